@@ -1,0 +1,48 @@
+"""The oracle's pins must catch plausible mistakes.  Each case compiles a copy
+of the oracle source with one planted mistake (on the CPU, into a temporary
+directory), loads it through GDN_ORACLE_LIB in a child pytest run of the pin
+suite, and expects that run to fail."""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "gdn_oracle.c")
+
+MUTANTS = {
+    "delta_sign": ("u[j] = beta[t] * (vt[j] - kS);", "u[j] = beta[t] * (vt[j] + kS);"),
+    "no_decay": ("for (int i = 0; i < dk * dv; ++i) S[i] *= decay;", "(void)decay;"),
+    "write_with_query": ("S[(int64_t)i * dv + j] += kt[i] * u[j];", "S[(int64_t)i * dv + j] += qt[i] * u[j];"),
+    "no_scale": ("o[(int64_t)t * dv + j] = scale * acc;\n        }\n        if (states)",
+                 "o[(int64_t)t * dv + j] = acc;\n        }\n        if (states)"),
+    "conv_reversed": ("acc += w[(int64_t)c * K + j] * xv;", "acc += w[(int64_t)c * K + (K - 1 - j)] * xv;"),
+    "softplus_no_one": ("log1p(exp(x))", "log(exp(x))"),
+    "gqa_interleaved": ("int hk = h / G;", "int hk = h % HK;"),
+    "l2_eps_outside": ("double inv = 1.0 / sqrt(ss + eps);", "double inv = 1.0 / (sqrt(ss) + eps);"),
+    "chunk_no_beta_in_A": ("val = bb[r] * exp(gam[r] - gam[s]) * kk;", "val = exp(gam[r] - gam[s]) * kk;"),
+    "chunk_decay_sign": ("intra += exp(gam[r] - gam[s]) * qk", "intra += exp(gam[s] - gam[r]) * qk"),
+    "conv_tail_shift": ("int64_t pos = (int64_t)L + i;", "int64_t pos = (int64_t)L + i - 1;"),
+    "verify_ckpt_window": ("int src = t + 1 - (K - 1) + j;", "int src = t - (K - 1) + j;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "mut.c")
+        so = os.path.join(d, "libmut.so")
+        open(c, "w").write(src.replace(old, new))
+        subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, c, "-lm"], check=True)
+        env = dict(os.environ, GDN_ORACLE_LIB=so)
+        r = subprocess.run(
+            [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+             os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600,
+        )
+        assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"

@@ -1,0 +1,41 @@
+"""Parity tolerances of the CUDA path against the fp64 oracle.
+
+Outputs: relative L2 <= 2e-3 and max-abs <= 1e-2; final fp32 states:
+relative L2 <= 1e-3; slot indexing and conv-state carry: bit-exact.  These are
+the layer description's parity bar and are far stricter than the 3e-2
+tolerances the SGLang GDN test matrix page uses (tests/golden/page_tolerances.txt).
+"""
+import numpy as np
+
+OUT_REL_L2 = 2e-3
+OUT_MAX_ABS = 1e-2
+STATE_REL_L2 = 1e-3
+
+
+def rel_l2(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    num = np.linalg.norm(got - ref)
+    return float(num / den) if den > 0 else float(num)
+
+
+def assert_out_close(got, ref, what="out"):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    r = rel_l2(got, ref)
+    m = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    assert r <= OUT_REL_L2 and m <= OUT_MAX_ABS, f"{what}: rel_l2={r:.3e} max_abs={m:.3e}"
+    return r, m
+
+
+def assert_state_close(got, ref, what="state"):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    r = rel_l2(got, ref)
+    assert r <= STATE_REL_L2, f"{what}: rel_l2={r:.3e}"
+    return r

@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the GDN layer on B200: one step = one gdn_extend over the
+packed prefill batch + one gdn_decode over the decode batch + one gdn_verify
+over the verify batch (every mode of the layer), on synthetic inputs already
+resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill32k|prefill262k]
+    python bench.py --impl reference ...      # the fp64 CPU oracle on a bounded sample
+
+Prints one JSON line (rank 0).  `value` is prefill tokens/s over all ranks,
+from the device time of the gdn_extend launches inside the timed steps;
+decode and verify report their own state-traffic figures.  Multi-GPU runs are
+independent replicas (weak scaling): every rank runs its own batch, no
+collective touches the data path; the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "GDN prefill tokens/s + decode state GB/s (frac. of roofline), 1×B200"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+C = 64
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["prefill32k", "prefill262k"], default="prefill32k")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-tokens", type=int, default=16384)
+    p.add_argument("--ref-sample-tokens", type=int, default=4096)
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ plumbing
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    try:
+        d = json.load(open(PEAKS_FILE))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def source_digest(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    if there is none or the kernel's source changed since it was taken."""
+    try:
+        d = json.load(open(TRAFFIC_FILE))[kernel]
+    except Exception:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or source_digest(src) != d["source_sha256_16"]:
+        return None
+    return float(d["bytes_per_launch"]) * float(d.get("scale_to_bench", 1.0))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        self.file.flush()
+        rows = []
+        for line in open(self.file.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        smax = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.5 * smax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+
+def prefill_work(spec, T):
+    """Algorithmic FLOPs and bytes of one prefill of T tokens (per value head and
+    chunk of C rows: intra 4C^2 d / G (q.k, k.k shared by the G value heads)
+    + 4C^2 d (W, U) + C^3/3 (triangular solve); state pass 6 C d^2 (W S, q^T S,
+    K^T V') + 2 C^2 d (decayed q.k times V'))."""
+    d, G, HV = spec.dk, spec.HV // spec.HK, spec.HV
+    per_chunk_intra = 4 * C * C * d / G + 4 * C * C * d + C ** 3 / 3
+    per_chunk_state = 6 * C * d * d + 2 * C * C * d
+    chunks = T / C
+    flops_intra = per_chunk_intra * chunks * HV
+    flops_state = per_chunk_state * chunks * HV
+    es = 2 if spec.dtype == torch.bfloat16 else 4
+    bytes_tok = spec.conv_dim * es + 2 * HV * es + HV * spec.dv * es
+    return {"flops_intra": flops_intra, "flops_state": flops_state, "flops": flops_intra + flops_state,
+            "bytes": bytes_tok * T, "bytes_per_token": bytes_tok}
+
+
+def decode_bytes(spec, B):
+    es = 2 if spec.dtype == torch.bfloat16 else 4
+    state = 2 * spec.HV * spec.dk * spec.dv * 4 * B
+    conv = 2 * spec.conv_dim * 3 * es * B
+    io = (spec.conv_dim + 2 * spec.HV + spec.HV * spec.dv) * es * B
+    return state, state + conv + io
+
+
+def verify_bytes(spec, B, D):
+    es = 2 if spec.dtype == torch.bfloat16 else 4
+    state = (1 + D) * spec.HV * spec.dk * spec.dv * 4 * B
+    conv = (1 + D) * spec.conv_dim * 3 * es * B
+    io = (spec.conv_dim + 2 * spec.HV + spec.HV * spec.dv) * es * B * D
+    return state, state + conv + io
+
+
+# ------------------------------------------------------------------ reference arm
+
+
+def oracle_sample(pre, ntok):
+    """The first `ntok` packed rows of the prefill batch (whole sequences, then
+    a cut of the next one), all heads, from the batch's initial slot contents."""
+    from oracle import oracle as O
+
+    spec = pre.spec
+    cu = pre.cu_seqlens.cpu().tolist()
+    n = min(ntok, cu[-1])
+    lens = []
+    for i in range(len(cu) - 1):
+        take = min(cu[i + 1], n) - cu[i]
+        if take <= 0:
+            break
+        lens.append(take)
+    N = len(lens)
+    cfg = O.OracleCfg(HK=spec.HK, HV=spec.HV, dk=spec.dk, dv=spec.dv)
+    slots = pre.state_indices[:N].cpu()
+    cs = pre.conv_state.cpu()
+    ss = pre.ssm_state.cpu()
+    cu_s = torch.tensor([0] + [sum(lens[:i + 1]) for i in range(N)], dtype=torch.int32)
+    args = (cfg, {k: (None if v is None else v.cpu()) for k, v in pre.params.items()}, pre.x[:n].cpu(),
+            pre.a[:n].cpu(), pre.b[:n].cpu(), cu_s, slots, cs, ss)
+    hi = None if pre.has_initial_state is None else pre.has_initial_state[:N].cpu()
+
+    def run():
+        O.extend(*args, has_initial_state=hi)
+
+    workers = min(O.num_threads(), N * spec.HV)
+    return run, n, workers
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from hybrid_linear_attention_causal_b200 import workloads as W
+
+    pre = W.large_prefill(device="cpu") if args.workload == "prefill32k" else W.long_prefill(device="cpu", T=8192)
+    run, n, workers = oracle_sample(pre, args.ref_sample_tokens)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    val = n / dt
+    sample = f"first {n} packed rows of the {pre.name} batch, all {pre.spec.HV} value heads, per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(pre, args),
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": workers, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def workload_config(pre, args):
+    s = pre.spec
+    return {"workload": pre.name, "prefill_tokens": pre.T, "prefill_seqs": pre.N,
+            "heads_qk_v": [s.HK, s.HV], "dk_dv": [s.dk, s.dv], "chunk": C, "io_dtype": str(s.dtype).split(".")[-1],
+            "decode_requests": 256, "decode_pool_slots": 1024, "verify_draft_tokens": 4,
+            "l2": "inputs larger than L2 (prefill input 512 MiB+, decode state 1 GiB touched per step)"}
+
+
+# ------------------------------------------------------------------ our arm
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        init_dist(world, "gloo")
+        run_reference(args, rank, world)
+        return
+    import hybrid_linear_attention_causal_b200 as gdn
+    from hybrid_linear_attention_causal_b200 import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+
+    seed_off = 1000 * rank  # every rank runs its own independent batch
+    if args.workload == "prefill32k":
+        pre = W.large_prefill(device=dev, seed=2 + seed_off)
+    else:
+        pre = W.long_prefill(device=dev, seed=4 + seed_off)
+    dv = W.decode_verify(device=dev, seed=3 + seed_off)
+    spec, dspec = pre.spec, dv.spec
+    cfg, dcfg = gdn.GdnConfig.from_spec(spec), gdn.GdnConfig.from_spec(dspec)
+    D = dv.extra["D"]
+    xv, av, bv = dv.extra["verify"]
+    Bn = dv.N
+
+    ws_pre = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, pre.N, pre.T), dev)
+    out_pre = torch.empty(pre.T, spec.HV, spec.dv, dtype=spec.dtype, device=dev)
+    ws_d = gdn.alloc_workspace(gdn.gdn_decode_workspace_size(dcfg, Bn), dev)
+    out_d = torch.empty(Bn, dspec.HV, dspec.dv, dtype=dspec.dtype, device=dev)
+    ws_v = gdn.alloc_workspace(gdn.gdn_verify_workspace_size(dcfg, Bn, D), dev)
+    out_v = torch.empty(Bn * D, dspec.HV, dspec.dv, dtype=dspec.dtype, device=dev)
+    ck = torch.empty(Bn, D, dspec.HV, dspec.dk, dspec.dv, dtype=torch.float32, device=dev)
+    cck = torch.empty(Bn, D, dspec.conv_dim, 3, dtype=dspec.dtype, device=dev)
+
+    def extend(x=pre.x, a=pre.a, b=pre.b, out=out_pre):
+        gdn.gdn_extend(cfg, pre.params, x, a, b, pre.cu_seqlens, pre.state_indices, pre.has_initial_state,
+                       pre.conv_state, pre.ssm_state, out, ws_pre)
+
+    def decode(x=dv.x, a=dv.a, b=dv.b, out=out_d):
+        gdn.gdn_decode(dcfg, dv.params, x, a, b, dv.state_indices, dv.conv_state, dv.ssm_state, out, ws_d)
+
+    def verify(x=xv, a=av, b=bv, out=out_v):
+        gdn.gdn_verify(dcfg, dv.params, x, a, b, dv.state_indices, D, dv.conv_state, dv.ssm_state, ck, cck, out,
+                       ws_v)
+
+    EXT_K = ["chunk_map", "prep", "conv_tail", "intra", "state"]
+    n_ev = len(EXT_K) + 1 + 2 + 2
+
+    def make_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+
+    def step(ev=None):
+        if ev is not None:
+            gdn.gdn_set_launch_events(ev[:len(EXT_K) + 1])
+        extend()
+        if ev is not None:
+            gdn.gdn_set_launch_events(ev[len(EXT_K) + 1:len(EXT_K) + 3])
+        decode()
+        if ev is not None:
+            gdn.gdn_set_launch_events(ev[len(EXT_K) + 3:])
+        verify()
+        if ev is not None:
+            gdn.gdn_set_launch_events([])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_error(ws_pre) == 0 and gdn.gdn_get_device_error(ws_d) == 0
+
+    evs = [make_events() for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for k in range(args.steps):
+            step(evs[k])
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    clocks = clk.summary()
+    total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    ms_step = total_ms / args.steps
+
+    def span(k, i, j):
+        return evs[k][i].elapsed_time(evs[k][j])
+
+    nE = len(EXT_K)
+    kern_ms = {name: statistics.mean(span(k, i, i + 1) for k in range(args.steps)) for i, name in enumerate(EXT_K)}
+    kern_ms["decode"] = statistics.mean(span(k, nE + 1, nE + 2) for k in range(args.steps))
+    kern_ms["verify"] = statistics.mean(span(k, nE + 3, nE + 4) for k in range(args.steps))
+    ext_ms = max_over_ranks(statistics.mean(span(k, 0, nE) for k in range(args.steps)), world, dev)
+    dec_ms = max_over_ranks(kern_ms["decode"], world, dev)
+    ver_ms = max_over_ranks(kern_ms["verify"], world, dev)
+
+    hbm, bf16, bf16_sus, peak_src = peaks()
+    pw = prefill_work(spec, pre.T)
+    st_dec, by_dec = decode_bytes(dspec, Bn)
+    st_ver, by_ver = verify_bytes(dspec, Bn, D)
+    value = world * pre.T / (ext_ms * 1e-3)
+
+    kernels = {
+        "state": {"bound": "alu", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": FP32_ALU_TFLOPS,
+                  "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+        "intra": {"bound": "alu", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": FP32_ALU_TFLOPS,
+                  "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+        "prep": {"bound": "hbm", "work": pre.T * (spec.conv_dim * 2 + 2 * spec.HV * 2), "unit": "GB/s",
+                 "peak": hbm, "peak_src": peak_src},
+        "decode": {"bound": "hbm", "work": by_dec, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
+        "verify": {"bound": "hbm", "work": by_ver, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
+    }
+    for name, k in kernels.items():
+        t = kern_ms[name] * 1e-3
+        scale = 1e12 if k["unit"] == "TFLOP/s" else 1e9
+        k["ms"] = kern_ms[name]
+        k["achieved"] = k["work"] / t / scale
+        k["frac"] = k["achieved"] / k["peak"]
+    dom = max(kern_ms, key=lambda n: kern_ms[n] if n in kernels else -1)
+    dk = kernels[dom]
+    roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                "unit": dk["unit"], "frac": dk["frac"], "traffic": ncu_traffic(dom),
+                "peak_source": dk["peak_src"] + (" (of measured)" if dk["peak_src"] == "measured" else "")}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hx, ha, hb = (t.cpu().pin_memory() for t in (pre.x, pre.a, pre.b))
+        hmeta = [t.cpu().pin_memory() for t in (pre.cu_seqlens, pre.state_indices, pre.has_initial_state)]
+        dmeta = [torch.empty_like(t) for t in (pre.cu_seqlens, pre.state_indices, pre.has_initial_state)]
+        dx, da, db = torch.empty_like(pre.x), torch.empty_like(pre.a), torch.empty_like(pre.b)
+        hout = torch.empty(out_pre.shape, dtype=out_pre.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in [hx, ha, hb] + hmeta)
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for h, d_ in zip([hx, ha, hb] + hmeta, [dx, da, db] + dmeta):
+                d_.copy_(h, non_blocking=True)
+            gdn.gdn_extend(cfg, pre.params, dx, da, db, dmeta[0], dmeta[1], dmeta[2], pre.conv_state, pre.ssm_state,
+                           out_pre, ws_pre)
+            hout.copy_(out_pre, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps, world, dev)
+        e2e = {"value": world * pre.T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
+               "what": "pinned host -> device copy of the prefill inputs, gdn_extend, device -> host copy of out"}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        run, n, workers = oracle_sample(pre, args.cpu_sample_tokens)
+        t0 = time.perf_counter()
+        run()
+        dt = time.perf_counter() - t0
+        cpu_baseline = {"value": n / dt, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                        "sample": f"fp64 oracle, first {n} packed rows of the batch, all {spec.HV} value heads"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(pre, args),
+            "roofline": roofline,
+            "cpu_baseline": cpu_baseline,
+            "e2e": e2e,
+            "gpu_launches": args.steps * (len(EXT_K) + 2),
+            "clocks": clocks,
+            "decode": {"ms": dec_ms, "requests_per_s": world * Bn / (dec_ms * 1e-3),
+                       "state_gbs": world * st_dec / (dec_ms * 1e-3) / 1e9,
+                       "total_gbs": world * by_dec / (dec_ms * 1e-3) / 1e9,
+                       "frac_of_8tbs_state": st_dec / (dec_ms * 1e-3) / 8e12,
+                       "frac_of_measured_hbm": by_dec / (dec_ms * 1e-3) / 1e9 / hbm},
+            "verify": {"ms": ver_ms, "state_gbs": world * st_ver / (ver_ms * 1e-3) / 1e9,
+                       "total_gbs": world * by_ver / (ver_ms * 1e-3) / 1e9,
+                       "frac_of_measured_hbm": by_ver / (ver_ms * 1e-3) / 1e9 / hbm},
+            "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12,
+                        "gbs_algorithmic": pw["bytes"] / (ext_ms * 1e-3) / 1e9,
+                        "kernel_ms": {k: kern_ms[k] for k in EXT_K}},
+            "kernels": {k: {kk: v[kk] for kk in ("bound", "ms", "achieved", "peak", "unit", "frac")}
+                        for k, v in kernels.items()},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,27 @@
+"""B200 (sm_100a) Gated DeltaNet layer: extend / decode / verify behind a C ABI.
+
+The compute lives in libgdn.so (csrc/, declared in include/gdn.h); this
+package holds its ctypes binding, the in-tree build step and seeded synthetic
+workloads.  Calls fail loudly when libgdn.so has not been built.
+"""
+from .binding import (  # noqa: F401
+    GDN_DEVERR_SEQLENS,
+    GDN_DEVERR_SLOT_RANGE,
+    GDN_ERR_CUDA,
+    GDN_ERR_INVALID_ARG,
+    GDN_ERR_UNSUPPORTED,
+    GDN_ERR_WORKSPACE,
+    GDN_OK,
+    GdnConfig,
+    GdnError,
+    alloc_workspace,
+    gdn_decode,
+    gdn_decode_workspace_size,
+    gdn_extend,
+    gdn_extend_workspace_size,
+    gdn_get_device_error,
+    gdn_reset_device_error,
+    gdn_set_launch_events,
+    gdn_verify,
+    gdn_verify_workspace_size,
+)

@@ -1,0 +1,125 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libgdn.
+// Not part of the public interface (include/gdn.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+constexpr int kChunk = 64;          // prefill chunk length C
+constexpr int kConvK = 4;           // conv width K
+constexpr int kHeaderBytes = 256;   // workspace header (error word + counters)
+constexpr int kMaxVerifyDraft = 16; // D limit of gdn_verify
+
+// header layout (int32 words)
+constexpr int kHdrError = 0;        // sticky GDN_DEVERR_* bits
+constexpr int kHdrNumChunks = 1;    // chunk count of the current extend batch
+
+struct LayerDims {
+    int HK, HV, dk, dv, G;  // G = HV / HK
+    int conv_dim;           // 2*HK*dk + HV*dv
+    float scale;            // resolved (> 0)
+    float eps;
+};
+
+// ---- element access -------------------------------------------------------
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// SiLU, softplus and sigmoid in fp32 from the CUDA math library's expf/log1pf.
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+__device__ __forceinline__ float softplus_f(float x) { return x > 20.0f ? x : log1pf(expf(x)); }
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ void raise_error(int32_t* hdr, int bits) {
+    if (hdr) atomicOr(reinterpret_cast<int*>(hdr) + kHdrError, bits);
+}
+
+// ---- launch argument blocks ----------------------------------------------
+
+struct DecodeArgs {
+    LayerDims d;
+    const float* A_log;
+    const float* dt_bias;
+    const void* conv_w;
+    const void* conv_b;
+    const void* x;      // [B*D, conv_dim]
+    const void* a;      // [B*D, HV]
+    const void* b;      // [B*D, HV]
+    const int32_t* slots;
+    int B, D, P;
+    void* conv_state;   // decode: read/write; verify: read only
+    float* ssm_state;   // decode: read/write; verify: read only
+    float* state_ckpt;  // verify only
+    void* conv_ckpt;    // verify only, nullable
+    void* out;          // [B*D, HV, dv]
+    int32_t* hdr;       // workspace header (error word)
+};
+
+struct ExtendArgs {
+    LayerDims d;
+    const float* A_log;
+    const float* dt_bias;
+    const void* conv_w;
+    const void* conv_b;
+    const void* x;      // [T, conv_dim]
+    const void* a;      // [T, HV]
+    const void* b;      // [T, HV]
+    const int32_t* cu;  // [N+1]
+    const int32_t* slots;
+    const int32_t* has_init;  // nullable
+    int N, T, P;
+    int max_chunks;     // upper bound on sum_n ceil(L_n / C)
+    void* conv_state;
+    float* ssm_state;
+    void* out;          // [T, HV, dv]
+    // workspace carve-out
+    int32_t* hdr;
+    int4* chunk_tab;    // [max_chunks] {seq, first row, length, chunk index within seq}
+    int32_t* seq_chunk0;// [N+1] first chunk id of each sequence
+    float* qn;          // [T, HK, dk] normalised q times scale
+    float* kn;          // [T, HK, dk] normalised k
+    float* vv;          // [T, HV, dv] SiLU(conv) values
+    float2* gb;         // [T, HV] (g, beta)
+    float* W;           // [max_chunks, HV, C, dk]
+    float* U;           // [max_chunks, HV, C, dv]
+    float* Aqk;         // [max_chunks, HV, C, C]
+    float* gam;         // [max_chunks, HV, C] in-chunk cumulative g
+};
+
+// Dispatch on the supported (dk, dv) pairs; expects a LayerDims `p.d` in scope.
+#define GDN_DISPATCH_DIMS(T, FN, ...)                                                   \
+    do {                                                                                \
+        if (p.d.dk == 128 && p.d.dv == 128) return FN<T, 128, 128>(__VA_ARGS__);        \
+        if (p.d.dk == 128 && p.d.dv == 64) return FN<T, 128, 64>(__VA_ARGS__);          \
+        if (p.d.dk == 64 && p.d.dv == 128) return FN<T, 64, 128>(__VA_ARGS__);          \
+        if (p.d.dk == 64 && p.d.dv == 64) return FN<T, 64, 64>(__VA_ARGS__);            \
+        return cudaErrorInvalidValue;                                                   \
+    } while (0)
+
+// Records the calling thread's i-th profiling event on `s` if one is set
+// (see gdn_set_launch_events); a no-op otherwise.
+void mark_launch(cudaStream_t s, int i);
+
+size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max_chunks_out);
+void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T);
+
+cudaError_t launch_decode(const DecodeArgs& args, int dtype, cudaStream_t s);
+cudaError_t launch_verify(const DecodeArgs& args, int dtype, cudaStream_t s);
+cudaError_t launch_extend(const ExtendArgs& args, int dtype, cudaStream_t s);
+
+}  // namespace gdn

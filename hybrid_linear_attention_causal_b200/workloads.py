@@ -280,7 +280,7 @@ def random_case(spec: LayerSpec, lengths, P: int, seed: int, device="cpu", init_
     else:
         slots = torch.tensor(list(slots), dtype=torch.int32, device=device)
     conv_state, ssm_state = make_pools(spec, P, device)
-    live = [int(s) for s in slots.tolist() if s >= 0]
+    live = [int(s) for s in slots.tolist() if 0 <= s < P]
     if init_random and live:
         fill_slots_random_(spec, conv_state, ssm_state, live, g, device)
     x, a, b = make_tokens(spec, sum(int(n) for n in lengths), g, device, a_mean=a_mean)

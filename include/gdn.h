@@ -1,0 +1,207 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet layer library (libgdn.so).
+ *
+ * The library runs the linear-attention half of a hybrid full-attention + GDN
+ * model: the call that page "pymllm.layers.attention.hybrid_backend" shows as
+ * HybridAttnBackend.forward_gdn(layer, forward_batch, mixed_qkv, a, b), with
+ * the per-layer parameters that `layer` carries (A_log, dt_bias, conv weight)
+ * passed explicitly.  The forward modes of page "SGLang GDN hybrid linear
+ * attention test matrix" (section on the forward-mode contract: decode/idle,
+ * extend and target-verify are the legal modes) map onto three entry points:
+ *
+ *   gdn_extend  EXTEND / MIXED / DRAFT_EXTEND: ragged packed-varlen prefill
+ *   gdn_decode  DECODE / IDLE: one token per request (IDLE = zero requests)
+ *   gdn_verify  TARGET_VERIFY: D draft tokens per request, state checkpoints
+ *
+ * What every mode computes, per request and value head h (qk head h / (HV/HK)):
+ *   conv:  y_t = SiLU(sum_{j<K} w[c,j] x_{t-K+1+j}[c] (+ bias[c])) per channel c,
+ *          rows before the request's first new row come from its conv-state slot;
+ *   split: y = [q (HK*dk) | k (HK*dk) | v (HV*dv)], head-major, dim-minor;
+ *   norm:  q <- q / sqrt(|q|^2 + l2_eps), likewise k;
+ *   gates: g = -exp(A_log[h]) * softplus(a_t[h] + dt_bias[h]), beta = sigmoid(b_t[h]);
+ *   rule:  S_t = exp(g_t) (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+ *          o_t = scale * S_t^T q_t   (S in R^{dk x dv}, fp32),
+ * which is the gated delta rule of Gated DeltaNet (Yang, Kautz, Hatamizadeh,
+ * ICLR 2025).  scale <= 0 selects 1/sqrt(dk), the default of page
+ * "pymllm.layers.attention.radix_attention" (RadixAttention, `scaling`).
+ *
+ * Conventions shared by all calls
+ *   - Every pointer argument is DEVICE memory owned by the caller unless its
+ *     comment says host.  The library allocates nothing and keeps no mutable
+ *     global state; calls on different streams with disjoint outputs may run
+ *     concurrently.
+ *   - Every call is asynchronous and stream-ordered on `stream` (a
+ *     cudaStream_t; NULL is the legacy default stream).  No call synchronises
+ *     the host, so decode and verify can be captured in a CUDA graph, and so
+ *     can extend for a fixed (N, T).
+ *   - dtype GDN_DTYPE_BF16 or GDN_DTYPE_F32 applies to mixed_qkv, a, b, out,
+ *     conv_weight, conv_bias and the conv-state pool.  A_log, dt_bias and the
+ *     ssm-state pool (and verify checkpoints) are always fp32.
+ *   - Pool layouts: conv_state [P, conv_dim, K-1] (the K-1 most recent raw rows
+ *     of each channel, index 0 oldest), ssm_state [P, HV, dk, dv] (dv fastest),
+ *     conv_dim = 2*HK*dk + HV*dv.
+ *   - state_indices[i] names request i's pool slot.  A negative entry marks a
+ *     padded request: its output rows are written as zeros and nothing else is
+ *     touched.  An entry >= P is a caller error detected on the device: the
+ *     request is treated as padded and GDN_DEVERR_SLOT_RANGE is raised in the
+ *     workspace error word.  Slots not named by any request are never read or
+ *     written.  Two live requests naming the same slot race (undefined).
+ *   - Supported shapes: dk, dv in {64, 128}; HV % HK == 0; K == 4.  Every
+ *     pointer must be 16-byte aligned.
+ *   - Return value: GDN_OK, or a GDN_ERR_* code with nothing launched.
+ *     Launch failures return GDN_ERR_CUDA; gdn_last_cuda_error() gives the
+ *     CUDA error string of the most recent one on the calling thread.
+ *   - Workspace: caller-allocated device memory of at least the size the
+ *     matching *_workspace_size() returns.  Its first 256 bytes are a header
+ *     whose first int32 is a sticky device error word: kernels OR GDN_DEVERR_*
+ *     bits into it and never clear it.  Zero it once after allocation with
+ *     gdn_reset_device_error() (or cudaMemset) and read it with
+ *     gdn_get_device_error().
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
+
+/* return codes */
+#define GDN_OK 0
+#define GDN_ERR_INVALID_ARG 1 /* null required pointer, bad shape, misalignment, negative size */
+#define GDN_ERR_UNSUPPORTED 2 /* well-formed but outside the supported set (dk/dv/K/dtype) */
+#define GDN_ERR_WORKSPACE 3   /* workspace too small for (N, T) or (B, D) */
+#define GDN_ERR_CUDA 4        /* a kernel launch failed */
+
+/* device error bits (sticky word at the start of the workspace) */
+#define GDN_DEVERR_SLOT_RANGE 0x1 /* a state index >= P was skipped */
+#define GDN_DEVERR_SEQLENS 0x2    /* cu_seqlens not non-decreasing from 0 to T; the batch was skipped */
+
+/* element types */
+#define GDN_DTYPE_F32 0
+#define GDN_DTYPE_BF16 1
+
+typedef struct {
+    int32_t num_qk_heads; /* HK */
+    int32_t num_v_heads;  /* HV, multiple of HK */
+    int32_t head_k_dim;   /* dk: 64 or 128 */
+    int32_t head_v_dim;   /* dv: 64 or 128 */
+    int32_t conv_kernel;  /* K: 4 */
+    int32_t dtype;        /* GDN_DTYPE_* */
+    float scale;          /* <= 0: 1/sqrt(dk) */
+    float l2_eps;         /* L2-norm epsilon, e.g. 1e-6 */
+} gdn_config_t;
+
+typedef struct {
+    const float* A_log;      /* [HV] fp32 */
+    const float* dt_bias;    /* [HV] fp32 */
+    const void* conv_weight; /* [conv_dim, K], cfg dtype */
+    const void* conv_bias;   /* [conv_dim], cfg dtype, or NULL for no bias */
+} gdn_params_t;
+
+/*
+ * Workspace bytes for gdn_extend over at most max_N sequences and max_T
+ * packed tokens (holds the chunk table and the fp32 intermediates of the
+ * chunked prefill).  Returns 0 for an invalid configuration.
+ */
+GDN_API size_t gdn_extend_workspace_size(const gdn_config_t* cfg, int32_t max_N, int32_t max_T);
+
+/*
+ * EXTEND (prefill): sequence n owns rows cu_seqlens[n] .. cu_seqlens[n+1]-1
+ * of the packed inputs and continues from pool slot state_indices[n].
+ *
+ *   mixed_qkv          [T, conv_dim] raw (pre-conv) rows, cfg dtype
+ *   a, b               [T, HV] gate pre-activations, cfg dtype
+ *   cu_seqlens         [N+1] int32 device, 0 = cu[0] <= cu[1] <= ... <= cu[N] = T
+ *   state_indices      [N] int32 device, see the conventions above
+ *   has_initial_state  [N] int32 device or NULL (= all 1); 0 reads the slot's
+ *                      conv and ssm contents as zeros (they are overwritten)
+ *   conv_state, ssm_state  pools of P slots, read and written in place
+ *   out                [T, HV, dv] cfg dtype
+ * Zero-length sequences are no-ops.  N == 0 or T == 0 returns GDN_OK with
+ * nothing launched.  The final state of each sequence is written to its slot,
+ * and the conv slot receives the K-1 most recent raw rows of (old conv state |
+ * the sequence's rows).
+ */
+GDN_API int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+               const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
+               const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
+               void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* Workspace bytes for gdn_decode (the error header only). */
+GDN_API size_t gdn_decode_workspace_size(const gdn_config_t* cfg, int32_t max_B);
+
+/*
+ * DECODE: request i has one new row (row i of mixed_qkv [B, conv_dim], a and
+ * b [B, HV]) and continues from slot state_indices[i]; its conv and ssm slots
+ * are updated in place and out [B, HV, dv] receives the outputs.  B == 0
+ * (IDLE) returns GDN_OK with nothing launched.
+ */
+GDN_API int gdn_decode(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+               const void* b, const int32_t* state_indices, int32_t B, void* conv_state, float* ssm_state,
+               int32_t P, void* out, void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* Workspace bytes for gdn_verify (the error header only). */
+GDN_API size_t gdn_verify_workspace_size(const gdn_config_t* cfg, int32_t max_B, int32_t D);
+
+/*
+ * TARGET_VERIFY: request i has D draft rows (rows i*D .. i*D+D-1 of
+ * mixed_qkv [B*D, conv_dim], a and b [B*D, HV]) and runs them in order from
+ * slot state_indices[i].  Both pools are read only.  state_ckpt
+ * [B, D, HV, dk, dv] fp32 receives the state after every draft token;
+ * conv_ckpt [B, D, conv_dim, K-1] (cfg dtype, or NULL) the conv window after
+ * every token; out [B*D, HV, dv] the outputs.  Checkpoints of padded requests
+ * are left untouched.  1 <= D <= 16.  This is the speculative Mamba-state
+ * buffer that the target-verify path of page "SGLang GDN hybrid linear
+ * attention test matrix" (verification conventions) fills; committing an
+ * accepted prefix back into the pool is a separate step.
+ */
+GDN_API int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+               const void* b, const int32_t* state_indices, int32_t B, int32_t D, const void* conv_state,
+               const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt, void* out, void* workspace,
+               size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * Reads the sticky device error word of `workspace` into *err_out (host).
+ * Enqueues a device-to-host copy on `stream` and waits for that stream, so it
+ * must not be called during stream capture.  Returns GDN_ERR_CUDA on failure.
+ */
+GDN_API int gdn_get_device_error(const void* workspace, int32_t* err_out, gdn_stream_t stream);
+
+/* Clears the device error word of `workspace` (an async memset on `stream`). */
+GDN_API int gdn_reset_device_error(void* workspace, gdn_stream_t stream);
+
+/*
+ * Profiling aid (off by default).  With n > 0, the calling thread's later
+ * gdn_extend / gdn_decode / gdn_verify calls record events[i] (each a
+ * cudaEvent_t created by the caller) on their stream just before their i-th
+ * kernel launch, and events[L] right after the last one, L being the number
+ * of kernels the call launches (5 for extend, 1 for decode and verify);
+ * indices >= n are not recorded.  n == 0 turns recording off.  The events
+ * bracket each kernel, so elapsed times between consecutive events are
+ * per-kernel device times.  Returns GDN_ERR_INVALID_ARG for n < 0, n > 16 or
+ * events == NULL with n > 0.
+ */
+GDN_API int gdn_set_launch_events(void* const* events, int32_t n);
+
+/* Static description of a return code. */
+GDN_API const char* gdn_strerror(int code);
+
+/* CUDA error string of the most recent GDN_ERR_CUDA on the calling thread ("" if none). */
+GDN_API const char* gdn_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -48,6 +48,9 @@
  */
 #include <math.h>
 #include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdlib.h>
 #include <string.h>
 
@@ -70,6 +73,15 @@ static int64_t ora_conv_dim(const ora_cfg* c) { return 2LL * c->HK * c->dk + (in
 double ora_gate_g(double A_log, double a, double dt_bias) { return -exp(A_log) * ora_softplus(a + dt_bias); }
 double ora_gate_beta(double b) { return ora_sigmoid(b); }
 double ora_softplus_exported(double x) { return ora_softplus(x); }
+
+/* number of OpenMP threads the layer functions use (1 without OpenMP) */
+int ora_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* x <- x / sqrt(sum x^2 + eps) over n entries */
 void ora_l2norm(double* x, int n, double eps) {

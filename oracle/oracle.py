@@ -123,6 +123,11 @@ def _p(a, kind=_dbl_p):
 # ---------------------------------------------------------------------------
 
 
+def num_threads() -> int:
+    """OpenMP threads the layer functions run on."""
+    return int(_L().ora_num_threads())
+
+
 def gate_g(A_log: float, a: float, dt_bias: float) -> float:
     return _L().ora_gate_g(float(A_log), float(a), float(dt_bias))
 

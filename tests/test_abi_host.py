@@ -1,0 +1,129 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/gdn.h declares, sizes workspaces, and rejects bad
+arguments before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hybrid_linear_attention_causal_b200 as gdn
+from hybrid_linear_attention_causal_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+FAKE = 0x10000  # aligned, never dereferenced by the host-side validation
+FAKE_MIS = 0x10004
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    L = B.lib()
+    for s in syms:
+        assert hasattr(L, s), f"libgdn.so does not export {s}"
+
+
+def test_strerror_codes():
+    for code in (gdn.GDN_OK, gdn.GDN_ERR_INVALID_ARG, gdn.GDN_ERR_UNSUPPORTED, gdn.GDN_ERR_WORKSPACE,
+                 gdn.GDN_ERR_CUDA):
+        assert B.strerror(code) and "unknown" not in B.strerror(code)
+    assert "unknown" in B.strerror(99)
+
+
+def cfg(**kw):
+    base = dict(num_qk_heads=16, num_v_heads=32, head_k_dim=128, head_v_dim=128)
+    base.update(kw)
+    return gdn.GdnConfig(**base)
+
+
+def test_workspace_sizes():
+    c = cfg()
+    small = gdn.gdn_extend_workspace_size(c, 1, 64)
+    big = gdn.gdn_extend_workspace_size(c, 8, 32768)
+    assert 0 < small < big
+    assert gdn.gdn_extend_workspace_size(c, 8, 32768) >= 32768 * (2 * 16 * 128 + 32 * 128) * 4
+    assert gdn.gdn_decode_workspace_size(c, 256) == B.HEADER_BYTES
+    assert gdn.gdn_verify_workspace_size(c, 256, 4) == B.HEADER_BYTES
+    assert gdn.gdn_verify_workspace_size(c, 256, 17) == 0
+    assert gdn.gdn_extend_workspace_size(cfg(head_k_dim=96), 1, 64) == 0
+    assert gdn.gdn_extend_workspace_size(cfg(num_v_heads=24, num_qk_heads=16), 1, 64) == 0
+
+
+def _params(mis=False):
+    p = B.GdnParamsC(FAKE, FAKE, FAKE_MIS if mis else FAKE, None)
+    return ctypes.byref(p)
+
+
+def _extend(c, N=2, T=100, ws_bytes=1 << 40, params=None, x=FAKE, cu=FAKE, ws=FAKE, out=FAKE):
+    return B.lib().gdn_extend(ctypes.byref(c.c()), params or _params(), x, FAKE, FAKE, cu, N, T, FAKE, None, FAKE,
+                              FAKE, 4, out, ws, ws_bytes, None)
+
+
+def _decode(c, Bn=3, ws_bytes=256, ws=FAKE, slots=FAKE):
+    return B.lib().gdn_decode(ctypes.byref(c.c()), _params(), FAKE, FAKE, FAKE, slots, Bn, FAKE, FAKE, 8, FAKE, ws,
+                              ws_bytes, None)
+
+
+def _verify(c, Bn=3, D=4, ckpt=FAKE):
+    return B.lib().gdn_verify(ctypes.byref(c.c()), _params(), FAKE, FAKE, FAKE, FAKE, Bn, D, FAKE, FAKE, 8, ckpt,
+                              None, FAKE, FAKE, 256, None)
+
+
+def test_extend_argument_validation():
+    c = cfg()
+    assert _extend(c, N=0) == gdn.GDN_OK  # nothing to do, nothing launched
+    assert _extend(c, T=0) == gdn.GDN_OK
+    assert _extend(c, N=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, x=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, out=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, cu=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, ws=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, x=FAKE_MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, params=_params(mis=True)) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend(c, ws_bytes=1024) == gdn.GDN_ERR_WORKSPACE
+    assert _extend(cfg(num_v_heads=20)) == gdn.GDN_ERR_INVALID_ARG  # HV % HK != 0
+    assert _extend(cfg(head_k_dim=96)) == gdn.GDN_ERR_UNSUPPORTED
+    assert _extend(cfg(head_v_dim=256)) == gdn.GDN_ERR_UNSUPPORTED
+    assert _extend(cfg(conv_kernel=3)) == gdn.GDN_ERR_UNSUPPORTED
+    assert _extend(gdn.GdnConfig(16, 32, 128, 128, dtype=__import__("torch").float16)) == gdn.GDN_ERR_UNSUPPORTED
+    assert B.lib().gdn_extend(None, _params(), FAKE, FAKE, FAKE, FAKE, 1, 1, FAKE, None, FAKE, FAKE, 4, FAKE, FAKE,
+                              1 << 40, None) == gdn.GDN_ERR_INVALID_ARG
+    assert B.lib().gdn_extend(ctypes.byref(cfg().c()), None, FAKE, FAKE, FAKE, FAKE, 1, 1, FAKE, None, FAKE, FAKE,
+                              4, FAKE, FAKE, 1 << 40, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_decode_and_verify_argument_validation():
+    c = cfg()
+    assert _decode(c, Bn=0) == gdn.GDN_OK  # IDLE
+    assert _decode(c, Bn=-2) == gdn.GDN_ERR_INVALID_ARG
+    assert _decode(c, ws=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _decode(c, slots=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _decode(c, ws_bytes=16) == gdn.GDN_ERR_WORKSPACE
+    assert _decode(cfg(head_k_dim=32)) == gdn.GDN_ERR_UNSUPPORTED
+    assert _verify(c, Bn=0) == gdn.GDN_OK
+    assert _verify(c, D=0) == gdn.GDN_ERR_INVALID_ARG
+    assert _verify(c, D=17) == gdn.GDN_ERR_INVALID_ARG
+    assert _verify(c, ckpt=None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_error_helpers_reject_null():
+    v = ctypes.c_int32(0)
+    assert B.lib().gdn_get_device_error(None, ctypes.byref(v), None) == gdn.GDN_ERR_INVALID_ARG
+    assert B.lib().gdn_reset_device_error(None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+
+    c = gdn.GdnConfig(2, 2, 64, 64, dtype=torch.float32)
+    t = torch.zeros(4)
+    with pytest.raises(ValueError):
+        gdn.gdn_decode(c, {"A_log": t, "dt_bias": t, "conv_w": t}, t, t, t, torch.zeros(1, dtype=torch.int32), t, t,
+                       t, t)

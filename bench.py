@@ -53,6 +53,10 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample-tokens", type=int, default=16384)
     p.add_argument("--ref-sample-tokens", type=int, default=4096)
+    p.add_argument("--profile", choices=["extend", "decode", "verify"], default=None,
+                   help="run only this call on a reduced case (an ncu target); prints timings, not the bench line")
+    p.add_argument("--profile-tokens", type=int, default=8192, help="prefill rows of the --profile extend case")
+    p.add_argument("--profile-requests", type=int, default=64, help="requests of the --profile decode/verify case")
     return p.parse_args()
 
 
@@ -273,6 +277,51 @@ def workload_config(pre, args):
 # ------------------------------------------------------------------ our arm
 
 
+def run_profile_case(args, dev):
+    """A reduced case of one call, for ncu captures: `--profile extend` runs the
+    prefill layer (16/32 heads, d=128) on --profile-tokens rows in 4 sequences;
+    decode/verify run --profile-requests requests on a pool of twice as many
+    slots.  Inputs stay larger than L2 for the default sizes."""
+    import hybrid_linear_attention_causal_b200 as gdn
+    from hybrid_linear_attention_causal_b200 import workloads as W
+
+    if args.profile == "extend":
+        w = W.large_prefill(device=dev, total=args.profile_tokens, nseq=4)
+        cfg = gdn.GdnConfig.from_spec(w.spec)
+        ws = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, w.N, w.T), dev)
+        out = torch.empty(w.T, w.spec.HV, w.spec.dv, dtype=w.spec.dtype, device=dev)
+        call = lambda: gdn.gdn_extend(cfg, w.params, w.x, w.a, w.b, w.cu_seqlens, w.state_indices,
+                                      w.has_initial_state, w.conv_state, w.ssm_state, out, ws)
+    else:
+        Bn = args.profile_requests
+        w = W.decode_verify(device=dev, B=Bn, P=2 * Bn)
+        cfg = gdn.GdnConfig.from_spec(w.spec)
+        if args.profile == "decode":
+            ws = gdn.alloc_workspace(gdn.gdn_decode_workspace_size(cfg, Bn), dev)
+            out = torch.empty(Bn, w.spec.HV, w.spec.dv, dtype=w.spec.dtype, device=dev)
+            call = lambda: gdn.gdn_decode(cfg, w.params, w.x, w.a, w.b, w.state_indices, w.conv_state,
+                                          w.ssm_state, out, ws)
+        else:
+            D = w.extra["D"]
+            xv, av, bv = w.extra["verify"]
+            ws = gdn.alloc_workspace(gdn.gdn_verify_workspace_size(cfg, Bn, D), dev)
+            out = torch.empty(Bn * D, w.spec.HV, w.spec.dv, dtype=w.spec.dtype, device=dev)
+            ck = torch.empty(Bn, D, w.spec.HV, w.spec.dk, w.spec.dv, device=dev)
+            call = lambda: gdn.gdn_verify(cfg, w.params, xv, av, bv, w.state_indices, D, w.conv_state,
+                                          w.ssm_state, ck, None, out, ws)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(args.steps):
+        call()
+    s1.record()
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_error(ws) == 0
+    print(json.dumps({"profile": args.profile, "workload": w.name, "ms_per_call": s0.elapsed_time(s1) / args.steps}))
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
@@ -285,6 +334,8 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.profile:
+        return run_profile_case(args, dev)
     init_dist(world, "nccl")
 
     seed_off = 1000 * rank  # every rank runs its own independent batch

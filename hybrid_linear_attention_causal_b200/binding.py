@@ -228,5 +228,8 @@ def gdn_set_launch_events(events) -> None:
     """Profiling aid: record these torch.cuda.Event objects around each kernel
     the following calls launch (see include/gdn.h); [] turns it off."""
     n = len(events)
+    for e in events:
+        if not e.cuda_event:  # torch creates the underlying cudaEvent_t on first record
+            e.record()
     arr = (ctypes.c_void_p * max(n, 1))(*[e.cuda_event for e in events])
     _check(lib().gdn_set_launch_events(arr if n else None, n), "gdn_set_launch_events")

@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     gdn_decode,
     gdn_decode_workspace_size,
     gdn_extend,
+    gdn_extend_static_scratch,
     gdn_extend_workspace_size,
     gdn_get_device_error,
     gdn_reset_device_error,

@@ -108,6 +108,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_verify_workspace_size.restype = sz
         L.gdn_extend.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp, sz, vp]
         L.gdn_extend.restype = ctypes.c_int
+        L.gdn_extend_static_scratch.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp]
+        L.gdn_extend_static_scratch.restype = ctypes.c_int
         L.gdn_decode.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_verify.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
@@ -188,6 +190,24 @@ def gdn_extend(cfg: GdnConfig, params: dict, mixed_qkv, a, b, cu_seqlens, state_
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
     )
     _check(rc, "gdn_extend")
+
+
+EXTEND_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def gdn_extend_static_scratch(cfg: GdnConfig, params: dict, mixed_qkv, a, b, cu_seqlens, state_indices,
+                              has_initial_state, conv_state, ssm_state, out, stream=None) -> None:
+    """gdn_extend for callers that cannot allocate: the scratch is the library's
+    fixed 64 MiB device array (see include/gdn.h); calls must not overlap on the GPU."""
+    N = int(state_indices.shape[0])
+    T = int(mixed_qkv.shape[0])
+    P = int(ssm_state.shape[0])
+    rc = lib().gdn_extend_static_scratch(
+        ctypes.byref(cfg.c()), ctypes.byref(_params(params)), _ptr(mixed_qkv), _ptr(a), _ptr(b), _ptr(cu_seqlens),
+        N, T, _ptr(state_indices), _ptr(has_initial_state), _ptr(conv_state), _ptr(ssm_state), P, _ptr(out),
+        _stream(stream),
+    )
+    _check(rc, "gdn_extend_static_scratch")
 
 
 def gdn_decode(cfg: GdnConfig, params: dict, mixed_qkv, a, b, state_indices, conv_state, ssm_state, out, workspace,

@@ -138,6 +138,42 @@ GDN_API int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, cons
                const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
                void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
+/* Size of the fixed device scratch behind gdn_extend_static_scratch. */
+#define GDN_EXTEND_STATIC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * EXTEND for callers that cannot allocate device memory.  The paper has no
+ * counterpart to this entry point; it exists for callers such as engine
+ * plugins whose enqueue step may not allocate (the host framework's allocator
+ * owns device memory), latency-critical paths that cannot take the device
+ * synchronisation cudaMalloc/cudaFree may cause, and hosts that pass the
+ * layer only its inputs and outputs.
+ *
+ * Same arguments and results as gdn_extend, minus the workspace: the scratch
+ * comes from a fixed GDN_EXTEND_STATIC_SCRATCH_BYTES (64 MiB) array in the
+ * library's own device memory, which every GPU that loads the library holds
+ * until the process exits.  Nothing is allocated: no cudaMalloc, no cudaFree,
+ * no allocating library routine.
+ *   - Sizes whose gdn_extend_workspace_size(cfg, N, T) exceeds
+ *     GDN_EXTEND_STATIC_SCRATCH_BYTES are rejected with GDN_ERR_WORKSPACE and
+ *     nothing is launched (one sequence of up to 837 tokens for the
+ *     16/32-head, dk = dv = 128 layer; 6439 for the 4/8-head, 64 layer).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make
+ *     that first call outside any stream capture.  A failure there returns
+ *     GDN_ERR_CUDA with the cause left in the CUDA runtime's last error.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; each call clears the part that must start at zero
+ *     before its kernels run.  Calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on the array: order them.
+ *   - Device-detected argument errors are handled as in gdn_extend (the
+ *     request or batch is skipped), but their error bits are not readable.
+ */
+GDN_API int gdn_extend_static_scratch(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv,
+                                      const void* a, const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T,
+                                      const int32_t* state_indices, const int32_t* has_initial_state,
+                                      void* conv_state, float* ssm_state, int32_t P, void* out, gdn_stream_t stream);
+
 /* Workspace bytes for gdn_decode (the error header only). */
 GDN_API size_t gdn_decode_workspace_size(const gdn_config_t* cfg, int32_t max_B);
 

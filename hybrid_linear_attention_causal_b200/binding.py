@@ -22,6 +22,7 @@ GDN_ERR_WORKSPACE = 3
 GDN_ERR_CUDA = 4
 GDN_DEVERR_SLOT_RANGE = 0x1
 GDN_DEVERR_SEQLENS = 0x2
+GDN_DEVERR_TIMEOUT = 0x4
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 HEADER_BYTES = 256

@@ -95,10 +95,14 @@ struct ExtendArgs {
     float* kn;          // [T, HK, dk] normalised k
     float* vv;          // [T, HV, dv] SiLU(conv) values
     float2* gb;         // [T, HV] (g, beta)
-    float* W;           // [max_chunks, HV, C, dk]
-    float* U;           // [max_chunks, HV, C, dv]
-    float* Aqk;         // [max_chunks, HV, C, C]
-    float* gam;         // [max_chunks, HV, C] in-chunk cumulative g
+    // per (chunk, value head), written by the intra kernel, read by the state
+    // pass; the three tiles are tf32 values already in the tensor-core
+    // shared-memory layout, so the state pass copies them verbatim
+    float* WQ;          // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], K-major, 128 rows
+    float* AQ;          // [max_chunks, HV, C*C]     masked decayed q.k, K-major, C rows
+    float* KT;          // [max_chunks, HV, dk*C]    (diag(e^{gamma_n-gamma}) K)^T, K-major, dk rows
+    float* U;           // [max_chunks, HV, C, dv]   fp32, row-major
+    float* gam;         // [max_chunks, HV, C]       in-chunk cumulative g
 };
 
 // Dispatch on the supported (dk, dv) pairs; expects a LayerDims `p.d` in scope.
@@ -110,6 +114,17 @@ struct ExtendArgs {
         if (p.d.dk == 64 && p.d.dv == 64) return FN<T, 64, 64>(__VA_ARGS__);            \
         return cudaErrorInvalidValue;                                                   \
     } while (0)
+
+// True when chunk_map rejected the batch (it then publishes zero chunks).
+__device__ __forceinline__ bool batch_rejected(const ExtendArgs& p) { return p.hdr[kHdrNumChunks] == 0; }
+
+// Intra-chunk step on tensor cores (gdn_intra_tc.cu): grid (max_chunks, HK).
+template <int DK, int DV>
+cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s);
+
+// Serial state pass + outputs on tensor cores (gdn_state_tc.cu): grid (N, HV).
+template <typename T, int DK, int DV>
+cudaError_t launch_state(const ExtendArgs& p, cudaStream_t s);
 
 // Records the calling thread's i-th profiling event on `s` if one is set
 // (see gdn_set_launch_events); a no-op otherwise.

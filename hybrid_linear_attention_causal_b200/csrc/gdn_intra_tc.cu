@@ -1,0 +1,377 @@
+// Intra-chunk step of the chunked GDN prefill on tcgen05 tensor cores (sm_100a).
+//
+// One CTA per (chunk, qk head); it serves the G value heads that share the qk
+// head.  For a chunk of n <= 64 rows with normalised k_r, q_r (q carries the
+// output scale), gates g_r, beta_r and gamma_r = sum_{s<=r} g_s:
+//
+//   D1  = [K; Q] K^T                          (tf32 MMA, M=128 N=64 K=dk)
+//   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
+//   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
+//   T   = (I + A)^{-1}                        (fp32, blocked 16x16 forward substitution)
+//   [W | U] = T [diag(beta e^gamma) K | diag(beta) V]   (tf32 MMA, M=64 N=dk+dv K=64)
+//
+// (the WY/UT form of the gated delta rule).  For the serial state pass it
+// writes, per (chunk, value head): the tile [W ; diag(e^gamma) Q], the Aqk
+// tile and the tile (diag(e^{gamma_n-gamma}) K)^T -- tf32, already in the
+// tensor core's shared-memory layout so the state pass bulk-copies them --
+// plus U (fp32) and gamma.  Operands are staged in shared memory as K-major
+// no-swizzle tiles rounded to tf32 (round to nearest); accumulators live in
+// tensor memory.  One thread issues the MMAs; all four warps read their
+// 32-lane slice of tensor memory for the CUDA-core steps.
+
+#include "gdn_internal.cuh"
+#include "gdn_tc.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int C = kChunk;
+constexpr int NT = 128;
+
+template <int DK, int DV>
+struct IntraTcSmem {
+    float kq[2 * C * DK];      // [K; Q] as a K-major tile of 128 rows
+    float bkv[(DK + DV) * C];  // [(diag(beta e^gamma) K)^T ; (diag(beta) V)^T], K-major, DK+DV rows x C
+    float t[C * C];            // T as a K-major tile, C rows x C
+    float a[C][C + 1];         // A (fp32)
+    float tf[C][C + 1];        // T (fp32)
+    float m[3][16][17];        // off-diagonal block products
+    float gam[C], beta[C], eg[C];
+    unsigned long long bar;
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ void store_f4(float* tile, uint32_t off, float4 v) {
+    *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + off) = v;
+}
+
+// idx -> (row, first column) of a K-major tile with R rows, chosen so that the
+// 32 lanes of a warp cover 8 consecutive rows x 4 column quads: each group of
+// 8 lanes then stores one contiguous 128-byte core matrix (no bank conflicts,
+// full 128-byte segments when the tile is written to global memory).
+template <int R>
+__device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
+    const int rr = idx & 7, cc = (idx >> 3) & 3, rest = idx >> 5;
+    const int rg = rest % (R / 8), cg = rest / (R / 8);
+    r = 8 * rg + rr;
+    k4 = 4 * (4 * cg + cc);
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
+    if (batch_rejected(p)) return;
+    const int id = blockIdx.x, hk = blockIdx.y;
+    if (id >= p.hdr[kHdrNumChunks]) return;
+    const int4 ch = p.chunk_tab[id];
+    const int slot = p.slots[ch.x];
+    if (slot < 0 || slot >= p.P) return;
+    const LayerDims& d = p.d;
+    const int t0 = ch.y, n = ch.z, G = d.G, HV = d.HV;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    IntraTcSmem<DK, DV>& sm = *reinterpret_cast<IntraTcSmem<DK, DV>*>(smem_raw);
+    const uint32_t bar = tc::smem_u32(&sm.bar);
+
+    if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::fence_mbar_init();
+    }
+    // [K; Q] rows -> K-major tile; 8 loads in flight per thread
+    {
+        constexpr int NV = 2 * C * DK / 4;
+        static_assert(NV % (NT * 8) == 0, "tile split");
+        for (int base = 0; base < NV; base += NT * 8) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                int r, k4;
+                tile_coord<2 * C>(base + u * NT + tid, r, k4);
+                const int row = r & (C - 1);
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (row < n)
+                    v[u] = *reinterpret_cast<const float4*>((r < C ? p.kn : p.qn) +
+                                                            ((size_t)(t0 + row) * d.HK + hk) * DK + k4);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                int r, k4;
+                tile_coord<2 * C>(base + u * NT + tid, r, k4);
+                store_f4(sm.kq, tc::kmajor_off(r, k4, 2 * C), tc::round_tf32(v[u]));
+            }
+        }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tm = sm.tmem_base;
+    const uint32_t tD1 = tm, tD2 = tm + 64;  // D1: 64 columns; D2: DK + DV columns (M = 64 layout)
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    if (tid == 0) {
+        const uint32_t base = tc::smem_u32(sm.kq);
+        constexpr uint32_t idesc = tc::idesc_tf32(128, 64);
+#pragma unroll
+        for (int s = 0; s < DK / 8; ++s)
+            tc::mma_tf32(tD1, tc::desc_kmajor(base, 2 * C, s), tc::desc_kmajor(base, 2 * C, s), idesc, s > 0);
+        tc::mma_commit(bar);
+    }
+    // upper off-diagonal blocks of T are zero for every head
+    for (int e = tid; e < C * C; e += NT) {
+        const int r = e / C, s = e % C;
+        if ((s >> 4) > (r >> 4)) sm.tf[r][s] = 0.f;
+    }
+
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int j = 0; j < G && ok; ++j) {
+        const int h = hk * G + j;
+        const size_t ch_h = (size_t)id * HV + h;
+        char* WQg = reinterpret_cast<char*>(p.WQ + ch_h * (2 * C * DK));
+        char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
+        char* KTg = reinterpret_cast<char*>(p.KT + ch_h * (DK * C));
+        float* Ug = p.U + ch_h * (C * DV);
+        if (warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
+            const float2 z = make_float2(0.f, 0.f);
+            const float2 g0 = 2 * lane < n ? p.gb[(size_t)(t0 + 2 * lane) * HV + h] : z;
+            const float2 g1 = 2 * lane + 1 < n ? p.gb[(size_t)(t0 + 2 * lane + 1) * HV + h] : z;
+            const float pair = g0.x + g1.x;
+            float incl = pair;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const float gA = incl - pair + g0.x;
+            sm.gam[2 * lane] = gA;
+            sm.gam[2 * lane + 1] = incl;
+            sm.beta[2 * lane] = g0.y;
+            sm.beta[2 * lane + 1] = g1.y;
+            sm.eg[2 * lane] = expf(gA);
+            sm.eg[2 * lane + 1] = expf(incl);
+        }
+        if (j == 0) {
+            ok = tc::mbar_wait(bar, phase);
+            phase ^= 1;
+        }
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const float gl = sm.gam[n - 1];
+        {  // A (warps 0-1, k.k rows) and the masked decayed q.k tile (warps 2-3) from D1
+            const int r = (warp & 1) * 32 + lane;
+            float row[C];
+#pragma unroll
+            for (int c0 = 0; c0 < C; c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tD1 + lane_base + c0, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) row[c0 + i] = v[i];
+            }
+            tc::tmem_ld_wait();
+            const float gr = sm.gam[r], br = sm.beta[r];
+            if (warp < 2) {
+#pragma unroll
+                for (int s = 0; s < C; ++s) sm.a[r][s] = (s < r && r < n) ? br * expf(gr - sm.gam[s]) * row[s] : 0.f;
+            } else {
+#pragma unroll
+                for (int s = 0; s < C; s += 4) {
+                    float o[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        o[u] = (s + u <= r && r < n) ? tc::round_tf32(expf(gr - sm.gam[s + u]) * row[s + u]) : 0.f;
+                    store_f4(reinterpret_cast<float*>(AQg), tc::kmajor_off(r, s, C), make_float4(o[0], o[1], o[2], o[3]));
+                }
+            }
+        }
+        __syncthreads();
+        // T = (I + A)^{-1}: diagonal 16x16 blocks, one column per thread
+        if (tid < 64) {
+            const int o = 16 * (tid >> 4), c = tid & 15;
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float v = (r == c) ? 1.f : 0.f;
+#pragma unroll
+                for (int s = 0; s < r; ++s) v = fmaf(-sm.a[o + r][o + s], t[s], v);
+                t[r] = v;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sm.tf[o + r][o + c] = t[r];
+        }
+        __syncthreads();
+        // off-diagonal blocks by distance: T_ij = -T_ii (sum_{k=j}^{i-1} A_ik T_kj)
+        for (int dist = 1; dist < 4; ++dist) {
+            const int nel = (4 - dist) * 256;
+            for (int e = tid; e < nel; e += NT) {
+                const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                const int bi = blk + dist, bj = blk;
+                float acc = 0.f;
+                for (int k = bj; k < bi; ++k)
+#pragma unroll
+                    for (int s = 0; s < 16; ++s) acc = fmaf(sm.a[16 * bi + r][16 * k + s], sm.tf[16 * k + s][16 * bj + c], acc);
+                sm.m[blk][r][c] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < nel; e += NT) {
+                const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+                const int bi = blk + dist, bj = blk;
+                float acc = 0.f;
+#pragma unroll
+                for (int s = 0; s < 16; ++s) acc = fmaf(sm.tf[16 * bi + r][16 * bi + s], sm.m[blk][s][c], acc);
+                sm.tf[16 * bi + r][16 * bj + c] = -acc;
+            }
+            __syncthreads();
+        }
+        // T -> K-major tf32 tile
+        for (int idx = tid; idx < C * C / 4; idx += NT) {
+            int r, s4;
+            tile_coord<C>(idx, r, s4);
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = (s4 + u <= r) ? tc::round_tf32(sm.tf[r][s4 + u]) : 0.f;
+            store_f4(sm.t, tc::kmajor_off(r, s4, C), make_float4(v[0], v[1], v[2], v[3]));
+        }
+        // feature-major tiles: row f holds one feature across the chunk rows s (loads coalesced over f);
+        // the k rows also give the state pass its (diag(e^{gamma_n - gamma}) K)^T tile
+        {
+            constexpr int NI = (DK + DV) * (C / 4);
+            static_assert(NI % (NT * 4) == 0, "tile split");
+            for (int base = 0; base < NI; base += NT * 4) {
+                float x[4][4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * NT + tid;
+                    const int fin = idx & 31, rest = idx >> 5;
+                    const int fg = rest % ((DK + DV) / 32), q = rest / ((DK + DV) / 32);
+                    const int f = 32 * fg + fin;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int s = 4 * q + w;
+                        x[u][w] = 0.f;
+                        if (s < n)
+                            x[u][w] = f < DK ? p.kn[((size_t)(t0 + s) * d.HK + hk) * DK + f]
+                                             : p.vv[((size_t)(t0 + s) * HV + h) * DV + (f - DK)];
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * NT + tid;
+                    const int fin = idx & 31, rest = idx >> 5;
+                    const int fg = rest % ((DK + DV) / 32), q = rest / ((DK + DV) / 32);
+                    const int f = 32 * fg + fin;
+                    float b[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int s = 4 * q + w;
+                        b[w] = tc::round_tf32(x[u][w] * sm.beta[s] * (f < DK ? sm.eg[s] : 1.f));
+                    }
+                    store_f4(sm.bkv, tc::kmajor_off(f, 4 * q, DK + DV), make_float4(b[0], b[1], b[2], b[3]));
+                    if (f < DK) {
+                        float kt[4];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const int s = 4 * q + w;
+                            kt[w] = s < n ? tc::round_tf32(x[u][w] * expf(gl - sm.gam[s])) : 0.f;
+                        }
+                        store_f4(reinterpret_cast<float*>(KTg), tc::kmajor_off(f, 4 * q, DK),
+                                 make_float4(kt[0], kt[1], kt[2], kt[3]));
+                    }
+                }
+            }
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (tid == 0) {  // [W | U] = T [diag(beta e^gamma) K | diag(beta) V]   (M = 64, N = DK + DV)
+            const uint32_t bt = tc::smem_u32(sm.t), bb = tc::smem_u32(sm.bkv);
+            constexpr uint32_t idesc = tc::idesc_tf32(64, DK + DV);
+#pragma unroll
+            for (int s = 0; s < C / 8; ++s)
+                tc::mma_tf32(tD2, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bb, DK + DV, s), idesc, s > 0);
+            tc::mma_commit(bar);
+        }
+        // while the MMA runs: rows 64..127 of the [W ; Qg] tile, Qg = diag(e^gamma) Q
+        {
+            constexpr int NV = C * DK / 4;
+            static_assert(NV % (NT * 4) == 0, "tile split");
+            for (int base = 0; base < NV; base += NT * 4) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    int r, k4;
+                    tile_coord<C>(base + u * NT + tid, r, k4);
+                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (r < n) v[u] = *reinterpret_cast<const float4*>(p.qn + ((size_t)(t0 + r) * d.HK + hk) * DK + k4);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    int r, k4;
+                    tile_coord<C>(base + u * NT + tid, r, k4);
+                    const float e = sm.eg[r];
+                    const float4 q = make_float4(v[u].x * e, v[u].y * e, v[u].z * e, v[u].w * e);
+                    store_f4(reinterpret_cast<float*>(WQg), tc::kmajor_off(C + r, k4, 2 * C), tc::round_tf32(q));
+                }
+            }
+        }
+        if (tid < C) p.gam[ch_h * C + tid] = sm.gam[tid];
+        ok = tc::mbar_wait(bar, phase);
+        phase ^= 1;
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        tc::fence_after_sync();
+        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major
+            const bool valid = lane < 16;
+            const int r = warp * 16 + lane;
+#pragma unroll
+            for (int c0 = 0; c0 < DK; c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tD2 + lane_base + c0, v);
+                tc::tmem_ld_wait();
+                if (valid)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        store_f4(reinterpret_cast<float*>(WQg), tc::kmajor_off(r, c0 + 4 * q, 2 * C),
+                                 make_float4(tc::round_tf32(v[4 * q]), tc::round_tf32(v[4 * q + 1]),
+                                             tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
+            }
+#pragma unroll
+            for (int c0 = 0; c0 < DV; c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tD2 + lane_base + DK + c0, v);
+                tc::tmem_ld_wait();
+                if (valid)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<float4*>(Ug + (size_t)r * DV + c0 + 4 * q) =
+                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    }
+    if (!ok && tid == 0) raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+}  // namespace
+
+template <int DK, int DV>
+cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s) {
+    const size_t shm = sizeof(IntraTcSmem<DK, DV>);
+    cudaError_t e = cudaFuncSetAttribute(intra_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
+    if (e != cudaSuccess) return e;
+    intra_tc_kernel<DK, DV><<<dim3(p.max_chunks, p.d.HK), NT, shm, s>>>(p);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_intra<64, 64>(const ExtendArgs&, cudaStream_t);
+template cudaError_t launch_intra<64, 128>(const ExtendArgs&, cudaStream_t);
+template cudaError_t launch_intra<128, 64>(const ExtendArgs&, cudaStream_t);
+template cudaError_t launch_intra<128, 128>(const ExtendArgs&, cudaStream_t);
+
+}  // namespace gdn

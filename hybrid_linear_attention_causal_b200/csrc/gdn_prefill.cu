@@ -14,11 +14,14 @@
 //   1. chunk_map:  validates cu_seqlens and lays out the chunk table
 //   2. prep:       conv1d + SiLU, L2 norm, gates -> fp32 q, k, v, (g, beta)
 //   3. conv_tail:  writes each sequence's new conv window into its slot
-//   4. intra:      per (chunk, value head): gamma, A, W, U, masked decayed q.k
-//   5. state:      per (sequence, value head, dv tile): the serial chunk pass
-//                  V' = U - W S, the outputs and S <- e^{gamma_n} S + K~^T V'
-// Every intermediate is fp32: the parity bar leaves no room for bf16 rounding
-// of q, k, v, W, U or V' (each alone adds ~1.7e-3 relative error).
+//   4. intra:      per (chunk, qk head) on tensor cores: gamma, A, T, W, U and
+//                  the masked decayed q.k of each value head (gdn_intra_tc.cu)
+//   5. state:      per (sequence, value head) on tensor cores: the serial chunk
+//                  pass V' = U - W S, the outputs and S <- e^{gamma_n} S + K~^T V'
+//                  (gdn_state_tc.cu)
+// Every intermediate is fp32 and every tensor-core operand is rounded to tf32
+// (round to nearest): the parity bar leaves no room for bf16 rounding of q, k,
+// v, W, U or V', and truncating to tf32 instead of rounding fails it too.
 
 #include "gdn_internal.cuh"
 
@@ -26,8 +29,6 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-
-__device__ __forceinline__ bool batch_rejected(const ExtendArgs& p) { return p.hdr[kHdrNumChunks] == 0; }
 
 // ---------------------------------------------------------------- 1. chunk map
 
@@ -190,244 +191,14 @@ __global__ void __launch_bounds__(256) conv_tail_kernel(ExtendArgs p) {
 }
 
 // ---------------------------------------------------------------- 4. intra
-
-template <int DK, int DV>
-struct IntraSmem {
-    float K[C][DK + 1];
-    float Q[C][DK + 1];
-    float X[C][DK + DV + 1];
-    float A[C][C + 1];
-    float gam[C];
-    float beta[C];
-};
-
-template <int DK, int DV>
-__global__ void __launch_bounds__(256) intra_kernel(ExtendArgs p) {
-    if (batch_rejected(p)) return;
-    const int id = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-    if (id >= p.hdr[kHdrNumChunks]) return;
-    const int4 ch = p.chunk_tab[id];
-    const int slot = p.slots[ch.x];
-    if (slot < 0 || slot >= p.P) return;
-    const LayerDims& d = p.d;
-    const int hk = h / d.G, t0 = ch.y, n = ch.z;
-    extern __shared__ float4 smem4[];
-    IntraSmem<DK, DV>& sm = *reinterpret_cast<IntraSmem<DK, DV>*>(smem4);
-
-    for (int e = tid; e < C * DK; e += 256) {
-        const int r = e / DK, i = e % DK;
-        const bool live = r < n;
-        sm.K[r][i] = live ? p.kn[((size_t)(t0 + r) * d.HK + hk) * DK + i] : 0.f;
-        sm.Q[r][i] = live ? p.qn[((size_t)(t0 + r) * d.HK + hk) * DK + i] : 0.f;
-    }
-    for (int e = tid; e < C * DV; e += 256) {
-        const int r = e / DV, j = e % DV;
-        sm.X[r][DK + j] = r < n ? p.vv[((size_t)(t0 + r) * d.HV + h) * DV + j] : 0.f;
-    }
-    if (tid < 32) {  // inclusive scan of g over the chunk (two rows per lane)
-        float2 gb0 = tid * 2 < n ? p.gb[(size_t)(t0 + tid * 2) * d.HV + h] : make_float2(0.f, 0.f);
-        float2 gb1 = tid * 2 + 1 < n ? p.gb[(size_t)(t0 + tid * 2 + 1) * d.HV + h] : make_float2(0.f, 0.f);
-        float pair = gb0.x + gb1.x;
-        float incl = pair;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (tid >= o) incl += v;
-        }
-        const float excl = incl - pair;
-        sm.gam[tid * 2] = excl + gb0.x;
-        sm.gam[tid * 2 + 1] = incl;
-        sm.beta[tid * 2] = gb0.y;
-        sm.beta[tid * 2 + 1] = gb1.y;
-    }
-    __syncthreads();
-
-    // k.k (s < r) and q.k (s <= r): thread owns row r = tid/4 and columns s = tid%4 + 4m
-    {
-        const int r = tid >> 2, s0 = tid & 3;
-        float kk[16], qk[16];
-#pragma unroll
-        for (int m = 0; m < 16; ++m) { kk[m] = 0.f; qk[m] = 0.f; }
-        for (int i = 0; i < DK; ++i) {
-            const float kr = sm.K[r][i], qr = sm.Q[r][i];
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float ks = sm.K[s0 + 4 * m][i];
-                kk[m] = fmaf(kr, ks, kk[m]);
-                qk[m] = fmaf(qr, ks, qk[m]);
-            }
-        }
-        const float gr = sm.gam[r], br = sm.beta[r];
-        float* aq = p.Aqk + (((size_t)id * d.HV + h) * C + r) * C;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int s = s0 + 4 * m;
-            const bool valid = r < n && s < n;
-            const float dec = valid && s <= r ? expf(gr - sm.gam[s]) : 0.f;
-            sm.A[r][s] = (s < r) ? br * dec * kk[m] : 0.f;
-            aq[s] = dec * qk[m];
-        }
-    }
-    // right-hand sides: rows of diag(beta e^gamma) K and diag(beta) V
-    for (int e = tid; e < C * DK; e += 256) {
-        const int r = e / DK, i = e % DK;
-        sm.X[r][i] = sm.beta[r] * expf(sm.gam[r]) * sm.K[r][i];
-    }
-    for (int e = tid; e < C * DV; e += 256) {
-        const int r = e / DV, j = e % DV;
-        sm.X[r][DK + j] *= sm.beta[r];
-    }
-    __syncthreads();
-    // forward substitution, one column per thread: X[r] -= sum_{s<r} A[r,s] X[s]
-    for (int col = tid; col < DK + DV; col += 256) {
-        for (int r = 1; r < n; ++r) {
-            float acc = sm.X[r][col];
-            for (int s = 0; s < r; ++s) acc = fmaf(-sm.A[r][s], sm.X[s][col], acc);
-            sm.X[r][col] = acc;
-        }
-    }
-    __syncthreads();
-    float* Wd = p.W + ((size_t)id * d.HV + h) * C * DK;
-    float* Ud = p.U + ((size_t)id * d.HV + h) * C * DV;
-    for (int e = tid; e < C * DK; e += 256) Wd[e] = sm.X[e / DK][e % DK];
-    for (int e = tid; e < C * DV; e += 256) Ud[e] = sm.X[e / DV][DK + e % DV];
-    if (tid < C) p.gam[((size_t)id * d.HV + h) * C + tid] = sm.gam[tid];
-}
+// on tensor cores, in gdn_intra_tc.cu
 
 // ---------------------------------------------------------------- 5. state pass
-
-template <int DK, int DT>
-struct StateSmem {
-    float S[DK][DT];
-    float W[C][DK];
-    float Q[C][DK];
-    float K[C][DK];
-    float Aqk[C][C];
-    float U[C][DT];
-    float Vn[C][DT];
-    float gam[C];
-};
-
-template <typename T, int DK, int DV, int DT>
-__global__ void __launch_bounds__(256) state_kernel(ExtendArgs p) {
-    static_assert(DT == 32, "one warp spans the dv tile");
-    if (batch_rejected(p)) return;
-    const int nseq = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DT, tid = threadIdx.x;
-    const LayerDims& d = p.d;
-    const int hk = h / d.G;
-    const int len = p.cu[nseq + 1] - p.cu[nseq];
-    if (len == 0) return;
-    const int slot = p.slots[nseq];
-    T* out = reinterpret_cast<T*>(p.out);
-    if (slot < 0 || slot >= p.P) {
-        if (slot >= p.P && tid == 0 && h == 0 && blockIdx.z == 0) raise_error(p.hdr, GDN_DEVERR_SLOT_RANGE);
-        for (int e = tid; e < len * DT; e += 256) {
-            const int r = e / DT, j = e % DT;
-            out[((size_t)(p.cu[nseq] + r) * d.HV + h) * DV + j0 + j] = from_f<T>(0.f);
-        }
-        return;
-    }
-    extern __shared__ float4 smem4[];
-    StateSmem<DK, DT>& sm = *reinterpret_cast<StateSmem<DK, DT>*>(smem4);
-    const bool init = p.has_init ? p.has_init[nseq] != 0 : true;
-    float* Sg = p.ssm_state + ((size_t)slot * d.HV + h) * DK * DV;
-    for (int e = tid; e < DK * DT; e += 256) {
-        const int i = e / DT, j = e % DT;
-        sm.S[i][j] = init ? Sg[(size_t)i * DV + j0 + j] : 0.f;
-    }
-    const int lane = tid & 31, wg = tid >> 5;  // lane = column j, warp = row group
-    const int c_begin = p.seq_chunk0[nseq], c_end = p.seq_chunk0[nseq + 1];
-    for (int id = c_begin; id < c_end; ++id) {
-        const int4 ch = p.chunk_tab[id];
-        const int t0 = ch.y, n = ch.z;
-        const float* Wg = p.W + ((size_t)id * d.HV + h) * C * DK;
-        const float* Ug = p.U + ((size_t)id * d.HV + h) * C * DV;
-        const float* Ag = p.Aqk + ((size_t)id * d.HV + h) * C * C;
-        for (int e = tid; e < C * DK / 4; e += 256) {
-            const int r = (e * 4) / DK, i = (e * 4) % DK;
-            reinterpret_cast<float4*>(&sm.W[r][i])[0] = reinterpret_cast<const float4*>(Wg)[e];
-            const bool live = r < n;
-            const size_t qo = ((size_t)(t0 + r) * d.HK + hk) * DK + i;
-            reinterpret_cast<float4*>(&sm.Q[r][i])[0] =
-                live ? *reinterpret_cast<const float4*>(p.qn + qo) : make_float4(0.f, 0.f, 0.f, 0.f);
-            reinterpret_cast<float4*>(&sm.K[r][i])[0] =
-                live ? *reinterpret_cast<const float4*>(p.kn + qo) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int e = tid; e < C * C / 4; e += 256)
-            reinterpret_cast<float4*>(&sm.Aqk[0][0])[e] = reinterpret_cast<const float4*>(Ag)[e];
-        for (int e = tid; e < C * DT; e += 256) {
-            const int r = e / DT, j = e % DT;
-            sm.U[r][j] = Ug[(size_t)r * DV + j0 + j];
-        }
-        if (tid < C) sm.gam[tid] = p.gam[((size_t)id * d.HV + h) * C + tid];
-        __syncthreads();
-        // V' = U - W S   (rows r = wg + 8m)
-        {
-            float acc[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) acc[m] = sm.U[wg + 8 * m][lane];
-            for (int i = 0; i < DK; ++i) {
-                const float sv = sm.S[i][lane];
-#pragma unroll
-                for (int m = 0; m < 8; ++m) acc[m] = fmaf(-sm.W[wg + 8 * m][i], sv, acc[m]);
-            }
-#pragma unroll
-            for (int m = 0; m < 8; ++m) sm.Vn[wg + 8 * m][lane] = acc[m];
-        }
-        __syncthreads();
-        // outputs: e^{gamma_r} q_r^T S + sum_{s<=r} Aqk[r,s] V'_s
-        {
-            float acc[8];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-            for (int i = 0; i < DK; ++i) {
-                const float sv = sm.S[i][lane];
-#pragma unroll
-                for (int m = 0; m < 8; ++m) acc[m] = fmaf(sm.Q[wg + 8 * m][i], sv, acc[m]);
-            }
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int r = wg + 8 * m;
-                float o = expf(sm.gam[r]) * acc[m];
-                for (int s = 0; s <= r; ++s) o = fmaf(sm.Aqk[r][s], sm.Vn[s][lane], o);
-                if (r < n) out[((size_t)(t0 + r) * d.HV + h) * DV + j0 + lane] = from_f<T>(o);
-            }
-        }
-        // S <- e^{gamma_n} S + sum_r e^{gamma_n - gamma_r} k_r V'_r^T   (rows i = wg + 8m)
-        {
-            const float gl = sm.gam[n - 1];
-            float acc[DK / 8];
-#pragma unroll
-            for (int m = 0; m < DK / 8; ++m) acc[m] = expf(gl) * sm.S[wg + 8 * m][lane];
-            for (int r = 0; r < n; ++r) {
-                const float vr = sm.Vn[r][lane] * expf(gl - sm.gam[r]);
-#pragma unroll
-                for (int m = 0; m < DK / 8; ++m) acc[m] = fmaf(sm.K[r][wg + 8 * m], vr, acc[m]);
-            }
-            __syncthreads();
-#pragma unroll
-            for (int m = 0; m < DK / 8; ++m) sm.S[wg + 8 * m][lane] = acc[m];
-        }
-        __syncthreads();
-    }
-    for (int e = tid; e < DK * DT; e += 256) {
-        const int i = e / DT, j = e % DT;
-        Sg[(size_t)i * DV + j0 + j] = sm.S[i][j];
-    }
-}
+// on tensor cores, in gdn_state_tc.cu
 
 template <typename T, int DK, int DV>
 cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
-    constexpr int DT = 32;
-    const size_t shm_intra = sizeof(IntraSmem<DK, DV>);
-    const size_t shm_state = sizeof(StateSmem<DK, DT>);
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(intra_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)shm_intra)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(state_kernel<T, DK, DV, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)shm_state)) != cudaSuccess)
-        return e;
     mark_launch(s, 0);
     chunk_map_kernel<<<1, 1024, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -438,11 +209,9 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 3);
-    intra_kernel<DK, DV><<<dim3(p.max_chunks, p.d.HV), 256, shm_intra, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_intra<DK, DV>(p, s)) != cudaSuccess) return e;
     mark_launch(s, 4);
-    state_kernel<T, DK, DV, DT><<<dim3(p.N, p.d.HV, DV / DT), 256, shm_state, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_state<T, DK, DV>(p, s)) != cudaSuccess) return e;
     mark_launch(s, 5);
     return cudaSuccess;
 }
@@ -453,16 +222,18 @@ size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max
     const size_t mc = (size_t)max_T / C + (size_t)max_N + 1;
     if (max_chunks_out) *max_chunks_out = (int)mc;
     auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+    const size_t per = mc * d.HV * sizeof(float);
     size_t off = kHeaderBytes;
     off += al(mc * sizeof(int4));
     off += al(((size_t)max_N + 1) * sizeof(int32_t));
     off += al((size_t)max_T * d.HK * d.dk * sizeof(float)) * 2;
     off += al((size_t)max_T * d.HV * d.dv * sizeof(float));
     off += al((size_t)max_T * d.HV * sizeof(float2));
-    off += al(mc * d.HV * C * d.dk * sizeof(float));
-    off += al(mc * d.HV * C * d.dv * sizeof(float));
-    off += al(mc * d.HV * C * C * sizeof(float));
-    off += al(mc * d.HV * C * sizeof(float));
+    off += al(per * 2 * C * d.dk);
+    off += al(per * C * C);
+    off += al(per * d.dk * C);
+    off += al(per * C * d.dv);
+    off += al(per * C);
     return off;
 }
 
@@ -472,6 +243,7 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
     extend_workspace_bytes(d, max_N, max_T, &mc);
     e.max_chunks = mc;
     auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+    const size_t per = (size_t)mc * d.HV * sizeof(float);
     char* base = static_cast<char*>(ws);
     e.hdr = reinterpret_cast<int32_t*>(base);
     size_t off = kHeaderBytes;
@@ -481,9 +253,10 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
     e.kn = reinterpret_cast<float*>(base + off); off += al((size_t)max_T * d.HK * d.dk * sizeof(float));
     e.vv = reinterpret_cast<float*>(base + off); off += al((size_t)max_T * d.HV * d.dv * sizeof(float));
     e.gb = reinterpret_cast<float2*>(base + off); off += al((size_t)max_T * d.HV * sizeof(float2));
-    e.W = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HV * C * d.dk * sizeof(float));
-    e.U = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HV * C * d.dv * sizeof(float));
-    e.Aqk = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HV * C * C * sizeof(float));
+    e.WQ = reinterpret_cast<float*>(base + off); off += al(per * 2 * C * d.dk);
+    e.AQ = reinterpret_cast<float*>(base + off); off += al(per * C * C);
+    e.KT = reinterpret_cast<float*>(base + off); off += al(per * d.dk * C);
+    e.U = reinterpret_cast<float*>(base + off); off += al(per * C * d.dv);
     e.gam = reinterpret_cast<float*>(base + off);
 }
 

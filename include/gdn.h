@@ -86,6 +86,7 @@ typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
 /* device error bits (sticky word at the start of the workspace) */
 #define GDN_DEVERR_SLOT_RANGE 0x1 /* a state index >= P was skipped */
 #define GDN_DEVERR_SEQLENS 0x2    /* cu_seqlens not non-decreasing from 0 to T; the batch was skipped */
+#define GDN_DEVERR_TIMEOUT 0x4    /* a tensor-core wait gave up after its time limit; results are invalid */
 
 /* element types */
 #define GDN_DTYPE_F32 0

@@ -4,11 +4,14 @@
 // head.  For a chunk of n <= 64 rows with normalised k_r, q_r (q carries the
 // output scale), gates g_r, beta_r and gamma_r = sum_{s<=r} g_s:
 //
+// The prep kernel's [K ; Q] tile and the V^T tiles and gates of the value
+// heads arrive by asynchronous bulk copies (two value heads in flight).
+//
 //   D1  = [K; Q] K^T                          (tf32 MMA, M=128 N=64 K=dk)
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
 //   T   = (I + A)^{-1}                        (fp32, blocked 16x16 forward substitution)
-//   [W | U] = T [diag(beta e^gamma) K | diag(beta) V]   (tf32 MMA, M=64 N=dk+dv K=64)
+//   W   = T diag(beta e^gamma) K, U = T diag(beta) V   (tf32 MMAs, M=64 K=64)
 //
 // (the WY/UT form of the gated delta rule).  For the serial state pass it
 // writes, per (chunk, value head): the tile [W ; diag(e^gamma) Q], the Aqk
@@ -30,25 +33,29 @@ constexpr int NT = 128;
 
 template <int DK, int DV>
 struct IntraTcSmem {
-    float kq[2 * C * DK];      // [K; Q] as a K-major tile of 128 rows
-    float bkv[(DK + DV) * C];  // [(diag(beta e^gamma) K)^T ; (diag(beta) V)^T], K-major, DK+DV rows x C
-    float t[C * C];            // T as a K-major tile, C rows x C
-    float a[C][C + 1];         // A (fp32)
-    float tf[C][C + 1];        // T (fp32)
-    float m[3][16][17];        // off-diagonal block products
+    float kq[2 * C * DK];  // [K ; Q*scale] tile from the prep kernel (bulk copy), K-major, 128 rows
+    float bk[DK * C];      // (diag(beta e^gamma) K)^T, K-major, DK rows x C
+    float bv[2][DV * C];   // V^T tiles (bulk copies, two heads in flight), scaled in place by beta
+    float t[C * C];        // T as a K-major tile, C rows x C
+    float a[C][C + 1];     // A (fp32)
+    float tf[C][C + 1];    // T (fp32)
+    float m[3][16][17];    // off-diagonal block products
+    float2 gb[2][C];       // (g, beta) of the two heads in flight
     float gam[C], beta[C], eg[C];
-    unsigned long long bar;
+    unsigned long long bar_mma, bar_kq, bar_v[2];
     uint32_t tmem_base;
 };
 
 __device__ __forceinline__ void store_f4(float* tile, uint32_t off, float4 v) {
     *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + off) = v;
 }
+__device__ __forceinline__ float load_f(const float* tile, uint32_t off) {
+    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(tile) + off);
+}
 
 // idx -> (row, first column) of a K-major tile with R rows, chosen so that the
 // 32 lanes of a warp cover 8 consecutive rows x 4 column quads: each group of
-// 8 lanes then stores one contiguous 128-byte core matrix (no bank conflicts,
-// full 128-byte segments when the tile is written to global memory).
+// 8 lanes then touches one contiguous 128-byte core matrix.
 template <int R>
 __device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
     const int rr = idx & 7, cc = (idx >> 3) & 3, rest = idx >> 5;
@@ -66,75 +73,69 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
     const int slot = p.slots[ch.x];
     if (slot < 0 || slot >= p.P) return;
     const LayerDims& d = p.d;
-    const int t0 = ch.y, n = ch.z, G = d.G, HV = d.HV;
+    const int n = ch.z, G = d.G, HV = d.HV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     IntraTcSmem<DK, DV>& sm = *reinterpret_cast<IntraTcSmem<DK, DV>*>(smem_raw);
-    const uint32_t bar = tc::smem_u32(&sm.bar);
+    const uint32_t bar = tc::smem_u32(&sm.bar_mma), bar_kq = tc::smem_u32(&sm.bar_kq);
+    constexpr uint32_t KQ_BYTES = 2 * C * DK * 4, VT_BYTES = DV * C * 4, GB_BYTES = C * 8;
+    auto fetch_v = [&](int jj) {  // V^T tile and gates of value head hk*G + jj into buffer jj & 1
+        const int b = jj & 1;
+        const size_t ch_h = (size_t)id * HV + hk * G + jj;
+        const uint32_t bv = tc::smem_u32(&sm.bar_v[b]);
+        tc::mbar_expect_tx(bv, VT_BYTES + GB_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.bv[b]), p.VT + ch_h * (DV * C), VT_BYTES, bv);
+        tc::bulk_g2s(tc::smem_u32(sm.gb[b]), p.GB + ch_h * C, GB_BYTES, bv);
+    };
 
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
+        tc::mbar_init(bar_kq, 1);
+        tc::mbar_init(tc::smem_u32(&sm.bar_v[0]), 1);
+        tc::mbar_init(tc::smem_u32(&sm.bar_v[1]), 1);
         tc::fence_mbar_init();
+        tc::mbar_expect_tx(bar_kq, KQ_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.kq), p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK), KQ_BYTES, bar_kq);
+        fetch_v(0);
+        if (G > 1) fetch_v(1);
     }
-    // [K; Q] rows -> K-major tile; 8 loads in flight per thread
-    {
-        constexpr int NV = 2 * C * DK / 4;
-        static_assert(NV % (NT * 8) == 0, "tile split");
-        for (int base = 0; base < NV; base += NT * 8) {
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                int r, k4;
-                tile_coord<2 * C>(base + u * NT + tid, r, k4);
-                const int row = r & (C - 1);
-                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (row < n)
-                    v[u] = *reinterpret_cast<const float4*>((r < C ? p.kn : p.qn) +
-                                                            ((size_t)(t0 + row) * d.HK + hk) * DK + k4);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                int r, k4;
-                tile_coord<2 * C>(base + u * NT + tid, r, k4);
-                store_f4(sm.kq, tc::kmajor_off(r, k4, 2 * C), tc::round_tf32(v[u]));
-            }
-        }
-    }
-    tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
-    const uint32_t tD1 = tm, tD2 = tm + 64;  // D1: 64 columns; D2: DK + DV columns (M = 64 layout)
+    const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;  // D1: 64 cols; W, U: M = 64 layout
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    bool ok = true;
     if (tid == 0) {
-        const uint32_t base = tc::smem_u32(sm.kq);
-        constexpr uint32_t idesc = tc::idesc_tf32(128, 64);
+        ok = tc::mbar_wait(bar_kq, 0);
+        if (ok) {  // D1 = [K ; Q] K^T
+            const uint32_t base = tc::smem_u32(sm.kq);
+            constexpr uint32_t idesc = tc::idesc_tf32(128, 64);
 #pragma unroll
-        for (int s = 0; s < DK / 8; ++s)
-            tc::mma_tf32(tD1, tc::desc_kmajor(base, 2 * C, s), tc::desc_kmajor(base, 2 * C, s), idesc, s > 0);
-        tc::mma_commit(bar);
+            for (int s = 0; s < DK / 8; ++s)
+                tc::mma_tf32(tD1, tc::desc_kmajor(base, 2 * C, s), tc::desc_kmajor(base, 2 * C, s), idesc, s > 0);
+            tc::mma_commit(bar);
+        }
     }
     // upper off-diagonal blocks of T are zero for every head
     for (int e = tid; e < C * C; e += NT) {
         const int r = e / C, s = e % C;
         if ((s >> 4) > (r >> 4)) sm.tf[r][s] = 0.f;
     }
+    ok = __syncthreads_and(ok);
 
-    uint32_t phase = 0;
-    bool ok = true;
+    uint32_t ph_mma = 0;
     for (int j = 0; j < G && ok; ++j) {
-        const int h = hk * G + j;
+        const int h = hk * G + j, b = j & 1;
         const size_t ch_h = (size_t)id * HV + h;
         char* WQg = reinterpret_cast<char*>(p.WQ + ch_h * (2 * C * DK));
         char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
         char* KTg = reinterpret_cast<char*>(p.KT + ch_h * (DK * C));
         float* Ug = p.U + ch_h * (C * DV);
-        if (warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
-            const float2 z = make_float2(0.f, 0.f);
-            const float2 g0 = 2 * lane < n ? p.gb[(size_t)(t0 + 2 * lane) * HV + h] : z;
-            const float2 g1 = 2 * lane + 1 < n ? p.gb[(size_t)(t0 + 2 * lane + 1) * HV + h] : z;
+        bool okv = tc::mbar_wait(tc::smem_u32(&sm.bar_v[b]), (uint32_t)(j >> 1) & 1u);
+        if (okv && warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
+            const float2 g0 = sm.gb[b][2 * lane], g1 = sm.gb[b][2 * lane + 1];
             const float pair = g0.x + g1.x;
             float incl = pair;
 #pragma unroll
@@ -151,10 +152,10 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             sm.eg[2 * lane + 1] = expf(incl);
         }
         if (j == 0) {
-            ok = tc::mbar_wait(bar, phase);
-            phase ^= 1;
+            okv = okv && tc::mbar_wait(bar, ph_mma);
+            ph_mma ^= 1;
         }
-        ok = __syncthreads_and(ok);
+        ok = __syncthreads_and(okv);
         if (!ok) break;
         tc::fence_after_sync();
         const float gl = sm.gam[n - 1];
@@ -232,102 +233,71 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             for (int u = 0; u < 4; ++u) v[u] = (s4 + u <= r) ? tc::round_tf32(sm.tf[r][s4 + u]) : 0.f;
             store_f4(sm.t, tc::kmajor_off(r, s4, C), make_float4(v[0], v[1], v[2], v[3]));
         }
-        // feature-major tiles: row f holds one feature across the chunk rows s (loads coalesced over f);
-        // the k rows also give the state pass its (diag(e^{gamma_n - gamma}) K)^T tile
-        {
-            constexpr int NI = (DK + DV) * (C / 4);
-            static_assert(NI % (NT * 4) == 0, "tile split");
-            for (int base = 0; base < NI; base += NT * 4) {
-                float x[4][4];
+        // (diag(beta e^gamma) K)^T into shared memory and (diag(e^{gamma_n - gamma}) K)^T to the
+        // workspace, both from the k rows of the [K ; Q] tile (row f = one feature across the rows s)
+        for (int idx = tid; idx < DK * (C / 4); idx += NT) {
+            const int f = idx % DK, q = idx / DK;
+            float kb[4], kt[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int idx = base + u * NT + tid;
-                    const int fin = idx & 31, rest = idx >> 5;
-                    const int fg = rest % ((DK + DV) / 32), q = rest / ((DK + DV) / 32);
-                    const int f = 32 * fg + fin;
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const int s = 4 * q + w;
-                        x[u][w] = 0.f;
-                        if (s < n)
-                            x[u][w] = f < DK ? p.kn[((size_t)(t0 + s) * d.HK + hk) * DK + f]
-                                             : p.vv[((size_t)(t0 + s) * HV + h) * DV + (f - DK)];
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int idx = base + u * NT + tid;
-                    const int fin = idx & 31, rest = idx >> 5;
-                    const int fg = rest % ((DK + DV) / 32), q = rest / ((DK + DV) / 32);
-                    const int f = 32 * fg + fin;
-                    float b[4];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const int s = 4 * q + w;
-                        b[w] = tc::round_tf32(x[u][w] * sm.beta[s] * (f < DK ? sm.eg[s] : 1.f));
-                    }
-                    store_f4(sm.bkv, tc::kmajor_off(f, 4 * q, DK + DV), make_float4(b[0], b[1], b[2], b[3]));
-                    if (f < DK) {
-                        float kt[4];
-#pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const int s = 4 * q + w;
-                            kt[w] = s < n ? tc::round_tf32(x[u][w] * expf(gl - sm.gam[s])) : 0.f;
-                        }
-                        store_f4(reinterpret_cast<float*>(KTg), tc::kmajor_off(f, 4 * q, DK),
-                                 make_float4(kt[0], kt[1], kt[2], kt[3]));
-                    }
-                }
+            for (int w = 0; w < 4; ++w) {
+                const int s = 4 * q + w;
+                const float kv = load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
+                kb[w] = tc::round_tf32(kv * sm.beta[s] * sm.eg[s]);
+                kt[w] = s < n ? tc::round_tf32(kv * expf(gl - sm.gam[s])) : 0.f;
             }
+            store_f4(sm.bk, tc::kmajor_off(f, 4 * q, DK), make_float4(kb[0], kb[1], kb[2], kb[3]));
+            store_f4(reinterpret_cast<float*>(KTg), tc::kmajor_off(f, 4 * q, DK), make_float4(kt[0], kt[1], kt[2], kt[3]));
+        }
+        // V^T scaled by beta, in place (tile layout unchanged)
+        for (int idx = tid; idx < DV * (C / 4); idx += NT) {
+            int f, s4;
+            tile_coord<DV>(idx, f, s4);
+            const uint32_t off = tc::kmajor_off(f, s4, DV);
+            float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.bv[b]) + off);
+            v = make_float4(tc::round_tf32(v.x * sm.beta[s4]), tc::round_tf32(v.y * sm.beta[s4 + 1]),
+                            tc::round_tf32(v.z * sm.beta[s4 + 2]), tc::round_tf32(v.w * sm.beta[s4 + 3]));
+            store_f4(sm.bv[b], off, v);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        if (tid == 0) {  // [W | U] = T [diag(beta e^gamma) K | diag(beta) V]   (M = 64, N = DK + DV)
-            const uint32_t bt = tc::smem_u32(sm.t), bb = tc::smem_u32(sm.bkv);
-            constexpr uint32_t idesc = tc::idesc_tf32(64, DK + DV);
+        if (tid == 0) {  // W = T diag(beta e^gamma) K,  U = T diag(beta) V   (M = 64)
+            const uint32_t bt = tc::smem_u32(sm.t), bkk = tc::smem_u32(sm.bk), bvv = tc::smem_u32(sm.bv[b]);
+            constexpr uint32_t iw = tc::idesc_tf32(64, DK), iu = tc::idesc_tf32(64, DV);
 #pragma unroll
             for (int s = 0; s < C / 8; ++s)
-                tc::mma_tf32(tD2, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bb, DK + DV, s), idesc, s > 0);
+                tc::mma_tf32(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
+#pragma unroll
+            for (int s = 0; s < C / 8; ++s)
+                tc::mma_tf32(tU, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bvv, DV, s), iu, s > 0);
             tc::mma_commit(bar);
         }
-        // while the MMA runs: rows 64..127 of the [W ; Qg] tile, Qg = diag(e^gamma) Q
-        {
-            constexpr int NV = C * DK / 4;
-            static_assert(NV % (NT * 4) == 0, "tile split");
-            for (int base = 0; base < NV; base += NT * 4) {
-                float4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    int r, k4;
-                    tile_coord<C>(base + u * NT + tid, r, k4);
-                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (r < n) v[u] = *reinterpret_cast<const float4*>(p.qn + ((size_t)(t0 + r) * d.HK + hk) * DK + k4);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    int r, k4;
-                    tile_coord<C>(base + u * NT + tid, r, k4);
-                    const float e = sm.eg[r];
-                    const float4 q = make_float4(v[u].x * e, v[u].y * e, v[u].z * e, v[u].w * e);
-                    store_f4(reinterpret_cast<float*>(WQg), tc::kmajor_off(C + r, k4, 2 * C), tc::round_tf32(q));
-                }
-            }
+        // while the MMA runs: rows 64..127 of the [W ; Qg] tile, Qg = diag(e^gamma) Q (same tile offsets)
+        for (int idx = tid; idx < C * DK / 4; idx += NT) {
+            int r, k4;
+            tile_coord<C>(idx, r, k4);
+            const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
+            const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
+            const float e = sm.eg[r];
+            store_f4(reinterpret_cast<float*>(WQg), off,
+                     make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
+                                 tc::round_tf32(q.w * e)));
         }
         if (tid < C) p.gam[ch_h * C + tid] = sm.gam[tid];
-        ok = tc::mbar_wait(bar, phase);
-        phase ^= 1;
+        ok = tc::mbar_wait(bar, ph_mma);
+        ph_mma ^= 1;
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc::fence_after_sync();
+        if (tid == 0 && j + 2 < G) fetch_v(j + 2);  // buffer b is free again
         {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major
             const bool valid = lane < 16;
             const int r = warp * 16 + lane;
 #pragma unroll
             for (int c0 = 0; c0 < DK; c0 += 16) {
                 float v[16];
-                tc::tmem_ld16(tD2 + lane_base + c0, v);
+                tc::tmem_ld16(tW + lane_base + c0, v);
                 tc::tmem_ld_wait();
                 if (valid)
 #pragma unroll
@@ -339,7 +309,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
 #pragma unroll
             for (int c0 = 0; c0 < DV; c0 += 16) {
                 float v[16];
-                tc::tmem_ld16(tD2 + lane_base + DK + c0, v);
+                tc::tmem_ld16(tU + lane_base + c0, v);
                 tc::tmem_ld_wait();
                 if (valid)
 #pragma unroll
@@ -352,7 +322,13 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         __syncthreads();
         tc::fence_after_sync();
     }
-    if (!ok && tid == 0) raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+    if (!ok && tid == 0) {
+        raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+        // let copies already in flight land before the CTA's shared memory goes away
+        for (int b = 0; b < 2; ++b)
+            for (uint32_t par = 0; par < 2; ++par) tc::mbar_wait(tc::smem_u32(&sm.bar_v[b]), par, 100000000ull);
+        tc::mbar_wait(bar_kq, 0, 100000000ull);
+    }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tm, 512);

@@ -12,7 +12,7 @@
 //
 // Launch sequence (all stream-ordered, no host synchronisation):
 //   1. chunk_map:  validates cu_seqlens and lays out the chunk table
-//   2. prep:       conv1d + SiLU, L2 norm, gates -> fp32 q, k, v, (g, beta)
+//   2. prep:       per (chunk, head): conv1d + SiLU, L2 norm, gates -> tiles
 //   3. conv_tail:  writes each sequence's new conv window into its slot
 //   4. intra:      per (chunk, qk head) on tensor cores: gamma, A, T, W, U and
 //                  the masked decayed q.k of each value head (gdn_intra_tc.cu)
@@ -24,6 +24,7 @@
 // v, W, U or V', and truncating to tf32 instead of rounding fails it too.
 
 #include "gdn_internal.cuh"
+#include "gdn_tc.cuh"
 
 namespace gdn {
 namespace {
@@ -90,76 +91,174 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
 
 // ---------------------------------------------------------------- 2. prep
 
-__device__ __forceinline__ int seq_of_row(const int32_t* cu, int N, int t) {
-    int lo = 0, hi = N - 1;  // last n with cu[n] <= t
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (cu[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
+// One CTA per (chunk, head unit): a unit is either a qk head (its q and k
+// channels) or a value head (its v channels and gates).  The chunk's raw rows
+// and the 3 rows before it (from the previous chunk of the same sequence, or
+// from the conv-state slot for a sequence's first chunk) are staged in shared
+// memory; every output row is then conv1d + SiLU (+ L2 norm for q, k) of
+// shared-memory data.  Results are assembled as tiles in the tensor core's
+// shared-memory layout and written with one bulk store:
+//   qk unit: [K ; Q*scale] tf32, K-major, 128 rows x dk
+//   v unit:  V^T fp32, K-major, dv rows x C, and (g, beta) for the C rows
+// Rows past the end of a ragged chunk are written as zeros.
+constexpr int kPrepThreads = 256;
 
-// One CTA per packed row.  Warps take whole heads: the 2*HK q/k heads are
-// normalised with a warp reduction, the HV value heads are stored as is.
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(256) prep_kernel(ExtendArgs p) {
+struct PrepShape {
+    static constexpr int NCH = 2 * DK > DV ? 2 * DK : DV;  // staged channels per row (max over units)
+    static constexpr int VE = 16 / sizeof(T);              // elements per 16-byte vector
+    static constexpr size_t XS_BYTES = (((size_t)(C + 3) * NCH * sizeof(T)) + 15) & ~(size_t)15;
+    static constexpr size_t TILE_BYTES = (2 * C * DK > DV * C ? 2 * C * DK : DV * C) * sizeof(float);
+    static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + C * sizeof(float2);
+};
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
+    using S = PrepShape<T, DK, DV>;
     if (batch_rejected(p)) return;
-    const LayerDims& d = p.d;
-    const int t = blockIdx.x, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int n = seq_of_row(p.cu, p.N, t);
-    const int slot = p.slots[n];
+    const int id = blockIdx.x, unit = blockIdx.y;
+    if (id >= p.hdr[kHdrNumChunks]) return;
+    const int4 ch = p.chunk_tab[id];
+    const int seq = ch.x, t0 = ch.y, n = ch.z, cidx = ch.w;
+    const int slot = p.slots[seq];
     if (slot < 0 || slot >= p.P) return;
-    const int pos = t - p.cu[n];
-    const bool init = p.has_init ? p.has_init[n] != 0 : true;
+    const LayerDims& d = p.d;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool isqk = unit < d.HK;
+    const int nch = isqk ? 2 * DK : DV;
+    // staged column c -> channel of mixed_qkv
+    const int hk = unit, h = unit - d.HK;
+    auto channel = [&](int c) -> int {
+        if (!isqk) return 2 * d.HK * DK + h * DV + c;
+        return c < DK ? hk * DK + c : d.HK * DK + hk * DK + (c - DK);
+    };
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T* xs = reinterpret_cast<T*>(smem_raw);  // row i <-> token t0 - 3 + i
+    float* tile = reinterpret_cast<float*>(smem_raw + S::XS_BYTES);
+    float2* gbs = reinterpret_cast<float2*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);
     const T* x = reinterpret_cast<const T*>(p.x);
+
+    // stage rows 3 .. n+2 (this chunk) with 16-byte loads; the 3 halo rows element-wise
+    {
+        const int vpr = nch / S::VE;  // vectors per row (segments never straddle a vector)
+        const int nv = n * vpr;
+        for (int base = 0; base < nv; base += kPrepThreads * 4) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = base + u * kPrepThreads + tid;
+                if (e < nv) {
+                    const int r = e / vpr, c = (e % vpr) * S::VE;
+                    v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d.conv_dim + channel(c));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = base + u * kPrepThreads + tid;
+                if (e < nv) {
+                    const int r = e / vpr, c = (e % vpr) * S::VE;
+                    *reinterpret_cast<uint4*>(xs + (size_t)(r + 3) * nch + c) = v[u];
+                }
+            }
+        }
+        const bool init = p.has_init ? p.has_init[seq] != 0 : true;
+        const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
+        for (int e = tid; e < 3 * nch; e += kPrepThreads) {
+            const int i = e / nch, c = e % nch;
+            T v;
+            if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + channel(c)];
+            else v = init ? cs[(size_t)channel(c) * 3 + i] : from_f<T>(0.f);
+            xs[(size_t)i * nch + c] = v;
+        }
+    }
+    __syncthreads();
     const T* w = reinterpret_cast<const T*>(p.conv_w);
     const T* bias = reinterpret_cast<const T*>(p.conv_b);
-    const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
-
-    auto conv = [&](int c) -> float {
-        float acc = bias ? to_f(bias[c]) : 0.f;
+    if (isqk) {
+        constexpr int PL = DK / 32;  // channels per lane and part
+        float wk[2][PL][4], bk[2][PL];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int src = pos - 3 + j;
-            float xv;
-            if (src >= 0) xv = to_f(x[(size_t)(t - 3 + j) * d.conv_dim + c]);
-            else xv = init ? to_f(cs[c * 3 + 3 + src]) : 0.f;
-            acc = fmaf(to_f(w[c * 4 + j]), xv, acc);
-        }
-        return silu_f(acc);
-    };
-
-    const int units = 2 * d.HK + d.HV;
-    for (int u = warp; u < units; u += 8) {
-        if (u < 2 * d.HK) {
-            const bool isq = u < d.HK;
-            const int hk = isq ? u : u - d.HK;
-            const int c0 = isq ? hk * DK : d.HK * DK + hk * DK;
-            float vals[DK / 32];
-            float ss = 0.f;
+        for (int part = 0; part < 2; ++part)
 #pragma unroll
-            for (int i = 0; i < DK / 32; ++i) {
-                vals[i] = conv(c0 + lane * (DK / 32) + i);
-                ss += vals[i] * vals[i];
+            for (int u = 0; u < PL; ++u) {
+                const int cg = channel(part * DK + PL * lane + u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) wk[part][u][j] = to_f(w[(size_t)cg * 4 + j]);
+                bk[part][u] = bias ? to_f(bias[cg]) : 0.f;
             }
-            ss = warp_sum(ss);
-            const float r = rsqrtf(ss + d.eps) * (isq ? d.scale : 1.0f);
-            float* dst = (isq ? p.qn : p.kn) + ((size_t)t * d.HK + hk) * DK + lane * (DK / 32);
+        for (int r = warp; r < C; r += kPrepThreads / 32) {
 #pragma unroll
-            for (int i = 0; i < DK / 32; ++i) dst[i] = vals[i] * r;
-        } else {
-            const int h = u - 2 * d.HK;
-            const int c0 = 2 * d.HK * DK + h * DV;
-            float* dst = p.vv + ((size_t)t * d.HV + h) * DV + lane * (DV / 32);
+            for (int part = 0; part < 2; ++part) {  // part 0: q (tile rows C + r), part 1: k (tile rows r)
+                float y[PL];
+                float ss = 0.f;
 #pragma unroll
-            for (int i = 0; i < DV / 32; ++i) dst[i] = conv(c0 + lane * (DV / 32) + i);
+                for (int u = 0; u < PL; ++u) {
+                    float acc = bk[part][u];
+                    if (r < n) {
+                        const int c = part * DK + PL * lane + u;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc = fmaf(wk[part][u][j], to_f(xs[(size_t)(r + j) * nch + c]), acc);
+                    }
+                    y[u] = r < n ? silu_f(acc) : 0.f;
+                    ss += y[u] * y[u];
+                }
+                ss = warp_sum(ss);
+                const float sc = (r < n) ? rsqrtf(ss + d.eps) * (part == 0 ? d.scale : 1.f) : 0.f;
+                const int row = part == 0 ? C + r : r;
+                char* dst = reinterpret_cast<char*>(tile) + tc::kmajor_off(row, PL * lane, 2 * C);
+                if constexpr (PL == 4)
+                    *reinterpret_cast<float4*>(dst) = make_float4(tc::round_tf32(y[0] * sc), tc::round_tf32(y[1] * sc),
+                                                                  tc::round_tf32(y[2] * sc), tc::round_tf32(y[3] * sc));
+                else
+                    *reinterpret_cast<float2*>(dst) = make_float2(tc::round_tf32(y[0] * sc), tc::round_tf32(y[1] * sc));
+            }
+        }
+    } else {
+        constexpr int PL = DV / 32;  // channels per lane: f = lane + 32 u
+        float wv[PL][4], bv[PL];
+#pragma unroll
+        for (int u = 0; u < PL; ++u) {
+            const int cg = channel(lane + 32 * u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) wv[u][j] = to_f(w[(size_t)cg * 4 + j]);
+            bv[u] = bias ? to_f(bias[cg]) : 0.f;
+        }
+        for (int r = warp; r < C; r += kPrepThreads / 32) {
+#pragma unroll
+            for (int u = 0; u < PL; ++u) {
+                const int f = lane + 32 * u;
+                float y = 0.f;
+                if (r < n) {
+                    float acc = bv[u];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc = fmaf(wv[u][j], to_f(xs[(size_t)(r + j) * nch + f]), acc);
+                    y = silu_f(acc);
+                }
+                *reinterpret_cast<float*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(f, r, DV)) = y;
+            }
+        }
+        if (tid < C) {
+            float2 gb = make_float2(0.f, 0.f);
+            if (tid < n) {
+                const size_t row = (size_t)(t0 + tid) * d.HV + h;
+                const float av = to_f(reinterpret_cast<const T*>(p.a)[row]);
+                const float bv2 = to_f(reinterpret_cast<const T*>(p.b)[row]);
+                gb = make_float2(-expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]), sigmoid_f(bv2));
+            }
+            gbs[tid] = gb;
         }
     }
-    for (int h = threadIdx.x; h < d.HV; h += 256) {
-        const float av = to_f(reinterpret_cast<const T*>(p.a)[(size_t)t * d.HV + h]);
-        const float bv = to_f(reinterpret_cast<const T*>(p.b)[(size_t)t * d.HV + h]);
-        const float g = -expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]);
-        p.gb[(size_t)t * d.HV + h] = make_float2(g, sigmoid_f(bv));
+    tc::fence_smem_to_async();
+    __syncthreads();
+    if (tid == 0) {
+        if (isqk) {
+            tc::bulk_s2g(p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK), tc::smem_u32(tile), 2 * C * DK * 4);
+        } else {
+            tc::bulk_s2g(p.VT + ((size_t)id * d.HV + h) * (DV * C), tc::smem_u32(tile), DV * C * 4);
+            tc::bulk_s2g(p.GB + ((size_t)id * d.HV + h) * C, tc::smem_u32(gbs), C * 8);
+        }
+        tc::bulk_commit();
+        tc::bulk_wait_read_all();
     }
 }
 
@@ -203,7 +302,13 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     chunk_map_kernel<<<1, 1024, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 1);
-    prep_kernel<T, DK, DV><<<p.T, 256, 0, s>>>(p);
+    {
+        const size_t shm = PrepShape<T, DK, DV>::SMEM;
+        if ((e = cudaFuncSetAttribute(prep_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)shm)) != cudaSuccess)
+            return e;
+        prep_kernel<T, DK, DV><<<dim3(p.max_chunks, p.d.HK + p.d.HV), kPrepThreads, shm, s>>>(p);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 2);
     conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
@@ -226,9 +331,9 @@ size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max
     size_t off = kHeaderBytes;
     off += al(mc * sizeof(int4));
     off += al(((size_t)max_N + 1) * sizeof(int32_t));
-    off += al((size_t)max_T * d.HK * d.dk * sizeof(float)) * 2;
-    off += al((size_t)max_T * d.HV * d.dv * sizeof(float));
-    off += al((size_t)max_T * d.HV * sizeof(float2));
+    off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
+    off += al(per * d.dv * C);
+    off += al(per * C * 2);
     off += al(per * 2 * C * d.dk);
     off += al(per * C * C);
     off += al(per * d.dk * C);
@@ -249,10 +354,9 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
     size_t off = kHeaderBytes;
     e.chunk_tab = reinterpret_cast<int4*>(base + off); off += al((size_t)mc * sizeof(int4));
     e.seq_chunk0 = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
-    e.qn = reinterpret_cast<float*>(base + off); off += al((size_t)max_T * d.HK * d.dk * sizeof(float));
-    e.kn = reinterpret_cast<float*>(base + off); off += al((size_t)max_T * d.HK * d.dk * sizeof(float));
-    e.vv = reinterpret_cast<float*>(base + off); off += al((size_t)max_T * d.HV * d.dv * sizeof(float));
-    e.gb = reinterpret_cast<float2*>(base + off); off += al((size_t)max_T * d.HV * sizeof(float2));
+    e.KQ = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
+    e.VT = reinterpret_cast<float*>(base + off); off += al(per * d.dv * C);
+    e.GB = reinterpret_cast<float2*>(base + off); off += al(per * C * 2);
     e.WQ = reinterpret_cast<float*>(base + off); off += al(per * 2 * C * d.dk);
     e.AQ = reinterpret_cast<float*>(base + off); off += al(per * C * C);
     e.KT = reinterpret_cast<float*>(base + off); off += al(per * d.dk * C);

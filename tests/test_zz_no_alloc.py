@@ -65,12 +65,19 @@ def test_static_scratch_matches_workspace_entry_point_on_two_calls_in_a_row():
 def test_static_scratch_rejects_sizes_beyond_its_maximum():
     """No GPU needed: the size check runs before anything touches the device."""
     cfg = gdn.GdnConfig(16, 32, 128, 128)
-    assert gdn.gdn_extend_workspace_size(cfg, 1, 837) <= B.EXTEND_STATIC_SCRATCH_BYTES
-    assert gdn.gdn_extend_workspace_size(cfg, 1, 838) > B.EXTEND_STATIC_SCRATCH_BYTES
+    lo, hi = 1, 1 << 20  # largest single-sequence batch that fits the fixed scratch
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if gdn.gdn_extend_workspace_size(cfg, 1, mid) <= B.EXTEND_STATIC_SCRATCH_BYTES:
+            lo = mid
+        else:
+            hi = mid - 1
+    assert lo >= 256, "the fixed scratch should hold a useful batch of the large layer"
+    too_big = lo + 1
     F = 0x10000
     params = B.GdnParamsC(F, F, F, None)
-    rc = B.lib().gdn_extend_static_scratch(ctypes.byref(cfg.c()), ctypes.byref(params), F, F, F, F, 1, 838, F, None,
-                                           F, F, 4, F, None)
+    rc = B.lib().gdn_extend_static_scratch(ctypes.byref(cfg.c()), ctypes.byref(params), F, F, F, F, 1, too_big, F,
+                                           None, F, F, 4, F, None)
     assert rc == gdn.GDN_ERR_WORKSPACE
     bad = gdn.GdnConfig(16, 32, 96, 128)
     rc = B.lib().gdn_extend_static_scratch(ctypes.byref(bad.c()), ctypes.byref(params), F, F, F, F, 1, 8, F, None,

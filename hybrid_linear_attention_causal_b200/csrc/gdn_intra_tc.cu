@@ -19,8 +19,9 @@
 // tensor core's shared-memory layout so the state pass bulk-copies them --
 // plus U (fp32) and gamma.  Operands are staged in shared memory as K-major
 // no-swizzle tiles rounded to tf32 (round to nearest); accumulators live in
-// tensor memory.  One thread issues the MMAs; all four warps read their
-// 32-lane slice of tensor memory for the CUDA-core steps.
+// tensor memory.  One thread issues the MMAs; the eight warps read their
+// sub-partition's 32-lane slice of tensor memory (two warps per slice, one
+// half of the columns each) for the CUDA-core steps.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -29,7 +30,7 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NT = 128;
+constexpr int NT = 256;  // 8 warps; warp w reads TMEM sub-partition w % 4
 
 template <int DK, int DV>
 struct IntraTcSmem {
@@ -105,7 +106,8 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
     const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;  // D1: 64 cols; W, U: M = 64 layout
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int sp = warp & 3, half = warp >> 2;  // TMEM sub-partition, column half
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     bool ok = true;
     if (tid == 0) {
         ok = tc::mbar_wait(bar_kq, 0);
@@ -148,8 +150,8 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             sm.gam[2 * lane + 1] = incl;
             sm.beta[2 * lane] = g0.y;
             sm.beta[2 * lane + 1] = g1.y;
-            sm.eg[2 * lane] = expf(gA);
-            sm.eg[2 * lane + 1] = expf(incl);
+            sm.eg[2 * lane] = __expf(gA);
+            sm.eg[2 * lane + 1] = __expf(incl);
         }
         if (j == 0) {
             okv = okv && tc::mbar_wait(bar, ph_mma);
@@ -159,29 +161,35 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         if (!ok) break;
         tc::fence_after_sync();
         const float gl = sm.gam[n - 1];
-        {  // A (warps 0-1, k.k rows) and the masked decayed q.k tile (warps 2-3) from D1
-            const int r = (warp & 1) * 32 + lane;
-            float row[C];
+        {  // A (sub-partitions 0-1: k.k rows) and the masked decayed q.k tile (2-3: q.k rows) from D1;
+           // the two warps of a sub-partition take one half of the 64 columns each
+            const int r = (sp & 1) * 32 + lane, c0 = 32 * half;
+            float row[32];
 #pragma unroll
-            for (int c0 = 0; c0 < C; c0 += 16) {
+            for (int c = 0; c < 32; c += 16) {
                 float v[16];
-                tc::tmem_ld16(tD1 + lane_base + c0, v);
+                tc::tmem_ld16(tD1 + lane_base + c0 + c, v);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) row[c0 + i] = v[i];
+                for (int i = 0; i < 16; ++i) row[c + i] = v[i];
             }
             tc::tmem_ld_wait();
             const float gr = sm.gam[r], br = sm.beta[r];
-            if (warp < 2) {
+            if (sp < 2) {
 #pragma unroll
-                for (int s = 0; s < C; ++s) sm.a[r][s] = (s < r && r < n) ? br * expf(gr - sm.gam[s]) * row[s] : 0.f;
+                for (int i = 0; i < 32; ++i) {
+                    const int s = c0 + i;
+                    sm.a[r][s] = (s < r && r < n) ? br * __expf(gr - sm.gam[s]) * row[i] : 0.f;
+                }
             } else {
 #pragma unroll
-                for (int s = 0; s < C; s += 4) {
+                for (int i = 0; i < 32; i += 4) {
                     float o[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        o[u] = (s + u <= r && r < n) ? tc::round_tf32(expf(gr - sm.gam[s + u]) * row[s + u]) : 0.f;
-                    store_f4(reinterpret_cast<float*>(AQg), tc::kmajor_off(r, s, C), make_float4(o[0], o[1], o[2], o[3]));
+                    for (int u = 0; u < 4; ++u) {
+                        const int s = c0 + i + u;
+                        o[u] = (s <= r && r < n) ? tc::round_tf32(__expf(gr - sm.gam[s]) * row[i + u]) : 0.f;
+                    }
+                    store_f4(reinterpret_cast<float*>(AQg), tc::kmajor_off(r, c0 + i, C), make_float4(o[0], o[1], o[2], o[3]));
                 }
             }
         }
@@ -243,7 +251,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 const int s = 4 * q + w;
                 const float kv = load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
                 kb[w] = tc::round_tf32(kv * sm.beta[s] * sm.eg[s]);
-                kt[w] = s < n ? tc::round_tf32(kv * expf(gl - sm.gam[s])) : 0.f;
+                kt[w] = s < n ? tc::round_tf32(kv * __expf(gl - sm.gam[s])) : 0.f;
             }
             store_f4(sm.bk, tc::kmajor_off(f, 4 * q, DK), make_float4(kb[0], kb[1], kb[2], kb[3]));
             store_f4(reinterpret_cast<float*>(KTg), tc::kmajor_off(f, 4 * q, DK), make_float4(kt[0], kt[1], kt[2], kt[3]));
@@ -291,11 +299,13 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         if (!ok) break;
         tc::fence_after_sync();
         if (tid == 0 && j + 2 < G) fetch_v(j + 2);  // buffer b is free again
-        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major
+        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major.
+           // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15;
+           // the two warps of a sub-partition take one half of the columns each
             const bool valid = lane < 16;
-            const int r = warp * 16 + lane;
+            const int r = sp * 16 + lane;
 #pragma unroll
-            for (int c0 = 0; c0 < DK; c0 += 16) {
+            for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 16) {
                 float v[16];
                 tc::tmem_ld16(tW + lane_base + c0, v);
                 tc::tmem_ld_wait();
@@ -307,7 +317,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                                              tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
             }
 #pragma unroll
-            for (int c0 = 0; c0 < DV; c0 += 16) {
+            for (int c0 = half * (DV / 2); c0 < (half + 1) * (DV / 2); c0 += 16) {
                 float v[16];
                 tc::tmem_ld16(tU + lane_base + c0, v);
                 tc::tmem_ld_wait();

@@ -107,9 +107,11 @@ template <typename T, int DK, int DV>
 struct PrepShape {
     static constexpr int NCH = 2 * DK > DV ? 2 * DK : DV;  // staged channels per row (max over units)
     static constexpr int VE = 16 / sizeof(T);              // elements per 16-byte vector
-    static constexpr size_t XS_BYTES = (((size_t)(C + 3) * NCH * sizeof(T)) + 15) & ~(size_t)15;
+    static constexpr int PAD = VE;                         // row padding: spreads rows over banks
+    static constexpr size_t XS_BYTES = (((size_t)(C + 3) * (NCH + PAD) * sizeof(T)) + 15) & ~(size_t)15;
     static constexpr size_t TILE_BYTES = (2 * C * DK > DV * C ? 2 * C * DK : DV * C) * sizeof(float);
-    static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + C * sizeof(float2);
+    static constexpr size_t W_BYTES = (size_t)NCH * 5 * sizeof(float);  // 4 taps + bias per channel
+    static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + W_BYTES + C * sizeof(float2);
 };
 
 template <typename T, int DK, int DV>
@@ -126,7 +128,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool isqk = unit < d.HK;
     const int nch = isqk ? 2 * DK : DV;
-    // staged column c -> channel of mixed_qkv
+    const int ld = nch + S::PAD;  // staged row stride (elements)
+    // staged column c -> channel of mixed_qkv: qk unit [q (DK) | k (DK)], v unit [v (DV)]
     const int hk = unit, h = unit - d.HK;
     auto channel = [&](int c) -> int {
         if (!isqk) return 2 * d.HK * DK + h * DV + c;
@@ -135,10 +138,13 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T* xs = reinterpret_cast<T*>(smem_raw);  // row i <-> token t0 - 3 + i
     float* tile = reinterpret_cast<float*>(smem_raw + S::XS_BYTES);
-    float2* gbs = reinterpret_cast<float2*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);
+    float* wsm = reinterpret_cast<float*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);  // [nch][5]
+    float2* gbs = reinterpret_cast<float2*>(smem_raw + S::XS_BYTES + S::TILE_BYTES + S::W_BYTES);
     const T* x = reinterpret_cast<const T*>(p.x);
+    const T* w = reinterpret_cast<const T*>(p.conv_w);
+    const T* bias = reinterpret_cast<const T*>(p.conv_b);
 
-    // stage rows 3 .. n+2 (this chunk) with 16-byte loads; the 3 halo rows element-wise
+    // stage rows 3 .. n+2 (this chunk) with 16-byte loads; the 3 halo rows and the weights element-wise
     {
         const int vpr = nch / S::VE;  // vectors per row (segments never straddle a vector)
         const int nv = n * vpr;
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
                 const int e = base + u * kPrepThreads + tid;
                 if (e < nv) {
                     const int r = e / vpr, c = (e % vpr) * S::VE;
-                    *reinterpret_cast<uint4*>(xs + (size_t)(r + 3) * nch + c) = v[u];
+                    *reinterpret_cast<uint4*>(xs + (size_t)(r + 3) * ld + c) = v[u];
                 }
             }
         }
@@ -168,74 +174,61 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
             T v;
             if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + channel(c)];
             else v = init ? cs[(size_t)channel(c) * 3 + i] : from_f<T>(0.f);
-            xs[(size_t)i * nch + c] = v;
+            xs[(size_t)i * ld + c] = v;
+        }
+        for (int e = tid; e < nch * 5; e += kPrepThreads) {
+            const int c = e / 5, j = e % 5;
+            const int cg = channel(c);
+            wsm[e] = j < 4 ? to_f(w[(size_t)cg * 4 + j]) : (bias ? to_f(bias[cg]) : 0.f);
         }
     }
     __syncthreads();
-    const T* w = reinterpret_cast<const T*>(p.conv_w);
-    const T* bias = reinterpret_cast<const T*>(p.conv_b);
+    // conv + SiLU of staged column c at output row r (r < n)
+    auto conv = [&](int c, int r) -> float {
+        const float* wc = wsm + c * 5;
+        float acc = wc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc = fmaf(wc[j], to_f(xs[(size_t)(r + j) * ld + c]), acc);
+        return silu_f(acc);
+    };
     if (isqk) {
-        constexpr int PL = DK / 32;  // channels per lane and part
-        float wk[2][PL][4], bk[2][PL];
+        // warp w: rows 8w .. 8w+7; lane (rr = lane & 7, cc = lane >> 3) takes row 8w + rr and the
+        // column quads 4 cg + cc of both parts, so every 8-lane group writes whole 128-byte core
+        // matrices of the tile; the L2 norm reduces over the 4 lanes of a row
+        const int rr = lane & 7, cc = lane >> 3;
+        const int r = 8 * warp + rr;
+        for (int part = 0; part < 2; ++part) {  // part 0: q (tile rows C + r), part 1: k (tile rows r)
+            float y[DK / 16][4];
+            float ss = 0.f;
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
+            for (int cg = 0; cg < DK / 16; ++cg)
 #pragma unroll
-            for (int u = 0; u < PL; ++u) {
-                const int cg = channel(part * DK + PL * lane + u);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) wk[part][u][j] = to_f(w[(size_t)cg * 4 + j]);
-                bk[part][u] = bias ? to_f(bias[cg]) : 0.f;
-            }
-        for (int r = warp; r < C; r += kPrepThreads / 32) {
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {  // part 0: q (tile rows C + r), part 1: k (tile rows r)
-                float y[PL];
-                float ss = 0.f;
-#pragma unroll
-                for (int u = 0; u < PL; ++u) {
-                    float acc = bk[part][u];
-                    if (r < n) {
-                        const int c = part * DK + PL * lane + u;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) acc = fmaf(wk[part][u][j], to_f(xs[(size_t)(r + j) * nch + c]), acc);
-                    }
-                    y[u] = r < n ? silu_f(acc) : 0.f;
-                    ss += y[u] * y[u];
+                for (int u = 0; u < 4; ++u) {
+                    const int c = part * DK + 4 * (4 * cg + cc) + u;
+                    y[cg][u] = r < n ? conv(c, r) : 0.f;
+                    ss += y[cg][u] * y[cg][u];
                 }
-                ss = warp_sum(ss);
-                const float sc = (r < n) ? rsqrtf(ss + d.eps) * (part == 0 ? d.scale : 1.f) : 0.f;
-                const int row = part == 0 ? C + r : r;
-                char* dst = reinterpret_cast<char*>(tile) + tc::kmajor_off(row, PL * lane, 2 * C);
-                if constexpr (PL == 4)
-                    *reinterpret_cast<float4*>(dst) = make_float4(tc::round_tf32(y[0] * sc), tc::round_tf32(y[1] * sc),
-                                                                  tc::round_tf32(y[2] * sc), tc::round_tf32(y[3] * sc));
-                else
-                    *reinterpret_cast<float2*>(dst) = make_float2(tc::round_tf32(y[0] * sc), tc::round_tf32(y[1] * sc));
-            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+            const float sc = (r < n) ? rsqrtf(ss + d.eps) * (part == 0 ? d.scale : 1.f) : 0.f;
+            const int row = part == 0 ? C + r : r;
+#pragma unroll
+            for (int cg = 0; cg < DK / 16; ++cg)
+                *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(row, 4 * (4 * cg + cc), 2 * C)) =
+                    make_float4(tc::round_tf32(y[cg][0] * sc), tc::round_tf32(y[cg][1] * sc),
+                                tc::round_tf32(y[cg][2] * sc), tc::round_tf32(y[cg][3] * sc));
         }
     } else {
-        constexpr int PL = DV / 32;  // channels per lane: f = lane + 32 u
-        float wv[PL][4], bv[PL];
+        // V^T tile: thread (f, 4 consecutive rows) -> one float4 of the K-major tile (8 lanes per core matrix)
+        for (int idx = tid; idx < DV * (C / 4); idx += kPrepThreads) {
+            const int ff = idx & 7, cq = (idx >> 3) & 3, rest = idx >> 5;
+            const int fg = rest % (DV / 8), rg = rest / (DV / 8);
+            const int f = 8 * fg + ff, r4 = 4 * (4 * rg + cq);
+            float y[4];
 #pragma unroll
-        for (int u = 0; u < PL; ++u) {
-            const int cg = channel(lane + 32 * u);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) wv[u][j] = to_f(w[(size_t)cg * 4 + j]);
-            bv[u] = bias ? to_f(bias[cg]) : 0.f;
-        }
-        for (int r = warp; r < C; r += kPrepThreads / 32) {
-#pragma unroll
-            for (int u = 0; u < PL; ++u) {
-                const int f = lane + 32 * u;
-                float y = 0.f;
-                if (r < n) {
-                    float acc = bv[u];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc = fmaf(wv[u][j], to_f(xs[(size_t)(r + j) * nch + f]), acc);
-                    y = silu_f(acc);
-                }
-                *reinterpret_cast<float*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(f, r, DV)) = y;
-            }
+            for (int u = 0; u < 4; ++u) y[u] = r4 + u < n ? conv(f, r4 + u) : 0.f;
+            *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(f, r4, DV)) =
+                make_float4(y[0], y[1], y[2], y[3]);
         }
         if (tid < C) {
             float2 gb = make_float2(0.f, 0.f);

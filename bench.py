@@ -37,8 +37,8 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# nominal dense tf32 / bf16 tensor throughput ratio of B200 (1.1 vs 2.25 PFLOP/s)
+TF32_PER_BF16 = 1.1 / 2.25
 C = 64
 
 
@@ -319,7 +319,10 @@ def run_profile_case(args, dev):
     s1.record()
     torch.cuda.synchronize()
     assert gdn.gdn_get_device_error(ws) == 0
-    print(json.dumps({"profile": args.profile, "workload": w.name, "ms_per_call": s0.elapsed_time(s1) / args.steps}))
+    cu = w.cu_seqlens.cpu().tolist() if args.profile == "extend" else list(range(w.N + 1))
+    chunks = sum((cu[i + 1] - cu[i] + C - 1) // C for i in range(len(cu) - 1))
+    print(json.dumps({"profile": args.profile, "workload": w.name, "chunks": chunks,
+                      "ms_per_call": s0.elapsed_time(s1) / args.steps}))
 
 
 def main():
@@ -426,11 +429,11 @@ def main():
     st_ver, by_ver = verify_bytes(dspec, Bn, D)
     value = world * pre.T / (ext_ms * 1e-3)
 
+    tf32 = bf16 * TF32_PER_BF16
+    tf32_src = f"{peak_src} bf16 burst {bf16:.1f} TFLOP/s x nominal tf32/bf16 ratio 1.1/2.25"
     kernels = {
-        "state": {"bound": "alu", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": FP32_ALU_TFLOPS,
-                  "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
-        "intra": {"bound": "alu", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": FP32_ALU_TFLOPS,
-                  "peak_src": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+        "state": {"bound": "tensor", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": tf32, "peak_src": tf32_src},
+        "intra": {"bound": "tensor", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": tf32, "peak_src": tf32_src},
         "prep": {"bound": "hbm", "work": pre.T * (spec.conv_dim * 2 + 2 * spec.HV * 2), "unit": "GB/s",
                  "peak": hbm, "peak_src": peak_src},
         "decode": {"bound": "hbm", "work": by_dec, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
@@ -446,7 +449,13 @@ def main():
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
                 "unit": dk["unit"], "frac": dk["frac"], "traffic": ncu_traffic(dom),
-                "peak_source": dk["peak_src"] + (" (of measured)" if dk["peak_src"] == "measured" else "")}
+                "peak_source": dk["peak_src"] + (" (of measured)" if peak_src == "measured" else " (of fallback)")}
+    # the whole prefill against its own roofline: max(algorithmic FLOPs at the tf32 peak,
+    # algorithmic bytes at the HBM peak)
+    t_floor = max(pw["flops"] / (tf32 * 1e12), pw["bytes"] / (hbm * 1e9))
+    prefill_roofline = {"floor_ms": t_floor * 1e3, "bound": "tensor" if pw["flops"] / (tf32 * 1e12) >= pw["bytes"] / (hbm * 1e9) else "hbm",
+                        "frac": t_floor / (ext_ms * 1e-3), "tensor_frac": pw["flops"] / (ext_ms * 1e-3) / (tf32 * 1e12),
+                        "hbm_frac": pw["bytes"] / (ext_ms * 1e-3) / (hbm * 1e9)}
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -493,7 +502,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "tf32/f32", "data": "synthetic",
             "config": workload_config(pre, args),
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,
@@ -508,7 +517,7 @@ def main():
             "verify": {"ms": ver_ms, "state_gbs": world * st_ver / (ver_ms * 1e-3) / 1e9,
                        "total_gbs": world * by_ver / (ver_ms * 1e-3) / 1e9,
                        "frac_of_measured_hbm": by_ver / (ver_ms * 1e-3) / 1e9 / hbm},
-            "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12,
+            "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12, "roofline": prefill_roofline,
                         "gbs_algorithmic": pw["bytes"] / (ext_ms * 1e-3) / 1e9,
                         "kernel_ms": {k: kern_ms[k] for k in EXT_K}},
             "kernels": {k: {kk: v[kk] for kk in ("bound", "ms", "achieved", "peak", "unit", "frac")}

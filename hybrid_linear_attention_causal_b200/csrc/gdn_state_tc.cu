@@ -138,11 +138,17 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
 
     uint32_t ph_mma = 0;
     bool ok = true;
+    // gamma of the next chunk, loaded one chunk ahead so no global load sits before an MMA issue
+    float g_next = tid < C ? p.gam[((size_t)c_begin * HV + h) * C + tid] : 0.f;
     for (int id = c_begin; id < c_end; ++id) {
         const uint32_t ph_ld = (uint32_t)(id - c_begin) & 1u;
         const int4 ch = p.chunk_tab[id];
         const int t0 = ch.y, n = ch.z;
         const size_t ch_h = (size_t)id * HV + h;
+        if (tid < C) {
+            sm.gam[tid] = g_next;
+            if (id + 1 < c_end) g_next = p.gam[(ch_h + HV) * C + tid];
+        }
         // U column j of this chunk (consumed after the first MMA)
         float u[C];
         {
@@ -150,7 +156,6 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
 #pragma unroll
             for (int s = 0; s < C; ++s) u[s] = rowv ? Ug[(size_t)s * DV + j] : 0.f;
         }
-        if (tid < C) sm.gam[tid] = p.gam[ch_h * C + tid];
         bool okw = true;
         if (tid == 0) {
             okw = tc::mbar_wait(bar_wq, ph_ld);
@@ -222,7 +227,9 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
         if (!ok) break;
         tc::fence_after_sync();
         if (tid == 0 && id + 1 < c_end) fetch_ak(id + 1);  // the Aqk and K~^T tiles are free again
-        // outputs O^T row j -> out[t0 + r][h][j]; new state -> next chunk's operand tile
+        // outputs: O^T row j is staged as column j of O [C][DV] in the (now free) V'^T tile, then the
+        // chunk's rows leave as 16-byte vectors
+        T* ostage = reinterpret_cast<T*>(sm.vt);
 #pragma unroll
         for (int c0 = 0; c0 < C; c0 += 16) {
             float o[16];
@@ -230,8 +237,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
             tc::tmem_ld_wait();
             if (rowv)
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + j] = from_f<T>(o[i]);
+                for (int i = 0; i < 16; ++i) ostage[(c0 + i) * DV + j] = from_f<T>(o[i]);
         }
 #pragma unroll
         for (int c0 = 0; c0 < DK; c0 += 16) {
@@ -244,6 +250,14 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
+        {
+            constexpr int VPR = DV * (int)sizeof(T) / 16;  // 16-byte vectors per output row
+            for (int e = tid; e < n * VPR; e += NT) {
+                const int r = e / VPR, v = e % VPR;
+                reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * HV + h) * DV)[v] =
+                    reinterpret_cast<const uint4*>(ostage + r * DV)[v];
+            }
+        }
     }
     if (ok) {  // final state: column j of S
 #pragma unroll

@@ -43,6 +43,8 @@ struct IntraTcSmem {
     float m[3][16][17];    // off-diagonal block products
     float2 gb[2][C];       // (g, beta) of the two heads in flight
     float gam[C], beta[C], eg[C];
+    float fbk[C];          // beta_s e^{gamma_s}: column factor of (diag(beta e^gamma) K)^T
+    float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
     unsigned long long bar_mma, bar_kq, bar_v[2];
     uint32_t tmem_base;
 };
@@ -152,6 +154,11 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             sm.beta[2 * lane + 1] = g1.y;
             sm.eg[2 * lane] = __expf(gA);
             sm.eg[2 * lane + 1] = __expf(incl);
+            const float gn = __shfl_sync(0xffffffffu, (n - 1) & 1 ? incl : gA, (n - 1) >> 1);
+            sm.fbk[2 * lane] = g0.y * __expf(gA);
+            sm.fbk[2 * lane + 1] = g1.y * __expf(incl);
+            sm.fkt[2 * lane] = 2 * lane < n ? __expf(gn - gA) : 0.f;
+            sm.fkt[2 * lane + 1] = 2 * lane + 1 < n ? __expf(gn - incl) : 0.f;
         }
         if (j == 0) {
             okv = okv && tc::mbar_wait(bar, ph_mma);
@@ -209,26 +216,29 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             for (int r = 0; r < 16; ++r) sm.tf[o + r][o + c] = t[r];
         }
         __syncthreads();
-        // off-diagonal blocks by distance: T_ij = -T_ii (sum_{k=j}^{i-1} A_ik T_kj)
+        // off-diagonal blocks by distance: T_ij = -T_ii (sum_{k=j}^{i-1} A_ik T_kj); four partial sums
+        // per element keep the dependent FMA chains short
         for (int dist = 1; dist < 4; ++dist) {
             const int nel = (4 - dist) * 256;
             for (int e = tid; e < nel; e += NT) {
                 const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
                 const int bi = blk + dist, bj = blk;
-                float acc = 0.f;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int k = bj; k < bi; ++k)
 #pragma unroll
-                    for (int s = 0; s < 16; ++s) acc = fmaf(sm.a[16 * bi + r][16 * k + s], sm.tf[16 * k + s][16 * bj + c], acc);
-                sm.m[blk][r][c] = acc;
+                    for (int s = 0; s < 16; ++s)
+                        acc[s & 3] = fmaf(sm.a[16 * bi + r][16 * k + s], sm.tf[16 * k + s][16 * bj + c], acc[s & 3]);
+                sm.m[blk][r][c] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
             __syncthreads();
             for (int e = tid; e < nel; e += NT) {
                 const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
                 const int bi = blk + dist, bj = blk;
-                float acc = 0.f;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int s = 0; s < 16; ++s) acc = fmaf(sm.tf[16 * bi + r][16 * bi + s], sm.m[blk][s][c], acc);
-                sm.tf[16 * bi + r][16 * bj + c] = -acc;
+                for (int s = 0; s < 16; ++s)
+                    acc[s & 3] = fmaf(sm.tf[16 * bi + r][16 * bi + s], sm.m[blk][s][c], acc[s & 3]);
+                sm.tf[16 * bi + r][16 * bj + c] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
             }
             __syncthreads();
         }
@@ -242,19 +252,14 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             store_f4(sm.t, tc::kmajor_off(r, s4, C), make_float4(v[0], v[1], v[2], v[3]));
         }
         // (diag(beta e^gamma) K)^T into shared memory and (diag(e^{gamma_n - gamma}) K)^T to the
-        // workspace, both from the k rows of the [K ; Q] tile (row f = one feature across the rows s)
-        for (int idx = tid; idx < DK * (C / 4); idx += NT) {
-            const int f = idx % DK, q = idx / DK;
-            float kb[4], kt[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const int s = 4 * q + w;
-                const float kv = load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
-                kb[w] = tc::round_tf32(kv * sm.beta[s] * sm.eg[s]);
-                kt[w] = s < n ? tc::round_tf32(kv * __expf(gl - sm.gam[s])) : 0.f;
-            }
-            store_f4(sm.bk, tc::kmajor_off(f, 4 * q, DK), make_float4(kb[0], kb[1], kb[2], kb[3]));
-            store_f4(reinterpret_cast<float*>(KTg), tc::kmajor_off(f, 4 * q, DK), make_float4(kt[0], kt[1], kt[2], kt[3]));
+        // workspace, both from the k rows of the [K ; Q] tile (row f = one feature across the rows s).
+        // A warp reads one 128-byte core matrix of the tile (8 rows s x 4 features f): no bank conflicts.
+        for (int idx = tid; idx < DK * C; idx += NT) {
+            const int s = (idx & 7) + 8 * ((idx >> 5) & 7), f = ((idx >> 3) & 3) + 4 * (idx >> 8);
+            const float kv = load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
+            const uint32_t off = tc::kmajor_off(f, s, DK);
+            *reinterpret_cast<float*>(reinterpret_cast<char*>(sm.bk) + off) = tc::round_tf32(kv * sm.fbk[s]);
+            *reinterpret_cast<float*>(KTg + off) = tc::round_tf32(kv * sm.fkt[s]);
         }
         // V^T scaled by beta, in place (tile layout unchanged)
         for (int idx = tid; idx < DV * (C / 4); idx += NT) {

@@ -91,25 +91,25 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
 
 // ---------------------------------------------------------------- 2. prep
 
-// One CTA per (chunk, head unit): a unit is either a qk head (its q and k
-// channels) or a value head (its v channels and gates).  The chunk's raw rows
-// and the 3 rows before it (from the previous chunk of the same sequence, or
-// from the conv-state slot for a sequence's first chunk) are staged in shared
-// memory; every output row is then conv1d + SiLU (+ L2 norm for q, k) of
-// shared-memory data.  Results are assembled as tiles in the tensor core's
-// shared-memory layout and written with one bulk store:
-//   qk unit: [K ; Q*scale] tf32, K-major, 128 rows x dk
-//   v unit:  V^T fp32, K-major, dv rows x C, and (g, beta) for the C rows
+// One CTA per (chunk, unit); a unit is the q channels of a qk head, the k
+// channels of a qk head, or the v channels (and gates) of a value head.  The
+// chunk's raw rows and the 3 rows before it (from the previous chunk of the
+// same sequence, or from the conv-state slot for a sequence's first chunk)
+// are staged in shared memory; every output row is then conv1d + SiLU (+ L2
+// norm for q, k) of shared-memory data.  Results are assembled as tiles in the
+// tensor core's shared-memory layout and leave by bulk stores:
+//   q / k unit: rows C..2C-1 / 0..C-1 of [K ; Q*scale] (tf32, K-major, 128 rows x dk)
+//   v unit:     V^T fp32 (K-major, dv rows x C) and (g, beta) for the C rows
 // Rows past the end of a ragged chunk are written as zeros.
 constexpr int kPrepThreads = 256;
 
 template <typename T, int DK, int DV>
 struct PrepShape {
-    static constexpr int NCH = 2 * DK > DV ? 2 * DK : DV;  // staged channels per row (max over units)
-    static constexpr int VE = 16 / sizeof(T);              // elements per 16-byte vector
-    static constexpr int PAD = VE;                         // row padding: spreads rows over banks
+    static constexpr int NCH = DK > DV ? DK : DV;  // staged channels per row (max over units)
+    static constexpr int VE = 16 / sizeof(T);      // elements per 16-byte vector
+    static constexpr int PAD = VE;                 // row padding: spreads rows over banks
     static constexpr size_t XS_BYTES = (((size_t)(C + 3) * (NCH + PAD) * sizeof(T)) + 15) & ~(size_t)15;
-    static constexpr size_t TILE_BYTES = (2 * C * DK > DV * C ? 2 * C * DK : DV * C) * sizeof(float);
+    static constexpr size_t TILE_BYTES = (size_t)C * NCH * sizeof(float);
     static constexpr size_t W_BYTES = (size_t)NCH * 5 * sizeof(float);  // 4 taps + bias per channel
     static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + W_BYTES + C * sizeof(float2);
 };
@@ -126,15 +126,11 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     if (slot < 0 || slot >= p.P) return;
     const LayerDims& d = p.d;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool isqk = unit < d.HK;
-    const int nch = isqk ? 2 * DK : DV;
+    const bool isq = unit < d.HK, isk = !isq && unit < 2 * d.HK, isv = !isq && !isk;
+    const int nch = isv ? DV : DK;
     const int ld = nch + S::PAD;  // staged row stride (elements)
-    // staged column c -> channel of mixed_qkv: qk unit [q (DK) | k (DK)], v unit [v (DV)]
-    const int hk = unit, h = unit - d.HK;
-    auto channel = [&](int c) -> int {
-        if (!isqk) return 2 * d.HK * DK + h * DV + c;
-        return c < DK ? hk * DK + c : d.HK * DK + hk * DK + (c - DK);
-    };
+    const int hk = isq ? unit : unit - d.HK, h = unit - 2 * d.HK;
+    const int c_first = isq ? hk * DK : isk ? d.HK * DK + hk * DK : 2 * d.HK * DK + h * DV;  // first channel
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T* xs = reinterpret_cast<T*>(smem_raw);  // row i <-> token t0 - 3 + i
     float* tile = reinterpret_cast<float*>(smem_raw + S::XS_BYTES);
@@ -146,7 +142,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
 
     // stage rows 3 .. n+2 (this chunk) with 16-byte loads; the 3 halo rows and the weights element-wise
     {
-        const int vpr = nch / S::VE;  // vectors per row (segments never straddle a vector)
+        const int vpr = nch / S::VE;  // vectors per row
         const int nv = n * vpr;
         for (int base = 0; base < nv; base += kPrepThreads * 4) {
             uint4 v[4];
@@ -155,7 +151,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
                 const int e = base + u * kPrepThreads + tid;
                 if (e < nv) {
                     const int r = e / vpr, c = (e % vpr) * S::VE;
-                    v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d.conv_dim + channel(c));
+                    v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d.conv_dim + c_first + c);
                 }
             }
 #pragma unroll
@@ -172,13 +168,13 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
         for (int e = tid; e < 3 * nch; e += kPrepThreads) {
             const int i = e / nch, c = e % nch;
             T v;
-            if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + channel(c)];
-            else v = init ? cs[(size_t)channel(c) * 3 + i] : from_f<T>(0.f);
+            if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + c_first + c];
+            else v = init ? cs[(size_t)(c_first + c) * 3 + i] : from_f<T>(0.f);
             xs[(size_t)i * ld + c] = v;
         }
         for (int e = tid; e < nch * 5; e += kPrepThreads) {
             const int c = e / 5, j = e % 5;
-            const int cg = channel(c);
+            const int cg = c_first + c;
             wsm[e] = j < 4 ? to_f(w[(size_t)cg * 4 + j]) : (bias ? to_f(bias[cg]) : 0.f);
         }
     }
@@ -191,33 +187,29 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
         for (int j = 0; j < 4; ++j) acc = fmaf(wc[j], to_f(xs[(size_t)(r + j) * ld + c]), acc);
         return silu_f(acc);
     };
-    if (isqk) {
+    if (!isv) {
         // warp w: rows 8w .. 8w+7; lane (rr = lane & 7, cc = lane >> 3) takes row 8w + rr and the
-        // column quads 4 cg + cc of both parts, so every 8-lane group writes whole 128-byte core
-        // matrices of the tile; the L2 norm reduces over the 4 lanes of a row
+        // column quads 4 cg + cc, so every 8-lane group writes whole 128-byte core matrices of the
+        // half tile (a K-major 64-row tile); the L2 norm reduces over the 4 lanes of a row
         const int rr = lane & 7, cc = lane >> 3;
         const int r = 8 * warp + rr;
-        for (int part = 0; part < 2; ++part) {  // part 0: q (tile rows C + r), part 1: k (tile rows r)
-            float y[DK / 16][4];
-            float ss = 0.f;
+        float y[DK / 16][4];
+        float ss = 0.f;
 #pragma unroll
-            for (int cg = 0; cg < DK / 16; ++cg)
+        for (int cg = 0; cg < DK / 16; ++cg)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = part * DK + 4 * (4 * cg + cc) + u;
-                    y[cg][u] = r < n ? conv(c, r) : 0.f;
-                    ss += y[cg][u] * y[cg][u];
-                }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-            const float sc = (r < n) ? rsqrtf(ss + d.eps) * (part == 0 ? d.scale : 1.f) : 0.f;
-            const int row = part == 0 ? C + r : r;
+            for (int u = 0; u < 4; ++u) {
+                y[cg][u] = r < n ? conv(4 * (4 * cg + cc) + u, r) : 0.f;
+                ss += y[cg][u] * y[cg][u];
+            }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+        const float sc = (r < n) ? rsqrtf(ss + d.eps) * (isq ? d.scale : 1.f) : 0.f;
 #pragma unroll
-            for (int cg = 0; cg < DK / 16; ++cg)
-                *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(row, 4 * (4 * cg + cc), 2 * C)) =
-                    make_float4(tc::round_tf32(y[cg][0] * sc), tc::round_tf32(y[cg][1] * sc),
-                                tc::round_tf32(y[cg][2] * sc), tc::round_tf32(y[cg][3] * sc));
-        }
+        for (int cg = 0; cg < DK / 16; ++cg)
+            *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(r, 4 * (4 * cg + cc), C)) =
+                make_float4(tc::round_tf32(y[cg][0] * sc), tc::round_tf32(y[cg][1] * sc),
+                            tc::round_tf32(y[cg][2] * sc), tc::round_tf32(y[cg][3] * sc));
     } else {
         // V^T tile: thread (f, 4 consecutive rows) -> one float4 of the K-major tile (8 lanes per core matrix)
         for (int idx = tid; idx < DV * (C / 4); idx += kPrepThreads) {
@@ -244,8 +236,11 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     tc::fence_smem_to_async();
     __syncthreads();
     if (tid == 0) {
-        if (isqk) {
-            tc::bulk_s2g(p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK), tc::smem_u32(tile), 2 * C * DK * 4);
+        if (!isv) {
+            // the 64-row half tile holds DK/4 blocks of 1 KB (one per column quad); in the 128-row
+            // [K ; Q] tile those blocks sit 2 KB apart, the q half 1 KB after the k half
+            char* dst = reinterpret_cast<char*>(p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK)) + (isq ? 1024 : 0);
+            for (int q = 0; q < DK / 4; ++q) tc::bulk_s2g(dst + 2048 * q, tc::smem_u32(tile) + 1024 * q, 1024);
         } else {
             tc::bulk_s2g(p.VT + ((size_t)id * d.HV + h) * (DV * C), tc::smem_u32(tile), DV * C * 4);
             tc::bulk_s2g(p.GB + ((size_t)id * d.HV + h) * C, tc::smem_u32(gbs), C * 8);
@@ -300,7 +295,7 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
         if ((e = cudaFuncSetAttribute(prep_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)shm)) != cudaSuccess)
             return e;
-        prep_kernel<T, DK, DV><<<dim3(p.max_chunks, p.d.HK + p.d.HV), kPrepThreads, shm, s>>>(p);
+        prep_kernel<T, DK, DV><<<dim3(p.max_chunks, 2 * p.d.HK + p.d.HV), kPrepThreads, shm, s>>>(p);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 2);

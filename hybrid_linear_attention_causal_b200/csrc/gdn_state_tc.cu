@@ -13,7 +13,9 @@
 //
 // where Qg = diag(e^gamma) Q (q carries the output scale).  The fp32 state
 // S^T lives in tensor memory (the MMA accumulates onto it in fp32); a tf32
-// copy in shared memory is the operand of the next chunk.  The intra-chunk
+// copy in shared memory is the operand of the next chunk.  Eight warps: the
+// two warps of a TMEM sub-partition share its 32 accumulator rows and take
+// one half of the columns each.  The intra-chunk
 // kernel wrote [W ; Qg], Aqk and K~^T already as tf32 tiles in the tensor
 // core's shared-memory layout; they arrive by asynchronous bulk copies, each
 // reissued for the next chunk as soon as the MMA that reads it has finished,
@@ -26,7 +28,7 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NT = 128;
+constexpr int NT = 256;  // 8 warps: two per TMEM sub-partition, each taking half of the columns
 
 template <int DK, int DV>
 struct StateTcSmem {
@@ -114,16 +116,18 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
     const uint32_t tXO = tm, tS = tm + 128;  // [X^T | O^T] (128 columns), S^T (DK columns)
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int sp = warp & 3, half = warp >> 2;  // TMEM sub-partition, column half
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     // this thread's accumulator row j (the value-dimension index)
     const bool rowv = DV == 128 || lane < 16;
-    const int j = DV == 128 ? warp * 32 + lane : warp * 16 + lane;
+    const int j = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
 
     // initial state: S^T row j = column j of S
     const bool init = p.has_init ? p.has_init[nseq] != 0 : true;
     float* Sg = p.ssm_state + ((size_t)slot * HV + h) * DK * DV;
 #pragma unroll
-    for (int c0 = 0; c0 < DK; c0 += 16) {
+    for (int cc = 0; cc < DK / 2; cc += 16) {
+        const int c0 = half * (DK / 2) + cc;
         float v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = (init && rowv) ? Sg[(size_t)(c0 + i) * DV + j] : 0.f;
@@ -149,12 +153,12 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
             sm.gam[tid] = g_next;
             if (id + 1 < c_end) g_next = p.gam[(ch_h + HV) * C + tid];
         }
-        // U column j of this chunk (consumed after the first MMA)
-        float u[C];
+        // U column j of this chunk, rows of this warp's half (consumed after the first MMA)
+        float u[C / 2];
         {
-            const float* Ug = p.U + ch_h * (C * DV);
+            const float* Ug = p.U + ch_h * (C * DV) + (size_t)half * (C / 2) * DV;
 #pragma unroll
-            for (int s = 0; s < C; ++s) u[s] = rowv ? Ug[(size_t)s * DV + j] : 0.f;
+            for (int s = 0; s < C / 2; ++s) u[s] = rowv ? Ug[(size_t)s * DV + j] : 0.f;
         }
         bool okw = true;
         if (tid == 0) {
@@ -178,7 +182,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
         const float egl = expf(sm.gam[n - 1]);
         // V'^T row j = U^T row j - X^T row j; the fp32 state is scaled by e^{gamma_n}
 #pragma unroll
-        for (int c0 = 0; c0 < C; c0 += 16) {
+        for (int cc = 0; cc < C / 2; cc += 16) {
+            const int c0 = half * (C / 2) + cc;
             float x[16];
             tc::tmem_ld16(tXO + lane_base + c0, x);
             tc::tmem_ld_wait();
@@ -186,13 +191,14 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     store_f4(sm.vt, tc::kmajor_off(j, c0 + 4 * q, DV),
-                             make_float4(tc::round_tf32(u[c0 + 4 * q] - x[4 * q]),
-                                         tc::round_tf32(u[c0 + 4 * q + 1] - x[4 * q + 1]),
-                                         tc::round_tf32(u[c0 + 4 * q + 2] - x[4 * q + 2]),
-                                         tc::round_tf32(u[c0 + 4 * q + 3] - x[4 * q + 3])));
+                             make_float4(tc::round_tf32(u[cc + 4 * q] - x[4 * q]),
+                                         tc::round_tf32(u[cc + 4 * q + 1] - x[4 * q + 1]),
+                                         tc::round_tf32(u[cc + 4 * q + 2] - x[4 * q + 2]),
+                                         tc::round_tf32(u[cc + 4 * q + 3] - x[4 * q + 3])));
         }
 #pragma unroll
-        for (int c0 = 0; c0 < DK; c0 += 16) {
+        for (int cc = 0; cc < DK / 2; cc += 16) {
+            const int c0 = half * (DK / 2) + cc;
             float v[16];
             tc::tmem_ld16(tS + lane_base + c0, v);
             tc::tmem_ld_wait();
@@ -231,7 +237,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
         // chunk's rows leave as 16-byte vectors
         T* ostage = reinterpret_cast<T*>(sm.vt);
 #pragma unroll
-        for (int c0 = 0; c0 < C; c0 += 16) {
+        for (int cc = 0; cc < C / 2; cc += 16) {
+            const int c0 = half * (C / 2) + cc;
             float o[16];
             tc::tmem_ld16(tXO + lane_base + 64 + c0, o);
             tc::tmem_ld_wait();
@@ -240,7 +247,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
                 for (int i = 0; i < 16; ++i) ostage[(c0 + i) * DV + j] = from_f<T>(o[i]);
         }
 #pragma unroll
-        for (int c0 = 0; c0 < DK; c0 += 16) {
+        for (int cc = 0; cc < DK / 2; cc += 16) {
+            const int c0 = half * (DK / 2) + cc;
             float v[16];
             tc::tmem_ld16(tS + lane_base + c0, v);
             tc::tmem_ld_wait();
@@ -261,7 +269,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
     }
     if (ok) {  // final state: column j of S
 #pragma unroll
-        for (int c0 = 0; c0 < DK; c0 += 16) {
+        for (int cc = 0; cc < DK / 2; cc += 16) {
+            const int c0 = half * (DK / 2) + cc;
             float v[16];
             tc::tmem_ld16(tS + lane_base + c0, v);
             tc::tmem_ld_wait();

@@ -119,6 +119,23 @@ def test_edge_lengths_and_shapes(HK, HV, dk, dv, dtype):
     check_extend(w, gpu_extend(to_device(w)), oracle_extend(w))
 
 
+@pytest.mark.parametrize("HK,HV,dk,dv,dtype", SHAPES)
+def test_many_sequences_per_head_state_pass(HK, HV, dk, dv, dtype):
+    """Enough sequences that the per-(sequence, head) state pass is chosen over
+    the sliced one (the sliced grid, four CTAs per head, no longer fits on the
+    SMs); the small cases above run the sliced pass."""
+    spec = W.LayerSpec(HK=HK, HV=HV, dk=dk, dv=dv, dtype=dtype)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pattern = [1, 0, 63, 64, 65, 130, 3, 200, 17, 128, 5, 70]
+    n = sms // (4 * HV) + 1
+    lengths = (pattern * (n // len(pattern) + 1))[:n]
+    hi = [(i % 3) != 1 for i in range(n)]
+    slots = list(range(n))
+    slots[2] = -1
+    w = W.random_case(spec, lengths, P=n + 2, seed=HV * 10 + dk + dv, has_init=hi, slots=slots)
+    check_extend(w, gpu_extend(to_device(w)), oracle_extend(w))
+
+
 def test_page_shapes_with_nonzero_prefix_state():
     """The ragged page-boundary, exact-page and checkpoint-boundary shapes of the
     SGLang GDN test matrix (prefix (0,8,16) / extend (15,8,1); extend (16,);

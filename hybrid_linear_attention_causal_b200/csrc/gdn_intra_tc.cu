@@ -10,8 +10,12 @@
 //   D1  = [K; Q] K^T                          (tf32 MMA, M=128 N=64 K=dk)
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
-//   T   = (I + A)^{-1}                        (fp32, blocked 16x16 forward substitution)
+//   T   = (I + A)^{-1}                        (fp32, 32x32 blocks: forward substitution + block products)
 //   W   = T diag(beta e^gamma) K, U = T diag(beta) V   (tf32 MMAs, M=64 K=64)
+//
+// Both products share the A operand T diag(beta): W takes (diag(e^gamma) K)^T
+// and U the V^T tile as delivered.  K^T is transposed once per CTA from the
+// [K ; Q] tile and serves every value head through column scalings.
 //
 // (the WY/UT form of the gated delta rule).  For the serial state pass it
 // writes, per (chunk, value head): the tile [W ; diag(e^gamma) Q], the Aqk
@@ -35,17 +39,17 @@ constexpr int NT = 256;  // 8 warps; warp w reads TMEM sub-partition w % 4
 template <int DK, int DV>
 struct IntraTcSmem {
     float kq[2 * C * DK];  // [K ; Q*scale] tile from the prep kernel (bulk copy), K-major, 128 rows
-    float bk[DK * C];      // (diag(beta e^gamma) K)^T, K-major, DK rows x C
-    float bv[2][DV * C];   // V^T tiles (bulk copies, two heads in flight), scaled in place by beta
-    float t[C * C];        // T as a K-major tile, C rows x C
+    float kt[DK * C];      // K^T, K-major, DK rows x C (built once, shared by the value heads)
+    float kte[DK * C];     // (diag(e^gamma) K)^T of the current head, same layout
+    float bv[DV * C];      // V^T tile of the current head (bulk copy), K-major, DV rows x C
+    float t[C * C];        // T diag(beta) as a K-major tile, C rows x C
     float a[C][C + 1];     // A (fp32)
     float tf[C][C + 1];    // T (fp32)
-    float m[3][16][17];    // off-diagonal block products
+    float m[32][33];       // A21 T11
     float2 gb[2][C];       // (g, beta) of the two heads in flight
     float gam[C], beta[C], eg[C];
-    float fbk[C];          // beta_s e^{gamma_s}: column factor of (diag(beta e^gamma) K)^T
     float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
-    unsigned long long bar_mma, bar_kq, bar_v[2];
+    unsigned long long bar_mma, bar_kq, bar_v, bar_g[2];
     uint32_t tmem_base;
 };
 
@@ -70,39 +74,63 @@ __device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
     if (batch_rejected(p)) return;
-    const int id = blockIdx.x, hk = blockIdx.y;
-    if (id >= p.hdr[kHdrNumChunks]) return;
-    const int4 ch = p.chunk_tab[id];
-    const int slot = p.slots[ch.x];
-    if (slot < 0 || slot >= p.P) return;
     const LayerDims& d = p.d;
-    const int n = ch.z, G = d.G, HV = d.HV;
+    const int G = d.G, HV = d.HV, HK = d.HK;
+    // work items (chunk, qk head) in order; CTA b takes items b, b + gridDim.x, ... skipping padded requests
+    const int nitems = p.hdr[kHdrNumChunks] * HK;
+    auto next_item = [&](int it) {
+        for (; it < nitems; it += gridDim.x) {
+            const int sl = p.slots[p.chunk_tab[it / HK].x];
+            if (sl >= 0 && sl < p.P) break;
+        }
+        return it;
+    };
+    int item = next_item(blockIdx.x);
+    if (item >= nitems) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     IntraTcSmem<DK, DV>& sm = *reinterpret_cast<IntraTcSmem<DK, DV>*>(smem_raw);
     const uint32_t bar = tc::smem_u32(&sm.bar_mma), bar_kq = tc::smem_u32(&sm.bar_kq);
     constexpr uint32_t KQ_BYTES = 2 * C * DK * 4, VT_BYTES = DV * C * 4, GB_BYTES = C * 8;
-    auto fetch_v = [&](int jj) {  // V^T tile and gates of value head hk*G + jj into buffer jj & 1
-        const int b = jj & 1;
-        const size_t ch_h = (size_t)id * HV + hk * G + jj;
-        const uint32_t bv = tc::smem_u32(&sm.bar_v[b]);
-        tc::mbar_expect_tx(bv, VT_BYTES + GB_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.bv[b]), p.VT + ch_h * (DV * C), VT_BYTES, bv);
-        tc::bulk_g2s(tc::smem_u32(sm.gb[b]), p.GB + ch_h * C, GB_BYTES, bv);
+    const uint32_t bar_v = tc::smem_u32(&sm.bar_v);
+    auto kq_src = [&](int it) { return p.KQ + (size_t)it * (2 * C * DK); };  // item = chunk * HK + hk
+    auto head_row = [&](int it, int jj) { return (size_t)(it / HK) * HV + (it % HK) * G + jj; };
+    auto fetch_kq = [&](int it) {
+        tc::mbar_expect_tx(bar_kq, KQ_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.kq), kq_src(it), KQ_BYTES, bar_kq);
+    };
+    auto fetch_v = [&](int it, int jj) {  // V^T tile of value head jj of the item's group
+        tc::mbar_expect_tx(bar_v, VT_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.bv), p.VT + head_row(it, jj) * (DV * C), VT_BYTES, bar_v);
+    };
+    auto fetch_g = [&](int it, int jj) {  // gates of value head jj of the item's group into buffer jj & 1
+        const uint32_t bg = tc::smem_u32(&sm.bar_g[jj & 1]);
+        tc::mbar_expect_tx(bg, GB_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.gb[jj & 1]), p.GB + head_row(it, jj) * C, GB_BYTES, bg);
+    };
+    auto prefetch_l2 = [&](int it) {  // the next item's inputs, while this one computes
+        tc::bulk_prefetch_l2(kq_src(it), KQ_BYTES);
+        for (int jj = 0; jj < G; ++jj) {
+            tc::bulk_prefetch_l2(p.VT + head_row(it, jj) * (DV * C), VT_BYTES);
+            tc::bulk_prefetch_l2(p.GB + head_row(it, jj) * C, GB_BYTES);
+        }
     };
 
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(bar_kq, 1);
-        tc::mbar_init(tc::smem_u32(&sm.bar_v[0]), 1);
-        tc::mbar_init(tc::smem_u32(&sm.bar_v[1]), 1);
+        tc::mbar_init(bar_v, 1);
+        tc::mbar_init(tc::smem_u32(&sm.bar_g[0]), 1);
+        tc::mbar_init(tc::smem_u32(&sm.bar_g[1]), 1);
         tc::fence_mbar_init();
-        tc::mbar_expect_tx(bar_kq, KQ_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.kq), p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK), KQ_BYTES, bar_kq);
-        fetch_v(0);
-        if (G > 1) fetch_v(1);
+        fetch_kq(item);
+        fetch_g(item, 0);
+        if (G > 1) fetch_g(item, 1);
+        fetch_v(item, 0);
     }
+    // the upper off-diagonal block of T is zero for every head
+    for (int e = tid; e < 32 * 32; e += NT) sm.tf[e >> 5][32 + (e & 31)] = 0.f;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -110,9 +138,16 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
     const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;  // D1: 64 cols; W, U: M = 64 layout
     const int sp = warp & 3, half = warp >> 2;  // TMEM sub-partition, column half
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    // completed uses of each barrier so far, identical in every thread (parity = count & 1)
+    uint32_t n_kq = 0, n_v = 0, n_g[2] = {0u, 0u}, ph_mma = 0;
     bool ok = true;
+    while (ok && item < nitems) {
+    const int nxt = next_item(item + gridDim.x);
+    const int id = item / HK, hk = item % HK;
+    const int n = p.chunk_tab[id].z;
+    if (tid == 0 && nxt < nitems) prefetch_l2(nxt);
     if (tid == 0) {
-        ok = tc::mbar_wait(bar_kq, 0);
+        ok = tc::mbar_wait(bar_kq, n_kq & 1u);
         if (ok) {  // D1 = [K ; Q] K^T
             const uint32_t base = tc::smem_u32(sm.kq);
             constexpr uint32_t idesc = tc::idesc_tf32(128, 64);
@@ -122,14 +157,18 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             tc::mma_commit(bar);
         }
     }
-    // upper off-diagonal blocks of T are zero for every head
-    for (int e = tid; e < C * C; e += NT) {
-        const int r = e / C, s = e % C;
-        if ((s >> 4) > (r >> 4)) sm.tf[r][s] = 0.f;
-    }
+    // K^T (feature rows) from the k rows of the [K ; Q] tile, once for all value heads.  A warp reads
+    // one 128-byte core matrix of the tile (8 rows s x 4 features f): no bank conflicts.
+    ok = ok && tc::mbar_wait(bar_kq, n_kq & 1u);
+    ++n_kq;
+    if (ok)
+        for (int idx = tid; idx < DK * C; idx += NT) {
+            const int s = (idx & 7) + 8 * ((idx >> 5) & 7), f = ((idx >> 3) & 3) + 4 * (idx >> 8);
+            *reinterpret_cast<float*>(reinterpret_cast<char*>(sm.kt) + tc::kmajor_off(f, s, DK)) =
+                load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
+        }
     ok = __syncthreads_and(ok);
 
-    uint32_t ph_mma = 0;
     for (int j = 0; j < G && ok; ++j) {
         const int h = hk * G + j, b = j & 1;
         const size_t ch_h = (size_t)id * HV + h;
@@ -137,7 +176,8 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
         char* KTg = reinterpret_cast<char*>(p.KT + ch_h * (DK * C));
         float* Ug = p.U + ch_h * (C * DV);
-        bool okv = tc::mbar_wait(tc::smem_u32(&sm.bar_v[b]), (uint32_t)(j >> 1) & 1u);
+        bool okv = tc::mbar_wait(tc::smem_u32(&sm.bar_g[b]), n_g[b] & 1u);
+        ++n_g[b];
         if (okv && warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
             const float2 g0 = sm.gb[b][2 * lane], g1 = sm.gb[b][2 * lane + 1];
             const float pair = g0.x + g1.x;
@@ -155,8 +195,6 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             sm.eg[2 * lane] = __expf(gA);
             sm.eg[2 * lane + 1] = __expf(incl);
             const float gn = __shfl_sync(0xffffffffu, (n - 1) & 1 ? incl : gA, (n - 1) >> 1);
-            sm.fbk[2 * lane] = g0.y * __expf(gA);
-            sm.fbk[2 * lane + 1] = g1.y * __expf(incl);
             sm.fkt[2 * lane] = 2 * lane < n ? __expf(gn - gA) : 0.f;
             sm.fkt[2 * lane + 1] = 2 * lane + 1 < n ? __expf(gn - incl) : 0.f;
         }
@@ -201,109 +239,125 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             }
         }
         __syncthreads();
-        // T = (I + A)^{-1}: diagonal 16x16 blocks, one column per thread
-        if (tid < 64) {
-            const int o = 16 * (tid >> 4), c = tid & 15;
-            float t[16];
+        // T = (I + A)^{-1} in 32-row blocks: T = [[T11, 0], [T21, T22]], T21 = -T22 (A21 T11).
+        // Warps 0-1 invert the diagonal blocks, one column per lane held in registers, by forward
+        // substitution (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so that only
+        // one FMA per row sits on the dependent chain).  Meanwhile warps 2-7 write what needs only the
+        // gates: (diag(e^gamma) K)^T for W, the state pass's (diag(e^{gamma_n-gamma}) K)^T and the
+        // rows Qg = diag(e^gamma) Q of the [W ; Qg] tile.
+        if (warp < 2) {
+            const int o = 32 * warp;
+            float t[32];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float v = (r == c) ? 1.f : 0.f;
+            for (int r = 0; r < 32; ++r) {
+                const float* arow = &sm.a[o + r][o];
+                float acc[4] = {r == lane ? 1.f : 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int s = 0; s < r; ++s) v = fmaf(-sm.a[o + r][o + s], t[s], v);
-                t[r] = v;
+                for (int s = 0; s + 1 < r; ++s) acc[s & 3] = fmaf(-arow[s], t[s], acc[s & 3]);
+                const float base = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                t[r] = r > 0 ? fmaf(-arow[r - 1], t[r - 1], base) : base;
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sm.tf[o + r][o + c] = t[r];
+            for (int r = 0; r < 32; ++r) sm.tf[o + r][o + lane] = t[r];
+        } else {
+            constexpr int NW = NT - 64;
+            const int wt = tid - 64;
+            for (int idx = wt; idx < DK * C / 4; idx += NW) {
+                int f, s4;
+                tile_coord<DK>(idx, f, s4);
+                const uint32_t off = tc::kmajor_off(f, s4, DK);
+                const float4 k = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) + off);
+                store_f4(sm.kte, off,
+                         make_float4(tc::round_tf32(k.x * sm.eg[s4]), tc::round_tf32(k.y * sm.eg[s4 + 1]),
+                                     tc::round_tf32(k.z * sm.eg[s4 + 2]), tc::round_tf32(k.w * sm.eg[s4 + 3])));
+                store_f4(reinterpret_cast<float*>(KTg), off,
+                         make_float4(tc::round_tf32(k.x * sm.fkt[s4]), tc::round_tf32(k.y * sm.fkt[s4 + 1]),
+                                     tc::round_tf32(k.z * sm.fkt[s4 + 2]), tc::round_tf32(k.w * sm.fkt[s4 + 3])));
+            }
+            for (int idx = wt; idx < C * DK / 4; idx += NW) {  // same tile offsets as the q rows of [K ; Q]
+                int r, k4;
+                tile_coord<C>(idx, r, k4);
+                const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
+                const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
+                const float e = sm.eg[r];
+                store_f4(reinterpret_cast<float*>(WQg), off,
+                         make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
+                                     tc::round_tf32(q.w * e)));
+            }
+            if (wt < C) p.gam[ch_h * C + wt] = sm.gam[wt];
         }
         __syncthreads();
-        // off-diagonal blocks by distance: T_ij = -T_ii (sum_{k=j}^{i-1} A_ik T_kj); four partial sums
-        // per element keep the dependent FMA chains short
-        for (int dist = 1; dist < 4; ++dist) {
-            const int nel = (4 - dist) * 256;
-            for (int e = tid; e < nel; e += NT) {
-                const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const int bi = blk + dist, bj = blk;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int k = bj; k < bi; ++k)
+        {  // P = A21 T11 (T11 lower triangular): thread -> row r, columns c, c + 8, c + 16, c + 24
+            const int r = tid >> 3, c = tid & 7;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int s = 0; s < 32; ++s) {
+                const float av = sm.a[32 + r][s];
 #pragma unroll
-                    for (int s = 0; s < 16; ++s)
-                        acc[s & 3] = fmaf(sm.a[16 * bi + r][16 * k + s], sm.tf[16 * k + s][16 * bj + c], acc[s & 3]);
-                sm.m[blk][r][c] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                for (int k = 0; k < 4; ++k) acc[k] = fmaf(av, sm.tf[s][c + 8 * k], acc[k]);
             }
-            __syncthreads();
-            for (int e = tid; e < nel; e += NT) {
-                const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-                const int bi = blk + dist, bj = blk;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int s = 0; s < 16; ++s)
-                    acc[s & 3] = fmaf(sm.tf[16 * bi + r][16 * bi + s], sm.m[blk][s][c], acc[s & 3]);
-                sm.tf[16 * bi + r][16 * bj + c] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-            }
-            __syncthreads();
+            for (int k = 0; k < 4; ++k) sm.m[r][c + 8 * k] = acc[k];
         }
-        // T -> K-major tf32 tile
+        __syncthreads();
+        {  // T21 = -T22 P (T22 lower triangular)
+            const int r = tid >> 3, c = tid & 7;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int s = 0; s < 32; ++s) {
+                const float tv = sm.tf[32 + r][32 + s];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[k] = fmaf(tv, sm.m[s][c + 8 * k], acc[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sm.tf[32 + r][c + 8 * k] = -acc[k];
+        }
+        __syncthreads();
+        // T diag(beta) -> K-major tf32 tile
         for (int idx = tid; idx < C * C / 4; idx += NT) {
             int r, s4;
             tile_coord<C>(idx, r, s4);
             float v[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = (s4 + u <= r) ? tc::round_tf32(sm.tf[r][s4 + u]) : 0.f;
+            for (int u = 0; u < 4; ++u)
+                v[u] = (s4 + u <= r) ? tc::round_tf32(sm.tf[r][s4 + u] * sm.beta[s4 + u]) : 0.f;
             store_f4(sm.t, tc::kmajor_off(r, s4, C), make_float4(v[0], v[1], v[2], v[3]));
-        }
-        // (diag(beta e^gamma) K)^T into shared memory and (diag(e^{gamma_n - gamma}) K)^T to the
-        // workspace, both from the k rows of the [K ; Q] tile (row f = one feature across the rows s).
-        // A warp reads one 128-byte core matrix of the tile (8 rows s x 4 features f): no bank conflicts.
-        for (int idx = tid; idx < DK * C; idx += NT) {
-            const int s = (idx & 7) + 8 * ((idx >> 5) & 7), f = ((idx >> 3) & 3) + 4 * (idx >> 8);
-            const float kv = load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
-            const uint32_t off = tc::kmajor_off(f, s, DK);
-            *reinterpret_cast<float*>(reinterpret_cast<char*>(sm.bk) + off) = tc::round_tf32(kv * sm.fbk[s]);
-            *reinterpret_cast<float*>(KTg + off) = tc::round_tf32(kv * sm.fkt[s]);
-        }
-        // V^T scaled by beta, in place (tile layout unchanged)
-        for (int idx = tid; idx < DV * (C / 4); idx += NT) {
-            int f, s4;
-            tile_coord<DV>(idx, f, s4);
-            const uint32_t off = tc::kmajor_off(f, s4, DV);
-            float4 v = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.bv[b]) + off);
-            v = make_float4(tc::round_tf32(v.x * sm.beta[s4]), tc::round_tf32(v.y * sm.beta[s4 + 1]),
-                            tc::round_tf32(v.z * sm.beta[s4 + 2]), tc::round_tf32(v.w * sm.beta[s4 + 3]));
-            store_f4(sm.bv[b], off, v);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        if (tid == 0) {  // W = T diag(beta e^gamma) K,  U = T diag(beta) V   (M = 64)
-            const uint32_t bt = tc::smem_u32(sm.t), bkk = tc::smem_u32(sm.bk), bvv = tc::smem_u32(sm.bv[b]);
-            constexpr uint32_t iw = tc::idesc_tf32(64, DK), iu = tc::idesc_tf32(64, DV);
+        bool okm = true;
+        if (tid == 0) {  // W = (T diag(beta)) (diag(e^gamma) K),  U = (T diag(beta)) V   (M = 64)
+            okm = tc::mbar_wait(bar_v, n_v & 1u);
+            if (okm) {
+                const uint32_t bt = tc::smem_u32(sm.t), bkk = tc::smem_u32(sm.kte), bvv = tc::smem_u32(sm.bv);
+                constexpr uint32_t iw = tc::idesc_tf32(64, DK), iu = tc::idesc_tf32(64, DV);
 #pragma unroll
-            for (int s = 0; s < C / 8; ++s)
-                tc::mma_tf32(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
+                for (int s = 0; s < C / 8; ++s)
+                    tc::mma_tf32(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
 #pragma unroll
-            for (int s = 0; s < C / 8; ++s)
-                tc::mma_tf32(tU, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bvv, DV, s), iu, s > 0);
-            tc::mma_commit(bar);
+                for (int s = 0; s < C / 8; ++s)
+                    tc::mma_tf32(tU, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bvv, DV, s), iu, s > 0);
+                tc::mma_commit(bar);
+            }
         }
-        // while the MMA runs: rows 64..127 of the [W ; Qg] tile, Qg = diag(e^gamma) Q (same tile offsets)
-        for (int idx = tid; idx < C * DK / 4; idx += NT) {
-            int r, k4;
-            tile_coord<C>(idx, r, k4);
-            const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
-            const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
-            const float e = sm.eg[r];
-            store_f4(reinterpret_cast<float*>(WQg), off,
-                     make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
-                                 tc::round_tf32(q.w * e)));
-        }
-        if (tid < C) p.gam[ch_h * C + tid] = sm.gam[tid];
-        ok = tc::mbar_wait(bar, ph_mma);
+        ++n_v;
+        ok = okm && tc::mbar_wait(bar, ph_mma);  // okm is false only on tid 0, if the V tile never came
         ph_mma ^= 1;
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc::fence_after_sync();
-        if (tid == 0 && j + 2 < G) fetch_v(j + 2);  // buffer b is free again
+        if (tid == 0) {  // the V^T tile and gate buffer b are free again; after the last head, so is [K ; Q]
+            if (j + 1 < G) fetch_v(item, j + 1);
+            if (j + 2 < G) fetch_g(item, j + 2);
+            if (j == G - 1 && nxt < nitems) {  // the next item's tiles land during this epilogue
+                fetch_kq(nxt);
+                fetch_g(nxt, 0);
+                if (G > 1) fetch_g(nxt, 1);
+                fetch_v(nxt, 0);
+            }
+        }
         {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major.
            // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15;
            // the two warps of a sub-partition take one half of the columns each
@@ -337,12 +391,15 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         __syncthreads();
         tc::fence_after_sync();
     }
+    item = nxt;
+    }
     if (!ok && tid == 0) {
         raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
         // let copies already in flight land before the CTA's shared memory goes away
         for (int b = 0; b < 2; ++b)
-            for (uint32_t par = 0; par < 2; ++par) tc::mbar_wait(tc::smem_u32(&sm.bar_v[b]), par, 100000000ull);
-        tc::mbar_wait(bar_kq, 0, 100000000ull);
+            for (uint32_t par = 0; par < 2; ++par) tc::mbar_wait(tc::smem_u32(&sm.bar_g[b]), par, 100000000ull);
+        for (uint32_t par = 0; par < 2; ++par) tc::mbar_wait(bar_v, par, 100000000ull);
+        for (uint32_t par = 0; par < 2; ++par) tc::mbar_wait(bar_kq, par, 100000000ull);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -356,7 +413,13 @@ cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s) {
     const size_t shm = sizeof(IntraTcSmem<DK, DV>);
     cudaError_t e = cudaFuncSetAttribute(intra_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
-    intra_tc_kernel<DK, DV><<<dim3(p.max_chunks, p.d.HK), NT, shm, s>>>(p);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // persistent: one CTA per SM walks the (chunk, qk head) items
+    const long long items = (long long)p.max_chunks * p.d.HK;
+    const int grid = (int)(items < sms ? items : sms);
+    intra_tc_kernel<DK, DV><<<grid, NT, shm, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
 // norm for q, k) of shared-memory data.  Results are assembled as tiles in the
 // tensor core's shared-memory layout and leave by bulk stores:
 //   q / k unit: rows C..2C-1 / 0..C-1 of [K ; Q*scale] (tf32, K-major, 128 rows x dk)
-//   v unit:     V^T fp32 (K-major, dv rows x C) and (g, beta) for the C rows
+//   v unit:     V^T tf32 (K-major, dv rows x C) and (g, beta) for the C rows
 // Rows past the end of a ragged chunk are written as zeros.
 constexpr int kPrepThreads = 256;
 
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
             const int f = 8 * fg + ff, r4 = 4 * (4 * rg + cq);
             float y[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) y[u] = r4 + u < n ? conv(f, r4 + u) : 0.f;
+            for (int u = 0; u < 4; ++u) y[u] = r4 + u < n ? tc::round_tf32(conv(f, r4 + u)) : 0.f;
             *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(f, r4, DV)) =
                 make_float4(y[0], y[1], y[2], y[3]);
         }

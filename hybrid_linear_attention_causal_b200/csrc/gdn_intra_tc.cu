@@ -10,7 +10,7 @@
 //   D1  = [K; Q] K^T                          (tf32 MMA, M=128 N=64 K=dk)
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
-//   T   = (I + A)^{-1}                        (fp32, 32x32 blocks: forward substitution + block products)
+//   T   = (I + A)^{-1}                        (fp32: 16x16 forward substitution + block products)
 //   W   = T diag(beta e^gamma) K, U = T diag(beta) V   (tf32 MMAs, M=64 K=64)
 //
 // Both products share the A operand T diag(beta): W takes (diag(e^gamma) K)^T
@@ -23,9 +23,9 @@
 // tensor core's shared-memory layout so the state pass bulk-copies them --
 // plus U (fp32) and gamma.  Operands are staged in shared memory as K-major
 // no-swizzle tiles rounded to tf32 (round to nearest); accumulators live in
-// tensor memory.  One thread issues the MMAs; the eight warps read their
-// sub-partition's 32-lane slice of tensor memory (two warps per slice, one
-// half of the columns each) for the CUDA-core steps.
+// tensor memory.  One thread issues the MMAs; the sixteen warps read their
+// sub-partition's 32-lane slice of tensor memory (four warps per slice, one
+// group of columns each) for the CUDA-core steps.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -34,7 +34,8 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NT = 256;  // 8 warps; warp w reads TMEM sub-partition w % 4
+constexpr int NT = 512;        // 16 warps; warp w reads TMEM sub-partition w % 4
+constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
 
 template <int DK, int DV>
 struct IntraTcSmem {
@@ -44,8 +45,9 @@ struct IntraTcSmem {
     float bv[DV * C];      // V^T tile of the current head (bulk copy), K-major, DV rows x C
     float t[C * C];        // T diag(beta) as a K-major tile, C rows x C
     float a[C][C + 1];     // A (fp32)
-    float tf[C][C + 1];    // T (fp32)
-    float m[32][33];       // A21 T11
+    float tf[C][C + 4];    // T (fp32), the blocks the next level of the inverse reads
+    float m[32][36];       // A21 T11
+    float y[2][16][17];    // A21 D1 inside each 32x32 diagonal block
     float2 gb[2][C];       // (g, beta) of the two heads in flight
     float gam[C], beta[C], eg[C];
     float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
@@ -129,14 +131,19 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         if (G > 1) fetch_g(item, 1);
         fetch_v(item, 0);
     }
-    // the upper off-diagonal block of T is zero for every head
-    for (int e = tid; e < 32 * 32; e += NT) sm.tf[e >> 5][32 + (e & 31)] = 0.f;
+    // blocks of T above the diagonal are zero for every head: in the tile, and in the two 16x16
+    // corners of the 32x32 diagonal blocks that the inverse reads back
+    for (int e = tid; e < C * C; e += NT) sm.t[e] = 0.f;
+    for (int e = tid; e < 2 * 256; e += NT) {
+        const int o = 32 * (e >> 8);
+        sm.tf[o + ((e >> 4) & 15)][o + 16 + (e & 15)] = 0.f;
+    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
     const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;  // D1: 64 cols; W, U: M = 64 layout
-    const int sp = warp & 3, half = warp >> 2;  // TMEM sub-partition, column half
+    const int sp = warp & 3, cg = warp >> 2;  // TMEM sub-partition, column group
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     // completed uses of each barrier so far, identical in every thread (parity = count & 1)
     uint32_t n_kq = 0, n_v = 0, n_g[2] = {0u, 0u}, ph_mma = 0;
@@ -207,11 +214,12 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         tc::fence_after_sync();
         const float gl = sm.gam[n - 1];
         {  // A (sub-partitions 0-1: k.k rows) and the masked decayed q.k tile (2-3: q.k rows) from D1;
-           // the two warps of a sub-partition take one half of the 64 columns each
-            const int r = (sp & 1) * 32 + lane, c0 = 32 * half;
-            float row[32];
+           // the warps of a sub-partition take one group of C / NCG columns each
+            constexpr int NC = C / NCG;
+            const int r = (sp & 1) * 32 + lane, c0 = NC * cg;
+            float row[NC];
 #pragma unroll
-            for (int c = 0; c < 32; c += 16) {
+            for (int c = 0; c < NC; c += 16) {
                 float v[16];
                 tc::tmem_ld16(tD1 + lane_base + c0 + c, v);
 #pragma unroll
@@ -221,13 +229,13 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
             const float gr = sm.gam[r], br = sm.beta[r];
             if (sp < 2) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < NC; ++i) {
                     const int s = c0 + i;
                     sm.a[r][s] = (s < r && r < n) ? br * __expf(gr - sm.gam[s]) * row[i] : 0.f;
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
+                for (int i = 0; i < NC; i += 4) {
                     float o[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
@@ -238,31 +246,64 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 }
             }
         }
+        // what needs only the gates and goes to the workspace: the state pass's
+        // (diag(e^{gamma_n-gamma}) K)^T and the rows Qg = diag(e^gamma) Q of the [W ; Qg] tile; these
+        // stores drain while the exponentials above and the inverse below compute
+        for (int idx = tid; idx < DK * C / 4; idx += NT) {
+            int f, s4;
+            tile_coord<DK>(idx, f, s4);
+            const uint32_t off = tc::kmajor_off(f, s4, DK);
+            const float4 k = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) + off);
+            store_f4(reinterpret_cast<float*>(KTg), off,
+                     make_float4(tc::round_tf32(k.x * sm.fkt[s4]), tc::round_tf32(k.y * sm.fkt[s4 + 1]),
+                                 tc::round_tf32(k.z * sm.fkt[s4 + 2]), tc::round_tf32(k.w * sm.fkt[s4 + 3])));
+        }
+        for (int idx = tid; idx < C * DK / 4; idx += NT) {  // same tile offsets as the q rows of [K ; Q]
+            int r, k4;
+            tile_coord<C>(idx, r, k4);
+            const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
+            const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
+            const float e = sm.eg[r];
+            store_f4(reinterpret_cast<float*>(WQg), off,
+                     make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
+                                 tc::round_tf32(q.w * e)));
+        }
+        if (tid < C) p.gam[ch_h * C + tid] = sm.gam[tid];
         __syncthreads();
-        // T = (I + A)^{-1} in 32-row blocks: T = [[T11, 0], [T21, T22]], T21 = -T22 (A21 T11).
-        // Warps 0-1 invert the diagonal blocks, one column per lane held in registers, by forward
-        // substitution (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so that only
-        // one FMA per row sits on the dependent chain).  Meanwhile warps 2-7 write what needs only the
-        // gates: (diag(e^gamma) K)^T for W, the state pass's (diag(e^{gamma_n-gamma}) K)^T and the
-        // rows Qg = diag(e^gamma) Q of the [W ; Qg] tile.
-        if (warp < 2) {
-            const int o = 32 * warp;
-            float t[32];
+        // T = (I + A)^{-1}, by blocks.  Every final entry goes straight into the K-major tf32 tile of
+        // T diag(beta) (the A operand of W and U); the fp32 copy tf holds what the next level reads.
+        //   level 1: the four diagonal 16x16 blocks by forward substitution, one column per lane held
+        //            in registers (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so
+        //            one FMA per row sits on the dependent chain); warps 4-7 meanwhile build
+        //            (diag(e^gamma) K)^T for W.
+        //   level 2: within each 32x32 diagonal block, X = -D2 (A21 D1).
+        //   level 3: T21 = -T22 (A21 T11) for the lower-left 32x32 block.
+        auto put_t = [&](int r, int c, float v) {
+            *reinterpret_cast<float*>(reinterpret_cast<char*>(sm.t) + tc::kmajor_off(r, c, C)) =
+                tc::round_tf32(v * sm.beta[c]);
+        };
+        if (warp < 4) {
+            if (lane < 16) {
+                const int o = 16 * warp, c = lane;
+                float t[16];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const float* arow = &sm.a[o + r][o];
-                float acc[4] = {r == lane ? 1.f : 0.f, 0.f, 0.f, 0.f};
+                for (int r = 0; r < 16; ++r) {
+                    const float* arow = &sm.a[o + r][o];
+                    float acc[2] = {r == c ? 1.f : 0.f, 0.f};
 #pragma unroll
-                for (int s = 0; s + 1 < r; ++s) acc[s & 3] = fmaf(-arow[s], t[s], acc[s & 3]);
-                const float base = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                t[r] = r > 0 ? fmaf(-arow[r - 1], t[r - 1], base) : base;
+                    for (int s = 0; s + 1 < r; ++s) acc[s & 1] = fmaf(-arow[s], t[s], acc[s & 1]);
+                    const float base = acc[0] + acc[1];
+                    t[r] = r > 0 ? fmaf(-arow[r - 1], t[r - 1], base) : base;
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    sm.tf[o + r][o + c] = t[r];
+                    put_t(o + r, o + c, t[r]);
+                }
             }
-#pragma unroll
-            for (int r = 0; r < 32; ++r) sm.tf[o + r][o + lane] = t[r];
         } else {
-            constexpr int NW = NT - 64;
-            const int wt = tid - 64;
-            for (int idx = wt; idx < DK * C / 4; idx += NW) {
+            constexpr int NW = NT - 128;
+            for (int idx = tid - 128; idx < DK * C / 4; idx += NW) {
                 int f, s4;
                 tile_coord<DK>(idx, f, s4);
                 const uint32_t off = tc::kmajor_off(f, s4, DK);
@@ -270,58 +311,50 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 store_f4(sm.kte, off,
                          make_float4(tc::round_tf32(k.x * sm.eg[s4]), tc::round_tf32(k.y * sm.eg[s4 + 1]),
                                      tc::round_tf32(k.z * sm.eg[s4 + 2]), tc::round_tf32(k.w * sm.eg[s4 + 3])));
-                store_f4(reinterpret_cast<float*>(KTg), off,
-                         make_float4(tc::round_tf32(k.x * sm.fkt[s4]), tc::round_tf32(k.y * sm.fkt[s4 + 1]),
-                                     tc::round_tf32(k.z * sm.fkt[s4 + 2]), tc::round_tf32(k.w * sm.fkt[s4 + 3])));
             }
-            for (int idx = wt; idx < C * DK / 4; idx += NW) {  // same tile offsets as the q rows of [K ; Q]
-                int r, k4;
-                tile_coord<C>(idx, r, k4);
-                const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
-                const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
-                const float e = sm.eg[r];
-                store_f4(reinterpret_cast<float*>(WQg), off,
-                         make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
-                                     tc::round_tf32(q.w * e)));
-            }
-            if (wt < C) p.gam[ch_h * C + wt] = sm.gam[wt];
         }
         __syncthreads();
-        {  // P = A21 T11 (T11 lower triangular): thread -> row r, columns c, c + 8, c + 16, c + 24
-            const int r = tid >> 3, c = tid & 7;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        static_assert(NT == 512, "the level 2 and 3 thread maps below assume 512 threads");
+        {  // level 2: thread -> 32-block bb, row r, column c
+            const int bb = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
+            const int o0 = 32 * bb, o1 = o0 + 16;
+            float y[2] = {0.f, 0.f};
+#pragma unroll
+            for (int s = 0; s < 16; ++s)  // Y = A21 D1
+                y[s & 1] = fmaf(sm.a[o1 + r][o0 + s], sm.tf[o0 + s][o0 + c], y[s & 1]);
+            sm.y[bb][r][c] = y[0] + y[1];
+            __syncthreads();
+            float x[2] = {0.f, 0.f};
+#pragma unroll
+            for (int s = 0; s < 16; ++s)  // X = -D2 Y
+                x[s & 1] = fmaf(sm.tf[o1 + r][o1 + s], sm.y[bb][s][c], x[s & 1]);
+            sm.tf[o1 + r][o0 + c] = -(x[0] + x[1]);
+            put_t(o1 + r, o0 + c, -(x[0] + x[1]));
+        }
+        __syncthreads();
+        {  // level 3: thread -> row r, columns c2, c2 + 1
+            const int r = tid >> 4, c2 = 2 * (tid & 15);
+            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll 8
-            for (int s = 0; s < 32; ++s) {
+            for (int s = 0; s < 32; ++s) {  // P = A21 T11
                 const float av = sm.a[32 + r][s];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) acc[k] = fmaf(av, sm.tf[s][c + 8 * k], acc[k]);
+                const float2 tv = *reinterpret_cast<const float2*>(&sm.tf[s][c2]);
+                acc[s & 1].x = fmaf(av, tv.x, acc[s & 1].x);
+                acc[s & 1].y = fmaf(av, tv.y, acc[s & 1].y);
             }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sm.m[r][c + 8 * k] = acc[k];
-        }
-        __syncthreads();
-        {  // T21 = -T22 P (T22 lower triangular)
-            const int r = tid >> 3, c = tid & 7;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            *reinterpret_cast<float2*>(&sm.m[r][c2]) =
+                make_float2(acc[0].x + acc[1].x, acc[0].y + acc[1].y);
+            __syncthreads();
+            acc[0] = acc[1] = make_float2(0.f, 0.f);
 #pragma unroll 8
-            for (int s = 0; s < 32; ++s) {
+            for (int s = 0; s < 32; ++s) {  // T21 = -T22 P
                 const float tv = sm.tf[32 + r][32 + s];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) acc[k] = fmaf(tv, sm.m[s][c + 8 * k], acc[k]);
+                const float2 pv = *reinterpret_cast<const float2*>(&sm.m[s][c2]);
+                acc[s & 1].x = fmaf(tv, pv.x, acc[s & 1].x);
+                acc[s & 1].y = fmaf(tv, pv.y, acc[s & 1].y);
             }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sm.tf[32 + r][c + 8 * k] = -acc[k];
-        }
-        __syncthreads();
-        // T diag(beta) -> K-major tf32 tile
-        for (int idx = tid; idx < C * C / 4; idx += NT) {
-            int r, s4;
-            tile_coord<C>(idx, r, s4);
-            float v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                v[u] = (s4 + u <= r) ? tc::round_tf32(sm.tf[r][s4 + u] * sm.beta[s4 + u]) : 0.f;
-            store_f4(sm.t, tc::kmajor_off(r, s4, C), make_float4(v[0], v[1], v[2], v[3]));
+            put_t(32 + r, c2, -(acc[0].x + acc[1].x));
+            put_t(32 + r, c2 + 1, -(acc[0].y + acc[1].y));
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -360,11 +393,11 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         }
         {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major.
            // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15;
-           // the two warps of a sub-partition take one half of the columns each
+           // the warps of a sub-partition take one group of columns each
             const bool valid = lane < 16;
             const int r = sp * 16 + lane;
 #pragma unroll
-            for (int c0 = half * (DK / 2); c0 < (half + 1) * (DK / 2); c0 += 16) {
+            for (int c0 = cg * (DK / NCG); c0 < (cg + 1) * (DK / NCG); c0 += 16) {
                 float v[16];
                 tc::tmem_ld16(tW + lane_base + c0, v);
                 tc::tmem_ld_wait();
@@ -376,7 +409,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                                              tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
             }
 #pragma unroll
-            for (int c0 = half * (DV / 2); c0 < (half + 1) * (DV / 2); c0 += 16) {
+            for (int c0 = cg * (DV / NCG); c0 < (cg + 1) * (DV / NCG); c0 += 16) {
                 float v[16];
                 tc::tmem_ld16(tU + lane_base + c0, v);
                 tc::tmem_ld_wait();

@@ -91,6 +91,7 @@ struct ExtendArgs {
     int32_t* hdr;
     int4* chunk_tab;    // [max_chunks] {seq, first row, length, chunk index within seq}
     int32_t* seq_chunk0;// [N+1] first chunk id of each sequence
+    int32_t* seq_order; // [N] sequences by decreasing chunk count (the state pass's launch order)
     // per chunk, written by the prep kernel (conv + SiLU + L2 norm + gates):
     float* KQ;          // [max_chunks, HK, 2*C*dk] [K ; Q*scale] tf32, K-major tile of 128 rows
     float* VT;          // [max_chunks, HV, dv*C]   V^T tf32, K-major tile of dv rows x C

@@ -77,6 +77,24 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     __threadfence_block();
     __syncthreads();
     const int total = s_base;
+    // Longest sequences first: the state pass runs each sequence's chunks in series, so its grid
+    // starts the long chains before the short ones.  (Rank by chunk count, ties by index; more
+    // than 1024 sequences keep their order.)
+    if (p.N <= 1024) {
+        if (tid < p.N) s_scan[tid] = p.seq_chunk0[tid + 1] - p.seq_chunk0[tid];
+        __syncthreads();
+        if (tid < p.N) {
+            const int mine = s_scan[tid];
+            int rank = 0;
+            for (int j = 0; j < p.N; ++j) {
+                const int o = s_scan[j];
+                rank += (o > mine || (o == mine && j < tid)) ? 1 : 0;
+            }
+            p.seq_order[rank] = tid;
+        }
+    } else {
+        for (int i = tid; i < p.N; i += 1024) p.seq_order[i] = i;
+    }
     for (int id = tid; id < total; id += 1024) {
         int lo = 0, hi = p.N - 1;  // last sequence whose first chunk id <= id
         while (lo < hi) {
@@ -319,6 +337,7 @@ size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max
     size_t off = kHeaderBytes;
     off += al(mc * sizeof(int4));
     off += al(((size_t)max_N + 1) * sizeof(int32_t));
+    off += al((size_t)max_N * sizeof(int32_t));
     off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
     off += al(per * d.dv * C);
     off += al(per * C * 2);
@@ -342,6 +361,7 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
     size_t off = kHeaderBytes;
     e.chunk_tab = reinterpret_cast<int4*>(base + off); off += al((size_t)mc * sizeof(int4));
     e.seq_chunk0 = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
+    e.seq_order = reinterpret_cast<int32_t*>(base + off); off += al((size_t)max_N * sizeof(int32_t));
     e.KQ = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
     e.VT = reinterpret_cast<float*>(base + off); off += al(per * d.dv * C);
     e.GB = reinterpret_cast<float2*>(base + off); off += al(per * C * 2);

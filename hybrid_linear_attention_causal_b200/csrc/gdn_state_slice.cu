@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(NT, 1) state_slice_kernel(ExtendArgs p) {
     const LayerDims& d = p.d;
     const int HV = d.HV;
     // slices of one head are adjacent in launch order, so they run together and share the tiles in L2
-    const int sl = blockIdx.x % NSL, h = (blockIdx.x / NSL) % HV, nseq = blockIdx.x / (NSL * HV);
+    const int sl = blockIdx.x % NSL, h = (blockIdx.x / NSL) % HV, nseq = p.seq_order[blockIdx.x / (NSL * HV)];
     const int j0 = sl * SW;
     const int len = p.cu[nseq + 1] - p.cu[nseq];
     if (len == 0) return;

@@ -73,9 +73,10 @@ __device__ __forceinline__ void put_st_row(float* st, int j, int c0, const float
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
     if (batch_rejected(p)) return;
-    const int nseq = blockIdx.x, h = blockIdx.y;
     const LayerDims& d = p.d;
     const int HV = d.HV;
+    // all heads of the longest sequence first, then the next longest, ...
+    const int h = blockIdx.x % HV, nseq = p.seq_order[blockIdx.x / HV];
     const int len = p.cu[nseq + 1] - p.cu[nseq];
     if (len == 0) return;
     const int slot = p.slots[nseq];
@@ -299,7 +300,7 @@ cudaError_t launch_state_head(const ExtendArgs& p, cudaStream_t s) {
     cudaError_t e =
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
-    state_tc_kernel<T, DK, DV><<<dim3(p.N, p.d.HV), NT, shm, s>>>(p);
+    state_tc_kernel<T, DK, DV><<<(unsigned)p.N * (unsigned)p.d.HV, NT, shm, s>>>(p);
     return cudaGetLastError();
 }
 

@@ -8,18 +8,26 @@
 //
 //   [X^T | O^T]  = S^T [W ; Qg]^T           M=dv N=128 K=dk   (X = W S, O = Qg S)
 //   V'^T         = U^T - X^T                 CUDA cores, per thread row j
+//   Snew^T       = V'^T K~                   M=dv N=dk  K=64  (K~ = diag(e^{gamma_n-gamma}) K)
+//   S^T         <- e^{gamma_n} S^T + Snew^T  CUDA cores, fp32 in registers
 //   O^T         += V'^T Aqk^T                M=dv N=64  K=64
-//   S^T         <- e^{gamma_n} S^T + V'^T K~ M=dv N=dk  K=64  (K~ = diag(e^{gamma_n-gamma}) K)
 //
-// where Qg = diag(e^gamma) Q (q carries the output scale).  The fp32 state
-// S^T lives in tensor memory (the MMA accumulates onto it in fp32); a tf32
-// copy in shared memory is the operand of the next chunk.  Eight warps: the
-// two warps of a TMEM sub-partition share its 32 accumulator rows and take
-// one half of the columns each.  The intra-chunk
-// kernel wrote [W ; Qg], Aqk and K~^T already as tf32 tiles in the tensor
-// core's shared-memory layout; they arrive by asynchronous bulk copies, each
-// reissued for the next chunk as soon as the MMA that reads it has finished,
-// so the copies overlap the rest of the chunk.  U (fp32) is read per thread.
+// where Qg = diag(e^gamma) Q (q carries the output scale).  The chain from one
+// chunk's state to the next runs through the first product, V', the state
+// product and the update; everything else is kept off it:
+//   - a ninth warp only issues the MMAs and the bulk copies, so the eight
+//     compute warps never wait behind an issue loop; it issues the output
+//     product only once the state product has completed;
+//   - the fp32 state lives in registers (each thread holds one half of row j
+//     of S^T), the state product goes to a fresh accumulator and the update
+//     is one FMA per element, written straight into the tf32 operand copy;
+//   - [X^T | O^T] is double-buffered in tensor memory: a chunk's outputs are
+//     read and stored while the next chunk's first product runs;
+//   - the tiles [W ; Qg], K~^T and Aqk (written by the intra-chunk kernel as
+//     tf32 in the tensor core's layout) each have their own barrier and are
+//     refetched as soon as the product that reads them completes.
+// The two compute warps of a TMEM sub-partition share its 32 accumulator rows
+// and take one half of the columns each.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -28,17 +36,25 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NT = 256;  // 8 warps: two per TMEM sub-partition, each taking half of the columns
+constexpr int NCW = 8;               // compute warps
+constexpr int NT = (NCW + 1) * 32;   // + the issuing warp
+constexpr int ISSUER = NCW * 32;     // its lane 0
 
-template <int DK, int DV>
+// bf16 outputs are staged in shared memory and leave as 16-byte vectors while
+// the next state product runs; fp32 outputs (whose staging tile would not fit)
+// are stored by each thread
+template <typename T>
+constexpr bool kStageOut = sizeof(T) == 2;
+
+template <typename T, int DK, int DV>
 struct StateTcSmem {
     float st[DV * DK];     // S^T tile, K-major: DV rows x DK (tf32 copy of the state)
     float wq[2 * C * DK];  // [W ; Qg] tile (bulk copy), K-major: 128 rows x DK
     float aq[C * C];       // Aqk tile (bulk copy), K-major: C rows (r) x C (s)
     float kt[DK * C];      // K~^T tile (bulk copy), K-major: DK rows (i) x C (s)
     float vt[DV * C];      // V'^T tile, K-major: DV rows (j) x C (s)
-    float gam[C];
-    unsigned long long bar_mma, bar_wq, bar_ak;
+    T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
+    unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq;
     uint32_t tmem_base;
 };
 
@@ -46,23 +62,9 @@ __device__ __forceinline__ void store_f4(float* tile, uint32_t off, float4 v) {
     *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + off) = v;
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-        "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-        "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Writes 16 consecutive fp32 values of S^T row j (columns c0..c0+15) into the
-// K-major tf32 operand tile.
-template <int DK, int DV>
-__device__ __forceinline__ void put_st_row(float* st, int j, int c0, const float (&v)[16]) {
+// tf32 copies of 16 consecutive values of S^T row j (columns c0..c0+15) into the operand tile
+template <int DV>
+__device__ __forceinline__ void put_st16(float* st, int j, int c0, const float* v) {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
         store_f4(st, tc::kmajor_off(j, c0 + 4 * q, DV),
@@ -89,154 +91,72 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
         return;
     }
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    StateTcSmem<DK, DV>& sm = *reinterpret_cast<StateTcSmem<DK, DV>*>(smem_raw);
-    const uint32_t bar_mma = tc::smem_u32(&sm.bar_mma), bar_wq = tc::smem_u32(&sm.bar_wq),
-                   bar_ak = tc::smem_u32(&sm.bar_ak);
+    StateTcSmem<T, DK, DV>& sm = *reinterpret_cast<StateTcSmem<T, DK, DV>*>(smem_raw);
+    const uint32_t bar_x = tc::smem_u32(&sm.bar_x), bar_s = tc::smem_u32(&sm.bar_s),
+                   bar_o = tc::smem_u32(&sm.bar_o), bar_wq = tc::smem_u32(&sm.bar_wq),
+                   bar_kt = tc::smem_u32(&sm.bar_kt), bar_aq = tc::smem_u32(&sm.bar_aq);
     constexpr uint32_t WQ_BYTES = 2 * C * DK * 4, AQ_BYTES = C * C * 4, KT_BYTES = DK * C * 4;
     const int c_begin = p.seq_chunk0[nseq], c_end = p.seq_chunk0[nseq + 1];
     auto fetch_wq = [&](int id) {
         tc::mbar_expect_tx(bar_wq, WQ_BYTES);
         tc::bulk_g2s(tc::smem_u32(sm.wq), p.WQ + ((size_t)id * HV + h) * (2 * C * DK), WQ_BYTES, bar_wq);
     };
-    auto fetch_ak = [&](int id) {
-        tc::mbar_expect_tx(bar_ak, AQ_BYTES + KT_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.aq), p.AQ + ((size_t)id * HV + h) * (C * C), AQ_BYTES, bar_ak);
-        tc::bulk_g2s(tc::smem_u32(sm.kt), p.KT + ((size_t)id * HV + h) * (DK * C), KT_BYTES, bar_ak);
+    auto fetch_kt = [&](int id) {
+        tc::mbar_expect_tx(bar_kt, KT_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.kt), p.KT + ((size_t)id * HV + h) * (DK * C), KT_BYTES, bar_kt);
     };
-    if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 256);
-    if (tid == 0) {
-        tc::mbar_init(bar_mma, 1);
+    auto fetch_aq = [&](int id) {
+        tc::mbar_expect_tx(bar_aq, AQ_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.aq), p.AQ + ((size_t)id * HV + h) * (C * C), AQ_BYTES, bar_aq);
+    };
+    if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
+    if (tid == ISSUER) {
+        tc::mbar_init(bar_x, 1);
+        tc::mbar_init(bar_s, 1);
+        tc::mbar_init(bar_o, 1);
         tc::mbar_init(bar_wq, 1);
-        tc::mbar_init(bar_ak, 1);
+        tc::mbar_init(bar_kt, 1);
+        tc::mbar_init(bar_aq, 1);
         tc::fence_mbar_init();
         fetch_wq(c_begin);
-        fetch_ak(c_begin);
+        fetch_kt(c_begin);
+        fetch_aq(c_begin);
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tm = sm.tmem_base;
-    const uint32_t tXO = tm, tS = tm + 128;  // [X^T | O^T] (128 columns), S^T (DK columns)
-    const int sp = warp & 3, half = warp >> 2;  // TMEM sub-partition, column half
-    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
-    // this thread's accumulator row j (the value-dimension index)
-    const bool rowv = DV == 128 || lane < 16;
-    const int j = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
 
-    // initial state: S^T row j = column j of S
+    // compute warps: thread (sp, half, lane) owns row j of S^T, columns half * DK/2 .. + DK/2
+    const int sp = warp & 3, half = (warp >> 2) & 1;
+    const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
+    const bool rowv = warp < NCW && (DV == 128 || lane < 16);
+    const int j = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
     const bool init = p.has_init ? p.has_init[nseq] != 0 : true;
     float* Sg = p.ssm_state + ((size_t)slot * HV + h) * DK * DV;
+    float s[DK / 2];
 #pragma unroll
-    for (int cc = 0; cc < DK / 2; cc += 16) {
-        const int c0 = half * (DK / 2) + cc;
-        float v[16];
+    for (int i = 0; i < DK / 2; ++i) s[i] = (init && rowv) ? Sg[(size_t)(half * (DK / 2) + i) * DV + j] : 0.f;
+    if (rowv)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = (init && rowv) ? Sg[(size_t)(c0 + i) * DV + j] : 0.f;
-        tmem_st16(tS + lane_base + c0, v);
-        if (rowv) put_st_row<DK, DV>(sm.st, j, c0, v);
-    }
-    tmem_st_wait();
+        for (int cc = 0; cc < DK / 2; cc += 16) put_st16<DV>(sm.st, j, half * (DK / 2) + cc, &s[cc]);
+    // U column j of a chunk, rows of this thread's half
+    float u[C / 2];
+    auto load_u = [&](int id) {
+        const float* Ug = p.U + ((size_t)id * HV + h) * (C * DV) + (size_t)half * (C / 2) * DV + j;
+#pragma unroll
+        for (int q = 0; q < C / 2; ++q) u[q] = rowv ? Ug[(size_t)q * DV] : 0.f;
+    };
+    load_u(c_begin);
+    int4 ch = p.chunk_tab[c_begin];
+    float gl = p.gam[((size_t)c_begin * HV + h) * C + ch.z - 1];  // gamma_n of this chunk
+    int4 ch_nx = c_begin + 1 < c_end ? p.chunk_tab[c_begin + 1] : ch;
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    const uint32_t tm = sm.tmem_base;
+    const uint32_t tS = tm + 256;  // Snew^T (DK columns); [X^T | O^T] double buffer at tm, tm + 128
 
-    uint32_t ph_mma = 0;
-    bool ok = true;
-    // gamma of the next chunk, loaded one chunk ahead so no global load sits before an MMA issue
-    float g_next = tid < C ? p.gam[((size_t)c_begin * HV + h) * C + tid] : 0.f;
-    for (int id = c_begin; id < c_end; ++id) {
-        const uint32_t ph_ld = (uint32_t)(id - c_begin) & 1u;
-        const int4 ch = p.chunk_tab[id];
-        const int t0 = ch.y, n = ch.z;
-        const size_t ch_h = (size_t)id * HV + h;
-        if (tid < C) {
-            sm.gam[tid] = g_next;
-            if (id + 1 < c_end) g_next = p.gam[(ch_h + HV) * C + tid];
-        }
-        // U column j of this chunk, rows of this warp's half (consumed after the first MMA)
-        float u[C / 2];
-        {
-            const float* Ug = p.U + ch_h * (C * DV) + (size_t)half * (C / 2) * DV;
-#pragma unroll
-            for (int s = 0; s < C / 2; ++s) u[s] = rowv ? Ug[(size_t)s * DV + j] : 0.f;
-        }
-        bool okw = true;
-        if (tid == 0) {
-            okw = tc::mbar_wait(bar_wq, ph_ld);
-            if (okw) {  // [X^T | O^T] = S^T [W ; Qg]^T
-                const uint32_t a = tc::smem_u32(sm.st), b = tc::smem_u32(sm.wq);
-                constexpr uint32_t idesc = tc::idesc_tf32(DV, 128);
-#pragma unroll
-                for (int s = 0; s < DK / 8; ++s)
-                    tc::mma_tf32(tXO, tc::desc_kmajor(a, DV, s), tc::desc_kmajor(b, 2 * C, s), idesc, s > 0);
-                tc::mma_commit(bar_mma);
-            }
-        }
-        ok = __syncthreads_and(okw);
-        if (!ok) break;
-        ok = __syncthreads_and(tc::mbar_wait(bar_mma, ph_mma));
-        ph_mma ^= 1;
-        if (!ok) break;
-        tc::fence_after_sync();
-        if (tid == 0 && id + 1 < c_end) fetch_wq(id + 1);  // the [W ; Qg] tile is free again
-        const float egl = expf(sm.gam[n - 1]);
-        // V'^T row j = U^T row j - X^T row j; the fp32 state is scaled by e^{gamma_n}
-#pragma unroll
-        for (int cc = 0; cc < C / 2; cc += 16) {
-            const int c0 = half * (C / 2) + cc;
-            float x[16];
-            tc::tmem_ld16(tXO + lane_base + c0, x);
-            tc::tmem_ld_wait();
-            if (rowv)
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    store_f4(sm.vt, tc::kmajor_off(j, c0 + 4 * q, DV),
-                             make_float4(tc::round_tf32(u[cc + 4 * q] - x[4 * q]),
-                                         tc::round_tf32(u[cc + 4 * q + 1] - x[4 * q + 1]),
-                                         tc::round_tf32(u[cc + 4 * q + 2] - x[4 * q + 2]),
-                                         tc::round_tf32(u[cc + 4 * q + 3] - x[4 * q + 3])));
-        }
-#pragma unroll
-        for (int cc = 0; cc < DK / 2; cc += 16) {
-            const int c0 = half * (DK / 2) + cc;
-            float v[16];
-            tc::tmem_ld16(tS + lane_base + c0, v);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= egl;
-            tmem_st16(tS + lane_base + c0, v);
-        }
-        tmem_st_wait();
-        tc::fence_smem_to_async();
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
-        bool oka = true;
-        if (tid == 0) {
-            oka = tc::mbar_wait(bar_ak, ph_ld);
-            if (oka) {  // O^T += V'^T Aqk^T ;  S^T += V'^T K~
-                const uint32_t av = tc::smem_u32(sm.vt), bq = tc::smem_u32(sm.aq), bk = tc::smem_u32(sm.kt);
-                constexpr uint32_t io = tc::idesc_tf32(DV, 64), is = tc::idesc_tf32(DV, DK);
-#pragma unroll
-                for (int s = 0; s < C / 8; ++s)
-                    tc::mma_tf32(tXO + 64, tc::desc_kmajor(av, DV, s), tc::desc_kmajor(bq, C, s), io, true);
-#pragma unroll
-                for (int s = 0; s < C / 8; ++s)
-                    tc::mma_tf32(tS, tc::desc_kmajor(av, DV, s), tc::desc_kmajor(bk, DK, s), is, true);
-                tc::mma_commit(bar_mma);
-            }
-        }
-        ok = __syncthreads_and(oka);
-        if (!ok) break;
-        ok = __syncthreads_and(tc::mbar_wait(bar_mma, ph_mma));
-        ph_mma ^= 1;
-        if (!ok) break;
-        tc::fence_after_sync();
-        if (tid == 0 && id + 1 < c_end) fetch_ak(id + 1);  // the Aqk and K~^T tiles are free again
-        // outputs: O^T row j is staged as column j of O [C][DV] in the (now free) V'^T tile, then the
-        // chunk's rows leave as 16-byte vectors
-        T* ostage = reinterpret_cast<T*>(sm.vt);
+    // rows t < n of O (chunk at row t0), this thread's column j and half of the rows, from the
+    // O^T half of an [X^T | O^T] buffer: into the staging tile, or straight to global memory
+    auto put_out = [&](uint32_t tXO, int t0, int n) {
 #pragma unroll
         for (int cc = 0; cc < C / 2; cc += 16) {
             const int c0 = half * (C / 2) + cc;
@@ -245,58 +165,177 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
             tc::tmem_ld_wait();
             if (rowv)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) ostage[(c0 + i) * DV + j] = from_f<T>(o[i]);
+                for (int i = 0; i < 16; ++i) {
+                    if constexpr (kStageOut<T>) sm.ostage[(c0 + i) * DV + j] = from_f<T>(o[i]);
+                    else if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + j] = from_f<T>(o[i]);
+                }
         }
+    };
+    // (compute warps) the staged rows t < n leave as 16-byte vectors
+    auto send_out = [&](int t0, int n) {
+        if constexpr (kStageOut<T>) {
+            constexpr int VPR = DV * (int)sizeof(T) / 16;  // vectors per row
+            for (int e = tid; e < n * VPR; e += NCW * 32) {
+                const int r = e / VPR, v = e % VPR;
+                reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * HV + h) * DV)[v] =
+                    reinterpret_cast<const uint4*>(sm.ostage + r * DV)[v];
+            }
+        }
+    };
+
+    bool ok = true;
+    int prev_t0 = 0, prev_n = 0;  // the chunk whose outputs are still in tensor memory
+    for (int id = c_begin; id < c_end; ++id) {
+        const uint32_t ph = (uint32_t)(id - c_begin) & 1u;
+        const uint32_t tXO = tm + ph * 128;
+        // loads one chunk ahead: the next chunk's gamma_n; two ahead: its table entry
+        float gl_nx = 0.f;
+        int4 ch_nx2 = ch_nx;
+        if (id + 1 < c_end) gl_nx = p.gam[((size_t)(id + 1) * HV + h) * C + ch_nx.z - 1];
+        if (id + 2 < c_end) ch_nx2 = p.chunk_tab[id + 2];
+        bool okl = true;
+        if (tid == ISSUER) {
+            okl = tc::mbar_wait(bar_wq, ph);
+            if (okl) {  // [X^T | O^T] = S^T [W ; Qg]^T
+                const uint32_t a = tc::smem_u32(sm.st), b = tc::smem_u32(sm.wq);
+                constexpr uint32_t idesc = tc::idesc_tf32(DV, 128);
 #pragma unroll
-        for (int cc = 0; cc < DK / 2; cc += 16) {
-            const int c0 = half * (DK / 2) + cc;
-            float v[16];
-            tc::tmem_ld16(tS + lane_base + c0, v);
-            tc::tmem_ld_wait();
-            if (rowv) put_st_row<DK, DV>(sm.st, j, c0, v);
+                for (int k = 0; k < DK / 8; ++k)
+                    tc::mma_tf32(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
+                tc::mma_commit(bar_x);
+            }
+            if (okl && id > c_begin) {  // this chunk's Aqk, once the previous output product is done with the tile
+                okl = tc::mbar_wait(bar_o, ph ^ 1u);
+                if (okl) fetch_aq(id);
+            }
+            if (okl) {
+                okl = tc::mbar_wait(bar_x, ph);
+                if (okl && id + 1 < c_end) fetch_wq(id + 1);  // the [W ; Qg] tile is free again
+            }
+        } else if (warp < NCW) {
+            if (id > c_begin) {  // the previous chunk's outputs leave while this chunk's first product runs
+                okl = __all_sync(0xffffffffu, tc::mbar_wait(bar_o, ph ^ 1u));
+                if (okl) {
+                    tc::fence_after_sync();
+                    put_out(tm + (ph ^ 1u) * 128, prev_t0, prev_n);
+                }
+            }
+            okl = __all_sync(0xffffffffu, okl && tc::mbar_wait(bar_x, ph));
+            tc::fence_after_sync();
+            if (okl) {  // V'^T row j = U^T row j - X^T row j
+#pragma unroll
+                for (int cc = 0; cc < C / 2; cc += 16) {
+                    const int c0 = half * (C / 2) + cc;
+                    float x[16];
+                    tc::tmem_ld16(tXO + lane_base + c0, x);
+                    tc::tmem_ld_wait();
+                    if (rowv)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            store_f4(sm.vt, tc::kmajor_off(j, c0 + 4 * q, DV),
+                                     make_float4(tc::round_tf32(u[cc + 4 * q] - x[4 * q]),
+                                                 tc::round_tf32(u[cc + 4 * q + 1] - x[4 * q + 1]),
+                                                 tc::round_tf32(u[cc + 4 * q + 2] - x[4 * q + 2]),
+                                                 tc::round_tf32(u[cc + 4 * q + 3] - x[4 * q + 3])));
+                }
+                if (id + 1 < c_end) load_u(id + 1);
+            }
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
-        __syncthreads();
+        ok = __syncthreads_and(okl);
+        if (!ok) break;
         tc::fence_after_sync();
-        {
-            constexpr int VPR = DV * (int)sizeof(T) / 16;  // 16-byte vectors per output row
-            for (int e = tid; e < n * VPR; e += NT) {
-                const int r = e / VPR, v = e % VPR;
-                reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * HV + h) * DV)[v] =
-                    reinterpret_cast<const uint4*>(ostage + r * DV)[v];
+        if (tid == ISSUER) {
+            okl = tc::mbar_wait(bar_kt, ph);
+            if (okl) {  // Snew^T = V'^T K~
+                const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt);
+                constexpr uint32_t is = tc::idesc_tf32(DV, DK);
+#pragma unroll
+                for (int k = 0; k < C / 8; ++k)
+                    tc::mma_tf32(tS, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bk, DK, k), is, k > 0);
+                tc::mma_commit(bar_s);
+                okl = tc::mbar_wait(bar_s, ph);
+            }
+            if (okl && id + 1 < c_end) fetch_kt(id + 1);  // the K~^T tile is free again
+            if (okl) okl = tc::mbar_wait(bar_aq, ph);
+            if (okl) {  // O^T += V'^T Aqk^T, off the state chain
+                const uint32_t av = tc::smem_u32(sm.vt), bq = tc::smem_u32(sm.aq);
+                constexpr uint32_t io = tc::idesc_tf32(DV, 64);
+#pragma unroll
+                for (int k = 0; k < C / 8; ++k)
+                    tc::mma_tf32(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
+                tc::mma_commit(bar_o);
+            }
+        } else if (warp < NCW) {
+            if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
+                                                          // state product runs meanwhile
+            okl = __all_sync(0xffffffffu, tc::mbar_wait(bar_s, ph));
+            if (okl) {  // S^T <- e^{gamma_n} S^T + Snew^T, and its tf32 copy for the next chunk
+                tc::fence_after_sync();
+                const float egl = expf(gl);
+#pragma unroll
+                for (int cc = 0; cc < DK / 2; cc += 16) {
+                    const int c0 = half * (DK / 2) + cc;
+                    float v[16];
+                    tc::tmem_ld16(tS + lane_base + c0, v);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) s[cc + i] = fmaf(egl, s[cc + i], v[i]);
+                    if (rowv) put_st16<DV>(sm.st, j, c0, &s[cc]);
+                }
             }
         }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        ok = __syncthreads_and(okl);
+        if (!ok) break;
+        tc::fence_after_sync();
+        prev_t0 = ch.y;
+        prev_n = ch.z;
+        ch = ch_nx;
+        ch_nx = ch_nx2;
+        gl = gl_nx;
     }
-    if (ok) {  // final state: column j of S
+    if (ok) {
+        if (warp < NCW) {
+            const uint32_t ph = (uint32_t)(c_end - 1 - c_begin) & 1u;
+            const bool okw = __all_sync(0xffffffffu, tc::mbar_wait(bar_o, ph));
+            if (okw) {  // the last chunk's outputs
+                tc::fence_after_sync();
+                put_out(tm + ph * 128, prev_t0, prev_n);
+            } else if (lane == 0) {
+                raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+            }
+            if (rowv)  // final state: column j of S
 #pragma unroll
-        for (int cc = 0; cc < DK / 2; cc += 16) {
-            const int c0 = half * (DK / 2) + cc;
-            float v[16];
-            tc::tmem_ld16(tS + lane_base + c0, v);
-            tc::tmem_ld_wait();
-            if (rowv)
-#pragma unroll
-                for (int i = 0; i < 16; ++i) Sg[(size_t)(c0 + i) * DV + j] = v[i];
+                for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
         }
-    } else if (tid == 0) {
+        if constexpr (kStageOut<T>) {
+            __syncthreads();
+            if (warp < NCW) send_out(prev_t0, prev_n);
+        }
+    } else if (tid == ISSUER) {
         raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
-        // let copies already in flight land before the CTA's shared memory goes away
-        tc::mbar_wait(bar_wq, 0, 100000000ull);
-        tc::mbar_wait(bar_wq, 1, 100000000ull);
-        tc::mbar_wait(bar_ak, 0, 100000000ull);
-        tc::mbar_wait(bar_ak, 1, 100000000ull);
+        // let copies and products already in flight finish before the CTA's shared and tensor
+        // memory go away
+        for (uint32_t par = 0; par < 2; ++par) {
+            tc::mbar_wait(bar_wq, par, 100000000ull);
+            tc::mbar_wait(bar_kt, par, 100000000ull);
+            tc::mbar_wait(bar_aq, par, 100000000ull);
+            tc::mbar_wait(bar_o, par, 100000000ull);
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tm, 256);
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
 }
 
 }  // namespace
 
 template <typename T, int DK, int DV>
 cudaError_t launch_state_head(const ExtendArgs& p, cudaStream_t s) {
-    const size_t shm = sizeof(StateTcSmem<DK, DV>);
+    const size_t shm = sizeof(StateTcSmem<T, DK, DV>);
     cudaError_t e =
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;

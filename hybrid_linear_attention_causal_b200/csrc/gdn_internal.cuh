@@ -102,7 +102,7 @@ struct ExtendArgs {
     float* WQ;          // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], K-major, 128 rows
     float* AQ;          // [max_chunks, HV, C*C]     masked decayed q.k, K-major, C rows
     float* KT;          // [max_chunks, HV, dk*C]    (diag(e^{gamma_n-gamma}) K)^T, K-major, dk rows
-    float* U;           // [max_chunks, HV, C, dv]   fp32, row-major
+    float* U;           // [max_chunks, HV, dv*C]    U^T fp32, K-major tile of dv rows (j) x C
     float* gam;         // [max_chunks, HV, C]       in-chunk cumulative g
 };
 

@@ -11,7 +11,8 @@
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
 //   T   = (I + A)^{-1}                        (fp32: 16x16 forward substitution + block products)
-//   W   = T diag(beta e^gamma) K, U = T diag(beta) V   (tf32 MMAs, M=64 K=64)
+//   W   = T diag(beta e^gamma) K, U = T diag(beta) V   (tf32 MMAs, K=64; U formed
+//                                                       transposed, U^T = V^T (T diag(beta))^T)
 //
 // Both products share the A operand T diag(beta): W takes (diag(e^gamma) K)^T
 // and U the V^T tile as delivered.  K^T is transposed once per CTA from the
@@ -142,7 +143,8 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
-    const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;  // D1: 64 cols; W, U: M = 64 layout
+    // D1: 64 columns; W: M = 64 layout, DK columns; U^T: M = DV, 64 columns
+    const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;
     const int sp = warp & 3, cg = warp >> 2;  // TMEM sub-partition, column group
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     // completed uses of each barrier so far, identical in every thread (parity = count & 1)
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         char* WQg = reinterpret_cast<char*>(p.WQ + ch_h * (2 * C * DK));
         char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
         char* KTg = reinterpret_cast<char*>(p.KT + ch_h * (DK * C));
-        float* Ug = p.U + ch_h * (C * DV);
+        char* Ug = reinterpret_cast<char*>(p.U + ch_h * (DV * C));  // U^T, K-major tile: DV rows (j) x C
         bool okv = tc::mbar_wait(tc::smem_u32(&sm.bar_g[b]), n_g[b] & 1u);
         ++n_g[b];
         if (okv && warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
@@ -361,17 +363,17 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         __syncthreads();
         tc::fence_after_sync();
         bool okm = true;
-        if (tid == 0) {  // W = (T diag(beta)) (diag(e^gamma) K),  U = (T diag(beta)) V   (M = 64)
+        if (tid == 0) {  // W = (T diag(beta)) (diag(e^gamma) K) (M = 64), U^T = V^T (T diag(beta))^T (M = DV)
             okm = tc::mbar_wait(bar_v, n_v & 1u);
             if (okm) {
                 const uint32_t bt = tc::smem_u32(sm.t), bkk = tc::smem_u32(sm.kte), bvv = tc::smem_u32(sm.bv);
-                constexpr uint32_t iw = tc::idesc_tf32(64, DK), iu = tc::idesc_tf32(64, DV);
+                constexpr uint32_t iw = tc::idesc_tf32(64, DK), iu = tc::idesc_tf32(DV, 64);
 #pragma unroll
                 for (int s = 0; s < C / 8; ++s)
                     tc::mma_tf32(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 8; ++s)
-                    tc::mma_tf32(tU, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bvv, DV, s), iu, s > 0);
+                    tc::mma_tf32(tU, tc::desc_kmajor(bvv, DV, s), tc::desc_kmajor(bt, C, s), iu, s > 0);
                 tc::mma_commit(bar);
             }
         }
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 fetch_v(nxt, 0);
             }
         }
-        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U rows -> fp32 row-major.
+        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U -> U^T tile (fp32, K-major).
            // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15;
            // the warps of a sub-partition take one group of columns each
             const bool valid = lane < 16;
@@ -408,16 +410,19 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                                  make_float4(tc::round_tf32(v[4 * q]), tc::round_tf32(v[4 * q + 1]),
                                              tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
             }
-#pragma unroll
-            for (int c0 = cg * (DV / NCG); c0 < (cg + 1) * (DV / NCG); c0 += 16) {
+            {  // U^T row j (M = DV layout), the warp's group of C / NCG columns r
+                static_assert(C / NCG == 16, "one 16-column load per warp");
+                const bool vj = DV == 128 || lane < 16;
+                const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
+                const int c0 = cg * 16;
                 float v[16];
                 tc::tmem_ld16(tU + lane_base + c0, v);
                 tc::tmem_ld_wait();
-                if (valid)
+                if (vj)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<float4*>(Ug + (size_t)r * DV + c0 + 4 * q) =
-                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                        store_f4(reinterpret_cast<float*>(Ug), tc::kmajor_off(jr, c0 + 4 * q, DV),
+                                 make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
             }
         }
         tc::fence_before_sync();

@@ -195,9 +195,14 @@ __global__ void __launch_bounds__(NT, 1) state_slice_kernel(ExtendArgs p) {
         for (int c = 0; c < SW; ++c) s[c] = 0.f;
     }
     if (own) put_col<SW>(sm.st, i_row, s);
-    // threads 0..C-1 own row t of X and V'; their U row is loaded one chunk ahead
+    // threads 0..C-1 own row t of X and V'; U row t (column t of the U^T tile), this slice's
+    // columns, is loaded one chunk ahead
     float u[SW];
-    auto load_u = [&](int id) { load_row<SW>(p.U + ((size_t)id * HV + h) * (C * DV) + (size_t)tid * DV + j0, u); };
+    auto load_u = [&](int id) {
+        const char* Ut = reinterpret_cast<const char*>(p.U + ((size_t)id * HV + h) * (DV * C));
+#pragma unroll
+        for (int c = 0; c < SW; ++c) u[c] = *reinterpret_cast<const float*>(Ut + tc::kmajor_off(j0 + c, tid, DV));
+    };
     if (tid < C) load_u(c_begin);
     int4 ch = p.chunk_tab[c_begin];
     float gl = p.gam[((size_t)c_begin * HV + h) * C + ch.z - 1];  // gamma_n of this chunk

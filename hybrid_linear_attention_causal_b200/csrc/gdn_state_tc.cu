@@ -25,7 +25,10 @@
 //     read and stored while the next chunk's first product runs;
 //   - the tiles [W ; Qg], K~^T and Aqk (written by the intra-chunk kernel as
 //     tf32 in the tensor core's layout) each have their own barrier and are
-//     refetched as soon as the product that reads them completes.
+//     refetched as soon as the product that reads them completes;
+//   - the intra-chunk kernel writes U^T in the layout of the V'^T operand
+//     tile, so it lands in that tile by one bulk copy and V' is formed in
+//     place (each thread rewrites exactly the elements it read).
 // The two compute warps of a TMEM sub-partition share its 32 accumulator rows
 // and take one half of the columns each.
 
@@ -52,9 +55,9 @@ struct StateTcSmem {
     float wq[2 * C * DK];  // [W ; Qg] tile (bulk copy), K-major: 128 rows x DK
     float aq[C * C];       // Aqk tile (bulk copy), K-major: C rows (r) x C (s)
     float kt[DK * C];      // K~^T tile (bulk copy), K-major: DK rows (i) x C (s)
-    float vt[DV * C];      // V'^T tile, K-major: DV rows (j) x C (s)
+    float vt[DV * C];      // U^T tile (bulk copy), overwritten in place by V'^T: K-major, DV rows (j) x C (s)
     T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
-    unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq;
+    unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq, bar_u;
     uint32_t tmem_base;
 };
 
@@ -94,7 +97,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
     StateTcSmem<T, DK, DV>& sm = *reinterpret_cast<StateTcSmem<T, DK, DV>*>(smem_raw);
     const uint32_t bar_x = tc::smem_u32(&sm.bar_x), bar_s = tc::smem_u32(&sm.bar_s),
                    bar_o = tc::smem_u32(&sm.bar_o), bar_wq = tc::smem_u32(&sm.bar_wq),
-                   bar_kt = tc::smem_u32(&sm.bar_kt), bar_aq = tc::smem_u32(&sm.bar_aq);
+                   bar_kt = tc::smem_u32(&sm.bar_kt), bar_aq = tc::smem_u32(&sm.bar_aq),
+                   bar_u = tc::smem_u32(&sm.bar_u);
     constexpr uint32_t WQ_BYTES = 2 * C * DK * 4, AQ_BYTES = C * C * 4, KT_BYTES = DK * C * 4;
     const int c_begin = p.seq_chunk0[nseq], c_end = p.seq_chunk0[nseq + 1];
     auto fetch_wq = [&](int id) {
@@ -104,6 +108,11 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
     auto fetch_kt = [&](int id) {
         tc::mbar_expect_tx(bar_kt, KT_BYTES);
         tc::bulk_g2s(tc::smem_u32(sm.kt), p.KT + ((size_t)id * HV + h) * (DK * C), KT_BYTES, bar_kt);
+    };
+    auto u_src = [&](int id) { return p.U + ((size_t)id * HV + h) * (DV * C); };
+    auto fetch_u = [&](int id) {
+        tc::mbar_expect_tx(bar_u, DV * C * 4);
+        tc::bulk_g2s(tc::smem_u32(sm.vt), u_src(id), DV * C * 4, bar_u);
     };
     auto fetch_aq = [&](int id) {
         tc::mbar_expect_tx(bar_aq, AQ_BYTES);
@@ -117,10 +126,12 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
         tc::mbar_init(bar_wq, 1);
         tc::mbar_init(bar_kt, 1);
         tc::mbar_init(bar_aq, 1);
+        tc::mbar_init(bar_u, 1);
         tc::fence_mbar_init();
         fetch_wq(c_begin);
         fetch_kt(c_begin);
         fetch_aq(c_begin);
+        fetch_u(c_begin);
     }
 
     // compute warps: thread (sp, half, lane) owns row j of S^T, columns half * DK/2 .. + DK/2
@@ -136,14 +147,6 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
     if (rowv)
 #pragma unroll
         for (int cc = 0; cc < DK / 2; cc += 16) put_st16<DV>(sm.st, j, half * (DK / 2) + cc, &s[cc]);
-    // U column j of a chunk, rows of this thread's half
-    float u[C / 2];
-    auto load_u = [&](int id) {
-        const float* Ug = p.U + ((size_t)id * HV + h) * (C * DV) + (size_t)half * (C / 2) * DV + j;
-#pragma unroll
-        for (int q = 0; q < C / 2; ++q) u[q] = rowv ? Ug[(size_t)q * DV] : 0.f;
-    };
-    load_u(c_begin);
     int4 ch = p.chunk_tab[c_begin];
     float gl = p.gam[((size_t)c_begin * HV + h) * C + ch.z - 1];  // gamma_n of this chunk
     int4 ch_nx = c_begin + 1 < c_end ? p.chunk_tab[c_begin + 1] : ch;
@@ -204,10 +207,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
                     tc::mma_tf32(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
                 tc::mma_commit(bar_x);
             }
-            if (okl && id > c_begin) {  // this chunk's Aqk, once the previous output product is done with the tile
-                okl = tc::mbar_wait(bar_o, ph ^ 1u);
-                if (okl) fetch_aq(id);
-            }
+            if (okl && id + 1 < c_end) tc::bulk_prefetch_l2(u_src(id + 1), DV * C * 4);
             if (okl) {
                 okl = tc::mbar_wait(bar_x, ph);
                 if (okl && id + 1 < c_end) fetch_wq(id + 1);  // the [W ; Qg] tile is free again
@@ -220,9 +220,9 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
                     put_out(tm + (ph ^ 1u) * 128, prev_t0, prev_n);
                 }
             }
-            okl = __all_sync(0xffffffffu, okl && tc::mbar_wait(bar_x, ph));
+            okl = __all_sync(0xffffffffu, okl && tc::mbar_wait(bar_x, ph) && tc::mbar_wait(bar_u, ph));
             tc::fence_after_sync();
-            if (okl) {  // V'^T row j = U^T row j - X^T row j
+            if (okl) {  // V'^T row j = U^T row j - X^T row j, in place: each thread rewrites what it read
 #pragma unroll
                 for (int cc = 0; cc < C / 2; cc += 16) {
                     const int c0 = half * (C / 2) + cc;
@@ -231,14 +231,14 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
                     tc::tmem_ld_wait();
                     if (rowv)
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            store_f4(sm.vt, tc::kmajor_off(j, c0 + 4 * q, DV),
-                                     make_float4(tc::round_tf32(u[cc + 4 * q] - x[4 * q]),
-                                                 tc::round_tf32(u[cc + 4 * q + 1] - x[4 * q + 1]),
-                                                 tc::round_tf32(u[cc + 4 * q + 2] - x[4 * q + 2]),
-                                                 tc::round_tf32(u[cc + 4 * q + 3] - x[4 * q + 3])));
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t off = tc::kmajor_off(j, c0 + 4 * q, DV);
+                            const float4 u = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.vt) + off);
+                            store_f4(sm.vt, off,
+                                     make_float4(tc::round_tf32(u.x - x[4 * q]), tc::round_tf32(u.y - x[4 * q + 1]),
+                                                 tc::round_tf32(u.z - x[4 * q + 2]), tc::round_tf32(u.w - x[4 * q + 3])));
+                        }
                 }
-                if (id + 1 < c_end) load_u(id + 1);
             }
         }
         tc::fence_smem_to_async();
@@ -266,6 +266,12 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
                 for (int k = 0; k < C / 8; ++k)
                     tc::mma_tf32(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
                 tc::mma_commit(bar_o);
+                // the next chunk's Aqk and U^T, once the output product is done with the Aqk and V'^T tiles
+                okl = tc::mbar_wait(bar_o, ph);
+                if (okl && id + 1 < c_end) {
+                    fetch_aq(id + 1);
+                    fetch_u(id + 1);
+                }
             }
         } else if (warp < NCW) {
             if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
@@ -324,6 +330,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
             tc::mbar_wait(bar_kt, par, 100000000ull);
             tc::mbar_wait(bar_aq, par, 100000000ull);
             tc::mbar_wait(bar_o, par, 100000000ull);
+            tc::mbar_wait(bar_u, par, 100000000ull);
         }
     }
     tc::fence_before_sync();

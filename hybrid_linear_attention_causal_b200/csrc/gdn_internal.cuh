@@ -123,17 +123,10 @@ __device__ __forceinline__ bool batch_rejected(const ExtendArgs& p) { return p.h
 template <int DK, int DV>
 cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s);
 
-// Serial state pass + outputs on tensor cores.  launch_state picks one of:
-//   launch_state_head  (gdn_state_tc.cu):    one CTA per (sequence, value head)
-//   launch_state_slice (gdn_state_slice.cu): one CTA per (sequence, value head,
-//                                            slice of dv / kStateSlices columns)
-constexpr int kStateSlices = 4;
+// Serial state pass + outputs on tensor cores (gdn_state_tc.cu): one CTA per
+// (sequence, value head), longest sequences first.
 template <typename T, int DK, int DV>
 cudaError_t launch_state(const ExtendArgs& p, cudaStream_t s);
-template <typename T, int DK, int DV>
-cudaError_t launch_state_head(const ExtendArgs& p, cudaStream_t s);
-template <typename T, int DK, int DV>
-cudaError_t launch_state_slice(const ExtendArgs& p, cudaStream_t s);
 
 // Records the calling thread's i-th profiling event on `s` if one is set
 // (see gdn_set_launch_events); a no-op otherwise.

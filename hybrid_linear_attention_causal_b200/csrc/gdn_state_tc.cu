@@ -341,29 +341,13 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
 }  // namespace
 
 template <typename T, int DK, int DV>
-cudaError_t launch_state_head(const ExtendArgs& p, cudaStream_t s) {
+cudaError_t launch_state(const ExtendArgs& p, cudaStream_t s) {
     const size_t shm = sizeof(StateTcSmem<T, DK, DV>);
     cudaError_t e =
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     state_tc_kernel<T, DK, DV><<<(unsigned)p.N * (unsigned)p.d.HV, NT, shm, s>>>(p);
     return cudaGetLastError();
-}
-
-// One CTA per (sequence, head) runs each head's chunks with the whole value
-// dimension; the sliced kernel spends four times the MMA instructions on the
-// same work (a tcgen05 MMA costs about the same few dozen cycles whatever its
-// N), so it only pays when the per-head grid leaves most SMs idle: when the
-// sliced grid still fits in one wave, the slices shorten each sequence's
-// serial chain instead.
-template <typename T, int DK, int DV>
-cudaError_t launch_state(const ExtendArgs& p, cudaStream_t s) {
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    if ((long long)p.N * p.d.HV * kStateSlices <= (long long)sms) return launch_state_slice<T, DK, DV>(p, s);
-    return launch_state_head<T, DK, DV>(p, s);
 }
 
 #define GDN_STATE_INST(T)                                                        \

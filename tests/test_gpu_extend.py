@@ -120,10 +120,10 @@ def test_edge_lengths_and_shapes(HK, HV, dk, dv, dtype):
 
 
 @pytest.mark.parametrize("HK,HV,dk,dv,dtype", SHAPES)
-def test_many_sequences_per_head_state_pass(HK, HV, dk, dv, dtype):
-    """Enough sequences that the per-(sequence, head) state pass is chosen over
-    the sliced one (the sliced grid, four CTAs per head, no longer fits on the
-    SMs); the small cases above run the sliced pass."""
+def test_many_sequences(HK, HV, dk, dv, dtype):
+    """More (sequence, head) state-pass CTAs than one wave of the SMs, with
+    ragged lengths, padded and fresh requests: the longest-first launch order
+    and the CTAs that start late."""
     spec = W.LayerSpec(HK=HK, HV=HV, dk=dk, dv=dv, dtype=dtype)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     pattern = [1, 0, 63, 64, 65, 130, 3, 200, 17, 128, 5, 70]

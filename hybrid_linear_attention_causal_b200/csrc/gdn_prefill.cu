@@ -128,7 +128,7 @@ struct PrepShape {
     static constexpr int PAD = VE;                 // row padding: spreads rows over banks
     static constexpr size_t XS_BYTES = (((size_t)(C + 3) * (NCH + PAD) * sizeof(T)) + 15) & ~(size_t)15;
     static constexpr size_t TILE_BYTES = (size_t)C * NCH * sizeof(float);
-    static constexpr size_t W_BYTES = (size_t)NCH * 5 * sizeof(float);  // 4 taps + bias per channel
+    static constexpr size_t W_BYTES = (size_t)NCH * 5 * sizeof(float);  // 4 taps per channel, then the biases
     static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + W_BYTES + C * sizeof(float2);
 };
 
@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T* xs = reinterpret_cast<T*>(smem_raw);  // row i <-> token t0 - 3 + i
     float* tile = reinterpret_cast<float*>(smem_raw + S::XS_BYTES);
-    float* wsm = reinterpret_cast<float*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);  // [nch][5]
+    float4* wsm = reinterpret_cast<float4*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);  // [nch] taps
+    float* bsm = reinterpret_cast<float*>(wsm + S::NCH);                                // [nch] biases
     float2* gbs = reinterpret_cast<float2*>(smem_raw + S::XS_BYTES + S::TILE_BYTES + S::W_BYTES);
     const T* x = reinterpret_cast<const T*>(p.x);
     const T* w = reinterpret_cast<const T*>(p.conv_w);
@@ -190,20 +191,26 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
             else v = init ? cs[(size_t)(c_first + c) * 3 + i] : from_f<T>(0.f);
             xs[(size_t)i * ld + c] = v;
         }
-        for (int e = tid; e < nch * 5; e += kPrepThreads) {
-            const int c = e / 5, j = e % 5;
+        for (int c = tid; c < nch; c += kPrepThreads) {
             const int cg = c_first + c;
-            wsm[e] = j < 4 ? to_f(w[(size_t)cg * 4 + j]) : (bias ? to_f(bias[cg]) : 0.f);
+            wsm[c] = make_float4(to_f(w[(size_t)cg * 4]), to_f(w[(size_t)cg * 4 + 1]), to_f(w[(size_t)cg * 4 + 2]),
+                                 to_f(w[(size_t)cg * 4 + 3]));
+            bsm[c] = bias ? to_f(bias[cg]) : 0.f;
         }
     }
     __syncthreads();
+    // SiLU with the fast exponential and division: their error (a few ulp) is far below the
+    // tf32 rounding every prep output goes through
+    auto silu = [](float x) { return __fdividef(x, 1.0f + __expf(-x)); };
     // conv + SiLU of staged column c at output row r (r < n)
     auto conv = [&](int c, int r) -> float {
-        const float* wc = wsm + c * 5;
-        float acc = wc[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc = fmaf(wc[j], to_f(xs[(size_t)(r + j) * ld + c]), acc);
-        return silu_f(acc);
+        const float4 wc = wsm[c];
+        float acc = bsm[c];
+        acc = fmaf(wc.x, to_f(xs[(size_t)r * ld + c]), acc);
+        acc = fmaf(wc.y, to_f(xs[(size_t)(r + 1) * ld + c]), acc);
+        acc = fmaf(wc.z, to_f(xs[(size_t)(r + 2) * ld + c]), acc);
+        acc = fmaf(wc.w, to_f(xs[(size_t)(r + 3) * ld + c]), acc);
+        return silu(acc);
     };
     if (!isv) {
         // warp w: rows 8w .. 8w+7; lane (rr = lane & 7, cc = lane >> 3) takes row 8w + rr and the
@@ -234,9 +241,21 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
             const int ff = idx & 7, cq = (idx >> 3) & 3, rest = idx >> 5;
             const int fg = rest % (DV / 8), rg = rest / (DV / 8);
             const int f = 8 * fg + ff, r4 = 4 * (4 * rg + cq);
+            // four consecutive rows of channel f from a sliding window of 7 staged rows
+            const float4 wc = wsm[f];
+            const float b0 = bsm[f];
+            float xw[7];
+#pragma unroll
+            for (int i = 0; i < 7; ++i) xw[i] = to_f(xs[(size_t)(r4 + i) * ld + f]);
             float y[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) y[u] = r4 + u < n ? tc::round_tf32(conv(f, r4 + u)) : 0.f;
+            for (int u = 0; u < 4; ++u) {
+                float acc = fmaf(wc.x, xw[u], b0);
+                acc = fmaf(wc.y, xw[u + 1], acc);
+                acc = fmaf(wc.z, xw[u + 2], acc);
+                acc = fmaf(wc.w, xw[u + 3], acc);
+                y[u] = r4 + u < n ? tc::round_tf32(silu(acc)) : 0.f;
+            }
             *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(f, r4, DV)) =
                 make_float4(y[0], y[1], y[2], y[3]);
         }

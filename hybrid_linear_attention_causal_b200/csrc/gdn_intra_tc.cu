@@ -248,36 +248,14 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 }
             }
         }
-        // what needs only the gates and goes to the workspace: the state pass's
-        // (diag(e^{gamma_n-gamma}) K)^T and the rows Qg = diag(e^gamma) Q of the [W ; Qg] tile; these
-        // stores drain while the exponentials above and the inverse below compute
-        for (int idx = tid; idx < DK * C / 4; idx += NT) {
-            int f, s4;
-            tile_coord<DK>(idx, f, s4);
-            const uint32_t off = tc::kmajor_off(f, s4, DK);
-            const float4 k = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) + off);
-            store_f4(reinterpret_cast<float*>(KTg), off,
-                     make_float4(tc::round_tf32(k.x * sm.fkt[s4]), tc::round_tf32(k.y * sm.fkt[s4 + 1]),
-                                 tc::round_tf32(k.z * sm.fkt[s4 + 2]), tc::round_tf32(k.w * sm.fkt[s4 + 3])));
-        }
-        for (int idx = tid; idx < C * DK / 4; idx += NT) {  // same tile offsets as the q rows of [K ; Q]
-            int r, k4;
-            tile_coord<C>(idx, r, k4);
-            const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
-            const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
-            const float e = sm.eg[r];
-            store_f4(reinterpret_cast<float*>(WQg), off,
-                     make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
-                                 tc::round_tf32(q.w * e)));
-        }
-        if (tid < C) p.gam[ch_h * C + tid] = sm.gam[tid];
         __syncthreads();
         // T = (I + A)^{-1}, by blocks.  Every final entry goes straight into the K-major tf32 tile of
         // T diag(beta) (the A operand of W and U); the fp32 copy tf holds what the next level reads.
         //   level 1: the four diagonal 16x16 blocks by forward substitution, one column per lane held
         //            in registers (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so
-        //            one FMA per row sits on the dependent chain); warps 4-7 meanwhile build
-        //            (diag(e^gamma) K)^T for W.
+        //            one FMA per row sits on the dependent chain); warps 4-15 meanwhile build
+        //            (diag(e^gamma) K)^T for W and write the tiles that need only the gates (the
+        //            state pass's (diag(e^{gamma_n-gamma}) K)^T, the rows Qg = diag(e^gamma) Q).
         //   level 2: within each 32x32 diagonal block, X = -D2 (A21 D1).
         //   level 3: T21 = -T22 (A21 T11) for the lower-left 32x32 block.
         auto put_t = [&](int r, int c, float v) {
@@ -313,7 +291,22 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 store_f4(sm.kte, off,
                          make_float4(tc::round_tf32(k.x * sm.eg[s4]), tc::round_tf32(k.y * sm.eg[s4 + 1]),
                                      tc::round_tf32(k.z * sm.eg[s4 + 2]), tc::round_tf32(k.w * sm.eg[s4 + 3])));
+                // the state pass's (diag(e^{gamma_n-gamma}) K)^T, same tile offsets
+                store_f4(reinterpret_cast<float*>(KTg), off,
+                         make_float4(tc::round_tf32(k.x * sm.fkt[s4]), tc::round_tf32(k.y * sm.fkt[s4 + 1]),
+                                     tc::round_tf32(k.z * sm.fkt[s4 + 2]), tc::round_tf32(k.w * sm.fkt[s4 + 3])));
             }
+            for (int idx = tid - 128; idx < C * DK / 4; idx += NW) {  // rows Qg = diag(e^gamma) Q of [W ; Qg]
+                int r, k4;
+                tile_coord<C>(idx, r, k4);
+                const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
+                const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
+                const float e = sm.eg[r];
+                store_f4(reinterpret_cast<float*>(WQg), off,
+                         make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
+                                     tc::round_tf32(q.w * e)));
+            }
+            if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[tid - 128];
         }
         __syncthreads();
         static_assert(NT == 512, "the level 2 and 3 thread maps below assume 512 threads");

@@ -374,20 +374,25 @@ def main():
                        ws_v)
 
     EXT_K = ["chunk_map", "prep", "conv_tail", "intra", "state"]
-    n_ev = len(EXT_K) + 1 + 2 + 2
+    # gdn_extend's profiling marks: 0 start, 1 chunk table, 2 prep, 3 conv tail, 4 intra of the
+    # longest sequences, 5 intra of the rest (first launch), 10 join, 6 state pass of the rest, 7 end;
+    # on the library's second stream 8 / 9 bracket the state pass of the longest sequences
+    # (alongside 4 -> 5) and 11 ends a second intra launch for the rest
+    EXT_EV = 12
+    n_ev = EXT_EV + 2 + 2
 
     def make_events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
 
     def step(ev=None):
         if ev is not None:
-            gdn.gdn_set_launch_events(ev[:len(EXT_K) + 1])
+            gdn.gdn_set_launch_events(ev[:EXT_EV])
         extend()
         if ev is not None:
-            gdn.gdn_set_launch_events(ev[len(EXT_K) + 1:len(EXT_K) + 3])
+            gdn.gdn_set_launch_events(ev[EXT_EV:EXT_EV + 2])
         decode()
         if ev is not None:
-            gdn.gdn_set_launch_events(ev[len(EXT_K) + 3:])
+            gdn.gdn_set_launch_events(ev[EXT_EV + 2:])
         verify()
         if ev is not None:
             gdn.gdn_set_launch_events([])
@@ -415,11 +420,16 @@ def main():
     def span(k, i, j):
         return evs[k][i].elapsed_time(evs[k][j])
 
-    nE = len(EXT_K)
-    kern_ms = {name: statistics.mean(span(k, i, i + 1) for k in range(args.steps)) for i, name in enumerate(EXT_K)}
-    kern_ms["decode"] = statistics.mean(span(k, nE + 1, nE + 2) for k in range(args.steps))
-    kern_ms["verify"] = statistics.mean(span(k, nE + 3, nE + 4) for k in range(args.steps))
-    ext_ms = max_over_ranks(statistics.mean(span(k, 0, nE) for k in range(args.steps)), world, dev)
+    def mean_span(*pairs):  # summed over the pairs, averaged over the steps
+        return statistics.mean(sum(span(k, i, j) for i, j in pairs) for k in range(args.steps))
+
+    # per-kernel device times; the two intra launches run back to back, the two state passes
+    # partly alongside the second intra launch
+    kern_ms = {"chunk_map": mean_span((0, 1)), "prep": mean_span((1, 2)), "conv_tail": mean_span((2, 3)),
+               "intra": mean_span((3, 4), (4, 5)), "state": mean_span((8, 9), (10, 6))}
+    kern_ms["decode"] = mean_span((EXT_EV, EXT_EV + 1))
+    kern_ms["verify"] = mean_span((EXT_EV + 2, EXT_EV + 3))
+    ext_ms = max_over_ranks(mean_span((0, 7)), world, dev)
     dec_ms = max_over_ranks(kern_ms["decode"], world, dev)
     ver_ms = max_over_ranks(kern_ms["verify"], world, dev)
 
@@ -536,7 +546,7 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
-            "gpu_launches": args.steps * (len(EXT_K) + 2),
+            "gpu_launches": args.steps * (8 + 2),  # extend: 8 kernels (intra 3x, state 2x); decode; verify
             "clocks": clocks,
             "decode": {"ms": dec_ms, "requests_per_s": world * Bn / (dec_ms * 1e-3),
                        "state_gbs": world * st_dec / (dec_ms * 1e-3) / 1e9,

@@ -18,6 +18,13 @@ constexpr int kMaxVerifyDraft = 16; // D limit of gdn_verify
 // header layout (int32 words)
 constexpr int kHdrError = 0;        // sticky GDN_DEVERR_* bits
 constexpr int kHdrNumChunks = 1;    // chunk count of the current extend batch
+constexpr int kHdrItemNext = 2;     // [2]: next intra work item of group 0, 1 (dynamic scheduling)
+constexpr int kHdrGroupSeqs = 4;    // sequences of group 0 (the longest; ranks 0 .. value-1)
+constexpr int kHdrGroupChunks = 5;  // [2]: chunks of group 0, 1 in chunk_list (live sequences only)
+
+// An extend batch is processed as two groups of sequences: group 0 holds the
+// longest ones (chunk count at least half the longest), group 1 the rest.  The
+// state pass of group 0 runs on a second stream while intra works on group 1.
 
 struct LayerDims {
     int HK, HV, dk, dv, G;  // G = HV / HK
@@ -92,6 +99,8 @@ struct ExtendArgs {
     int4* chunk_tab;    // [max_chunks] {seq, first row, length, chunk index within seq}
     int32_t* seq_chunk0;// [N+1] first chunk id of each sequence
     int32_t* seq_order; // [N] sequences by decreasing chunk count (the state pass's launch order)
+    int32_t* seq_rank;  // [N] inverse of seq_order
+    int32_t* chunk_list;// [max_chunks] chunk ids of group 0's live sequences, then group 1's
     // per chunk, written by the prep kernel (conv + SiLU + L2 norm + gates):
     float* KQ;          // [max_chunks, HK, 2*C*dk] [K ; Q*scale] tf32, K-major tile of 128 rows
     float* VT;          // [max_chunks, HV, dv*C]   V^T tf32, K-major tile of dv rows x C
@@ -119,14 +128,16 @@ struct ExtendArgs {
 // True when chunk_map rejected the batch (it then publishes zero chunks).
 __device__ __forceinline__ bool batch_rejected(const ExtendArgs& p) { return p.hdr[kHdrNumChunks] == 0; }
 
-// Intra-chunk step on tensor cores (gdn_intra_tc.cu): grid (max_chunks, HK).
+// Intra-chunk step on tensor cores (gdn_intra_tc.cu) for the chunks of one
+// sequence group: persistent CTAs taking (chunk, qk head) items dynamically;
+// with `reserve`, the CTAs leave group 0's state pass its SMs.
 template <int DK, int DV>
-cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s);
+cudaError_t launch_intra(const ExtendArgs& p, int group, bool reserve, cudaStream_t s);
 
-// Serial state pass + outputs on tensor cores (gdn_state_tc.cu): one CTA per
-// (sequence, value head), longest sequences first.
+// Serial state pass + outputs on tensor cores (gdn_state_tc.cu) for one
+// sequence group: one CTA per (sequence, value head), longest sequences first.
 template <typename T, int DK, int DV>
-cudaError_t launch_state(const ExtendArgs& p, cudaStream_t s);
+cudaError_t launch_state(const ExtendArgs& p, int group, cudaStream_t s);
 
 // Records the calling thread's i-th profiling event on `s` if one is set
 // (see gdn_set_launch_events); a no-op otherwise.

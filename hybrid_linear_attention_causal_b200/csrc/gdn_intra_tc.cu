@@ -54,6 +54,7 @@ struct IntraTcSmem {
     float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
     unsigned long long bar_mma, bar_kq, bar_v, bar_g[2];
     uint32_t tmem_base;
+    int next_item;         // thread 0's latest grab, for the other threads
 };
 
 __device__ __forceinline__ void store_f4(float* tile, uint32_t off, float4 v) {
@@ -75,28 +76,40 @@ __device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
+__global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int group, int reserve) {
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int G = d.G, HV = d.HV, HK = d.HK;
-    // work items (chunk, qk head) in order; CTA b takes items b, b + gridDim.x, ... skipping padded requests
-    const int nitems = p.hdr[kHdrNumChunks] * HK;
-    auto next_item = [&](int it) {
-        for (; it < nitems; it += gridDim.x) {
-            const int sl = p.slots[p.chunk_tab[it / HK].x];
-            if (sl >= 0 && sl < p.P) break;
+    // This group's (chunk, qk head) items, handed out dynamically from one counter: CTAs that start
+    // late (while the other stream's state pass holds SMs) still find work.  An item is named by
+    // chunk * HK + hk; padded requests are skipped; -1 = none left.
+    const int base = group ? p.hdr[kHdrGroupChunks] : 0;
+    const int nlist = p.hdr[kHdrGroupChunks + group] * HK;
+    int* next_ctr = p.hdr + kHdrItemNext + group;
+    auto grab = [&]() -> int {
+        while (true) {
+            const int li = atomicAdd(next_ctr, 1);
+            if (li >= nlist) return -1;
+            const int cid = p.chunk_list[base + li / HK];
+            const int sl = p.slots[p.chunk_tab[cid].x];
+            if (sl >= 0 && sl < p.P) return cid * HK + li % HK;
         }
-        return it;
     };
-    int item = next_item(blockIdx.x);
-    if (item >= nitems) return;
+    // group 1's first launch runs while the state pass of group 0 (one CTA per SM, kA x HV of them)
+    // runs on the other stream: it leaves that pass those SMs.  A second launch for group 1 on the
+    // other stream, after that pass, takes the remaining items from the same counter.
+    if (reserve && (int)blockIdx.x >= (int)gridDim.x - min(p.hdr[kHdrGroupSeqs] * HV, (int)gridDim.x / 2)) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     IntraTcSmem<DK, DV>& sm = *reinterpret_cast<IntraTcSmem<DK, DV>*>(smem_raw);
+    if (tid == 0) sm.next_item = grab();
+    __syncthreads();
+    int item = sm.next_item;
+    if (item < 0) return;
     const uint32_t bar = tc::smem_u32(&sm.bar_mma), bar_kq = tc::smem_u32(&sm.bar_kq);
     constexpr uint32_t KQ_BYTES = 2 * C * DK * 4, VT_BYTES = DV * C * 4, GB_BYTES = C * 8;
     const uint32_t bar_v = tc::smem_u32(&sm.bar_v);
-    auto kq_src = [&](int it) { return p.KQ + (size_t)it * (2 * C * DK); };  // item = chunk * HK + hk
+    auto kq_src = [&](int it) { return p.KQ + (size_t)it * (2 * C * DK); };  // [K ; Q] tiles are [chunk][hk]
     auto head_row = [&](int it, int jj) { return (size_t)(it / HK) * HV + (it % HK) * G + jj; };
     auto fetch_kq = [&](int it) {
         tc::mbar_expect_tx(bar_kq, KQ_BYTES);
@@ -150,11 +163,15 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
     // completed uses of each barrier so far, identical in every thread (parity = count & 1)
     uint32_t n_kq = 0, n_v = 0, n_g[2] = {0u, 0u}, ph_mma = 0;
     bool ok = true;
-    while (ok && item < nitems) {
-    const int nxt = next_item(item + gridDim.x);
+    while (ok && item >= 0) {
+    int nxt = -1;
+    if (tid == 0) {
+        nxt = grab();
+        sm.next_item = nxt;  // read by every thread after the K^T barrier below
+    }
     const int id = item / HK, hk = item % HK;
     const int n = p.chunk_tab[id].z;
-    if (tid == 0 && nxt < nitems) prefetch_l2(nxt);
+    if (tid == 0 && nxt >= 0) prefetch_l2(nxt);
     if (tid == 0) {
         ok = tc::mbar_wait(bar_kq, n_kq & 1u);
         if (ok) {  // D1 = [K ; Q] K^T
@@ -177,6 +194,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
                 load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
         }
     ok = __syncthreads_and(ok);
+    nxt = sm.next_item;
 
     for (int j = 0; j < G && ok; ++j) {
         const int h = hk * G + j, b = j & 1;
@@ -379,7 +397,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
         if (tid == 0) {  // the V^T tile and gate buffer b are free again; after the last head, so is [K ; Q]
             if (j + 1 < G) fetch_v(item, j + 1);
             if (j + 2 < G) fetch_g(item, j + 2);
-            if (j == G - 1 && nxt < nitems) {  // the next item's tiles land during this epilogue
+            if (j == G - 1 && nxt >= 0) {  // the next item's tiles land during this epilogue
                 fetch_kq(nxt);
                 fetch_g(nxt, 0);
                 if (G > 1) fetch_g(nxt, 1);
@@ -440,7 +458,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p) {
 }  // namespace
 
 template <int DK, int DV>
-cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s) {
+cudaError_t launch_intra(const ExtendArgs& p, int group, bool reserve, cudaStream_t s) {
     const size_t shm = sizeof(IntraTcSmem<DK, DV>);
     cudaError_t e = cudaFuncSetAttribute(intra_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
@@ -450,13 +468,13 @@ cudaError_t launch_intra(const ExtendArgs& p, cudaStream_t s) {
     // persistent: one CTA per SM walks the (chunk, qk head) items
     const long long items = (long long)p.max_chunks * p.d.HK;
     const int grid = (int)(items < sms ? items : sms);
-    intra_tc_kernel<DK, DV><<<grid, NT, shm, s>>>(p);
+    intra_tc_kernel<DK, DV><<<grid, NT, shm, s>>>(p, group, reserve ? 1 : 0);
     return cudaGetLastError();
 }
 
-template cudaError_t launch_intra<64, 64>(const ExtendArgs&, cudaStream_t);
-template cudaError_t launch_intra<64, 128>(const ExtendArgs&, cudaStream_t);
-template cudaError_t launch_intra<128, 64>(const ExtendArgs&, cudaStream_t);
-template cudaError_t launch_intra<128, 128>(const ExtendArgs&, cudaStream_t);
+template cudaError_t launch_intra<64, 64>(const ExtendArgs&, int, bool, cudaStream_t);
+template cudaError_t launch_intra<64, 128>(const ExtendArgs&, int, bool, cudaStream_t);
+template cudaError_t launch_intra<128, 64>(const ExtendArgs&, int, bool, cudaStream_t);
+template cudaError_t launch_intra<128, 128>(const ExtendArgs&, int, bool, cudaStream_t);
 
 }  // namespace gdn

@@ -37,6 +37,8 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     __shared__ int s_bad;
     __shared__ int s_scan[1024];
     __shared__ int s_base;
+    __shared__ int s_rank[1024], s_off[1024];  // (N <= 1024) rank of each sequence, chunk offset by rank
+    __shared__ int s_maxc, s_kA;
     const int tid = threadIdx.x;
     if (tid == 0) {
         s_bad = (p.cu[0] != 0 || p.cu[p.N] != p.T) ? 1 : 0;
@@ -78,22 +80,60 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     __syncthreads();
     const int total = s_base;
     // Longest sequences first: the state pass runs each sequence's chunks in series, so its grid
-    // starts the long chains before the short ones.  (Rank by chunk count, ties by index; more
-    // than 1024 sequences keep their order.)
-    if (p.N <= 1024) {
-        if (tid < p.N) s_scan[tid] = p.seq_chunk0[tid + 1] - p.seq_chunk0[tid];
+    // starts the long chains before the short ones (rank by chunk count, ties by index).  Group 0
+    // is the sequences with at least half the longest one's chunks, ranks 0 .. kA-1; chunk_list
+    // holds the chunk ids by rank, so each group's chunks are one contiguous run.  More than 1024
+    // sequences keep their order and form group 0 alone.
+    const bool small = p.N <= 1024;
+    if (small) {
+        const int nc_t = tid < p.N ? p.seq_chunk0[tid + 1] - p.seq_chunk0[tid] : 0;
+        if (tid == 0) {
+            s_maxc = 0;
+            s_kA = 0;
+        }
         __syncthreads();
         if (tid < p.N) {
-            const int mine = s_scan[tid];
+            s_scan[tid] = nc_t;
+            atomicMax(&s_maxc, nc_t);
+        }
+        __syncthreads();
+        if (tid < p.N) {
             int rank = 0;
             for (int j = 0; j < p.N; ++j) {
                 const int o = s_scan[j];
-                rank += (o > mine || (o == mine && j < tid)) ? 1 : 0;
+                rank += (o > nc_t || (o == nc_t && j < tid)) ? 1 : 0;
             }
             p.seq_order[rank] = tid;
+            p.seq_rank[tid] = rank;
+            s_rank[tid] = rank;
+            s_off[rank] = nc_t;
+            if (nc_t > 0 && 2 * nc_t >= s_maxc) atomicAdd(&s_kA, 1);
         }
+        __syncthreads();
+        // exclusive scan of the chunk counts in rank order
+        const int own = tid < p.N ? s_off[tid] : 0;
+        for (int off = 1; off < 1024; off <<= 1) {
+            const int v = tid >= off ? s_off[tid - off] : 0;
+            __syncthreads();
+            if (tid < p.N) s_off[tid] += v;
+            __syncthreads();
+        }
+        if (tid < p.N) s_off[tid] -= own;
+        __syncthreads();
     } else {
-        for (int i = tid; i < p.N; i += 1024) p.seq_order[i] = i;
+        for (int i = tid; i < p.N; i += 1024) {
+            p.seq_order[i] = i;
+            p.seq_rank[i] = i;
+        }
+    }
+    if (tid == 0) {
+        const int kA = small ? s_kA : p.N;
+        const int cA = small ? (kA < p.N ? s_off[kA] : total) : total;
+        p.hdr[kHdrGroupSeqs] = kA;
+        p.hdr[kHdrGroupChunks] = cA;
+        p.hdr[kHdrGroupChunks + 1] = total - cA;
+        p.hdr[kHdrItemNext] = 0;
+        p.hdr[kHdrItemNext + 1] = 0;
     }
     for (int id = tid; id < total; id += 1024) {
         int lo = 0, hi = p.N - 1;  // last sequence whose first chunk id <= id
@@ -104,6 +144,7 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
         const int c = id - p.seq_chunk0[lo];
         const int len = p.cu[lo + 1] - p.cu[lo];
         p.chunk_tab[id] = make_int4(lo, p.cu[lo] + c * C, min(C, len - c * C), c);
+        p.chunk_list[small ? s_off[s_rank[lo]] + c : id] = id;
     }
 }
 
@@ -317,6 +358,42 @@ __global__ void __launch_bounds__(256) conv_tail_kernel(ExtendArgs p) {
 // ---------------------------------------------------------------- 4. intra
 // on tensor cores, in gdn_intra_tc.cu
 
+// A second stream (at the device's greatest priority) with a fork and a join
+// event, per host thread and device, created by the first extend call there
+// and kept until the process exits.  Inside a stream capture the fork / join
+// pair makes it part of the captured graph.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+constexpr int kMaxSideDevices = 64;
+
+cudaError_t side_stream(SideStream** out) {
+    thread_local SideStream per_device[kMaxSideDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+    SideStream& ss = per_device[dev];
+    if (!ss.s) {
+        SideStream n;
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) == cudaSuccess &&
+            (e = cudaStreamCreateWithPriority(&n.s, cudaStreamNonBlocking, greatest)) == cudaSuccess &&
+            (e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) == cudaSuccess &&
+            (e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming)) == cudaSuccess) {
+            ss = n;
+        } else {  // nothing half-made is kept
+            if (n.fork) cudaEventDestroy(n.fork);
+            if (n.s) cudaStreamDestroy(n.s);
+            return e;
+        }
+    }
+    *out = &ss;
+    return cudaSuccess;
+}
+
 // ---------------------------------------------------------------- 5. state pass
 // on tensor cores, in gdn_state_tc.cu
 
@@ -339,10 +416,29 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 3);
-    if ((e = launch_intra<DK, DV>(p, s)) != cudaSuccess) return e;
+    // group 0 (the longest sequences): intra; then, on the side stream, its state pass and after it
+    // a second intra launch for group 1, while on `s` intra of group 1 runs on the SMs that the
+    // state pass leaves (both intra launches take items from one counter); then the state pass of
+    // group 1
+    SideStream* side = nullptr;
+    if ((e = side_stream(&side)) != cudaSuccess) return e;
+    if ((e = launch_intra<DK, DV>(p, 0, false, s)) != cudaSuccess) return e;
     mark_launch(s, 4);
-    if ((e = launch_state<T, DK, DV>(p, s)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(side->fork, s)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
+    mark_launch(side->s, 8);
+    if ((e = launch_state<T, DK, DV>(p, 0, side->s)) != cudaSuccess) return e;
+    mark_launch(side->s, 9);
+    if ((e = launch_intra<DK, DV>(p, 1, false, side->s)) != cudaSuccess) return e;
+    mark_launch(side->s, 11);
+    if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
+    if ((e = launch_intra<DK, DV>(p, 1, true, s)) != cudaSuccess) return e;
     mark_launch(s, 5);
+    if ((e = cudaStreamWaitEvent(s, side->join, 0)) != cudaSuccess) return e;
+    mark_launch(s, 10);
+    if ((e = launch_state<T, DK, DV>(p, 1, s)) != cudaSuccess) return e;
+    mark_launch(s, 6);
+    mark_launch(s, 7);
     return cudaSuccess;
 }
 
@@ -357,6 +453,8 @@ size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max
     off += al(mc * sizeof(int4));
     off += al(((size_t)max_N + 1) * sizeof(int32_t));
     off += al((size_t)max_N * sizeof(int32_t));
+    off += al((size_t)max_N * sizeof(int32_t));
+    off += al(mc * sizeof(int32_t));
     off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
     off += al(per * d.dv * C);
     off += al(per * C * 2);
@@ -381,6 +479,8 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
     e.chunk_tab = reinterpret_cast<int4*>(base + off); off += al((size_t)mc * sizeof(int4));
     e.seq_chunk0 = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
     e.seq_order = reinterpret_cast<int32_t*>(base + off); off += al((size_t)max_N * sizeof(int32_t));
+    e.seq_rank = reinterpret_cast<int32_t*>(base + off); off += al((size_t)max_N * sizeof(int32_t));
+    e.chunk_list = reinterpret_cast<int32_t*>(base + off); off += al((size_t)mc * sizeof(int32_t));
     e.KQ = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
     e.VT = reinterpret_cast<float*>(base + off); off += al(per * d.dv * C);
     e.GB = reinterpret_cast<float2*>(base + off); off += al(per * C * 2);

@@ -76,12 +76,15 @@ __device__ __forceinline__ void put_st16(float* st, int j, int c0, const float* 
 }
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
+__global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int group) {
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int HV = d.HV;
-    // all heads of the longest sequence first, then the next longest, ...
-    const int h = blockIdx.x % HV, nseq = p.seq_order[blockIdx.x / HV];
+    // all heads of the longest sequence first, then the next longest, ...; group 0 is ranks
+    // 0 .. kA-1, group 1 the rest
+    const int rank = blockIdx.x / HV, kA = p.hdr[kHdrGroupSeqs];
+    if (group == 0 ? rank >= kA : rank < kA) return;
+    const int h = blockIdx.x % HV, nseq = p.seq_order[rank];
     const int len = p.cu[nseq + 1] - p.cu[nseq];
     if (len == 0) return;
     const int slot = p.slots[nseq];
@@ -207,7 +210,13 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
                     tc::mma_tf32(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
                 tc::mma_commit(bar_x);
             }
-            if (okl && id + 1 < c_end) tc::bulk_prefetch_l2(u_src(id + 1), DV * C * 4);
+            if (okl && id + 1 < c_end) {  // the next chunk's tiles into L2, so their copies wait on L2 only
+                const size_t nx = (size_t)(id + 1) * HV + h;
+                tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
+                tc::bulk_prefetch_l2(p.KT + nx * (DK * C), KT_BYTES);
+                tc::bulk_prefetch_l2(p.AQ + nx * (C * C), AQ_BYTES);
+                tc::bulk_prefetch_l2(u_src(id + 1), DV * C * 4);
+            }
             if (okl) {
                 okl = tc::mbar_wait(bar_x, ph);
                 if (okl && id + 1 < c_end) fetch_wq(id + 1);  // the [W ; Qg] tile is free again
@@ -341,20 +350,20 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p) {
 }  // namespace
 
 template <typename T, int DK, int DV>
-cudaError_t launch_state(const ExtendArgs& p, cudaStream_t s) {
+cudaError_t launch_state(const ExtendArgs& p, int group, cudaStream_t s) {
     const size_t shm = sizeof(StateTcSmem<T, DK, DV>);
     cudaError_t e =
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
-    state_tc_kernel<T, DK, DV><<<(unsigned)p.N * (unsigned)p.d.HV, NT, shm, s>>>(p);
+    state_tc_kernel<T, DK, DV><<<(unsigned)p.N * (unsigned)p.d.HV, NT, shm, s>>>(p, group);
     return cudaGetLastError();
 }
 
 #define GDN_STATE_INST(T)                                                        \
-    template cudaError_t launch_state<T, 64, 64>(const ExtendArgs&, cudaStream_t);   \
-    template cudaError_t launch_state<T, 64, 128>(const ExtendArgs&, cudaStream_t);  \
-    template cudaError_t launch_state<T, 128, 64>(const ExtendArgs&, cudaStream_t);  \
-    template cudaError_t launch_state<T, 128, 128>(const ExtendArgs&, cudaStream_t);
+    template cudaError_t launch_state<T, 64, 64>(const ExtendArgs&, int, cudaStream_t);   \
+    template cudaError_t launch_state<T, 64, 128>(const ExtendArgs&, int, cudaStream_t);  \
+    template cudaError_t launch_state<T, 128, 64>(const ExtendArgs&, int, cudaStream_t);  \
+    template cudaError_t launch_state<T, 128, 128>(const ExtendArgs&, int, cudaStream_t);
 GDN_STATE_INST(float)
 GDN_STATE_INST(__nv_bfloat16)
 

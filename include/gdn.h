@@ -133,6 +133,14 @@ GDN_API size_t gdn_extend_workspace_size(const gdn_config_t* cfg, int32_t max_N,
  * nothing launched.  The final state of each sequence is written to its slot,
  * and the conv slot receives the K-1 most recent raw rows of (old conv state |
  * the sequence's rows).
+ *
+ * All work is ordered after earlier work on `stream` and complete before
+ * later work on it.  Internally the call also uses a second stream of the
+ * library (one per host thread and device, at the device's greatest stream
+ * priority) that forks from and joins back into `stream`, so it is captured
+ * along with `stream` into a CUDA graph; the first call on a device from a
+ * host thread creates that stream and its two events, so make it before any
+ * capture.
  */
 GDN_API int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
                const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
@@ -221,13 +229,18 @@ GDN_API int gdn_reset_device_error(void* workspace, gdn_stream_t stream);
 /*
  * Profiling aid (off by default).  With n > 0, the calling thread's later
  * gdn_extend / gdn_decode / gdn_verify calls record events[i] (each a
- * cudaEvent_t created by the caller) on their stream just before their i-th
- * kernel launch, and events[L] right after the last one, L being the number
- * of kernels the call launches (5 for extend, 1 for decode and verify);
- * indices >= n are not recorded.  n == 0 turns recording off.  The events
- * bracket each kernel, so elapsed times between consecutive events are
- * per-kernel device times.  Returns GDN_ERR_INVALID_ARG for n < 0, n > 16 or
- * events == NULL with n > 0.
+ * cudaEvent_t created by the caller) at fixed points of the call; indices
+ * >= n are not recorded.  n == 0 turns recording off.
+ *   decode, verify: 0 before the kernel, 1 after it (on `stream`).
+ *   extend: on `stream`: 0 start, 1 after the chunk table, 2 after the
+ *     conv + norm + gate pass, 3 after the conv-state update, 4 after the
+ *     intra-chunk pass of the longest sequences, 5 after the intra-chunk
+ *     pass of the others, 10 after joining the second stream, 6 after the
+ *     state pass of the others, 7 end; on the library's second stream: 8
+ *     before and 9 after the state pass of the longest sequences (alongside
+ *     4 -> 5), 11 after a second intra-chunk launch for the others that
+ *     takes the items left when that state pass ends.
+ * Returns GDN_ERR_INVALID_ARG for n < 0, n > 16 or events == NULL with n > 0.
  */
 GDN_API int gdn_set_launch_events(void* const* events, int32_t n);
 

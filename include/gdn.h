@@ -168,8 +168,10 @@ GDN_API int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, cons
  *     nothing is launched (one sequence of up to 511 tokens for the
  *     16/32-head, dk = dv = 128 layer; 4543 for the 4/8-head, 64 layer).
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and keeps it; make
- *     that first call outside any stream capture.  A failure there returns
+ *     (cudaGetSymbolAddress, with that device current) and keeps it, and,
+ *     like gdn_extend, creates the library's second stream and its two
+ *     events for the calling host thread (no device memory); make that first
+ *     call outside any stream capture.  A failure there returns
  *     GDN_ERR_CUDA with the cause left in the CUDA runtime's last error.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents; each call clears the part that must start at zero

@@ -374,11 +374,10 @@ def main():
                        ws_v)
 
     EXT_K = ["chunk_map", "prep", "conv_tail", "intra", "state"]
-    # gdn_extend's profiling marks: 0 start, 1 chunk table, 2 prep, 3 conv tail, 4 intra of the
-    # longest sequences, 5 intra of the rest (first launch), 10 join, 6 state pass of the rest, 7 end;
-    # on the library's second stream 8 / 9 bracket the state pass of the longest sequences
-    # (alongside 4 -> 5) and 11 ends a second intra launch for the rest
-    EXT_EV = 12
+    # gdn_extend's profiling marks: 0 start, 1 chunk table, 2 prep, 3 conv tail, 4 after the last intra
+    # segment, 5 end; on the library's second stream 6 / 7 bracket the state-pass segments, which run
+    # alongside the intra segments after the first
+    EXT_EV = 8
     n_ev = EXT_EV + 2 + 2
 
     def make_events():
@@ -423,13 +422,13 @@ def main():
     def mean_span(*pairs):  # summed over the pairs, averaged over the steps
         return statistics.mean(sum(span(k, i, j) for i, j in pairs) for k in range(args.steps))
 
-    # per-kernel device times; the two intra launches run back to back, the two state passes
-    # partly alongside the second intra launch
+    # per-kernel device times: the spans of the intra segments (on the caller's stream) and of the
+    # state-pass segments (on the second stream) overlap
     kern_ms = {"chunk_map": mean_span((0, 1)), "prep": mean_span((1, 2)), "conv_tail": mean_span((2, 3)),
-               "intra": mean_span((3, 4), (4, 5)), "state": mean_span((8, 9), (10, 6))}
+               "intra": mean_span((3, 4)), "state": mean_span((6, 7))}
     kern_ms["decode"] = mean_span((EXT_EV, EXT_EV + 1))
     kern_ms["verify"] = mean_span((EXT_EV + 2, EXT_EV + 3))
-    ext_ms = max_over_ranks(mean_span((0, 7)), world, dev)
+    ext_ms = max_over_ranks(mean_span((0, 5)), world, dev)
     dec_ms = max_over_ranks(kern_ms["decode"], world, dev)
     ver_ms = max_over_ranks(kern_ms["verify"], world, dev)
 
@@ -546,7 +545,8 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
-            "gpu_launches": args.steps * (8 + 2),  # extend: 8 kernels (intra 3x, state 2x); decode; verify
+            # extend: chunk table, prep, conv tail + intra and state per segment; decode; verify
+            "gpu_launches": args.steps * (3 + 2 * min(16, max(1, pre.T // 16384)) + 2),
             "clocks": clocks,
             "decode": {"ms": dec_ms, "requests_per_s": world * Bn / (dec_ms * 1e-3),
                        "state_gbs": world * st_dec / (dec_ms * 1e-3) / 1e9,

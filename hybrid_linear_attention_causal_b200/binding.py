@@ -25,7 +25,7 @@ GDN_DEVERR_SEQLENS = 0x2
 GDN_DEVERR_TIMEOUT = 0x4
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
-HEADER_BYTES = 256
+HEADER_BYTES = 512
 MAX_VERIFY_DRAFT = 16
 
 _DTYPES = {torch.float32: GDN_DTYPE_F32, torch.bfloat16: GDN_DTYPE_BF16}

@@ -12,19 +12,29 @@ namespace gdn {
 
 constexpr int kChunk = 64;          // prefill chunk length C
 constexpr int kConvK = 4;           // conv width K
-constexpr int kHeaderBytes = 256;   // workspace header (error word + counters)
+constexpr int kHeaderBytes = 512;   // workspace header (error word + counters)
 constexpr int kMaxVerifyDraft = 16; // D limit of gdn_verify
 
 // header layout (int32 words)
 constexpr int kHdrError = 0;        // sticky GDN_DEVERR_* bits
 constexpr int kHdrNumChunks = 1;    // chunk count of the current extend batch
-constexpr int kHdrItemNext = 2;     // [2]: next intra work item of group 0, 1 (dynamic scheduling)
-constexpr int kHdrGroupSeqs = 4;    // sequences of group 0 (the longest; ranks 0 .. value-1)
-constexpr int kHdrGroupChunks = 5;  // [2]: chunks of group 0, 1 in chunk_list (live sequences only)
+constexpr int kMaxSegments = 16;    // segments of an extend batch (see below)
+constexpr int kHdrSegLen = 2;       // P: chunks per segment (the last may hold fewer)
+constexpr int kHdrSegOff = 3;       // [kMaxSegments]: first chunk_list entry of segment k
+constexpr int kHdrSegCnt = kHdrSegOff + kMaxSegments;    // [kMaxSegments]: chunks in segment k
+constexpr int kHdrSegSeqs = kHdrSegCnt + kMaxSegments;   // [kMaxSegments]: sequences with chunks in segment k
+constexpr int kHdrItemNext = kHdrSegSeqs + kMaxSegments; // [kMaxSegments]: next intra item of segment k
+constexpr int kHdrSegRank = kHdrItemNext + kMaxSegments; // [kMaxSegments]: first rank with chunks in segment k
+static_assert((kHdrSegRank + kMaxSegments) * 4 <= kHeaderBytes, "header too small");
 
-// An extend batch is processed as two groups of sequences: group 0 holds the
-// longest ones (chunk count at least half the longest), group 1 the rest.  The
-// state pass of group 0 runs on a second stream while intra works on group 1.
+// An extend batch is cut into S segments (S chosen by the host, at most
+// kMaxSegments): the chunks, listed longest sequence first, in S pieces of P
+// consecutive list entries.  The intra step runs segment by segment on the
+// caller's stream; the state pass of segment k runs on a second stream once
+// intra has finished segment k, taking each sequence's chunks inside the piece
+// and continuing from the state the previous piece left in its slot,
+// alongside intra of segment k+1.  A piece holds few sequences, so its state
+// pass needs few SMs; the shortest sequences come last.
 
 struct LayerDims {
     int HK, HV, dk, dv, G;  // G = HV / HK
@@ -99,8 +109,9 @@ struct ExtendArgs {
     int4* chunk_tab;    // [max_chunks] {seq, first row, length, chunk index within seq}
     int32_t* seq_chunk0;// [N+1] first chunk id of each sequence
     int32_t* seq_order; // [N] sequences by decreasing chunk count (the state pass's launch order)
-    int32_t* seq_rank;  // [N] inverse of seq_order
-    int32_t* chunk_list;// [max_chunks] chunk ids of group 0's live sequences, then group 1's
+    int32_t* rank_off;  // [N+1] chunk_list position of each rank's first chunk
+    int32_t* chunk_list;// [max_chunks] chunk ids, rank by rank (longest sequence first)
+    int nseg;           // S
     // per chunk, written by the prep kernel (conv + SiLU + L2 norm + gates):
     float* KQ;          // [max_chunks, HK, 2*C*dk] [K ; Q*scale] tf32, K-major tile of 128 rows
     float* VT;          // [max_chunks, HV, dv*C]   V^T tf32, K-major tile of dv rows x C
@@ -129,15 +140,15 @@ struct ExtendArgs {
 __device__ __forceinline__ bool batch_rejected(const ExtendArgs& p) { return p.hdr[kHdrNumChunks] == 0; }
 
 // Intra-chunk step on tensor cores (gdn_intra_tc.cu) for the chunks of one
-// sequence group: persistent CTAs taking (chunk, qk head) items dynamically;
-// with `reserve`, the CTAs leave group 0's state pass its SMs.
+// segment: persistent CTAs taking (chunk, qk head) items dynamically; for
+// segment k > 0 they leave one SM per CTA of segment k-1's state pass free.
 template <int DK, int DV>
-cudaError_t launch_intra(const ExtendArgs& p, int group, bool reserve, cudaStream_t s);
+cudaError_t launch_intra(const ExtendArgs& p, int seg, cudaStream_t s);
 
 // Serial state pass + outputs on tensor cores (gdn_state_tc.cu) for one
-// sequence group: one CTA per (sequence, value head), longest sequences first.
+// segment: one CTA per (sequence, value head), longest sequences first.
 template <typename T, int DK, int DV>
-cudaError_t launch_state(const ExtendArgs& p, int group, cudaStream_t s);
+cudaError_t launch_state(const ExtendArgs& p, int seg, cudaStream_t s);
 
 // Records the calling thread's i-th profiling event on `s` if one is set
 // (see gdn_set_launch_events); a no-op otherwise.

@@ -37,6 +37,7 @@ namespace {
 constexpr int C = kChunk;
 constexpr int NT = 512;        // 16 warps; warp w reads TMEM sub-partition w % 4
 constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
+constexpr int kItemsPerCta = 4;
 
 template <int DK, int DV>
 struct IntraTcSmem {
@@ -76,16 +77,16 @@ __device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
 }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int group, int reserve) {
+__global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) {
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int G = d.G, HV = d.HV, HK = d.HK;
-    // This group's (chunk, qk head) items, handed out dynamically from one counter: CTAs that start
+    // This segment's (chunk, qk head) items, handed out dynamically from one counter: CTAs that start
     // late (while the other stream's state pass holds SMs) still find work.  An item is named by
     // chunk * HK + hk; padded requests are skipped; -1 = none left.
-    const int base = group ? p.hdr[kHdrGroupChunks] : 0;
-    const int nlist = p.hdr[kHdrGroupChunks + group] * HK;
-    int* next_ctr = p.hdr + kHdrItemNext + group;
+    const int base = p.hdr[kHdrSegOff + seg];
+    const int nlist = p.hdr[kHdrSegCnt + seg] * HK;
+    int* next_ctr = p.hdr + kHdrItemNext + seg;
     auto grab = [&]() -> int {
         while (true) {
             const int li = atomicAdd(next_ctr, 1);
@@ -95,10 +96,6 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int group
             if (sl >= 0 && sl < p.P) return cid * HK + li % HK;
         }
     };
-    // group 1's first launch runs while the state pass of group 0 (one CTA per SM, kA x HV of them)
-    // runs on the other stream: it leaves that pass those SMs.  A second launch for group 1 on the
-    // other stream, after that pass, takes the remaining items from the same counter.
-    if (reserve && (int)blockIdx.x >= (int)gridDim.x - min(p.hdr[kHdrGroupSeqs] * HV, (int)gridDim.x / 2)) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     IntraTcSmem<DK, DV>& sm = *reinterpret_cast<IntraTcSmem<DK, DV>*>(smem_raw);
@@ -163,12 +160,13 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int group
     // completed uses of each barrier so far, identical in every thread (parity = count & 1)
     uint32_t n_kq = 0, n_v = 0, n_g[2] = {0u, 0u}, ph_mma = 0;
     bool ok = true;
+    int done = 0;
     while (ok && item >= 0) {
     int nxt = -1;
-    if (tid == 0) {
-        nxt = grab();
-        sm.next_item = nxt;  // read by every thread after the K^T barrier below
-    }
+    // At most kItemsPerCta items, then the CTA ends: its SM goes to whatever waits, first of all a
+    // state-pass CTA of the previous segment (its stream has the higher priority).
+    if (tid == 0 && ++done < kItemsPerCta) nxt = grab();
+    if (tid == 0) sm.next_item = nxt;  // read by every thread after the K^T barrier below
     const int id = item / HK, hk = item % HK;
     const int n = p.chunk_tab[id].z;
     if (tid == 0 && nxt >= 0) prefetch_l2(nxt);
@@ -458,23 +456,24 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int group
 }  // namespace
 
 template <int DK, int DV>
-cudaError_t launch_intra(const ExtendArgs& p, int group, bool reserve, cudaStream_t s) {
+cudaError_t launch_intra(const ExtendArgs& p, int seg, cudaStream_t s) {
     const size_t shm = sizeof(IntraTcSmem<DK, DV>);
     cudaError_t e = cudaFuncSetAttribute(intra_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    // persistent: one CTA per SM walks the (chunk, qk head) items
-    const long long items = (long long)p.max_chunks * p.d.HK;
-    const int grid = (int)(items < sms ? items : sms);
-    intra_tc_kernel<DK, DV><<<grid, NT, shm, s>>>(p, group, reserve ? 1 : 0);
+    // CTAs of up to kItemsPerCta (chunk, qk head) items each, enough for the most a segment can hold
+    (void)sms;
+    const long long items = ((long long)p.max_chunks + p.nseg - 1) / p.nseg * p.d.HK;
+    const int grid = (int)((items + kItemsPerCta - 1) / kItemsPerCta);
+    intra_tc_kernel<DK, DV><<<grid, NT, shm, s>>>(p, seg);
     return cudaGetLastError();
 }
 
-template cudaError_t launch_intra<64, 64>(const ExtendArgs&, int, bool, cudaStream_t);
-template cudaError_t launch_intra<64, 128>(const ExtendArgs&, int, bool, cudaStream_t);
-template cudaError_t launch_intra<128, 64>(const ExtendArgs&, int, bool, cudaStream_t);
-template cudaError_t launch_intra<128, 128>(const ExtendArgs&, int, bool, cudaStream_t);
+template cudaError_t launch_intra<64, 64>(const ExtendArgs&, int, cudaStream_t);
+template cudaError_t launch_intra<64, 128>(const ExtendArgs&, int, cudaStream_t);
+template cudaError_t launch_intra<128, 64>(const ExtendArgs&, int, cudaStream_t);
+template cudaError_t launch_intra<128, 128>(const ExtendArgs&, int, cudaStream_t);
 
 }  // namespace gdn

@@ -37,8 +37,7 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     __shared__ int s_bad;
     __shared__ int s_scan[1024];
     __shared__ int s_base;
-    __shared__ int s_rank[1024], s_off[1024];  // (N <= 1024) rank of each sequence, chunk offset by rank
-    __shared__ int s_maxc, s_kA;
+    __shared__ int s_rank[1024], s_off[1024];  // (N <= 1024) rank of each sequence; list offset by rank
     const int tid = threadIdx.x;
     if (tid == 0) {
         s_bad = (p.cu[0] != 0 || p.cu[p.N] != p.T) ? 1 : 0;
@@ -79,23 +78,13 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     __threadfence_block();
     __syncthreads();
     const int total = s_base;
-    // Longest sequences first: the state pass runs each sequence's chunks in series, so its grid
-    // starts the long chains before the short ones (rank by chunk count, ties by index).  Group 0
-    // is the sequences with at least half the longest one's chunks, ranks 0 .. kA-1; chunk_list
-    // holds the chunk ids by rank, so each group's chunks are one contiguous run.  More than 1024
-    // sequences keep their order and form group 0 alone.
+    // Longest sequences first (rank by chunk count, ties by index; more than 1024 sequences keep
+    // their order).  This is the state pass's launch order and the order of chunk_list, which holds
+    // the chunks rank by rank; rank_off[r] is the list position of rank r's first chunk.
     const bool small = p.N <= 1024;
     if (small) {
         const int nc_t = tid < p.N ? p.seq_chunk0[tid + 1] - p.seq_chunk0[tid] : 0;
-        if (tid == 0) {
-            s_maxc = 0;
-            s_kA = 0;
-        }
-        __syncthreads();
-        if (tid < p.N) {
-            s_scan[tid] = nc_t;
-            atomicMax(&s_maxc, nc_t);
-        }
+        if (tid < p.N) s_scan[tid] = nc_t;
         __syncthreads();
         if (tid < p.N) {
             int rank = 0;
@@ -104,10 +93,8 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
                 rank += (o > nc_t || (o == nc_t && j < tid)) ? 1 : 0;
             }
             p.seq_order[rank] = tid;
-            p.seq_rank[tid] = rank;
             s_rank[tid] = rank;
             s_off[rank] = nc_t;
-            if (nc_t > 0 && 2 * nc_t >= s_maxc) atomicAdd(&s_kA, 1);
         }
         __syncthreads();
         // exclusive scan of the chunk counts in rank order
@@ -118,23 +105,46 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
             if (tid < p.N) s_off[tid] += v;
             __syncthreads();
         }
-        if (tid < p.N) s_off[tid] -= own;
-        __syncthreads();
+        if (tid < p.N) {
+            s_off[tid] -= own;
+            p.rank_off[tid] = s_off[tid];
+        }
     } else {
         for (int i = tid; i < p.N; i += 1024) {
             p.seq_order[i] = i;
-            p.seq_rank[i] = i;
+            p.rank_off[i] = p.seq_chunk0[i];
         }
     }
-    if (tid == 0) {
-        const int kA = small ? s_kA : p.N;
-        const int cA = small ? (kA < p.N ? s_off[kA] : total) : total;
-        p.hdr[kHdrGroupSeqs] = kA;
-        p.hdr[kHdrGroupChunks] = cA;
-        p.hdr[kHdrGroupChunks + 1] = total - cA;
-        p.hdr[kHdrItemNext] = 0;
-        p.hdr[kHdrItemNext + 1] = 0;
+    if (tid == 0) p.rank_off[p.N] = total;
+    __threadfence_block();
+    __syncthreads();
+    // Segments: the list cut into nseg pieces of P chunks.  The state pass of segment k takes, for
+    // each sequence, its chunks inside piece k, continuing from the state the previous piece left.
+    const int P = max(1, (total + p.nseg - 1) / p.nseg);
+    if (tid < kMaxSegments) {
+        const int k = tid, lo = min(k * P, total), hi = min(lo + P, total);
+        p.hdr[kHdrSegOff + k] = lo;
+        p.hdr[kHdrSegCnt + k] = hi - lo;
+        p.hdr[kHdrItemNext + k] = 0;
+        int first = p.N, last = p.N - 1;
+        if (lo < hi) {  // ranks holding list positions lo and hi - 1
+            int a = 0, b = p.N - 1;
+            while (a < b) {
+                const int m = (a + b + 1) >> 1;
+                if (p.rank_off[m] <= lo) a = m; else b = m - 1;
+            }
+            first = a;
+            b = p.N - 1;
+            while (a < b) {
+                const int m = (a + b + 1) >> 1;
+                if (p.rank_off[m] <= hi - 1) a = m; else b = m - 1;
+            }
+            last = a;
+        }
+        p.hdr[kHdrSegRank + k] = first;
+        p.hdr[kHdrSegSeqs + k] = last - first + 1;
     }
+    if (tid == 0) p.hdr[kHdrSegLen] = P;
     for (int id = tid; id < total; id += 1024) {
         int lo = 0, hi = p.N - 1;  // last sequence whose first chunk id <= id
         while (lo < hi) {
@@ -144,7 +154,7 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
         const int c = id - p.seq_chunk0[lo];
         const int len = p.cu[lo + 1] - p.cu[lo];
         p.chunk_tab[id] = make_int4(lo, p.cu[lo] + c * C, min(C, len - c * C), c);
-        p.chunk_list[small ? s_off[s_rank[lo]] + c : id] = id;
+        p.chunk_list[(small ? s_off[s_rank[lo]] : p.seq_chunk0[lo]) + c] = id;
     }
 }
 
@@ -358,13 +368,14 @@ __global__ void __launch_bounds__(256) conv_tail_kernel(ExtendArgs p) {
 // ---------------------------------------------------------------- 4. intra
 // on tensor cores, in gdn_intra_tc.cu
 
-// A second stream (at the device's greatest priority) with a fork and a join
-// event, per host thread and device, created by the first extend call there
-// and kept until the process exits.  Inside a stream capture the fork / join
-// pair makes it part of the captured graph.
+// A second stream (at the device's greatest priority) with one fork event per
+// segment and a join event, per host thread and device, created by the first
+// extend call there and kept until the process exits.  Inside a stream
+// capture the fork / join events make it part of the captured graph.
 struct SideStream {
     cudaStream_t s = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t seg[kMaxSegments] = {};
+    cudaEvent_t join = nullptr;
 };
 
 constexpr int kMaxSideDevices = 64;
@@ -379,16 +390,18 @@ cudaError_t side_stream(SideStream** out) {
     if (!ss.s) {
         SideStream n;
         int least = 0, greatest = 0;
-        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) == cudaSuccess &&
-            (e = cudaStreamCreateWithPriority(&n.s, cudaStreamNonBlocking, greatest)) == cudaSuccess &&
-            (e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming)) == cudaSuccess &&
-            (e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming)) == cudaSuccess) {
-            ss = n;
-        } else {  // nothing half-made is kept
-            if (n.fork) cudaEventDestroy(n.fork);
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) == cudaSuccess)
+            e = cudaStreamCreateWithPriority(&n.s, cudaStreamNonBlocking, greatest);
+        for (int k = 0; k < kMaxSegments && e == cudaSuccess; ++k)
+            e = cudaEventCreateWithFlags(&n.seg[k], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) {  // nothing half-made is kept
+            for (int k = 0; k < kMaxSegments; ++k)
+                if (n.seg[k]) cudaEventDestroy(n.seg[k]);
             if (n.s) cudaStreamDestroy(n.s);
             return e;
         }
+        ss = n;
     }
     *out = &ss;
     return cudaSuccess;
@@ -416,29 +429,22 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 3);
-    // group 0 (the longest sequences): intra; then, on the side stream, its state pass and after it
-    // a second intra launch for group 1, while on `s` intra of group 1 runs on the SMs that the
-    // state pass leaves (both intra launches take items from one counter); then the state pass of
-    // group 1
+    // segment by segment: intra on `s`; the state pass of segment k on the side stream once intra
+    // has finished segment k, alongside intra of segment k+1
     SideStream* side = nullptr;
     if ((e = side_stream(&side)) != cudaSuccess) return e;
-    if ((e = launch_intra<DK, DV>(p, 0, false, s)) != cudaSuccess) return e;
+    for (int k = 0; k < p.nseg; ++k) {
+        if ((e = launch_intra<DK, DV>(p, k, s)) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(side->seg[k], s)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(side->s, side->seg[k], 0)) != cudaSuccess) return e;
+        if (k == 0) mark_launch(side->s, 6);
+        if ((e = launch_state<T, DK, DV>(p, k, side->s)) != cudaSuccess) return e;
+    }
     mark_launch(s, 4);
-    if ((e = cudaEventRecord(side->fork, s)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(side->s, side->fork, 0)) != cudaSuccess) return e;
-    mark_launch(side->s, 8);
-    if ((e = launch_state<T, DK, DV>(p, 0, side->s)) != cudaSuccess) return e;
-    mark_launch(side->s, 9);
-    if ((e = launch_intra<DK, DV>(p, 1, false, side->s)) != cudaSuccess) return e;
-    mark_launch(side->s, 11);
+    mark_launch(side->s, 7);
     if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
-    if ((e = launch_intra<DK, DV>(p, 1, true, s)) != cudaSuccess) return e;
-    mark_launch(s, 5);
     if ((e = cudaStreamWaitEvent(s, side->join, 0)) != cudaSuccess) return e;
-    mark_launch(s, 10);
-    if ((e = launch_state<T, DK, DV>(p, 1, s)) != cudaSuccess) return e;
-    mark_launch(s, 6);
-    mark_launch(s, 7);
+    mark_launch(s, 5);
     return cudaSuccess;
 }
 
@@ -453,7 +459,7 @@ size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max
     off += al(mc * sizeof(int4));
     off += al(((size_t)max_N + 1) * sizeof(int32_t));
     off += al((size_t)max_N * sizeof(int32_t));
-    off += al((size_t)max_N * sizeof(int32_t));
+    off += al(((size_t)max_N + 1) * sizeof(int32_t));
     off += al(mc * sizeof(int32_t));
     off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
     off += al(per * d.dv * C);
@@ -479,7 +485,7 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
     e.chunk_tab = reinterpret_cast<int4*>(base + off); off += al((size_t)mc * sizeof(int4));
     e.seq_chunk0 = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
     e.seq_order = reinterpret_cast<int32_t*>(base + off); off += al((size_t)max_N * sizeof(int32_t));
-    e.seq_rank = reinterpret_cast<int32_t*>(base + off); off += al((size_t)max_N * sizeof(int32_t));
+    e.rank_off = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
     e.chunk_list = reinterpret_cast<int32_t*>(base + off); off += al((size_t)mc * sizeof(int32_t));
     e.KQ = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
     e.VT = reinterpret_cast<float*>(base + off); off += al(per * d.dv * C);

@@ -76,24 +76,29 @@ __device__ __forceinline__ void put_st16(float* st, int j, int c0, const float* 
 }
 
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int group) {
+__global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) {
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int HV = d.HV;
-    // all heads of the longest sequence first, then the next longest, ...; group 0 is ranks
-    // 0 .. kA-1, group 1 the rest
-    const int rank = blockIdx.x / HV, kA = p.hdr[kHdrGroupSeqs];
-    if (group == 0 ? rank >= kA : rank < kA) return;
-    const int h = blockIdx.x % HV, nseq = p.seq_order[rank];
-    const int len = p.cu[nseq + 1] - p.cu[nseq];
-    if (len == 0) return;
+    // the ranks holding chunks of this segment's piece of the chunk list (all heads of the longer
+    // sequence first); each CTA takes its sequence's chunks inside the piece
+    const int r = p.hdr[kHdrSegRank + seg] + (int)(blockIdx.x / HV);
+    if (r >= p.N) return;
+    const int h = blockIdx.x % HV, nseq = p.seq_order[r];
+    const int lo = p.hdr[kHdrSegOff + seg], hi = lo + p.hdr[kHdrSegCnt + seg];
+    const int ro = p.rank_off[r];
+    const int a = max(lo, ro), b = min(hi, p.rank_off[r + 1]);
+    if (a >= b) return;
+    const int c_first = p.seq_chunk0[nseq];
+    const int c_begin = c_first + (a - ro), c_end = c_begin + (b - a);
     const int slot = p.slots[nseq];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     T* out = reinterpret_cast<T*>(p.out);
     if (slot < 0 || slot >= p.P) {
-        if (slot >= p.P && tid == 0 && h == 0) raise_error(p.hdr, GDN_DEVERR_SLOT_RANGE);
-        for (int e = tid; e < len * DV; e += NT)
-            out[((size_t)(p.cu[nseq] + e / DV) * HV + h) * DV + e % DV] = from_f<T>(0.f);
+        if (slot >= p.P && tid == 0 && h == 0 && a == ro) raise_error(p.hdr, GDN_DEVERR_SLOT_RANGE);
+        const int r0 = p.cu[nseq] + (c_begin - c_first) * C, r1 = min(p.cu[nseq + 1], r0 + (c_end - c_begin) * C);
+        for (int e = tid; e < (r1 - r0) * DV; e += NT)
+            out[((size_t)(r0 + e / DV) * HV + h) * DV + e % DV] = from_f<T>(0.f);
         return;
     }
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -103,7 +108,6 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int group
                    bar_kt = tc::smem_u32(&sm.bar_kt), bar_aq = tc::smem_u32(&sm.bar_aq),
                    bar_u = tc::smem_u32(&sm.bar_u);
     constexpr uint32_t WQ_BYTES = 2 * C * DK * 4, AQ_BYTES = C * C * 4, KT_BYTES = DK * C * 4;
-    const int c_begin = p.seq_chunk0[nseq], c_end = p.seq_chunk0[nseq + 1];
     auto fetch_wq = [&](int id) {
         tc::mbar_expect_tx(bar_wq, WQ_BYTES);
         tc::bulk_g2s(tc::smem_u32(sm.wq), p.WQ + ((size_t)id * HV + h) * (2 * C * DK), WQ_BYTES, bar_wq);
@@ -142,7 +146,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int group
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     const bool rowv = warp < NCW && (DV == 128 || lane < 16);
     const int j = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
-    const bool init = p.has_init ? p.has_init[nseq] != 0 : true;
+    // a range after the sequence's first chunk continues from the state the previous piece left
+    const bool init = a > ro || (p.has_init ? p.has_init[nseq] != 0 : true);
     float* Sg = p.ssm_state + ((size_t)slot * HV + h) * DK * DV;
     float s[DK / 2];
 #pragma unroll
@@ -350,12 +355,15 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int group
 }  // namespace
 
 template <typename T, int DK, int DV>
-cudaError_t launch_state(const ExtendArgs& p, int group, cudaStream_t s) {
+cudaError_t launch_state(const ExtendArgs& p, int seg, cudaStream_t s) {
     const size_t shm = sizeof(StateTcSmem<T, DK, DV>);
     cudaError_t e =
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
-    state_tc_kernel<T, DK, DV><<<(unsigned)p.N * (unsigned)p.d.HV, NT, shm, s>>>(p, group);
+    // a piece of P chunks touches at most P + 1 sequences
+    const long long piece = ((long long)p.max_chunks + p.nseg - 1) / p.nseg;
+    const long long seqs = piece + 1 < p.N ? piece + 1 : p.N;
+    state_tc_kernel<T, DK, DV><<<(unsigned)(seqs * p.d.HV), NT, shm, s>>>(p, seg);
     return cudaGetLastError();
 }
 

@@ -52,7 +52,7 @@
  *     Launch failures return GDN_ERR_CUDA; gdn_last_cuda_error() gives the
  *     CUDA error string of the most recent one on the calling thread.
  *   - Workspace: caller-allocated device memory of at least the size the
- *     matching *_workspace_size() returns.  Its first 256 bytes are a header
+ *     matching *_workspace_size() returns.  Its first 512 bytes are a header
  *     whose first int32 is a sticky device error word: kernels OR GDN_DEVERR_*
  *     bits into it and never clear it.  Zero it once after allocation with
  *     gdn_reset_device_error() (or cudaMemset) and read it with
@@ -236,12 +236,12 @@ GDN_API int gdn_reset_device_error(void* workspace, gdn_stream_t stream);
  *   decode, verify: 0 before the kernel, 1 after it (on `stream`).
  *   extend: on `stream`: 0 start, 1 after the chunk table, 2 after the
  *     conv + norm + gate pass, 3 after the conv-state update, 4 after the
- *     intra-chunk pass of the longest sequences, 5 after the intra-chunk
- *     pass of the others, 10 after joining the second stream, 6 after the
- *     state pass of the others, 7 end; on the library's second stream: 8
- *     before and 9 after the state pass of the longest sequences (alongside
- *     4 -> 5), 11 after a second intra-chunk launch for the others that
- *     takes the items left when that state pass ends.
+ *     last intra-chunk segment, 5 end (second stream joined); on the
+ *     library's second stream: 6 before the first and 7 after the last
+ *     state-pass segment.  The batch is processed in segments of chunks
+ *     (about one per 16384 packed rows, at most 16): the state pass of segment
+ *     k runs on the second stream alongside the intra-chunk pass of segment
+ *     k+1, so the two spans overlap.
  * Returns GDN_ERR_INVALID_ARG for n < 0, n > 16 or events == NULL with n > 0.
  */
 GDN_API int gdn_set_launch_events(void* const* events, int32_t n);

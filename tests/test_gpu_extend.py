@@ -136,6 +136,22 @@ def test_many_sequences(HK, HV, dk, dv, dtype):
     check_extend(w, gpu_extend(to_device(w)), oracle_extend(w))
 
 
+@pytest.mark.parametrize("lengths,slots,hi", [
+    # 33000 packed rows -> 2 segments: long, medium, short, single-row, empty and padded requests
+    ([16000, 12000, 4000, 1, 0, 999], [3, 0, 5, 1, 2, -1], [1, 0, 1, 1, 1, 1]),
+    # one sequence of 49152 rows -> 3 segments, each continuing from the previous one's state
+    ([49152], [2], [1]),
+])
+def test_segmented_batches(lengths, slots, hi):
+    """Batches of 32768 packed rows or more run as several segments (the state
+    pass of segment k alongside intra of segment k+1, each segment a piece of
+    the chunks listed longest sequence first); every sequence's chain must
+    continue across the segment boundaries."""
+    spec = W.LayerSpec(HK=2, HV=4, dk=128, dv=128, dtype=torch.bfloat16)
+    w = W.random_case(spec, lengths, P=6, seed=sum(lengths), has_init=hi, slots=slots, a_mean=-2.0)
+    check_extend(w, gpu_extend(to_device(w)), oracle_extend(w))
+
+
 def test_page_shapes_with_nonzero_prefix_state():
     """The ragged page-boundary, exact-page and checkpoint-boundary shapes of the
     SGLang GDN test matrix (prefix (0,8,16) / extend (15,8,1); extend (16,);

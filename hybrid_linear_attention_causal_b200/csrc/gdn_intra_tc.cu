@@ -194,17 +194,52 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     ok = __syncthreads_and(ok);
     nxt = sm.next_item;
 
-    for (int j = 0; j < G && ok; ++j) {
-        const int h = hk * G + j, b = j & 1;
-        const size_t ch_h = (size_t)id * HV + h;
-        char* WQg = reinterpret_cast<char*>(p.WQ + ch_h * (2 * C * DK));
-        char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
-        char* KTg = reinterpret_cast<char*>(p.KT + ch_h * (DK * C));
-        char* Ug = reinterpret_cast<char*>(p.U + ch_h * (DV * C));  // U^T, K-major tile: DV rows (j) x C
-        bool okv = tc::mbar_wait(tc::smem_u32(&sm.bar_g[b]), n_g[b] & 1u);
-        ++n_g[b];
-        if (okv && warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
-            const float2 g0 = sm.gb[b][2 * lane], g1 = sm.gb[b][2 * lane + 1];
+    // W and U^T of value head jj (accumulators in tensor memory) -> their workspace tiles
+    auto epilogue = [&](int jj) {
+        const size_t hrow = (size_t)id * HV + hk * G + jj;
+        char* WQg = reinterpret_cast<char*>(p.WQ + hrow * (2 * C * DK));
+        char* Ug = reinterpret_cast<char*>(p.U + hrow * (DV * C));  // U^T, K-major tile: DV rows (j) x C
+        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U -> U^T tile (fp32, K-major).
+           // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15;
+           // the warps of a sub-partition take one group of columns each
+            const bool valid = lane < 16;
+            const int r = sp * 16 + lane;
+#pragma unroll
+            for (int c0 = cg * (DK / NCG); c0 < (cg + 1) * (DK / NCG); c0 += 16) {
+                float v[16];
+                tc::tmem_ld16(tW + lane_base + c0, v);
+                tc::tmem_ld_wait();
+                if (valid)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        store_f4(reinterpret_cast<float*>(WQg), tc::kmajor_off(r, c0 + 4 * q, 2 * C),
+                                 make_float4(tc::round_tf32(v[4 * q]), tc::round_tf32(v[4 * q + 1]),
+                                             tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
+            }
+            {  // U^T row j (M = DV layout), the warp's group of C / NCG columns r
+                static_assert(C / NCG == 16, "one 16-column load per warp");
+                const bool vj = DV == 128 || lane < 16;
+                const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
+                const int c0 = cg * 16;
+                float v[16];
+                tc::tmem_ld16(tU + lane_base + c0, v);
+                tc::tmem_ld_wait();
+                if (vj)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        store_f4(reinterpret_cast<float*>(Ug), tc::kmajor_off(jr, c0 + 4 * q, DV),
+                                 make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+            }
+        }
+    };
+    // warp 0: wait for value head jj's gates and scan them (warp-uniform result)
+    auto scan_gates = [&](int jj) -> bool {
+        const int bb = jj & 1;
+        bool okg = tc::mbar_wait(tc::smem_u32(&sm.bar_g[bb]), n_g[bb] & 1u);
+        ++n_g[bb];
+        okg = __all_sync(0xffffffffu, okg);
+        if (okg) {  // inclusive scan of g over the chunk, two rows per lane
+            const float2 g0 = sm.gb[bb][2 * lane], g1 = sm.gb[bb][2 * lane + 1];
             const float pair = g0.x + g1.x;
             float incl = pair;
 #pragma unroll
@@ -223,13 +258,22 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             sm.fkt[2 * lane] = 2 * lane < n ? __expf(gn - gA) : 0.f;
             sm.fkt[2 * lane + 1] = 2 * lane + 1 < n ? __expf(gn - incl) : 0.f;
         }
-        if (j == 0) {
+        return okg;
+    };
+    for (int j = 0; j < G && ok; ++j) {
+        const int h = hk * G + j;
+        const size_t ch_h = (size_t)id * HV + h;
+        char* WQg = reinterpret_cast<char*>(p.WQ + ch_h * (2 * C * DK));
+        char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
+        char* KTg = reinterpret_cast<char*>(p.KT + ch_h * (DK * C));
+        if (j == 0) {  // head 0's gates, and D1; later heads' gates are scanned during the previous head's MMA
+            bool okv = warp == 0 ? scan_gates(0) : true;
             okv = okv && tc::mbar_wait(bar, ph_mma);
             ph_mma ^= 1;
+            ok = __syncthreads_and(okv);
+            if (!ok) break;
+            tc::fence_after_sync();
         }
-        ok = __syncthreads_and(okv);
-        if (!ok) break;
-        tc::fence_after_sync();
         const float gl = sm.gam[n - 1];
         {  // A (sub-partitions 0-1: k.k rows) and the masked decayed q.k tile (2-3: q.k rows) from D1;
            // the warps of a sub-partition take one group of C / NCG columns each
@@ -264,7 +308,10 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 }
             }
         }
+        if (j > 0) epilogue(j - 1);  // the previous head's W and U^T, from other tensor-memory columns
+        tc::fence_before_sync();
         __syncthreads();
+        tc::fence_after_sync();
         // T = (I + A)^{-1}, by blocks.  Every final entry goes straight into the K-major tf32 tile of
         // T diag(beta) (the A operand of W and U); the fp32 copy tf holds what the next level reads.
         //   level 1: the four diagonal 16x16 blocks by forward substitution, one column per lane held
@@ -386,13 +433,16 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 tc::mma_commit(bar);
             }
         }
+        bool okn = true;
+        if (warp == 0 && j + 1 < G) okn = scan_gates(j + 1);  // head j's gate arrays are no longer read
         ++n_v;
-        ok = okm && tc::mbar_wait(bar, ph_mma);  // okm is false only on tid 0, if the V tile never came
+        ok = okm && okn && tc::mbar_wait(bar, ph_mma);  // okm is false only on tid 0, if the V tile never came
         ph_mma ^= 1;
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc::fence_after_sync();
         if (tid == 0) {  // the V^T tile and gate buffer b are free again; after the last head, so is [K ; Q]
+                         // (the last head's epilogue reads only tensor memory)
             if (j + 1 < G) fetch_v(item, j + 1);
             if (j + 2 < G) fetch_g(item, j + 2);
             if (j == G - 1 && nxt >= 0) {  // the next item's tiles land during this epilogue
@@ -402,38 +452,12 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 fetch_v(nxt, 0);
             }
         }
-        {  // W rows -> [W ; Qg] tile rows 0..63 (tf32, K-major); U -> U^T tile (fp32, K-major).
-           // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15;
-           // the warps of a sub-partition take one group of columns each
-            const bool valid = lane < 16;
-            const int r = sp * 16 + lane;
-#pragma unroll
-            for (int c0 = cg * (DK / NCG); c0 < (cg + 1) * (DK / NCG); c0 += 16) {
-                float v[16];
-                tc::tmem_ld16(tW + lane_base + c0, v);
-                tc::tmem_ld_wait();
-                if (valid)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        store_f4(reinterpret_cast<float*>(WQg), tc::kmajor_off(r, c0 + 4 * q, 2 * C),
-                                 make_float4(tc::round_tf32(v[4 * q]), tc::round_tf32(v[4 * q + 1]),
-                                             tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
-            }
-            {  // U^T row j (M = DV layout), the warp's group of C / NCG columns r
-                static_assert(C / NCG == 16, "one 16-column load per warp");
-                const bool vj = DV == 128 || lane < 16;
-                const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
-                const int c0 = cg * 16;
-                float v[16];
-                tc::tmem_ld16(tU + lane_base + c0, v);
-                tc::tmem_ld_wait();
-                if (vj)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        store_f4(reinterpret_cast<float*>(Ug), tc::kmajor_off(jr, c0 + 4 * q, DV),
-                                 make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
-            }
-        }
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    }
+    if (ok) {
+        epilogue(G - 1);
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();

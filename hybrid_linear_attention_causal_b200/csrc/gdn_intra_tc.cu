@@ -49,7 +49,7 @@ struct IntraTcSmem {
     float a[C][C + 1];     // A (fp32)
     float tf[C][C + 4];    // T (fp32), the blocks the next level of the inverse reads
     float m[32][36];       // A21 T11
-    float y[2][16][17];    // A21 D1 inside each 32x32 diagonal block
+    float y[2][16][20];    // A21 D1 inside each 32x32 diagonal block (rows 16-byte aligned)
     float2 gb[2][C];       // (g, beta) of the two heads in flight
     float gam[C], beta[C], eg[C];
     float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
@@ -372,47 +372,62 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[tid - 128];
         }
         __syncthreads();
-        static_assert(NT == 512, "the level 2 and 3 thread maps below assume 512 threads");
-        {  // level 2: thread -> 32-block bb, row r, column c
-            const int bb = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
+        // Levels 2 and 3 tile the outputs in registers: a thread takes four consecutive columns of
+        // one row, so each step of a dot product is one (broadcast) load of the left factor and one
+        // 16-byte load of the right one for four FMAs; the shared-memory pipe, not the FMAs, bounds
+        // these small products.
+        static_assert(NT >= 256, "level 3 takes 256 threads");
+        auto fma4 = [](float4& acc, float a, const float4& b) {
+            acc.x = fmaf(a, b.x, acc.x);
+            acc.y = fmaf(a, b.y, acc.y);
+            acc.z = fmaf(a, b.z, acc.z);
+            acc.w = fmaf(a, b.w, acc.w);
+        };
+        {  // level 2 (threads 0..127): 32-block bb, row r, columns c4 .. c4 + 3
+            const int bb = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
             const int o0 = 32 * bb, o1 = o0 + 16;
-            float y[2] = {0.f, 0.f};
+            if (tid < 128) {
+                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int s = 0; s < 16; ++s)  // Y = A21 D1
-                y[s & 1] = fmaf(sm.a[o1 + r][o0 + s], sm.tf[o0 + s][o0 + c], y[s & 1]);
-            sm.y[bb][r][c] = y[0] + y[1];
+                for (int s = 0; s < 16; ++s)  // Y = A21 D1
+                    fma4(y, sm.a[o1 + r][o0 + s], *reinterpret_cast<const float4*>(&sm.tf[o0 + s][o0 + c4]));
+                *reinterpret_cast<float4*>(&sm.y[bb][r][c4]) = y;
+            }
             __syncthreads();
-            float x[2] = {0.f, 0.f};
+            if (tid < 128) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int s = 0; s < 16; ++s)  // X = -D2 Y
-                x[s & 1] = fmaf(sm.tf[o1 + r][o1 + s], sm.y[bb][s][c], x[s & 1]);
-            sm.tf[o1 + r][o0 + c] = -(x[0] + x[1]);
-            put_t(o1 + r, o0 + c, -(x[0] + x[1]));
+                for (int s = 0; s < 16; ++s)  // X = -D2 Y
+                    fma4(x, sm.tf[o1 + r][o1 + s], *reinterpret_cast<const float4*>(&sm.y[bb][s][c4]));
+                x = make_float4(-x.x, -x.y, -x.z, -x.w);
+                *reinterpret_cast<float4*>(&sm.tf[o1 + r][o0 + c4]) = x;
+                put_t(o1 + r, o0 + c4, x.x);
+                put_t(o1 + r, o0 + c4 + 1, x.y);
+                put_t(o1 + r, o0 + c4 + 2, x.z);
+                put_t(o1 + r, o0 + c4 + 3, x.w);
+            }
         }
         __syncthreads();
-        {  // level 3: thread -> row r, columns c2, c2 + 1
-            const int r = tid >> 4, c2 = 2 * (tid & 15);
-            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        {  // level 3 (threads 0..255): row r, columns c4 .. c4 + 3
+            const int r = tid >> 3, c4 = 4 * (tid & 7);
+            if (tid < 256) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
-            for (int s = 0; s < 32; ++s) {  // P = A21 T11
-                const float av = sm.a[32 + r][s];
-                const float2 tv = *reinterpret_cast<const float2*>(&sm.tf[s][c2]);
-                acc[s & 1].x = fmaf(av, tv.x, acc[s & 1].x);
-                acc[s & 1].y = fmaf(av, tv.y, acc[s & 1].y);
+                for (int s = 0; s < 32; ++s)  // P = A21 T11
+                    fma4(acc, sm.a[32 + r][s], *reinterpret_cast<const float4*>(&sm.tf[s][c4]));
+                *reinterpret_cast<float4*>(&sm.m[r][c4]) = acc;
             }
-            *reinterpret_cast<float2*>(&sm.m[r][c2]) =
-                make_float2(acc[0].x + acc[1].x, acc[0].y + acc[1].y);
             __syncthreads();
-            acc[0] = acc[1] = make_float2(0.f, 0.f);
+            if (tid < 256) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
-            for (int s = 0; s < 32; ++s) {  // T21 = -T22 P
-                const float tv = sm.tf[32 + r][32 + s];
-                const float2 pv = *reinterpret_cast<const float2*>(&sm.m[s][c2]);
-                acc[s & 1].x = fmaf(tv, pv.x, acc[s & 1].x);
-                acc[s & 1].y = fmaf(tv, pv.y, acc[s & 1].y);
+                for (int s = 0; s < 32; ++s)  // T21 = -T22 P
+                    fma4(acc, sm.tf[32 + r][32 + s], *reinterpret_cast<const float4*>(&sm.m[s][c4]));
+                // the four columns are contiguous in the K-major tile
+                store_f4(sm.t, tc::kmajor_off(32 + r, c4, C),
+                         make_float4(tc::round_tf32(-acc.x * sm.beta[c4]), tc::round_tf32(-acc.y * sm.beta[c4 + 1]),
+                                     tc::round_tf32(-acc.z * sm.beta[c4 + 2]), tc::round_tf32(-acc.w * sm.beta[c4 + 3])));
             }
-            put_t(32 + r, c2, -(acc[0].x + acc[1].x));
-            put_t(32 + r, c2 + 1, -(acc[0].y + acc[1].y));
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();

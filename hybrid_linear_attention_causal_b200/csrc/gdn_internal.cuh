@@ -119,10 +119,10 @@ struct ExtendArgs {
     // per (chunk, value head), written by the intra kernel, read by the state
     // pass; the three tiles are tf32 values already in the tensor-core
     // shared-memory layout, so the state pass copies them verbatim
-    float* WQ;          // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], K-major, 128 rows
-    float* AQ;          // [max_chunks, HV, C*C]     masked decayed q.k, K-major, C rows
-    float* KT;          // [max_chunks, HV, dk*C]    (diag(e^{gamma_n-gamma}) K)^T, K-major, dk rows
-    float* U;           // [max_chunks, HV, dv*C]    U^T fp32, K-major tile of dv rows (j) x C
+    uint16_t* WQ;       // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], fp16, K-major, 128 rows
+    uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, fp16, K-major, C rows
+    uint16_t* KT;       // [max_chunks, HV, dk*C]    (diag(e^{gamma_n-gamma}) K)^T, fp16, K-major, dk rows
+    uint16_t* U;        // [max_chunks, HV, dv*C]    U^T, fp16, K-major tile of dv rows (j) x C
     float* gam;         // [max_chunks, HV, C]       in-chunk cumulative g
 };
 

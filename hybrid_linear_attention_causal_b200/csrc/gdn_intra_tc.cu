@@ -68,6 +68,22 @@ __device__ __forceinline__ float load_f(const float* tile, uint32_t off) {
 // idx -> (row, first column) of a K-major tile with R rows, chosen so that the
 // 32 lanes of a warp cover 8 consecutive rows x 4 column quads: each group of
 // 8 lanes then touches one contiguous 128-byte core matrix.
+// idx -> (row, first column) of an 8-column group of a 16-bit K-major tile with R rows: 8
+// consecutive lanes take 8 consecutive rows, i.e. one 128-byte core matrix
+template <int R>
+__device__ __forceinline__ void tile_coord8(int idx, int& r, int& k8) {
+    const int rr = idx & 7, rest = idx >> 3;
+    r = 8 * (rest % (R / 8)) + rr;
+    k8 = 8 * (rest / (R / 8));
+}
+
+// 8 floats -> 8 fp16 at byte offset `off` of a 16-bit tile (one 16-byte store)
+__device__ __forceinline__ void store_h8(void* tile, uint32_t off, const float* v) {
+    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(tile) + off) =
+        make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]), tc::pack_f16(v[4], v[5]),
+                   tc::pack_f16(v[6], v[7]));
+}
+
 template <int R>
 __device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
     const int rr = idx & 7, cc = (idx >> 3) & 3, rest = idx >> 5;
@@ -209,12 +225,10 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 float v[16];
                 tc::tmem_ld16(tW + lane_base + c0, v);
                 tc::tmem_ld_wait();
-                if (valid)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        store_f4(reinterpret_cast<float*>(WQg), tc::kmajor_off(r, c0 + 4 * q, 2 * C),
-                                 make_float4(tc::round_tf32(v[4 * q]), tc::round_tf32(v[4 * q + 1]),
-                                             tc::round_tf32(v[4 * q + 2]), tc::round_tf32(v[4 * q + 3])));
+                if (valid) {
+                    store_h8(WQg, tc::kmajor_off16(r, c0, 2 * C), v);
+                    store_h8(WQg, tc::kmajor_off16(r, c0 + 8, 2 * C), v + 8);
+                }
             }
             {  // U^T row j (M = DV layout), the warp's group of C / NCG columns r
                 static_assert(C / NCG == 16, "one 16-column load per warp");
@@ -224,11 +238,10 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 float v[16];
                 tc::tmem_ld16(tU + lane_base + c0, v);
                 tc::tmem_ld_wait();
-                if (vj)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        store_f4(reinterpret_cast<float*>(Ug), tc::kmajor_off(jr, c0 + 4 * q, DV),
-                                 make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+                if (vj) {
+                    store_h8(Ug, tc::kmajor_off16(jr, c0, DV), v);
+                    store_h8(Ug, tc::kmajor_off16(jr, c0 + 8, DV), v + 8);
+                }
             }
         }
     };
@@ -297,14 +310,14 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < NC; i += 4) {
-                    float o[4];
+                for (int i = 0; i < NC; i += 8) {
+                    float o[8];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < 8; ++u) {
                         const int s = c0 + i + u;
-                        o[u] = (s <= r && r < n) ? tc::round_tf32(__expf(gr - sm.gam[s]) * row[i + u]) : 0.f;
+                        o[u] = (s <= r && r < n) ? __expf(gr - sm.gam[s]) * row[i + u] : 0.f;
                     }
-                    store_f4(reinterpret_cast<float*>(AQg), tc::kmajor_off(r, c0 + i, C), make_float4(o[0], o[1], o[2], o[3]));
+                    store_h8(AQg, tc::kmajor_off16(r, c0 + i, C), o);
                 }
             }
         }
@@ -354,20 +367,29 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 store_f4(sm.kte, off,
                          make_float4(tc::round_tf32(k.x * sm.eg[s4]), tc::round_tf32(k.y * sm.eg[s4 + 1]),
                                      tc::round_tf32(k.z * sm.eg[s4 + 2]), tc::round_tf32(k.w * sm.eg[s4 + 3])));
-                // the state pass's (diag(e^{gamma_n-gamma}) K)^T, same tile offsets
-                store_f4(reinterpret_cast<float*>(KTg), off,
-                         make_float4(tc::round_tf32(k.x * sm.fkt[s4]), tc::round_tf32(k.y * sm.fkt[s4 + 1]),
-                                     tc::round_tf32(k.z * sm.fkt[s4 + 2]), tc::round_tf32(k.w * sm.fkt[s4 + 3])));
             }
-            for (int idx = tid - 128; idx < C * DK / 4; idx += NW) {  // rows Qg = diag(e^gamma) Q of [W ; Qg]
-                int r, k4;
-                tile_coord<C>(idx, r, k4);
-                const uint32_t off = tc::kmajor_off(C + r, k4, 2 * C);
-                const float4 q = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) + off);
+            for (int idx = tid - 128; idx < DK * C / 8; idx += NW) {  // the state pass's (diag(e^{gamma_n-gamma}) K)^T
+                int f, s8;
+                tile_coord8<DK>(idx, f, s8);
+                const float4 k0 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) +
+                                                                   tc::kmajor_off(f, s8, DK));
+                const float4 k1 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) +
+                                                                   tc::kmajor_off(f, s8 + 4, DK));
+                const float v[8] = {k0.x * sm.fkt[s8],     k0.y * sm.fkt[s8 + 1], k0.z * sm.fkt[s8 + 2],
+                                    k0.w * sm.fkt[s8 + 3], k1.x * sm.fkt[s8 + 4], k1.y * sm.fkt[s8 + 5],
+                                    k1.z * sm.fkt[s8 + 6], k1.w * sm.fkt[s8 + 7]};
+                store_h8(KTg, tc::kmajor_off16(f, s8, DK), v);
+            }
+            for (int idx = tid - 128; idx < C * DK / 8; idx += NW) {  // rows Qg = diag(e^gamma) Q of [W ; Qg]
+                int r, k8;
+                tile_coord8<C>(idx, r, k8);
+                const float4 q0 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) +
+                                                                   tc::kmajor_off(C + r, k8, 2 * C));
+                const float4 q1 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) +
+                                                                   tc::kmajor_off(C + r, k8 + 4, 2 * C));
                 const float e = sm.eg[r];
-                store_f4(reinterpret_cast<float*>(WQg), off,
-                         make_float4(tc::round_tf32(q.x * e), tc::round_tf32(q.y * e), tc::round_tf32(q.z * e),
-                                     tc::round_tf32(q.w * e)));
+                const float v[8] = {q0.x * e, q0.y * e, q0.z * e, q0.w * e, q1.x * e, q1.y * e, q1.z * e, q1.w * e};
+                store_h8(WQg, tc::kmajor_off16(C + r, k8, 2 * C), v);
             }
             if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[tid - 128];
         }

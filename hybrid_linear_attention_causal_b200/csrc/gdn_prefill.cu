@@ -450,51 +450,60 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
 
 }  // namespace
 
-size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max_chunks_out) {
-    const size_t mc = (size_t)max_T / C + (size_t)max_N + 1;
-    if (max_chunks_out) *max_chunks_out = (int)mc;
-    auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
-    const size_t per = mc * d.HV * sizeof(float);
+namespace {
+
+// One walk over the extend workspace: the total size, and with `e` set the carved pointers.
+size_t walk_extend_workspace(const LayerDims& d, int max_N, int max_T, char* base, ExtendArgs* e) {
+    const size_t mc = (size_t)max_T / C + (size_t)max_N + 1;  // chunk capacity
+    const size_t units = mc * d.HV;                           // (chunk, value head) units
     size_t off = kHeaderBytes;
-    off += al(mc * sizeof(int4));
-    off += al(((size_t)max_N + 1) * sizeof(int32_t));
-    off += al((size_t)max_N * sizeof(int32_t));
-    off += al(((size_t)max_N + 1) * sizeof(int32_t));
-    off += al(mc * sizeof(int32_t));
-    off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
-    off += al(per * d.dv * C);
-    off += al(per * C * 2);
-    off += al(per * 2 * C * d.dk);
-    off += al(per * C * C);
-    off += al(per * d.dk * C);
-    off += al(per * C * d.dv);
-    off += al(per * C);
+    auto take = [&](size_t bytes) {
+        char* ptr = base ? base + off : nullptr;
+        off += (bytes + 255) & ~(size_t)255;
+        return ptr;
+    };
+    char* chunk_tab = take(mc * sizeof(int4));
+    char* seq_chunk0 = take(((size_t)max_N + 1) * sizeof(int32_t));
+    char* seq_order = take((size_t)max_N * sizeof(int32_t));
+    char* rank_off = take(((size_t)max_N + 1) * sizeof(int32_t));
+    char* chunk_list = take(mc * sizeof(int32_t));
+    char* kq = take(mc * d.HK * 2 * C * d.dk * sizeof(float));
+    char* vt = take(units * d.dv * C * sizeof(float));
+    char* gb = take(units * C * sizeof(float2));
+    char* wq = take(units * 2 * C * d.dk * sizeof(uint16_t));
+    char* aq = take(units * C * C * sizeof(uint16_t));
+    char* kt = take(units * d.dk * C * sizeof(uint16_t));
+    char* u = take(units * d.dv * C * sizeof(uint16_t));
+    char* gam = take(units * C * sizeof(float));
+    if (e) {
+        e->max_chunks = (int)mc;
+        e->hdr = reinterpret_cast<int32_t*>(base);
+        e->chunk_tab = reinterpret_cast<int4*>(chunk_tab);
+        e->seq_chunk0 = reinterpret_cast<int32_t*>(seq_chunk0);
+        e->seq_order = reinterpret_cast<int32_t*>(seq_order);
+        e->rank_off = reinterpret_cast<int32_t*>(rank_off);
+        e->chunk_list = reinterpret_cast<int32_t*>(chunk_list);
+        e->KQ = reinterpret_cast<float*>(kq);
+        e->VT = reinterpret_cast<float*>(vt);
+        e->GB = reinterpret_cast<float2*>(gb);
+        e->WQ = reinterpret_cast<uint16_t*>(wq);
+        e->AQ = reinterpret_cast<uint16_t*>(aq);
+        e->KT = reinterpret_cast<uint16_t*>(kt);
+        e->U = reinterpret_cast<uint16_t*>(u);
+        e->gam = reinterpret_cast<float*>(gam);
+    }
     return off;
 }
 
+}  // namespace
+
+size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max_chunks_out) {
+    if (max_chunks_out) *max_chunks_out = (int)((size_t)max_T / C + (size_t)max_N + 1);
+    return walk_extend_workspace(d, max_N, max_T, nullptr, nullptr);
+}
+
 void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T) {
-    const LayerDims& d = e.d;
-    int mc = 0;
-    extend_workspace_bytes(d, max_N, max_T, &mc);
-    e.max_chunks = mc;
-    auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
-    const size_t per = (size_t)mc * d.HV * sizeof(float);
-    char* base = static_cast<char*>(ws);
-    e.hdr = reinterpret_cast<int32_t*>(base);
-    size_t off = kHeaderBytes;
-    e.chunk_tab = reinterpret_cast<int4*>(base + off); off += al((size_t)mc * sizeof(int4));
-    e.seq_chunk0 = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
-    e.seq_order = reinterpret_cast<int32_t*>(base + off); off += al((size_t)max_N * sizeof(int32_t));
-    e.rank_off = reinterpret_cast<int32_t*>(base + off); off += al(((size_t)max_N + 1) * sizeof(int32_t));
-    e.chunk_list = reinterpret_cast<int32_t*>(base + off); off += al((size_t)mc * sizeof(int32_t));
-    e.KQ = reinterpret_cast<float*>(base + off); off += al((size_t)mc * d.HK * 2 * C * d.dk * sizeof(float));
-    e.VT = reinterpret_cast<float*>(base + off); off += al(per * d.dv * C);
-    e.GB = reinterpret_cast<float2*>(base + off); off += al(per * C * 2);
-    e.WQ = reinterpret_cast<float*>(base + off); off += al(per * 2 * C * d.dk);
-    e.AQ = reinterpret_cast<float*>(base + off); off += al(per * C * C);
-    e.KT = reinterpret_cast<float*>(base + off); off += al(per * d.dk * C);
-    e.U = reinterpret_cast<float*>(base + off); off += al(per * C * d.dv);
-    e.gam = reinterpret_cast<float*>(base + off);
+    walk_extend_workspace(e.d, max_N, max_T, static_cast<char*>(ws), &e);
 }
 
 cudaError_t launch_extend(const ExtendArgs& p, int dtype, cudaStream_t s) {

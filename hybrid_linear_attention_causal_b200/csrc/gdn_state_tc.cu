@@ -20,11 +20,11 @@
 //     product only once the state product has completed;
 //   - the fp32 state lives in registers (each thread holds one half of row j
 //     of S^T), the state product goes to a fresh accumulator and the update
-//     is one FMA per element, written straight into the tf32 operand copy;
+//     is one FMA per element, written straight into the fp16 operand copy;
 //   - [X^T | O^T] is double-buffered in tensor memory: a chunk's outputs are
 //     read and stored while the next chunk's first product runs;
 //   - the tiles [W ; Qg], K~^T and Aqk (written by the intra-chunk kernel as
-//     tf32 in the tensor core's layout) each have their own barrier and are
+//     fp16 in the tensor core's layout) each have their own barrier and are
 //     refetched as soon as the product that reads them completes;
 //   - the intra-chunk kernel writes U^T in the layout of the V'^T operand
 //     tile, so it lands in that tile by one bulk copy and V' is formed in
@@ -51,28 +51,27 @@ constexpr bool kStageOut = sizeof(T) == 2;
 
 template <typename T, int DK, int DV>
 struct StateTcSmem {
-    float st[DV * DK];     // S^T tile, K-major: DV rows x DK (tf32 copy of the state)
-    float wq[2 * C * DK];  // [W ; Qg] tile (bulk copy), K-major: 128 rows x DK
-    float aq[C * C];       // Aqk tile (bulk copy), K-major: C rows (r) x C (s)
-    float kt[DK * C];      // K~^T tile (bulk copy), K-major: DK rows (i) x C (s)
-    float vt[DV * C];      // U^T tile (bulk copy), overwritten in place by V'^T: K-major, DV rows (j) x C (s)
+    // fp16 operand tiles (16-bit K-major layout)
+    uint16_t st[DV * DK];     // S^T tile: DV rows x DK (fp16 copy of the state)
+    uint16_t wq[2 * C * DK];  // [W ; Qg] tile (bulk copy): 128 rows x DK
+    uint16_t aq[C * C];       // Aqk tile (bulk copy): C rows (r) x C (s)
+    uint16_t kt[DK * C];      // K~^T tile (bulk copy): DK rows (i) x C (s)
+    uint16_t vt[DV * C];      // U^T tile (bulk copy), overwritten in place by V'^T: DV rows (j) x C (s)
     T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
     unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq, bar_u;
     uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void store_f4(float* tile, uint32_t off, float4 v) {
-    *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + off) = v;
-}
 
-// tf32 copies of 16 consecutive values of S^T row j (columns c0..c0+15) into the operand tile
+// fp16 copies of 16 consecutive values of S^T row j (columns c0..c0+15, c0 a multiple of 8) into
+// the operand tile: two 16-byte vectors
 template <int DV>
-__device__ __forceinline__ void put_st16(float* st, int j, int c0, const float* v) {
+__device__ __forceinline__ void put_st16(uint16_t* st, int j, int c0, const float* v) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-        store_f4(st, tc::kmajor_off(j, c0 + 4 * q, DV),
-                 make_float4(tc::round_tf32(v[4 * q]), tc::round_tf32(v[4 * q + 1]), tc::round_tf32(v[4 * q + 2]),
-                             tc::round_tf32(v[4 * q + 3])));
+    for (int q = 0; q < 2; ++q)
+        *reinterpret_cast<uint4*>(reinterpret_cast<char*>(st) + tc::kmajor_off16(j, c0 + 8 * q, DV)) =
+            make_uint4(tc::pack_f16(v[8 * q], v[8 * q + 1]), tc::pack_f16(v[8 * q + 2], v[8 * q + 3]),
+                       tc::pack_f16(v[8 * q + 4], v[8 * q + 5]), tc::pack_f16(v[8 * q + 6], v[8 * q + 7]));
 }
 
 template <typename T, int DK, int DV>
@@ -107,7 +106,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                    bar_o = tc::smem_u32(&sm.bar_o), bar_wq = tc::smem_u32(&sm.bar_wq),
                    bar_kt = tc::smem_u32(&sm.bar_kt), bar_aq = tc::smem_u32(&sm.bar_aq),
                    bar_u = tc::smem_u32(&sm.bar_u);
-    constexpr uint32_t WQ_BYTES = 2 * C * DK * 4, AQ_BYTES = C * C * 4, KT_BYTES = DK * C * 4;
+    constexpr uint32_t WQ_BYTES = 2 * C * DK * 2, AQ_BYTES = C * C * 2, KT_BYTES = DK * C * 2, U_BYTES = DV * C * 2;
     auto fetch_wq = [&](int id) {
         tc::mbar_expect_tx(bar_wq, WQ_BYTES);
         tc::bulk_g2s(tc::smem_u32(sm.wq), p.WQ + ((size_t)id * HV + h) * (2 * C * DK), WQ_BYTES, bar_wq);
@@ -118,8 +117,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     };
     auto u_src = [&](int id) { return p.U + ((size_t)id * HV + h) * (DV * C); };
     auto fetch_u = [&](int id) {
-        tc::mbar_expect_tx(bar_u, DV * C * 4);
-        tc::bulk_g2s(tc::smem_u32(sm.vt), u_src(id), DV * C * 4, bar_u);
+        tc::mbar_expect_tx(bar_u, U_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.vt), u_src(id), U_BYTES, bar_u);
     };
     auto fetch_aq = [&](int id) {
         tc::mbar_expect_tx(bar_aq, AQ_BYTES);
@@ -209,10 +208,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             okl = tc::mbar_wait(bar_wq, ph);
             if (okl) {  // [X^T | O^T] = S^T [W ; Qg]^T
                 const uint32_t a = tc::smem_u32(sm.st), b = tc::smem_u32(sm.wq);
-                constexpr uint32_t idesc = tc::idesc_tf32(DV, 128);
+                constexpr uint32_t idesc = tc::idesc_f16(DV, 128);
 #pragma unroll
-                for (int k = 0; k < DK / 8; ++k)
-                    tc::mma_tf32(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
+                for (int k = 0; k < DK / 16; ++k)
+                    tc::mma_f16(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
                 tc::mma_commit(bar_x);
             }
             if (okl && id + 1 < c_end) {  // the next chunk's tiles into L2, so their copies wait on L2 only
@@ -220,7 +219,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
                 tc::bulk_prefetch_l2(p.KT + nx * (DK * C), KT_BYTES);
                 tc::bulk_prefetch_l2(p.AQ + nx * (C * C), AQ_BYTES);
-                tc::bulk_prefetch_l2(u_src(id + 1), DV * C * 4);
+                tc::bulk_prefetch_l2(u_src(id + 1), U_BYTES);
             }
             if (okl) {
                 okl = tc::mbar_wait(bar_x, ph);
@@ -245,12 +244,15 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     tc::tmem_ld_wait();
                     if (rowv)
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t off = tc::kmajor_off(j, c0 + 4 * q, DV);
-                            const float4 u = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.vt) + off);
-                            store_f4(sm.vt, off,
-                                     make_float4(tc::round_tf32(u.x - x[4 * q]), tc::round_tf32(u.y - x[4 * q + 1]),
-                                                 tc::round_tf32(u.z - x[4 * q + 2]), tc::round_tf32(u.w - x[4 * q + 3])));
+                        for (int q = 0; q < 2; ++q) {  // 8 fp16 values per 16-byte vector
+                            uint4* pv = reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.vt) +
+                                                                 tc::kmajor_off16(j, c0 + 8 * q, DV));
+                            const uint4 u = *pv;
+                            const float2 u0 = tc::unpack_f16(u.x), u1 = tc::unpack_f16(u.y), u2 = tc::unpack_f16(u.z),
+                                         u3 = tc::unpack_f16(u.w);
+                            const float* xq = x + 8 * q;
+                            *pv = make_uint4(tc::pack_f16(u0.x - xq[0], u0.y - xq[1]), tc::pack_f16(u1.x - xq[2], u1.y - xq[3]),
+                                             tc::pack_f16(u2.x - xq[4], u2.y - xq[5]), tc::pack_f16(u3.x - xq[6], u3.y - xq[7]));
                         }
                 }
             }
@@ -264,10 +266,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             okl = tc::mbar_wait(bar_kt, ph);
             if (okl) {  // Snew^T = V'^T K~
                 const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt);
-                constexpr uint32_t is = tc::idesc_tf32(DV, DK);
+                constexpr uint32_t is = tc::idesc_f16(DV, DK);
 #pragma unroll
-                for (int k = 0; k < C / 8; ++k)
-                    tc::mma_tf32(tS, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bk, DK, k), is, k > 0);
+                for (int k = 0; k < C / 16; ++k)
+                    tc::mma_f16(tS, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bk, DK, k), is, k > 0);
                 tc::mma_commit(bar_s);
                 okl = tc::mbar_wait(bar_s, ph);
             }
@@ -275,10 +277,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             if (okl) okl = tc::mbar_wait(bar_aq, ph);
             if (okl) {  // O^T += V'^T Aqk^T, off the state chain
                 const uint32_t av = tc::smem_u32(sm.vt), bq = tc::smem_u32(sm.aq);
-                constexpr uint32_t io = tc::idesc_tf32(DV, 64);
+                constexpr uint32_t io = tc::idesc_f16(DV, 64);
 #pragma unroll
-                for (int k = 0; k < C / 8; ++k)
-                    tc::mma_tf32(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
+                for (int k = 0; k < C / 16; ++k)
+                    tc::mma_f16(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
                 tc::mma_commit(bar_o);
                 // the next chunk's Aqk and U^T, once the output product is done with the Aqk and V'^T tiles
                 okl = tc::mbar_wait(bar_o, ph);
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
                                                           // state product runs meanwhile
             okl = __all_sync(0xffffffffu, tc::mbar_wait(bar_s, ph));
-            if (okl) {  // S^T <- e^{gamma_n} S^T + Snew^T, and its tf32 copy for the next chunk
+            if (okl) {  // S^T <- e^{gamma_n} S^T + Snew^T, and its fp16 copy for the next chunk
                 tc::fence_after_sync();
                 const float egl = expf(gl);
 #pragma unroll

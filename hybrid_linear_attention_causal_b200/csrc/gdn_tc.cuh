@@ -43,6 +43,12 @@ __device__ __forceinline__ uint32_t kmajor_off(int r, int k, int R) {
     return (uint32_t)(((k >> 2) * (R >> 3) + (r >> 3)) * 128 + (r & 7) * 16 + (k & 3) * 4);
 }
 
+// byte offset of element (r, k) of a 16-bit K-major tile with R rows: core matrices of 8 rows x
+// 8 elements (16 bytes), the same 128-byte blocks as above
+__device__ __forceinline__ uint32_t kmajor_off16(int r, int k, int R) {
+    return (uint32_t)(((k >> 3) * (R >> 3) + (r >> 3)) * 128 + (r & 7) * 16 + (k & 7) * 2);
+}
+
 // 64-bit shared-memory matrix descriptor, no swizzle, sm_100 version field.
 __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
@@ -53,7 +59,7 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint
     return d;                // base offset 0, legacy LBO mode, layout type 0 (no swizzle)
 }
 
-// descriptor of MMA k-step `s` (8 tf32 along K) of a K-major tile with R rows
+// descriptor of MMA k-step `s` (8 tf32 or 16 fp16 along K: 32 bytes) of a K-major tile with R rows
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int R, int s) {
     const uint32_t lbo = (uint32_t)(R >> 3) * 128;
     return make_desc(base + 2 * s * lbo, lbo, 128);
@@ -67,6 +73,39 @@ __device__ __forceinline__ constexpr uint32_t idesc_tf32(int M, int N) {
            | (2u << 10)                   // B format: tf32
            | ((uint32_t)(N >> 3) << 17)
            | ((uint32_t)(M >> 4) << 24);
+}
+
+// 32-bit instruction descriptor: kind::f16 with fp16 A and B, fp32 accumulate, shape M x N,
+// both operands K-major.  fp16 keeps tf32's 10-bit mantissa, so an operand rounded to fp16 is
+// the value a tf32 operand would be, within fp16's range, at half the bytes and with 16 K per MMA.
+__device__ __forceinline__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4)                      // D format: f32 (A, B format fields 0: f16)
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// two floats -> one 32-bit word of two fp16 (round to nearest even), low half first
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 unpack_f16(uint32_t w) {
+    float2 f;
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(f.x), "=f"(f.y) : "r"(w));
+    return f;
 }
 
 __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,

@@ -113,8 +113,8 @@ struct ExtendArgs {
     int32_t* chunk_list;// [max_chunks] chunk ids, rank by rank (longest sequence first)
     int nseg;           // S
     // per chunk, written by the prep kernel (conv + SiLU + L2 norm + gates):
-    float* KQ;          // [max_chunks, HK, 2*C*dk] [K ; Q*scale] tf32, K-major tile of 128 rows
-    float* VT;          // [max_chunks, HV, dv*C]   V^T tf32, K-major tile of dv rows x C
+    uint16_t* KQ;       // [max_chunks, HK, 2*C*dk] [K ; Q*scale] fp16, K-major tile of 128 rows
+    uint16_t* VT;       // [max_chunks, HV, dv*C]   V^T fp16, K-major tile of dv rows x C
     float2* GB;         // [max_chunks, HV, C]      (g, beta); rows past the chunk end are zero
     // per (chunk, value head), written by the intra kernel, read by the state
     // pass; the three tiles are tf32 values already in the tensor-core

@@ -41,11 +41,12 @@ constexpr int kItemsPerCta = 4;
 
 template <int DK, int DV>
 struct IntraTcSmem {
-    float kq[2 * C * DK];  // [K ; Q*scale] tile from the prep kernel (bulk copy), K-major, 128 rows
-    float kt[DK * C];      // K^T, K-major, DK rows x C (built once, shared by the value heads)
-    float kte[DK * C];     // (diag(e^gamma) K)^T of the current head, same layout
-    float bv[DV * C];      // V^T tile of the current head (bulk copy), K-major, DV rows x C
-    float t[C * C];        // T diag(beta) as a K-major tile, C rows x C
+    // fp16 operand tiles (16-bit K-major layout)
+    uint16_t kq[2 * C * DK];  // [K ; Q*scale] tile from the prep kernel (bulk copy), 128 rows
+    uint16_t kt[DK * C];      // K^T, DK rows x C (built once, shared by the value heads)
+    uint16_t kte[DK * C];     // (diag(e^gamma) K)^T of the current head, same layout
+    uint16_t bv[DV * C];      // V^T tile of the current head (bulk copy), DV rows x C
+    uint16_t t[C * C];        // T diag(beta), C rows x C
     float a[C][C + 1];     // A (fp32)
     float tf[C][C + 4];    // T (fp32), the blocks the next level of the inverse reads
     float m[32][36];       // A21 T11
@@ -58,16 +59,6 @@ struct IntraTcSmem {
     int next_item;         // thread 0's latest grab, for the other threads
 };
 
-__device__ __forceinline__ void store_f4(float* tile, uint32_t off, float4 v) {
-    *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + off) = v;
-}
-__device__ __forceinline__ float load_f(const float* tile, uint32_t off) {
-    return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(tile) + off);
-}
-
-// idx -> (row, first column) of a K-major tile with R rows, chosen so that the
-// 32 lanes of a warp cover 8 consecutive rows x 4 column quads: each group of
-// 8 lanes then touches one contiguous 128-byte core matrix.
 // idx -> (row, first column) of an 8-column group of a 16-bit K-major tile with R rows: 8
 // consecutive lanes take 8 consecutive rows, i.e. one 128-byte core matrix
 template <int R>
@@ -77,6 +68,13 @@ __device__ __forceinline__ void tile_coord8(int idx, int& r, int& k8) {
     k8 = 8 * (rest / (R / 8));
 }
 
+// 8 fp16 at byte offset `off` of a 16-bit tile (one 16-byte load) -> 8 floats
+__device__ __forceinline__ void load_h8(const void* tile, uint32_t off, float* v) {
+    const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(tile) + off);
+    const float2 a = tc::unpack_f16(w.x), b = tc::unpack_f16(w.y), c = tc::unpack_f16(w.z), e = tc::unpack_f16(w.w);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y; v[4] = c.x; v[5] = c.y; v[6] = e.x; v[7] = e.y;
+}
+
 // 8 floats -> 8 fp16 at byte offset `off` of a 16-bit tile (one 16-byte store)
 __device__ __forceinline__ void store_h8(void* tile, uint32_t off, const float* v) {
     *reinterpret_cast<uint4*>(reinterpret_cast<char*>(tile) + off) =
@@ -84,13 +82,6 @@ __device__ __forceinline__ void store_h8(void* tile, uint32_t off, const float* 
                    tc::pack_f16(v[6], v[7]));
 }
 
-template <int R>
-__device__ __forceinline__ void tile_coord(int idx, int& r, int& k4) {
-    const int rr = idx & 7, cc = (idx >> 3) & 3, rest = idx >> 5;
-    const int rg = rest % (R / 8), cg = rest / (R / 8);
-    r = 8 * rg + rr;
-    k4 = 4 * (4 * cg + cc);
-}
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) {
@@ -120,7 +111,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     int item = sm.next_item;
     if (item < 0) return;
     const uint32_t bar = tc::smem_u32(&sm.bar_mma), bar_kq = tc::smem_u32(&sm.bar_kq);
-    constexpr uint32_t KQ_BYTES = 2 * C * DK * 4, VT_BYTES = DV * C * 4, GB_BYTES = C * 8;
+    constexpr uint32_t KQ_BYTES = 2 * C * DK * 2, VT_BYTES = DV * C * 2, GB_BYTES = C * 8;
     const uint32_t bar_v = tc::smem_u32(&sm.bar_v);
     auto kq_src = [&](int it) { return p.KQ + (size_t)it * (2 * C * DK); };  // [K ; Q] tiles are [chunk][hk]
     auto head_row = [&](int it, int jj) { return (size_t)(it / HK) * HV + (it % HK) * G + jj; };
@@ -160,7 +151,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     }
     // blocks of T above the diagonal are zero for every head: in the tile, and in the two 16x16
     // corners of the 32x32 diagonal blocks that the inverse reads back
-    for (int e = tid; e < C * C; e += NT) sm.t[e] = 0.f;
+    for (int e = tid; e < C * C; e += NT) sm.t[e] = 0;
     for (int e = tid; e < 2 * 256; e += NT) {
         const int o = 32 * (e >> 8);
         sm.tf[o + ((e >> 4) & 15)][o + 16 + (e & 15)] = 0.f;
@@ -190,22 +181,22 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         ok = tc::mbar_wait(bar_kq, n_kq & 1u);
         if (ok) {  // D1 = [K ; Q] K^T
             const uint32_t base = tc::smem_u32(sm.kq);
-            constexpr uint32_t idesc = tc::idesc_tf32(128, 64);
+            constexpr uint32_t idesc = tc::idesc_f16(128, 64);
 #pragma unroll
-            for (int s = 0; s < DK / 8; ++s)
-                tc::mma_tf32(tD1, tc::desc_kmajor(base, 2 * C, s), tc::desc_kmajor(base, 2 * C, s), idesc, s > 0);
+            for (int s = 0; s < DK / 16; ++s)
+                tc::mma_f16(tD1, tc::desc_kmajor(base, 2 * C, s), tc::desc_kmajor(base, 2 * C, s), idesc, s > 0);
             tc::mma_commit(bar);
         }
     }
     // K^T (feature rows) from the k rows of the [K ; Q] tile, once for all value heads.  A warp reads
-    // one 128-byte core matrix of the tile (8 rows s x 4 features f): no bank conflicts.
+    // 8 rows s x 4 features f of one 128-byte core matrix of the tile.
     ok = ok && tc::mbar_wait(bar_kq, n_kq & 1u);
     ++n_kq;
     if (ok)
         for (int idx = tid; idx < DK * C; idx += NT) {
             const int s = (idx & 7) + 8 * ((idx >> 5) & 7), f = ((idx >> 3) & 3) + 4 * (idx >> 8);
-            *reinterpret_cast<float*>(reinterpret_cast<char*>(sm.kt) + tc::kmajor_off(f, s, DK)) =
-                load_f(sm.kq, tc::kmajor_off(s, f, 2 * C));
+            *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.kt) + tc::kmajor_off16(f, s, DK)) =
+                *reinterpret_cast<const uint16_t*>(reinterpret_cast<const char*>(sm.kq) + tc::kmajor_off16(s, f, 2 * C));
         }
     ok = __syncthreads_and(ok);
     nxt = sm.next_item;
@@ -335,8 +326,8 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         //   level 2: within each 32x32 diagonal block, X = -D2 (A21 D1).
         //   level 3: T21 = -T22 (A21 T11) for the lower-left 32x32 block.
         auto put_t = [&](int r, int c, float v) {
-            *reinterpret_cast<float*>(reinterpret_cast<char*>(sm.t) + tc::kmajor_off(r, c, C)) =
-                tc::round_tf32(v * sm.beta[c]);
+            *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.t) + tc::kmajor_off16(r, c, C)) =
+                (uint16_t)(tc::pack_f16(v * sm.beta[c], 0.f) & 0xffffu);
         };
         if (warp < 4) {
             if (lane < 16) {
@@ -359,37 +350,33 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             }
         } else {
             constexpr int NW = NT - 128;
-            for (int idx = tid - 128; idx < DK * C / 4; idx += NW) {
-                int f, s4;
-                tile_coord<DK>(idx, f, s4);
-                const uint32_t off = tc::kmajor_off(f, s4, DK);
-                const float4 k = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) + off);
-                store_f4(sm.kte, off,
-                         make_float4(tc::round_tf32(k.x * sm.eg[s4]), tc::round_tf32(k.y * sm.eg[s4 + 1]),
-                                     tc::round_tf32(k.z * sm.eg[s4 + 2]), tc::round_tf32(k.w * sm.eg[s4 + 3])));
-            }
-            for (int idx = tid - 128; idx < DK * C / 8; idx += NW) {  // the state pass's (diag(e^{gamma_n-gamma}) K)^T
+            // (diag(e^gamma) K)^T for W and the state pass's (diag(e^{gamma_n-gamma}) K)^T: column
+            // scalings of K^T, 8 columns s per 16-byte vector, same tile offsets in both
+            for (int idx = tid - 128; idx < DK * C / 8; idx += NW) {
                 int f, s8;
                 tile_coord8<DK>(idx, f, s8);
-                const float4 k0 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) +
-                                                                   tc::kmajor_off(f, s8, DK));
-                const float4 k1 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kt) +
-                                                                   tc::kmajor_off(f, s8 + 4, DK));
-                const float v[8] = {k0.x * sm.fkt[s8],     k0.y * sm.fkt[s8 + 1], k0.z * sm.fkt[s8 + 2],
-                                    k0.w * sm.fkt[s8 + 3], k1.x * sm.fkt[s8 + 4], k1.y * sm.fkt[s8 + 5],
-                                    k1.z * sm.fkt[s8 + 6], k1.w * sm.fkt[s8 + 7]};
-                store_h8(KTg, tc::kmajor_off16(f, s8, DK), v);
+                const uint32_t off = tc::kmajor_off16(f, s8, DK);
+                float k[8];
+                load_h8(sm.kt, off, k);
+                float ve[8], vk[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    ve[i] = k[i] * sm.eg[s8 + i];
+                    vk[i] = k[i] * sm.fkt[s8 + i];
+                }
+                store_h8(sm.kte, off, ve);
+                store_h8(KTg, off, vk);
             }
             for (int idx = tid - 128; idx < C * DK / 8; idx += NW) {  // rows Qg = diag(e^gamma) Q of [W ; Qg]
                 int r, k8;
                 tile_coord8<C>(idx, r, k8);
-                const float4 q0 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) +
-                                                                   tc::kmajor_off(C + r, k8, 2 * C));
-                const float4 q1 = *reinterpret_cast<const float4*>(reinterpret_cast<const char*>(sm.kq) +
-                                                                   tc::kmajor_off(C + r, k8 + 4, 2 * C));
+                const uint32_t off = tc::kmajor_off16(C + r, k8, 2 * C);  // same offsets in both tiles
+                float q[8];
+                load_h8(sm.kq, off, q);
                 const float e = sm.eg[r];
-                const float v[8] = {q0.x * e, q0.y * e, q0.z * e, q0.w * e, q1.x * e, q1.y * e, q1.z * e, q1.w * e};
-                store_h8(WQg, tc::kmajor_off16(C + r, k8, 2 * C), v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q[i] *= e;
+                store_h8(WQg, off, q);
             }
             if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[tid - 128];
         }
@@ -446,9 +433,9 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 for (int s = 0; s < 32; ++s)  // T21 = -T22 P
                     fma4(acc, sm.tf[32 + r][32 + s], *reinterpret_cast<const float4*>(&sm.m[s][c4]));
                 // the four columns are contiguous in the K-major tile
-                store_f4(sm.t, tc::kmajor_off(32 + r, c4, C),
-                         make_float4(tc::round_tf32(-acc.x * sm.beta[c4]), tc::round_tf32(-acc.y * sm.beta[c4 + 1]),
-                                     tc::round_tf32(-acc.z * sm.beta[c4 + 2]), tc::round_tf32(-acc.w * sm.beta[c4 + 3])));
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.t) + tc::kmajor_off16(32 + r, c4, C)) =
+                    make_uint2(tc::pack_f16(-acc.x * sm.beta[c4], -acc.y * sm.beta[c4 + 1]),
+                               tc::pack_f16(-acc.z * sm.beta[c4 + 2], -acc.w * sm.beta[c4 + 3]));
             }
         }
         tc::fence_smem_to_async();
@@ -460,13 +447,13 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             okm = tc::mbar_wait(bar_v, n_v & 1u);
             if (okm) {
                 const uint32_t bt = tc::smem_u32(sm.t), bkk = tc::smem_u32(sm.kte), bvv = tc::smem_u32(sm.bv);
-                constexpr uint32_t iw = tc::idesc_tf32(64, DK), iu = tc::idesc_tf32(DV, 64);
+                constexpr uint32_t iw = tc::idesc_f16(64, DK), iu = tc::idesc_f16(DV, 64);
 #pragma unroll
-                for (int s = 0; s < C / 8; ++s)
-                    tc::mma_tf32(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
+                for (int s = 0; s < C / 16; ++s)
+                    tc::mma_f16(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
 #pragma unroll
-                for (int s = 0; s < C / 8; ++s)
-                    tc::mma_tf32(tU, tc::desc_kmajor(bvv, DV, s), tc::desc_kmajor(bt, C, s), iu, s > 0);
+                for (int s = 0; s < C / 16; ++s)
+                    tc::mma_f16(tU, tc::desc_kmajor(bvv, DV, s), tc::desc_kmajor(bt, C, s), iu, s > 0);
                 tc::mma_commit(bar);
             }
         }

@@ -167,8 +167,8 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
 // are staged in shared memory; every output row is then conv1d + SiLU (+ L2
 // norm for q, k) of shared-memory data.  Results are assembled as tiles in the
 // tensor core's shared-memory layout and leave by bulk stores:
-//   q / k unit: rows C..2C-1 / 0..C-1 of [K ; Q*scale] (tf32, K-major, 128 rows x dk)
-//   v unit:     V^T tf32 (K-major, dv rows x C) and (g, beta) for the C rows
+//   q / k unit: rows C..2C-1 / 0..C-1 of [K ; Q*scale] (fp16, K-major, 128 rows x dk)
+//   v unit:     V^T fp16 (K-major, dv rows x C) and (g, beta) for the C rows
 // Rows past the end of a ragged chunk are written as zeros.
 constexpr int kPrepThreads = 256;
 
@@ -178,7 +178,7 @@ struct PrepShape {
     static constexpr int VE = 16 / sizeof(T);      // elements per 16-byte vector
     static constexpr int PAD = VE;                 // row padding: spreads rows over banks
     static constexpr size_t XS_BYTES = (((size_t)(C + 3) * (NCH + PAD) * sizeof(T)) + 15) & ~(size_t)15;
-    static constexpr size_t TILE_BYTES = (size_t)C * NCH * sizeof(float);
+    static constexpr size_t TILE_BYTES = (size_t)C * NCH * sizeof(uint16_t);  // fp16 tile
     static constexpr size_t W_BYTES = (size_t)NCH * 5 * sizeof(float);  // 4 taps per channel, then the biases
     static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + W_BYTES + C * sizeof(float2);
 };
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     const int c_first = isq ? hk * DK : isk ? d.HK * DK + hk * DK : 2 * d.HK * DK + h * DV;  // first channel
     extern __shared__ __align__(16) unsigned char smem_raw[];
     T* xs = reinterpret_cast<T*>(smem_raw);  // row i <-> token t0 - 3 + i
-    float* tile = reinterpret_cast<float*>(smem_raw + S::XS_BYTES);
+    char* tile = reinterpret_cast<char*>(smem_raw + S::XS_BYTES);
     float4* wsm = reinterpret_cast<float4*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);  // [nch] taps
     float* bsm = reinterpret_cast<float*>(wsm + S::NCH);                                // [nch] biases
     float2* gbs = reinterpret_cast<float2*>(smem_raw + S::XS_BYTES + S::TILE_BYTES + S::W_BYTES);
@@ -283,11 +283,10 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
         const float sc = (r < n) ? rsqrtf(ss + d.eps) * (isq ? d.scale : 1.f) : 0.f;
 #pragma unroll
         for (int cg = 0; cg < DK / 16; ++cg)
-            *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(r, 4 * (4 * cg + cc), C)) =
-                make_float4(tc::round_tf32(y[cg][0] * sc), tc::round_tf32(y[cg][1] * sc),
-                            tc::round_tf32(y[cg][2] * sc), tc::round_tf32(y[cg][3] * sc));
+            *reinterpret_cast<uint2*>(tile + tc::kmajor_off16(r, 4 * (4 * cg + cc), C)) =
+                make_uint2(tc::pack_f16(y[cg][0] * sc, y[cg][1] * sc), tc::pack_f16(y[cg][2] * sc, y[cg][3] * sc));
     } else {
-        // V^T tile: thread (f, 4 consecutive rows) -> one float4 of the K-major tile (8 lanes per core matrix)
+        // V^T tile: thread (f, 4 consecutive rows) -> 4 fp16 of the K-major tile (8 lanes per core matrix)
         for (int idx = tid; idx < DV * (C / 4); idx += kPrepThreads) {
             const int ff = idx & 7, cq = (idx >> 3) & 3, rest = idx >> 5;
             const int fg = rest % (DV / 8), rg = rest / (DV / 8);
@@ -305,10 +304,10 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
                 acc = fmaf(wc.y, xw[u + 1], acc);
                 acc = fmaf(wc.z, xw[u + 2], acc);
                 acc = fmaf(wc.w, xw[u + 3], acc);
-                y[u] = r4 + u < n ? tc::round_tf32(silu(acc)) : 0.f;
+                y[u] = r4 + u < n ? silu(acc) : 0.f;
             }
-            *reinterpret_cast<float4*>(reinterpret_cast<char*>(tile) + tc::kmajor_off(f, r4, DV)) =
-                make_float4(y[0], y[1], y[2], y[3]);
+            *reinterpret_cast<uint2*>(tile + tc::kmajor_off16(f, r4, DV)) =
+                make_uint2(tc::pack_f16(y[0], y[1]), tc::pack_f16(y[2], y[3]));
         }
         if (tid < C) {
             float2 gb = make_float2(0.f, 0.f);
@@ -325,12 +324,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
     __syncthreads();
     if (tid == 0) {
         if (!isv) {
-            // the 64-row half tile holds DK/4 blocks of 1 KB (one per column quad); in the 128-row
-            // [K ; Q] tile those blocks sit 2 KB apart, the q half 1 KB after the k half
+            // the 64-row half tile holds DK/8 blocks of 1 KB (one per group of 8 columns); in the
+            // 128-row [K ; Q] tile those blocks sit 2 KB apart, the q half 1 KB after the k half
             char* dst = reinterpret_cast<char*>(p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK)) + (isq ? 1024 : 0);
-            for (int q = 0; q < DK / 4; ++q) tc::bulk_s2g(dst + 2048 * q, tc::smem_u32(tile) + 1024 * q, 1024);
+            for (int q = 0; q < DK / 8; ++q) tc::bulk_s2g(dst + 2048 * q, tc::smem_u32(tile) + 1024 * q, 1024);
         } else {
-            tc::bulk_s2g(p.VT + ((size_t)id * d.HV + h) * (DV * C), tc::smem_u32(tile), DV * C * 4);
+            tc::bulk_s2g(p.VT + ((size_t)id * d.HV + h) * (DV * C), tc::smem_u32(tile), DV * C * 2);
             tc::bulk_s2g(p.GB + ((size_t)id * d.HV + h) * C, tc::smem_u32(gbs), C * 8);
         }
         tc::bulk_commit();
@@ -467,8 +466,8 @@ size_t walk_extend_workspace(const LayerDims& d, int max_N, int max_T, char* bas
     char* seq_order = take((size_t)max_N * sizeof(int32_t));
     char* rank_off = take(((size_t)max_N + 1) * sizeof(int32_t));
     char* chunk_list = take(mc * sizeof(int32_t));
-    char* kq = take(mc * d.HK * 2 * C * d.dk * sizeof(float));
-    char* vt = take(units * d.dv * C * sizeof(float));
+    char* kq = take(mc * d.HK * 2 * C * d.dk * sizeof(uint16_t));
+    char* vt = take(units * d.dv * C * sizeof(uint16_t));
     char* gb = take(units * C * sizeof(float2));
     char* wq = take(units * 2 * C * d.dk * sizeof(uint16_t));
     char* aq = take(units * C * C * sizeof(uint16_t));
@@ -483,8 +482,8 @@ size_t walk_extend_workspace(const LayerDims& d, int max_N, int max_T, char* bas
         e->seq_order = reinterpret_cast<int32_t*>(seq_order);
         e->rank_off = reinterpret_cast<int32_t*>(rank_off);
         e->chunk_list = reinterpret_cast<int32_t*>(chunk_list);
-        e->KQ = reinterpret_cast<float*>(kq);
-        e->VT = reinterpret_cast<float*>(vt);
+        e->KQ = reinterpret_cast<uint16_t*>(kq);
+        e->VT = reinterpret_cast<uint16_t*>(vt);
         e->GB = reinterpret_cast<float2*>(gb);
         e->WQ = reinterpret_cast<uint16_t*>(wq);
         e->AQ = reinterpret_cast<uint16_t*>(aq);

@@ -165,8 +165,8 @@ GDN_API int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, cons
  * no allocating library routine.
  *   - Sizes whose gdn_extend_workspace_size(cfg, N, T) exceeds
  *     GDN_EXTEND_STATIC_SCRATCH_BYTES are rejected with GDN_ERR_WORKSPACE and
- *     nothing is launched (one sequence of up to 831 tokens for the
- *     16/32-head, dk = dv = 128 layer; 7103 for the 4/8-head, 64 layer).
+ *     nothing is launched (one sequence of up to 1151 tokens for the
+ *     16/32-head, dk = dv = 128 layer; 9151 for the 4/8-head, 64 layer).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and keeps it, and,
  *     like gdn_extend, creates the library's second stream and its two

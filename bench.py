@@ -37,8 +37,8 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-# nominal dense tf32 / bf16 tensor throughput ratio of B200 (1.1 vs 2.25 PFLOP/s)
-TF32_PER_BF16 = 1.1 / 2.25
+# The prefill's tensor-core products are kind::f16 MMAs (fp16 operands, fp32 accumulation): their
+# peak is the dense fp16 rate, which equals the bf16 rate the peaks file measures.
 C = 64
 
 
@@ -438,11 +438,11 @@ def main():
     st_ver, by_ver = verify_bytes(dspec, Bn, D)
     value = world * pre.T / (ext_ms * 1e-3)
 
-    tf32 = bf16 * TF32_PER_BF16
-    tf32_src = f"{peak_src} bf16 burst {bf16:.1f} TFLOP/s x nominal tf32/bf16 ratio 1.1/2.25"
+    f16 = bf16
+    f16_src = f"{peak_src} bf16 burst {bf16:.1f} TFLOP/s (fp16 and bf16 share the dense tensor rate)"
     kernels = {
-        "state": {"bound": "tensor", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": tf32, "peak_src": tf32_src},
-        "intra": {"bound": "tensor", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": tf32, "peak_src": tf32_src},
+        "state": {"bound": "tensor", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": f16, "peak_src": f16_src},
+        "intra": {"bound": "tensor", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": f16, "peak_src": f16_src},
         "prep": {"bound": "hbm", "work": pre.T * (spec.conv_dim * 2 + 2 * spec.HV * 2), "unit": "GB/s",
                  "peak": hbm, "peak_src": peak_src},
         "decode": {"bound": "hbm", "work": by_dec, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
@@ -459,11 +459,11 @@ def main():
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
                 "unit": dk["unit"], "frac": dk["frac"], "traffic": ncu_traffic(dom),
                 "peak_source": dk["peak_src"] + (" (of measured)" if peak_src == "measured" else " (of fallback)")}
-    # the whole prefill against its own roofline: max(algorithmic FLOPs at the tf32 peak,
+    # the whole prefill against its own roofline: max(algorithmic FLOPs at the fp16 tensor peak,
     # algorithmic bytes at the HBM peak)
-    t_floor = max(pw["flops"] / (tf32 * 1e12), pw["bytes"] / (hbm * 1e9))
-    prefill_roofline = {"floor_ms": t_floor * 1e3, "bound": "tensor" if pw["flops"] / (tf32 * 1e12) >= pw["bytes"] / (hbm * 1e9) else "hbm",
-                        "frac": t_floor / (ext_ms * 1e-3), "tensor_frac": pw["flops"] / (ext_ms * 1e-3) / (tf32 * 1e12),
+    t_floor = max(pw["flops"] / (f16 * 1e12), pw["bytes"] / (hbm * 1e9))
+    prefill_roofline = {"floor_ms": t_floor * 1e3, "bound": "tensor" if pw["flops"] / (f16 * 1e12) >= pw["bytes"] / (hbm * 1e9) else "hbm",
+                        "frac": t_floor / (ext_ms * 1e-3), "tensor_frac": pw["flops"] / (ext_ms * 1e-3) / (f16 * 1e12),
                         "hbm_frac": pw["bytes"] / (ext_ms * 1e-3) / (hbm * 1e9)}
 
     # End to end through the public API with pinned host buffers.  The layer is independent per
@@ -540,7 +540,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "tf32/f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f16/f32", "data": "synthetic",
             "config": workload_config(pre, args),
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,

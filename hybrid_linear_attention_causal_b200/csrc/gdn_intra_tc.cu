@@ -381,11 +381,10 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[tid - 128];
         }
         __syncthreads();
-        // Levels 2 and 3 tile the outputs in registers: a thread takes four consecutive columns of
-        // one row, so each step of a dot product is one (broadcast) load of the left factor and one
-        // 16-byte load of the right one for four FMAs; the shared-memory pipe, not the FMAs, bounds
-        // these small products.
-        static_assert(NT >= 256, "level 3 takes 256 threads");
+        // Level 2 tiles the outputs in registers: a thread takes four consecutive columns of one row,
+        // so each step of a dot product is one (broadcast) load of the left factor and one 16-byte
+        // load of the right one for four FMAs; the shared-memory pipe, not the FMAs, bounds these
+        // small products.
         auto fma4 = [](float4& acc, float a, const float4& b) {
             acc.x = fmaf(a, b.x, acc.x);
             acc.y = fmaf(a, b.y, acc.y);
@@ -417,26 +416,30 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             }
         }
         __syncthreads();
-        {  // level 3 (threads 0..255): row r, columns c4 .. c4 + 3
-            const int r = tid >> 3, c4 = 4 * (tid & 7);
-            if (tid < 256) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                for (int s = 0; s < 32; ++s)  // P = A21 T11
-                    fma4(acc, sm.a[32 + r][s], *reinterpret_cast<const float4*>(&sm.tf[s][c4]));
-                *reinterpret_cast<float4*>(&sm.m[r][c4]) = acc;
+        // Level 3 reads one operand as a warp-wide broadcast and skips the zero blocks of the
+        // triangular factors: T11[s][c] = 0 for s < c and T22[r][s] = 0 for s > r.
+        static_assert(NT == 512, "level 3 maps 8 column groups, then 16 row pairs, onto the warps");
+        if (warp < 8) {  // level 3a: P = A21 T11; warp w takes columns 4w .. 4w + 3, lane = row
+            const int r = lane, c4 = 4 * warp;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int s = c4; s < 32; ++s)
+                fma4(acc, sm.a[32 + r][s], *reinterpret_cast<const float4*>(&sm.tf[s][c4]));
+            *reinterpret_cast<float4*>(&sm.m[r][c4]) = acc;
+        }
+        __syncthreads();
+        {  // level 3b: T21 = -T22 P; warp w takes rows 2w, 2w + 1 of the block, lane = column
+            const int r0 = 2 * warp, c = lane;
+            float acc0 = 0.f, acc1 = 0.f;
+            for (int s4 = 0; s4 < r0 + 2; s4 += 4) {
+                const float4 t0 = *reinterpret_cast<const float4*>(&sm.tf[32 + r0][32 + s4]);
+                const float4 t1 = *reinterpret_cast<const float4*>(&sm.tf[33 + r0][32 + s4]);
+                const float p0 = sm.m[s4][c], p1 = sm.m[s4 + 1][c], p2 = sm.m[s4 + 2][c], p3 = sm.m[s4 + 3][c];
+                acc0 = fmaf(t0.x, p0, fmaf(t0.y, p1, fmaf(t0.z, p2, fmaf(t0.w, p3, acc0))));
+                acc1 = fmaf(t1.x, p0, fmaf(t1.y, p1, fmaf(t1.z, p2, fmaf(t1.w, p3, acc1))));
             }
-            __syncthreads();
-            if (tid < 256) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-                for (int s = 0; s < 32; ++s)  // T21 = -T22 P
-                    fma4(acc, sm.tf[32 + r][32 + s], *reinterpret_cast<const float4*>(&sm.m[s][c4]));
-                // the four columns are contiguous in the K-major tile
-                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.t) + tc::kmajor_off16(32 + r, c4, C)) =
-                    make_uint2(tc::pack_f16(-acc.x * sm.beta[c4], -acc.y * sm.beta[c4 + 1]),
-                               tc::pack_f16(-acc.z * sm.beta[c4 + 2], -acc.w * sm.beta[c4 + 3]));
-            }
+            put_t(32 + r0, c, -acc0);
+            put_t(33 + r0, c, -acc1);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();

@@ -38,6 +38,7 @@ constexpr int C = kChunk;
 constexpr int NT = 512;        // 16 warps; warp w reads TMEM sub-partition w % 4
 constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
 constexpr int kItemsPerCta = 4;
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
 template <int DK, int DV>
 struct IntraTcSmem {
@@ -53,6 +54,7 @@ struct IntraTcSmem {
     float y[2][16][20];    // A21 D1 inside each 32x32 diagonal block (rows 16-byte aligned)
     float2 gb[2][C];       // (g, beta) of the two heads in flight
     float gam[C], beta[C], eg[C];
+    float gam2[C];         // gamma * log2(e): the exponents of the decay factors in base 2
     float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
     unsigned long long bar_mma, bar_kq, bar_v, bar_g[2];
     uint32_t tmem_base;
@@ -254,6 +256,8 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             const float gA = incl - pair + g0.x;
             sm.gam[2 * lane] = gA;
             sm.gam[2 * lane + 1] = incl;
+            sm.gam2[2 * lane] = gA * kLog2e;
+            sm.gam2[2 * lane + 1] = incl * kLog2e;
             sm.beta[2 * lane] = g0.y;
             sm.beta[2 * lane + 1] = g1.y;
             sm.eg[2 * lane] = __expf(gA);
@@ -280,36 +284,44 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         }
         const float gl = sm.gam[n - 1];
         {  // A (sub-partitions 0-1: k.k rows) and the masked decayed q.k tile (2-3: q.k rows) from D1;
-           // the warps of a sub-partition take one group of C / NCG columns each
+           // the warps of a sub-partition take one group of C / NCG columns each.  The exponents are
+           // formed without branches (a masked entry gets -inf, whose exponential is 0) so the
+           // sixteen exponentials of a thread issue back to back; a warp whose whole block lies
+           // above the diagonal only writes zeros.
             constexpr int NC = C / NCG;
+            static_assert(NC == 16, "one 16-column load per warp");
             const int r = (sp & 1) * 32 + lane, c0 = NC * cg;
-            float row[NC];
+            const bool qrow = sp >= 2;
+            const bool live = c0 <= (sp & 1) * 32 + 31;  // warp-uniform
+            float v[NC], e[NC];
+            if (live) {
+                tc::tmem_ld16(tD1 + lane_base + c0, v);
+                tc::tmem_ld_wait();
+                // entry i is kept when column c0 + i lies below the diagonal (on it, for q.k) of a row
+                // inside the chunk
+                const int lim = r < n ? r - c0 + (qrow ? 1 : 0) : 0;
+                const float gr = sm.gam2[r];
 #pragma unroll
-            for (int c = 0; c < NC; c += 16) {
-                float v[16];
-                tc::tmem_ld16(tD1 + lane_base + c0 + c, v);
+                for (int q = 0; q < NC; q += 4) {
+                    const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[c0 + q]);
+                    const float gq[4] = {gs.x, gs.y, gs.z, gs.w};
 #pragma unroll
-                for (int i = 0; i < 16; ++i) row[c + i] = v[i];
-            }
-            tc::tmem_ld_wait();
-            const float gr = sm.gam[r], br = sm.beta[r];
-            if (sp < 2) {
-#pragma unroll
-                for (int i = 0; i < NC; ++i) {
-                    const int s = c0 + i;
-                    sm.a[r][s] = (s < r && r < n) ? br * __expf(gr - sm.gam[s]) * row[i] : 0.f;
+                    for (int u = 0; u < 4; ++u)
+                        e[q + u] = q + u < lim ? gr - gq[u] : __int_as_float(0xff800000u);  // -inf
                 }
+#pragma unroll
+                for (int i = 0; i < NC; ++i) e[i] = tc::ex2_approx(e[i]) * v[i];
             } else {
 #pragma unroll
-                for (int i = 0; i < NC; i += 8) {
-                    float o[8];
+                for (int i = 0; i < NC; ++i) e[i] = 0.f;
+            }
+            if (!qrow) {
+                const float br = sm.beta[r];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int s = c0 + i + u;
-                        o[u] = (s <= r && r < n) ? __expf(gr - sm.gam[s]) * row[i + u] : 0.f;
-                    }
-                    store_h8(AQg, tc::kmajor_off16(r, c0 + i, C), o);
-                }
+                for (int i = 0; i < NC; ++i) sm.a[r][c0 + i] = br * e[i];
+            } else {
+                store_h8(AQg, tc::kmajor_off16(r, c0, C), e);
+                store_h8(AQg, tc::kmajor_off16(r, c0 + 8, C), e + 8);
             }
         }
         if (j > 0) epilogue(j - 1);  // the previous head's W and U^T, from other tensor-memory columns

@@ -95,6 +95,14 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         : "memory");
 }
 
+// 2^x with the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32): one
+// instruction; 2^-inf = +0 and results below the normal range flush to zero
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // two floats -> one 32-bit word of two fp16 (round to nearest even), low half first
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     uint32_t r;

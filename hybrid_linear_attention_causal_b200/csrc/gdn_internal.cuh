@@ -121,7 +121,7 @@ struct ExtendArgs {
     // shared-memory layout, so the state pass copies them verbatim
     uint16_t* WQ;       // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], fp16, K-major, 128 rows
     uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, fp16, K-major, C rows
-    uint16_t* KT;       // [max_chunks, HV, dk*C]    (diag(e^{gamma_n-gamma}) K)^T, fp16, K-major, dk rows
+    uint16_t* KT;       // [max_chunks, HV, C*dk]    K~ = diag(e^{gamma_n-gamma}) K, fp16, tile of C rows s
     uint16_t* U;        // [max_chunks, HV, dv*C]    U^T, fp16, K-major tile of dv rows (j) x C
     float* gam;         // [max_chunks, HV, C]       in-chunk cumulative g
 };

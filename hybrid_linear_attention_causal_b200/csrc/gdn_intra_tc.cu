@@ -1,32 +1,27 @@
 // Intra-chunk step of the chunked GDN prefill on tcgen05 tensor cores (sm_100a).
 //
-// One CTA per (chunk, qk head); it serves the G value heads that share the qk
-// head.  For a chunk of n <= 64 rows with normalised k_r, q_r (q carries the
-// output scale), gates g_r, beta_r and gamma_r = sum_{s<=r} g_s:
+// One (chunk, qk head) item at a time; an item serves the G value heads that
+// share the qk head.  For a chunk of n <= 64 rows with normalised k_r, q_r (q
+// carries the output scale), gates g_r, beta_r and gamma_r = sum_{s<=r} g_s:
 //
-// The prep kernel's [K ; Q] tile and the V^T tiles and gates of the value
-// heads arrive by asynchronous bulk copies (two value heads in flight).
-//
-//   D1  = [K; Q] K^T                          (tf32 MMA, M=128 N=64 K=dk)
+//   D1  = [K; Q] K^T                          (fp16 MMA, M=128 N=64 K=dk)
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
 //   T   = (I + A)^{-1}                        (fp32: 16x16 forward substitution + block products)
-//   W   = T diag(beta e^gamma) K, U = T diag(beta) V   (tf32 MMAs, K=64; U formed
-//                                                       transposed, U^T = V^T (T diag(beta))^T)
+//   W   = T diag(beta e^gamma) K              (fp16 MMA, M=64 N=dk K=64; K read MN-major
+//                                              straight from the [K ; Q] tile)
+//   U^T = V^T (T diag(beta))^T                (fp16 MMA, M=dv N=64 K=64)
 //
-// Both products share the A operand T diag(beta): W takes (diag(e^gamma) K)^T
-// and U the V^T tile as delivered.  K^T is transposed once per CTA from the
-// [K ; Q] tile and serves every value head through column scalings.
-//
-// (the WY/UT form of the gated delta rule).  For the serial state pass it
-// writes, per (chunk, value head): the tile [W ; diag(e^gamma) Q], the Aqk
-// tile and the tile (diag(e^{gamma_n-gamma}) K)^T -- tf32, already in the
-// tensor core's shared-memory layout so the state pass bulk-copies them --
-// plus U (fp32) and gamma.  Operands are staged in shared memory as K-major
-// no-swizzle tiles rounded to tf32 (round to nearest); accumulators live in
-// tensor memory.  One thread issues the MMAs; the sixteen warps read their
-// sub-partition's 32-lane slice of tensor memory (four warps per slice, one
-// group of columns each) for the CUDA-core steps.
+// (the WY/UT form of the gated delta rule).  The prep kernel's [K ; Q] tile and
+// the V^T tiles and gates of the value heads arrive by asynchronous bulk copies.
+// For the serial state pass it writes, per (chunk, value head), fp16 tiles in
+// the tensor core's shared-memory layout, so the state pass bulk-copies them:
+// [W ; diag(e^gamma) Q], Aqk, K~ = diag(e^{gamma_n-gamma}) K (rows s; read
+// MN-major) and U^T; plus gamma.  Operands are staged in shared memory as
+// no-swizzle tiles rounded to fp16; accumulators live in tensor memory.  One
+// thread issues the MMAs; the sixteen warps read their sub-partition's 32-lane
+// slice of tensor memory (four warps per slice, one group of columns each) for
+// the CUDA-core steps.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -43,19 +38,22 @@ constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 template <int DK, int DV>
 struct IntraTcSmem {
     // fp16 operand tiles (16-bit K-major layout)
-    uint16_t kq[2 * C * DK];  // [K ; Q*scale] tile from the prep kernel (bulk copy), 128 rows
-    uint16_t kt[DK * C];      // K^T, DK rows x C (built once, shared by the value heads)
-    uint16_t kte[DK * C];     // (diag(e^gamma) K)^T of the current head, same layout
+    uint16_t kq[2 * C * DK];  // [K ; Q*scale] tile from the prep kernel (bulk copy), 128 rows; its
+                              // K rows are also W's B operand, read MN-major
     uint16_t bv[DV * C];      // V^T tile of the current head (bulk copy), DV rows x C
-    uint16_t t[C * C];        // T diag(beta), C rows x C
+    uint16_t t[C * C];        // T diag(beta), C rows x C: U's operand
+    uint16_t te[C * C];       // T diag(beta e^gamma), same layout: W's operand
     float a[C][C + 1];     // A (fp32)
     float tf[C][C + 4];    // T (fp32), the blocks the next level of the inverse reads
     float m[32][36];       // A21 T11
     float y[2][16][20];    // A21 D1 inside each 32x32 diagonal block (rows 16-byte aligned)
     float2 gb[2][C];       // (g, beta) of the two heads in flight
-    float gam[C], beta[C], eg[C];
-    float gam2[C];         // gamma * log2(e): the exponents of the decay factors in base 2
-    float fkt[C];          // e^{gamma_n - gamma_s} (0 past the chunk end): column factor of K~^T
+    // per-row gate quantities of a value head, double-buffered by head parity: the tiles that need
+    // only head j's gates are written while head j + 1's gates are scanned
+    float gam[2][C], beta[2][C], eg[2][C];
+    float gam2[2][C];      // gamma * log2(e): the exponents of the decay factors in base 2
+    float bge[2][C];       // beta e^gamma: the column factor of W's operand
+    float fkt[2][C];       // e^{gamma_n - gamma_s} (0 past the chunk end): row factor of K~
     unsigned long long bar_mma, bar_kq, bar_v, bar_g[2];
     uint32_t tmem_base;
     int next_item;         // thread 0's latest grab, for the other threads
@@ -153,7 +151,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     }
     // blocks of T above the diagonal are zero for every head: in the tile, and in the two 16x16
     // corners of the 32x32 diagonal blocks that the inverse reads back
-    for (int e = tid; e < C * C; e += NT) sm.t[e] = 0;
+    for (int e = tid; e < C * C; e += NT) sm.t[e] = sm.te[e] = 0;
     for (int e = tid; e < 2 * 256; e += NT) {
         const int o = 32 * (e >> 8);
         sm.tf[o + ((e >> 4) & 15)][o + 16 + (e & 15)] = 0.f;
@@ -175,7 +173,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     // At most kItemsPerCta items, then the CTA ends: its SM goes to whatever waits, first of all a
     // state-pass CTA of the previous segment (its stream has the higher priority).
     if (tid == 0 && ++done < kItemsPerCta) nxt = grab();
-    if (tid == 0) sm.next_item = nxt;  // read by every thread after the K^T barrier below
+    if (tid == 0) sm.next_item = nxt;  // read by every thread after the barrier below
     const int id = item / HK, hk = item % HK;
     const int n = p.chunk_tab[id].z;
     if (tid == 0 && nxt >= 0) prefetch_l2(nxt);
@@ -190,16 +188,9 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             tc::mma_commit(bar);
         }
     }
-    // K^T (feature rows) from the k rows of the [K ; Q] tile, once for all value heads.  A warp reads
-    // 8 rows s x 4 features f of one 128-byte core matrix of the tile.
+    // every thread reads the [K ; Q] tile below
     ok = ok && tc::mbar_wait(bar_kq, n_kq & 1u);
     ++n_kq;
-    if (ok)
-        for (int idx = tid; idx < DK * C; idx += NT) {
-            const int s = (idx & 7) + 8 * ((idx >> 5) & 7), f = ((idx >> 3) & 3) + 4 * (idx >> 8);
-            *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.kt) + tc::kmajor_off16(f, s, DK)) =
-                *reinterpret_cast<const uint16_t*>(reinterpret_cast<const char*>(sm.kq) + tc::kmajor_off16(s, f, 2 * C));
-        }
     ok = __syncthreads_and(ok);
     nxt = sm.next_item;
 
@@ -254,22 +245,24 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 if (lane >= o) incl += v;
             }
             const float gA = incl - pair + g0.x;
-            sm.gam[2 * lane] = gA;
-            sm.gam[2 * lane + 1] = incl;
-            sm.gam2[2 * lane] = gA * kLog2e;
-            sm.gam2[2 * lane + 1] = incl * kLog2e;
-            sm.beta[2 * lane] = g0.y;
-            sm.beta[2 * lane + 1] = g1.y;
-            sm.eg[2 * lane] = __expf(gA);
-            sm.eg[2 * lane + 1] = __expf(incl);
+            sm.gam[bb][2 * lane] = gA;
+            sm.gam[bb][2 * lane + 1] = incl;
+            sm.gam2[bb][2 * lane] = gA * kLog2e;
+            sm.gam2[bb][2 * lane + 1] = incl * kLog2e;
+            sm.beta[bb][2 * lane] = g0.y;
+            sm.beta[bb][2 * lane + 1] = g1.y;
+            sm.eg[bb][2 * lane] = __expf(gA);
+            sm.eg[bb][2 * lane + 1] = __expf(incl);
+            sm.bge[bb][2 * lane] = g0.y * sm.eg[bb][2 * lane];
+            sm.bge[bb][2 * lane + 1] = g1.y * sm.eg[bb][2 * lane + 1];
             const float gn = __shfl_sync(0xffffffffu, (n - 1) & 1 ? incl : gA, (n - 1) >> 1);
-            sm.fkt[2 * lane] = 2 * lane < n ? __expf(gn - gA) : 0.f;
-            sm.fkt[2 * lane + 1] = 2 * lane + 1 < n ? __expf(gn - incl) : 0.f;
+            sm.fkt[bb][2 * lane] = 2 * lane < n ? __expf(gn - gA) : 0.f;
+            sm.fkt[bb][2 * lane + 1] = 2 * lane + 1 < n ? __expf(gn - incl) : 0.f;
         }
         return okg;
     };
     for (int j = 0; j < G && ok; ++j) {
-        const int h = hk * G + j;
+        const int h = hk * G + j, hb = j & 1;
         const size_t ch_h = (size_t)id * HV + h;
         char* WQg = reinterpret_cast<char*>(p.WQ + ch_h * (2 * C * DK));
         char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
@@ -282,7 +275,6 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             if (!ok) break;
             tc::fence_after_sync();
         }
-        const float gl = sm.gam[n - 1];
         {  // A (sub-partitions 0-1: k.k rows) and the masked decayed q.k tile (2-3: q.k rows) from D1;
            // the warps of a sub-partition take one group of C / NCG columns each.  The exponents are
            // formed without branches (a masked entry gets -inf, whose exponential is 0) so the
@@ -300,10 +292,10 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 // entry i is kept when column c0 + i lies below the diagonal (on it, for q.k) of a row
                 // inside the chunk
                 const int lim = r < n ? r - c0 + (qrow ? 1 : 0) : 0;
-                const float gr = sm.gam2[r];
+                const float gr = sm.gam2[hb][r];
 #pragma unroll
                 for (int q = 0; q < NC; q += 4) {
-                    const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[c0 + q]);
+                    const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[hb][c0 + q]);
                     const float gq[4] = {gs.x, gs.y, gs.z, gs.w};
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
@@ -316,7 +308,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 for (int i = 0; i < NC; ++i) e[i] = 0.f;
             }
             if (!qrow) {
-                const float br = sm.beta[r];
+                const float br = sm.beta[hb][r];
 #pragma unroll
                 for (int i = 0; i < NC; ++i) sm.a[r][c0 + i] = br * e[i];
             } else {
@@ -328,18 +320,20 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        // T = (I + A)^{-1}, by blocks.  Every final entry goes straight into the K-major tf32 tile of
+        // T = (I + A)^{-1}, by blocks.  Every final entry goes straight into the K-major fp16 tile of
         // T diag(beta) (the A operand of W and U); the fp32 copy tf holds what the next level reads.
         //   level 1: the four diagonal 16x16 blocks by forward substitution, one column per lane held
         //            in registers (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so
-        //            one FMA per row sits on the dependent chain); warps 4-15 meanwhile build
-        //            (diag(e^gamma) K)^T for W and write the tiles that need only the gates (the
-        //            state pass's (diag(e^{gamma_n-gamma}) K)^T, the rows Qg = diag(e^gamma) Q).
+        //            one FMA per row sits on the dependent chain); warps 4-15 meanwhile write the
+        //            tiles that need only the gates: the state pass's K~ = diag(e^{gamma_n-gamma}) K
+        //            and the rows Qg = diag(e^gamma) Q of [W ; Qg], and gamma.
         //   level 2: within each 32x32 diagonal block, X = -D2 (A21 D1).
         //   level 3: T21 = -T22 (A21 T11) for the lower-left 32x32 block.
-        auto put_t = [&](int r, int c, float v) {
-            *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.t) + tc::kmajor_off16(r, c, C)) =
-                (uint16_t)(tc::pack_f16(v * sm.beta[c], 0.f) & 0xffffu);
+        auto put_t = [&](int r, int c, float v) {  // T entry (r, c) into both operand tiles
+            const uint32_t off = tc::kmajor_off16(r, c, C);
+            const uint32_t w = tc::pack_f16(v * sm.beta[hb][c], v * sm.bge[hb][c]);
+            *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.t) + off) = (uint16_t)(w & 0xffffu);
+            *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.te) + off) = (uint16_t)(w >> 16);
         };
         if (warp < 4) {
             if (lane < 16) {
@@ -360,37 +354,23 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                     put_t(o + r, o + c, t[r]);
                 }
             }
-        } else {
+        } else {  // row scalings of the [K ; Q] tile, 8 features per 16-byte vector
             constexpr int NW = NT - 128;
-            // (diag(e^gamma) K)^T for W and the state pass's (diag(e^{gamma_n-gamma}) K)^T: column
-            // scalings of K^T, 8 columns s per 16-byte vector, same tile offsets in both
-            for (int idx = tid - 128; idx < DK * C / 8; idx += NW) {
-                int f, s8;
-                tile_coord8<DK>(idx, f, s8);
-                const uint32_t off = tc::kmajor_off16(f, s8, DK);
-                float k[8];
-                load_h8(sm.kt, off, k);
-                float ve[8], vk[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    ve[i] = k[i] * sm.eg[s8 + i];
-                    vk[i] = k[i] * sm.fkt[s8 + i];
-                }
-                store_h8(sm.kte, off, ve);
-                store_h8(KTg, off, vk);
-            }
-            for (int idx = tid - 128; idx < C * DK / 8; idx += NW) {  // rows Qg = diag(e^gamma) Q of [W ; Qg]
+            for (int idx = tid - 128; idx < 2 * C * DK / 8; idx += NW) {
                 int r, k8;
-                tile_coord8<C>(idx, r, k8);
-                const uint32_t off = tc::kmajor_off16(C + r, k8, 2 * C);  // same offsets in both tiles
-                float q[8];
-                load_h8(sm.kq, off, q);
-                const float e = sm.eg[r];
+                tile_coord8<2 * C>(idx, r, k8);  // a warp's 32 rows lie in one half of the tile
+                const uint32_t off = tc::kmajor_off16(r, k8, 2 * C);
+                float v[8];
+                load_h8(sm.kq, off, v);
+                const float e = r < C ? sm.fkt[hb][r] : sm.eg[hb][r - C];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] *= e;
-                store_h8(WQg, off, q);
+                for (int i = 0; i < 8; ++i) v[i] *= e;
+                if (r < C)
+                    store_h8(KTg, tc::kmajor_off16(r, k8, C), v);  // K~: a tile of C rows s
+                else
+                    store_h8(WQg, off, v);  // rows Qg: same offsets in [W ; Qg]
             }
-            if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[tid - 128];
+            if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[hb][tid - 128];
         }
         __syncthreads();
         // Level 2 tiles the outputs in registers: a thread takes four consecutive columns of one row,
@@ -458,14 +438,16 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         __syncthreads();
         tc::fence_after_sync();
         bool okm = true;
-        if (tid == 0) {  // W = (T diag(beta)) (diag(e^gamma) K) (M = 64), U^T = V^T (T diag(beta))^T (M = DV)
+        if (tid == 0) {  // W = (T diag(beta e^gamma)) K (M = 64, K read MN-major from the [K ; Q] tile),
+                         // U^T = V^T (T diag(beta))^T (M = DV)
             okm = tc::mbar_wait(bar_v, n_v & 1u);
             if (okm) {
-                const uint32_t bt = tc::smem_u32(sm.t), bkk = tc::smem_u32(sm.kte), bvv = tc::smem_u32(sm.bv);
-                constexpr uint32_t iw = tc::idesc_f16(64, DK), iu = tc::idesc_f16(DV, 64);
+                const uint32_t bt = tc::smem_u32(sm.t), bte = tc::smem_u32(sm.te), bkq = tc::smem_u32(sm.kq);
+                const uint32_t bvv = tc::smem_u32(sm.bv);
+                constexpr uint32_t iw = tc::idesc_f16(64, DK) | tc::kTransposeB, iu = tc::idesc_f16(DV, 64);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    tc::mma_f16(tW, tc::desc_kmajor(bt, C, s), tc::desc_kmajor(bkk, DK, s), iw, s > 0);
+                    tc::mma_f16(tW, tc::desc_kmajor(bte, C, s), tc::desc_mnmajor16(bkq, 2 * C, s), iw, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
                     tc::mma_f16(tU, tc::desc_kmajor(bvv, DV, s), tc::desc_kmajor(bt, C, s), iu, s > 0);
@@ -473,7 +455,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
             }
         }
         bool okn = true;
-        if (warp == 0 && j + 1 < G) okn = scan_gates(j + 1);  // head j's gate arrays are no longer read
+        if (warp == 0 && j + 1 < G) okn = scan_gates(j + 1);  // into the other gate buffer
         ++n_v;
         ok = okm && okn && tc::mbar_wait(bar, ph_mma);  // okm is false only on tid 0, if the V tile never came
         ph_mma ^= 1;

@@ -3,8 +3,8 @@
 //
 // One CTA per (sequence, value head), looping over the sequence's chunks.  The
 // products are formed transposed, with the value dimension (dv) as the MMA's
-// M, so that every shared-memory operand is K-major and every accumulator row
-// belongs to one thread:
+// M, so that every accumulator row belongs to one thread; K~ is read MN-major
+// (its rows s run along the product's K), every other operand K-major:
 //
 //   [X^T | O^T]  = S^T [W ; Qg]^T           M=dv N=128 K=dk   (X = W S, O = Qg S)
 //   V'^T         = U^T - X^T                 CUDA cores, per thread row j
@@ -23,7 +23,7 @@
 //     is one FMA per element, written straight into the fp16 operand copy;
 //   - [X^T | O^T] is double-buffered in tensor memory: a chunk's outputs are
 //     read and stored while the next chunk's first product runs;
-//   - the tiles [W ; Qg], K~^T and Aqk (written by the intra-chunk kernel as
+//   - the tiles [W ; Qg], K~ and Aqk (written by the intra-chunk kernel as
 //     fp16 in the tensor core's layout) each have their own barrier and are
 //     refetched as soon as the product that reads them completes;
 //   - the intra-chunk kernel writes U^T in the layout of the V'^T operand
@@ -55,7 +55,7 @@ struct StateTcSmem {
     uint16_t st[DV * DK];     // S^T tile: DV rows x DK (fp16 copy of the state)
     uint16_t wq[2 * C * DK];  // [W ; Qg] tile (bulk copy): 128 rows x DK
     uint16_t aq[C * C];       // Aqk tile (bulk copy): C rows (r) x C (s)
-    uint16_t kt[DK * C];      // K~^T tile (bulk copy): DK rows (i) x C (s)
+    uint16_t kt[C * DK];      // K~ tile (bulk copy): C rows (s) x DK (i), the MN-major B of Snew^T
     uint16_t vt[DV * C];      // U^T tile (bulk copy), overwritten in place by V'^T: DV rows (j) x C (s)
     T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
     unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq, bar_u;
@@ -264,16 +264,16 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         tc::fence_after_sync();
         if (tid == ISSUER) {
             okl = tc::mbar_wait(bar_kt, ph);
-            if (okl) {  // Snew^T = V'^T K~
+            if (okl) {  // Snew^T = V'^T K~, K~ (rows s) read MN-major
                 const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt);
-                constexpr uint32_t is = tc::idesc_f16(DV, DK);
+                constexpr uint32_t is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    tc::mma_f16(tS, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bk, DK, k), is, k > 0);
+                    tc::mma_f16(tS, tc::desc_kmajor(av, DV, k), tc::desc_mnmajor16(bk, C, k), is, k > 0);
                 tc::mma_commit(bar_s);
                 okl = tc::mbar_wait(bar_s, ph);
             }
-            if (okl && id + 1 < c_end) fetch_kt(id + 1);  // the K~^T tile is free again
+            if (okl && id + 1 < c_end) fetch_kt(id + 1);  // the K~ tile is free again
             if (okl) okl = tc::mbar_wait(bar_aq, ph);
             if (okl) {  // O^T += V'^T Aqk^T, off the state chain
                 const uint32_t av = tc::smem_u32(sm.vt), bq = tc::smem_u32(sm.aq);

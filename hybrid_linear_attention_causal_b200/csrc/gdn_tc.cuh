@@ -2,19 +2,22 @@
 // PTX from the PTX ISA's tcgen05 / mbarrier instruction descriptions.
 //
 // Conventions used by the GDN kernels:
-//   - kind::tf32 MMAs, fp32 accumulators in tensor memory (TMEM), one CTA
-//     (cta_group::1), one elected thread issues.
-//   - shared-memory operands use the K-major no-swizzle canonical layout built
-//     from 8 x 16-byte "core matrices" (128 contiguous bytes each):
-//       tile [R rows][Kt cols]: element (r, k) at byte
-//           ((k/4) * (R/8) + r/8) * 128 + (r%8) * 16 + (k%4) * 4
-//         -> leading-dimension offset (next 4 k)  = (R/8) * 128
-//            stride-dimension offset  (next 8 r)  = 128
-//     Both operands of every MMA are K-major (tf32 with a transposed,
-//     MN-major operand in the no-swizzle layout produced zeros on B200 in a
-//     standalone check, so the kernels arrange their products to avoid it).
-//   - every operand value is rounded to tf32 (round to nearest) before it is
-//     stored, so the tensor core sees exactly the value the kernel chose.
+//   - kind::f16 MMAs with fp16 operands and fp32 accumulators in tensor memory
+//     (TMEM), one CTA (cta_group::1), one elected thread issues.  (kind::tf32
+//     helpers are kept for reference products; the kernels do not use them.)
+//   - shared-memory operands use the no-swizzle canonical layout built from
+//     8 x 16-byte "core matrices" (128 contiguous bytes each).  A tile of R rows
+//     keeps element (r, k) of a 16-bit tile at byte
+//           ((k/8) * (R/8) + r/8) * 128 + (r%8) * 16 + (k%8) * 2      (kmajor_off16)
+//     As a K-major operand (rows r along M or N, k along K) its descriptor has
+//     LBO = (R/8) * 128 (next 8 k) and SBO = 128 (next 8 r).  The same bytes
+//     serve as an MN-major operand whose K runs along the rows r and whose M or
+//     N runs along k: LBO = 128 (next 8 along K), SBO = (R/8) * 128 (next 8
+//     along M or N), and the instruction descriptor's transpose bit for that
+//     operand set (checked on B200 against an fp64 product: max abs error 5e-7
+//     on a 128 x 128 x 64 product; the other LBO/SBO assignment gives garbage).
+//   - every operand value is rounded to fp16 (round to nearest even) before it
+//     is stored, so the tensor core sees exactly the value the kernel chose.
 //   - every wait on an mbarrier gives up after a time limit and reports it,
 //     so a kernel can never hang the GPU.
 #pragma once
@@ -64,6 +67,14 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int R, int s) {
     const uint32_t lbo = (uint32_t)(R >> 3) * 128;
     return make_desc(base + 2 * s * lbo, lbo, 128);
 }
+
+// descriptor of MMA k-step `s` (16 fp16 along K) of an MN-major operand held as a tile of R rows
+// whose rows run along K (see the layout above): the step starts 16 rows (two core matrices) on
+__device__ __forceinline__ uint64_t desc_mnmajor16(uint32_t base, int R, int s) {
+    return make_desc(base + (uint32_t)s * 256, 128, (uint32_t)(R >> 3) * 128);
+}
+// instruction-descriptor bit: the B operand is MN-major (transposed)
+constexpr uint32_t kTransposeB = 1u << 16;
 
 // 32-bit instruction descriptor: kind::tf32, fp32 accumulate, shape M x N.
 // Both operands K-major (bits 15 and 16 clear).

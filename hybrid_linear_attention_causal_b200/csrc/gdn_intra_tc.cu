@@ -19,9 +19,10 @@
 // [W ; diag(e^gamma) Q], Aqk, K~ = diag(e^{gamma_n-gamma}) K (rows s; read
 // MN-major) and U^T; plus gamma.  Operands are staged in shared memory as
 // no-swizzle tiles rounded to fp16; accumulators live in tensor memory.  One
-// thread issues the MMAs; the sixteen warps read their sub-partition's 32-lane
-// slice of tensor memory (four warps per slice, one group of columns each) for
-// the CUDA-core steps.
+// thread issues the MMAs; the eight warps read their sub-partition's 32-lane
+// slice of tensor memory (two warps per slice, one group of columns each) for
+// the CUDA-core steps.  Two CTAs share an SM (half of its tensor memory and
+// shared memory each), so one CTA's barrier waits are covered by the other.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -30,8 +31,10 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NT = 512;        // 16 warps; warp w reads TMEM sub-partition w % 4
+constexpr int NT = 256;        // 8 warps; warp w reads TMEM sub-partition w % 4
+constexpr int kCtasPerSm = 2;  // two CTAs share an SM: one's barrier waits are the other's issue slots
 constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
+constexpr uint32_t kTmemCols = 256;  // D1 (64 columns) + W (DK) + U^T (64), a half of tensor memory
 constexpr int kItemsPerCta = 4;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
@@ -44,7 +47,7 @@ struct IntraTcSmem {
     uint16_t t[C * C];        // T diag(beta), C rows x C: U's operand
     uint16_t te[C * C];       // T diag(beta e^gamma), same layout: W's operand
     float a[C][C + 1];     // A (fp32)
-    float tf[C][C + 4];    // T (fp32), the blocks the next level of the inverse reads
+    float tf[2][32][36];   // T (fp32) in its two 32x32 diagonal blocks: what the next levels read
     float m[32][36];       // A21 T11
     float y[2][16][20];    // A21 D1 inside each 32x32 diagonal block (rows 16-byte aligned)
     float2 gb[2][C];       // (g, beta) of the two heads in flight
@@ -84,7 +87,7 @@ __device__ __forceinline__ void store_h8(void* tile, uint32_t off, const float* 
 
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) {
+__global__ void __launch_bounds__(NT, kCtasPerSm) intra_tc_kernel(ExtendArgs p, int seg) {
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int G = d.G, HV = d.HV, HK = d.HK;
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         }
     };
 
-    if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
+    if (warp == 0) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(bar_kq, 1);
@@ -152,10 +155,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     // blocks of T above the diagonal are zero for every head: in the tile, and in the two 16x16
     // corners of the 32x32 diagonal blocks that the inverse reads back
     for (int e = tid; e < C * C; e += NT) sm.t[e] = sm.te[e] = 0;
-    for (int e = tid; e < 2 * 256; e += NT) {
-        const int o = 32 * (e >> 8);
-        sm.tf[o + ((e >> 4) & 15)][o + 16 + (e & 15)] = 0.f;
-    }
+    for (int e = tid; e < 2 * 256; e += NT) sm.tf[e >> 8][(e >> 4) & 15][16 + (e & 15)] = 0.f;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -215,16 +215,17 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 }
             }
             {  // U^T row j (M = DV layout), the warp's group of C / NCG columns r
-                static_assert(C / NCG == 16, "one 16-column load per warp");
                 const bool vj = DV == 128 || lane < 16;
                 const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
-                const int c0 = cg * 16;
-                float v[16];
-                tc::tmem_ld16(tU + lane_base + c0, v);
-                tc::tmem_ld_wait();
-                if (vj) {
-                    store_h8(Ug, tc::kmajor_off16(jr, c0, DV), v);
-                    store_h8(Ug, tc::kmajor_off16(jr, c0 + 8, DV), v + 8);
+#pragma unroll
+                for (int c0 = cg * (C / NCG); c0 < (cg + 1) * (C / NCG); c0 += 16) {
+                    float v[16];
+                    tc::tmem_ld16(tU + lane_base + c0, v);
+                    tc::tmem_ld_wait();
+                    if (vj) {
+                        store_h8(Ug, tc::kmajor_off16(jr, c0, DV), v);
+                        store_h8(Ug, tc::kmajor_off16(jr, c0 + 8, DV), v + 8);
+                    }
                 }
             }
         }
@@ -278,42 +279,45 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         {  // A (sub-partitions 0-1: k.k rows) and the masked decayed q.k tile (2-3: q.k rows) from D1;
            // the warps of a sub-partition take one group of C / NCG columns each.  The exponents are
            // formed without branches (a masked entry gets -inf, whose exponential is 0) so the
-           // sixteen exponentials of a thread issue back to back; a warp whose whole block lies
-           // above the diagonal only writes zeros.
+           // sixteen exponentials of a 16-column block issue back to back; a block that lies wholly
+           // above the diagonal only gets zeros.
             constexpr int NC = C / NCG;
-            static_assert(NC == 16, "one 16-column load per warp");
-            const int r = (sp & 1) * 32 + lane, c0 = NC * cg;
+            static_assert(NC % 16 == 0, "16-column loads");
+            const int r = (sp & 1) * 32 + lane;
             const bool qrow = sp >= 2;
-            const bool live = c0 <= (sp & 1) * 32 + 31;  // warp-uniform
-            float v[NC], e[NC];
-            if (live) {
-                tc::tmem_ld16(tD1 + lane_base + c0, v);
-                tc::tmem_ld_wait();
-                // entry i is kept when column c0 + i lies below the diagonal (on it, for q.k) of a row
-                // inside the chunk
-                const int lim = r < n ? r - c0 + (qrow ? 1 : 0) : 0;
-                const float gr = sm.gam2[hb][r];
 #pragma unroll
-                for (int q = 0; q < NC; q += 4) {
-                    const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[hb][c0 + q]);
-                    const float gq[4] = {gs.x, gs.y, gs.z, gs.w};
+            for (int c0 = NC * cg; c0 < NC * (cg + 1); c0 += 16) {
+                const bool live = c0 <= (sp & 1) * 32 + 31;  // warp-uniform
+                float v[16], e[16];
+                if (live) {
+                    tc::tmem_ld16(tD1 + lane_base + c0, v);
+                    tc::tmem_ld_wait();
+                    // entry i is kept when column c0 + i lies below the diagonal (on it, for q.k) of a
+                    // row inside the chunk
+                    const int lim = r < n ? r - c0 + (qrow ? 1 : 0) : 0;
+                    const float gr = sm.gam2[hb][r];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        e[q + u] = q + u < lim ? gr - gq[u] : __int_as_float(0xff800000u);  // -inf
+                    for (int q = 0; q < 16; q += 4) {
+                        const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[hb][c0 + q]);
+                        const float gq[4] = {gs.x, gs.y, gs.z, gs.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            e[q + u] = q + u < lim ? gr - gq[u] : __int_as_float(0xff800000u);  // -inf
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) e[i] = tc::ex2_approx(e[i]) * v[i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) e[i] = 0.f;
                 }
+                if (!qrow) {
+                    const float br = sm.beta[hb][r];
 #pragma unroll
-                for (int i = 0; i < NC; ++i) e[i] = tc::ex2_approx(e[i]) * v[i];
-            } else {
-#pragma unroll
-                for (int i = 0; i < NC; ++i) e[i] = 0.f;
-            }
-            if (!qrow) {
-                const float br = sm.beta[hb][r];
-#pragma unroll
-                for (int i = 0; i < NC; ++i) sm.a[r][c0 + i] = br * e[i];
-            } else {
-                store_h8(AQg, tc::kmajor_off16(r, c0, C), e);
-                store_h8(AQg, tc::kmajor_off16(r, c0 + 8, C), e + 8);
+                    for (int i = 0; i < 16; ++i) sm.a[r][c0 + i] = br * e[i];
+                } else {
+                    store_h8(AQg, tc::kmajor_off16(r, c0, C), e);
+                    store_h8(AQg, tc::kmajor_off16(r, c0 + 8, C), e + 8);
+                }
             }
         }
         if (j > 0) epilogue(j - 1);  // the previous head's W and U^T, from other tensor-memory columns
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         // T diag(beta) (the A operand of W and U); the fp32 copy tf holds what the next level reads.
         //   level 1: the four diagonal 16x16 blocks by forward substitution, one column per lane held
         //            in registers (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so
-        //            one FMA per row sits on the dependent chain); warps 4-15 meanwhile write the
+        //            one FMA per row sits on the dependent chain); the other warps meanwhile write the
         //            tiles that need only the gates: the state pass's K~ = diag(e^{gamma_n-gamma}) K
         //            and the rows Qg = diag(e^gamma) Q of [W ; Qg], and gamma.
         //   level 2: within each 32x32 diagonal block, X = -D2 (A21 D1).
@@ -350,7 +354,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 }
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    sm.tf[o + r][o + c] = t[r];
+                    sm.tf[warp >> 1][16 * (warp & 1) + r][16 * (warp & 1) + c] = t[r];
                     put_t(o + r, o + c, t[r]);
                 }
             }
@@ -390,7 +394,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int s = 0; s < 16; ++s)  // Y = A21 D1
-                    fma4(y, sm.a[o1 + r][o0 + s], *reinterpret_cast<const float4*>(&sm.tf[o0 + s][o0 + c4]));
+                    fma4(y, sm.a[o1 + r][o0 + s], *reinterpret_cast<const float4*>(&sm.tf[bb][s][c4]));
                 *reinterpret_cast<float4*>(&sm.y[bb][r][c4]) = y;
             }
             __syncthreads();
@@ -398,9 +402,9 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int s = 0; s < 16; ++s)  // X = -D2 Y
-                    fma4(x, sm.tf[o1 + r][o1 + s], *reinterpret_cast<const float4*>(&sm.y[bb][s][c4]));
+                    fma4(x, sm.tf[bb][16 + r][16 + s], *reinterpret_cast<const float4*>(&sm.y[bb][s][c4]));
                 x = make_float4(-x.x, -x.y, -x.z, -x.w);
-                *reinterpret_cast<float4*>(&sm.tf[o1 + r][o0 + c4]) = x;
+                *reinterpret_cast<float4*>(&sm.tf[bb][16 + r][c4]) = x;
                 put_t(o1 + r, o0 + c4, x.x);
                 put_t(o1 + r, o0 + c4 + 1, x.y);
                 put_t(o1 + r, o0 + c4 + 2, x.z);
@@ -410,28 +414,32 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
         __syncthreads();
         // Level 3 reads one operand as a warp-wide broadcast and skips the zero blocks of the
         // triangular factors: T11[s][c] = 0 for s < c and T22[r][s] = 0 for s > r.
-        static_assert(NT == 512, "level 3 maps 8 column groups, then 16 row pairs, onto the warps");
+        static_assert(NT / 32 >= 8 && 32 % (NT / 32) == 0, "level 3 maps 8 column groups, then row groups, onto the warps");
         if (warp < 8) {  // level 3a: P = A21 T11; warp w takes columns 4w .. 4w + 3, lane = row
             const int r = lane, c4 = 4 * warp;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
             for (int s = c4; s < 32; ++s)
-                fma4(acc, sm.a[32 + r][s], *reinterpret_cast<const float4*>(&sm.tf[s][c4]));
+                fma4(acc, sm.a[32 + r][s], *reinterpret_cast<const float4*>(&sm.tf[0][s][c4]));
             *reinterpret_cast<float4*>(&sm.m[r][c4]) = acc;
         }
         __syncthreads();
-        {  // level 3b: T21 = -T22 P; warp w takes rows 2w, 2w + 1 of the block, lane = column
-            const int r0 = 2 * warp, c = lane;
-            float acc0 = 0.f, acc1 = 0.f;
-            for (int s4 = 0; s4 < r0 + 2; s4 += 4) {
-                const float4 t0 = *reinterpret_cast<const float4*>(&sm.tf[32 + r0][32 + s4]);
-                const float4 t1 = *reinterpret_cast<const float4*>(&sm.tf[33 + r0][32 + s4]);
+        {  // level 3b: T21 = -T22 P; warp w takes RPW consecutive rows of the block, lane = column
+            constexpr int RPW = 32 / (NT / 32);
+            const int r0 = RPW * warp, c = lane;
+            float acc[RPW];
+#pragma unroll
+            for (int i = 0; i < RPW; ++i) acc[i] = 0.f;
+            for (int s4 = 0; s4 < r0 + RPW; s4 += 4) {
                 const float p0 = sm.m[s4][c], p1 = sm.m[s4 + 1][c], p2 = sm.m[s4 + 2][c], p3 = sm.m[s4 + 3][c];
-                acc0 = fmaf(t0.x, p0, fmaf(t0.y, p1, fmaf(t0.z, p2, fmaf(t0.w, p3, acc0))));
-                acc1 = fmaf(t1.x, p0, fmaf(t1.y, p1, fmaf(t1.z, p2, fmaf(t1.w, p3, acc1))));
+#pragma unroll
+                for (int i = 0; i < RPW; ++i) {
+                    const float4 t = *reinterpret_cast<const float4*>(&sm.tf[1][r0 + i][s4]);
+                    acc[i] = fmaf(t.x, p0, fmaf(t.y, p1, fmaf(t.z, p2, fmaf(t.w, p3, acc[i]))));
+                }
             }
-            put_t(32 + r0, c, -acc0);
-            put_t(33 + r0, c, -acc1);
+#pragma unroll
+            for (int i = 0; i < RPW; ++i) put_t(32 + r0 + i, c, -acc[i]);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -495,7 +503,7 @@ __global__ void __launch_bounds__(NT, 1) intra_tc_kernel(ExtendArgs p, int seg) 
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tm, 512);
+    if (warp == 0) tc::tmem_dealloc(tm, kTmemCols);
 }
 
 }  // namespace

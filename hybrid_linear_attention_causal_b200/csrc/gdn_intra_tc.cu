@@ -35,7 +35,7 @@ constexpr int NT = 256;        // 8 warps; warp w reads TMEM sub-partition w % 4
 constexpr int kCtasPerSm = 2;  // two CTAs share an SM: one's barrier waits are the other's issue slots
 constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
 constexpr uint32_t kTmemCols = 256;  // D1 (64 columns) + W (DK) + U^T (64), a half of tensor memory
-constexpr int kItemsPerCta = 4;
+constexpr int kItemsPerCta = 2;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
 template <int DK, int DV>

@@ -16,8 +16,10 @@
 // chunk's state to the next runs through the first product, V', the state
 // product and the update; everything else is kept off it:
 //   - a ninth warp only issues the MMAs and the bulk copies, so the eight
-//     compute warps never wait behind an issue loop; it issues the output
-//     product only once the state product has completed;
+//     compute warps never wait behind an issue loop; it queues the output
+//     product right behind the state product and waits for it only in the
+//     next chunk, after issuing that chunk's first product (the tensor core
+//     runs them in order), before refetching the Aqk tile;
 //   - the fp32 state lives in registers (each thread holds one half of row j
 //     of S^T), the state product goes to a fresh accumulator and the update
 //     is one FMA per element, written straight into the fp16 operand copy;
@@ -27,8 +29,8 @@
 //     fp16 in the tensor core's layout) each have their own barrier and are
 //     refetched as soon as the product that reads them completes;
 //   - the intra-chunk kernel writes U^T in the layout of the V'^T operand
-//     tile, so it lands in that tile by one bulk copy and V' is formed in
-//     place (each thread rewrites exactly the elements it read).
+//     tile; it lands in a tile of its own, so the next chunk's copy starts
+//     as soon as V' has been formed from it.
 // The two compute warps of a TMEM sub-partition share its 32 accumulator rows
 // and take one half of the columns each.
 
@@ -56,7 +58,8 @@ struct StateTcSmem {
     uint16_t wq[2 * C * DK];  // [W ; Qg] tile (bulk copy): 128 rows x DK
     uint16_t aq[C * C];       // Aqk tile (bulk copy): C rows (r) x C (s)
     uint16_t kt[C * DK];      // K~ tile (bulk copy): C rows (s) x DK (i), the MN-major B of Snew^T
-    uint16_t vt[DV * C];      // U^T tile (bulk copy), overwritten in place by V'^T: DV rows (j) x C (s)
+    uint16_t ut[DV * C];      // U^T tile (bulk copy): DV rows (j) x C (s)
+    uint16_t vt[DV * C];      // V'^T = U^T - X^T, same layout: the A operand of the state and output products
     T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
     unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq, bar_u;
     uint32_t tmem_base;
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     auto u_src = [&](int id) { return p.U + ((size_t)id * HV + h) * (DV * C); };
     auto fetch_u = [&](int id) {
         tc::mbar_expect_tx(bar_u, U_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.vt), u_src(id), U_BYTES, bar_u);
+        tc::bulk_g2s(tc::smem_u32(sm.ut), u_src(id), U_BYTES, bar_u);
     };
     auto fetch_aq = [&](int id) {
         tc::mbar_expect_tx(bar_aq, AQ_BYTES);
@@ -214,6 +217,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     tc::mma_f16(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
                 tc::mma_commit(bar_x);
             }
+            if (okl && id > c_begin) {  // the previous chunk's output product is done with the Aqk tile
+                okl = tc::mbar_wait(bar_o, ph ^ 1u);
+                if (okl) fetch_aq(id);
+            }
             if (okl && id + 1 < c_end) {  // the next chunk's tiles into L2, so their copies wait on L2 only
                 const size_t nx = (size_t)(id + 1) * HV + h;
                 tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             }
             okl = __all_sync(0xffffffffu, okl && tc::mbar_wait(bar_x, ph) && tc::mbar_wait(bar_u, ph));
             tc::fence_after_sync();
-            if (okl) {  // V'^T row j = U^T row j - X^T row j, in place: each thread rewrites what it read
+            if (okl) {  // V'^T row j = U^T row j - X^T row j
 #pragma unroll
                 for (int cc = 0; cc < C / 2; cc += 16) {
                     const int c0 = half * (C / 2) + cc;
@@ -245,9 +252,9 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     if (rowv)
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {  // 8 fp16 values per 16-byte vector
-                            uint4* pv = reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.vt) +
-                                                                 tc::kmajor_off16(j, c0 + 8 * q, DV));
-                            const uint4 u = *pv;
+                            const uint32_t off = tc::kmajor_off16(j, c0 + 8 * q, DV);
+                            uint4* pv = reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.vt) + off);
+                            const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(sm.ut) + off);
                             const float2 u0 = tc::unpack_f16(u.x), u1 = tc::unpack_f16(u.y), u2 = tc::unpack_f16(u.z),
                                          u3 = tc::unpack_f16(u.w);
                             const float* xq = x + 8 * q;
@@ -263,6 +270,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         if (!ok) break;
         tc::fence_after_sync();
         if (tid == ISSUER) {
+            if (id + 1 < c_end) fetch_u(id + 1);  // V' has read the U^T tile
             okl = tc::mbar_wait(bar_kt, ph);
             if (okl) {  // Snew^T = V'^T K~, K~ (rows s) read MN-major
                 const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt);
@@ -271,24 +279,19 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 for (int k = 0; k < C / 16; ++k)
                     tc::mma_f16(tS, tc::desc_kmajor(av, DV, k), tc::desc_mnmajor16(bk, C, k), is, k > 0);
                 tc::mma_commit(bar_s);
-                okl = tc::mbar_wait(bar_s, ph);
             }
-            if (okl && id + 1 < c_end) fetch_kt(id + 1);  // the K~ tile is free again
             if (okl) okl = tc::mbar_wait(bar_aq, ph);
-            if (okl) {  // O^T += V'^T Aqk^T, off the state chain
+            if (okl) {  // O^T += V'^T Aqk^T: queued behind the state product, off the state chain; the
+                        // next chunk's first product waits for it (the tensor core runs them in order)
                 const uint32_t av = tc::smem_u32(sm.vt), bq = tc::smem_u32(sm.aq);
                 constexpr uint32_t io = tc::idesc_f16(DV, 64);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
                     tc::mma_f16(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
                 tc::mma_commit(bar_o);
-                // the next chunk's Aqk and U^T, once the output product is done with the Aqk and V'^T tiles
-                okl = tc::mbar_wait(bar_o, ph);
-                if (okl && id + 1 < c_end) {
-                    fetch_aq(id + 1);
-                    fetch_u(id + 1);
-                }
             }
+            if (okl) okl = tc::mbar_wait(bar_s, ph);
+            if (okl && id + 1 < c_end) fetch_kt(id + 1);  // the K~ tile is free again
         } else if (warp < NCW) {
             if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
                                                           // state product runs meanwhile

@@ -216,9 +216,24 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // Waits until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// One non-blocking test of the phase with parity `parity` of the mbarrier.
+__device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
+    uint32_t done = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Waits for the phase with parity `parity` of the mbarrier to complete.
-// Gives up after `limit_ns` nanoseconds and returns false.
+// Gives up after `limit_ns` nanoseconds and returns false.  A phase that has already completed
+// costs one test: the clock is read only once the wait is real.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+    if (mbar_test(mbar, parity)) return true;
     uint32_t done = 0;
     const uint64_t t0 = globaltimer_ns();
     while (true) {

@@ -22,9 +22,12 @@
 //     runs them in order), before refetching the Aqk tile;
 //   - the fp32 state lives in registers (each thread holds one half of row j
 //     of S^T), the state product goes to a fresh accumulator and the update
-//     is one FMA per element, written straight into the fp16 operand copy;
+//     is one FMA per element, written straight into the fp16 copy of S^T that
+//     the first product reads from tensor memory (so that product reads only
+//     [W ; Qg] from shared memory);
 //   - [X^T | O^T] is double-buffered in tensor memory: a chunk's outputs are
 //     read and stored while the next chunk's first product runs;
+//   - [W ; Qg] and K~ are double-buffered and copied two chunks ahead;
 //   - the tiles [W ; Qg], K~ and Aqk (written by the intra-chunk kernel as
 //     fp16 in the tensor core's layout) each have their own barrier and are
 //     refetched as soon as the product that reads them completes;
@@ -53,28 +56,26 @@ constexpr bool kStageOut = sizeof(T) == 2;
 
 template <typename T, int DK, int DV>
 struct StateTcSmem {
-    // fp16 operand tiles (16-bit K-major layout)
-    uint16_t st[DV * DK];     // S^T tile: DV rows x DK (fp16 copy of the state)
-    uint16_t wq[2 * C * DK];  // [W ; Qg] tile (bulk copy): 128 rows x DK
+    // fp16 operand tiles (16-bit K-major layout); [W ; Qg] and K~ are double-buffered and copied
+    // two chunks ahead
+    uint16_t wq[2][2 * C * DK];  // [W ; Qg] tiles (bulk copy): 128 rows x DK
+    uint16_t kt[2][C * DK];      // K~ tiles (bulk copy): C rows (s) x DK (i), the MN-major B of Snew^T
     uint16_t aq[C * C];       // Aqk tile (bulk copy): C rows (r) x C (s)
-    uint16_t kt[C * DK];      // K~ tile (bulk copy): C rows (s) x DK (i), the MN-major B of Snew^T
     uint16_t ut[DV * C];      // U^T tile (bulk copy): DV rows (j) x C (s)
     uint16_t vt[DV * C];      // V'^T = U^T - X^T, same layout: the A operand of the state and output products
     T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
-    unsigned long long bar_x, bar_s, bar_o, bar_wq, bar_kt, bar_aq, bar_u;
+    unsigned long long bar_x, bar_s, bar_o, bar_wq[2], bar_kt[2], bar_aq, bar_u;
     uint32_t tmem_base;
 };
 
 
-// fp16 copies of 16 consecutive values of S^T row j (columns c0..c0+15, c0 a multiple of 8) into
-// the operand tile: two 16-byte vectors
-template <int DV>
-__device__ __forceinline__ void put_st16(uint16_t* st, int j, int c0, const float* v) {
+// fp16 copy of 32 consecutive values of S^T row j (this thread's lane) into 16 columns of the
+// tensor-memory A operand: two fp16 per column, the even column of S^T in the low half
+__device__ __forceinline__ void put_sa32(uint32_t taddr, const float* v) {
+    uint32_t w[16];
 #pragma unroll
-    for (int q = 0; q < 2; ++q)
-        *reinterpret_cast<uint4*>(reinterpret_cast<char*>(st) + tc::kmajor_off16(j, c0 + 8 * q, DV)) =
-            make_uint4(tc::pack_f16(v[8 * q], v[8 * q + 1]), tc::pack_f16(v[8 * q + 2], v[8 * q + 3]),
-                       tc::pack_f16(v[8 * q + 4], v[8 * q + 5]), tc::pack_f16(v[8 * q + 6], v[8 * q + 7]));
+    for (int i = 0; i < 16; ++i) w[i] = tc::pack_f16(v[2 * i], v[2 * i + 1]);
+    tc::tmem_st16(taddr, w);
 }
 
 template <typename T, int DK, int DV>
@@ -106,17 +107,22 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StateTcSmem<T, DK, DV>& sm = *reinterpret_cast<StateTcSmem<T, DK, DV>*>(smem_raw);
     const uint32_t bar_x = tc::smem_u32(&sm.bar_x), bar_s = tc::smem_u32(&sm.bar_s),
-                   bar_o = tc::smem_u32(&sm.bar_o), bar_wq = tc::smem_u32(&sm.bar_wq),
-                   bar_kt = tc::smem_u32(&sm.bar_kt), bar_aq = tc::smem_u32(&sm.bar_aq),
+                   bar_o = tc::smem_u32(&sm.bar_o), bar_aq = tc::smem_u32(&sm.bar_aq),
                    bar_u = tc::smem_u32(&sm.bar_u);
     constexpr uint32_t WQ_BYTES = 2 * C * DK * 2, AQ_BYTES = C * C * 2, KT_BYTES = DK * C * 2, U_BYTES = DV * C * 2;
+    // buffer b = (id - c_begin) & 1 of the double-buffered tiles; its barrier completes once every
+    // other chunk, so a chunk waits on parity ((id - c_begin) >> 1) & 1
+    auto bar_wq = [&](int b) { return tc::smem_u32(&sm.bar_wq[b]); };
+    auto bar_kt = [&](int b) { return tc::smem_u32(&sm.bar_kt[b]); };
     auto fetch_wq = [&](int id) {
-        tc::mbar_expect_tx(bar_wq, WQ_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.wq), p.WQ + ((size_t)id * HV + h) * (2 * C * DK), WQ_BYTES, bar_wq);
+        const int b = (id - c_begin) & 1;
+        tc::mbar_expect_tx(bar_wq(b), WQ_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.wq[b]), p.WQ + ((size_t)id * HV + h) * (2 * C * DK), WQ_BYTES, bar_wq(b));
     };
     auto fetch_kt = [&](int id) {
-        tc::mbar_expect_tx(bar_kt, KT_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.kt), p.KT + ((size_t)id * HV + h) * (DK * C), KT_BYTES, bar_kt);
+        const int b = (id - c_begin) & 1;
+        tc::mbar_expect_tx(bar_kt(b), KT_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.kt[b]), p.KT + ((size_t)id * HV + h) * (DK * C), KT_BYTES, bar_kt(b));
     };
     auto u_src = [&](int id) { return p.U + ((size_t)id * HV + h) * (DV * C); };
     auto fetch_u = [&](int id) {
@@ -132,13 +138,17 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         tc::mbar_init(bar_x, 1);
         tc::mbar_init(bar_s, 1);
         tc::mbar_init(bar_o, 1);
-        tc::mbar_init(bar_wq, 1);
-        tc::mbar_init(bar_kt, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(bar_wq(b), 1);
+            tc::mbar_init(bar_kt(b), 1);
+        }
         tc::mbar_init(bar_aq, 1);
         tc::mbar_init(bar_u, 1);
         tc::fence_mbar_init();
-        fetch_wq(c_begin);
-        fetch_kt(c_begin);
+        for (int id = c_begin; id < c_end && id < c_begin + 2; ++id) {
+            fetch_wq(id);
+            fetch_kt(id);
+        }
         fetch_aq(c_begin);
         fetch_u(c_begin);
     }
@@ -154,9 +164,6 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     float s[DK / 2];
 #pragma unroll
     for (int i = 0; i < DK / 2; ++i) s[i] = (init && rowv) ? Sg[(size_t)(half * (DK / 2) + i) * DV + j] : 0.f;
-    if (rowv)
-#pragma unroll
-        for (int cc = 0; cc < DK / 2; cc += 16) put_st16<DV>(sm.st, j, half * (DK / 2) + cc, &s[cc]);
     int4 ch = p.chunk_tab[c_begin];
     float gl = p.gam[((size_t)c_begin * HV + h) * C + ch.z - 1];  // gamma_n of this chunk
     int4 ch_nx = c_begin + 1 < c_end ? p.chunk_tab[c_begin + 1] : ch;
@@ -165,7 +172,21 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
-    const uint32_t tS = tm + 256;  // Snew^T (DK columns); [X^T | O^T] double buffer at tm, tm + 128
+    // [X^T | O^T] double buffer at tm, tm + 128; Snew^T (DK columns) at tm + 256; the fp16 copy of
+    // S^T, the A operand of the first product (DK / 2 columns), at tm + 384
+    const uint32_t tS = tm + 256, tA = tm + 384;
+    static_assert(DK <= 128, "tensor-memory layout");
+    // this thread's DK / 2 state columns of row j into the A operand (lanes past the rows of a
+    // 64-row tile hold values no product reads)
+    const uint32_t tA_row = tA + lane_base + half * (DK / 4);
+    if (warp < NCW) {
+#pragma unroll
+        for (int cc = 0; cc < DK / 2; cc += 32) put_sa32(tA_row + cc / 2, &s[cc]);
+        tc::tmem_st_wait();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
 
     // rows t < n of O (chunk at row t0), this thread's column j and half of the rows, from the
     // O^T half of an [X^T | O^T] buffer: into the staging tile, or straight to global memory
@@ -207,30 +228,32 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         if (id + 1 < c_end) gl_nx = p.gam[((size_t)(id + 1) * HV + h) * C + ch_nx.z - 1];
         if (id + 2 < c_end) ch_nx2 = p.chunk_tab[id + 2];
         bool okl = true;
+        const int bb = (id - c_begin) & 1;
+        const uint32_t pb = (uint32_t)((id - c_begin) >> 1) & 1u;
         if (tid == ISSUER) {
-            okl = tc::mbar_wait(bar_wq, ph);
-            if (okl) {  // [X^T | O^T] = S^T [W ; Qg]^T
-                const uint32_t a = tc::smem_u32(sm.st), b = tc::smem_u32(sm.wq);
+            okl = tc::mbar_wait(bar_wq(bb), pb);
+            if (okl) {  // [X^T | O^T] = S^T [W ; Qg]^T, S^T from tensor memory
+                const uint32_t b = tc::smem_u32(sm.wq[bb]);
                 constexpr uint32_t idesc = tc::idesc_f16(DV, 128);
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k)
-                    tc::mma_f16(tXO, tc::desc_kmajor(a, DV, k), tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
+                    tc::mma_f16_ta(tXO, tA + 8 * k, tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
                 tc::mma_commit(bar_x);
             }
             if (okl && id > c_begin) {  // the previous chunk's output product is done with the Aqk tile
                 okl = tc::mbar_wait(bar_o, ph ^ 1u);
                 if (okl) fetch_aq(id);
             }
-            if (okl && id + 1 < c_end) {  // the next chunk's tiles into L2, so their copies wait on L2 only
-                const size_t nx = (size_t)(id + 1) * HV + h;
+            if (okl && id + 2 < c_end) {  // tiles two chunks ahead into L2, so their copies wait on L2 only
+                const size_t nx = (size_t)(id + 2) * HV + h;
                 tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
                 tc::bulk_prefetch_l2(p.KT + nx * (DK * C), KT_BYTES);
                 tc::bulk_prefetch_l2(p.AQ + nx * (C * C), AQ_BYTES);
-                tc::bulk_prefetch_l2(u_src(id + 1), U_BYTES);
+                tc::bulk_prefetch_l2(u_src(id + 2), U_BYTES);
             }
             if (okl) {
                 okl = tc::mbar_wait(bar_x, ph);
-                if (okl && id + 1 < c_end) fetch_wq(id + 1);  // the [W ; Qg] tile is free again
+                if (okl && id + 2 < c_end) fetch_wq(id + 2);  // this [W ; Qg] buffer is free again
             }
         } else if (warp < NCW) {
             if (id > c_begin) {  // the previous chunk's outputs leave while this chunk's first product runs
@@ -271,9 +294,9 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         tc::fence_after_sync();
         if (tid == ISSUER) {
             if (id + 1 < c_end) fetch_u(id + 1);  // V' has read the U^T tile
-            okl = tc::mbar_wait(bar_kt, ph);
+            okl = tc::mbar_wait(bar_kt(bb), pb);
             if (okl) {  // Snew^T = V'^T K~, K~ (rows s) read MN-major
-                const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt);
+                const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt[bb]);
                 constexpr uint32_t is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
@@ -291,7 +314,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 tc::mma_commit(bar_o);
             }
             if (okl) okl = tc::mbar_wait(bar_s, ph);
-            if (okl && id + 1 < c_end) fetch_kt(id + 1);  // the K~ tile is free again
+            if (okl && id + 2 < c_end) fetch_kt(id + 2);  // this K~ buffer is free again
         } else if (warp < NCW) {
             if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
                                                           // state product runs meanwhile
@@ -300,18 +323,19 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 tc::fence_after_sync();
                 const float egl = expf(gl);
 #pragma unroll
-                for (int cc = 0; cc < DK / 2; cc += 16) {
+                for (int cc = 0; cc < DK / 2; cc += 32) {
                     const int c0 = half * (DK / 2) + cc;
-                    float v[16];
-                    tc::tmem_ld16(tS + lane_base + c0, v);
+                    float v[32];
+                    tc::tmem_ld16(tS + lane_base + c0, *reinterpret_cast<float(*)[16]>(v));
+                    tc::tmem_ld16(tS + lane_base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) s[cc + i] = fmaf(egl, s[cc + i], v[i]);
-                    if (rowv) put_st16<DV>(sm.st, j, c0, &s[cc]);
+                    for (int i = 0; i < 32; ++i) s[cc + i] = fmaf(egl, s[cc + i], v[i]);
+                    put_sa32(tA_row + cc / 2, &s[cc]);
                 }
+                tc::tmem_st_wait();
             }
         }
-        tc::fence_smem_to_async();
         tc::fence_before_sync();
         ok = __syncthreads_and(okl);
         if (!ok) break;
@@ -345,8 +369,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         // let copies and products already in flight finish before the CTA's shared and tensor
         // memory go away
         for (uint32_t par = 0; par < 2; ++par) {
-            tc::mbar_wait(bar_wq, par, 100000000ull);
-            tc::mbar_wait(bar_kt, par, 100000000ull);
+            for (int b = 0; b < 2; ++b) {
+                tc::mbar_wait(bar_wq(b), par, 100000000ull);
+                tc::mbar_wait(bar_kt(b), par, 100000000ull);
+            }
             tc::mbar_wait(bar_aq, par, 100000000ull);
             tc::mbar_wait(bar_o, par, 100000000ull);
             tc::mbar_wait(bar_u, par, 100000000ull);

@@ -35,6 +35,7 @@ constexpr int NT = 256;        // 8 warps; warp w reads TMEM sub-partition w % 4
 constexpr int kCtasPerSm = 2;  // two CTAs share an SM: one's barrier waits are the other's issue slots
 constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
 constexpr uint32_t kTmemCols = 256;  // D1 (64 columns) + W (DK) + U^T (64), a half of tensor memory
+constexpr int kInvBarrier = 1;       // named barrier of warps 0-3, which take levels 1 and 2 of the inverse
 constexpr int kItemsPerCta = 2;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
@@ -61,6 +62,8 @@ struct IntraTcSmem {
     uint32_t tmem_base;
     int next_item;         // thread 0's latest grab, for the other threads
 };
+
+__device__ __forceinline__ void bar_sync_n(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // idx -> (row, first column) of an 8-column group of a 16-bit K-major tile with R rows: 8
 // consecutive lanes take 8 consecutive rows, i.e. one 128-byte core matrix
@@ -339,6 +342,12 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) intra_tc_kernel(ExtendArgs p, 
             *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.t) + off) = (uint16_t)(w & 0xffffu);
             *reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(sm.te) + off) = (uint16_t)(w >> 16);
         };
+        auto fma4 = [](float4& acc, float a, const float4& b) {
+            acc.x = fmaf(a, b.x, acc.x);
+            acc.y = fmaf(a, b.y, acc.y);
+            acc.z = fmaf(a, b.z, acc.z);
+            acc.w = fmaf(a, b.w, acc.w);
+        };
         if (warp < 4) {
             if (lane < 16) {
                 const int o = 16 * warp, c = lane;
@@ -358,6 +367,37 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) intra_tc_kernel(ExtendArgs p, 
                     put_t(o + r, o + c, t[r]);
                 }
             }
+            // levels 1 -> 2 synchronise warps 0-3 only: the other warps keep writing the gate-only
+            // tiles meanwhile
+            bar_sync_n(kInvBarrier, 128);
+            // Level 2 tiles the outputs in registers: a thread takes four consecutive columns of one
+            // row, so each step of a dot product is one (broadcast) load of the left factor and one
+            // 16-byte load of the right one for four FMAs; the shared-memory pipe, not the FMAs,
+            // bounds these small products.
+            {  // level 2 (threads 0..127): 32-block bb, row r, columns c4 .. c4 + 3
+                const int bb = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
+                const int o0 = 32 * bb, o1 = o0 + 16;
+                {
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int s = 0; s < 16; ++s)  // Y = A21 D1
+                        fma4(y, sm.a[o1 + r][o0 + s], *reinterpret_cast<const float4*>(&sm.tf[bb][s][c4]));
+                    *reinterpret_cast<float4*>(&sm.y[bb][r][c4]) = y;
+                }
+                bar_sync_n(kInvBarrier, 128);
+                {
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int s = 0; s < 16; ++s)  // X = -D2 Y
+                        fma4(x, sm.tf[bb][16 + r][16 + s], *reinterpret_cast<const float4*>(&sm.y[bb][s][c4]));
+                    x = make_float4(-x.x, -x.y, -x.z, -x.w);
+                    *reinterpret_cast<float4*>(&sm.tf[bb][16 + r][c4]) = x;
+                    put_t(o1 + r, o0 + c4, x.x);
+                    put_t(o1 + r, o0 + c4 + 1, x.y);
+                    put_t(o1 + r, o0 + c4 + 2, x.z);
+                    put_t(o1 + r, o0 + c4 + 3, x.w);
+                }
+            }
         } else {  // row scalings of the [K ; Q] tile, 8 features per 16-byte vector
             constexpr int NW = NT - 128;
             for (int idx = tid - 128; idx < 2 * C * DK / 8; idx += NW) {
@@ -375,41 +415,6 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) intra_tc_kernel(ExtendArgs p, 
                     store_h8(WQg, off, v);  // rows Qg: same offsets in [W ; Qg]
             }
             if (tid - 128 < C) p.gam[ch_h * C + tid - 128] = sm.gam[hb][tid - 128];
-        }
-        __syncthreads();
-        // Level 2 tiles the outputs in registers: a thread takes four consecutive columns of one row,
-        // so each step of a dot product is one (broadcast) load of the left factor and one 16-byte
-        // load of the right one for four FMAs; the shared-memory pipe, not the FMAs, bounds these
-        // small products.
-        auto fma4 = [](float4& acc, float a, const float4& b) {
-            acc.x = fmaf(a, b.x, acc.x);
-            acc.y = fmaf(a, b.y, acc.y);
-            acc.z = fmaf(a, b.z, acc.z);
-            acc.w = fmaf(a, b.w, acc.w);
-        };
-        {  // level 2 (threads 0..127): 32-block bb, row r, columns c4 .. c4 + 3
-            const int bb = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-            const int o0 = 32 * bb, o1 = o0 + 16;
-            if (tid < 128) {
-                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int s = 0; s < 16; ++s)  // Y = A21 D1
-                    fma4(y, sm.a[o1 + r][o0 + s], *reinterpret_cast<const float4*>(&sm.tf[bb][s][c4]));
-                *reinterpret_cast<float4*>(&sm.y[bb][r][c4]) = y;
-            }
-            __syncthreads();
-            if (tid < 128) {
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int s = 0; s < 16; ++s)  // X = -D2 Y
-                    fma4(x, sm.tf[bb][16 + r][16 + s], *reinterpret_cast<const float4*>(&sm.y[bb][s][c4]));
-                x = make_float4(-x.x, -x.y, -x.z, -x.w);
-                *reinterpret_cast<float4*>(&sm.tf[bb][16 + r][c4]) = x;
-                put_t(o1 + r, o0 + c4, x.x);
-                put_t(o1 + r, o0 + c4 + 1, x.y);
-                put_t(o1 + r, o0 + c4 + 2, x.z);
-                put_t(o1 + r, o0 + c4 + 3, x.w);
-            }
         }
         __syncthreads();
         // Level 3 reads one operand as a warp-wide broadcast and skips the zero blocks of the

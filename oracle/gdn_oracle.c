@@ -496,3 +496,32 @@ int ora_verify(const ora_cfg* cfg, const double* A_log, const double* dt_bias, c
     free(cs); free(ss); free(st); free(cu); free(loc);
     return rc;
 }
+
+/*
+ * Speculative commit, the step after verify: request i accepted acc[i] of its D
+ * draft tokens; for acc[i] >= 1 its slot takes the checkpoints recorded after
+ * token acc[i]-1 (state and, when conv_ckpt is non-NULL, conv window), so the
+ * pools hold what running the accepted tokens from the slot would have left;
+ * acc[i] == 0 and padded requests (slot < 0) leave everything untouched.  The
+ * commit of the speculative state buffer for the accepted draft prefix, page
+ * "SGLang GDN hybrid linear attention test matrix", verification conventions.
+ * Returns 2 for a slot >= P and 3 for an accepted count outside 0..D (nothing
+ * written for that request).
+ */
+int ora_commit(const ora_cfg* cfg, int B, int D, const int32_t* slots, const int32_t* acc, const double* ckpt,
+               const double* conv_ckpt, double* conv_state, double* ssm_state, int P) {
+    const int HV = cfg->HV, dk = cfg->dk, dv = cfg->dv, K = cfg->K;
+    const int64_t CD = ora_conv_dim(cfg);
+    const int64_t sslot = (int64_t)HV * dk * dv, cslot = CD * (K - 1);
+    int rc = 0;
+    for (int i = 0; i < B; ++i) {
+        if (slots[i] < 0) continue;
+        if (slots[i] >= P) { rc = 2; continue; }
+        if (acc[i] < 0 || acc[i] > D) { rc = 3; continue; }
+        if (acc[i] == 0) continue;
+        const int64_t t = (int64_t)i * D + (acc[i] - 1);
+        memcpy(ssm_state + slots[i] * sslot, ckpt + t * sslot, sizeof(double) * sslot);
+        if (conv_ckpt) memcpy(conv_state + slots[i] * cslot, conv_ckpt + t * cslot, sizeof(double) * cslot);
+    }
+    return rc;
+}

@@ -295,3 +295,22 @@ def verify(cfg: OracleCfg, params: dict, x, a, b, state_indices, D: int, conv_st
     if rc != 0:
         raise ValueError(f"oracle verify rejected its arguments (code {rc})")
     return out, ckpt, cck
+
+
+def commit(cfg: OracleCfg, state_indices, accepted, D: int, ckpt, conv_ckpt, conv_state, ssm_state):
+    """Pools after committing each request's last accepted draft token (copies; inputs untouched).
+
+    ckpt [B,D,HV,dk,dv] and conv_ckpt [B,D,conv_dim,K-1] (or None) as verify returns them.
+    Returns (conv_state, ssm_state, code): code 0, 2 (a slot >= P) or 3 (an accepted count
+    outside 0..D); such requests are skipped.
+    """
+    slots = _i32(state_indices)
+    acc = _i32(accepted)
+    cs = _f64(conv_state).copy()
+    ss = _f64(ssm_state).copy()
+    ck = _f64(ckpt)
+    cck = _f64(conv_ckpt) if conv_ckpt is not None else None
+    c = cfg._c()
+    code = _L().ora_commit(ctypes.byref(c), ctypes.c_int(len(slots)), ctypes.c_int(D), _p(slots, _i32_p),
+                           _p(acc, _i32_p), _p(ck), _p(cck), _p(cs), _p(ss), ctypes.c_int(ss.shape[0]))
+    return cs, ss, int(code)

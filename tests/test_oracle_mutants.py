@@ -26,6 +26,7 @@ MUTANTS = {
     "chunk_decay_sign": ("intra += exp(gam[r] - gam[s]) * qk", "intra += exp(gam[s] - gam[r]) * qk"),
     "conv_tail_shift": ("int64_t pos = (int64_t)L + i;", "int64_t pos = (int64_t)L + i - 1;"),
     "verify_ckpt_window": ("int src = t + 1 - (K - 1) + j;", "int src = t - (K - 1) + j;"),
+    "commit_off_by_one": ("const int64_t t = (int64_t)i * D + (acc[i] - 1);", "const int64_t t = (int64_t)i * D + acc[i] % D;"),
 }
 
 

@@ -261,6 +261,50 @@ def test_verify_checkpoints_and_read_only_pools():
             np.testing.assert_allclose(out[i * D + t], o_e[t], rtol=1e-12, atol=1e-13)
 
 
+def test_commit_equals_extend_of_the_accepted_prefix():
+    """verify, then commit(a), leaves each slot as an extend over the request's first a draft
+    tokens would; a = 0 and padded requests leave their slots alone."""
+    D = 4
+    w = _layer_case([D] * 5, P=8, seed=11)
+    slots = w.state_indices.clone()
+    slots[3] = -1  # padding
+    accepted = np.array([1, 4, 0, 2, 3], dtype=np.int32)
+    out, ck, cck = O.verify(CFG, w.params, w.x, w.a, w.b, slots, D, w.conv_state, w.ssm_state)
+    cs, ss, code = O.commit(CFG, slots, accepted, D, ck, cck, w.conv_state, w.ssm_state)
+    assert code == 0
+    for i in range(5):
+        slot = int(slots[i])
+        if slot < 0:
+            continue
+        if accepted[i] == 0:
+            np.testing.assert_array_equal(ss[slot], O._f64(w.ssm_state)[slot])
+            np.testing.assert_array_equal(cs[slot], O._f64(w.conv_state)[slot])
+            continue
+        rows = slice(i * D, i * D + int(accepted[i]))
+        cu = torch.tensor([0, int(accepted[i])], dtype=torch.int32)
+        _, c_e, s_e = O.extend(CFG, w.params, w.x[rows], w.a[rows], w.b[rows], cu, slots[i:i + 1], w.conv_state,
+                               w.ssm_state)
+        np.testing.assert_allclose(ss[slot], s_e[slot], rtol=1e-12, atol=1e-13)
+        np.testing.assert_array_equal(cs[slot], c_e[slot])
+    # slots no request names are untouched
+    named = {int(x) for x in slots if int(x) >= 0}
+    for sl in range(8):
+        if sl not in named:
+            np.testing.assert_array_equal(ss[sl], O._f64(w.ssm_state)[sl])
+
+
+def test_commit_rejects_out_of_range_counts():
+    D = 3
+    w = _layer_case([D, D], P=4, seed=12)
+    out, ck, cck = O.verify(CFG, w.params, w.x, w.a, w.b, w.state_indices, D, w.conv_state, w.ssm_state)
+    cs, ss, code = O.commit(CFG, w.state_indices, np.array([D + 1, 2], dtype=np.int32), D, ck, cck, w.conv_state,
+                            w.ssm_state)
+    assert code == 3
+    s0 = int(w.state_indices[0])
+    np.testing.assert_array_equal(ss[s0], O._f64(w.ssm_state)[s0])  # the bad request wrote nothing
+    np.testing.assert_array_equal(ss[int(w.state_indices[1])], ck[1, 1])
+
+
 def test_head_independence_and_gqa_mapping():
     w = _layer_case([23, 9], seed=8)
     base, _, _ = _run(w)

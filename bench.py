@@ -1,15 +1,15 @@
 #!/usr/bin/env python
 """Benchmark of the GDN layer on B200: one step = one gdn_extend over the
 packed prefill batch + one gdn_decode over the decode batch + one gdn_verify
-over the verify batch (every mode of the layer), on synthetic inputs already
-resident in HBM.
+over the verify batch + one gdn_commit of each verify request's accepted
+prefix (every mode of the layer), on synthetic inputs already resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill32k|prefill262k]
     python bench.py --impl reference ...      # the fp64 CPU oracle on a bounded sample
 
 Prints one JSON line (rank 0).  `value` is prefill tokens/s over all ranks,
 from the device time of the gdn_extend launches inside the timed steps;
-decode and verify report their own state-traffic figures.  Multi-GPU runs are
+decode, verify and commit report their own state-traffic figures.  Multi-GPU runs are
 independent replicas (weak scaling): every rank runs its own batch, no
 collective touches the data path; the timing is the max over ranks.
 """
@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 METRIC = "GDN prefill tokens/s + decode state GB/s (frac. of roofline), 1×B200"
@@ -199,6 +200,15 @@ def decode_bytes(spec, B):
     return state, state + conv + io
 
 
+def commit_bytes(spec, accepted):
+    """Bytes one commit moves: for every request with a >= 1 accepted tokens, its checkpoint
+    (every head's fp32 state and the conv window) read and written into the slot."""
+    es = 2 if spec.dtype == torch.bfloat16 else 4
+    n = int((accepted > 0).sum())
+    state = 2 * spec.HV * spec.dk * spec.dv * 4 * n
+    return state, state + 2 * spec.conv_dim * 3 * es * n
+
+
 def verify_bytes(spec, B, D):
     es = 2 if spec.dtype == torch.bfloat16 else 4
     state = (1 + D) * spec.HV * spec.dk * spec.dv * 4 * B
@@ -361,6 +371,10 @@ def main():
     out_v = torch.empty(Bn * D, dspec.HV, dspec.dv, dtype=dspec.dtype, device=dev)
     ck = torch.empty(Bn, D, dspec.HV, dspec.dk, dspec.dv, dtype=torch.float32, device=dev)
     cck = torch.empty(Bn, D, dspec.conv_dim, 3, dtype=dspec.dtype, device=dev)
+    ws_c = gdn.alloc_workspace(gdn.gdn_commit_workspace_size(dcfg, Bn), dev)
+    # accepted draft tokens per request: seeded, 0 .. D
+    acc_h = torch.from_numpy(np.random.default_rng(5 + seed_off).integers(0, D + 1, Bn).astype(np.int32))
+    acc = acc_h.to(dev)
 
     def extend(x=pre.x, a=pre.a, b=pre.b, out=out_pre):
         gdn.gdn_extend(cfg, pre.params, x, a, b, pre.cu_seqlens, pre.state_indices, pre.has_initial_state,
@@ -373,12 +387,15 @@ def main():
         gdn.gdn_verify(dcfg, dv.params, x, a, b, dv.state_indices, D, dv.conv_state, dv.ssm_state, ck, cck, out,
                        ws_v)
 
+    def commit():
+        gdn.gdn_commit(dcfg, dv.state_indices, acc, D, ck, cck, dv.conv_state, dv.ssm_state, ws_c)
+
     EXT_K = ["chunk_map", "prep", "conv_tail", "intra", "state"]
     # gdn_extend's profiling marks: 0 start, 1 chunk table, 2 prep, 3 conv tail, 4 after the last intra
     # segment, 5 end; on the library's second stream 6 / 7 bracket the state-pass segments, which run
     # alongside the intra segments after the first
     EXT_EV = 8
-    n_ev = EXT_EV + 2 + 2
+    n_ev = EXT_EV + 2 + 2 + 2
 
     def make_events():
         return [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
@@ -391,8 +408,11 @@ def main():
             gdn.gdn_set_launch_events(ev[EXT_EV:EXT_EV + 2])
         decode()
         if ev is not None:
-            gdn.gdn_set_launch_events(ev[EXT_EV + 2:])
+            gdn.gdn_set_launch_events(ev[EXT_EV + 2:EXT_EV + 4])
         verify()
+        if ev is not None:
+            gdn.gdn_set_launch_events(ev[EXT_EV + 4:])
+        commit()
         if ev is not None:
             gdn.gdn_set_launch_events([])
 
@@ -400,6 +420,7 @@ def main():
         step()
     torch.cuda.synchronize()
     assert gdn.gdn_get_device_error(ws_pre) == 0 and gdn.gdn_get_device_error(ws_d) == 0
+    assert gdn.gdn_get_device_error(ws_v) == 0 and gdn.gdn_get_device_error(ws_c) == 0
 
     evs = [make_events() for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -428,14 +449,17 @@ def main():
                "intra": mean_span((3, 4)), "state": mean_span((6, 7))}
     kern_ms["decode"] = mean_span((EXT_EV, EXT_EV + 1))
     kern_ms["verify"] = mean_span((EXT_EV + 2, EXT_EV + 3))
+    kern_ms["commit"] = mean_span((EXT_EV + 4, EXT_EV + 5))
     ext_ms = max_over_ranks(mean_span((0, 5)), world, dev)
     dec_ms = max_over_ranks(kern_ms["decode"], world, dev)
     ver_ms = max_over_ranks(kern_ms["verify"], world, dev)
+    com_ms = max_over_ranks(kern_ms["commit"], world, dev)
 
     hbm, bf16, bf16_sus, peak_src = peaks()
     pw = prefill_work(spec, pre.T)
     st_dec, by_dec = decode_bytes(dspec, Bn)
     st_ver, by_ver = verify_bytes(dspec, Bn, D)
+    st_com, by_com = commit_bytes(dspec, acc_h)
     value = world * pre.T / (ext_ms * 1e-3)
 
     f16 = bf16
@@ -447,6 +471,7 @@ def main():
                  "peak": hbm, "peak_src": peak_src},
         "decode": {"bound": "hbm", "work": by_dec, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
         "verify": {"bound": "hbm", "work": by_ver, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
+        "commit": {"bound": "hbm", "work": by_com, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
     }
     for name, k in kernels.items():
         t = kern_ms[name] * 1e-3
@@ -545,8 +570,8 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
-            # extend: chunk table, prep, conv tail + intra and state per segment; decode; verify
-            "gpu_launches": args.steps * (3 + 2 * min(16, max(1, pre.T // 16384)) + 2),
+            # extend: chunk table, prep, conv tail + intra and state per segment; decode; verify; commit
+            "gpu_launches": args.steps * (3 + 2 * min(16, max(1, pre.T // 16384)) + 3),
             "clocks": clocks,
             "decode": {"ms": dec_ms, "requests_per_s": world * Bn / (dec_ms * 1e-3),
                        "state_gbs": world * st_dec / (dec_ms * 1e-3) / 1e9,
@@ -556,6 +581,9 @@ def main():
             "verify": {"ms": ver_ms, "state_gbs": world * st_ver / (ver_ms * 1e-3) / 1e9,
                        "total_gbs": world * by_ver / (ver_ms * 1e-3) / 1e9,
                        "frac_of_measured_hbm": by_ver / (ver_ms * 1e-3) / 1e9 / hbm},
+            "commit": {"ms": com_ms, "accepted_requests": int((acc_h > 0).sum()),
+                       "total_gbs": world * by_com / (com_ms * 1e-3) / 1e9,
+                       "frac_of_measured_hbm": by_com / (com_ms * 1e-3) / 1e9 / hbm},
             "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12, "roofline": prefill_roofline,
                         "gbs_algorithmic": pw["bytes"] / (ext_ms * 1e-3) / 1e9,
                         "kernel_ms": {k: kern_ms[k] for k in EXT_K}},

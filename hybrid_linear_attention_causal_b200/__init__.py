@@ -1,10 +1,11 @@
-"""B200 (sm_100a) Gated DeltaNet layer: extend / decode / verify behind a C ABI.
+"""B200 (sm_100a) Gated DeltaNet layer: extend / decode / verify / commit behind a C ABI.
 
 The compute lives in libgdn.so (csrc/, declared in include/gdn.h); this
 package holds its ctypes binding, the in-tree build step and seeded synthetic
 workloads.  Calls fail loudly when libgdn.so has not been built.
 """
 from .binding import (  # noqa: F401
+    GDN_DEVERR_ACCEPT_RANGE,
     GDN_DEVERR_SEQLENS,
     GDN_DEVERR_SLOT_RANGE,
     GDN_ERR_CUDA,
@@ -15,6 +16,8 @@ from .binding import (  # noqa: F401
     GdnConfig,
     GdnError,
     alloc_workspace,
+    gdn_commit,
+    gdn_commit_workspace_size,
     gdn_decode,
     gdn_decode_workspace_size,
     gdn_extend,

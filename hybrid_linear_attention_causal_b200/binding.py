@@ -23,6 +23,7 @@ GDN_ERR_CUDA = 4
 GDN_DEVERR_SLOT_RANGE = 0x1
 GDN_DEVERR_SEQLENS = 0x2
 GDN_DEVERR_TIMEOUT = 0x4
+GDN_DEVERR_ACCEPT_RANGE = 0x8
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 HEADER_BYTES = 512
@@ -115,6 +116,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_verify.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
         L.gdn_verify.restype = ctypes.c_int
+        L.gdn_commit_workspace_size.argtypes = [cfg_p, i32]
+        L.gdn_commit_workspace_size.restype = sz
+        L.gdn_commit.argtypes = [cfg_p, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, sz, vp]
+        L.gdn_commit.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_reset_device_error.argtypes = [vp, vp]
@@ -233,6 +238,23 @@ def gdn_verify(cfg: GdnConfig, params: dict, mixed_qkv, a, b, state_indices, D: 
         _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
     )
     _check(rc, "gdn_verify")
+
+
+def gdn_commit_workspace_size(cfg: GdnConfig, max_B: int) -> int:
+    return int(lib().gdn_commit_workspace_size(ctypes.byref(cfg.c()), max_B))
+
+
+def gdn_commit(cfg: GdnConfig, state_indices, accepted, D: int, state_ckpt, conv_ckpt, conv_state, ssm_state,
+               workspace, stream=None) -> None:
+    """Write the checkpoints of each request's last accepted draft token into its pool slot."""
+    B = int(state_indices.shape[0])
+    P = int(ssm_state.shape[0])
+    rc = lib().gdn_commit(
+        ctypes.byref(cfg.c()), _ptr(state_indices), _ptr(accepted), B, int(D), _ptr(state_ckpt), _ptr(conv_ckpt),
+        _ptr(conv_state), _ptr(ssm_state), P, _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream),
+    )
+    _check(rc, "gdn_commit")
 
 
 def gdn_get_device_error(workspace, stream=None) -> int:

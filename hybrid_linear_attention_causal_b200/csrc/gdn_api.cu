@@ -223,6 +223,42 @@ int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, const void* 
     return err == cudaSuccess ? GDN_OK : cuda_fail(err);
 }
 
+size_t gdn_commit_workspace_size(const gdn_config_t* cfg, int32_t max_B) {
+    if (check_cfg(cfg, nullptr) != GDN_OK || max_B < 0) return 0;
+    return gdn::kHeaderBytes;
+}
+
+int gdn_commit(const gdn_config_t* cfg, const int32_t* state_indices, const int32_t* accepted, int32_t B, int32_t D,
+               const float* state_ckpt, const void* conv_ckpt, void* conv_state, float* ssm_state, int32_t P,
+               void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    gdn::LayerDims d;
+    int rc = check_cfg(cfg, &d);
+    if (rc != GDN_OK) return rc;
+    if (B < 0 || P < 0 || D < 1 || D > gdn::kMaxVerifyDraft) return GDN_ERR_INVALID_ARG;
+    if (!workspace) return GDN_ERR_INVALID_ARG;
+    if (B == 0) return GDN_OK;
+    if (!state_indices || !accepted || !state_ckpt || !ssm_state) return GDN_ERR_INVALID_ARG;
+    if (conv_ckpt && !conv_state) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned(state_indices, accepted, state_ckpt, ssm_state, workspace)) return GDN_ERR_INVALID_ARG;
+    if (conv_ckpt && (!aligned16(conv_ckpt) || !aligned16(conv_state))) return GDN_ERR_INVALID_ARG;
+    if (workspace_bytes < (size_t)gdn::kHeaderBytes) return GDN_ERR_WORKSPACE;
+    gdn::CommitArgs p{};
+    p.d = d;
+    p.slots = state_indices;
+    p.accepted = accepted;
+    p.B = B;
+    p.D = D;
+    p.P = P;
+    p.state_ckpt = state_ckpt;
+    p.conv_ckpt = conv_ckpt;
+    p.conv_state = conv_state;
+    p.ssm_state = ssm_state;
+    p.conv_elem = cfg->dtype == GDN_DTYPE_BF16 ? 2 : 4;
+    p.hdr = static_cast<int32_t*>(workspace);
+    cudaError_t err = gdn::launch_commit(p, reinterpret_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? GDN_OK : cuda_fail(err);
+}
+
 int gdn_get_device_error(const void* workspace, int32_t* err_out, gdn_stream_t stream) {
     if (!workspace || !err_out) return GDN_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

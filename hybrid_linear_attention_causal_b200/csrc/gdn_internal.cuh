@@ -87,6 +87,19 @@ struct DecodeArgs {
     int32_t* hdr;       // workspace header (error word)
 };
 
+struct CommitArgs {
+    LayerDims d;
+    const int32_t* slots;     // [B]
+    const int32_t* accepted;  // [B], 0..D
+    int B, D, P;
+    const float* state_ckpt;  // [B, D, HV, dk, dv]
+    const void* conv_ckpt;    // [B, D, conv_dim, K-1], nullable
+    void* conv_state;         // [P, conv_dim, K-1]
+    float* ssm_state;         // [P, HV, dk, dv]
+    size_t conv_elem;         // bytes per conv element
+    int32_t* hdr;             // workspace header (error word)
+};
+
 struct ExtendArgs {
     LayerDims d;
     const float* A_log;
@@ -159,6 +172,7 @@ void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T);
 
 cudaError_t launch_decode(const DecodeArgs& args, int dtype, cudaStream_t s);
 cudaError_t launch_verify(const DecodeArgs& args, int dtype, cudaStream_t s);
+cudaError_t launch_commit(const CommitArgs& args, cudaStream_t s);
 cudaError_t launch_extend(const ExtendArgs& args, int dtype, cudaStream_t s);
 
 }  // namespace gdn

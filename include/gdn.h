@@ -12,6 +12,7 @@
  *   gdn_extend  EXTEND / MIXED / DRAFT_EXTEND: ragged packed-varlen prefill
  *   gdn_decode  DECODE / IDLE: one token per request (IDLE = zero requests)
  *   gdn_verify  TARGET_VERIFY: D draft tokens per request, state checkpoints
+ *   gdn_commit  the accepted prefix of a verify pass back into the pools
  *
  * What every mode computes, per request and value head h (qk head h / (HV/HK)):
  *   conv:  y_t = SiLU(sum_{j<K} w[c,j] x_{t-K+1+j}[c] (+ bias[c])) per channel c,
@@ -87,6 +88,7 @@ typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
 #define GDN_DEVERR_SLOT_RANGE 0x1 /* a state index >= P was skipped */
 #define GDN_DEVERR_SEQLENS 0x2    /* cu_seqlens not non-decreasing from 0 to T; the batch was skipped */
 #define GDN_DEVERR_TIMEOUT 0x4    /* a tensor-core wait gave up after its time limit; results are invalid */
+#define GDN_DEVERR_ACCEPT_RANGE 0x8 /* a commit's accepted count was outside 0..D; that request was skipped */
 
 /* element types */
 #define GDN_DTYPE_F32 0
@@ -218,6 +220,30 @@ GDN_API int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, cons
                const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt, void* out, void* workspace,
                size_t workspace_bytes, gdn_stream_t stream);
 
+/* Workspace bytes for gdn_commit (the error header only). */
+GDN_API size_t gdn_commit_workspace_size(const gdn_config_t* cfg, int32_t max_B);
+
+/*
+ * Speculative commit, the step after gdn_verify: request i accepted accepted[i]
+ * of its D draft tokens (accepted: device int32 [B]).  For accepted[i] >= 1
+ * its pool slot state_indices[i] receives the checkpoints of its last accepted
+ * token: ssm_state[slot] = state_ckpt[i, accepted[i] - 1] and, when conv_ckpt
+ * is non-NULL, conv_state[slot] = conv_ckpt[i, accepted[i] - 1] (layouts as
+ * gdn_verify writes them: state_ckpt [B, D, HV, dk, dv] fp32, conv_ckpt
+ * [B, D, conv_dim, K-1] in the cfg dtype).  The pool then holds what
+ * gdn_extend over the accepted tokens would have left.  accepted[i] == 0 leaves
+ * the slot untouched (verify never writes the pool).  A negative slot is
+ * padding and is skipped; a slot >= P raises GDN_DEVERR_SLOT_RANGE and an
+ * accepted count outside 0..D raises GDN_DEVERR_ACCEPT_RANGE, and that request
+ * is skipped.  1 <= D <= 16.  This is the accept step that follows the
+ * target-verify pass of page "SGLang GDN hybrid linear attention test matrix"
+ * (verification conventions: the speculative state buffer is committed for
+ * the accepted draft prefix).
+ */
+GDN_API int gdn_commit(const gdn_config_t* cfg, const int32_t* state_indices, const int32_t* accepted, int32_t B,
+                       int32_t D, const float* state_ckpt, const void* conv_ckpt, void* conv_state, float* ssm_state,
+                       int32_t P, void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
 /*
  * Reads the sticky device error word of `workspace` into *err_out (host).
  * Enqueues a device-to-host copy on `stream` and waits for that stream, so it
@@ -230,10 +256,10 @@ GDN_API int gdn_reset_device_error(void* workspace, gdn_stream_t stream);
 
 /*
  * Profiling aid (off by default).  With n > 0, the calling thread's later
- * gdn_extend / gdn_decode / gdn_verify calls record events[i] (each a
+ * gdn_extend / gdn_decode / gdn_verify / gdn_commit calls record events[i] (each a
  * cudaEvent_t created by the caller) at fixed points of the call; indices
  * >= n are not recorded.  n == 0 turns recording off.
- *   decode, verify: 0 before the kernel, 1 after it (on `stream`).
+ *   decode, verify, commit: 0 before the kernel, 1 after it (on `stream`).
  *   extend: on `stream`: 0 start, 1 after the chunk table, 2 after the
  *     conv + norm + gate pass, 3 after the conv-state update, 4 after the
  *     last intra-chunk segment, 5 end (second stream joined); on the

@@ -113,6 +113,30 @@ def test_decode_and_verify_argument_validation():
     assert _verify(c, ckpt=None) == gdn.GDN_ERR_INVALID_ARG
 
 
+def _commit(c, Bn=3, D=4, slots=FAKE, acc=FAKE, ckpt=FAKE, cck=None, cs=None, ss=FAKE, ws=FAKE, ws_bytes=256):
+    return B.lib().gdn_commit(ctypes.byref(c.c()), slots, acc, Bn, D, ckpt, cck, cs, ss, 8, ws, ws_bytes, None)
+
+
+def test_commit_argument_validation():
+    c = cfg()
+    assert gdn.gdn_commit_workspace_size(c, 256) == B.HEADER_BYTES
+    assert gdn.gdn_commit_workspace_size(cfg(head_k_dim=96), 256) == 0
+    assert _commit(c, Bn=0) == gdn.GDN_OK  # nothing to commit, nothing launched
+    assert _commit(c, Bn=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, D=0) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, D=17) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, slots=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, acc=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, ckpt=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, ss=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, cck=FAKE, cs=None) == gdn.GDN_ERR_INVALID_ARG  # a conv checkpoint needs the conv pool
+    assert _commit(c, cck=FAKE_MIS, cs=FAKE) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, acc=FAKE_MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, ws=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _commit(c, ws_bytes=16) == gdn.GDN_ERR_WORKSPACE
+    assert _commit(cfg(head_v_dim=256)) == gdn.GDN_ERR_UNSUPPORTED
+
+
 def test_error_helpers_reject_null():
     v = ctypes.c_int32(0)
     assert B.lib().gdn_get_device_error(None, ctypes.byref(v), None) == gdn.GDN_ERR_INVALID_ARG

@@ -207,3 +207,78 @@ def test_decode_and_verify_in_cuda_graph_with_padded_batch():
     g2.replay()
     torch.cuda.synchronize()
     assert same_bits(out2, out_v) and same_bits(ck2, ck_v) and same_bits(cck2, cck_v)
+
+
+def run_commit(wd, slots, accepted, D, ck, cck, conv, ssm):
+    cfg = gcfg(wd.spec)
+    ws = gdn.alloc_workspace(gdn.gdn_commit_workspace_size(cfg, int(slots.shape[0])), "cuda")
+    gdn.gdn_commit(cfg, slots, accepted, D, ck, cck, conv, ssm, ws)
+    torch.cuda.synchronize()
+    return gdn.gdn_get_device_error(ws)
+
+
+@pytest.mark.parametrize("HK,HV,dk,dv,dtype", [(2, 4, 64, 64, torch.float32), (4, 8, 128, 128, torch.bfloat16),
+                                               (1, 4, 128, 64, torch.bfloat16)])
+def test_commit_after_verify_equals_extend_of_accepted_prefix(HK, HV, dk, dv, dtype):
+    """verify, then commit: each slot holds the checkpoint of its last accepted token (a copy, bit
+    for bit) and matches the oracle's extend over the accepted prefix; zero accepted, padded and
+    unnamed slots keep their bits."""
+    spec = W.LayerSpec(HK=HK, HV=HV, dk=dk, dv=dv, dtype=dtype)
+    D = 4
+    slots = [5, -1, 0, 7, 2, 3]
+    accepted = [1, 3, 0, 4, 2, 4]
+    w = W.random_case(spec, [D] * len(slots), P=9, seed=dk + HV + 3, slots=slots)
+    wd = to_device(w)
+    out, ck, cck, err = run_verify(wd, wd.x, wd.a, wd.b, wd.state_indices, D, wd.conv_state, wd.ssm_state)
+    assert err == 0
+    conv, ssm = wd.conv_state.clone(), wd.ssm_state.clone()
+    acc = torch.tensor(accepted, dtype=torch.int32, device="cuda")
+    assert run_commit(wd, wd.state_indices, acc, D, ck, cck, conv, ssm) == 0
+    touched = set()
+    for i, (s, a) in enumerate(zip(slots, accepted)):
+        if s < 0 or a == 0:
+            continue
+        touched.add(s)
+        assert same_bits(ssm[s], ck[i, a - 1]) and same_bits(conv[s], cck[i, a - 1])
+        rows = torch.arange(i * D, i * D + a)
+        _, r_cs, r_ss = O.extend(ocfg(spec), w.params, w.x[rows], w.a[rows], w.b[rows],
+                                 torch.tensor([0, a], dtype=torch.int32), torch.tensor([s], dtype=torch.int32),
+                                 w.conv_state, w.ssm_state)
+        assert_state_close(f64(ssm[s]), r_ss[s], what=f"slot {s}")
+        assert same_bits(conv[s], torch.from_numpy(r_cs[s]).to(dtype))
+    for s in range(9):
+        if s not in touched:
+            assert same_bits(ssm[s], wd.ssm_state[s]) and same_bits(conv[s], wd.conv_state[s])
+
+
+def test_commit_full_size_pool_and_range_errors():
+    """The decode-verify workload's pool: 256 requests commit 0..4 accepted tokens; then counts and
+    slots out of range are flagged and skipped."""
+    w = W.decode_verify(device="cpu")
+    wd = to_device(w)
+    D = w.extra["D"]
+    xv, av, bv = w.extra["verify"]
+    out, ck, cck, err = run_verify(wd, xv.cuda(), av.cuda(), bv.cuda(), wd.state_indices, D, wd.conv_state,
+                                   wd.ssm_state)
+    assert err == 0
+    acc = torch.from_numpy(np.random.default_rng(3).integers(0, D + 1, w.N).astype(np.int32)).cuda()
+    conv, ssm = wd.conv_state.clone(), wd.ssm_state.clone()
+    assert run_commit(wd, wd.state_indices, acc, D, ck, cck, conv, ssm) == 0
+    expect_ssm, expect_conv = wd.ssm_state.clone(), wd.conv_state.clone()
+    for i in range(w.N):
+        a = int(acc[i])
+        if a > 0:
+            s = int(w.state_indices[i])
+            expect_ssm[s] = ck[i, a - 1]
+            expect_conv[s] = cck[i, a - 1]
+    assert same_bits(ssm, expect_ssm) and same_bits(conv, expect_conv)
+    # an accepted count past D and a slot past the pool: both flagged, neither written
+    bad_acc = acc.clone()
+    bad_acc[0] = D + 1
+    bad_slots = wd.state_indices.clone()
+    bad_slots[1] = w.ssm_state.shape[0]
+    conv2, ssm2 = wd.conv_state.clone(), wd.ssm_state.clone()
+    err = run_commit(wd, bad_slots, bad_acc, D, ck, cck, conv2, ssm2)
+    assert err == gdn.GDN_DEVERR_ACCEPT_RANGE | gdn.GDN_DEVERR_SLOT_RANGE
+    s0 = int(w.state_indices[0])
+    assert same_bits(ssm2[s0], wd.ssm_state[s0])

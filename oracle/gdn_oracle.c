@@ -525,3 +525,62 @@ int ora_commit(const ora_cfg* cfg, int B, int D, const int32_t* slots, const int
     }
     return rc;
 }
+
+/*
+ * Extend with one state checkpoint per sequence (prefix caching): sequence n
+ * names an exclusive absolute packed-row boundary ck_idx[n] with
+ * cu[n] <= ck_idx[n] <= cu[n+1] and a row ck_slot[n] of ck_states
+ * [num_ck, HV, dk, dv]; that row receives the state after rows
+ * cu[n] .. ck_idx[n]-1 (the state the sequence started from when the boundary
+ * is its first row), and ck_conv [num_ck, conv_dim, K-1] (nullable) the conv
+ * window there: the K-1 raw rows before the boundary, reaching into the
+ * sequence's starting conv window.  Page "flashinfer ... ssd_combined"
+ * (checkpoint_token_indices: one exclusive boundary per sequence, absolute for
+ * packed varlen, negative disables; checkpoint_state_slots: the row, negative
+ * disables; checkpoint_states: [num_checkpoints, nheads, headdim, dstate]).
+ * Padded sequences (slot < 0) capture nothing.  Everything else is ora_extend.
+ * Returns 4 when a boundary lies outside its sequence or a row >= num_ck
+ * (that sequence is skipped), else ora_extend's code.
+ */
+int ora_extend_ckpt(const ora_cfg* cfg, const double* A_log, const double* dt_bias, const double* conv_w,
+                    const double* conv_b, const double* x, const double* a, const double* b, const int32_t* cu,
+                    int N, const int32_t* slots, const int32_t* has_init, double* conv_state, double* ssm_state,
+                    int P, double* out, const int32_t* ck_idx, const int32_t* ck_slot, double* ck_states,
+                    double* ck_conv, int num_ck) {
+    const int HV = cfg->HV, dk = cfg->dk, dv = cfg->dv, K = cfg->K;
+    const int64_t CD = ora_conv_dim(cfg);
+    const int64_t sslot = (int64_t)HV * dk * dv, cslot = CD * (K - 1);
+    const int64_t T = cu[N];
+    double* st = (double*)malloc(sizeof(double) * (T > 0 ? T : 1) * sslot);
+    double* ss0 = (double*)malloc(sizeof(double) * (P > 0 ? P : 1) * sslot);
+    double* cs0 = (double*)malloc(sizeof(double) * (P > 0 ? P : 1) * cslot);
+    memcpy(ss0, ssm_state, sizeof(double) * P * sslot);
+    memcpy(cs0, conv_state, sizeof(double) * P * cslot);
+    int rc = ora_layer(cfg, A_log, dt_bias, conv_w, conv_b, x, a, b, cu, N, slots, has_init, conv_state, ssm_state,
+                       P, out, 0, NULL, st);
+    if (rc == 0) {
+        for (int n = 0; n < N; ++n) {
+            if (ck_idx[n] < 0 || ck_slot[n] < 0 || slots[n] < 0) continue;
+            if (ck_idx[n] < cu[n] || ck_idx[n] > cu[n + 1] || ck_slot[n] >= num_ck) { rc = 4; continue; }
+            const int64_t bnd = ck_idx[n];
+            const int init = has_init ? has_init[n] != 0 : 1;
+            double* dst = ck_states + (int64_t)ck_slot[n] * sslot;
+            if (bnd > cu[n]) memcpy(dst, st + (bnd - 1) * sslot, sizeof(double) * sslot);
+            else if (init) memcpy(dst, ss0 + (int64_t)slots[n] * sslot, sizeof(double) * sslot);
+            else memset(dst, 0, sizeof(double) * sslot);
+            if (ck_conv) {
+                double* cdst = ck_conv + (int64_t)ck_slot[n] * cslot;
+                for (int64_t c = 0; c < CD; ++c)
+                    for (int j = 0; j < K - 1; ++j) {
+                        const int64_t r = bnd - (K - 1) + j; /* raw row j of the window, index 0 oldest */
+                        double v;
+                        if (r >= cu[n]) v = x[r * CD + c];
+                        else v = init ? cs0[(int64_t)slots[n] * cslot + c * (K - 1) + (K - 1) + (r - cu[n])] : 0.0;
+                        cdst[c * (K - 1) + j] = v;
+                    }
+            }
+        }
+    }
+    free(st); free(ss0); free(cs0);
+    return rc;
+}

@@ -314,3 +314,37 @@ def commit(cfg: OracleCfg, state_indices, accepted, D: int, ckpt, conv_ckpt, con
     code = _L().ora_commit(ctypes.byref(c), ctypes.c_int(len(slots)), ctypes.c_int(D), _p(slots, _i32_p),
                            _p(acc, _i32_p), _p(ck), _p(cck), _p(cs), _p(ss), ctypes.c_int(ss.shape[0]))
     return cs, ss, int(code)
+
+
+def extend_ckpt(cfg: OracleCfg, params: dict, x, a, b, cu_seqlens, state_indices, conv_state, ssm_state,
+                ckpt_token_indices, ckpt_state_slots, num_ckpt: int, has_initial_state=None, want_conv: bool = True):
+    """extend that also captures, per sequence, the state (and conv window) at one exclusive absolute
+    packed-row boundary into row ckpt_state_slots[n] of the checkpoint buffers.
+
+    Returns (out, conv_state, ssm_state, ckpt_states [num_ckpt,HV,dk,dv] (zeros where nothing was
+    captured), ckpt_conv [num_ckpt,conv_dim,K-1] or None, code): code 0, or 4 when a boundary lies
+    outside its sequence or a row >= num_ckpt (that sequence is skipped).
+    """
+    A_log, dt_bias, conv_w, conv_b, x, a, b = _layer_args(cfg, params, x, a, b)
+    cu = _i32(cu_seqlens)
+    slots = _i32(state_indices)
+    hi = _i32(has_initial_state)
+    idx = _i32(ckpt_token_indices)
+    cks = _i32(ckpt_state_slots)
+    cs = _f64(conv_state).copy()
+    ss = _f64(ssm_state).copy()
+    N = len(slots)
+    T = int(cu[-1])
+    P = cs.shape[0]
+    out = np.zeros((T, cfg.HV, cfg.dv))
+    ck = np.zeros((num_ckpt, cfg.HV, cfg.dk, cfg.dv))
+    ckc = np.zeros((num_ckpt, cfg.conv_dim, cfg.K - 1)) if want_conv else None
+    c = cfg._c()
+    rc = _L().ora_extend_ckpt(
+        ctypes.byref(c), _p(A_log), _p(dt_bias), _p(conv_w), _p(conv_b), _p(x), _p(a), _p(b), _p(cu, _i32_p),
+        ctypes.c_int(N), _p(slots, _i32_p), _p(hi, _i32_p), _p(cs), _p(ss), ctypes.c_int(P), _p(out),
+        _p(idx, _i32_p), _p(cks, _i32_p), _p(ck), _p(ckc), ctypes.c_int(num_ckpt),
+    )
+    if rc not in (0, 4):
+        raise ValueError(f"oracle extend_ckpt rejected its arguments (code {rc})")
+    return out, cs, ss, ck, ckc, int(rc)

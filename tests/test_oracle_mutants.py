@@ -26,6 +26,8 @@ MUTANTS = {
     "chunk_decay_sign": ("intra += exp(gam[r] - gam[s]) * qk", "intra += exp(gam[s] - gam[r]) * qk"),
     "conv_tail_shift": ("int64_t pos = (int64_t)L + i;", "int64_t pos = (int64_t)L + i - 1;"),
     "verify_ckpt_window": ("int src = t + 1 - (K - 1) + j;", "int src = t - (K - 1) + j;"),
+    "ckpt_one_token_early": ("if (bnd > cu[n]) memcpy(dst, st + (bnd - 1) * sslot, sizeof(double) * sslot);",
+                             "if (bnd > cu[n] + 1) memcpy(dst, st + (bnd - 2) * sslot, sizeof(double) * sslot);"),
     "commit_off_by_one": ("const int64_t t = (int64_t)i * D + (acc[i] - 1);", "const int64_t t = (int64_t)i * D + acc[i] % D;"),
 }
 

@@ -305,6 +305,100 @@ def test_commit_rejects_out_of_range_counts():
     np.testing.assert_array_equal(ss[int(w.state_indices[1])], ck[1, 1])
 
 
+def test_extend_checkpoints_equal_extends_of_the_prefixes():
+    """A checkpoint at boundary b of sequence n is the slot state (and conv window) that extending
+    only rows cu[n] .. b-1 leaves; the boundary may sit at the start, mid chunk, on a chunk edge or at
+    the end; checkpointing leaves the outputs and pools of the extend unchanged."""
+    lens = [70, 130, 5, 64, 40]
+    w = _layer_case(lens, P=8, seed=13)
+    w.has_initial_state = torch.tensor([1, 0, 0, 1, 1], dtype=torch.int32)
+    cu = [int(v) for v in w.cu_seqlens]
+    offs = [37, 64, 0, 64, -1]  # boundary offsets inside each sequence; -1 disables
+    idx = torch.tensor([cu[n] + o if o >= 0 else -1 for n, o in enumerate(offs)], dtype=torch.int32)
+    rows_of = torch.tensor([2, 0, 3, 1, 4], dtype=torch.int32)
+    out, cs, ss, ck, ckc, code = O.extend_ckpt(CFG, w.params, w.x, w.a, w.b, w.cu_seqlens, w.state_indices,
+                                               w.conv_state, w.ssm_state, idx, rows_of, 5,
+                                               has_initial_state=w.has_initial_state)
+    assert code == 0
+    o_ref, cs_ref, ss_ref = _run(w)
+    np.testing.assert_array_equal(out, o_ref)
+    np.testing.assert_array_equal(ss, ss_ref)
+    np.testing.assert_array_equal(cs, cs_ref)
+    for n, o in enumerate(offs):
+        r = int(rows_of[n])
+        if o < 0:
+            assert not ck[r].any() and not ckc[r].any()
+            continue
+        sl = w.state_indices[n:n + 1]
+        rows = slice(cu[n], cu[n] + o)
+        _, c_p, s_p = O.extend(CFG, w.params, w.x[rows], w.a[rows], w.b[rows],
+                               torch.tensor([0, o], dtype=torch.int32), sl, w.conv_state, w.ssm_state,
+                               has_initial_state=w.has_initial_state[n:n + 1])
+        slot = int(sl[0])
+        if o == 0:  # nothing run: the slot as the sequence found it (zeros without an initial state)
+            init = bool(w.has_initial_state[n])
+            np.testing.assert_array_equal(ck[r], O._f64(w.ssm_state)[slot] * init)
+            np.testing.assert_array_equal(ckc[r], O._f64(w.conv_state)[slot] * init)
+        else:
+            np.testing.assert_allclose(ck[r], s_p[slot], rtol=1e-12, atol=1e-13)
+            np.testing.assert_array_equal(ckc[r], c_p[slot])
+    # the end of a sequence is its final state
+    n = 1
+    _, _, _, ck2, _, _ = O.extend_ckpt(CFG, w.params, w.x, w.a, w.b, w.cu_seqlens, w.state_indices, w.conv_state,
+                                       w.ssm_state, torch.tensor([-1, cu[2], -1, -1, -1], dtype=torch.int32),
+                                       torch.tensor([-1, 0, -1, -1, -1], dtype=torch.int32), 1,
+                                       has_initial_state=w.has_initial_state)
+    np.testing.assert_allclose(ck2[0], ss_ref[int(w.state_indices[n])], rtol=1e-12, atol=1e-13)
+
+
+def test_extend_checkpoints_prefix_cache_case():
+    """Cached prefixes (0, 64, 128) continued by extends (64, 65, 129) with a checkpoint on the last
+    chunk edge of each extend: the checkpoint equals the state after the whole-sequence prefix."""
+    prefix, ext = [0, 64, 128], [64, 65, 129]
+    full = _layer_case([p + e for p, e in zip(prefix, ext)], P=4, seed=14)
+    full.has_initial_state = torch.tensor([0, 1, 1], dtype=torch.int32)
+    xs, a_s, bs, pre_rows, ext_rows = [], [], [], [], []
+    cu_full = [int(v) for v in full.cu_seqlens]
+    for n in range(3):
+        pre_rows += list(range(cu_full[n], cu_full[n] + prefix[n]))
+        ext_rows += list(range(cu_full[n] + prefix[n], cu_full[n + 1]))
+    pr, er = torch.tensor(pre_rows, dtype=torch.long), torch.tensor(ext_rows, dtype=torch.long)
+    cu_pre = torch.tensor(np.cumsum([0] + prefix), dtype=torch.int32)
+    cu_ext = torch.tensor(np.cumsum([0] + ext), dtype=torch.int32)
+    _, cs1, ss1 = O.extend(CFG, full.params, full.x[pr], full.a[pr], full.b[pr], cu_pre, full.state_indices,
+                           full.conv_state, full.ssm_state, has_initial_state=full.has_initial_state)
+    # after the prefix the slots hold the prefix state; the extend starts from it
+    hi = torch.ones(3, dtype=torch.int32)
+    bnd = [int(cu_ext[n]) + (ext[n] // 64) * 64 for n in range(3)]
+    out, cs2, ss2, ck, ckc, code = O.extend_ckpt(CFG, full.params, full.x[er], full.a[er], full.b[er], cu_ext,
+                                                 full.state_indices, cs1, ss1, torch.tensor(bnd, dtype=torch.int32),
+                                                 torch.arange(3, dtype=torch.int32), 3, has_initial_state=hi)
+    assert code == 0
+    for n in range(3):
+        upto = prefix[n] + (ext[n] // 64) * 64
+        rows = slice(cu_full[n], cu_full[n] + upto)
+        _, c_w, s_w = O.extend(CFG, full.params, full.x[rows], full.a[rows], full.b[rows],
+                               torch.tensor([0, upto], dtype=torch.int32), full.state_indices[n:n + 1],
+                               full.conv_state, full.ssm_state, has_initial_state=full.has_initial_state[n:n + 1])
+        slot = int(full.state_indices[n])
+        np.testing.assert_allclose(ck[n], s_w[slot], rtol=1e-11, atol=1e-12)
+        np.testing.assert_array_equal(ckc[n], c_w[slot])
+
+
+def test_extend_checkpoint_ranges():
+    w = _layer_case([20, 30], P=4, seed=15)
+    cu = [int(v) for v in w.cu_seqlens]
+    assert w.has_initial_state is None  # every slot holds a starting state
+    *_, code = O.extend_ckpt(CFG, w.params, w.x, w.a, w.b, w.cu_seqlens, w.state_indices, w.conv_state,
+                             w.ssm_state, torch.tensor([cu[1] + 1, cu[1]], dtype=torch.int32),
+                             torch.tensor([0, 1], dtype=torch.int32), 2, has_initial_state=w.has_initial_state)
+    assert code == 4  # the first boundary lies in the second sequence
+    *_, ck, _, code = O.extend_ckpt(CFG, w.params, w.x, w.a, w.b, w.cu_seqlens, w.state_indices, w.conv_state,
+                                    w.ssm_state, torch.tensor([5, cu[1] + 3], dtype=torch.int32),
+                                    torch.tensor([0, 2], dtype=torch.int32), 2, has_initial_state=w.has_initial_state)
+    assert code == 4 and ck[0].any() and not ck[1].any()  # row 2 >= 2 rows: skipped
+
+
 def test_head_independence_and_gqa_mapping():
     w = _layer_case([23, 9], seed=8)
     base, _, _ = _run(w)

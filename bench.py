@@ -491,6 +491,30 @@ def main():
                         "frac": t_floor / (ext_ms * 1e-3), "tensor_frac": pw["flops"] / (ext_ms * 1e-3) / (f16 * 1e12),
                         "hbm_frac": pw["bytes"] / (ext_ms * 1e-3) / (hbm * 1e9)}
 
+    # Prefill state checkpoints (prefix caching), outside the timed step: the same batch with one
+    # checkpoint per sequence at a boundary three fifths into it (mid chunk in general)
+    cu_h = pre.cu_seqlens.to("cpu").to(torch.int64)
+    ck_idx = (cu_h[:-1] + (cu_h[1:] - cu_h[:-1]) * 3 // 5).to(torch.int32).to(dev)
+    ck_rows = torch.arange(pre.N, dtype=torch.int32, device=dev)
+    ck_states = torch.empty(pre.N, spec.HV, spec.dk, spec.dv, dtype=torch.float32, device=dev)
+    ck_conv = torch.empty(pre.N, spec.conv_dim, 3, dtype=spec.dtype, device=dev)
+
+    def extend_ck():
+        gdn.gdn_extend_checkpoints(cfg, pre.params, pre.x, pre.a, pre.b, pre.cu_seqlens, pre.state_indices,
+                                   pre.has_initial_state, pre.conv_state, pre.ssm_state, out_pre, ck_idx, ck_rows,
+                                   ck_states, ck_conv, ws_pre)
+
+    for _ in range(2):
+        extend_ck()
+    ck_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+    for e0, e1 in ck_ev:
+        e0.record()
+        extend_ck()
+        e1.record()
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_error(ws_pre) == 0
+    ck_ms = max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in ck_ev), world, dev)
+
     # End to end through the public API with pinned host buffers.  The layer is independent per
     # sequence, so the step runs one gdn_extend call per sequence and overlaps the host -> device
     # copy of sequence i + 1 and the device -> host copy of sequence i - 1 with the call for
@@ -584,6 +608,8 @@ def main():
             "commit": {"ms": com_ms, "accepted_requests": int((acc_h > 0).sum()),
                        "total_gbs": world * by_com / (com_ms * 1e-3) / 1e9,
                        "frac_of_measured_hbm": by_com / (com_ms * 1e-3) / 1e9 / hbm},
+            "prefill_checkpoints": {"ms": ck_ms, "checkpoints": pre.N, "vs_prefill": ck_ms / ext_ms,
+                                    "note": "one state checkpoint per sequence, mid chunk; timed outside the step"},
             "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12, "roofline": prefill_roofline,
                         "gbs_algorithmic": pw["bytes"] / (ext_ms * 1e-3) / 1e9,
                         "kernel_ms": {k: kern_ms[k] for k in EXT_K}},

@@ -6,6 +6,7 @@ workloads.  Calls fail loudly when libgdn.so has not been built.
 """
 from .binding import (  # noqa: F401
     GDN_DEVERR_ACCEPT_RANGE,
+    GDN_DEVERR_CKPT_RANGE,
     GDN_DEVERR_SEQLENS,
     GDN_DEVERR_SLOT_RANGE,
     GDN_ERR_CUDA,
@@ -21,6 +22,7 @@ from .binding import (  # noqa: F401
     gdn_decode,
     gdn_decode_workspace_size,
     gdn_extend,
+    gdn_extend_checkpoints,
     gdn_extend_static_scratch,
     gdn_extend_workspace_size,
     gdn_get_device_error,

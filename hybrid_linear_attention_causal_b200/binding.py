@@ -24,6 +24,7 @@ GDN_DEVERR_SLOT_RANGE = 0x1
 GDN_DEVERR_SEQLENS = 0x2
 GDN_DEVERR_TIMEOUT = 0x4
 GDN_DEVERR_ACCEPT_RANGE = 0x8
+GDN_DEVERR_CKPT_RANGE = 0x10
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 HEADER_BYTES = 512
@@ -110,6 +111,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_verify_workspace_size.restype = sz
         L.gdn_extend.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp, sz, vp]
         L.gdn_extend.restype = ctypes.c_int
+        L.gdn_extend_checkpoints.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp,
+                                             vp, vp, i32, vp, sz, vp]
+        L.gdn_extend_checkpoints.restype = ctypes.c_int
         L.gdn_extend_static_scratch.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, vp]
         L.gdn_extend_static_scratch.restype = ctypes.c_int
         L.gdn_decode.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]
@@ -196,6 +200,23 @@ def gdn_extend(cfg: GdnConfig, params: dict, mixed_qkv, a, b, cu_seqlens, state_
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
     )
     _check(rc, "gdn_extend")
+
+
+def gdn_extend_checkpoints(cfg: GdnConfig, params: dict, mixed_qkv, a, b, cu_seqlens, state_indices,
+                           has_initial_state, conv_state, ssm_state, out, ckpt_token_indices, ckpt_state_slots,
+                           ckpt_states, ckpt_conv, workspace, stream=None) -> None:
+    """gdn_extend that also captures each sequence's state (and conv window) at one exclusive absolute
+    packed-row boundary into row ckpt_state_slots[i] of ckpt_states / ckpt_conv (see include/gdn.h)."""
+    N = int(state_indices.shape[0])
+    T = int(mixed_qkv.shape[0])
+    P = int(ssm_state.shape[0])
+    rc = lib().gdn_extend_checkpoints(
+        ctypes.byref(cfg.c()), ctypes.byref(_params(params)), _ptr(mixed_qkv), _ptr(a), _ptr(b), _ptr(cu_seqlens),
+        N, T, _ptr(state_indices), _ptr(has_initial_state), _ptr(conv_state), _ptr(ssm_state), P, _ptr(out),
+        _ptr(ckpt_token_indices), _ptr(ckpt_state_slots), _ptr(ckpt_states), _ptr(ckpt_conv),
+        int(ckpt_states.shape[0]), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(rc, "gdn_extend_checkpoints")
 
 
 EXTEND_STATIC_SCRATCH_BYTES = 64 << 20

@@ -104,10 +104,13 @@ size_t gdn_verify_workspace_size(const gdn_config_t* cfg, int32_t max_B, int32_t
     return gdn::kHeaderBytes;
 }
 
-int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
-               const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
-               const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
-               void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+namespace {
+
+// gdn_extend and gdn_extend_checkpoints: `ck` carries the checkpoint arguments (all null for none)
+int extend_impl(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+                const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
+                const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
+                const gdn::ExtendArgs& ck, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
     gdn::LayerDims d;
     int rc = check_cfg(cfg, &d);
     if (rc != GDN_OK) return rc;
@@ -139,6 +142,11 @@ int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, const void* 
     e.conv_state = conv_state;
     e.ssm_state = ssm_state;
     e.out = out;
+    e.ck_idx = ck.ck_idx;
+    e.ck_row = ck.ck_row;
+    e.ck_states = ck.ck_states;
+    e.ck_conv = ck.ck_conv;
+    e.num_ck = ck.num_ck;
     // about one segment per 16384 packed rows (measured best on B200 among 4096 .. 40000): a
     // segment's intra work then hides the previous segment's state pass, and each launch's
     // ramp-up and tail stay small against its work
@@ -146,6 +154,36 @@ int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, const void* 
     gdn::carve_extend_workspace(e, workspace, N, T);
     cudaError_t err = gdn::launch_extend(e, cfg->dtype, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : cuda_fail(err);
+}
+
+}  // namespace
+
+int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+               const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
+               const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
+               void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    const gdn::ExtendArgs none{};
+    return extend_impl(cfg, params, mixed_qkv, a, b, cu_seqlens, N, T, state_indices, has_initial_state, conv_state,
+                       ssm_state, P, out, none, workspace, workspace_bytes, stream);
+}
+
+int gdn_extend_checkpoints(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+                           const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T,
+                           const int32_t* state_indices, const int32_t* has_initial_state, void* conv_state,
+                           float* ssm_state, int32_t P, void* out, const int32_t* ckpt_token_indices,
+                           const int32_t* ckpt_state_slots, float* ckpt_states, void* ckpt_conv, int32_t num_ckpt,
+                           void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (num_ckpt < 0 || !ckpt_token_indices || !ckpt_state_slots || !ckpt_states) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned(ckpt_token_indices, ckpt_state_slots, ckpt_states)) return GDN_ERR_INVALID_ARG;
+    if (ckpt_conv && !aligned16(ckpt_conv)) return GDN_ERR_INVALID_ARG;
+    gdn::ExtendArgs ck{};
+    ck.ck_idx = ckpt_token_indices;
+    ck.ck_row = ckpt_state_slots;
+    ck.ck_states = ckpt_states;
+    ck.ck_conv = ckpt_conv;
+    ck.num_ck = num_ckpt;
+    return extend_impl(cfg, params, mixed_qkv, a, b, cu_seqlens, N, T, state_indices, has_initial_state, conv_state,
+                       ssm_state, P, out, ck, workspace, workspace_bytes, stream);
 }
 
 int gdn_decode(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,

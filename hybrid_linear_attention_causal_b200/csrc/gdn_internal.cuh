@@ -117,6 +117,12 @@ struct ExtendArgs {
     void* conv_state;
     float* ssm_state;
     void* out;          // [T, HV, dv]
+    // optional state checkpoints, one per sequence (all null when not asked for)
+    const int32_t* ck_idx;  // [N] exclusive absolute packed-row boundary; < 0 disables
+    const int32_t* ck_row;  // [N] row of ck_states; < 0 disables
+    float* ck_states;       // [num_ck, HV, dk, dv]
+    void* ck_conv;          // [num_ck, conv_dim, K-1] (cfg dtype), nullable
+    int num_ck;
     // workspace carve-out
     int32_t* hdr;
     int4* chunk_tab;    // [max_chunks] {seq, first row, length, chunk index within seq}
@@ -130,8 +136,8 @@ struct ExtendArgs {
     uint16_t* VT;       // [max_chunks, HV, dv*C]   V^T fp16, K-major tile of dv rows x C
     float2* GB;         // [max_chunks, HV, C]      (g, beta); rows past the chunk end are zero
     // per (chunk, value head), written by the intra kernel, read by the state
-    // pass; the three tiles are tf32 values already in the tensor-core
-    // shared-memory layout, so the state pass copies them verbatim
+    // pass; the tiles are fp16 values already in the tensor-core shared-memory
+    // layout, so the state pass copies them verbatim
     uint16_t* WQ;       // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], fp16, K-major, 128 rows
     uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, fp16, K-major, C rows
     uint16_t* KT;       // [max_chunks, HV, C*dk]    K~ = diag(e^{gamma_n-gamma}) K, fp16, tile of C rows s
@@ -151,6 +157,17 @@ struct ExtendArgs {
 
 // True when chunk_map rejected the batch (it then publishes zero chunks).
 __device__ __forceinline__ bool batch_rejected(const ExtendArgs& p) { return p.hdr[kHdrNumChunks] == 0; }
+
+// The state checkpoint of sequence n: its boundary's offset inside the sequence (with *row set),
+// -1 when none is asked for, -2 when the boundary lies outside the sequence or the row is out of range.
+__device__ __forceinline__ int ckpt_offset(const ExtendArgs& p, int n, int* row) {
+    if (!p.ck_idx) return -1;
+    const int b = p.ck_idx[n], r = p.ck_row[n];
+    if (b < 0 || r < 0) return -1;
+    if (b < p.cu[n] || b > p.cu[n + 1] || r >= p.num_ck) return -2;
+    *row = r;
+    return b - p.cu[n];
+}
 
 // Intra-chunk step on tensor cores (gdn_intra_tc.cu) for the chunks of one
 // segment: persistent CTAs taking (chunk, qk head) items dynamically; for

@@ -23,6 +23,8 @@
 // (round to nearest): the parity bar leaves no room for bf16 rounding of q, k,
 // v, W, U or V', and truncating to tf32 instead of rounding fails it too.
 
+#include <cuda_fp16.h>
+
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
 
@@ -406,6 +408,115 @@ cudaError_t side_stream(SideStream** out) {
     return cudaSuccess;
 }
 
+// ---------------------------------------------------------------- state checkpoints
+
+// The conv window at each sequence's checkpoint boundary: the K-1 raw rows before it, reaching into
+// the sequence's starting conv window (launched before the conv-state update overwrites that).
+// Raises GDN_DEVERR_CKPT_RANGE for a boundary outside its sequence or a row out of range.
+template <typename T>
+__global__ void __launch_bounds__(256) ckpt_conv_kernel(ExtendArgs p) {
+    if (batch_rejected(p)) return;
+    const int n = blockIdx.x;
+    const int slot = p.slots[n];
+    if (slot < 0 || slot >= p.P) return;  // padded sequences capture nothing
+    int row = 0;
+    const int t = ckpt_offset(p, n, &row);
+    if (t == -2 && blockIdx.y == 0 && threadIdx.x == 0) raise_error(p.hdr, GDN_DEVERR_CKPT_RANGE);
+    if (t < 0 || !p.ck_conv) return;
+    const int cd = p.d.conv_dim;
+    const int c = blockIdx.y * 256 + threadIdx.x;
+    if (c >= cd) return;
+    const bool init = p.has_init ? p.has_init[n] != 0 : true;
+    const int t0 = p.cu[n], bnd = t0 + t;
+    const T* x = reinterpret_cast<const T*>(p.x);
+    const T* cs = reinterpret_cast<const T*>(p.conv_state) + ((size_t)slot * cd + c) * (kConvK - 1);
+    T* dst = reinterpret_cast<T*>(p.ck_conv) + ((size_t)row * cd + c) * (kConvK - 1);
+#pragma unroll
+    for (int j = 0; j < kConvK - 1; ++j) {
+        const int r = bnd - (kConvK - 1) + j;  // window entry j (0 oldest)
+        dst[j] = r >= t0 ? x[(size_t)r * cd + c] : (init ? cs[kConvK - 1 + (r - t0)] : from_f<T>(0.f));
+    }
+}
+
+// The state at each checkpoint boundary that does not sit on a chunk edge.  The state pass stored
+// the state S_c entering the boundary's chunk; the m rows of that chunk before the boundary add
+//   S_m = e^{gamma_{m-1}} S_c + sum_{s<m} e^{gamma_{m-1} - gamma_s} k_s v'_s^T,   v'_s = u_s - S_c^T w_s,
+// where u_s and w_s are rows of the chunk's U and W: those rows depend only on the chunk's rows up
+// to s (T = (I + A)^{-1} is lower triangular), so cutting the chunk at the boundary leaves them as
+// they are.  fp32 on CUDA cores, from the fp16 tiles the prefill already holds.  One CTA per
+// (sequence, value head, quarter of the dv columns); a sequence with no rows gets the state it
+// started from.
+constexpr int kCkptSplit = 4;  // CTAs per (sequence, value head), one group of dv columns each
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
+    if (batch_rejected(p)) return;
+    constexpr int DVS = DV / kCkptSplit;  // this CTA's columns j0 .. j0 + DVS - 1
+    const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * DVS, tid = threadIdx.x;
+    const int slot = p.slots[n];
+    if (slot < 0 || slot >= p.P) return;
+    int row = 0;
+    const int t = ckpt_offset(p, n, &row);
+    if (t < 0) return;
+    const LayerDims& d = p.d;
+    float* dst = p.ck_states + ((size_t)row * d.HV + h) * DK * DV;
+    const int len = p.cu[n + 1] - p.cu[n];
+    if (len == 0) {
+        const bool init = p.has_init ? p.has_init[n] != 0 : true;
+        const float* src = p.ssm_state + ((size_t)slot * d.HV + h) * DK * DV;
+        for (int e = tid; e < DK * DVS; e += 256) {
+            const size_t o = (size_t)(e / DVS) * DV + j0 + e % DVS;
+            dst[o] = init ? src[o] : 0.f;
+        }
+        return;
+    }
+    const int cl = min(t / C, (len + C - 1) / C - 1), m = t - C * cl;
+    if (m == 0) return;  // on a chunk edge: the state pass stored it
+    const size_t id = (size_t)p.seq_chunk0[n] + cl;
+    extern __shared__ __align__(16) float fsm[];
+    float* Sc = fsm;            // [DK][DVS] this CTA's columns of S_c
+    float* Wf = Sc + DK * DVS;  // [C][DK] rows s < m of W
+    float* Kf = Wf + C * DK;    // [C][DK] rows s < m of K
+    float* Vp = Kf + C * DK;    // [C][DVS] v'_s, this CTA's columns
+    float* coef = Vp + C * DVS; // [C] e^{gamma_{m-1} - gamma_s}
+    const char* WQg = reinterpret_cast<const char*>(p.WQ + (id * d.HV + h) * (2 * C * DK));
+    const char* KQg = reinterpret_cast<const char*>(p.KQ + (id * d.HK + h / d.G) * (2 * C * DK));
+    const char* Ug = reinterpret_cast<const char*>(p.U + (id * d.HV + h) * (DV * C));
+    const float* gm = p.gam + (id * d.HV + h) * C;
+    auto h2f = [](const char* q) { return __half2float(*reinterpret_cast<const __half*>(q)); };
+    for (int e = tid; e < DK * DVS / 4; e += 256) {
+        const int f = e / (DVS / 4), j4 = e % (DVS / 4);
+        reinterpret_cast<float4*>(Sc)[e] = reinterpret_cast<const float4*>(dst + (size_t)f * DV + j0)[j4];
+    }
+    for (int e = tid; e < m * DK; e += 256) {
+        const int sr = e / DK, f = e % DK;
+        Wf[e] = h2f(WQg + tc::kmajor_off16(sr, f, 2 * C));
+        Kf[e] = h2f(KQg + tc::kmajor_off16(sr, f, 2 * C));
+    }
+    if (tid < m) coef[tid] = expf(gm[m - 1] - gm[tid]);
+    __syncthreads();
+    for (int e = tid; e < m * DVS; e += 256) {  // v'_s[j] = u_s[j] - sum_f w_s[f] S_c[f][j]
+        const int sr = e / DVS, jl = e % DVS;
+        float acc = h2f(Ug + tc::kmajor_off16(j0 + jl, sr, DV));
+#pragma unroll 8
+        for (int f = 0; f < DK; ++f) acc = fmaf(-Wf[sr * DK + f], Sc[f * DVS + jl], acc);
+        Vp[e] = acc;
+    }
+    __syncthreads();
+    const float eg = expf(gm[m - 1]);
+    for (int e = tid; e < DK * DVS; e += 256) {
+        const int f = e / DVS, jl = e % DVS;
+        float acc = eg * Sc[e];
+        for (int sr = 0; sr < m; ++sr) acc = fmaf(coef[sr] * Kf[sr * DK + f], Vp[sr * DVS + jl], acc);
+        dst[(size_t)f * DV + j0 + jl] = acc;
+    }
+}
+
+template <int DK, int DV>
+constexpr size_t ckpt_finish_smem() {
+    return sizeof(float) * ((size_t)DK * (DV / kCkptSplit) + 2 * (size_t)C * DK + (size_t)C * (DV / kCkptSplit) + C);
+}
+
 // ---------------------------------------------------------------- 5. state pass
 // on tensor cores, in gdn_state_tc.cu
 
@@ -425,6 +536,10 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 2);
+    if (p.ck_idx) {  // the conv windows at the checkpoint boundaries, before the conv-state update
+        ckpt_conv_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 3);
@@ -441,6 +556,14 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     }
     mark_launch(s, 4);
     mark_launch(side->s, 7);
+    if (p.ck_idx) {  // the checkpoint states off the chunk edges, once the state pass stored the edges
+        constexpr size_t shm = ckpt_finish_smem<DK, DV>();
+        if ((e = cudaFuncSetAttribute(ckpt_finish_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)shm)) != cudaSuccess)
+            return e;
+        ckpt_finish_kernel<DK, DV><<<dim3(p.N, p.d.HV, kCkptSplit), 256, shm, side->s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(s, side->join, 0)) != cudaSuccess) return e;
     mark_launch(s, 5);

@@ -164,6 +164,20 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     float s[DK / 2];
 #pragma unroll
     for (int i = 0; i < DK / 2; ++i) s[i] = (init && rowv) ? Sg[(size_t)(half * (DK / 2) + i) * DV + j] : 0.f;
+    // a state checkpoint of this sequence: the state entering the chunk that holds its boundary is
+    // stored when that chunk comes up (a boundary at the very end belongs to the last chunk); the
+    // rows of that chunk before the boundary are added afterwards, off the chain
+    int ck_chunk = -1;
+    float* ck_dst = nullptr;
+    {
+        int row = 0;
+        const int t = ckpt_offset(p, nseq, &row);
+        const int len = p.cu[nseq + 1] - p.cu[nseq];
+        if (t >= 0 && len > 0) {
+            ck_chunk = c_first + min(t / C, (len + C - 1) / C - 1);
+            ck_dst = p.ck_states + ((size_t)row * HV + h) * DK * DV;
+        }
+    }
     int4 ch = p.chunk_tab[c_begin];
     float gl = p.gam[((size_t)c_begin * HV + h) * C + ch.z - 1];  // gamma_n of this chunk
     int4 ch_nx = c_begin + 1 < c_end ? p.chunk_tab[c_begin + 1] : ch;
@@ -256,6 +270,9 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 if (okl && id + 2 < c_end) fetch_wq(id + 2);  // this [W ; Qg] buffer is free again
             }
         } else if (warp < NCW) {
+            if (id == ck_chunk && rowv)  // the state entering the checkpoint's chunk: column j of S
+#pragma unroll
+                for (int i = 0; i < DK / 2; ++i) ck_dst[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
             if (id > c_begin) {  // the previous chunk's outputs leave while this chunk's first product runs
                 okl = __all_sync(0xffffffffu, tc::mbar_wait(bar_o, ph ^ 1u));
                 if (okl) {

@@ -10,6 +10,8 @@
  * extend and target-verify are the legal modes) map onto three entry points:
  *
  *   gdn_extend  EXTEND / MIXED / DRAFT_EXTEND: ragged packed-varlen prefill
+ *               (gdn_extend_checkpoints: the same, also capturing each
+ *               sequence's state at one token boundary, for prefix caching)
  *   gdn_decode  DECODE / IDLE: one token per request (IDLE = zero requests)
  *   gdn_verify  TARGET_VERIFY: D draft tokens per request, state checkpoints
  *   gdn_commit  the accepted prefix of a verify pass back into the pools
@@ -89,6 +91,7 @@ typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
 #define GDN_DEVERR_SEQLENS 0x2    /* cu_seqlens not non-decreasing from 0 to T; the batch was skipped */
 #define GDN_DEVERR_TIMEOUT 0x4    /* a tensor-core wait gave up after its time limit; results are invalid */
 #define GDN_DEVERR_ACCEPT_RANGE 0x8 /* a commit's accepted count was outside 0..D; that request was skipped */
+#define GDN_DEVERR_CKPT_RANGE 0x10  /* a checkpoint boundary outside its sequence or a row >= num_ckpt; skipped */
 
 /* element types */
 #define GDN_DTYPE_F32 0
@@ -148,6 +151,34 @@ GDN_API int gdn_extend(const gdn_config_t* cfg, const gdn_params_t* params, cons
                const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
                const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
                void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_extend that also captures, for prefix caching, each sequence's state at
+ * one token boundary.  ckpt_token_indices [N] (device int32) holds an
+ * exclusive ABSOLUTE packed-row boundary b_i with cu_seqlens[i] <= b_i <=
+ * cu_seqlens[i+1]: the captured state is the one after rows
+ * cu_seqlens[i] .. b_i - 1 (b_i == cu_seqlens[i] gives the state the sequence
+ * started from, b_i == cu_seqlens[i+1] its final state).  ckpt_state_slots [N]
+ * names the row of ckpt_states [num_ckpt, HV, dk, dv] (fp32) that receives it;
+ * ckpt_conv [num_ckpt, conv_dim, K-1] (cfg dtype, or NULL) receives the conv
+ * window at the boundary, the K-1 raw rows before it (reaching into the
+ * sequence's starting conv window).  A negative boundary or row disables the
+ * capture of that sequence, and padded sequences capture nothing; a boundary
+ * outside its sequence or a row >= num_ckpt raises GDN_DEVERR_CKPT_RANGE and
+ * skips it.  Two sequences naming the same row race.  Outputs and pools are
+ * exactly those of gdn_extend, with the same workspace size.  Page
+ * "flashinfer ... ssd_combined": checkpoint_token_indices (one exclusive
+ * boundary per sequence, absolute for packed varlen, negative disables),
+ * checkpoint_state_slots, checkpoint_states [num_checkpoints, nheads, headdim,
+ * dstate]; and the tracked-state checkpoints of the prefill test on page
+ * "SGLang GDN hybrid linear attention test matrix".
+ */
+GDN_API int gdn_extend_checkpoints(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv,
+                                   const void* a, const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T,
+                                   const int32_t* state_indices, const int32_t* has_initial_state, void* conv_state,
+                                   float* ssm_state, int32_t P, void* out, const int32_t* ckpt_token_indices,
+                                   const int32_t* ckpt_state_slots, float* ckpt_states, void* ckpt_conv,
+                                   int32_t num_ckpt, void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /* Size of the fixed device scratch behind gdn_extend_static_scratch. */
 #define GDN_EXTEND_STATIC_SCRATCH_BYTES (64u << 20)

@@ -113,6 +113,22 @@ def test_decode_and_verify_argument_validation():
     assert _verify(c, ckpt=None) == gdn.GDN_ERR_INVALID_ARG
 
 
+def _extend_ckpt(c, idx=FAKE, rows=FAKE, states=FAKE, cconv=None, num=4, x=FAKE):
+    return B.lib().gdn_extend_checkpoints(ctypes.byref(c.c()), _params(), x, FAKE, FAKE, FAKE, 2, 100, FAKE, None,
+                                          FAKE, FAKE, 4, FAKE, idx, rows, states, cconv, num, FAKE, 1 << 40, None)
+
+
+def test_extend_checkpoints_argument_validation():
+    c = cfg()
+    assert _extend_ckpt(c, idx=None) == gdn.GDN_ERR_INVALID_ARG  # the three checkpoint arrays go together
+    assert _extend_ckpt(c, rows=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend_ckpt(c, states=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend_ckpt(c, num=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend_ckpt(c, idx=FAKE_MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend_ckpt(c, cconv=FAKE_MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert _extend_ckpt(c, x=None) == gdn.GDN_ERR_INVALID_ARG  # and the extend's own checks still apply
+
+
 def _commit(c, Bn=3, D=4, slots=FAKE, acc=FAKE, ckpt=FAKE, cck=None, cs=None, ss=FAKE, ws=FAKE, ws_bytes=256):
     return B.lib().gdn_commit(ctypes.byref(c.c()), slots, acc, Bn, D, ckpt, cck, cs, ss, 8, ws, ws_bytes, None)
 

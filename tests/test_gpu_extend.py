@@ -263,3 +263,103 @@ def test_extend_captured_in_cuda_graph_matches_eager():
     g.replay()
     torch.cuda.synchronize()
     assert same_bits(out, eager[0]) and same_bits(conv, eager[1]) and same_bits(ssm, eager[2])
+
+
+def gpu_extend_ckpt(wd, idx, rows, num):
+    spec = wd.spec
+    cfg = gcfg(spec)
+    T, N = int(wd.x.shape[0]), int(wd.state_indices.shape[0])
+    ws = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, N, T), "cuda")
+    out = torch.full((T, spec.HV, spec.dv), float("nan"), dtype=spec.dtype, device="cuda")
+    conv, ssm = wd.conv_state.clone(), wd.ssm_state.clone()
+    cks = W.sentinel_fill_(torch.empty(num, spec.HV, spec.dk, spec.dv, device="cuda"))
+    ckc = W.sentinel_fill_(torch.empty(num, spec.conv_dim, spec.K - 1, dtype=spec.dtype, device="cuda"))
+    gdn.gdn_extend_checkpoints(cfg, wd.params, wd.x, wd.a, wd.b, wd.cu_seqlens, wd.state_indices,
+                               wd.has_initial_state, conv, ssm, out, idx.cuda(), rows.cuda(), cks, ckc, ws)
+    torch.cuda.synchronize()
+    return out, conv, ssm, cks, ckc, gdn.gdn_get_device_error(ws)
+
+
+CKPT_SHAPES = [(2, 2, 64, 64, torch.float32), (4, 8, 128, 128, torch.bfloat16), (2, 4, 128, 64, torch.bfloat16),
+               (1, 2, 64, 128, torch.bfloat16)]
+
+
+@pytest.mark.parametrize("HK,HV,dk,dv,dtype", CKPT_SHAPES)
+def test_extend_checkpoints_match_oracle(HK, HV, dk, dv, dtype):
+    """Boundaries at a sequence's start, mid chunk (first and later chunks), on a chunk edge, at the
+    end of a ragged sequence, on an empty sequence, disabled, and on a padded request: checkpoint
+    states within the state tolerance of the oracle's, conv windows bit-exact, and the extend's own
+    outputs and pools bit-identical to gdn_extend's."""
+    spec = W.LayerSpec(HK=HK, HV=HV, dk=dk, dv=dv, dtype=dtype)
+    lens = [130, 70, 0, 64, 200, 9, 100]
+    slots = [3, 0, 6, 1, -1, 4, 2]
+    w = W.random_case(spec, lens, P=8, seed=dk + 2 * dv + HV, slots=slots)
+    w.has_initial_state = torch.tensor([1, 0, 1, 1, 1, 0, 1], dtype=torch.int32)
+    cu = [int(v) for v in w.cu_seqlens]
+    offs = [37, 70, 0, 64, 100, 0, -1]  # boundary inside each sequence; -1 disables
+    idx = torch.tensor([cu[n] + o if o >= 0 else -1 for n, o in enumerate(offs)], dtype=torch.int32)
+    rows = torch.tensor([1, 0, 2, 5, 3, 4, 6], dtype=torch.int32)
+    wd = to_device(w)
+    out, conv, ssm, cks, ckc, err = gpu_extend_ckpt(wd, idx, rows, 7)
+    assert err == 0, f"device error word {err:#x}"
+    b_out, b_conv, b_ssm, _ = gpu_extend(wd)
+    assert same_bits(out, b_out) and same_bits(ssm, b_ssm) and same_bits(conv, b_conv)
+    r_out, r_cs, r_ss, r_ck, r_ckc, code = O.extend_ckpt(ocfg(spec), w.params, w.x, w.a, w.b, w.cu_seqlens,
+                                                         w.state_indices, w.conv_state, w.ssm_state, idx, rows, 7,
+                                                         has_initial_state=w.has_initial_state)
+    assert code == 0
+    for n, o in enumerate(offs):
+        r = int(rows[n])
+        if o < 0 or slots[n] < 0:  # nothing captured: the sentinel is still there
+            assert same_bits(cks[r], W.sentinel_fill_(torch.empty_like(cks[r])))
+            continue
+        assert_state_close(f64(cks[r]), r_ck[r], what=f"checkpoint of sequence {n}")
+        assert same_bits(ckc[r], torch.from_numpy(r_ckc[r]).to(dtype)), f"conv checkpoint of sequence {n}"
+
+
+def test_extend_checkpoints_cached_prefix_case():
+    """Cached prefixes (0, 64, 128) extended by (64, 65, 129) rows, head dim 128, checkpoints on the
+    last chunk edge and mid chunk: against the oracle's checkpoints of the whole sequences."""
+    spec = W.LayerSpec(HK=2, HV=4, dk=128, dv=128, dtype=torch.bfloat16)
+    prefix, ext = [0, 64, 128], [64, 65, 129]
+    full = W.random_case(spec, [p + e for p, e in zip(prefix, ext)], P=4, seed=31)
+    full.has_initial_state = torch.zeros(3, dtype=torch.int32)
+    cu_f = [int(v) for v in full.cu_seqlens]
+    pre_rows = [r for n in range(3) for r in range(cu_f[n], cu_f[n] + prefix[n])]
+    ext_rows = [r for n in range(3) for r in range(cu_f[n] + prefix[n], cu_f[n + 1])]
+    pr, er = torch.tensor(pre_rows, dtype=torch.long), torch.tensor(ext_rows, dtype=torch.long)
+    # the prefixes' states (oracle) in the slots, then the extends on the GPU from them
+    _, cs1, ss1 = O.extend(ocfg(spec), full.params, full.x[pr], full.a[pr], full.b[pr],
+                           torch.tensor(np.cumsum([0] + prefix), dtype=torch.int32), full.state_indices,
+                           full.conv_state, full.ssm_state, has_initial_state=full.has_initial_state)
+    w = W.Workload(full.name, spec, full.params, full.x[er], full.a[er], full.b[er],
+                   torch.tensor(np.cumsum([0] + ext), dtype=torch.int32), full.state_indices,
+                   torch.tensor([1 if p > 0 else 0 for p in prefix], dtype=torch.int32),
+                   torch.from_numpy(cs1).to(spec.dtype), torch.from_numpy(ss1).float(), {})
+    cu_e = [int(v) for v in w.cu_seqlens]
+    for offs in ([64, 64, 128], [13, 65, 100]):
+        idx = torch.tensor([cu_e[n] + offs[n] for n in range(3)], dtype=torch.int32)
+        out, conv, ssm, cks, ckc, err = gpu_extend_ckpt(to_device(w), idx, torch.arange(3, dtype=torch.int32), 3)
+        assert err == 0
+        for n in range(3):
+            upto = prefix[n] + offs[n]
+            rows = torch.arange(cu_f[n], cu_f[n] + upto)
+            _, c_w, s_w = O.extend(ocfg(spec), full.params, full.x[rows], full.a[rows], full.b[rows],
+                                   torch.tensor([0, upto], dtype=torch.int32), full.state_indices[n:n + 1],
+                                   full.conv_state, full.ssm_state, has_initial_state=full.has_initial_state[n:n + 1])
+            slot = int(full.state_indices[n])
+            assert_state_close(f64(cks[n]), s_w[slot], what=f"checkpoint {n} at {offs[n]}")
+            assert same_bits(ckc[n], torch.from_numpy(c_w[slot]).to(spec.dtype))
+
+
+def test_extend_checkpoint_range_errors_flagged():
+    spec = W.LayerSpec(HK=2, HV=4, dk=64, dv=64, dtype=torch.bfloat16)
+    w = W.random_case(spec, [20, 30], P=4, seed=32)
+    cu = [int(v) for v in w.cu_seqlens]
+    idx = torch.tensor([cu[1] + 1, cu[1] + 5], dtype=torch.int32)  # the first lies in the second sequence
+    out, conv, ssm, cks, ckc, err = gpu_extend_ckpt(to_device(w), idx, torch.tensor([0, 1], dtype=torch.int32), 2)
+    assert err == gdn.GDN_DEVERR_CKPT_RANGE
+    assert same_bits(cks[0], W.sentinel_fill_(torch.empty_like(cks[0])))
+    r = O.extend_ckpt(ocfg(spec), w.params, w.x, w.a, w.b, w.cu_seqlens, w.state_indices, w.conv_state,
+                      w.ssm_state, idx, torch.tensor([0, 1], dtype=torch.int32), 2)
+    assert_state_close(f64(cks[1]), r[3][1])

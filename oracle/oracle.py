@@ -348,3 +348,40 @@ def extend_ckpt(cfg: OracleCfg, params: dict, x, a, b, cu_seqlens, state_indices
     if rc not in (0, 4):
         raise ValueError(f"oracle extend_ckpt rejected its arguments (code {rc})")
     return out, cs, ss, ck, ckc, int(rc)
+
+
+def verify_tree(cfg: OracleCfg, params: dict, x, a, b, state_indices, parents, D: int, conv_state, ssm_state):
+    """D draft tokens per request forming a tree: parents[i, t] is -1 (the slot) or an earlier token.
+    Each token's output, state and conv window are those of running, from the slot, the path from the
+    root to that token (the EAGLE tree verification of page "SGLang GDN hybrid linear attention test
+    matrix").  Written as a replay of every path through ``extend`` (plain Python over small trees).
+
+    Returns (out [B*D,HV,dv], ckpt [B,D,HV,dk,dv], conv_ckpt [B,D,conv_dim,K-1]); padded requests get
+    zero outputs and zero checkpoints.
+    """
+    slots = _i32(state_indices)
+    B = len(slots)
+    par = _i32(parents).reshape(B, D)
+    cs = _f64(conv_state)
+    ss = _f64(ssm_state)
+    xs, as_, bs = _f64(x), _f64(a), _f64(b)
+    out = np.zeros((B * D, cfg.HV, cfg.dv))
+    ckpt = np.zeros((B, D, cfg.HV, cfg.dk, cfg.dv))
+    cck = np.zeros((B, D, cfg.conv_dim, cfg.K - 1))
+    for i in range(B):
+        slot = int(slots[i])
+        if slot < 0:
+            continue
+        for t in range(D):
+            path, nd = [], t
+            while nd >= 0:
+                assert par[i, nd] < nd, "a parent must precede its token"
+                path.append(nd)
+                nd = int(par[i, nd])
+            rows = [i * D + q for q in reversed(path)]
+            o, c1, s1 = extend(cfg, params, xs[rows], as_[rows], bs[rows], np.array([0, len(rows)], np.int32),
+                               np.array([0], np.int32), cs[slot:slot + 1], ss[slot:slot + 1])
+            out[i * D + t] = o[-1]
+            ckpt[i, t] = s1[0]
+            cck[i, t] = c1[0]
+    return out, ckpt, cck

@@ -399,6 +399,54 @@ def test_extend_checkpoint_ranges():
     assert code == 4 and ck[0].any() and not ck[1].any()  # row 2 >= 2 rows: skipped
 
 
+def test_verify_tree_chain_equals_verify_and_star_equals_decodes():
+    """A chain tree (parent t-1) is verify; a star (every parent the slot) is D independent decodes
+    from the slot."""
+    D = 5
+    w = _layer_case([D, D, D], P=5, seed=16)
+    slots = w.state_indices.clone()
+    slots[1] = -1
+    chain = np.tile(np.arange(-1, D - 1, dtype=np.int32), (3, 1))
+    o_t, ck_t, cc_t = O.verify_tree(CFG, w.params, w.x, w.a, w.b, slots, chain, D, w.conv_state, w.ssm_state)
+    o_v, ck_v, cc_v = O.verify(CFG, w.params, w.x, w.a, w.b, slots, D, w.conv_state, w.ssm_state)
+    np.testing.assert_allclose(o_t, o_v, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ck_t[[0, 2]], ck_v[[0, 2]], rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(cc_t[[0, 2]], cc_v[[0, 2]])
+    star = np.full((3, D), -1, dtype=np.int32)
+    o_s, ck_s, cc_s = O.verify_tree(CFG, w.params, w.x, w.a, w.b, slots, star, D, w.conv_state, w.ssm_state)
+    for i in (0, 2):
+        for t in range(D):
+            r = slice(i * D + t, i * D + t + 1)
+            o_d, c_d, s_d = O.decode(CFG, w.params, w.x[r], w.a[r], w.b[r], slots[i:i + 1], w.conv_state,
+                                     w.ssm_state)
+            sl = int(slots[i])
+            np.testing.assert_allclose(o_s[i * D + t], o_d[0], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(ck_s[i, t], s_d[sl], rtol=1e-12, atol=1e-13)
+            np.testing.assert_array_equal(cc_s[i, t], c_d[sl])
+
+
+def test_verify_tree_node_is_one_step_from_its_parent():
+    """In a branching tree every node's state is one decode step, with its own token, from its
+    parent's checkpoint (the slot for the root's children)."""
+    D = 7
+    w = _layer_case([D, D], P=3, seed=17)
+    parents = np.array([[-1, 0, 0, 1, 1, 2, -1], [-1, -1, 1, 2, 0, 4, 3]], dtype=np.int32)
+    o, ck, cc = O.verify_tree(CFG, w.params, w.x, w.a, w.b, w.state_indices, parents, D, w.conv_state,
+                              w.ssm_state)
+    for i in range(2):
+        sl = int(w.state_indices[i])
+        for t in range(D):
+            pool_s, pool_c = O._f64(w.ssm_state).copy(), O._f64(w.conv_state).copy()
+            pt = int(parents[i, t])
+            if pt >= 0:
+                pool_s[sl], pool_c[sl] = ck[i, pt], cc[i, pt]
+            r = slice(i * D + t, i * D + t + 1)
+            o_d, c_d, s_d = O.decode(CFG, w.params, w.x[r], w.a[r], w.b[r], w.state_indices[i:i + 1], pool_c, pool_s)
+            np.testing.assert_allclose(ck[i, t], s_d[sl], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(o[i * D + t], o_d[0], rtol=1e-11, atol=1e-12)
+            np.testing.assert_array_equal(cc[i, t], c_d[sl])
+
+
 def test_head_independence_and_gqa_mapping():
     w = _layer_case([23, 9], seed=8)
     base, _, _ = _run(w)

@@ -515,6 +515,29 @@ def main():
     assert gdn.gdn_get_device_error(ws_pre) == 0
     ck_ms = max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in ck_ev), world, dev)
 
+    # Draft-tree verify (EAGLE topk 2), outside the timed step: the verify batch with each request's D
+    # draft tokens as a tree whose parents are [-1, 0, 0, 1, ...] (two children per node)
+    tree = torch.tensor([-1] + [(t - 1) // 2 for t in range(1, D)], dtype=torch.int32)
+    parents = tree.repeat(Bn, 1).contiguous().to(dev)
+
+    def verify_tree():
+        gdn.gdn_verify_tree(dcfg, dv.params, xv, av, bv, dv.state_indices, parents, D, dv.conv_state, dv.ssm_state,
+                            ck, cck, out_v, ws_v)
+
+    for _ in range(2):
+        verify_tree()
+    tr_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+    for e0, e1 in tr_ev:
+        e0.record()
+        verify_tree()
+        e1.record()
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_error(ws_v) == 0
+    tr_ms = max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in tr_ev), world, dev)
+    # the tree's algorithmic bytes: verify's, plus one parent checkpoint read per branching token
+    n_branch = sum(1 for t in range(D) if int(tree[t]) != t - 1)
+    by_tree = by_ver + n_branch * dspec.HV * dspec.dk * dspec.dv * 4 * Bn
+
     # End to end through the public API with pinned host buffers.  The layer is independent per
     # sequence, so the step runs one gdn_extend call per sequence and overlaps the host -> device
     # copy of sequence i + 1 and the device -> host copy of sequence i - 1 with the call for
@@ -608,6 +631,9 @@ def main():
             "commit": {"ms": com_ms, "accepted_requests": int((acc_h > 0).sum()),
                        "total_gbs": world * by_com / (com_ms * 1e-3) / 1e9,
                        "frac_of_measured_hbm": by_com / (com_ms * 1e-3) / 1e9 / hbm},
+            "verify_tree": {"ms": tr_ms, "parents": tree.tolist(), "total_gbs": world * by_tree / (tr_ms * 1e-3) / 1e9,
+                            "frac_of_measured_hbm": by_tree / (tr_ms * 1e-3) / 1e9 / hbm,
+                            "note": "timed outside the step"},
             "prefill_checkpoints": {"ms": ck_ms, "checkpoints": pre.N, "vs_prefill": ck_ms / ext_ms,
                                     "note": "one state checkpoint per sequence, mid chunk; timed outside the step"},
             "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12, "roofline": prefill_roofline,

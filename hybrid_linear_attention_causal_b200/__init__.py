@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     GDN_DEVERR_CKPT_RANGE,
     GDN_DEVERR_SEQLENS,
     GDN_DEVERR_SLOT_RANGE,
+    GDN_DEVERR_TREE,
     GDN_ERR_CUDA,
     GDN_ERR_INVALID_ARG,
     GDN_ERR_UNSUPPORTED,
@@ -29,5 +30,6 @@ from .binding import (  # noqa: F401
     gdn_reset_device_error,
     gdn_set_launch_events,
     gdn_verify,
+    gdn_verify_tree,
     gdn_verify_workspace_size,
 )

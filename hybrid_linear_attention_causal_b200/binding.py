@@ -25,6 +25,7 @@ GDN_DEVERR_SEQLENS = 0x2
 GDN_DEVERR_TIMEOUT = 0x4
 GDN_DEVERR_ACCEPT_RANGE = 0x8
 GDN_DEVERR_CKPT_RANGE = 0x10
+GDN_DEVERR_TREE = 0x20
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 HEADER_BYTES = 512
@@ -120,6 +121,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_verify.argtypes = [cfg_p, par_p, vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
         L.gdn_verify.restype = ctypes.c_int
+        L.gdn_verify_tree.argtypes = [cfg_p, par_p, vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+        L.gdn_verify_tree.restype = ctypes.c_int
         L.gdn_commit_workspace_size.argtypes = [cfg_p, i32]
         L.gdn_commit_workspace_size.restype = sz
         L.gdn_commit.argtypes = [cfg_p, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, sz, vp]
@@ -276,6 +279,19 @@ def gdn_commit(cfg: GdnConfig, state_indices, accepted, D: int, state_ckpt, conv
         _stream(stream),
     )
     _check(rc, "gdn_commit")
+
+
+def gdn_verify_tree(cfg: GdnConfig, params: dict, mixed_qkv, a, b, state_indices, parents, D: int, conv_state,
+                    ssm_state, state_ckpt, conv_ckpt, out, workspace, stream=None) -> None:
+    """gdn_verify over a draft tree: parents [B, D] int32, -1 = the slot state, else an earlier token."""
+    B = int(state_indices.shape[0])
+    P = int(ssm_state.shape[0])
+    rc = lib().gdn_verify_tree(
+        ctypes.byref(cfg.c()), ctypes.byref(_params(params)), _ptr(mixed_qkv), _ptr(a), _ptr(b),
+        _ptr(state_indices), _ptr(parents), B, int(D), _ptr(conv_state), _ptr(ssm_state), P, _ptr(state_ckpt),
+        _ptr(conv_ckpt), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(rc, "gdn_verify_tree")
 
 
 def gdn_get_device_error(workspace, stream=None) -> int:

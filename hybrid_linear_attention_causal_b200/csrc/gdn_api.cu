@@ -221,10 +221,12 @@ int gdn_decode(const gdn_config_t* cfg, const gdn_params_t* params, const void* 
     return err == cudaSuccess ? GDN_OK : cuda_fail(err);
 }
 
-int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
-               const void* b, const int32_t* state_indices, int32_t B, int32_t D, const void* conv_state,
-               const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt, void* out, void* workspace,
-               size_t workspace_bytes, gdn_stream_t stream) {
+namespace {
+
+int verify_impl(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+                const void* b, const int32_t* state_indices, const int32_t* parents, int32_t B, int32_t D,
+                const void* conv_state, const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt,
+                void* out, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
     gdn::LayerDims d;
     int rc = check_cfg(cfg, &d);
     if (rc != GDN_OK) return rc;
@@ -255,10 +257,30 @@ int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, const void* 
     p.ssm_state = const_cast<float*>(ssm_state);
     p.state_ckpt = state_ckpt;
     p.conv_ckpt = conv_ckpt;
+    p.parents = parents;
     p.out = out;
     p.hdr = static_cast<int32_t*>(workspace);
     cudaError_t err = gdn::launch_verify(p, cfg->dtype, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : cuda_fail(err);
+}
+
+}  // namespace
+
+int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+               const void* b, const int32_t* state_indices, int32_t B, int32_t D, const void* conv_state,
+               const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt, void* out, void* workspace,
+               size_t workspace_bytes, gdn_stream_t stream) {
+    return verify_impl(cfg, params, mixed_qkv, a, b, state_indices, nullptr, B, D, conv_state, ssm_state, P,
+                       state_ckpt, conv_ckpt, out, workspace, workspace_bytes, stream);
+}
+
+int gdn_verify_tree(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+                    const void* b, const int32_t* state_indices, const int32_t* parents, int32_t B, int32_t D,
+                    const void* conv_state, const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt,
+                    void* out, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (!parents || !aligned16(parents)) return GDN_ERR_INVALID_ARG;
+    return verify_impl(cfg, params, mixed_qkv, a, b, state_indices, parents, B, D, conv_state, ssm_state, P,
+                       state_ckpt, conv_ckpt, out, workspace, workspace_bytes, stream);
 }
 
 size_t gdn_commit_workspace_size(const gdn_config_t* cfg, int32_t max_B) {

@@ -194,11 +194,23 @@ __global__ void __launch_bounds__(kNT) verify_kernel(DecodeArgs p) {
     float* usm = red + 2 * kNW * DV;        // [DV]
     float* qk = usm + DV;                   // [D]
     float* gate = qk + kMaxVerifyDraft;     // [D][G] x (e^g, beta)
+    __shared__ int par[kMaxVerifyDraft];    // draft-tree parent of each token (-1 = the slot)
+    __shared__ int tree_bad;
 
+    // the draft tree: a chain (parent t-1) unless parents are given; every parent must precede its token
+    if (tid == 0) tree_bad = 0;
+    __syncthreads();
+    if (tid < D) {
+        const int pt = p.parents ? p.parents[(size_t)req * D + tid] : tid - 1;
+        par[tid] = pt;
+        if (pt < -1 || pt >= tid) atomicOr(&tree_bad, 1);
+    }
+    __syncthreads();
     const int slot = p.slots[req];
     T* out0 = reinterpret_cast<T*>(p.out);
-    if (slot < 0 || slot >= p.P) {
+    if (slot < 0 || slot >= p.P || tree_bad) {
         if (slot >= p.P && tid == 0 && hk == 0) raise_error(p.hdr, GDN_DEVERR_SLOT_RANGE);
+        if (tree_bad && slot >= 0 && tid == 0 && hk == 0) raise_error(p.hdr, GDN_DEVERR_TREE);
         for (int t = 0; t < D; ++t) {
             T* o = out0 + (((size_t)req * D + t) * d.HV + (size_t)hk * G) * DV;
             for (int i = tid; i < G * DV; i += kNT) o[i] = from_f<T>(0.f);
@@ -210,23 +222,36 @@ __global__ void __launch_bounds__(kNT) verify_kernel(DecodeArgs p) {
         const T* w = reinterpret_cast<const T*>(p.conv_w);
         const T* bias = reinterpret_cast<const T*>(p.conv_b);
         T* cck = reinterpret_cast<T*>(p.conv_ckpt);
+        const T* xq = reinterpret_cast<const T*>(p.x) + (size_t)req * D * d.conv_dim;
         for (int i = tid; i < nch; i += kNT) {
             const int c = owned_channel<DK, DV>(d, hk, i);
-            T s0 = cs[c * 3 + 0], s1 = cs[c * 3 + 1], s2 = cs[c * 3 + 2];
             const float w0 = to_f(w[c * 4 + 0]), w1 = to_f(w[c * 4 + 1]), w2 = to_f(w[c * 4 + 2]),
                         w3 = to_f(w[c * 4 + 3]);
             const float bc = bias ? to_f(bias[c]) : 0.f;
             for (int t = 0; t < D; ++t) {
-                const T xr = reinterpret_cast<const T*>(p.x)[((size_t)req * D + t) * d.conv_dim + c];
-                float acc = fmaf(w0, to_f(s0), bc);
-                acc = fmaf(w1, to_f(s1), acc);
-                acc = fmaf(w2, to_f(s2), acc);
+                // the 3 raw rows before token t, newest first: its ancestors' rows, then the slot's
+                // window from its newest row back (on a chain these are rows t-1, t-2, t-3)
+                T win[3];
+                int nd = par[t], sk = 2;
+#pragma unroll
+                for (int q = 0; q < 3; ++q) {
+                    if (nd >= 0) {
+                        win[q] = xq[(size_t)nd * d.conv_dim + c];
+                        nd = par[nd];
+                    } else {
+                        win[q] = cs[c * 3 + sk];
+                        --sk;
+                    }
+                }
+                const T xr = xq[(size_t)t * d.conv_dim + c];
+                float acc = fmaf(w0, to_f(win[2]), bc);
+                acc = fmaf(w1, to_f(win[1]), acc);
+                acc = fmaf(w2, to_f(win[0]), acc);
                 acc = fmaf(w3, to_f(xr), acc);
                 y[t * nchp + i] = silu_f(acc);
-                s0 = s1; s1 = s2; s2 = xr;
-                if (cck) {
+                if (cck) {  // the window after token t, oldest first
                     T* dst = cck + (((size_t)req * D + t) * d.conv_dim + c) * 3;
-                    dst[0] = s0; dst[1] = s1; dst[2] = s2;
+                    dst[0] = win[1]; dst[1] = win[0]; dst[2] = xr;
                 }
             }
         }
@@ -252,7 +277,17 @@ __global__ void __launch_bounds__(kNT) verify_kernel(DecodeArgs p) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k)
             s[k] = __ldcs(reinterpret_cast<const float4*>(Sp + (size_t)(r0 + k * RSTEP) * DV) + cg);
+        int cur = -1;  // the tree node whose state the registers hold
         for (int t = 0; t < D; ++t) {
+            if (par[t] != cur) {  // a branch: continue from the parent's checkpoint (or the slot), which
+                                  // this very thread wrote (or read) element for element
+                const float* src =
+                    par[t] < 0 ? Sp : p.state_ckpt + (((size_t)req * D + par[t]) * d.HV + h) * DK * DV;
+#pragma unroll
+                for (int k = 0; k < RPT; ++k)
+                    s[k] = reinterpret_cast<const float4*>(src + (size_t)(r0 + k * RSTEP) * DV)[cg];
+            }
+            cur = t;
             const float* yt = y + t * nchp;
             T* orow = out0 + (((size_t)req * D + t) * d.HV + h) * DV;
             state_step<DK, DV, RPT, RSTEP, CG>(s, yt, yt + DK, yt + 2 * DK + j * DV, gate[2 * (t * G + j)],
@@ -284,6 +319,7 @@ cudaError_t launch_decode_t(const DecodeArgs& p, cudaStream_t s) {
 
 template <typename T, int DK, int DV>
 cudaError_t launch_verify_t(const DecodeArgs& p, cudaStream_t s) {
+    static_assert(kMaxVerifyDraft <= kNT, "one thread per draft token reads the tree");
     const int nchp = (2 * DK + p.d.G * DV + 3) & ~3;
     const size_t shm =
         sizeof(float) * ((size_t)p.D * nchp + 2 * kNW * DV + DV + kMaxVerifyDraft + 2 * (size_t)p.D * p.d.G);

@@ -83,6 +83,7 @@ struct DecodeArgs {
     float* ssm_state;   // decode: read/write; verify: read only
     float* state_ckpt;  // verify only
     void* conv_ckpt;    // verify only, nullable
+    const int32_t* parents;  // verify only: [B, D] draft-tree parents (-1 = slot), nullable = a chain
     void* out;          // [B*D, HV, dv]
     int32_t* hdr;       // workspace header (error word)
 };

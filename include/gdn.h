@@ -14,6 +14,7 @@
  *               sequence's state at one token boundary, for prefix caching)
  *   gdn_decode  DECODE / IDLE: one token per request (IDLE = zero requests)
  *   gdn_verify  TARGET_VERIFY: D draft tokens per request, state checkpoints
+ *               (gdn_verify_tree: the draft tokens form a tree given by parent indices)
  *   gdn_commit  the accepted prefix of a verify pass back into the pools
  *
  * What every mode computes, per request and value head h (qk head h / (HV/HK)):
@@ -92,6 +93,7 @@ typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
 #define GDN_DEVERR_TIMEOUT 0x4    /* a tensor-core wait gave up after its time limit; results are invalid */
 #define GDN_DEVERR_ACCEPT_RANGE 0x8 /* a commit's accepted count was outside 0..D; that request was skipped */
 #define GDN_DEVERR_CKPT_RANGE 0x10  /* a checkpoint boundary outside its sequence or a row >= num_ckpt; skipped */
+#define GDN_DEVERR_TREE 0x20        /* a draft tree parent outside -1 .. t-1; that request was treated as padded */
 
 /* element types */
 #define GDN_DTYPE_F32 0
@@ -250,6 +252,25 @@ GDN_API int gdn_verify(const gdn_config_t* cfg, const gdn_params_t* params, cons
                const void* b, const int32_t* state_indices, int32_t B, int32_t D, const void* conv_state,
                const float* ssm_state, int32_t P, float* state_ckpt, void* conv_ckpt, void* out, void* workspace,
                size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * TARGET_VERIFY over a draft TREE (EAGLE topk > 1): as gdn_verify, except that
+ * draft token t of request i continues from its parent parents[i*D + t]
+ * (device int32 [B, D]) instead of from token t-1: -1 is the slot state, any
+ * other parent must be an earlier token (0 <= parent < t).  Each token's
+ * state, output, state_ckpt and conv_ckpt entries are those of the path from
+ * the root to it; the conv window of a token is made of its ancestors' rows,
+ * then the slot's window.  parents[i*D + t] == t-1 for every t is exactly
+ * gdn_verify.  A parent outside -1 .. t-1 raises GDN_DEVERR_TREE and the
+ * request is treated as padded.  Same workspace as gdn_verify.  The EAGLE
+ * tree verification (topk = 2) of page "SGLang GDN hybrid linear attention
+ * test matrix".
+ */
+GDN_API int gdn_verify_tree(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv,
+                            const void* a, const void* b, const int32_t* state_indices, const int32_t* parents,
+                            int32_t B, int32_t D, const void* conv_state, const float* ssm_state, int32_t P,
+                            float* state_ckpt, void* conv_ckpt, void* out, void* workspace, size_t workspace_bytes,
+                            gdn_stream_t stream);
 
 /* Workspace bytes for gdn_commit (the error header only). */
 GDN_API size_t gdn_commit_workspace_size(const gdn_config_t* cfg, int32_t max_B);

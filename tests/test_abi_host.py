@@ -153,6 +153,16 @@ def test_commit_argument_validation():
     assert _commit(cfg(head_v_dim=256)) == gdn.GDN_ERR_UNSUPPORTED
 
 
+def test_verify_tree_argument_validation():
+    c = cfg()
+    tree = lambda parents=FAKE, D=4: B.lib().gdn_verify_tree(ctypes.byref(c.c()), _params(), FAKE, FAKE, FAKE, FAKE,
+                                                            parents, 3, D, FAKE, FAKE, 8, FAKE, None, FAKE, FAKE,
+                                                            256, None)
+    assert tree(parents=None) == gdn.GDN_ERR_INVALID_ARG  # a tree needs its parents
+    assert tree(parents=FAKE_MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert tree(D=17) == gdn.GDN_ERR_INVALID_ARG
+
+
 def test_error_helpers_reject_null():
     v = ctypes.c_int32(0)
     assert B.lib().gdn_get_device_error(None, ctypes.byref(v), None) == gdn.GDN_ERR_INVALID_ARG

@@ -282,3 +282,60 @@ def test_commit_full_size_pool_and_range_errors():
     assert err == gdn.GDN_DEVERR_ACCEPT_RANGE | gdn.GDN_DEVERR_SLOT_RANGE
     s0 = int(w.state_indices[0])
     assert same_bits(ssm2[s0], wd.ssm_state[s0])
+
+
+def run_verify_tree(wd, parents, D, want_conv_ckpt=True):
+    cfg = gcfg(wd.spec)
+    Bn = int(wd.state_indices.shape[0])
+    ws = gdn.alloc_workspace(gdn.gdn_verify_workspace_size(cfg, Bn, D), "cuda")
+    out = torch.full((Bn * D, wd.spec.HV, wd.spec.dv), float("nan"), dtype=wd.spec.dtype, device="cuda")
+    ck = W.sentinel_fill_(torch.empty(Bn, D, wd.spec.HV, wd.spec.dk, wd.spec.dv, device="cuda"))
+    cck = (W.sentinel_fill_(torch.empty(Bn, D, wd.spec.conv_dim, 3, dtype=wd.spec.dtype, device="cuda"))
+           if want_conv_ckpt else None)
+    gdn.gdn_verify_tree(cfg, wd.params, wd.x, wd.a, wd.b, wd.state_indices, parents.cuda(), D, wd.conv_state,
+                        wd.ssm_state, ck, cck, out, ws)
+    torch.cuda.synchronize()
+    return out, ck, cck, gdn.gdn_get_device_error(ws)
+
+
+@pytest.mark.parametrize("HK,HV,dk,dv,dtype", [(2, 4, 64, 64, torch.float32), (4, 8, 128, 128, torch.bfloat16),
+                                               (1, 4, 128, 64, torch.bfloat16)])
+def test_verify_tree_matches_oracle(HK, HV, dk, dv, dtype):
+    """Branching draft trees (EAGLE topk 2 style) against the oracle's path replay; pools untouched."""
+    spec = W.LayerSpec(HK=HK, HV=HV, dk=dk, dv=dv, dtype=dtype)
+    D = 7
+    slots = [2, -1, 0, 4]
+    w = W.random_case(spec, [D] * 4, P=5, seed=dk + dv + 7, slots=slots)
+    parents = torch.tensor([[-1, 0, 0, 1, 1, 2, 2], [-1, 0, 1, 2, 3, 4, 5], [-1, -1, 0, 1, 3, 4, 1],
+                            [-1, 0, 1, 0, 3, -1, 5]], dtype=torch.int32)
+    wd = to_device(w)
+    out, ck, cck, err = run_verify_tree(wd, parents, D)
+    assert err == 0
+    assert same_bits(wd.ssm_state, w.ssm_state.cuda()) and same_bits(wd.conv_state, w.conv_state.cuda())
+    r_out, r_ck, r_cck = O.verify_tree(ocfg(spec), w.params, w.x, w.a, w.b, w.state_indices, parents, D,
+                                       w.conv_state, w.ssm_state)
+    assert_out_close(f64(out), r_out)
+    for i, s in enumerate(slots):
+        if s < 0:
+            continue
+        for t in range(D):
+            assert_state_close(f64(ck[i, t]), r_ck[i, t], what=f"ckpt {i},{t}")
+            assert same_bits(cck[i, t], torch.from_numpy(r_cck[i, t]).to(dtype)), f"conv ckpt {i},{t}"
+
+
+def test_verify_tree_chain_is_verify_bit_for_bit_and_bad_parent_flagged():
+    spec = W.LayerSpec(HK=2, HV=4, dk=128, dv=128, dtype=torch.bfloat16)
+    D = 6
+    w = W.random_case(spec, [D] * 3, P=4, seed=33)
+    wd = to_device(w)
+    chain = torch.arange(-1, D - 1, dtype=torch.int32).repeat(3, 1)
+    t_out, t_ck, t_cck, err = run_verify_tree(wd, chain, D)
+    v_out, v_ck, v_cck, err2 = run_verify(wd, wd.x, wd.a, wd.b, wd.state_indices, D, wd.conv_state, wd.ssm_state)
+    assert err == 0 and err2 == 0
+    assert same_bits(t_out, v_out) and same_bits(t_ck, v_ck) and same_bits(t_cck, v_cck)
+    bad = chain.clone()
+    bad[1, 3] = 3  # a token cannot be its own parent
+    b_out, b_ck, _, err = run_verify_tree(wd, bad, D)
+    assert err == gdn.GDN_DEVERR_TREE
+    assert torch.all(b_out[D:2 * D] == 0)  # that request is treated as padded
+    assert same_bits(b_out[:D], v_out[:D]) and same_bits(b_ck[0], v_ck[0])

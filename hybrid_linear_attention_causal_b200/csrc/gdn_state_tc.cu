@@ -15,11 +15,14 @@
 // where Qg = diag(e^gamma) Q (q carries the output scale).  The chain from one
 // chunk's state to the next runs through the first product, V', the state
 // product and the update; everything else is kept off it:
-//   - a ninth warp only issues the MMAs and the bulk copies, so the eight
-//     compute warps never wait behind an issue loop; it queues the output
-//     product right behind the state product and waits for it only in the
-//     next chunk, after issuing that chunk's first product (the tensor core
-//     runs them in order), before refetching the Aqk tile;
+//   - a ninth warp only issues the MMAs, so the eight compute warps never
+//     wait behind an issue loop; it queues the output product right behind
+//     the state product (the tensor core runs them in order) and never waits
+//     for it;
+//   - a tenth warp issues every bulk copy: each tile buffer has a "free"
+//     barrier that the product reading it signals on completion (or the
+//     compute warps, for U^T), and the copier refills the buffer as soon as
+//     it completes, so no copy issue or wait sits on the chain;
 //   - the fp32 state lives in registers (each thread holds one half of row j
 //     of S^T), the state product goes to a fresh accumulator and the update
 //     is one FMA per element, written straight into the fp16 copy of S^T that
@@ -44,9 +47,26 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NCW = 8;               // compute warps
-constexpr int NT = (NCW + 1) * 32;   // + the issuing warp
-constexpr int ISSUER = NCW * 32;     // its lane 0
+constexpr int NCW = 8;                  // compute warps
+constexpr int NCHAIN = (NCW + 1) * 32;  // + the issuing warp: the threads on the state chain
+constexpr int ISSUER = NCW * 32;        // its lane 0
+constexpr int COPIER = NCHAIN;          // lane 0 of a tenth warp, which issues every bulk copy
+constexpr int NT = NCHAIN + 32;
+constexpr int kChainBarrier = 1;        // named barrier of the chain threads
+
+// barrier among the `n` threads of named barrier `id`; true when `pred` holds in all of them
+__device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
 
 // bf16 outputs are staged in shared memory and leave as 16-byte vectors while
 // the next state product runs; fp32 outputs (whose staging tile would not fit)
@@ -65,6 +85,9 @@ struct StateTcSmem {
     uint16_t vt[DV * C];      // V'^T = U^T - X^T, same layout: the A operand of the state and output products
     T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
     unsigned long long bar_x, bar_s, bar_o, bar_wq[2], bar_kt[2], bar_aq, bar_u;
+    // the copier's signals that a tile buffer is free again: the product reading it has completed
+    // (tensor-core commits), or V' has read U^T (one arrival per compute warp)
+    unsigned long long free_wq[2], free_kt[2], free_aq, free_u;
     uint32_t tmem_base;
 };
 
@@ -144,6 +167,12 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         }
         tc::mbar_init(bar_aq, 1);
         tc::mbar_init(bar_u, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(tc::smem_u32(&sm.free_wq[b]), 1);
+            tc::mbar_init(tc::smem_u32(&sm.free_kt[b]), 1);
+        }
+        tc::mbar_init(tc::smem_u32(&sm.free_aq), 1);
+        tc::mbar_init(tc::smem_u32(&sm.free_u), NCW);
         tc::fence_mbar_init();
         for (int id = c_begin; id < c_end && id < c_begin + 2; ++id) {
             fetch_wq(id);
@@ -233,6 +262,41 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 
     bool ok = true;
     int prev_t0 = 0, prev_n = 0;  // the chunk whose outputs are still in tensor memory
+    if (warp > NCW) {
+        // ---- the copier: each tile buffer is refilled as soon as the chain frees it, in the order
+        // the chain frees them ([W ; Qg] after the first product, U^T after V', K~ after the state
+        // product, Aqk after the output product).  The next release of a buffer needs the copy issued
+        // here, so none of these barriers can complete twice before this lane has seen the first.
+        if (tid == COPIER) {
+            for (int id = c_begin; id < c_end && ok; ++id) {
+                const int it = id - c_begin, bb = it & 1;
+                const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
+                if (id + 2 < c_end) {  // tiles two chunks ahead into L2, so their copies wait on L2 only
+                    const size_t nx = (size_t)(id + 2) * HV + h;
+                    tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
+                    tc::bulk_prefetch_l2(p.KT + nx * (DK * C), KT_BYTES);
+                    tc::bulk_prefetch_l2(p.AQ + nx * (C * C), AQ_BYTES);
+                    tc::bulk_prefetch_l2(u_src(id + 2), U_BYTES);
+                }
+                if (id + 2 < c_end) {
+                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_wq[bb]), pb);
+                    if (ok) fetch_wq(id + 2);
+                }
+                if (ok && id + 1 < c_end) {
+                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_u), ph);
+                    if (ok) fetch_u(id + 1);
+                }
+                if (ok && id + 2 < c_end) {
+                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_kt[bb]), pb);
+                    if (ok) fetch_kt(id + 2);
+                }
+                if (ok && id + 1 < c_end) {
+                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_aq), ph);
+                    if (ok) fetch_aq(id + 1);
+                }
+            }
+        }
+    } else
     for (int id = c_begin; id < c_end; ++id) {
         const uint32_t ph = (uint32_t)(id - c_begin) & 1u;
         const uint32_t tXO = tm + ph * 128;
@@ -253,21 +317,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 for (int k = 0; k < DK / 16; ++k)
                     tc::mma_f16_ta(tXO, tA + 8 * k, tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
                 tc::mma_commit(bar_x);
-            }
-            if (okl && id > c_begin) {  // the previous chunk's output product is done with the Aqk tile
-                okl = tc::mbar_wait(bar_o, ph ^ 1u);
-                if (okl) fetch_aq(id);
-            }
-            if (okl && id + 2 < c_end) {  // tiles two chunks ahead into L2, so their copies wait on L2 only
-                const size_t nx = (size_t)(id + 2) * HV + h;
-                tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
-                tc::bulk_prefetch_l2(p.KT + nx * (DK * C), KT_BYTES);
-                tc::bulk_prefetch_l2(p.AQ + nx * (C * C), AQ_BYTES);
-                tc::bulk_prefetch_l2(u_src(id + 2), U_BYTES);
-            }
-            if (okl) {
-                okl = tc::mbar_wait(bar_x, ph);
-                if (okl && id + 2 < c_end) fetch_wq(id + 2);  // this [W ; Qg] buffer is free again
+                tc::mma_commit(tc::smem_u32(&sm.free_wq[bb]));
             }
         } else if (warp < NCW) {
             if (id == ck_chunk && rowv)  // the state entering the checkpoint's chunk: column j of S
@@ -303,14 +353,15 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                         }
                 }
             }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(tc::smem_u32(&sm.free_u));  // this warp has read its U^T rows
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
-        ok = __syncthreads_and(okl);
+        ok = bar_and(kChainBarrier, NCHAIN, okl);
         if (!ok) break;
         tc::fence_after_sync();
         if (tid == ISSUER) {
-            if (id + 1 < c_end) fetch_u(id + 1);  // V' has read the U^T tile
             okl = tc::mbar_wait(bar_kt(bb), pb);
             if (okl) {  // Snew^T = V'^T K~, K~ (rows s) read MN-major
                 const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt[bb]);
@@ -319,6 +370,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 for (int k = 0; k < C / 16; ++k)
                     tc::mma_f16(tS, tc::desc_kmajor(av, DV, k), tc::desc_mnmajor16(bk, C, k), is, k > 0);
                 tc::mma_commit(bar_s);
+                tc::mma_commit(tc::smem_u32(&sm.free_kt[bb]));
             }
             if (okl) okl = tc::mbar_wait(bar_aq, ph);
             if (okl) {  // O^T += V'^T Aqk^T: queued behind the state product, off the state chain; the
@@ -329,9 +381,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 for (int k = 0; k < C / 16; ++k)
                     tc::mma_f16(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
                 tc::mma_commit(bar_o);
+                tc::mma_commit(tc::smem_u32(&sm.free_aq));
             }
-            if (okl) okl = tc::mbar_wait(bar_s, ph);
-            if (okl && id + 2 < c_end) fetch_kt(id + 2);  // this K~ buffer is free again
         } else if (warp < NCW) {
             if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
                                                           // state product runs meanwhile
@@ -354,7 +405,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             }
         }
         tc::fence_before_sync();
-        ok = __syncthreads_and(okl);
+        ok = bar_and(kChainBarrier, NCHAIN, okl);
         if (!ok) break;
         tc::fence_after_sync();
         prev_t0 = ch.y;
@@ -363,6 +414,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         ch_nx = ch_nx2;
         gl = gl_nx;
     }
+    ok = __syncthreads_and(ok);  // the chain, the copier and the idle lanes agree
     if (ok) {
         if (warp < NCW) {
             const uint32_t ph = (uint32_t)(c_end - 1 - c_begin) & 1u;
@@ -377,12 +429,22 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 #pragma unroll
                 for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
         }
+        if (tid == ISSUER) {  // the releases nobody waited for, so that none lands after the CTA is gone
+            const int n = c_end - c_begin;
+            for (int it = max(0, n - 2); it < n; ++it) {
+                tc::mbar_wait(tc::smem_u32(&sm.free_wq[it & 1]), (uint32_t)(it >> 1) & 1u);
+                tc::mbar_wait(tc::smem_u32(&sm.free_kt[it & 1]), (uint32_t)(it >> 1) & 1u);
+            }
+            tc::mbar_wait(tc::smem_u32(&sm.free_aq), (uint32_t)(n - 1) & 1u);
+        }
         if constexpr (kStageOut<T>) {
             __syncthreads();
             if (warp < NCW) send_out(prev_t0, prev_n);
         }
     } else if (tid == ISSUER) {
         raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+        // (the copier has stopped issuing: its loop ends at its first failed wait, and every
+        // wait of the chain threads above has returned)
         // let copies and products already in flight finish before the CTA's shared and tensor
         // memory go away
         for (uint32_t par = 0; par < 2; ++par) {
@@ -393,6 +455,11 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             tc::mbar_wait(bar_aq, par, 100000000ull);
             tc::mbar_wait(bar_o, par, 100000000ull);
             tc::mbar_wait(bar_u, par, 100000000ull);
+            for (int b = 0; b < 2; ++b) {
+                tc::mbar_wait(tc::smem_u32(&sm.free_wq[b]), par, 100000000ull);
+                tc::mbar_wait(tc::smem_u32(&sm.free_kt[b]), par, 100000000ull);
+            }
+            tc::mbar_wait(tc::smem_u32(&sm.free_aq), par, 100000000ull);
         }
     }
     tc::fence_before_sync();

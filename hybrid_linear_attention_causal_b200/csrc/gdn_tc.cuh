@@ -215,6 +215,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// One plain arrival on the mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
 // One arrival on the mbarrier that also expects `bytes` of async-copy traffic.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");

@@ -49,3 +49,40 @@ def test_pins_catch_planted_mistake(name):
             cwd=ROOT, env=env, capture_output=True, text=True, timeout=600,
         )
         assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
+
+
+SSD_SRC = os.path.join(ROOT, "oracle", "ssd_oracle.c")
+
+SSD_MUTANTS = {
+    "ssd_exclusive_output": ("acc += v * Ct[i];", "acc += (v - d * xt[p] * Bt[i]) * Ct[i];"),
+    "ssd_decay_sign": ("const double decay = exp(d * A[h]);", "const double decay = exp(-d * A[h]);"),
+    "ssd_group_interleaved": ("h / hpg;\n            double* S = (double*)malloc(sizeof(double) * ss);\n            if (init)",
+                              "h % G;\n            double* S = (double*)malloc(sizeof(double) * ss);\n            if (init)"),
+    "ssd_gate_no_silu": ("v *= zt[p] * ssd_sigmoid(zt[p]);", "v *= ssd_sigmoid(zt[p]);"),
+    "ssd_bias_after_softplus": ("double v = dt + bias;\n    if (c->dt_softplus) v = ssd_softplus(v);",
+                                "double v = dt;\n    if (c->dt_softplus) v = ssd_softplus(v);\n    v += bias;"),
+    "ssd_input_without_step": ("+ d * xt[p] * Bt[i];", "+ xt[p] * Bt[i];"),
+    "ssd_ckpt_one_token_late": ("t + 1 - cu[n] == ck", "t - cu[n] == ck"),
+    "ssd_skip_index": ("D[(int64_t)h * c->P + p]", "D[(int64_t)p * c->H + h]"),
+    "ssd_chunk_state_decay": ("const double w = exp(gl - gam[s]) * dd[s];", "const double w = exp(gl) * dd[s];"),
+    "ssd_chunk_carry_undecayed": ("yr[p] = exp(gam[r]) * inter;", "yr[p] = inter;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SSD_MUTANTS))
+def test_ssd_pins_catch_planted_mistake(name):
+    old, new = SSD_MUTANTS[name]
+    src = open(SSD_SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "mut.c")
+        so = os.path.join(d, "libmut.so")
+        open(c, "w").write(src.replace(old, new))
+        subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", so, c, "-lm"], check=True)
+        env = dict(os.environ, SSD_ORACLE_LIB=so)
+        r = subprocess.run(
+            [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+             os.path.join(ROOT, "tests", "test_ssd_oracle_pins.py")],
+            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600,
+        )
+        assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"

@@ -17,6 +17,9 @@ from .binding import (  # noqa: F401
     GDN_OK,
     GdnConfig,
     GdnError,
+    SsdConfig,
+    ssd_combined_fwd,
+    ssd_workspace_size,
     alloc_workspace,
     gdn_commit,
     gdn_commit_workspace_size,

@@ -28,6 +28,7 @@ GDN_DEVERR_CKPT_RANGE = 0x10
 GDN_DEVERR_TREE = 0x20
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
+GDN_DTYPE_F16 = 2
 HEADER_BYTES = 512
 MAX_VERIFY_DRAFT = 16
 
@@ -44,6 +45,20 @@ class GdnConfigC(ctypes.Structure):
         ("dtype", ctypes.c_int32),
         ("scale", ctypes.c_float),
         ("l2_eps", ctypes.c_float),
+    ]
+
+
+class SsdConfigC(ctypes.Structure):
+    _fields_ = [
+        ("nheads", ctypes.c_int32),
+        ("headdim", ctypes.c_int32),
+        ("dstate", ctypes.c_int32),
+        ("ngroups", ctypes.c_int32),
+        ("state_dtype", ctypes.c_int32),
+        ("dt_softplus", ctypes.c_int32),
+        ("d_per_dim", ctypes.c_int32),
+        ("dt_min", ctypes.c_float),
+        ("dt_max", ctypes.c_float),
     ]
 
 
@@ -127,6 +142,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_commit_workspace_size.restype = sz
         L.gdn_commit.argtypes = [cfg_p, vp, vp, i32, i32, vp, vp, vp, vp, i32, vp, sz, vp]
         L.gdn_commit.restype = ctypes.c_int
+        ssd_p = ctypes.POINTER(SsdConfigC)
+        L.ssd_workspace_size.argtypes = [ssd_p, i32, i32]
+        L.ssd_workspace_size.restype = sz
+        L.ssd_combined_fwd.argtypes = [ssd_p, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, i32,
+                                       vp, vp, sz, vp]
+        L.ssd_combined_fwd.restype = ctypes.c_int
         L.gdn_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_reset_device_error.argtypes = [vp, vp]
@@ -313,3 +334,45 @@ def gdn_set_launch_events(events) -> None:
             e.record()
     arr = (ctypes.c_void_p * max(n, 1))(*[e.cuda_event for e in events])
     _check(lib().gdn_set_launch_events(arr if n else None, n), "gdn_set_launch_events")
+
+
+_STATE_DTYPES = {torch.float32: GDN_DTYPE_F32, torch.bfloat16: GDN_DTYPE_BF16, torch.float16: GDN_DTYPE_F16}
+
+
+@dataclass(frozen=True)
+class SsdConfig:
+    """Shape and options of the Mamba2 SSD scan (include/ssd.h, ssd_config_t)."""
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    state_dtype: torch.dtype = torch.bfloat16
+    dt_softplus: bool = True
+    d_per_dim: bool = False
+    dt_limit: tuple = (0.0, float("inf"))
+
+    def c(self) -> SsdConfigC:
+        return SsdConfigC(self.nheads, self.headdim, self.dstate, self.ngroups, _STATE_DTYPES[self.state_dtype],
+                          int(self.dt_softplus), int(self.d_per_dim), float(self.dt_limit[0]),
+                          float(self.dt_limit[1]))
+
+
+def ssd_workspace_size(cfg: SsdConfig, max_N: int, max_T: int) -> int:
+    return int(lib().ssd_workspace_size(ctypes.byref(cfg.c()), max_N, max_T))
+
+
+def ssd_combined_fwd(cfg: SsdConfig, x, dt, A, B, C, cu_seqlens, out, workspace, D=None, z=None, dt_bias=None,
+                     initial_states=None, final_states=None, ckpt_token_indices=None, ckpt_state_slots=None,
+                     ckpt_states=None, stream=None) -> None:
+    """The Mamba2 SSD scan over packed sequences (include/ssd.h): out [T, H, P] and, when given,
+    final_states / ckpt_states [.., H, P, N] in cfg.state_dtype."""
+    N = int(cu_seqlens.shape[0]) - 1
+    T = int(x.shape[0])
+    num_ck = int(ckpt_states.shape[0]) if ckpt_states is not None else 0
+    rc = lib().ssd_combined_fwd(
+        ctypes.byref(cfg.c()), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(dt_bias),
+        _ptr(cu_seqlens), N, T, _ptr(initial_states), _ptr(final_states), _ptr(ckpt_token_indices),
+        _ptr(ckpt_state_slots), _ptr(ckpt_states), num_ck, _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream),
+    )
+    _check(rc, "ssd_combined_fwd")

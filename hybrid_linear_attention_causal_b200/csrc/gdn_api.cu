@@ -62,6 +62,10 @@ bool all_aligned(P... ptrs) {
 
 }  // namespace
 
+namespace gdn {
+int record_cuda_failure(cudaError_t e) { return cuda_fail(e); }
+}  // namespace gdn
+
 void gdn::mark_launch(cudaStream_t s, int i) {
     if (i < g_num_events) cudaEventRecord(g_events[i], s);
 }

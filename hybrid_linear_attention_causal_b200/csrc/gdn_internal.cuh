@@ -185,6 +185,9 @@ cudaError_t launch_state(const ExtendArgs& p, int seg, cudaStream_t s);
 // (see gdn_set_launch_events); a no-op otherwise.
 void mark_launch(cudaStream_t s, int i);
 
+// Records a CUDA failure for gdn_last_cuda_error and returns GDN_ERR_CUDA.
+int record_cuda_failure(cudaError_t e);
+
 size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max_chunks_out);
 void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T);
 

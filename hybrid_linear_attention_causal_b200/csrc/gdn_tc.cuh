@@ -73,7 +73,8 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int R, int s) {
 __device__ __forceinline__ uint64_t desc_mnmajor16(uint32_t base, int R, int s) {
     return make_desc(base + (uint32_t)s * 256, 128, (uint32_t)(R >> 3) * 128);
 }
-// instruction-descriptor bit: the B operand is MN-major (transposed)
+// instruction-descriptor bits: the A (bit 15) or B (bit 16) operand is MN-major (transposed)
+constexpr uint32_t kTransposeA = 1u << 15;
 constexpr uint32_t kTransposeB = 1u << 16;
 
 // 32-bit instruction descriptor: kind::tf32, fp32 accumulate, shape M x N.

@@ -289,3 +289,87 @@ def random_case(spec: LayerSpec, lengths, P: int, seed: int, device="cpu", init_
         f"case_{spec.HK}x{spec.HV}_d{spec.dk}x{spec.dv}_{'_'.join(map(str, lengths))}", spec, params, x, a, b,
         cu_from_lengths(lengths, device), slots, hi, conv_state, ssm_state,
     )
+
+
+# ---------------------------------------------------------------------------
+# Mamba2 SSD chunk-scan workloads
+# ---------------------------------------------------------------------------
+#
+# x, z, B, C and the raw steps dt ~ N(0, 1) in bf16; A = -U(a_lo, a_hi) (fp32;
+# the Mamba2 initialisation draws -A from U(1, 16)); dt_bias ~ U(-4, -1) (fp32),
+# so that softplus(dt + dt_bias) lies mostly in (0.005, 1); D ~ N(0, 1) in bf16
+# per head (or per head and dim); random initial states ~ N(0, 0.02) in the
+# state dtype.
+
+
+@dataclass(frozen=True)
+class SsdSpec:
+    """Shape of one Mamba2 SSD layer."""
+
+    H: int  # heads
+    P: int  # head dim
+    N: int  # state dim
+    G: int  # groups of B / C
+    state_dtype: torch.dtype = torch.bfloat16
+
+
+@dataclass
+class SsdWorkload:
+    name: str
+    spec: SsdSpec
+    x: torch.Tensor       # [T, H, P] bf16
+    dt: torch.Tensor      # [T, H] bf16
+    A: torch.Tensor       # [H] fp32
+    B: torch.Tensor       # [T, G, N] bf16
+    C: torch.Tensor       # [T, G, N] bf16
+    D: torch.Tensor | None
+    z: torch.Tensor | None
+    dt_bias: torch.Tensor | None
+    cu: torch.Tensor      # [Nseq + 1] int32
+    init: torch.Tensor | None  # [Nseq, H, P, N] state dtype
+    lengths: list = field(default_factory=list)
+
+    @property
+    def T(self) -> int:
+        return int(self.x.shape[0])
+
+    def to(self, device) -> "SsdWorkload":
+        mv = lambda t: None if t is None else t.to(device)
+        return SsdWorkload(self.name, self.spec, mv(self.x), mv(self.dt), mv(self.A), mv(self.B), mv(self.C),
+                           mv(self.D), mv(self.z), mv(self.dt_bias), mv(self.cu), mv(self.init), list(self.lengths))
+
+
+def ssd_case(spec: SsdSpec, lengths, seed: int, device="cpu", with_D: bool = True, d_per_dim: bool = False,
+             with_z: bool = True, with_bias: bool = True, init_random: bool = True, a_range=(1.0, 16.0)) -> SsdWorkload:
+    """A seeded SSD case; tensors drawn in the order x, z, B, C, dt, A, dt_bias, D, init."""
+    g = _gen(seed, device)
+    T, H, P, N, G = sum(int(n) for n in lengths), spec.H, spec.P, spec.N, spec.G
+    bf = torch.bfloat16
+    x = torch.randn(T, H, P, generator=g, device=device).to(bf)
+    z = torch.randn(T, H, P, generator=g, device=device).to(bf)
+    B = torch.randn(T, G, N, generator=g, device=device).to(bf)
+    C = torch.randn(T, G, N, generator=g, device=device).to(bf)
+    dt = torch.randn(T, H, generator=g, device=device).to(bf)
+    A = -(a_range[0] + (a_range[1] - a_range[0]) * torch.rand(H, generator=g, device=device))
+    dt_bias = -4.0 + 3.0 * torch.rand(H, generator=g, device=device)
+    D = torch.randn((H, P) if d_per_dim else (H,), generator=g, device=device).to(bf)
+    init = (math.sqrt(0.02) * torch.randn(len(lengths), H, P, N, generator=g, device=device)).to(spec.state_dtype)
+    return SsdWorkload(
+        f"ssd_{H}h_p{P}_n{N}_g{G}_{'_'.join(map(str, lengths))}", spec, x, dt, A.float(), B, C,
+        D if with_D else None, z if with_z else None, dt_bias.float() if with_bias else None,
+        cu_from_lengths(lengths, device), init if init_random else None, list(lengths),
+    )
+
+
+SPEC_SSD = SsdSpec(H=128, P=64, N=128, G=8)
+
+
+def ssd_prefill(device="cpu", seed: int = 5, total: int = 32768, nseq: int = 8) -> SsdWorkload:
+    """The SSD bench workload: a Mamba2 layer of 128 heads (head dim 64, state 128, 8 groups) over
+    nseq packed sequences with lengths log-uniform in [512, 16384] summing to ``total`` (the same
+    length recipe as the large GDN prefill), bf16 states continuing from random initial states."""
+    g = _gen(seed, device)
+    lens = loguniform_lengths(nseq, 512, 16384, total, g)
+    w = ssd_case(SPEC_SSD, lens, seed + 1000, device=device)
+    w.name = f"ssd_prefill_{nseq}seq_{total}tok"
+    return w

@@ -98,6 +98,7 @@ typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
 /* element types */
 #define GDN_DTYPE_F32 0
 #define GDN_DTYPE_BF16 1
+#define GDN_DTYPE_F16 2 /* fp16: a state storage type of ssd.h only */
 
 typedef struct {
     int32_t num_qk_heads; /* HK */

@@ -11,20 +11,20 @@ import hybrid_linear_attention_causal_b200 as gdn
 from hybrid_linear_attention_causal_b200 import binding as B
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gdn.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("gdn.h", "ssd.h")]
 
 FAKE = 0x10000  # aligned, never dereferenced by the host-side validation
 FAKE_MIS = 0x10004
 
 
 def declared_symbols():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+    text = "".join(open(h).read() for h in HEADERS)
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b((?:gdn|ssd)_\w+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_symbol():
     syms = declared_symbols()
-    assert len(syms) >= 10
+    assert len(syms) >= 12 and "ssd_combined_fwd" in syms
     L = B.lib()
     for s in syms:
         assert hasattr(L, s), f"libgdn.so does not export {s}"
@@ -177,3 +177,36 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(ValueError):
         gdn.gdn_decode(c, {"A_log": t, "dt_bias": t, "conv_w": t}, t, t, t, torch.zeros(1, dtype=torch.int32), t, t,
                        t, t)
+
+
+def _ssd_call(c, x=FAKE, dt=FAKE, A=FAKE, Bm=FAKE, C=FAKE, D=None, z=None, bias=None, cu=FAKE, N=2, T=100,
+              init=None, fin=None, ck=(None, None, None), num_ck=0, out=FAKE, ws=FAKE, wsb=4096):
+    return B.lib().ssd_combined_fwd(ctypes.byref(c.c()), x, dt, A, Bm, C, D, z, bias, cu, N, T, init, fin, ck[0],
+                                    ck[1], ck[2], num_ck, out, ws, wsb, None)
+
+
+def test_ssd_workspace_and_argument_validation():
+    c = gdn.SsdConfig(nheads=8, headdim=64, dstate=128, ngroups=2)
+    assert gdn.ssd_workspace_size(c, 8, 32768) == B.HEADER_BYTES
+    assert B.lib().ssd_workspace_size(None, 1, 1) == 0
+    inv, uns, wsp = gdn.GDN_ERR_INVALID_ARG, gdn.GDN_ERR_UNSUPPORTED, gdn.GDN_ERR_WORKSPACE
+    assert _ssd_call(gdn.SsdConfig(nheads=6, headdim=64, dstate=128, ngroups=4)) == inv   # H % G
+    assert _ssd_call(gdn.SsdConfig(nheads=8, headdim=32, dstate=128, ngroups=2)) == uns   # headdim
+    assert _ssd_call(gdn.SsdConfig(nheads=8, headdim=64, dstate=96, ngroups=2)) == uns    # dstate
+    assert _ssd_call(gdn.SsdConfig(nheads=8, headdim=64, dstate=128, ngroups=2, dt_limit=(1.0, 0.5))) == inv
+    assert _ssd_call(c, N=-1) == inv
+    assert _ssd_call(c, x=None) == inv
+    assert _ssd_call(c, cu=None) == inv
+    assert _ssd_call(c, A=None) == inv
+    assert _ssd_call(c, out=None) == inv
+    assert _ssd_call(c, x=FAKE_MIS) == inv
+    assert _ssd_call(c, z=FAKE_MIS) == inv
+    assert _ssd_call(c, init=FAKE_MIS) == inv
+    assert _ssd_call(c, ck=(FAKE, None, FAKE), num_ck=1) == inv           # checkpoint arguments in part
+    assert _ssd_call(c, ck=(FAKE, FAKE, FAKE), num_ck=-1) == inv
+    assert _ssd_call(c, ws=None) == inv
+    assert _ssd_call(c, wsb=16) == wsp
+    assert _ssd_call(c, N=0, x=None, cu=None) == gdn.GDN_OK                # nothing to do
+    bad = B.SsdConfigC(8, 64, 128, 2, 7, 1, 0, 0.0, float("inf"))          # state dtype
+    assert B.lib().ssd_combined_fwd(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, 2,
+                                    100, None, None, None, None, None, 0, FAKE, FAKE, 4096, None) == uns

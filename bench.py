@@ -52,9 +52,10 @@ def parse():
     p.add_argument("--workload", choices=["prefill32k", "prefill262k"], default="prefill32k")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-ssd", action="store_true", help="skip the Mamba2 SSD scan timing")
     p.add_argument("--cpu-sample-tokens", type=int, default=16384)
     p.add_argument("--ref-sample-tokens", type=int, default=4096)
-    p.add_argument("--profile", choices=["extend", "decode", "verify"], default=None,
+    p.add_argument("--profile", choices=["extend", "decode", "verify", "ssd"], default=None,
                    help="run only this call on a reduced case (an ncu target); prints timings, not the bench line")
     p.add_argument("--profile-tokens", type=int, default=8192, help="prefill rows of the --profile extend case")
     p.add_argument("--profile-requests", type=int, default=64, help="requests of the --profile decode/verify case")
@@ -287,6 +288,32 @@ def workload_config(pre, args):
 # ------------------------------------------------------------------ our arm
 
 
+def ssd_work(w):
+    """Algorithmic bytes and FLOPs of one Mamba2 SSD scan over workload w (chunks of C rows).
+    Bytes: x, z, out (H P bf16 each), B and C (G N bf16 each) and dt (H bf16) per row, plus the
+    initial and final states once per sequence.  FLOPs per row and head: the group's C B^T shared
+    by its H / G heads (2 C N / (H / G)), the intra product Lm X (2 C P), and the state's read-out
+    C h^T and update B^T Xw (2 N P each)."""
+    s = w.spec
+    T, H, P, N, G = w.T, s.H, s.P, s.N, s.G
+    esz = torch.tensor([], dtype=s.state_dtype).element_size()
+    nseq = len(w.lengths)
+    byts = T * (3 * H * P * 2 + 2 * G * N * 2 + H * 2) + 2 * nseq * H * P * N * esz
+    flops = T * H * (2 * C * N / (H // G) + 2 * C * P + 4 * N * P)
+    return byts, flops
+
+
+def ssd_call(w, gdn, dev):
+    s = w.spec
+    cfg = gdn.SsdConfig(nheads=s.H, headdim=s.P, dstate=s.N, ngroups=s.G, state_dtype=s.state_dtype)
+    ws = gdn.alloc_workspace(gdn.ssd_workspace_size(cfg, len(w.lengths), w.T), dev)
+    out = torch.empty((w.T, s.H, s.P), dtype=torch.bfloat16, device=dev)
+    fin = torch.empty((len(w.lengths), s.H, s.P, s.N), dtype=s.state_dtype, device=dev)
+    call = lambda: gdn.ssd_combined_fwd(cfg, w.x, w.dt, w.A, w.B, w.C, w.cu, out, ws, D=w.D, z=w.z,
+                                        dt_bias=w.dt_bias, initial_states=w.init, final_states=fin)
+    return call, ws
+
+
 def run_profile_case(args, dev):
     """A reduced case of one call, for ncu captures: `--profile extend` runs the
     prefill layer (16/32 heads, d=128) on --profile-tokens rows in 4 sequences;
@@ -295,7 +322,11 @@ def run_profile_case(args, dev):
     import hybrid_linear_attention_causal_b200 as gdn
     from hybrid_linear_attention_causal_b200 import workloads as W
 
-    if args.profile == "extend":
+    if args.profile == "ssd":
+        w = W.ssd_prefill(device=dev, total=args.profile_tokens, nseq=4)
+        call, ws = ssd_call(w, gdn, dev)
+        w.cu_seqlens, w.N = w.cu, len(w.lengths)
+    elif args.profile == "extend":
         w = W.large_prefill(device=dev, total=args.profile_tokens, nseq=4)
         cfg = gdn.GdnConfig.from_spec(w.spec)
         ws = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, w.N, w.T), dev)
@@ -329,7 +360,7 @@ def run_profile_case(args, dev):
     s1.record()
     torch.cuda.synchronize()
     assert gdn.gdn_get_device_error(ws) == 0
-    cu = w.cu_seqlens.cpu().tolist() if args.profile == "extend" else list(range(w.N + 1))
+    cu = w.cu_seqlens.cpu().tolist() if args.profile in ("extend", "ssd") else list(range(w.N + 1))
     chunks = sum((cu[i + 1] - cu[i] + C - 1) // C for i in range(len(cu) - 1))
     print(json.dumps({"profile": args.profile, "workload": w.name, "chunks": chunks,
                       "ms_per_call": s0.elapsed_time(s1) / args.steps}))
@@ -538,6 +569,32 @@ def main():
     n_branch = sum(1 for t in range(D) if int(tree[t]) != t - 1)
     by_tree = by_ver + n_branch * dspec.HV * dspec.dk * dspec.dv * 4 * Bn
 
+    # Mamba2 SSD scan (the second workload), outside the timed step: its inputs (1.8 GB) exceed L2
+    ssd = None
+    if not args.no_ssd:
+        sw = W.ssd_prefill(device=dev)
+        ssd_run, ssd_ws = ssd_call(sw, gdn, dev)
+        for _ in range(3):
+            ssd_run()
+        sd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+        for e0, e1 in sd_ev:
+            e0.record()
+            ssd_run()
+            e1.record()
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_device_error(ssd_ws) == 0
+        sd_ms = max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in sd_ev), world, dev)
+        sb, sf = ssd_work(sw)
+        floor_ms = max(sb / (hbm * 1e9), sf / (bf16 * 1e12)) * 1e3
+        ssd = {"ms": sd_ms, "tokens_per_s": world * sw.T / (sd_ms * 1e-3), "workload": sw.name,
+               "config": {"heads": sw.spec.H, "headdim": sw.spec.P, "dstate": sw.spec.N, "groups": sw.spec.G,
+                          "lengths": sw.lengths, "state_dtype": "bf16", "D": True, "z": True},
+               "roofline": {"bound": "hbm", "achieved": sb / (sd_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                            "frac": sb / (sd_ms * 1e-3) / 1e9 / hbm, "floor_ms": floor_ms,
+                            "algorithmic_bytes": sb, "tensor_frac": sf / (sd_ms * 1e-3) / 1e12 / bf16},
+               "note": "timed outside the step; one ssd_combined_fwd per timing"}
+        del ssd_run, ssd_ws
+
     # End to end through the public API with pinned host buffers.  The layer is independent per
     # sequence, so the step runs one gdn_extend call per sequence and overlaps the host -> device
     # copy of sequence i + 1 and the device -> host copy of sequence i - 1 with the call for
@@ -634,6 +691,7 @@ def main():
             "verify_tree": {"ms": tr_ms, "parents": tree.tolist(), "total_gbs": world * by_tree / (tr_ms * 1e-3) / 1e9,
                             "frac_of_measured_hbm": by_tree / (tr_ms * 1e-3) / 1e9 / hbm,
                             "note": "timed outside the step"},
+            "ssd": ssd,
             "prefill_checkpoints": {"ms": ck_ms, "checkpoints": pre.N, "vs_prefill": ck_ms / ext_ms,
                                     "note": "one state checkpoint per sequence, mid chunk; timed outside the step"},
             "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12, "roofline": prefill_roofline,

@@ -13,13 +13,17 @@
 //   Gm     = C B^T             M=64 (r)  N=64 (s)  K=N   C and B rows K-major
 //   Z      = C h_in^T          M=64 (r)  N=P       K=N   h^T rows read MN-major
 //   Hnew^T = B^T Xw            M=N       N=P       K=64  B and Xw rows read MN-major
-//            (Xw = diag(e^{gamma_last - gamma} d) X)
+//            (Xw = diag(d e^{gamma_last - gamma}) X)
 //   Y      = Lm X              M=64 (r)  N=P       K=64  X rows read MN-major
 //            (Lm[r,s] = e^{gamma_r - gamma_s} d_s Gm[r,s] for s <= r, else 0)
 //
+// (C and B are exact in fp16, so Gm is exact up to fp32 accumulation; the step
+// d enters only through the rounded Lm and Xw.)
+//
 // then h_out^T = e^{gamma_last} h_in^T + Hnew^T in registers (thread row n of
 // h^T) and y_r = Y_r + e^{gamma_r} Z_r, plus the skip term D x_r and the gate
-// silu(z_r).  The first three products depend only on the chunk's inputs and
+// silu(z_r) (staged in fp32 with the chunk's rows).  Decays are powers of two
+// of base-2 cumulative sums (ex2.approx).  The first three products depend only on the chunk's inputs and
 // on h_in, so they are issued together; Y follows once Lm is formed.
 //
 // A state checkpoint inside a chunk is taken by ending the chunk at the
@@ -73,7 +77,9 @@ struct SsdSmem {
     uint16_t xw[SC * SP];  // Xw rows s x P
     uint16_t lm[SC * SC];  // Lm rows r x s
     uint16_t ht[N * SP];   // fp16 copy of h^T: rows n x P (R = N)
-    float gam[SC];         // gamma_r (rows past the chunk repeat gamma_last)
+    __nv_bfloat16 xs[SC][SP + 8];  // the chunk's x rows (bf16) and gates silu(z) (fp32), rows padded by
+    float zs[SC][SP + 4];          // 16 bytes so that the threads reading one row each spread over the banks
+    float g2[SC];          // gamma_r log2(e) (rows past the chunk repeat the last row's)
     float dd[SC];          // processed step d_r (0 past the chunk)
     float wl[SC];          // d_s e^{gamma_last - gamma_s}
     unsigned long long bar1, bar2;
@@ -117,9 +123,9 @@ __device__ __forceinline__ void st16(uint16_t* tile, uint32_t off, const uint4& 
     *reinterpret_cast<uint4*>(reinterpret_cast<char*>(tile) + off) = v;
 }
 
-// processed step of (row t, head h): clamp(softplus?(dt + dt_bias), lo, hi)
-__device__ __forceinline__ float ssd_step(const SsdArgs& p, int t, int h) {
-    float v = __bfloat162float(p.dt[(size_t)t * p.H + h]) + (p.dt_bias ? p.dt_bias[h] : 0.f);
+// processed step of a raw step dt of head h: clamp(softplus?(dt + dt_bias), lo, hi)
+__device__ __forceinline__ float ssd_step(const SsdArgs& p, float dt, int h) {
+    float v = dt + (p.dt_bias ? p.dt_bias[h] : 0.f);
     if (p.softplus) v = v > 20.f ? v : log1pf(expf(v));
     return fminf(fmaxf(v, p.dt_lo), p.dt_hi);
 }
@@ -187,21 +193,59 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
     const uint32_t tm = sm.tmem_base;
     const uint32_t tG = tm, tZ = tm + 64, tS = tm + 128, tY = tm + 192;  // 64 columns each
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float Ah = p.A[h];
+    const float Ah2 = p.A[h] * 1.4426950408889634f;  // A log2(e): decays are formed as powers of two
     const float Dh = (p.D && !p.d_per_dim) ? __bfloat162float(p.D[h]) : 0.f;
     constexpr uint32_t iG = tc::idesc_f16(SC, SC), iZ = tc::idesc_f16(SC, SP) | tc::kTransposeB,
                        iH = tc::idesc_f16(N, SP) | tc::kTransposeA | tc::kTransposeB;
 
+    // the next chunk's rows, fetched into registers one chunk ahead: thread j of each group of eight
+    // takes row 8 rg + j of one 16-byte column block, so that a warp reads 64 contiguous bytes of
+    // each of 8 rows and eight consecutive threads later store one 128-byte core-matrix block
+    constexpr int NBX = SP / 8, NBB = N / 8, KX = SC * NBX / SNT, KB = SC * NBB / SNT;
+    uint4 rx[KX], rz[KX], rb[KB], rc[KB];
+    float rdt0 = 0.f, rdt1 = 0.f;  // (warp 0) raw steps of rows lane and lane + 32
+    auto chunk_len = [&](int t0) {  // up to 64 rows, cut at the checkpoint boundary
+        int len = min(SC, s1 - t0);
+        if (ck_b > t0 && ck_b < t0 + len) len = ck_b - t0;
+        return len;
+    };
+    auto fetch = [&](int t0, int len) {
+#pragma unroll
+        for (int k = 0; k < KX; ++k) {
+            const int e = tid + k * SNT, j = e & 7, cb = (e >> 3) % NBX, r = ((e >> 3) / NBX) * 8 + j;
+            rx[k] = rz[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < len) {
+                const size_t o = ((size_t)(t0 + r) * p.H + h) * SP + cb * 8;
+                rx[k] = __ldcs(reinterpret_cast<const uint4*>(p.x + o));
+                if (p.z) rz[k] = __ldcs(reinterpret_cast<const uint4*>(p.z + o));
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            const int e = tid + k * SNT, j = e & 7, cb = (e >> 3) % NBB, r = ((e >> 3) / NBB) * 8 + j;
+            rb[k] = rc[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < len) {  // B and C rows are shared by the group's heads: kept in L2
+                const size_t o = ((size_t)(t0 + r) * p.G + g) * N + cb * 8;
+                rb[k] = __ldg(reinterpret_cast<const uint4*>(p.B + o));
+                rc[k] = __ldg(reinterpret_cast<const uint4*>(p.C + o));
+            }
+        }
+        if (warp == 0) {
+            rdt0 = lane < len ? __bfloat162float(p.dt[(size_t)(t0 + lane) * p.H + h]) : 0.f;
+            rdt1 = lane + 32 < len ? __bfloat162float(p.dt[(size_t)(t0 + lane + 32) * p.H + h]) : 0.f;
+        }
+    };
+    int len = s0 < s1 ? chunk_len(s0) : 0;
+    if (len > 0) fetch(s0, len);
+
     bool ok = true, okw = true;
     uint32_t ph = 0;
     for (int t0 = s0; t0 < s1; ph ^= 1u) {
-        int len = min(SC, s1 - t0);
-        if (ck_b > t0 && ck_b < t0 + len) len = ck_b - t0;  // the chunk ends at the checkpoint
         // ---- processed steps and in-chunk cumulative decay (warp 0, rows lane and lane + 32)
         if (warp == 0) {
-            const float d0 = lane < len ? ssd_step(p, t0 + lane, h) : 0.f;
-            const float d1 = lane + 32 < len ? ssd_step(p, t0 + lane + 32, h) : 0.f;
-            float c0 = d0 * Ah, c1 = d1 * Ah;
+            const float d0 = lane < len ? ssd_step(p, rdt0, h) : 0.f;
+            const float d1 = lane + 32 < len ? ssd_step(p, rdt1, h) : 0.f;
+            float c0 = d0 * Ah2, c1 = d1 * Ah2;  // base-2 exponents
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float v0 = __shfl_up_sync(0xffffffffu, c0, o), v1 = __shfl_up_sync(0xffffffffu, c1, o);
@@ -212,51 +256,46 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
             }
             c1 += __shfl_sync(0xffffffffu, c0, 31);
             const float gl = __shfl_sync(0xffffffffu, c1, 31);  // rows past the chunk add nothing
-            sm.gam[lane] = c0;
-            sm.gam[lane + 32] = c1;
+            sm.g2[lane] = c0;
+            sm.g2[lane + 32] = c1;
             sm.dd[lane] = d0;
             sm.dd[lane + 32] = d1;
-            sm.wl[lane] = d0 * expf(gl - c0);
-            sm.wl[lane + 32] = d1 * expf(gl - c1);
+            sm.wl[lane] = d0 * tc::ex2_approx(gl - c0);
+            sm.wl[lane + 32] = d1 * tc::ex2_approx(gl - c1);
         }
-        ok = __syncthreads_and(okw) != 0;  // (also: the previous chunk's products are all read)
+        ok = __syncthreads_and(okw) != 0;  // (also: the previous chunk's outputs are all read)
         if (!ok) break;
-        // ---- the chunk's rows into the fp16 operand tiles, zero past the chunk.  Thread j of each
-        // group of eight takes row 8 rg + j of one 16-byte column block: eight consecutive threads
-        // store one 128-byte core-matrix block, and a warp reads 64 contiguous bytes of 8 rows
-        {
-            constexpr int NBX = SP / 8;
+        // ---- the fetched rows into the fp16 operand tiles (zero past the chunk) and the bf16
+        // staging rows of x and z for the outputs
 #pragma unroll
-            for (int k = 0; k < SC * NBX / SNT; ++k) {
-                const int e = tid + k * SNT, j = e & 7, cb = (e >> 3) % NBX, r = ((e >> 3) / NBX) * 8 + j;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (r < len) v = *reinterpret_cast<const uint4*>(p.x + ((size_t)(t0 + r) * p.H + h) * SP + cb * 8);
-                float f[8];
-                bf16x8(v, f);
-                const uint32_t off = tc::kmajor_off16(r, cb * 8, SC);
-                st16(sm.xt, off, f16x8(f));
-                const float w = sm.wl[r];
+        for (int k = 0; k < KX; ++k) {
+            const int e = tid + k * SNT, j = e & 7, cb = (e >> 3) % NBX, r = ((e >> 3) / NBX) * 8 + j;
+            float f[8];
+            bf16x8(rx[k], f);
+            const uint32_t off = tc::kmajor_off16(r, cb * 8, SC);
+            st16(sm.xt, off, f16x8(f));
+            const float w = sm.wl[r];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] *= w;
-                st16(sm.xw, off, f16x8(f));
+            for (int i = 0; i < 8; ++i) f[i] *= w;
+            st16(sm.xw, off, f16x8(f));
+            *reinterpret_cast<uint4*>(&sm.xs[r][cb * 8]) = rx[k];
+            if (p.z) {  // the gate silu(z) = z / (1 + e^{-z})
+                bf16x8(rz[k], f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = __fdividef(f[i], 1.f + __expf(-f[i]));
+                *reinterpret_cast<float4*>(&sm.zs[r][cb * 8]) = make_float4(f[0], f[1], f[2], f[3]);
+                *reinterpret_cast<float4*>(&sm.zs[r][cb * 8 + 4]) = make_float4(f[4], f[5], f[6], f[7]);
             }
-            constexpr int NBB = N / 8;
+        }
 #pragma unroll
-            for (int k = 0; k < SC * NBB / SNT; ++k) {
-                const int e = tid + k * SNT, j = e & 7, cb = (e >> 3) % NBB, r = ((e >> 3) / NBB) * 8 + j;
-                uint4 vb = make_uint4(0u, 0u, 0u, 0u), vc = vb;
-                if (r < len) {
-                    const size_t o = ((size_t)(t0 + r) * p.G + g) * N + cb * 8;
-                    vb = *reinterpret_cast<const uint4*>(p.B + o);
-                    vc = *reinterpret_cast<const uint4*>(p.C + o);
-                }
-                float f[8];
-                const uint32_t off = tc::kmajor_off16(r, cb * 8, SC);
-                bf16x8(vb, f);
-                st16(sm.bt, off, f16x8(f));
-                bf16x8(vc, f);
-                st16(sm.ct, off, f16x8(f));
-            }
+        for (int k = 0; k < KB; ++k) {
+            const int e = tid + k * SNT, j = e & 7, cb = (e >> 3) % NBB, r = ((e >> 3) / NBB) * 8 + j;
+            float f[8];
+            const uint32_t off = tc::kmajor_off16(r, cb * 8, SC);
+            bf16x8(rb[k], f);
+            st16(sm.bt, off, f16x8(f));
+            bf16x8(rc[k], f);
+            st16(sm.ct, off, f16x8(f));
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -279,7 +318,7 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
         okw = tc::mbar_wait(bar1, ph);
         tc::fence_after_sync();
         {  // h^T <- e^{gamma_last} h^T + Hnew^T
-            const float egl = expf(sm.gam[SC - 1]);
+            const float egl = tc::ex2_approx(sm.g2[SC - 1]);
 #pragma unroll
             for (int c0 = 0; c0 < SP; c0 += 16) {
                 float v[16];
@@ -291,7 +330,7 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
         }
         put_ht();
         {  // Lm row r_own: e^{gamma_r - gamma_s} d_s Gm[r, s] for s <= r
-            const float gr = sm.gam[r_own];
+            const float gr = sm.g2[r_own];
             const bool rv = lane < 16 && r_own < len;
 #pragma unroll
             for (int c0 = 0; c0 < SC; c0 += 16) {
@@ -305,7 +344,7 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int s = c0 + q + i;
-                            f[i] = (rv && s <= r_own) ? v[q + i] * sm.dd[s] * expf(gr - sm.gam[s]) : 0.f;
+                            f[i] = (rv && s <= r_own) ? v[q + i] * sm.dd[s] * tc::ex2_approx(gr - sm.g2[s]) : 0.f;
                         }
                         st16(sm.lm, tc::kmajor_off16(r_own, c0 + q, SC), f16x8(f));
                     }
@@ -324,11 +363,14 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
                 tc::mma_f16(tY, tc::desc_kmajor(lm, SC, k), tc::desc_mnmajor16(xt, SC, k), iZ, k > 0);
             tc::mma_commit(bar2);
         }
+        // the next chunk's rows load while Y and this chunk's outputs complete
+        const int t0n = t0 + len, lenn = t0n < s1 ? chunk_len(t0n) : 0;
+        if (lenn > 0) fetch(t0n, lenn);
         okw = tc::mbar_wait(bar2, ph);
         tc::fence_after_sync();
         {  // y_r = Y_r + e^{gamma_r} Z_r, skip term, gate
             const bool live = okw && lane < 16 && r_own < len;
-            const float eg = expf(sm.gam[r_own]);
+            const float eg = tc::ex2_approx(sm.g2[r_own]);
             const size_t row = ((size_t)(t0 + r_own) * p.H + h) * SP;
 #pragma unroll
             for (int c0 = 0; c0 < SP; c0 += 16) {
@@ -344,22 +386,23 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
                         for (int i = 0; i < 8; ++i) o[i] = fmaf(eg, zv[q + i], yv[q + i]);
                         if (p.D) {
                             float xv[8], dv[8];
-                            bf16x8(*reinterpret_cast<const uint4*>(p.x + row + c0 + q), xv);
+                            bf16x8(*reinterpret_cast<const uint4*>(&sm.xs[r_own][c0 + q]), xv);
                             if (p.d_per_dim) bf16x8(*reinterpret_cast<const uint4*>(p.D + (size_t)h * SP + c0 + q), dv);
 #pragma unroll
                             for (int i = 0; i < 8; ++i) o[i] = fmaf(p.d_per_dim ? dv[i] : Dh, xv[i], o[i]);
                         }
                         if (p.z) {
-                            float zz[8];
-                            bf16x8(*reinterpret_cast<const uint4*>(p.z + row + c0 + q), zz);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) o[i] *= zz[i] / (1.f + expf(-zz[i]));
+                            const float4 g0 = *reinterpret_cast<const float4*>(&sm.zs[r_own][c0 + q]),
+                                         g1 = *reinterpret_cast<const float4*>(&sm.zs[r_own][c0 + q + 4]);
+                            o[0] *= g0.x; o[1] *= g0.y; o[2] *= g0.z; o[3] *= g0.w;
+                            o[4] *= g1.x; o[5] *= g1.y; o[6] *= g1.z; o[7] *= g1.w;
                         }
-                        *reinterpret_cast<uint4*>(p.out + row + c0 + q) = bf16x8_out(o);
+                        __stcs(reinterpret_cast<uint4*>(p.out + row + c0 + q), bf16x8_out(o));
                     }
             }
         }
-        t0 += len;
+        t0 = t0n;
+        len = lenn;
     }
     ok = __syncthreads_and(ok && okw) != 0;
     if (ok) {

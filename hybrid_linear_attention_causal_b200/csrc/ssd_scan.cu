@@ -59,6 +59,7 @@ struct SsdArgs {
     const __nv_bfloat16* z;
     const float* dt_bias;
     const int32_t* cu;
+    const int32_t* order;  // sequences, longest first
     const void* init;
     void* fin;
     const int32_t* ck_idx;
@@ -132,7 +133,7 @@ __device__ __forceinline__ float ssd_step(const SsdArgs& p, float dt, int h) {
 
 template <typename TS, int N>
 __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
-    const int seq = blockIdx.x / p.H, h = blockIdx.x % p.H;
+    const int seq = p.order[blockIdx.x / p.H], h = blockIdx.x % p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = h / (p.H / p.G);
     const int s0 = p.cu[seq], s1 = p.cu[seq + 1];
@@ -420,12 +421,38 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
     if (warp == 0) tc::tmem_dealloc(tm, 256);
 }
 
+// order[rank] = sequence: sequences by decreasing length (ties by index), so that the longest chains
+// start first; a sequence with invalid bounds counts as empty
+__global__ void ssd_order_kernel(const int32_t* cu, int nseq, int T, int32_t* order) {
+    __shared__ int lens[1024];
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    auto len_of = [&](int j) {
+        const int a = cu[j], b = cu[j + 1];
+        return (a < 0 || b < a || b > T) ? 0 : b - a;
+    };
+    const int li = i < nseq ? len_of(i) : 0;
+    int rank = 0;
+    for (int j0 = 0; j0 < nseq; j0 += 1024) {
+        __syncthreads();
+        for (int j = threadIdx.x; j < 1024 && j0 + j < nseq; j += blockDim.x) lens[j] = len_of(j0 + j);
+        __syncthreads();
+        const int m = min(1024, nseq - j0);
+        if (i < nseq)
+            for (int j = 0; j < m; ++j) {
+                const int lj = lens[j];
+                rank += (lj > li) || (lj == li && j0 + j < i);
+            }
+    }
+    if (i < nseq) order[rank] = i;
+}
+
 template <typename TS, int N>
 cudaError_t launch_ssd(const SsdArgs& a, cudaStream_t s) {
     // at most two CTAs per SM, whose 256 tensor-memory columns each fill the SM's 512
     const size_t shm = sizeof(SsdSmem<N>) > 80 * 1024 ? sizeof(SsdSmem<N>) : 80 * 1024;
     cudaError_t e = cudaFuncSetAttribute(ssd_scan_kernel<TS, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
+    ssd_order_kernel<<<(a.Nseq + 255) / 256, 256, 0, s>>>(a.cu, a.Nseq, a.T, const_cast<int32_t*>(a.order));
     ssd_scan_kernel<TS, N><<<(unsigned)(a.Nseq * a.H), SNT, shm, s>>>(a);
     return cudaGetLastError();
 }
@@ -442,7 +469,7 @@ bool al16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 
 extern "C" GDN_API size_t ssd_workspace_size(const ssd_config_t* cfg, int32_t max_N, int32_t max_T) {
     if (!cfg || max_N < 0 || max_T < 0) return 0;
-    return (size_t)gdn::kHeaderBytes;
+    return (size_t)gdn::kHeaderBytes + (((size_t)max_N * 4 + 15) & ~(size_t)15);  // header + sequence order
 }
 
 extern "C" GDN_API int ssd_combined_fwd(const ssd_config_t* cfg, const void* x, const void* dt, const float* A,
@@ -491,6 +518,7 @@ extern "C" GDN_API int ssd_combined_fwd(const ssd_config_t* cfg, const void* x, 
     a.z = static_cast<const __nv_bfloat16*>(z);
     a.dt_bias = dt_bias;
     a.cu = cu_seqlens;
+    a.order = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + gdn::kHeaderBytes);
     a.init = initial_states;
     a.fin = final_states;
     a.ck_idx = ckpt_token_indices;

@@ -45,7 +45,8 @@ typedef struct {
     float dt_max;
 } ssd_config_t;
 
-/* Bytes of workspace ssd_combined_fwd needs (the device error header). */
+/* Bytes of workspace ssd_combined_fwd needs for up to max_N sequences (the device error header and
+ * the order in which the sequences are scanned, longest first). */
 GDN_API size_t ssd_workspace_size(const ssd_config_t* cfg, int32_t max_N, int32_t max_T);
 
 /*

@@ -187,7 +187,8 @@ def _ssd_call(c, x=FAKE, dt=FAKE, A=FAKE, Bm=FAKE, C=FAKE, D=None, z=None, bias=
 
 def test_ssd_workspace_and_argument_validation():
     c = gdn.SsdConfig(nheads=8, headdim=64, dstate=128, ngroups=2)
-    assert gdn.ssd_workspace_size(c, 8, 32768) == B.HEADER_BYTES
+    assert gdn.ssd_workspace_size(c, 8, 32768) == B.HEADER_BYTES + 32
+    assert gdn.ssd_workspace_size(c, 5, 100) == B.HEADER_BYTES + 32
     assert B.lib().ssd_workspace_size(None, 1, 1) == 0
     inv, uns, wsp = gdn.GDN_ERR_INVALID_ARG, gdn.GDN_ERR_UNSUPPORTED, gdn.GDN_ERR_WORKSPACE
     assert _ssd_call(gdn.SsdConfig(nheads=6, headdim=64, dstate=128, ngroups=4)) == inv   # H % G
@@ -206,6 +207,7 @@ def test_ssd_workspace_and_argument_validation():
     assert _ssd_call(c, ck=(FAKE, FAKE, FAKE), num_ck=-1) == inv
     assert _ssd_call(c, ws=None) == inv
     assert _ssd_call(c, wsb=16) == wsp
+    assert _ssd_call(c, N=2, wsb=B.HEADER_BYTES) == wsp                    # no room for the order
     assert _ssd_call(c, N=0, x=None, cu=None) == gdn.GDN_OK                # nothing to do
     bad = B.SsdConfigC(8, 64, 128, 2, 7, 1, 0, 0.0, float("inf"))          # state dtype
     assert B.lib().ssd_combined_fwd(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, 2,

@@ -591,7 +591,8 @@ def main():
                           "lengths": sw.lengths, "state_dtype": "bf16", "D": True, "z": True},
                "roofline": {"bound": "hbm", "achieved": sb / (sd_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
                             "frac": sb / (sd_ms * 1e-3) / 1e9 / hbm, "floor_ms": floor_ms,
-                            "algorithmic_bytes": sb, "tensor_frac": sf / (sd_ms * 1e-3) / 1e12 / bf16},
+                            "algorithmic_bytes": sb, "tensor_frac": sf / (sd_ms * 1e-3) / 1e12 / bf16,
+                            "traffic": ncu_traffic("ssd")},
                "note": "timed outside the step; one ssd_combined_fwd per timing"}
         del ssd_run, ssd_ws
 

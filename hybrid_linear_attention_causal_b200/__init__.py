@@ -1,6 +1,7 @@
-"""B200 (sm_100a) Gated DeltaNet layer: extend / decode / verify / commit behind a C ABI.
+"""B200 (sm_100a) Gated DeltaNet layer: extend / decode / verify / commit behind a C ABI,
+and the Mamba2 SSD chunk scan (ssd_combined_fwd).
 
-The compute lives in libgdn.so (csrc/, declared in include/gdn.h); this
+The compute lives in libgdn.so (csrc/, declared in include/gdn.h and include/ssd.h); this
 package holds its ctypes binding, the in-tree build step and seeded synthetic
 workloads.  Calls fail loudly when libgdn.so has not been built.
 """

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import hybrid_linear_attention_causal_b200 as gdn
 from hybrid_linear_attention_causal_b200 import binding as B
@@ -212,3 +213,22 @@ def test_ssd_workspace_and_argument_validation():
     bad = B.SsdConfigC(8, 64, 128, 2, 7, 1, 0, 0.0, float("inf"))          # state dtype
     assert B.lib().ssd_combined_fwd(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, 2,
                                     100, None, None, None, None, None, 0, FAKE, FAKE, 4096, None) == uns
+
+
+def test_ssd_workload_recipe_is_seeded_and_shaped():
+    from hybrid_linear_attention_causal_b200 import workloads as W
+
+    spec = W.SsdSpec(H=6, P=64, N=64, G=3, state_dtype=torch.float16)
+    a = W.ssd_case(spec, [5, 0, 70], seed=3, d_per_dim=True)
+    b = W.ssd_case(spec, [5, 0, 70], seed=3, d_per_dim=True)
+    for name in ("x", "dt", "A", "B", "C", "D", "z", "dt_bias", "cu", "init"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    assert a.x.shape == (75, 6, 64) and a.x.dtype == torch.bfloat16
+    assert a.B.shape == (75, 3, 64) and a.C.shape == a.B.shape and a.dt.shape == (75, 6)
+    assert a.D.shape == (6, 64) and a.init.shape == (3, 6, 64, 64) and a.init.dtype == torch.float16
+    assert a.cu.tolist() == [0, 5, 5, 75]
+    assert (a.A < 0).all() and a.A.dtype == torch.float32
+    w = W.ssd_prefill()
+    assert w.T == 32768 and len(w.lengths) == 8 and all(512 <= n <= 16384 for n in w.lengths)
+    none = W.ssd_case(spec, [4], seed=1, with_D=False, with_z=False, with_bias=False, init_random=False)
+    assert none.D is None and none.z is None and none.dt_bias is None and none.init is None

@@ -152,3 +152,10 @@ def test_bench_workload_sampled_heads():
     assert_ssd_out_close(_f64(out[:, heads]), y, what="sampled heads out")
     assert_ssd_state_close(_f64(fin[:, heads]), f, "bfloat16", what="sampled heads final")
     assert torch.isfinite(out.float()).all()
+
+
+def test_many_short_sequences():
+    """1100 packed sequences of 0 to 9 rows: the longest-first order is ranked in tiles of 1024."""
+    lens = [(7 * i) % 10 for i in range(1100)]
+    w = W.ssd_case(W.SsdSpec(H=2, P=64, N=64, G=1, state_dtype=torch.float32), lens, seed=39)
+    check(w, gpu_ssd(w), oracle_ssd(w), "many sequences")

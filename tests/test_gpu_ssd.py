@@ -159,3 +159,34 @@ def test_many_short_sequences():
     lens = [(7 * i) % 10 for i in range(1100)]
     w = W.ssd_case(W.SsdSpec(H=2, P=64, N=64, G=1, state_dtype=torch.float32), lens, seed=39)
     check(w, gpu_ssd(w), oracle_ssd(w), "many sequences")
+
+
+def test_graph_capture_and_bit_reproducibility():
+    """Two eager calls and a CUDA-graph replay of the same call give bit-identical outputs and states."""
+    w = W.ssd_case(W.SsdSpec(H=4, P=64, N=128, G=2), [70, 1, 130], seed=40)
+    s = w.spec
+    wd = w.to("cuda")
+    cfg = gdn.SsdConfig(nheads=s.H, headdim=s.P, dstate=s.N, ngroups=s.G, state_dtype=s.state_dtype)
+    ws = gdn.alloc_workspace(gdn.ssd_workspace_size(cfg, 3, w.T), "cuda")
+    outs = [torch.empty((w.T, s.H, s.P), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    fins = [torch.empty_like(wd.init) for _ in range(3)]
+
+    def call(k):
+        gdn.ssd_combined_fwd(cfg, wd.x, wd.dt, wd.A, wd.B, wd.C, wd.cu, outs[k], ws, D=wd.D, z=wd.z,
+                             dt_bias=wd.dt_bias, initial_states=wd.init, final_states=fins[k])
+
+    call(0)
+    call(1)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            call(2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert gdn.gdn_get_device_error(ws) == 0
+    for k in (1, 2):
+        assert torch.equal(outs[k].view(torch.int16), outs[0].view(torch.int16))
+        assert torch.equal(fins[k].view(torch.int16), fins[0].view(torch.int16))

@@ -252,6 +252,33 @@ def oracle_sample(pre, ntok):
     return run, n, workers
 
 
+def ssd_oracle_sample(w, nrows):
+    """The fp64 SSD oracle on the first `nrows` packed rows of SSD workload w (the leading sequences,
+    the last one cut), all heads.  Returns (run, rows, workers)."""
+    from oracle import ssd as OS
+
+    s = w.spec
+    lens, n = [], 0
+    for L in w.lengths:
+        take = min(int(L), nrows - n)
+        if take <= 0:
+            break
+        lens.append(take)
+        n += take
+    cu = torch.tensor([0] + [sum(lens[:i + 1]) for i in range(len(lens))], dtype=torch.int32)
+    cpu = lambda t: None if t is None else t[:n].cpu() if t.dim() >= 2 and t.shape[0] == w.T else t.cpu()
+    cfg = OS.SsdCfg(H=s.H, P=s.P, N=s.N, G=s.G)
+    init = None if w.init is None else w.init[:len(lens)].cpu()
+    args = (cfg, cpu(w.x), cpu(w.dt), w.A.cpu(), cpu(w.B), cpu(w.C), cu)
+    kw = dict(D=None if w.D is None else w.D.cpu(), z=cpu(w.z), dt_bias=None if w.dt_bias is None else w.dt_bias.cpu(),
+              init=init)
+
+    def run():
+        OS.scan(*args, **kw)
+
+    return run, n, min(OS.num_threads(), len(lens) * s.H)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -267,6 +294,16 @@ def run_reference(args, rank, world):
     dt = (time.perf_counter() - t0) / args.steps
     val = n / dt
     sample = f"first {n} packed rows of the {pre.name} batch, all {pre.spec.HV} value heads, per step"
+    ssd = None
+    if not args.no_ssd:  # the SSD scan's oracle on a bounded sample of its workload, timed once
+        sw = W.ssd_prefill(device="cpu")
+        srun, sn, sworkers = ssd_oracle_sample(sw, args.ref_sample_tokens // 4)
+        srun()
+        t1 = time.perf_counter()
+        srun()
+        sdt = time.perf_counter() - t1
+        ssd = {"value": sn / sdt, "unit": "rows/s", "cores": sworkers, "kind": "oracle", "workload": sw.name,
+               "sample": f"first {sn} packed rows of the {sw.name} batch, all {sw.spec.H} heads"}
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
@@ -274,6 +311,7 @@ def run_reference(args, rank, world):
         "config": workload_config(pre, args),
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": workers, "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "ssd": ssd,
     }), flush=True)
 
 
@@ -594,6 +632,13 @@ def main():
                             "algorithmic_bytes": sb, "tensor_frac": sf / (sd_ms * 1e-3) / 1e12 / bf16,
                             "traffic": ncu_traffic("ssd")},
                "note": "timed outside the step; one ssd_combined_fwd per timing"}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            orun, on, oworkers = ssd_oracle_sample(sw, 1024)
+            t0 = time.perf_counter()
+            orun()
+            odt = time.perf_counter() - t0
+            ssd["cpu_baseline"] = {"value": on / odt, "unit": "rows/s", "cores": oworkers, "kind": "oracle",
+                                   "sample": f"fp64 oracle, first {on} packed rows of the batch, all {sw.spec.H} heads"}
         del ssd_run, ssd_ws
 
     # End to end through the public API with pinned host buffers.  The layer is independent per

@@ -17,6 +17,9 @@
  *               (gdn_verify_tree: the draft tokens form a tree given by parent indices)
  *   gdn_commit  the accepted prefix of a verify pass back into the pools
  *
+ * The same library also exports the Mamba2 SSD chunk scan (ssd_combined_fwd),
+ * declared in ssd.h, which shares this header's conventions and error codes.
+ *
  * What every mode computes, per request and value head h (qk head h / (HV/HK)):
  *   conv:  y_t = SiLU(sum_{j<K} w[c,j] x_{t-K+1+j}[c] (+ bias[c])) per channel c,
  *          rows before the request's first new row come from its conv-state slot;

@@ -132,18 +132,16 @@ struct ExtendArgs {
     int32_t* rank_off;  // [N+1] chunk_list position of each rank's first chunk
     int32_t* chunk_list;// [max_chunks] chunk ids, rank by rank (longest sequence first)
     int nseg;           // S
-    // per chunk, written by the prep kernel (conv + SiLU + L2 norm + gates):
-    uint16_t* KQ;       // [max_chunks, HK, 2*C*dk] [K ; Q*scale] fp16, K-major tile of 128 rows
-    uint16_t* VT;       // [max_chunks, HV, dv*C]   V^T fp16, K-major tile of dv rows x C
-    float2* GB;         // [max_chunks, HV, C]      (g, beta); rows past the chunk end are zero
-    // per (chunk, value head), written by the intra kernel, read by the state
-    // pass; the tiles are fp16 values already in the tensor-core shared-memory
-    // layout, so the state pass copies them verbatim
-    uint16_t* WQ;       // [max_chunks, HV, 2*C*dk]  [W ; diag(e^gamma) Q], fp16, K-major, 128 rows
-    uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, fp16, K-major, C rows
-    uint16_t* KT;       // [max_chunks, HV, C*dk]    K~ = diag(e^{gamma_n-gamma}) K, fp16, tile of C rows s
-    uint16_t* U;        // [max_chunks, HV, dv*C]    U^T, fp16, K-major tile of dv rows (j) x C
-    float* gam;         // [max_chunks, HV, C]       in-chunk cumulative g
+    // per chunk, written by the per-chunk step (conv + SiLU, L2 norm, gates and the intra-chunk
+    // products) and read by the state pass; the tiles are fp16 values already in the tensor core's
+    // 128-byte swizzled shared-memory layout, so the state pass copies them verbatim.  Rows past the
+    // end of a ragged chunk are zero.
+    uint16_t* KQ;       // [max_chunks, HK, 2*C*dk]  [K ; Q*scale] (L2-normalised), 128 rows x dk
+    uint16_t* W;        // [max_chunks, HV, C*dk]    W = T diag(beta e^gamma) K, C rows x dk
+    uint16_t* U;        // [max_chunks, HV, dv*C]    U^T = (T diag(beta) V)^T, dv rows x C
+    uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, C rows x C
+    float4* GV;         // [max_chunks, HV, C]       per row: e^{gamma_r}, f_r = e^{gamma_n - gamma_r}
+                        //                           (0 past the chunk end), gamma_r, e^{gamma_n}
 };
 
 // Dispatch on the supported (dk, dv) pairs; expects a LayerDims `p.d` in scope.
@@ -170,11 +168,11 @@ __device__ __forceinline__ int ckpt_offset(const ExtendArgs& p, int n, int* row)
     return b - p.cu[n];
 }
 
-// Intra-chunk step on tensor cores (gdn_intra_tc.cu) for the chunks of one
-// segment: persistent CTAs taking (chunk, qk head) items dynamically; for
-// segment k > 0 they leave one SM per CTA of segment k-1's state pass free.
-template <int DK, int DV>
-cudaError_t launch_intra(const ExtendArgs& p, int seg, cudaStream_t s);
+// Per-chunk step on tensor cores (gdn_chunk_tc.cu) for the chunks of one
+// segment: conv + SiLU, L2 norm, gates and the intra-chunk products of
+// (chunk, qk head) items, taken dynamically by persistent CTAs.
+template <typename T, int DK, int DV>
+cudaError_t launch_chunk(const ExtendArgs& p, int seg, cudaStream_t s);
 
 // Serial state pass + outputs on tensor cores (gdn_state_tc.cu) for one
 // segment: one CTA per (sequence, value head), longest sequences first.

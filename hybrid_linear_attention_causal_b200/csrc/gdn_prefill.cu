@@ -12,16 +12,16 @@
 //
 // Launch sequence (all stream-ordered, no host synchronisation):
 //   1. chunk_map:  validates cu_seqlens and lays out the chunk table
-//   2. prep:       per (chunk, head): conv1d + SiLU, L2 norm, gates -> tiles
-//   3. conv_tail:  writes each sequence's new conv window into its slot
-//   4. intra:      per (chunk, qk head) on tensor cores: gamma, A, T, W, U and
-//                  the masked decayed q.k of each value head (gdn_intra_tc.cu)
-//   5. state:      per (sequence, value head) on tensor cores: the serial chunk
+//   2. chunk:      per (chunk, qk head) on tensor cores: conv1d + SiLU, L2 norm,
+//                  gates, A, T, W, U and the masked decayed q.k of each value
+//                  head (gdn_chunk_tc.cu), segment by segment
+//   3. state:      per (sequence, value head) on tensor cores: the serial chunk
 //                  pass V' = U - W S, the outputs and S <- e^{gamma_n} S + K~^T V'
-//                  (gdn_state_tc.cu)
-// Every intermediate is fp32 and every tensor-core operand is rounded to tf32
-// (round to nearest): the parity bar leaves no room for bf16 rounding of q, k,
-// v, W, U or V', and truncating to tf32 instead of rounding fails it too.
+//                  (gdn_state_tc.cu), segment by segment on a second stream
+//   4. conv_tail:  writes each sequence's new conv window into its slot, once
+//                  every chunk has read the windows it started from
+// Every tensor-core operand is rounded to fp16 (round to nearest) with fp32
+// accumulation; the state, A, T and the gates stay fp32.
 
 #include <cuda_fp16.h>
 
@@ -160,186 +160,7 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     }
 }
 
-// ---------------------------------------------------------------- 2. prep
-
-// One CTA per (chunk, unit); a unit is the q channels of a qk head, the k
-// channels of a qk head, or the v channels (and gates) of a value head.  The
-// chunk's raw rows and the 3 rows before it (from the previous chunk of the
-// same sequence, or from the conv-state slot for a sequence's first chunk)
-// are staged in shared memory; every output row is then conv1d + SiLU (+ L2
-// norm for q, k) of shared-memory data.  Results are assembled as tiles in the
-// tensor core's shared-memory layout and leave by bulk stores:
-//   q / k unit: rows C..2C-1 / 0..C-1 of [K ; Q*scale] (fp16, K-major, 128 rows x dk)
-//   v unit:     V^T fp16 (K-major, dv rows x C) and (g, beta) for the C rows
-// Rows past the end of a ragged chunk are written as zeros.
-constexpr int kPrepThreads = 256;
-
-template <typename T, int DK, int DV>
-struct PrepShape {
-    static constexpr int NCH = DK > DV ? DK : DV;  // staged channels per row (max over units)
-    static constexpr int VE = 16 / sizeof(T);      // elements per 16-byte vector
-    static constexpr int PAD = VE;                 // row padding: spreads rows over banks
-    static constexpr size_t XS_BYTES = (((size_t)(C + 3) * (NCH + PAD) * sizeof(T)) + 15) & ~(size_t)15;
-    static constexpr size_t TILE_BYTES = (size_t)C * NCH * sizeof(uint16_t);  // fp16 tile
-    static constexpr size_t W_BYTES = (size_t)NCH * 5 * sizeof(float);  // 4 taps per channel, then the biases
-    static constexpr size_t SMEM = XS_BYTES + TILE_BYTES + W_BYTES + C * sizeof(float2);
-};
-
-template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(ExtendArgs p) {
-    using S = PrepShape<T, DK, DV>;
-    if (batch_rejected(p)) return;
-    const int id = blockIdx.x, unit = blockIdx.y;
-    if (id >= p.hdr[kHdrNumChunks]) return;
-    const int4 ch = p.chunk_tab[id];
-    const int seq = ch.x, t0 = ch.y, n = ch.z, cidx = ch.w;
-    const int slot = p.slots[seq];
-    if (slot < 0 || slot >= p.P) return;
-    const LayerDims& d = p.d;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool isq = unit < d.HK, isk = !isq && unit < 2 * d.HK, isv = !isq && !isk;
-    const int nch = isv ? DV : DK;
-    const int ld = nch + S::PAD;  // staged row stride (elements)
-    const int hk = isq ? unit : unit - d.HK, h = unit - 2 * d.HK;
-    const int c_first = isq ? hk * DK : isk ? d.HK * DK + hk * DK : 2 * d.HK * DK + h * DV;  // first channel
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    T* xs = reinterpret_cast<T*>(smem_raw);  // row i <-> token t0 - 3 + i
-    char* tile = reinterpret_cast<char*>(smem_raw + S::XS_BYTES);
-    float4* wsm = reinterpret_cast<float4*>(smem_raw + S::XS_BYTES + S::TILE_BYTES);  // [nch] taps
-    float* bsm = reinterpret_cast<float*>(wsm + S::NCH);                                // [nch] biases
-    float2* gbs = reinterpret_cast<float2*>(smem_raw + S::XS_BYTES + S::TILE_BYTES + S::W_BYTES);
-    const T* x = reinterpret_cast<const T*>(p.x);
-    const T* w = reinterpret_cast<const T*>(p.conv_w);
-    const T* bias = reinterpret_cast<const T*>(p.conv_b);
-
-    // stage rows 3 .. n+2 (this chunk) with 16-byte loads; the 3 halo rows and the weights element-wise
-    {
-        const int vpr = nch / S::VE;  // vectors per row
-        const int nv = n * vpr;
-        for (int base = 0; base < nv; base += kPrepThreads * 4) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = base + u * kPrepThreads + tid;
-                if (e < nv) {
-                    const int r = e / vpr, c = (e % vpr) * S::VE;
-                    v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d.conv_dim + c_first + c);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = base + u * kPrepThreads + tid;
-                if (e < nv) {
-                    const int r = e / vpr, c = (e % vpr) * S::VE;
-                    *reinterpret_cast<uint4*>(xs + (size_t)(r + 3) * ld + c) = v[u];
-                }
-            }
-        }
-        const bool init = p.has_init ? p.has_init[seq] != 0 : true;
-        const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
-        for (int e = tid; e < 3 * nch; e += kPrepThreads) {
-            const int i = e / nch, c = e % nch;
-            T v;
-            if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + c_first + c];
-            else v = init ? cs[(size_t)(c_first + c) * 3 + i] : from_f<T>(0.f);
-            xs[(size_t)i * ld + c] = v;
-        }
-        for (int c = tid; c < nch; c += kPrepThreads) {
-            const int cg = c_first + c;
-            wsm[c] = make_float4(to_f(w[(size_t)cg * 4]), to_f(w[(size_t)cg * 4 + 1]), to_f(w[(size_t)cg * 4 + 2]),
-                                 to_f(w[(size_t)cg * 4 + 3]));
-            bsm[c] = bias ? to_f(bias[cg]) : 0.f;
-        }
-    }
-    __syncthreads();
-    // SiLU with the fast exponential and division: their error (a few ulp) is far below the
-    // tf32 rounding every prep output goes through
-    auto silu = [](float x) { return __fdividef(x, 1.0f + __expf(-x)); };
-    // conv + SiLU of staged column c at output row r (r < n)
-    auto conv = [&](int c, int r) -> float {
-        const float4 wc = wsm[c];
-        float acc = bsm[c];
-        acc = fmaf(wc.x, to_f(xs[(size_t)r * ld + c]), acc);
-        acc = fmaf(wc.y, to_f(xs[(size_t)(r + 1) * ld + c]), acc);
-        acc = fmaf(wc.z, to_f(xs[(size_t)(r + 2) * ld + c]), acc);
-        acc = fmaf(wc.w, to_f(xs[(size_t)(r + 3) * ld + c]), acc);
-        return silu(acc);
-    };
-    if (!isv) {
-        // warp w: rows 8w .. 8w+7; lane (rr = lane & 7, cc = lane >> 3) takes row 8w + rr and the
-        // column quads 4 cg + cc, so every 8-lane group writes whole 128-byte core matrices of the
-        // half tile (a K-major 64-row tile); the L2 norm reduces over the 4 lanes of a row
-        const int rr = lane & 7, cc = lane >> 3;
-        const int r = 8 * warp + rr;
-        float y[DK / 16][4];
-        float ss = 0.f;
-#pragma unroll
-        for (int cg = 0; cg < DK / 16; ++cg)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                y[cg][u] = r < n ? conv(4 * (4 * cg + cc) + u, r) : 0.f;
-                ss += y[cg][u] * y[cg][u];
-            }
-        ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-        const float sc = (r < n) ? rsqrtf(ss + d.eps) * (isq ? d.scale : 1.f) : 0.f;
-#pragma unroll
-        for (int cg = 0; cg < DK / 16; ++cg)
-            *reinterpret_cast<uint2*>(tile + tc::kmajor_off16(r, 4 * (4 * cg + cc), C)) =
-                make_uint2(tc::pack_f16(y[cg][0] * sc, y[cg][1] * sc), tc::pack_f16(y[cg][2] * sc, y[cg][3] * sc));
-    } else {
-        // V^T tile: thread (f, 4 consecutive rows) -> 4 fp16 of the K-major tile (8 lanes per core matrix)
-        for (int idx = tid; idx < DV * (C / 4); idx += kPrepThreads) {
-            const int ff = idx & 7, cq = (idx >> 3) & 3, rest = idx >> 5;
-            const int fg = rest % (DV / 8), rg = rest / (DV / 8);
-            const int f = 8 * fg + ff, r4 = 4 * (4 * rg + cq);
-            // four consecutive rows of channel f from a sliding window of 7 staged rows
-            const float4 wc = wsm[f];
-            const float b0 = bsm[f];
-            float xw[7];
-#pragma unroll
-            for (int i = 0; i < 7; ++i) xw[i] = to_f(xs[(size_t)(r4 + i) * ld + f]);
-            float y[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float acc = fmaf(wc.x, xw[u], b0);
-                acc = fmaf(wc.y, xw[u + 1], acc);
-                acc = fmaf(wc.z, xw[u + 2], acc);
-                acc = fmaf(wc.w, xw[u + 3], acc);
-                y[u] = r4 + u < n ? silu(acc) : 0.f;
-            }
-            *reinterpret_cast<uint2*>(tile + tc::kmajor_off16(f, r4, DV)) =
-                make_uint2(tc::pack_f16(y[0], y[1]), tc::pack_f16(y[2], y[3]));
-        }
-        if (tid < C) {
-            float2 gb = make_float2(0.f, 0.f);
-            if (tid < n) {
-                const size_t row = (size_t)(t0 + tid) * d.HV + h;
-                const float av = to_f(reinterpret_cast<const T*>(p.a)[row]);
-                const float bv2 = to_f(reinterpret_cast<const T*>(p.b)[row]);
-                gb = make_float2(-expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]), sigmoid_f(bv2));
-            }
-            gbs[tid] = gb;
-        }
-    }
-    tc::fence_smem_to_async();
-    __syncthreads();
-    if (tid == 0) {
-        if (!isv) {
-            // the 64-row half tile holds DK/8 blocks of 1 KB (one per group of 8 columns); in the
-            // 128-row [K ; Q] tile those blocks sit 2 KB apart, the q half 1 KB after the k half
-            char* dst = reinterpret_cast<char*>(p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK)) + (isq ? 1024 : 0);
-            for (int q = 0; q < DK / 8; ++q) tc::bulk_s2g(dst + 2048 * q, tc::smem_u32(tile) + 1024 * q, 1024);
-        } else {
-            tc::bulk_s2g(p.VT + ((size_t)id * d.HV + h) * (DV * C), tc::smem_u32(tile), DV * C * 2);
-            tc::bulk_s2g(p.GB + ((size_t)id * d.HV + h) * C, tc::smem_u32(gbs), C * 8);
-        }
-        tc::bulk_commit();
-        tc::bulk_wait_read_all();
-    }
-}
-
-// ---------------------------------------------------------------- 3. conv tail
+// ---------------------------------------------------------------- conv tail
 
 template <typename T>
 __global__ void __launch_bounds__(256) conv_tail_kernel(ExtendArgs p) {
@@ -365,9 +186,6 @@ __global__ void __launch_bounds__(256) conv_tail_kernel(ExtendArgs p) {
     }
     cs[0] = nv[0]; cs[1] = nv[1]; cs[2] = nv[2];
 }
-
-// ---------------------------------------------------------------- 4. intra
-// on tensor cores, in gdn_intra_tc.cu
 
 // A second stream (at the device's greatest priority) with one fork event per
 // segment and a join event, per host thread and device, created by the first
@@ -479,10 +297,10 @@ __global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
     float* Kf = Wf + C * DK;    // [C][DK] rows s < m of K
     float* Vp = Kf + C * DK;    // [C][DVS] v'_s, this CTA's columns
     float* coef = Vp + C * DVS; // [C] e^{gamma_{m-1} - gamma_s}
-    const char* WQg = reinterpret_cast<const char*>(p.WQ + (id * d.HV + h) * (2 * C * DK));
+    const char* Wg = reinterpret_cast<const char*>(p.W + (id * d.HV + h) * (C * DK));
     const char* KQg = reinterpret_cast<const char*>(p.KQ + (id * d.HK + h / d.G) * (2 * C * DK));
     const char* Ug = reinterpret_cast<const char*>(p.U + (id * d.HV + h) * (DV * C));
-    const float* gm = p.gam + (id * d.HV + h) * C;
+    const float4* gv = p.GV + (id * d.HV + h) * C;  // .z = gamma
     auto h2f = [](const char* q) { return __half2float(*reinterpret_cast<const __half*>(q)); };
     for (int e = tid; e < DK * DVS / 4; e += 256) {
         const int f = e / (DVS / 4), j4 = e % (DVS / 4);
@@ -490,20 +308,20 @@ __global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
     }
     for (int e = tid; e < m * DK; e += 256) {
         const int sr = e / DK, f = e % DK;
-        Wf[e] = h2f(WQg + tc::kmajor_off16(sr, f, 2 * C));
-        Kf[e] = h2f(KQg + tc::kmajor_off16(sr, f, 2 * C));
+        Wf[e] = h2f(Wg + tc::sw128_off(sr, f, C));
+        Kf[e] = h2f(KQg + tc::sw128_off(sr, f, 2 * C));
     }
-    if (tid < m) coef[tid] = expf(gm[m - 1] - gm[tid]);
+    if (tid < m) coef[tid] = expf(gv[m - 1].z - gv[tid].z);
     __syncthreads();
     for (int e = tid; e < m * DVS; e += 256) {  // v'_s[j] = u_s[j] - sum_f w_s[f] S_c[f][j]
         const int sr = e / DVS, jl = e % DVS;
-        float acc = h2f(Ug + tc::kmajor_off16(j0 + jl, sr, DV));
+        float acc = h2f(Ug + tc::sw128_off(j0 + jl, sr, DV));
 #pragma unroll 8
         for (int f = 0; f < DK; ++f) acc = fmaf(-Wf[sr * DK + f], Sc[f * DVS + jl], acc);
         Vp[e] = acc;
     }
     __syncthreads();
-    const float eg = expf(gm[m - 1]);
+    const float eg = expf(gv[m - 1].z);
     for (int e = tid; e < DK * DVS; e += 256) {
         const int f = e / DVS, jl = e % DVS;
         float acc = eg * Sc[e];
@@ -517,9 +335,6 @@ constexpr size_t ckpt_finish_smem() {
     return sizeof(float) * ((size_t)DK * (DV / kCkptSplit) + 2 * (size_t)C * DK + (size_t)C * (DV / kCkptSplit) + C);
 }
 
-// ---------------------------------------------------------------- 5. state pass
-// on tensor cores, in gdn_state_tc.cu
-
 template <typename T, int DK, int DV>
 cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     cudaError_t e;
@@ -527,34 +342,26 @@ cudaError_t launch_extend_t(const ExtendArgs& p, cudaStream_t s) {
     chunk_map_kernel<<<1, 1024, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark_launch(s, 1);
-    {
-        const size_t shm = PrepShape<T, DK, DV>::SMEM;
-        if ((e = cudaFuncSetAttribute(prep_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)shm)) != cudaSuccess)
-            return e;
-        prep_kernel<T, DK, DV><<<dim3(p.max_chunks, 2 * p.d.HK + p.d.HV), kPrepThreads, shm, s>>>(p);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    mark_launch(s, 2);
     if (p.ck_idx) {  // the conv windows at the checkpoint boundaries, before the conv-state update
         ckpt_conv_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    mark_launch(s, 3);
-    // segment by segment: intra on `s`; the state pass of segment k on the side stream once intra
-    // has finished segment k, alongside intra of segment k+1
+    // segment by segment: the per-chunk step on `s`; the state pass of segment k on the side stream
+    // once the per-chunk step has finished segment k, alongside the per-chunk step of segment k+1
     SideStream* side = nullptr;
     if ((e = side_stream(&side)) != cudaSuccess) return e;
     for (int k = 0; k < p.nseg; ++k) {
-        if ((e = launch_intra<DK, DV>(p, k, s)) != cudaSuccess) return e;
+        if ((e = launch_chunk<T, DK, DV>(p, k, s)) != cudaSuccess) return e;
         if ((e = cudaEventRecord(side->seg[k], s)) != cudaSuccess) return e;
         if ((e = cudaStreamWaitEvent(side->s, side->seg[k], 0)) != cudaSuccess) return e;
         if (k == 0) mark_launch(side->s, 6);
         if ((e = launch_state<T, DK, DV>(p, k, side->s)) != cudaSuccess) return e;
     }
-    mark_launch(s, 4);
+    mark_launch(s, 2);
+    // the new conv windows, once every chunk has staged the windows its sequence started from
+    conv_tail_kernel<T><<<dim3(p.N, (p.d.conv_dim + 255) / 256), 256, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark_launch(s, 3);
     mark_launch(side->s, 7);
     if (p.ck_idx) {  // the checkpoint states off the chunk edges, once the state pass stored the edges
         constexpr size_t shm = ckpt_finish_smem<DK, DV>();
@@ -590,13 +397,10 @@ size_t walk_extend_workspace(const LayerDims& d, int max_N, int max_T, char* bas
     char* rank_off = take(((size_t)max_N + 1) * sizeof(int32_t));
     char* chunk_list = take(mc * sizeof(int32_t));
     char* kq = take(mc * d.HK * 2 * C * d.dk * sizeof(uint16_t));
-    char* vt = take(units * d.dv * C * sizeof(uint16_t));
-    char* gb = take(units * C * sizeof(float2));
-    char* wq = take(units * 2 * C * d.dk * sizeof(uint16_t));
-    char* aq = take(units * C * C * sizeof(uint16_t));
-    char* kt = take(units * d.dk * C * sizeof(uint16_t));
+    char* w = take(units * C * d.dk * sizeof(uint16_t));
     char* u = take(units * d.dv * C * sizeof(uint16_t));
-    char* gam = take(units * C * sizeof(float));
+    char* aq = take(units * C * C * sizeof(uint16_t));
+    char* gv = take(units * C * sizeof(float4));
     if (e) {
         e->max_chunks = (int)mc;
         e->hdr = reinterpret_cast<int32_t*>(base);
@@ -606,13 +410,10 @@ size_t walk_extend_workspace(const LayerDims& d, int max_N, int max_T, char* bas
         e->rank_off = reinterpret_cast<int32_t*>(rank_off);
         e->chunk_list = reinterpret_cast<int32_t*>(chunk_list);
         e->KQ = reinterpret_cast<uint16_t*>(kq);
-        e->VT = reinterpret_cast<uint16_t*>(vt);
-        e->GB = reinterpret_cast<float2*>(gb);
-        e->WQ = reinterpret_cast<uint16_t*>(wq);
-        e->AQ = reinterpret_cast<uint16_t*>(aq);
-        e->KT = reinterpret_cast<uint16_t*>(kt);
+        e->W = reinterpret_cast<uint16_t*>(w);
         e->U = reinterpret_cast<uint16_t*>(u);
-        e->gam = reinterpret_cast<float*>(gam);
+        e->AQ = reinterpret_cast<uint16_t*>(aq);
+        e->GV = reinterpret_cast<float4*>(gv);
     }
     return off;
 }

@@ -3,42 +3,34 @@
 //
 // One CTA per (sequence, value head), looping over the sequence's chunks.  The
 // products are formed transposed, with the value dimension (dv) as the MMA's
-// M, so that every accumulator row belongs to one thread; K~ is read MN-major
-// (its rows s run along the product's K), every other operand K-major:
+// M, so that every accumulator row belongs to one thread.  Per chunk, from the
+// tiles the per-chunk step wrote ([K ; Q], W, U^T, Aqk and the gate vectors):
 //
-//   [X^T | O^T]  = S^T [W ; Qg]^T           M=dv N=128 K=dk   (X = W S, O = Qg S)
-//   V'^T         = U^T - X^T                 CUDA cores, per thread row j
-//   Snew^T       = V'^T K~                   M=dv N=dk  K=64  (K~ = diag(e^{gamma_n-gamma}) K)
-//   S^T         <- e^{gamma_n} S^T + Snew^T  CUDA cores, fp32 in registers
-//   O^T         += V'^T Aqk^T                M=dv N=64  K=64
+//   X^T     = S^T W^T                       M=dv N=64 K=dk   (on the chain)
+//   Oi^T    = S^T Q^T                       M=dv N=64 K=dk   (off the chain)
+//   V'^T    = U^T - X^T,  Vs'^T = V'^T diag(f),  f_s = e^{gamma_n - gamma_s}
+//   Snew^T  = Vs'^T K                       M=dv N=dk K=64   (K read MN-major; on the chain)
+//   S^T    <- e^{gamma_n} S^T + Snew^T      CUDA cores, fp32 in registers
+//   Oq^T    = V'^T Aqk^T                    M=dv N=64 K=64   (off the chain)
+//   o_r     = e^{gamma_r} Oi_r + Oq_r
 //
-// where Qg = diag(e^gamma) Q (q carries the output scale).  The chain from one
-// chunk's state to the next runs through the first product, V', the state
-// product and the update; everything else is kept off it:
-//   - a ninth warp only issues the MMAs, so the eight compute warps never
-//     wait behind an issue loop; it queues the output product right behind
-//     the state product (the tensor core runs them in order) and never waits
-//     for it;
-//   - a tenth warp issues every bulk copy: each tile buffer has a "free"
-//     barrier that the product reading it signals on completion (or the
-//     compute warps, for U^T), and the copier refills the buffer as soon as
-//     it completes, so no copy issue or wait sits on the chain;
-//   - the fp32 state lives in registers (each thread holds one half of row j
-//     of S^T), the state product goes to a fresh accumulator and the update
-//     is one FMA per element, written straight into the fp16 copy of S^T that
-//     the first product reads from tensor memory (so that product reads only
-//     [W ; Qg] from shared memory);
-//   - [X^T | O^T] is double-buffered in tensor memory: a chunk's outputs are
-//     read and stored while the next chunk's first product runs;
-//   - [W ; Qg] and K~ are double-buffered and copied two chunks ahead;
-//   - the tiles [W ; Qg], K~ and Aqk (written by the intra-chunk kernel as
-//     fp16 in the tensor core's layout) each have their own barrier and are
-//     refetched as soon as the product that reads them completes;
-//   - the intra-chunk kernel writes U^T in the layout of the V'^T operand
-//     tile; it lands in a tile of its own, so the next chunk's copy starts
-//     as soon as V' has been formed from it.
-// The two compute warps of a TMEM sub-partition share its 32 accumulator rows
-// and take one half of the columns each.
+// (the chunked WY/UT form of the gated delta rule; q carries the output scale).
+// The chain from one chunk's state to the next is X, V', the state product and
+// the update, and every step of it is cut in two so the next one starts on the
+// first half:
+//   - the state update writes the fp16 copy of S^T (the A operand of X and Oi,
+//     in tensor memory) in two column halves, each released on its own
+//     barrier, so the next chunk's X issues its first k-steps while the second
+//     half is still being updated;
+//   - V' is formed in two halves of the chunk's rows, each released on its own
+//     barrier, so the state product issues its first k-steps meanwhile;
+//   - the output products run on the tensor core while the CUDA cores form V'
+//     and update the state; a chunk's outputs are read, scaled and staged while
+//     the next chunk's state product runs, and stored after its update.
+// A ninth warp only issues MMAs; a tenth issues every bulk copy, refilling
+// each double-buffered tile as soon as its last reader releases it.  The two
+// compute warps of a TMEM sub-partition share its 32 accumulator rows and
+// take one half of the columns each.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -48,14 +40,44 @@ namespace {
 
 constexpr int C = kChunk;
 constexpr int NCW = 8;                  // compute warps
-constexpr int NCHAIN = (NCW + 1) * 32;  // + the issuing warp: the threads on the state chain
-constexpr int ISSUER = NCW * 32;        // its lane 0
-constexpr int COPIER = NCHAIN;          // lane 0 of a tenth warp, which issues every bulk copy
-constexpr int NT = NCHAIN + 32;
-constexpr int kChainBarrier = 1;        // named barrier of the chain threads
+constexpr int ISSUER = NCW * 32;        // lane 0 of the ninth warp
+constexpr int COPIER = (NCW + 1) * 32;  // lane 0 of the tenth warp
+constexpr int NT = (NCW + 2) * 32;
+constexpr int kCwBarrier = 1;           // named barrier of the compute warps
 
-// barrier among the `n` threads of named barrier `id`; true when `pred` holds in all of them
-__device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
+// bf16 outputs are staged in shared memory and leave as 16-byte vectors; fp32 outputs (whose
+// staging tiles would not fit) are stored by each thread
+template <typename T>
+constexpr bool kStageOut = sizeof(T) == 2;
+
+template <typename T, int DK, int DV>
+struct StateSmem {
+    // fp16 operand tiles in the 128-byte swizzled layout (1024-byte aligned), double-buffered and
+    // copied two chunks ahead
+    uint16_t kq[2][2 * C * DK];  // [K ; Q]: K rows (MN-major B of Snew), Q rows (B of Oi)
+    uint16_t w[2][C * DK];       // W (B of X)
+    uint16_t ut[2][DV * C];      // U^T
+    uint16_t aq[2][C * C];       // Aqk (B of Oq)
+    uint16_t vt[DV * C];         // V'^T: A of Oq
+    uint16_t vs[DV * C];         // Vs'^T: A of Snew
+    T ostage[kStageOut<T> ? 2 : 1][kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV]
+    float4 gv[2][C];             // per row: e^{gamma_r}, f_r, gamma_r, e^{gamma_n}
+    float eg[2][C];              // e^{gamma_r} of the chunk whose outputs are pending
+    unsigned long long full_kq[2], full_w[2], full_u[2], full_aq[2];
+    unsigned long long free_kq[2], free_w[2], free_u[2], free_aq[2];
+    unsigned long long bar_x, bar_s, bar_o, bar_vp[2], bar_sa[2];
+    uint32_t tmem_base;
+};
+
+template <typename T, int DK, int DV>
+constexpr size_t state_smem_bytes() {
+    return sizeof(StateSmem<T, DK, DV>) + 1024;  // + room to align the tiles on 1024 bytes
+}
+static_assert(state_smem_bytes<__nv_bfloat16, 128, 128>() <= 227 * 1024, "state pass shared memory");
+static_assert(state_smem_bytes<float, 128, 128>() <= 227 * 1024, "state pass shared memory");
+
+// barrier among the compute warps; true when `pred` holds in all of them
+__device__ __forceinline__ bool cw_and(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -63,57 +85,34 @@ __device__ __forceinline__ bool bar_and(int id, int n, bool pred) {
         "barrier.red.and.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(n)
+        : "r"((uint32_t)pred), "r"(kCwBarrier), "r"(NCW * 32)
         : "memory");
     return r != 0;
 }
 
-// bf16 outputs are staged in shared memory and leave as 16-byte vectors while
-// the next state product runs; fp32 outputs (whose staging tile would not fit)
-// are stored by each thread
-template <typename T>
-constexpr bool kStageOut = sizeof(T) == 2;
-
-template <typename T, int DK, int DV>
-struct StateTcSmem {
-    // fp16 operand tiles (16-bit K-major layout); [W ; Qg] and K~ are double-buffered and copied
-    // two chunks ahead
-    uint16_t wq[2][2 * C * DK];  // [W ; Qg] tiles (bulk copy): 128 rows x DK
-    uint16_t kt[2][C * DK];      // K~ tiles (bulk copy): C rows (s) x DK (i), the MN-major B of Snew^T
-    uint16_t aq[C * C];       // Aqk tile (bulk copy): C rows (r) x C (s)
-    uint16_t ut[DV * C];      // U^T tile (bulk copy): DV rows (j) x C (s)
-    uint16_t vt[DV * C];      // V'^T = U^T - X^T, same layout: the A operand of the state and output products
-    T ostage[kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV] on their way out
-    unsigned long long bar_x, bar_s, bar_o, bar_wq[2], bar_kt[2], bar_aq, bar_u;
-    // the copier's signals that a tile buffer is free again: the product reading it has completed
-    // (tensor-core commits), or V' has read U^T (one arrival per compute warp)
-    unsigned long long free_wq[2], free_kt[2], free_aq, free_u;
-    uint32_t tmem_base;
-};
-
-
 // fp16 copy of 32 consecutive values of S^T row j (this thread's lane) into 16 columns of the
 // tensor-memory A operand: two fp16 per column, the even column of S^T in the low half
 __device__ __forceinline__ void put_sa32(uint32_t taddr, const float* v) {
-    uint32_t w[16];
+    uint32_t wv[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) w[i] = tc::pack_f16(v[2 * i], v[2 * i + 1]);
-    tc::tmem_st16(taddr, w);
+    for (int i = 0; i < 16; ++i) wv[i] = tc::pack_f16(v[2 * i], v[2 * i + 1]);
+    tc::tmem_st16(taddr, wv);
 }
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) {
+    using Sm = StateSmem<T, DK, DV>;
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int HV = d.HV;
     // the ranks holding chunks of this segment's piece of the chunk list (all heads of the longer
     // sequence first); each CTA takes its sequence's chunks inside the piece
-    const int r = p.hdr[kHdrSegRank + seg] + (int)(blockIdx.x / HV);
-    if (r >= p.N) return;
-    const int h = blockIdx.x % HV, nseq = p.seq_order[r];
+    const int rk = p.hdr[kHdrSegRank + seg] + (int)(blockIdx.x / HV);
+    if (rk >= p.N) return;
+    const int h = blockIdx.x % HV, hk = h / d.G, nseq = p.seq_order[rk];
     const int lo = p.hdr[kHdrSegOff + seg], hi = lo + p.hdr[kHdrSegCnt + seg];
-    const int ro = p.rank_off[r];
-    const int a = max(lo, ro), b = min(hi, p.rank_off[r + 1]);
+    const int ro = p.rank_off[rk];
+    const int a = max(lo, ro), b = min(hi, p.rank_off[rk + 1]);
     if (a >= b) return;
     const int c_first = p.seq_chunk0[nseq];
     const int c_begin = c_first + (a - ro), c_end = c_begin + (b - a);
@@ -127,59 +126,57 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             out[((size_t)(r0 + e / DV) * HV + h) * DV + e % DV] = from_f<T>(0.f);
         return;
     }
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    StateTcSmem<T, DK, DV>& sm = *reinterpret_cast<StateTcSmem<T, DK, DV>*>(smem_raw);
-    const uint32_t bar_x = tc::smem_u32(&sm.bar_x), bar_s = tc::smem_u32(&sm.bar_s),
-                   bar_o = tc::smem_u32(&sm.bar_o), bar_aq = tc::smem_u32(&sm.bar_aq),
-                   bar_u = tc::smem_u32(&sm.bar_u);
-    constexpr uint32_t WQ_BYTES = 2 * C * DK * 2, AQ_BYTES = C * C * 2, KT_BYTES = DK * C * 2, U_BYTES = DV * C * 2;
-    // buffer b = (id - c_begin) & 1 of the double-buffered tiles; its barrier completes once every
-    // other chunk, so a chunk waits on parity ((id - c_begin) >> 1) & 1
-    auto bar_wq = [&](int b) { return tc::smem_u32(&sm.bar_wq[b]); };
-    auto bar_kt = [&](int b) { return tc::smem_u32(&sm.bar_kt[b]); };
-    auto fetch_wq = [&](int id) {
-        const int b = (id - c_begin) & 1;
-        tc::mbar_expect_tx(bar_wq(b), WQ_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.wq[b]), p.WQ + ((size_t)id * HV + h) * (2 * C * DK), WQ_BYTES, bar_wq(b));
+    extern __shared__ unsigned char smem_raw[];
+    Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    constexpr uint32_t KQ_BYTES = 2 * C * DK * 2, W_BYTES = C * DK * 2, U_BYTES = DV * C * 2, AQ_BYTES = C * C * 2,
+                       GV_BYTES = C * 16;
+    auto bar = [](unsigned long long& m) { return tc::smem_u32(&m); };
+    auto fetch_kq = [&](int id) {
+        const int bb = (id - c_begin) & 1;
+        tc::mbar_expect_tx(bar(sm.full_kq[bb]), KQ_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.kq[bb]), p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK), KQ_BYTES,
+                     bar(sm.full_kq[bb]));
     };
-    auto fetch_kt = [&](int id) {
-        const int b = (id - c_begin) & 1;
-        tc::mbar_expect_tx(bar_kt(b), KT_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.kt[b]), p.KT + ((size_t)id * HV + h) * (DK * C), KT_BYTES, bar_kt(b));
+    auto fetch_w = [&](int id) {
+        const int bb = (id - c_begin) & 1;
+        tc::mbar_expect_tx(bar(sm.full_w[bb]), W_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.w[bb]), p.W + ((size_t)id * HV + h) * (C * DK), W_BYTES, bar(sm.full_w[bb]));
     };
-    auto u_src = [&](int id) { return p.U + ((size_t)id * HV + h) * (DV * C); };
     auto fetch_u = [&](int id) {
-        tc::mbar_expect_tx(bar_u, U_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.ut), u_src(id), U_BYTES, bar_u);
+        const int bb = (id - c_begin) & 1;
+        tc::mbar_expect_tx(bar(sm.full_u[bb]), U_BYTES + GV_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.ut[bb]), p.U + ((size_t)id * HV + h) * (DV * C), U_BYTES, bar(sm.full_u[bb]));
+        tc::bulk_g2s(tc::smem_u32(sm.gv[bb]), p.GV + ((size_t)id * HV + h) * C, GV_BYTES, bar(sm.full_u[bb]));
     };
     auto fetch_aq = [&](int id) {
-        tc::mbar_expect_tx(bar_aq, AQ_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.aq), p.AQ + ((size_t)id * HV + h) * (C * C), AQ_BYTES, bar_aq);
+        const int bb = (id - c_begin) & 1;
+        tc::mbar_expect_tx(bar(sm.full_aq[bb]), AQ_BYTES);
+        tc::bulk_g2s(tc::smem_u32(sm.aq[bb]), p.AQ + ((size_t)id * HV + h) * (C * C), AQ_BYTES, bar(sm.full_aq[bb]));
     };
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     if (tid == ISSUER) {
-        tc::mbar_init(bar_x, 1);
-        tc::mbar_init(bar_s, 1);
-        tc::mbar_init(bar_o, 1);
-        for (int b = 0; b < 2; ++b) {
-            tc::mbar_init(bar_wq(b), 1);
-            tc::mbar_init(bar_kt(b), 1);
+        for (int bb = 0; bb < 2; ++bb) {
+            tc::mbar_init(bar(sm.full_kq[bb]), 1);
+            tc::mbar_init(bar(sm.full_w[bb]), 1);
+            tc::mbar_init(bar(sm.full_u[bb]), 1);
+            tc::mbar_init(bar(sm.full_aq[bb]), 1);
+            tc::mbar_init(bar(sm.free_kq[bb]), 1);
+            tc::mbar_init(bar(sm.free_w[bb]), 1);
+            tc::mbar_init(bar(sm.free_u[bb]), NCW);
+            tc::mbar_init(bar(sm.free_aq[bb]), NCW + 1);  // the output product's commit + every compute warp
+            tc::mbar_init(bar(sm.bar_vp[bb]), NCW / 2);
+            tc::mbar_init(bar(sm.bar_sa[bb]), NCW / 2);
         }
-        tc::mbar_init(bar_aq, 1);
-        tc::mbar_init(bar_u, 1);
-        for (int b = 0; b < 2; ++b) {
-            tc::mbar_init(tc::smem_u32(&sm.free_wq[b]), 1);
-            tc::mbar_init(tc::smem_u32(&sm.free_kt[b]), 1);
-        }
-        tc::mbar_init(tc::smem_u32(&sm.free_aq), 1);
-        tc::mbar_init(tc::smem_u32(&sm.free_u), NCW);
+        tc::mbar_init(bar(sm.bar_x), 1);
+        tc::mbar_init(bar(sm.bar_s), 1);
+        tc::mbar_init(bar(sm.bar_o), 1);
         tc::fence_mbar_init();
         for (int id = c_begin; id < c_end && id < c_begin + 2; ++id) {
-            fetch_wq(id);
-            fetch_kt(id);
+            fetch_kq(id);
+            fetch_w(id);
+            fetch_u(id);
+            fetch_aq(id);
         }
-        fetch_aq(c_begin);
-        fetch_u(c_begin);
     }
 
     // compute warps: thread (sp, half, lane) owns row j of S^T, columns half * DK/2 .. + DK/2
@@ -207,259 +204,263 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             ck_dst = p.ck_states + ((size_t)row * HV + h) * DK * DV;
         }
     }
-    int4 ch = p.chunk_tab[c_begin];
-    float gl = p.gam[((size_t)c_begin * HV + h) * C + ch.z - 1];  // gamma_n of this chunk
-    int4 ch_nx = c_begin + 1 < c_end ? p.chunk_tab[c_begin + 1] : ch;
-    tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
-    // [X^T | O^T] double buffer at tm, tm + 128; Snew^T (DK columns) at tm + 256; the fp16 copy of
-    // S^T, the A operand of the first product (DK / 2 columns), at tm + 384
-    const uint32_t tS = tm + 256, tA = tm + 384;
-    static_assert(DK <= 128, "tensor-memory layout");
-    // this thread's DK / 2 state columns of row j into the A operand (lanes past the rows of a
-    // 64-row tile hold values no product reads)
+    // tensor memory: the fp16 copy of S^T (DK / 2 columns) at tm, X^T at tm + 64, Oi^T and Oq^T
+    // double-buffered at tm + 128 + 64 b and tm + 256 + 64 b, Snew^T (DK columns) at tm + 384
+    const uint32_t tA = tm, tX = tm + 64, tSn = tm + 384;
+    auto tOi = [&](int bb) { return tm + 128 + 64 * bb; };
+    auto tOq = [&](int bb) { return tm + 256 + 64 * bb; };
+    static_assert(DK <= 128 && DV <= 128, "tensor-memory layout");
     const uint32_t tA_row = tA + lane_base + half * (DK / 4);
-    if (warp < NCW) {
+    if (warp < NCW) {  // the starting state's fp16 copy, released as both halves of the first chunk's X
 #pragma unroll
         for (int cc = 0; cc < DK / 2; cc += 32) put_sa32(tA_row + cc / 2, &s[cc]);
         tc::tmem_st_wait();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
 
-    // rows t < n of O (chunk at row t0), this thread's column j and half of the rows, from the
-    // O^T half of an [X^T | O^T] buffer: into the staging tile, or straight to global memory
-    auto put_out = [&](uint32_t tXO, int t0, int n) {
+    // the outputs of chunk `it` (rows t < n at packed row t0), this thread's column j and half of the
+    // rows: o = e^{gamma_r} Oi + Oq, staged (bf16) or stored (fp32)
+    auto put_out = [&](int it, int t0, int n) {
+        const int bb = it & 1;
 #pragma unroll
         for (int cc = 0; cc < C / 2; cc += 16) {
             const int c0 = half * (C / 2) + cc;
-            float o[16];
-            tc::tmem_ld16(tXO + lane_base + 64 + c0, o);
+            float oi[16], oq[16];
+            tc::tmem_ld16(tOi(bb) + lane_base + c0, oi);
+            tc::tmem_ld16(tOq(bb) + lane_base + c0, oq);
             tc::tmem_ld_wait();
             if (rowv)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    if constexpr (kStageOut<T>) sm.ostage[(c0 + i) * DV + j] = from_f<T>(o[i]);
-                    else if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + j] = from_f<T>(o[i]);
+                    const float o = fmaf(sm.eg[bb][c0 + i], oi[i], oq[i]);
+                    if constexpr (kStageOut<T>) sm.ostage[bb][(c0 + i) * DV + j] = from_f<T>(o);
+                    else if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + j] = from_f<T>(o);
                 }
         }
     };
-    // (compute warps) the staged rows t < n leave as 16-byte vectors
-    auto send_out = [&](int t0, int n) {
+    // (compute warps, after the named barrier) the staged rows t < n leave as 16-byte vectors
+    auto send_out = [&](int it, int t0, int n) {
         if constexpr (kStageOut<T>) {
             constexpr int VPR = DV * (int)sizeof(T) / 16;  // vectors per row
             for (int e = tid; e < n * VPR; e += NCW * 32) {
                 const int r = e / VPR, v = e % VPR;
                 reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * HV + h) * DV)[v] =
-                    reinterpret_cast<const uint4*>(sm.ostage + r * DV)[v];
+                    reinterpret_cast<const uint4*>(sm.ostage[it & 1] + r * DV)[v];
             }
         }
     };
 
     bool ok = true;
-    int prev_t0 = 0, prev_n = 0;  // the chunk whose outputs are still in tensor memory
-    if (warp > NCW) {
-        // ---- the copier: each tile buffer is refilled as soon as the chain frees it, in the order
-        // the chain frees them ([W ; Qg] after the first product, U^T after V', K~ after the state
-        // product, Aqk after the output product).  The next release of a buffer needs the copy issued
-        // here, so none of these barriers can complete twice before this lane has seen the first.
-        if (tid == COPIER) {
+    if (warp == NCW + 1) {
+        // ---- the copier: each buffer is refilled for the chunk two ahead as soon as its readers have
+        // released it (W after X, [K ; Q] after the state product, U^T and the gate vectors once V'
+        // and the output scale have been formed, Aqk once its product and the outputs are done).
+        // The next release of a buffer needs the copy issued here, so none of these barriers can
+        // complete twice before this lane has seen the first.
+        if (lane == 0) {
+            for (int id = c_begin; id + 2 < c_end && ok; ++id) {
+                const int it = id - c_begin, bb = it & 1;
+                const uint32_t pb = (uint32_t)(it >> 1) & 1u;
+                ok = tc::mbar_wait(bar(sm.free_w[bb]), pb);
+                if (ok) fetch_w(id + 2);
+                if (ok) ok = tc::mbar_wait(bar(sm.free_u[bb]), pb);
+                if (ok) fetch_u(id + 2);
+                if (ok) ok = tc::mbar_wait(bar(sm.free_kq[bb]), pb);
+                if (ok) fetch_kq(id + 2);
+                if (ok) ok = tc::mbar_wait(bar(sm.free_aq[bb]), pb);
+                if (ok) fetch_aq(id + 2);
+            }
+        }
+    } else if (warp == NCW) {
+        // ---- the MMA issuer
+        if (lane == 0) {
             for (int id = c_begin; id < c_end && ok; ++id) {
                 const int it = id - c_begin, bb = it & 1;
                 const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
-                if (id + 2 < c_end) {  // tiles two chunks ahead into L2, so their copies wait on L2 only
-                    const size_t nx = (size_t)(id + 2) * HV + h;
-                    tc::bulk_prefetch_l2(p.WQ + nx * (2 * C * DK), WQ_BYTES);
-                    tc::bulk_prefetch_l2(p.KT + nx * (DK * C), KT_BYTES);
-                    tc::bulk_prefetch_l2(p.AQ + nx * (C * C), AQ_BYTES);
-                    tc::bulk_prefetch_l2(u_src(id + 2), U_BYTES);
+                ok = tc::mbar_wait(bar(sm.full_w[bb]), pb) && tc::mbar_wait(bar(sm.full_kq[bb]), pb);
+                const uint32_t bw = tc::smem_u32(sm.w[bb]), bkq = tc::smem_u32(sm.kq[bb]);
+                constexpr uint32_t ix = tc::idesc_f16(DV, 64);
+                // X^T = S^T W^T, each half of S^T's columns as soon as the update has written it
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (ok) ok = tc::mbar_wait(bar(sm.bar_sa[hh]), ph);
+                    tc::fence_after_sync();
+                    if (ok)
+#pragma unroll
+                        for (int k = hh * (DK / 32); k < (hh + 1) * (DK / 32); ++k)
+                            tc::mma_f16_ta(tX, tA + 8 * k, tc::desc_sw128_k(bw, C, k), ix, k > 0);
                 }
-                if (id + 2 < c_end) {
-                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_wq[bb]), pb);
-                    if (ok) fetch_wq(id + 2);
-                }
-                if (ok && id + 1 < c_end) {
-                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_u), ph);
-                    if (ok) fetch_u(id + 1);
-                }
-                if (ok && id + 2 < c_end) {
-                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_kt[bb]), pb);
-                    if (ok) fetch_kt(id + 2);
-                }
-                if (ok && id + 1 < c_end) {
-                    ok = tc::mbar_wait(tc::smem_u32(&sm.free_aq), ph);
-                    if (ok) fetch_aq(id + 1);
-                }
-            }
-        }
-    } else
-    for (int id = c_begin; id < c_end; ++id) {
-        const uint32_t ph = (uint32_t)(id - c_begin) & 1u;
-        const uint32_t tXO = tm + ph * 128;
-        // loads one chunk ahead: the next chunk's gamma_n; two ahead: its table entry
-        float gl_nx = 0.f;
-        int4 ch_nx2 = ch_nx;
-        if (id + 1 < c_end) gl_nx = p.gam[((size_t)(id + 1) * HV + h) * C + ch_nx.z - 1];
-        if (id + 2 < c_end) ch_nx2 = p.chunk_tab[id + 2];
-        bool okl = true;
-        const int bb = (id - c_begin) & 1;
-        const uint32_t pb = (uint32_t)((id - c_begin) >> 1) & 1u;
-        if (tid == ISSUER) {
-            okl = tc::mbar_wait(bar_wq(bb), pb);
-            if (okl) {  // [X^T | O^T] = S^T [W ; Qg]^T, S^T from tensor memory
-                const uint32_t b = tc::smem_u32(sm.wq[bb]);
-                constexpr uint32_t idesc = tc::idesc_f16(DV, 128);
+                if (!ok) break;
+                tc::mma_commit(bar(sm.bar_x));
+                tc::mma_commit(bar(sm.free_w[bb]));
+                // Oi^T = S^T Q^T (Q: rows C .. 2C-1 of the [K ; Q] tile)
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k)
-                    tc::mma_f16_ta(tXO, tA + 8 * k, tc::desc_kmajor(b, 2 * C, k), idesc, k > 0);
-                tc::mma_commit(bar_x);
-                tc::mma_commit(tc::smem_u32(&sm.free_wq[bb]));
+                    tc::mma_f16_ta(tOi(bb), tA + 8 * k, tc::desc_sw128_k(bkq + C * 128, 2 * C, k), ix, k > 0);
+                // Snew^T = Vs'^T K (K read MN-major), each half of the rows as soon as it is formed
+                const uint32_t bvs = tc::smem_u32(sm.vs), bvt = tc::smem_u32(sm.vt);
+                constexpr uint32_t is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    ok = tc::mbar_wait(bar(sm.bar_vp[hh]), ph);
+                    tc::fence_after_sync();
+                    if (!ok) break;
+#pragma unroll
+                    for (int k = 2 * hh; k < 2 * hh + 2; ++k)
+                        tc::mma_f16(tSn, tc::desc_sw128_k(bvs, DV, k), tc::desc_sw128_mn(bkq, 2 * C, k), is, k > 0);
+                }
+                if (!ok) break;
+                tc::mma_commit(bar(sm.bar_s));
+                tc::mma_commit(bar(sm.free_kq[bb]));
+                // Oq^T = V'^T Aqk^T: queued behind the state product, off the chain
+                ok = tc::mbar_wait(bar(sm.full_aq[bb]), pb);
+                if (!ok) break;
+                constexpr uint32_t io = tc::idesc_f16(DV, 64);
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    tc::mma_f16(tOq(bb), tc::desc_sw128_k(bvt, DV, k), tc::desc_sw128_k(tc::smem_u32(sm.aq[bb]), C, k),
+                                io, k > 0);
+                tc::mma_commit(bar(sm.bar_o));
+                tc::mma_commit(bar(sm.free_aq[bb]));
             }
-        } else if (warp < NCW) {
+        }
+    } else {
+        // ---- the compute warps.  Every wait is bounded; a failed one skips the work that needed it,
+        // and the compute warps agree on the outcome at one barrier per chunk, so they stop together.
+        int prev_t0 = 0, prev_n = 0;
+        int4 chn = p.chunk_tab[c_begin];
+        for (int id = c_begin; id < c_end; ++id) {
+            const int it = id - c_begin, bb = it & 1;
+            const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
+            const int4 ch = chn;
+            if (id + 1 < c_end) chn = p.chunk_tab[id + 1];
             if (id == ck_chunk && rowv)  // the state entering the checkpoint's chunk: column j of S
 #pragma unroll
                 for (int i = 0; i < DK / 2; ++i) ck_dst[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
-            if (id > c_begin) {  // the previous chunk's outputs leave while this chunk's first product runs
-                okl = __all_sync(0xffffffffu, tc::mbar_wait(bar_o, ph ^ 1u));
-                if (okl) {
-                    tc::fence_after_sync();
-                    put_out(tm + (ph ^ 1u) * 128, prev_t0, prev_n);
-                }
-            }
-            okl = __all_sync(0xffffffffu, okl && tc::mbar_wait(bar_x, ph) && tc::mbar_wait(bar_u, ph));
-            tc::fence_after_sync();
-            if (okl) {  // V'^T row j = U^T row j - X^T row j
+            // V'^T row j = U^T row j - X^T row j over this warp's half of the chunk's rows, and
+            // Vs'^T = V'^T diag(f)
+            bool okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_x), ph) && tc::mbar_wait(bar(sm.full_u[bb]), pb));
+            float egn = 0.f;
+            if (okl) {
+                tc::fence_after_sync();
+                char* vtb = reinterpret_cast<char*>(sm.vt);
+                char* vsb = reinterpret_cast<char*>(sm.vs);
+                const char* utb = reinterpret_cast<const char*>(sm.ut[bb]);
 #pragma unroll
                 for (int cc = 0; cc < C / 2; cc += 16) {
                     const int c0 = half * (C / 2) + cc;
-                    float x[16];
-                    tc::tmem_ld16(tXO + lane_base + c0, x);
+                    float xv[16];
+                    tc::tmem_ld16(tX + lane_base + c0, xv);
                     tc::tmem_ld_wait();
                     if (rowv)
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {  // 8 fp16 values per 16-byte vector
-                            const uint32_t off = tc::kmajor_off16(j, c0 + 8 * q, DV);
-                            uint4* pv = reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.vt) + off);
-                            const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(sm.ut) + off);
-                            const float2 u0 = tc::unpack_f16(u.x), u1 = tc::unpack_f16(u.y), u2 = tc::unpack_f16(u.z),
-                                         u3 = tc::unpack_f16(u.w);
-                            const float* xq = x + 8 * q;
-                            *pv = make_uint4(tc::pack_f16(u0.x - xq[0], u0.y - xq[1]), tc::pack_f16(u1.x - xq[2], u1.y - xq[3]),
-                                             tc::pack_f16(u2.x - xq[4], u2.y - xq[5]), tc::pack_f16(u3.x - xq[6], u3.y - xq[7]));
+                            const uint32_t off = tc::sw128_off(j, c0 + 8 * q, DV);
+                            const uint4 u = *reinterpret_cast<const uint4*>(utb + off);
+                            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                            uint32_t vw[4], sw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 uu = tc::unpack_f16(uw[e]);
+                                const int cl = c0 + 8 * q + 2 * e;
+                                const float v0 = uu.x - xv[8 * q + 2 * e], v1 = uu.y - xv[8 * q + 2 * e + 1];
+                                vw[e] = tc::pack_f16(v0, v1);
+                                sw[e] = tc::pack_f16(v0 * sm.gv[bb][cl].y, v1 * sm.gv[bb][cl + 1].y);
+                            }
+                            *reinterpret_cast<uint4*>(vtb + off) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+                            *reinterpret_cast<uint4*>(vsb + off) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
                         }
                 }
+                if (warp == 0 || warp == 4)  // the output scale of this chunk, for its outputs one chunk later
+                    sm.eg[bb][half * 32 + lane] = sm.gv[bb][half * 32 + lane].x;
+                egn = sm.gv[bb][0].w;  // e^{gamma_n}
+                tc::fence_smem_to_async();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(bar(sm.bar_vp[half]));
+                    tc::mbar_arrive(bar(sm.free_u[bb]));
+                }
             }
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(tc::smem_u32(&sm.free_u));  // this warp has read its U^T rows
-        }
-        tc::fence_smem_to_async();
-        tc::fence_before_sync();
-        ok = bar_and(kChainBarrier, NCHAIN, okl);
-        if (!ok) break;
-        tc::fence_after_sync();
-        if (tid == ISSUER) {
-            okl = tc::mbar_wait(bar_kt(bb), pb);
-            if (okl) {  // Snew^T = V'^T K~, K~ (rows s) read MN-major
-                const uint32_t av = tc::smem_u32(sm.vt), bk = tc::smem_u32(sm.kt[bb]);
-                constexpr uint32_t is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
-#pragma unroll
-                for (int k = 0; k < C / 16; ++k)
-                    tc::mma_f16(tS, tc::desc_kmajor(av, DV, k), tc::desc_mnmajor16(bk, C, k), is, k > 0);
-                tc::mma_commit(bar_s);
-                tc::mma_commit(tc::smem_u32(&sm.free_kt[bb]));
-            }
-            if (okl) okl = tc::mbar_wait(bar_aq, ph);
-            if (okl) {  // O^T += V'^T Aqk^T: queued behind the state product, off the state chain; the
-                        // next chunk's first product waits for it (the tensor core runs them in order)
-                const uint32_t av = tc::smem_u32(sm.vt), bq = tc::smem_u32(sm.aq);
-                constexpr uint32_t io = tc::idesc_f16(DV, 64);
-#pragma unroll
-                for (int k = 0; k < C / 16; ++k)
-                    tc::mma_f16(tXO + 64, tc::desc_kmajor(av, DV, k), tc::desc_kmajor(bq, C, k), io, true);
-                tc::mma_commit(bar_o);
-                tc::mma_commit(tc::smem_u32(&sm.free_aq));
-            }
-        } else if (warp < NCW) {
-            if (id > c_begin) send_out(prev_t0, prev_n);  // staged before the middle barrier; the
-                                                          // state product runs meanwhile
-            okl = __all_sync(0xffffffffu, tc::mbar_wait(bar_s, ph));
-            if (okl) {  // S^T <- e^{gamma_n} S^T + Snew^T, and its fp16 copy for the next chunk
+            // the previous chunk's outputs, while the state product runs (their products completed before
+            // this chunk's X did: a commit covers every earlier product of the issuing thread)
+            if (okl && it > 0) {
                 tc::fence_after_sync();
-                const float egl = expf(gl);
+                put_out(it - 1, prev_t0, prev_n);
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(sm.free_aq[bb ^ 1]));
+            }
+            // S^T <- e^{gamma_n} S^T + Snew^T, and its fp16 copy for the next chunk, half by half
+            if (okl) okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_s), ph));
+            if (okl) {
+                tc::fence_after_sync();
 #pragma unroll
                 for (int cc = 0; cc < DK / 2; cc += 32) {
                     const int c0 = half * (DK / 2) + cc;
                     float v[32];
-                    tc::tmem_ld16(tS + lane_base + c0, *reinterpret_cast<float(*)[16]>(v));
-                    tc::tmem_ld16(tS + lane_base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+                    tc::tmem_ld16(tSn + lane_base + c0, *reinterpret_cast<float(*)[16]>(v));
+                    tc::tmem_ld16(tSn + lane_base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[cc + i] = fmaf(egl, s[cc + i], v[i]);
+                    for (int i = 0; i < 32; ++i) s[cc + i] = fmaf(egn, s[cc + i], v[i]);
                     put_sa32(tA_row + cc / 2, &s[cc]);
                 }
                 tc::tmem_st_wait();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
             }
+            ok = cw_and(okl);  // also orders the output scale and the staged outputs between the warps
+            if (!ok) break;
+            if (it > 0) send_out(it - 1, prev_t0, prev_n);  // the previous chunk's staged outputs leave
+            prev_t0 = ch.y;
+            prev_n = ch.z;
         }
-        tc::fence_before_sync();
-        ok = bar_and(kChainBarrier, NCHAIN, okl);
-        if (!ok) break;
-        tc::fence_after_sync();
-        prev_t0 = ch.y;
-        prev_n = ch.z;
-        ch = ch_nx;
-        ch_nx = ch_nx2;
-        gl = gl_nx;
-    }
-    ok = __syncthreads_and(ok);  // the chain, the copier and the idle lanes agree
-    if (ok) {
-        if (warp < NCW) {
-            const uint32_t ph = (uint32_t)(c_end - 1 - c_begin) & 1u;
-            const bool okw = __all_sync(0xffffffffu, tc::mbar_wait(bar_o, ph));
-            if (okw) {  // the last chunk's outputs
+        if (ok) {  // the last chunk's outputs and the final state
+            const int it = c_end - 1 - c_begin;
+            bool okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_o), (uint32_t)it & 1u));
+            if (okl) {
                 tc::fence_after_sync();
-                put_out(tm + ph * 128, prev_t0, prev_n);
-            } else if (lane == 0) {
-                raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+                put_out(it, prev_t0, prev_n);
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(sm.free_aq[it & 1]));
             }
-            if (rowv)  // final state: column j of S
+            ok = cw_and(okl);
+            if (ok) send_out(it, prev_t0, prev_n);
+            if (ok && rowv)  // final state: column j of S
 #pragma unroll
                 for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
         }
-        if (tid == ISSUER) {  // the releases nobody waited for, so that none lands after the CTA is gone
-            const int n = c_end - c_begin;
-            for (int it = max(0, n - 2); it < n; ++it) {
-                tc::mbar_wait(tc::smem_u32(&sm.free_wq[it & 1]), (uint32_t)(it >> 1) & 1u);
-                tc::mbar_wait(tc::smem_u32(&sm.free_kt[it & 1]), (uint32_t)(it >> 1) & 1u);
-            }
-            tc::mbar_wait(tc::smem_u32(&sm.free_aq), (uint32_t)(n - 1) & 1u);
-        }
-        if constexpr (kStageOut<T>) {
-            __syncthreads();
-            if (warp < NCW) send_out(prev_t0, prev_n);
-        }
-    } else if (tid == ISSUER) {
+    }
+    ok = __syncthreads_and(ok);  // the chain, the issuer, the copier and the idle lanes agree
+    if (!ok && tid == ISSUER) {
         raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
-        // (the copier has stopped issuing: its loop ends at its first failed wait, and every
-        // wait of the chain threads above has returned)
         // let copies and products already in flight finish before the CTA's shared and tensor
         // memory go away
         for (uint32_t par = 0; par < 2; ++par) {
-            for (int b = 0; b < 2; ++b) {
-                tc::mbar_wait(bar_wq(b), par, 100000000ull);
-                tc::mbar_wait(bar_kt(b), par, 100000000ull);
+            for (int bb = 0; bb < 2; ++bb) {
+                tc::mbar_wait(bar(sm.full_kq[bb]), par, 100000000ull);
+                tc::mbar_wait(bar(sm.full_w[bb]), par, 100000000ull);
+                tc::mbar_wait(bar(sm.full_u[bb]), par, 100000000ull);
+                tc::mbar_wait(bar(sm.full_aq[bb]), par, 100000000ull);
             }
-            tc::mbar_wait(bar_aq, par, 100000000ull);
-            tc::mbar_wait(bar_o, par, 100000000ull);
-            tc::mbar_wait(bar_u, par, 100000000ull);
-            for (int b = 0; b < 2; ++b) {
-                tc::mbar_wait(tc::smem_u32(&sm.free_wq[b]), par, 100000000ull);
-                tc::mbar_wait(tc::smem_u32(&sm.free_kt[b]), par, 100000000ull);
-            }
-            tc::mbar_wait(tc::smem_u32(&sm.free_aq), par, 100000000ull);
+            tc::mbar_wait(bar(sm.bar_o), par, 100000000ull);
+        }
+    }
+    if (ok && tid == ISSUER) {  // the releases nobody waited for, so that none lands after the CTA is gone
+        const int n = c_end - c_begin;
+        for (int it = max(0, n - 2); it < n; ++it) {
+            tc::mbar_wait(bar(sm.free_w[it & 1]), (uint32_t)(it >> 1) & 1u);
+            tc::mbar_wait(bar(sm.free_kq[it & 1]), (uint32_t)(it >> 1) & 1u);
+            tc::mbar_wait(bar(sm.free_aq[it & 1]), (uint32_t)(it >> 1) & 1u);
         }
     }
     tc::fence_before_sync();
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 
 template <typename T, int DK, int DV>
 cudaError_t launch_state(const ExtendArgs& p, int seg, cudaStream_t s) {
-    const size_t shm = sizeof(StateTcSmem<T, DK, DV>);
+    constexpr size_t shm = state_smem_bytes<T, DK, DV>();
     cudaError_t e =
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;

@@ -62,6 +62,42 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint
     return d;                // base offset 0, legacy LBO mode, layout type 0 (no swizzle)
 }
 
+// ---- 128-byte swizzled tiles ------------------------------------------------
+// A 16-bit tile with R rows (R a multiple of 8) and a column count that is a multiple of 64 is
+// held as column blocks of 64 elements: block b is R rows of 128 bytes at b * R * 128, and inside
+// an 8-row group the 16-byte chunk c of row r sits at chunk position c ^ (r % 8).  The tile must
+// start on a 1024-byte boundary (the tensor core forms the XOR from address bits 7-9).  Writers
+// that put 8 consecutive rows of one chunk, or one row's consecutive chunks, into a warp's lanes
+// spread them over all 32 banks, so such stores run without bank conflicts.
+//
+// Read as a K-major operand (rows along M or N, columns along K): SBO = 1024 (next 8 rows), the
+// 32-byte k-step s of a 64-wide block starts 32 s bytes into it.  Read as an MN-major operand
+// (rows along K, columns along M or N): LBO = R * 128 (next 64 columns), SBO = 1024 (next 8 rows
+// along K), a 16-deep k-step spans 2048 bytes.
+__device__ __forceinline__ uint32_t sw128_off(int r, int k, int R) {
+    return (uint32_t)((k >> 6) * (R * 128) + r * 128 + ((((k >> 3) & 7) ^ (r & 7)) << 4) + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint64_t make_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
+    d |= (uint64_t)2 << 61;  // layout type: 128-byte swizzle
+    return d;
+}
+
+// K-major k-step `s` (16 fp16 along K) of a swizzled tile with R rows
+__device__ __forceinline__ uint64_t desc_sw128_k(uint32_t base, int R, int s) {
+    return make_desc_sw128(base + (uint32_t)(s >> 2) * (uint32_t)(R * 128) + (uint32_t)(s & 3) * 32, 16, 1024);
+}
+
+// MN-major k-step `s` (16 rows along K) of a swizzled tile with R rows
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t base, int R, int s) {
+    return make_desc_sw128(base + (uint32_t)s * 2048, (uint32_t)(R * 128), 1024);
+}
+
 // descriptor of MMA k-step `s` (8 tf32 or 16 fp16 along K: 32 bytes) of a K-major tile with R rows
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int R, int s) {
     const uint32_t lbo = (uint32_t)(R >> 3) * 128;

@@ -1,17 +1,21 @@
 #!/usr/bin/env python
 """Benchmark of the GDN layer on B200: one step = one gdn_extend over the
-packed prefill batch + one gdn_decode over the decode batch + one gdn_verify
-over the verify batch + one gdn_commit of each verify request's accepted
-prefix (every mode of the layer), on synthetic inputs already resident in HBM.
+prefill workload + one gdn_decode over the decode batch + one gdn_verify over
+the verify batch + one gdn_commit of each verify request's accepted prefix
+(every mode of the layer), on synthetic inputs already resident in HBM.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill32k|prefill262k]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill262k|prefill32k]
     python bench.py --impl reference ...      # the fp64 CPU oracle on a bounded sample
 
-Prints one JSON line (rank 0).  `value` is prefill tokens/s over all ranks,
-from the device time of the gdn_extend launches inside the timed steps;
-decode, verify and commit report their own state-traffic figures.  Multi-GPU runs are
-independent replicas (weak scaling): every rank runs its own batch, no
-collective touches the data path; the timing is the max over ranks.
+The default prefill workload is the long-context one (one sequence of 262144
+tokens continuing from a random state, 16/32 heads, d = 128): the largest
+configuration that fits one GPU.  The 32768-token packed batch (8 sequences)
+is timed beside it.  Prints one JSON line (rank 0).  `value` is prefill
+tokens/s over all ranks, from the device time of the gdn_extend launches
+inside the timed steps; decode, verify and commit report their own
+state-traffic figures.  Multi-GPU runs are independent replicas (weak
+scaling): every rank runs its own batch, no collective touches the data path;
+the timing is the max over ranks.
 """
 from __future__ import annotations
 
@@ -49,15 +53,18 @@ def parse():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=["prefill32k", "prefill262k"], default="prefill32k")
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--workload", choices=["prefill262k", "prefill32k"], default="prefill262k")
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--e2e-piece", type=int, default=16384, help="rows per call of the end-to-end pipeline")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-ssd", action="store_true", help="skip the Mamba2 SSD scan timing")
+    p.add_argument("--no-side", action="store_true", help="skip the prefill timings outside the step")
     p.add_argument("--cpu-sample-tokens", type=int, default=16384)
     p.add_argument("--ref-sample-tokens", type=int, default=4096)
     p.add_argument("--profile", choices=["extend", "decode", "verify", "ssd"], default=None,
                    help="run only this call on a reduced case (an ncu target); prints timings, not the bench line")
     p.add_argument("--profile-tokens", type=int, default=8192, help="prefill rows of the --profile extend case")
+    p.add_argument("--profile-seqs", type=int, default=4, help="sequences of the --profile extend case")
     p.add_argument("--profile-requests", type=int, default=64, help="requests of the --profile decode/verify case")
     return p.parse_args()
 
@@ -323,6 +330,54 @@ def workload_config(pre, args):
             "l2": "inputs larger than L2 (prefill input 512 MiB+, decode state 1 GiB touched per step)"}
 
 
+# gdn_extend's profiling marks (gdn_set_launch_events): 0 start, 1 chunk table, 2 after the last
+# per-chunk segment, 3 conv-state update, 5 end; on the library's second stream 6 / 7 bracket the
+# state-pass segments, which run alongside the per-chunk segments after the first
+EXT_EV = 8
+EXT_K = ["chunk_map", "chunk", "conv_tail", "state"]
+
+
+def extend_kernel_ms(ev):
+    sp = lambda i, j: ev[i].elapsed_time(ev[j])
+    return {"chunk_map": sp(0, 1), "chunk": sp(1, 2), "conv_tail": sp(2, 3), "state": sp(6, 7), "extend": sp(0, 5)}
+
+
+def prefill_kernel_roofline(spec, T, chunks, kms, hbm, f16):
+    """Per-kernel rooflines of one extend: the per-chunk step against the larger of its input read
+    (the bf16 rows and gates: the algorithmic bytes it must move) at the HBM peak and the intra-chunk
+    FLOPs at the tensor peak; the state pass against its FLOPs (the chain products and outputs)
+    at the tensor peak."""
+    pw = prefill_work(spec, T)
+    es = 2 if spec.dtype == torch.bfloat16 else 4
+    in_bytes = T * (spec.conv_dim + 2 * spec.HV) * es
+    out = {}
+    t_in, t_fi = in_bytes / (hbm * 1e9), pw["flops_intra"] / (f16 * 1e12)
+    if t_in >= t_fi:
+        out["chunk"] = {"bound": "hbm", "work": in_bytes, "unit": "GB/s", "peak": hbm}
+    else:
+        out["chunk"] = {"bound": "tensor", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": f16}
+    out["state"] = {"bound": "tensor", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": f16}
+    for name, k in out.items():
+        t = kms[name] * 1e-3
+        scale = 1e12 if k["unit"] == "TFLOP/s" else 1e9
+        k["ms"] = kms[name]
+        k["achieved"] = k["work"] / t / scale
+        k["frac"] = k["achieved"] / k["peak"]
+    return out, pw
+
+
+def prefill_summary(spec, T, chunks, ms, kms, hbm, f16, world):
+    pw = prefill_work(spec, T)
+    t_floor = max(pw["flops"] / (f16 * 1e12), pw["bytes"] / (hbm * 1e9))
+    return {"ms": ms, "tokens_per_s": world * T / (ms * 1e-3), "chunks": chunks,
+            "tflops": pw["flops"] / (ms * 1e-3) / 1e12, "gbs_algorithmic": pw["bytes"] / (ms * 1e-3) / 1e9,
+            "roofline": {"floor_ms": t_floor * 1e3,
+                         "bound": "tensor" if pw["flops"] / (f16 * 1e12) >= pw["bytes"] / (hbm * 1e9) else "hbm",
+                         "frac": t_floor / (ms * 1e-3), "tensor_frac": pw["flops"] / (ms * 1e-3) / (f16 * 1e12),
+                         "hbm_frac": pw["bytes"] / (ms * 1e-3) / (hbm * 1e9)},
+            "kernel_ms": {k: kms[k] for k in EXT_K}}
+
+
 # ------------------------------------------------------------------ our arm
 
 
@@ -365,7 +420,7 @@ def run_profile_case(args, dev):
         call, ws = ssd_call(w, gdn, dev)
         w.cu_seqlens, w.N = w.cu, len(w.lengths)
     elif args.profile == "extend":
-        w = W.large_prefill(device=dev, total=args.profile_tokens, nseq=4)
+        w = W.large_prefill(device=dev, total=args.profile_tokens, nseq=args.profile_seqs)
         cfg = gdn.GdnConfig.from_spec(w.spec)
         ws = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, w.N, w.T), dev)
         out = torch.empty(w.T, w.spec.HV, w.spec.dv, dtype=w.spec.dtype, device=dev)
@@ -400,8 +455,19 @@ def run_profile_case(args, dev):
     assert gdn.gdn_get_device_error(ws) == 0
     cu = w.cu_seqlens.cpu().tolist() if args.profile in ("extend", "ssd") else list(range(w.N + 1))
     chunks = sum((cu[i + 1] - cu[i] + C - 1) // C for i in range(len(cu) - 1))
-    print(json.dumps({"profile": args.profile, "workload": w.name, "chunks": chunks,
-                      "ms_per_call": s0.elapsed_time(s1) / args.steps}))
+    rec = {"profile": args.profile, "workload": w.name, "chunks": chunks,
+           "ms_per_call": s0.elapsed_time(s1) / args.steps}
+    if args.profile == "extend":  # kernel spans of one more call (one segment below 16384 rows: the
+        # state pass then starts after the per-chunk step, so its span is the serial chain alone)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(EXT_EV)]
+        gdn.gdn_set_launch_events(ev)
+        call()
+        gdn.gdn_set_launch_events([])
+        torch.cuda.synchronize()
+        rec["kernel_ms"] = extend_kernel_ms(ev)
+        longest = max((cu[i + 1] - cu[i] + C - 1) // C for i in range(len(cu) - 1))
+        rec["state_us_per_chunk_of_longest"] = rec["kernel_ms"]["state"] * 1e3 / longest
+    print(json.dumps(rec))
 
 
 def main():
@@ -431,6 +497,8 @@ def main():
     D = dv.extra["D"]
     xv, av, bv = dv.extra["verify"]
     Bn = dv.N
+    cu_list = pre.cu_seqlens.cpu().tolist()
+    chunks = sum((cu_list[i + 1] - cu_list[i] + C - 1) // C for i in range(pre.N))
 
     ws_pre = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, pre.N, pre.T), dev)
     out_pre = torch.empty(pre.T, spec.HV, spec.dv, dtype=spec.dtype, device=dev)
@@ -459,11 +527,6 @@ def main():
     def commit():
         gdn.gdn_commit(dcfg, dv.state_indices, acc, D, ck, cck, dv.conv_state, dv.ssm_state, ws_c)
 
-    EXT_K = ["chunk_map", "prep", "conv_tail", "intra", "state"]
-    # gdn_extend's profiling marks: 0 start, 1 chunk table, 2 prep, 3 conv tail, 4 after the last intra
-    # segment, 5 end; on the library's second stream 6 / 7 bracket the state-pass segments, which run
-    # alongside the intra segments after the first
-    EXT_EV = 8
     n_ev = EXT_EV + 2 + 2 + 2
 
     def make_events():
@@ -506,59 +569,83 @@ def main():
     total_ms = max_over_ranks(start.elapsed_time(end), world, dev)
     ms_step = total_ms / args.steps
 
-    def span(k, i, j):
-        return evs[k][i].elapsed_time(evs[k][j])
+    def mean_span(i, j):
+        return statistics.mean(evs[k][i].elapsed_time(evs[k][j]) for k in range(args.steps))
 
-    def mean_span(*pairs):  # summed over the pairs, averaged over the steps
-        return statistics.mean(sum(span(k, i, j) for i, j in pairs) for k in range(args.steps))
-
-    # per-kernel device times: the spans of the intra segments (on the caller's stream) and of the
-    # state-pass segments (on the second stream) overlap
-    kern_ms = {"chunk_map": mean_span((0, 1)), "prep": mean_span((1, 2)), "conv_tail": mean_span((2, 3)),
-               "intra": mean_span((3, 4)), "state": mean_span((6, 7))}
-    kern_ms["decode"] = mean_span((EXT_EV, EXT_EV + 1))
-    kern_ms["verify"] = mean_span((EXT_EV + 2, EXT_EV + 3))
-    kern_ms["commit"] = mean_span((EXT_EV + 4, EXT_EV + 5))
-    ext_ms = max_over_ranks(mean_span((0, 5)), world, dev)
+    ek = [extend_kernel_ms(evs[k][:EXT_EV]) for k in range(args.steps)]
+    kern_ms = {name: statistics.mean(e[name] for e in ek) for name in EXT_K}
+    kern_ms["decode"] = mean_span(EXT_EV, EXT_EV + 1)
+    kern_ms["verify"] = mean_span(EXT_EV + 2, EXT_EV + 3)
+    kern_ms["commit"] = mean_span(EXT_EV + 4, EXT_EV + 5)
+    ext_ms = max_over_ranks(statistics.mean(e["extend"] for e in ek), world, dev)
     dec_ms = max_over_ranks(kern_ms["decode"], world, dev)
     ver_ms = max_over_ranks(kern_ms["verify"], world, dev)
     com_ms = max_over_ranks(kern_ms["commit"], world, dev)
 
     hbm, bf16, bf16_sus, peak_src = peaks()
-    pw = prefill_work(spec, pre.T)
+    f16 = bf16
+    f16_src = f"{peak_src} bf16 burst {bf16:.1f} TFLOP/s (fp16 and bf16 share the dense tensor rate)"
     st_dec, by_dec = decode_bytes(dspec, Bn)
     st_ver, by_ver = verify_bytes(dspec, Bn, D)
     st_com, by_com = commit_bytes(dspec, acc_h)
     value = world * pre.T / (ext_ms * 1e-3)
 
-    f16 = bf16
-    f16_src = f"{peak_src} bf16 burst {bf16:.1f} TFLOP/s (fp16 and bf16 share the dense tensor rate)"
-    kernels = {
-        "state": {"bound": "tensor", "work": pw["flops_state"], "unit": "TFLOP/s", "peak": f16, "peak_src": f16_src},
-        "intra": {"bound": "tensor", "work": pw["flops_intra"], "unit": "TFLOP/s", "peak": f16, "peak_src": f16_src},
-        "prep": {"bound": "hbm", "work": pre.T * (spec.conv_dim * 2 + 2 * spec.HV * 2), "unit": "GB/s",
-                 "peak": hbm, "peak_src": peak_src},
-        "decode": {"bound": "hbm", "work": by_dec, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
-        "verify": {"bound": "hbm", "work": by_ver, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
-        "commit": {"bound": "hbm", "work": by_com, "unit": "GB/s", "peak": hbm, "peak_src": peak_src},
-    }
-    for name, k in kernels.items():
-        t = kern_ms[name] * 1e-3
-        scale = 1e12 if k["unit"] == "TFLOP/s" else 1e9
+    kernels, pw = prefill_kernel_roofline(spec, pre.T, chunks, kern_ms, hbm, f16)
+    kernels["decode"] = {"bound": "hbm", "work": by_dec, "unit": "GB/s", "peak": hbm}
+    kernels["verify"] = {"bound": "hbm", "work": by_ver, "unit": "GB/s", "peak": hbm}
+    kernels["commit"] = {"bound": "hbm", "work": by_com, "unit": "GB/s", "peak": hbm}
+    for name in ("decode", "verify", "commit"):
+        k = kernels[name]
         k["ms"] = kern_ms[name]
-        k["achieved"] = k["work"] / t / scale
+        k["achieved"] = k["work"] / (kern_ms[name] * 1e-3) / 1e9
         k["frac"] = k["achieved"] / k["peak"]
-    dom = max(kern_ms, key=lambda n: kern_ms[n] if n in kernels else -1)
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
     dk = kernels[dom]
     roofline = {"kernel": dom, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
-                "unit": dk["unit"], "frac": dk["frac"], "traffic": ncu_traffic(dom),
-                "peak_source": dk["peak_src"] + (" (of measured)" if peak_src == "measured" else " (of fallback)")}
-    # the whole prefill against its own roofline: max(algorithmic FLOPs at the fp16 tensor peak,
-    # algorithmic bytes at the HBM peak)
-    t_floor = max(pw["flops"] / (f16 * 1e12), pw["bytes"] / (hbm * 1e9))
-    prefill_roofline = {"floor_ms": t_floor * 1e3, "bound": "tensor" if pw["flops"] / (f16 * 1e12) >= pw["bytes"] / (hbm * 1e9) else "hbm",
-                        "frac": t_floor / (ext_ms * 1e-3), "tensor_frac": pw["flops"] / (ext_ms * 1e-3) / (f16 * 1e12),
-                        "hbm_frac": pw["bytes"] / (ext_ms * 1e-3) / (hbm * 1e9)}
+                "unit": dk["unit"], "frac": dk["frac"], "traffic": ncu_traffic(f"{dom}@{pre.name}"),
+                "peak_source": (f16_src if dk["unit"] == "TFLOP/s" else f"{peak_src} copy {hbm:.1f} GB/s")
+                + (" (of measured)" if peak_src == "measured" else " (of fallback)")}
+    prefill = prefill_summary(spec, pre.T, chunks, ext_ms, kern_ms, hbm, f16, world)
+    prefill["state_chain_us_per_chunk"] = kern_ms["state"] * 1e3 / max(1, max(
+        (cu_list[i + 1] - cu_list[i] + C - 1) // C for i in range(pre.N)))
+    prefill["kernel_roofline"] = {k: {kk: kernels[k][kk] for kk in ("bound", "ms", "achieved", "peak", "unit", "frac")}
+                                  for k in ("chunk", "state")}
+
+    # The other prefill workload (the 8-sequence packed batch, or the long one when it is the headline's
+    # alternative), outside the timed step: its own inputs, workspace and pools
+    other = None
+    if not args.no_side:
+        alt = W.large_prefill(device=dev, seed=2 + seed_off) if args.workload == "prefill262k" else \
+            W.long_prefill(device=dev, seed=4 + seed_off)
+        acu = alt.cu_seqlens.cpu().tolist()
+        achunks = sum((acu[i + 1] - acu[i] + C - 1) // C for i in range(alt.N))
+        acfg = gdn.GdnConfig.from_spec(alt.spec)
+        aws = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(acfg, alt.N, alt.T), dev)
+        aout = torch.empty(alt.T, alt.spec.HV, alt.spec.dv, dtype=alt.spec.dtype, device=dev)
+
+        def alt_extend():
+            gdn.gdn_extend(acfg, alt.params, alt.x, alt.a, alt.b, alt.cu_seqlens, alt.state_indices,
+                           alt.has_initial_state, alt.conv_state, alt.ssm_state, aout, aws)
+
+        for _ in range(3):
+            alt_extend()
+        aev = [make_events()[:EXT_EV] for _ in range(5)]
+        for ev in aev:
+            gdn.gdn_set_launch_events(ev)
+            alt_extend()
+        gdn.gdn_set_launch_events([])
+        torch.cuda.synchronize()
+        assert gdn.gdn_get_device_error(aws) == 0
+        aek = [extend_kernel_ms(ev) for ev in aev]
+        akms = {name: statistics.mean(e[name] for e in aek) for name in EXT_K}
+        a_ms = max_over_ranks(statistics.mean(e["extend"] for e in aek), world, dev)
+        other = prefill_summary(alt.spec, alt.T, achunks, a_ms, akms, hbm, f16, world)
+        other["workload"] = alt.name
+        akern, _ = prefill_kernel_roofline(alt.spec, alt.T, achunks, akms, hbm, f16)
+        other["kernel_roofline"] = {k: {kk: akern[k][kk] for kk in ("bound", "ms", "achieved", "peak", "unit", "frac")}
+                                    for k in akern}
+        other["note"] = "timed outside the step: 5 calls after 3 warm-up calls, CUDA events"
+        del aws, aout, alt
 
     # Prefill state checkpoints (prefix caching), outside the timed step: the same batch with one
     # checkpoint per sequence at a boundary three fifths into it (mid chunk in general)
@@ -575,7 +662,7 @@ def main():
 
     for _ in range(2):
         extend_ck()
-    ck_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+    ck_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
     for e0, e1 in ck_ev:
         e0.record()
         extend_ck()
@@ -603,9 +690,9 @@ def main():
     torch.cuda.synchronize()
     assert gdn.gdn_get_device_error(ws_v) == 0
     tr_ms = max_over_ranks(statistics.mean(e0.elapsed_time(e1) for e0, e1 in tr_ev), world, dev)
-    # the tree's algorithmic bytes: verify's, plus one parent checkpoint read per branching token
-    n_branch = sum(1 for t in range(D) if int(tree[t]) != t - 1)
-    by_tree = by_ver + n_branch * dspec.HV * dspec.dk * dspec.dv * 4 * Bn
+    # the tree's algorithmic bytes are verify's: a parent checkpoint it reloads was written by the same
+    # thread moments before and is not counted as HBM traffic
+    by_tree = by_ver
 
     # Mamba2 SSD scan (the second workload), outside the timed step: its inputs (1.8 GB) exceed L2
     ssd = None
@@ -641,46 +728,48 @@ def main():
                                    "sample": f"fp64 oracle, first {on} packed rows of the batch, all {sw.spec.H} heads"}
         del ssd_run, ssd_ws
 
-    # End to end through the public API with pinned host buffers.  The layer is independent per
-    # sequence, so the step runs one gdn_extend call per sequence and overlaps the host -> device
-    # copy of sequence i + 1 and the device -> host copy of sequence i - 1 with the call for
-    # sequence i (two copy streams, events between them): the same bytes and the same work as one
-    # call over the whole batch, with PCIe traffic in both directions hidden behind each other.
+    # End to end through the public API with pinned host buffers.  The layer is causal per sequence,
+    # so the step cuts every sequence into pieces of --e2e-piece rows and calls gdn_extend once per
+    # piece, each piece continuing from the state and conv window the previous one left in the slot
+    # (prefix-then-extend equals the whole sequence); the host -> device copy of piece i + 1 and the
+    # device -> host copy of piece i - 1 overlap the call for piece i (two copy streams, events
+    # between them): the same bytes and the same work as one call over the whole batch.
     e2e = None
     if args.e2e_steps > 0:
         hx, ha, hb = (t.cpu().pin_memory() for t in (pre.x, pre.a, pre.b))
         dx, da, db = torch.empty_like(pre.x), torch.empty_like(pre.a), torch.empty_like(pre.b)
         hout = torch.empty(out_pre.shape, dtype=out_pre.dtype).pin_memory()
-        cu_h = pre.cu_seqlens.cpu()
-        groups = []  # per sequence: row range, rebased cu_seqlens, slot and flag (host, pinned) + device copies
+        hi_h = pre.has_initial_state.cpu()
+        pieces = []  # (row range, host metadata [cu, slot, flag] pinned, device copies)
         for i in range(pre.N):
             r0, r1 = int(cu_h[i]), int(cu_h[i + 1])
-            if r1 == r0:
-                continue
-            hm = [torch.tensor([0, r1 - r0], dtype=torch.int32).pin_memory(),
-                  pre.state_indices[i:i + 1].cpu().pin_memory(), pre.has_initial_state[i:i + 1].cpu().pin_memory()]
-            groups.append((r0, r1, hm, [torch.empty_like(t, device=dev) for t in hm]))
-        groups.sort(key=lambda g: g[0] - g[1])  # longest first: short sequences end the pipeline
+            for q0 in range(r0, r1, args.e2e_piece):
+                q1 = min(r1, q0 + args.e2e_piece)
+                flag = hi_h[i:i + 1].clone() if q0 == r0 else torch.ones(1, dtype=torch.int32)
+                hm = [torch.tensor([0, q1 - q0], dtype=torch.int32).pin_memory(),
+                      pre.state_indices[i:i + 1].cpu().pin_memory(), flag.pin_memory()]
+                pieces.append((q0, q1, hm, [torch.empty_like(t, device=dev) for t in hm]))
+        ws_e2e = gdn.alloc_workspace(gdn.gdn_extend_workspace_size(cfg, 1, args.e2e_piece), dev)
         h2d = sum(t.numel() * t.element_size() for t in (hx, ha, hb)) + \
-            sum(t.numel() * t.element_size() for g in groups for t in g[2])
+            sum(t.numel() * t.element_size() for g in pieces for t in g[2])
         d2h = hout.numel() * hout.element_size()
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-        ev_in = [torch.cuda.Event() for _ in groups]
-        ev_out = [torch.cuda.Event() for _ in groups]
+        ev_in = [torch.cuda.Event() for _ in pieces]
+        ev_out = [torch.cuda.Event() for _ in pieces]
 
         def e2e_step():
             cur = torch.cuda.current_stream()
             s_in.wait_stream(cur)
             s_out.wait_stream(cur)
             with torch.cuda.stream(s_in):
-                for k, (r0, r1, hm, dm) in enumerate(groups):
+                for k, (r0, r1, hm, dm) in enumerate(pieces):
                     for h, d_ in zip((hx[r0:r1], ha[r0:r1], hb[r0:r1], *hm), (dx[r0:r1], da[r0:r1], db[r0:r1], *dm)):
                         d_.copy_(h, non_blocking=True)
                     ev_in[k].record(s_in)
-            for k, (r0, r1, hm, dm) in enumerate(groups):
+            for k, (r0, r1, hm, dm) in enumerate(pieces):
                 cur.wait_event(ev_in[k])
                 gdn.gdn_extend(cfg, pre.params, dx[r0:r1], da[r0:r1], db[r0:r1], dm[0], dm[1], dm[2],
-                               pre.conv_state, pre.ssm_state, out_pre[r0:r1], ws_pre)
+                               pre.conv_state, pre.ssm_state, out_pre[r0:r1], ws_e2e)
                 ev_out[k].record(cur)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev_out[k])
@@ -689,6 +778,7 @@ def main():
 
         e2e_step()
         torch.cuda.synchronize()
+        assert gdn.gdn_get_device_error(ws_e2e) == 0
         barrier(world)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s0.record()
@@ -699,8 +789,10 @@ def main():
         e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps, world, dev)
         e2e = {"value": world * pre.T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms,
-               "what": "pinned host buffers; per sequence: host -> device copy of its inputs, gdn_extend, "
-                       "device -> host copy of its out, pipelined across sequences on two copy streams"}
+               "what": f"pinned host buffers; per piece of {args.e2e_piece} rows: host -> device copy of its "
+                       "inputs, gdn_extend continuing from the slot, device -> host copy of its out, "
+                       "pipelined across pieces on two copy streams"}
+        del hx, ha, hb, dx, da, db, hout, ws_e2e
 
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -709,9 +801,11 @@ def main():
         run()
         dt = time.perf_counter() - t0
         cpu_baseline = {"value": n / dt, "unit": "tokens/s", "cores": workers, "kind": "oracle",
-                        "sample": f"fp64 oracle, first {n} packed rows of the batch, all {spec.HV} value heads"}
+                        "sample": f"fp64 oracle, first {n} packed rows of the {pre.name} batch, "
+                                  f"all {spec.HV} value heads"}
 
     if rank == 0:
+        nseg = min(16, max(1, pre.T // 16384))
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -720,9 +814,12 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu_baseline,
             "e2e": e2e,
-            # extend: chunk table, prep, conv tail + intra and state per segment; decode; verify; commit
-            "gpu_launches": args.steps * (3 + 2 * min(16, max(1, pre.T // 16384)) + 3),
+            # extend: chunk table, the per-chunk step and the state pass per segment, conv-state update;
+            # decode; verify; commit
+            "gpu_launches": args.steps * (2 + 2 * nseg + 3),
             "clocks": clocks,
+            "prefill": prefill,
+            "prefill_other": other,
             "decode": {"ms": dec_ms, "requests_per_s": world * Bn / (dec_ms * 1e-3),
                        "state_gbs": world * st_dec / (dec_ms * 1e-3) / 1e9,
                        "total_gbs": world * by_dec / (dec_ms * 1e-3) / 1e9,
@@ -730,19 +827,17 @@ def main():
                        "frac_of_measured_hbm": by_dec / (dec_ms * 1e-3) / 1e9 / hbm},
             "verify": {"ms": ver_ms, "state_gbs": world * st_ver / (ver_ms * 1e-3) / 1e9,
                        "total_gbs": world * by_ver / (ver_ms * 1e-3) / 1e9,
+                       "frac_of_8tbs_state": st_ver / (ver_ms * 1e-3) / 8e12,
                        "frac_of_measured_hbm": by_ver / (ver_ms * 1e-3) / 1e9 / hbm},
             "commit": {"ms": com_ms, "accepted_requests": int((acc_h > 0).sum()),
                        "total_gbs": world * by_com / (com_ms * 1e-3) / 1e9,
                        "frac_of_measured_hbm": by_com / (com_ms * 1e-3) / 1e9 / hbm},
             "verify_tree": {"ms": tr_ms, "parents": tree.tolist(), "total_gbs": world * by_tree / (tr_ms * 1e-3) / 1e9,
                             "frac_of_measured_hbm": by_tree / (tr_ms * 1e-3) / 1e9 / hbm,
-                            "note": "timed outside the step"},
+                            "note": "timed outside the step; bytes counted as verify's (parent reloads not counted)"},
             "ssd": ssd,
             "prefill_checkpoints": {"ms": ck_ms, "checkpoints": pre.N, "vs_prefill": ck_ms / ext_ms,
                                     "note": "one state checkpoint per sequence, mid chunk; timed outside the step"},
-            "prefill": {"ms": ext_ms, "tflops": pw["flops"] / (ext_ms * 1e-3) / 1e12, "roofline": prefill_roofline,
-                        "gbs_algorithmic": pw["bytes"] / (ext_ms * 1e-3) / 1e9,
-                        "kernel_ms": {k: kern_ms[k] for k in EXT_K}},
             "kernels": {k: {kk: v[kk] for kk in ("bound", "ms", "achieved", "peak", "unit", "frac")}
                         for k, v in kernels.items()},
         }

@@ -8,8 +8,10 @@ workloads.  Calls fail loudly when libgdn.so has not been built.
 from .binding import (  # noqa: F401
     GDN_DEVERR_ACCEPT_RANGE,
     GDN_DEVERR_CKPT_RANGE,
+    GDN_DEVERR_FP16_RANGE,
     GDN_DEVERR_SEQLENS,
     GDN_DEVERR_SLOT_RANGE,
+    GDN_DEVERR_TIMEOUT,
     GDN_DEVERR_TREE,
     GDN_ERR_CUDA,
     GDN_ERR_INVALID_ARG,
@@ -23,6 +25,7 @@ from .binding import (  # noqa: F401
     ssd_workspace_size,
     alloc_workspace,
     gdn_commit,
+    gdn_check_bounded_wait,
     gdn_commit_workspace_size,
     gdn_decode,
     gdn_decode_workspace_size,

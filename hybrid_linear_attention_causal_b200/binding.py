@@ -26,6 +26,7 @@ GDN_DEVERR_TIMEOUT = 0x4
 GDN_DEVERR_ACCEPT_RANGE = 0x8
 GDN_DEVERR_CKPT_RANGE = 0x10
 GDN_DEVERR_TREE = 0x20
+GDN_DEVERR_FP16_RANGE = 0x40
 GDN_DTYPE_F32 = 0
 GDN_DTYPE_BF16 = 1
 GDN_DTYPE_F16 = 2
@@ -152,6 +153,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_get_device_error.restype = ctypes.c_int
         L.gdn_reset_device_error.argtypes = [vp, vp]
         L.gdn_reset_device_error.restype = ctypes.c_int
+        L.gdn_check_bounded_wait.argtypes = [i32, ctypes.c_int64, vp, sz, vp]
+        L.gdn_check_bounded_wait.restype = ctypes.c_int
         L.gdn_set_launch_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
         L.gdn_set_launch_events.restype = ctypes.c_int
         L.gdn_strerror.argtypes = [ctypes.c_int]
@@ -323,6 +326,15 @@ def gdn_get_device_error(workspace, stream=None) -> int:
 
 def gdn_reset_device_error(workspace, stream=None) -> None:
     _check(lib().gdn_reset_device_error(_ptr(workspace), _stream(stream)), "gdn_reset_device_error")
+
+
+def gdn_check_bounded_wait(arrive: bool, limit_ns: int, workspace, stream=None) -> None:
+    """Runs the kernels' bounded mbarrier wait once on the device (see include/gdn.h): on a barrier
+    that completes (arrive=True) or that nothing completes (arrive=False: GDN_DEVERR_TIMEOUT after
+    limit_ns nanoseconds).  Asynchronous; read the outcome with gdn_get_device_error."""
+    _check(lib().gdn_check_bounded_wait(1 if arrive else 0, int(limit_ns), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "gdn_check_bounded_wait")
 
 
 def gdn_set_launch_events(events) -> None:

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include "gdn_internal.cuh"
+#include "gdn_tc.cuh"
 
 namespace {
 
@@ -64,7 +65,45 @@ bool all_aligned(P... ptrs) {
 
 namespace gdn {
 int record_cuda_failure(cudaError_t e) { return cuda_fail(e); }
+
+namespace {
+// The bounded mbarrier wait of the tensor-core kernels, on a barrier that this thread completes itself
+// (arrive) or that nothing completes; a wait that gives up raises GDN_DEVERR_TIMEOUT and returns.
+__global__ void bounded_wait_check_kernel(int32_t* hdr, int arrive, unsigned long long limit_ns) {
+    __shared__ __align__(8) unsigned long long bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = tc::smem_u32(&bar);
+    tc::mbar_init(b, 1);
+    tc::fence_mbar_init();
+    if (arrive) tc::mbar_arrive(b);
+    if (!tc::mbar_wait(b, 0, limit_ns)) raise_error(hdr, GDN_DEVERR_TIMEOUT);
+}
+}  // namespace
+
+
+int check_extend_args(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+                      const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
+                      const int32_t* has_initial_state, const void* conv_state, const float* ssm_state, int32_t P,
+                      const void* out, LayerDims* d, bool* nothing) {
+    *nothing = false;
+    int rc = check_cfg(cfg, d);
+    if (rc != GDN_OK) return rc;
+    if ((rc = check_params(params)) != GDN_OK) return rc;
+    if (N < 0 || T < 0 || P < 0) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens) return GDN_ERR_INVALID_ARG;
+    if (N == 0 || T == 0) {
+        *nothing = true;
+        return GDN_OK;
+    }
+    if (!mixed_qkv || !a || !b || !state_indices || !conv_state || !ssm_state || !out) return GDN_ERR_INVALID_ARG;
+    if (!all_aligned(mixed_qkv, a, b, cu_seqlens, state_indices, conv_state, ssm_state, out))
+        return GDN_ERR_INVALID_ARG;
+    if (has_initial_state && !aligned16(has_initial_state)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
 }  // namespace gdn
+
 
 void gdn::mark_launch(cudaStream_t s, int i) {
     if (i < g_num_events) cudaEventRecord(g_events[i], s);
@@ -116,16 +155,13 @@ int extend_impl(const gdn_config_t* cfg, const gdn_params_t* params, const void*
                 const int32_t* has_initial_state, void* conv_state, float* ssm_state, int32_t P, void* out,
                 const gdn::ExtendArgs& ck, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
     gdn::LayerDims d;
-    int rc = check_cfg(cfg, &d);
+    bool nothing = false;
+    int rc = gdn::check_extend_args(cfg, params, mixed_qkv, a, b, cu_seqlens, N, T, state_indices, has_initial_state,
+                                    conv_state, ssm_state, P, out, &d, &nothing);
     if (rc != GDN_OK) return rc;
-    if ((rc = check_params(params)) != GDN_OK) return rc;
-    if (N < 0 || T < 0 || P < 0) return GDN_ERR_INVALID_ARG;
-    if (!cu_seqlens || !workspace) return GDN_ERR_INVALID_ARG;
-    if (N == 0 || T == 0) return GDN_OK;
-    if (!mixed_qkv || !a || !b || !state_indices || !conv_state || !ssm_state || !out) return GDN_ERR_INVALID_ARG;
-    if (!all_aligned(mixed_qkv, a, b, cu_seqlens, state_indices, conv_state, ssm_state, out, workspace))
-        return GDN_ERR_INVALID_ARG;
-    if (has_initial_state && !aligned16(has_initial_state)) return GDN_ERR_INVALID_ARG;
+    if (!workspace) return GDN_ERR_INVALID_ARG;
+    if (nothing) return GDN_OK;
+    if (!aligned16(workspace)) return GDN_ERR_INVALID_ARG;
     if (workspace_bytes < gdn::extend_workspace_bytes(d, N, T, nullptr)) return GDN_ERR_WORKSPACE;
 
     gdn::ExtendArgs e{};
@@ -321,6 +357,16 @@ int gdn_commit(const gdn_config_t* cfg, const int32_t* state_indices, const int3
     p.hdr = static_cast<int32_t*>(workspace);
     cudaError_t err = gdn::launch_commit(p, reinterpret_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? GDN_OK : cuda_fail(err);
+}
+
+int gdn_check_bounded_wait(int32_t arrive, int64_t limit_ns, void* workspace, size_t workspace_bytes,
+                           gdn_stream_t stream) {
+    if (limit_ns <= 0 || limit_ns > 1000000000LL || !workspace || !aligned16(workspace)) return GDN_ERR_INVALID_ARG;
+    if (workspace_bytes < (size_t)gdn::kHeaderBytes) return GDN_ERR_WORKSPACE;
+    gdn::bounded_wait_check_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<int32_t*>(workspace), arrive != 0, (unsigned long long)limit_ns);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
 int gdn_get_device_error(const void* workspace, int32_t* err_out, gdn_stream_t stream) {

@@ -6,29 +6,43 @@
 // One (chunk, qk head) item at a time; an item serves the G value heads that
 // share the qk head.  For a chunk of n <= 64 rows starting at packed row t0:
 //
-//   rows t0-3 .. t0+n-1 of the item's channels are staged in shared memory
-//   (the 3 rows before the chunk come from the previous chunk of the same
-//   sequence, or from the conv-state slot for a sequence's first chunk);
-//   y = SiLU(conv1d(x)), q and k L2-normalised (q carries the output scale),
-//   g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b), gamma_r = sum_{s<=r} g_s;
+//   rows t0-3 .. t0+n-1 of the item's channels and their conv weights are
+//   staged in shared memory (the 3 rows before the chunk come from the
+//   previous chunk of the same sequence, or from the conv-state slot for a
+//   sequence's first chunk); y = SiLU(conv1d(x)), q and k L2-normalised (q
+//   carries the output scale), g = -exp(A_log) softplus(a + dt_bias),
+//   beta = sigmoid(b), gamma_r = sum_{s<=r} g_s;
 //
 //   D1  = [K; Q] K^T                          (fp16 MMA, M=128 N=64 K=dk)
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
-//   T   = (I + A)^{-1}                        (fp32: 16x16 forward substitution + block products)
+//   T   = (I + A)^{-1}
 //   W   = T diag(beta e^gamma) K              (fp16 MMA, M=64 N=dk K=64; K read MN-major)
-//   U^T = V^T (T diag(beta))^T                (fp16 MMA, M=dv N=64 K=64)
+//   U^T = V^T (T diag(beta))^T                (fp16 MMA, M=dv N=64 K=64; V read MN-major)
 //
 // (the WY/UT form of the gated delta rule, Gated DeltaNet, Yang, Kautz and
-// Hatamizadeh, ICLR 2025).  The item writes, as fp16 tiles in the tensor
-// core's 128-byte swizzled shared-memory layout (so the state pass copies
-// them verbatim): [K ; Q] once per (chunk, qk head), and per (chunk, value
-// head) W, U^T and the masked decayed q.k; plus gamma in fp32.  Rows past the
-// end of a ragged chunk are zero in every tile.  One thread issues the MMAs;
-// the eight warps read their sub-partition's 32-lane slice of tensor memory
-// (two warps per slice, one group of columns each) for the CUDA-core steps.
-// Two CTAs share an SM (half of its tensor memory and shared memory each), so
-// one CTA's barrier waits are covered by the other.
+// Hatamizadeh, ICLR 2025).  The triangular inverse runs in two stages: the
+// four 16x16 diagonal blocks of I + A by forward substitution in fp32 on the
+// CUDA cores (D = their inverses, block diagonal), then, with L the strictly
+// block-lower part of A and E = D L (nilpotent: E^4 = 0),
+//   T = (I + E)^{-1} D = (I - E)(I + E^2) D
+// as four fp16 products on the tensor core (E, E^2, P = (I + E^2) D and
+// T = (I - E) P), each result rounded to fp16 once on its way back to shared
+// memory.  T's diagonal blocks are D itself and E's entries are L's scaled by
+// D, so these roundings add nothing measurable to the fp16 rounding of
+// T diag(beta) that W and U need anyway.
+//
+// The item writes, as fp16 tiles in the tensor core's 128-byte swizzled
+// shared-memory layout (so the state pass copies them verbatim): [K ; Q] once
+// per (chunk, qk head), and per (chunk, value head) W, U^T and the masked
+// decayed q.k; plus a per-row gate vector in fp32.  Rows past the end of a
+// ragged chunk are zero in every tile.  One thread issues the MMAs; the eight
+// warps read their sub-partition's 32-lane slice of tensor memory (two warps
+// per slice, one group of columns each) for the CUDA-core steps.  Two CTAs
+// share an SM (half of its tensor memory and shared memory each), so one
+// CTA's barrier waits are covered by the other.
+
+#include <cuda_fp16.h>
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -39,9 +53,7 @@ namespace {
 constexpr int C = kChunk;
 constexpr int NT = 256;        // 8 warps; warp w reads TMEM sub-partition w % 4
 constexpr int kCtasPerSm = 2;
-constexpr int NCG = NT / 128;  // warps per TMEM sub-partition, each taking one group of columns
 constexpr uint32_t kTmemCols = 256;  // D1 (64 columns) + W (DK) + U^T (64), a half of tensor memory
-constexpr int kInvBarrier = 1;       // named barrier of warps 0-3, which take levels 1 and 2 of the inverse
 constexpr int kItemsPerCta = 2;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
@@ -52,6 +64,7 @@ struct ChunkShape {
     static constexpr int LDV = DV + PADE;                // staged v row
     static constexpr size_t XQK = (size_t)(C + 3) * LDQK * sizeof(T);
     static constexpr size_t XV = (size_t)(C + 3) * LDV * sizeof(T);
+    static constexpr size_t XMAX = XQK > XV ? XQK : XV;
 };
 
 template <typename T, int DK, int DV>
@@ -59,24 +72,27 @@ struct ChunkSmem {
     using S = ChunkShape<T, DK, DV>;
     // fp16 operand tiles in the 128-byte swizzled layout; each starts on a 1024-byte boundary
     uint16_t kq[2 * C * DK];  // [K ; Q*scale], 128 rows x DK: D1's operands, W's B (K rows read MN-major)
-    uint16_t bv[DV * C];      // V^T of the current value head, DV rows x C
-    uint16_t t[C * C];        // T diag(beta), C rows x C: U's operand
-    uint16_t te[C * C];       // T diag(beta e^gamma), same layout: W's operand
+    uint16_t vr[C * DV];      // V of the current value head, C rows x DV: U's A (read MN-major)
+    // the inverse's tiles (64 x 64 fp16 each) and fp32 diagonal blocks, or the raw rows being staged
     struct Inv {
-        float a[C][C + 1];     // A (fp32)
-        float tf[2][32][36];   // T (fp32) in its two 32x32 diagonal blocks: what the next levels read
-        float m[32][36];       // A21 T11
-        float y[2][16][20];    // A21 D1 inside each 32x32 diagonal block (rows 16-byte aligned)
+        uint16_t tile[4][C * C];  // roles rotate: D | L | E | I - E, then I + E^2 in L's, P in E's, and
+                                  // finally T diag(beta) in D's and T diag(beta e^gamma) in I - E's
+        float dg[4][16][20];      // the diagonal 16x16 blocks of A (fp32), rows padded
     };
-    // raw rows (q,k of the item, then v of one value head), or the inverse's fp32 work space
-    static constexpr size_t XMAX = S::XQK > S::XV ? S::XQK : S::XV;
-    static constexpr size_t UBYTES = XMAX > sizeof(Inv) ? XMAX : sizeof(Inv);
-    alignas(16) unsigned char u[UBYTES];
-    float2 gb[C];          // (g, beta) of the current value head
-    float gam[C], gam2[C], beta[C], bge[C];  // gamma, gamma log2(e), beta, beta e^gamma
+    static constexpr size_t UBYTES = S::XMAX > sizeof(Inv) ? S::XMAX : sizeof(Inv);
+    alignas(1024) unsigned char u[UBYTES];
+    alignas(16) T wq[2 * DK * 4];  // conv taps of the item's k then q channels
+    alignas(16) T wv[DV * 4];      // conv taps of the current value head's channels
+    float2 gb[C];                  // (g, beta) of the current value head
+    // gamma, gamma log2(e) (read as float4), beta, beta e^gamma
+    alignas(16) float gam[C];
+    alignas(16) float gam2[C];
+    alignas(16) float beta[C];
+    alignas(16) float bge[C];
     unsigned long long bar_mma;
     uint32_t tmem_base;
     int next_item;
+    int prefetch_item;        // the item after the current one, or -1
 };
 
 template <typename T, int DK, int DV>
@@ -84,9 +100,7 @@ constexpr size_t chunk_smem_bytes() {
     return sizeof(ChunkSmem<T, DK, DV>) + 1024;  // + room to align the tiles on 1024 bytes
 }
 
-__device__ __forceinline__ void bar_sync_n(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
-// 4 consecutive staged elements -> 4 floats (8-byte load for bf16, 16-byte for fp32)
+// 4 consecutive elements -> 4 floats (8-byte load for bf16, 16-byte for fp32)
 __device__ __forceinline__ void load4(const __nv_bfloat16* p, float* v) {
     const uint2 w = *reinterpret_cast<const uint2*>(p);
     v[0] = __uint_as_float(w.x << 16);
@@ -99,20 +113,53 @@ __device__ __forceinline__ void load4(const float* p, float* v) {
     v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
 }
 
-// SiLU with the fast exponential and division: their error (a few ulp) is far below the fp16
-// rounding every conv output goes through
-__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+// SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x / 2, with the hardware tanh (one MUFU operation;
+// its error is below the fp16 rounding every conv output goes through)
+__device__ __forceinline__ float silu_fast(float x) {
+    const float h = 0.5f * x;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
 
-// 8 floats -> 8 fp16 (one 16-byte store) at byte offset `off` of a tile in global memory
-__device__ __forceinline__ void store_h8_global(char* tile, uint32_t off, const float* v) {
+// 8 floats -> 8 fp16 (one 16-byte store) at byte offset `off` of a tile
+__device__ __forceinline__ void store_h8(char* tile, uint32_t off, const float* v) {
     *reinterpret_cast<uint4*>(tile + off) = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
                                                        tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
+}
+
+// conv1d (K = 4) + SiLU of 8 consecutive output rows r0 .. r0+7 (rows >= n give 0) of 4 consecutive
+// channels, from staged rows r0 .. r0+10 (staged row i holds packed row t0 - 3 + i) with a sliding
+// window; `xs` points at the first of the 4 channels in staged row 0, `w` at their 16 taps.
+template <typename T>
+__device__ __forceinline__ void conv8x4(const T* xs, int ld, const T* w, const T* bias, int r0, int n,
+                                        float (&y)[8][4]) {
+    float wt[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load4(w + 4 * u, wt[u]);
+    float b[4] = {0.f, 0.f, 0.f, 0.f};
+    if (bias) load4(bias, b);
+    float win[4][4];
+#pragma unroll
+    for (int i = 0; i < 3; ++i) load4(xs + (size_t)(r0 + i) * ld, win[i]);
+#pragma unroll
+    for (int o = 0; o < 8; ++o) {
+        load4(xs + (size_t)(r0 + o + 3) * ld, win[(o + 3) & 3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float acc = b[u];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc = fmaf(wt[u][j], win[(o + j) & 3][u], acc);
+            y[o][u] = r0 + o < n ? silu_fast(acc) : 0.f;
+        }
+    }
 }
 
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, int seg) {
     using S = ChunkShape<T, DK, DV>;
     using Sm = ChunkSmem<T, DK, DV>;
+    static_assert(DK % 32 == 0 && DV % 32 == 0, "channel groups of 4 per lane");
     if (batch_rejected(p)) return;
     const LayerDims& d = p.d;
     const int G = d.G, HV = d.HV, HK = d.HK;
@@ -144,52 +191,65 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
     const T* cbias = reinterpret_cast<const T*>(p.conv_b);
     T* xs = reinterpret_cast<T*>(sm.u);
     typename Sm::Inv& inv = *reinterpret_cast<typename Sm::Inv*>(sm.u);
+    char* tiles = reinterpret_cast<char*>(inv.tile);
+    auto tile_b = [&](int i) { return tiles + (size_t)i * C * C * 2; };
+    auto tile_s = [&](int i) { return tc::smem_u32(tiles) + (uint32_t)i * C * C * 2; };
 
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
     if (tid == 0) {
         tc::mbar_init(bar, 1);
         tc::fence_mbar_init();
     }
-    // blocks of T above the diagonal are zero for every head: in the tiles, and in the two 16x16
-    // corners of the 32x32 diagonal blocks that the inverse reads back
-    for (int e = tid; e < C * C; e += NT) sm.t[e] = sm.te[e] = 0;
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
-    // D1: 64 columns; W: M = 64 layout, DK columns; U^T: M = DV, 64 columns
-    const uint32_t tD1 = tm, tW = tm + 64, tU = tm + 64 + DK;
+    // D1: 64 columns; the inverse's accumulators X1, X2 (64 columns each, M = 64 layout) and then W
+    // (DK columns) at tm + 64; U^T (M = DV, 64 columns) at tm + 64 + DK
+    const uint32_t tD1 = tm, tX1 = tm + 64, tX2 = tm + 128, tW = tm + 64, tU = tm + 64 + DK;
+    static_assert(64 + DK + 64 <= (int)kTmemCols && 192 <= 64 + DK + 64, "tensor-memory layout");
     const int sp = warp & 3, cg = warp >> 2;  // TMEM sub-partition, column group
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     uint32_t ph_mma = 0;
     bool ok = true;
     int done = 0;
+    float amax = 0.f;  // largest magnitude this thread rounded to fp16 among v, T's tiles, W and U
+    // all threads wait for the tensor core's latest commit
+    auto wait_mma = [&]() -> bool {
+        const bool r = __syncthreads_and(tc::mbar_wait(bar, ph_mma));
+        ph_mma ^= 1;
+        tc::fence_after_sync();
+        return r;
+    };
+    // an M = 64 accumulator (rows 16 sp + lane in lanes 0-15 of sub-partition sp) -> 32 columns of this
+    // warp's group for row m: `f(m, c0, v16)` per 16 columns
+    auto read64 = [&](uint32_t t0, auto&& f) {
+#pragma unroll
+        for (int c0 = 32 * cg; c0 < 32 * cg + 32; c0 += 16) {
+            float v[16];
+            tc::tmem_ld16(t0 + lane_base + c0, v);
+            tc::tmem_ld_wait();
+            if (lane < 16) f(sp * 16 + lane, c0, v);
+        }
+    };
+
     while (ok && item >= 0) {
         int nxt = -1;
         // At most kItemsPerCta items, then the CTA ends: its SM goes to whatever waits, first of all a
         // state-pass CTA of the previous segment (its stream has the higher priority).
         if (tid == 0 && ++done < kItemsPerCta) nxt = grab();
+        if (tid == 0) sm.prefetch_item = nxt;  // read by every thread after the staging barrier
         const int id = item / HK, hk = item % HK;
         const int4 ch = p.chunk_tab[id];
         const int seq = ch.x, t0 = ch.y, n = ch.z, cidx = ch.w;
         const int slot = p.slots[seq];
         const bool init = p.has_init ? p.has_init[seq] != 0 : true;
         const int ck0 = d.HK * DK + hk * DK, cq0 = hk * DK;  // first k / q channel
-        if (tid == 0 && nxt >= 0) {  // the next item's rows into L2 while this one computes
-            const int4 chn = p.chunk_tab[nxt / HK];
-            const int hkn = nxt % HK;
-            const int r0 = chn.w > 0 ? chn.y - 3 : chn.y;
-            for (int r = r0; r < chn.y + chn.z; ++r) {
-                const T* row = x + (size_t)r * d.conv_dim;
-                tc::bulk_prefetch_l2(row + hkn * DK, DK * sizeof(T));
-                tc::bulk_prefetch_l2(row + d.HK * DK + hkn * DK, DK * sizeof(T));
-                tc::bulk_prefetch_l2(row + 2 * d.HK * DK + hkn * G * DV, G * DV * sizeof(T));
-            }
-        }
-        // ---- stage the q,k rows: staged row i <-> packed row t0 - 3 + i; columns k then q
+        const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
+        constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
+        // ---- stage the q,k rows (staged row i <-> packed row t0 - 3 + i; columns k then q) and taps
         {
-            constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
-            constexpr int VPR = 2 * DK / VE;         // vectors per staged row
+            constexpr int VPR = 2 * DK / VE;  // vectors per staged row
             const int nv = n * VPR;
             for (int b0 = 0; b0 < nv; b0 += NT * 4) {
                 uint4 v[4];
@@ -211,7 +271,6 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                     }
                 }
             }
-            const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
             for (int e = tid; e < 3 * 2 * DK; e += NT) {
                 const int i = e / (2 * DK), c = e % (2 * DK);
                 const int gc = c < DK ? ck0 + c : cq0 + (c - DK);
@@ -220,53 +279,55 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 else v = init ? cs[(size_t)gc * 3 + i] : from_f<T>(0.f);
                 xs[(size_t)i * S::LDQK + c] = v;
             }
+            constexpr int WV = DK * 4 / VE;  // vectors of one part's taps
+            for (int e = tid; e < 2 * WV; e += NT) {
+                const int c0 = e < WV ? ck0 : cq0, o = (e % WV) * VE;
+                *reinterpret_cast<uint4*>(sm.wq + (e < WV ? 0 : DK * 4) + o) =
+                    *reinterpret_cast<const uint4*>(w + (size_t)c0 * 4 + o);
+            }
         }
         __syncthreads();
-        // ---- conv + SiLU + L2 norm of k (tile rows 0..63) and q*scale (rows 64..127): warp w takes
-        // rows 8w .. 8w+7; lane (rr, cc) row 8w + rr and the column quads 16 c + 4 cc; a row's four
-        // lanes hold all DK channels, so the norm reduces over them
-        {
-            const int rr = lane & 7, cc = lane >> 3;
-            const int r = 8 * warp + rr;
-            char* kqb = reinterpret_cast<char*>(sm.kq);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int gc0 = part == 0 ? ck0 : cq0;
-                float y[DK / 16][4];
-                float ss = 0.f;
-#pragma unroll
-                for (int c16 = 0; c16 < DK / 16; ++c16) {
-                    const int cl = 16 * c16 + 4 * cc;  // first of 4 channels, within the part
-                    float acc[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int gc = gc0 + cl + u;
-                        acc[u] = cbias ? to_f(cbias[gc]) : 0.f;
-                    }
-                    if (r < n) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            float xv[4];
-                            load4(xs + (size_t)(r + j) * S::LDQK + part * DK + cl, xv);
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) acc[u] = fmaf(to_f(w[(size_t)(gc0 + cl + u) * 4 + j]), xv[u], acc[u]);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        y[c16][u] = r < n ? silu_fast(acc[u]) : 0.f;
-                        ss = fmaf(y[c16][u], y[c16][u], ss);
-                    }
+        {  // the next item's rows into L2 while this one computes: one 128-byte line per prefetch, spread
+           // over every thread (its q, k and v pieces of each row: 2 DK + G DV elements)
+            const int pi = sm.prefetch_item;
+            if (pi >= 0) {
+                const int4 chn = p.chunk_tab[pi / HK];
+                const int hkn = pi % HK;
+                const int r0 = chn.w > 0 ? chn.y - 3 : chn.y, nr = chn.y + chn.z - r0;
+                constexpr int LQ = DK * (int)sizeof(T) / 128, LV = DV * (int)sizeof(T) / 128;  // lines per piece
+                const int lpr = 2 * LQ + G * LV;                                                 // lines per row
+                for (int e = tid; e < nr * lpr; e += NT) {
+                    const int r = r0 + e / lpr, l = e % lpr;
+                    const T* row = x + (size_t)r * d.conv_dim;
+                    const T* a_ = l < LQ ? row + hkn * DK + l * (128 / sizeof(T))
+                                : l < 2 * LQ ? row + d.HK * DK + hkn * DK + (l - LQ) * (128 / sizeof(T))
+                                             : row + 2 * d.HK * DK + hkn * G * DV + (l - 2 * LQ) * (128 / sizeof(T));
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a_));
                 }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 8);
-                ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-                const float sc = r < n ? rsqrtf(ss + d.eps) * (part ? d.scale : 1.f) : 0.f;
-                const int tr = part * C + r;  // tile row
+            }
+        }
+        // ---- conv + SiLU + L2 norm of k (tile rows 0..63) and q*scale (rows 64..127).  A task is 8 rows
+        // of one part; its DK / 4 lanes take 4 channels each, so a row's norm reduces over them.
+        {
+            constexpr int LPP = DK / 4, PPW = 32 / LPP;  // lanes per part, parts per warp
+            const int l = lane % LPP;
+            char* kqb = reinterpret_cast<char*>(sm.kq);
+            for (int task = warp * PPW + lane / LPP; task < 2 * (C / 8); task += 8 * PPW) {
+                const int part = task & 1, r0 = 8 * (task >> 1);
+                const int gc0 = part == 0 ? ck0 : cq0;
+                float y[8][4];
+                conv8x4(xs + part * DK + 4 * l, S::LDQK, sm.wq + (part * DK + 4 * l) * 4,
+                        cbias ? cbias + gc0 + 4 * l : nullptr, r0, n, y);
 #pragma unroll
-                for (int c16 = 0; c16 < DK / 16; ++c16) {
-                    const int cl = 16 * c16 + 4 * cc;
-                    *reinterpret_cast<uint2*>(kqb + tc::sw128_off(tr, cl, 2 * C)) =
-                        make_uint2(tc::pack_f16(y[c16][0] * sc, y[c16][1] * sc), tc::pack_f16(y[c16][2] * sc, y[c16][3] * sc));
+                for (int o = 0; o < 8; ++o) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) ss = fmaf(y[o][u], y[o][u], ss);
+#pragma unroll
+                    for (int m = LPP / 2; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                    const float sc = r0 + o < n ? rsqrtf(ss + d.eps) * (part ? d.scale : 1.f) : 0.f;
+                    *reinterpret_cast<uint2*>(kqb + tc::sw128_off(part * C + r0 + o, 4 * l, 2 * C)) =
+                        make_uint2(tc::pack_f16(y[o][0] * sc, y[o][1] * sc), tc::pack_f16(y[o][2] * sc, y[o][3] * sc));
                 }
             }
         }
@@ -288,10 +349,9 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
         for (int j = 0; j < G && ok; ++j) {
             const int h = hk * G + j;
             const size_t ch_h = (size_t)id * HV + h;
-            // ---- stage this value head's v rows (the q,k rows are no longer needed), and its gates
+            const int cv0 = 2 * d.HK * DK + h * DV;  // first v channel of this head
+            // ---- stage this value head's v rows and taps (the q,k rows are no longer needed), and gates
             {
-                const int cv0 = 2 * d.HK * DK + h * DV;
-                constexpr int VE = 16 / (int)sizeof(T);
                 constexpr int VPR = DV / VE;
                 const int nv = n * VPR;
                 for (int b0 = 0; b0 < nv; b0 += NT * 4) {
@@ -309,7 +369,6 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                         if (e < nv) *reinterpret_cast<uint4*>(xs + (size_t)(e / VPR + 3) * S::LDV + (e % VPR) * VE) = v[u];
                     }
                 }
-                const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
                 for (int e = tid; e < 3 * DV; e += NT) {
                     const int i = e / DV, c = e % DV;
                     T v;
@@ -317,6 +376,8 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                     else v = init ? cs[(size_t)(cv0 + c) * 3 + i] : from_f<T>(0.f);
                     xs[(size_t)i * S::LDV + c] = v;
                 }
+                for (int e = tid; e < DV * 4 / VE; e += NT)
+                    *reinterpret_cast<uint4*>(sm.wv + e * VE) = *reinterpret_cast<const uint4*>(w + (size_t)cv0 * 4 + e * VE);
                 if (tid >= NT - C) {  // gates of the chunk's rows (zero past the end)
                     const int r = tid - (NT - C);
                     float2 gb = make_float2(0.f, 0.f);
@@ -330,33 +391,23 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 }
             }
             __syncthreads();
-            // ---- V^T tile: thread (f, 4 consecutive rows) from a sliding window of 7 staged rows; warp 0
-            // also scans the gates
+            // ---- V rows (conv + SiLU) into the V tile: a task is 8 rows of DV / 4 lanes; warp 0 also
+            // scans the gates
             {
-                char* bvb = reinterpret_cast<char*>(sm.bv);
-                for (int idx = tid; idx < DV * (C / 4); idx += NT) {
-                    const int ff = idx & 7, cq = (idx >> 3) & 3, rest = idx >> 5;
-                    const int fg = rest % (DV / 8), rg = rest / (DV / 8);
-                    const int f = 8 * fg + ff, r4 = 4 * (4 * rg + cq);
-                    const int gcv = 2 * d.HK * DK + h * DV + f;
-                    float wc[4];
+                constexpr int LPV = DV / 4, VPW = 32 / LPV;
+                const int l = lane % LPV;
+                char* vrb = reinterpret_cast<char*>(sm.vr);
+                for (int task = warp * VPW + lane / LPV; task < C / 8; task += 8 * VPW) {
+                    const int r0 = 8 * task;
+                    float y[8][4];
+                    conv8x4(xs + 4 * l, S::LDV, sm.wv + 16 * l, cbias ? cbias + cv0 + 4 * l : nullptr, r0, n, y);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) wc[q] = to_f(w[(size_t)gcv * 4 + q]);
-                    const float b0 = cbias ? to_f(cbias[gcv]) : 0.f;
-                    float xw[7];
+                    for (int o = 0; o < 8; ++o) {
 #pragma unroll
-                    for (int i = 0; i < 7; ++i) xw[i] = to_f(xs[(size_t)(r4 + i) * S::LDV + f]);
-                    float yv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        float acc = fmaf(wc[0], xw[u], b0);
-                        acc = fmaf(wc[1], xw[u + 1], acc);
-                        acc = fmaf(wc[2], xw[u + 2], acc);
-                        acc = fmaf(wc[3], xw[u + 3], acc);
-                        yv[u] = r4 + u < n ? silu_fast(acc) : 0.f;
+                        for (int u = 0; u < 4; ++u) amax = fmaxf(amax, fabsf(y[o][u]));
+                        *reinterpret_cast<uint2*>(vrb + tc::sw128_off(r0 + o, 4 * l, C)) =
+                            make_uint2(tc::pack_f16(y[o][0], y[o][1]), tc::pack_f16(y[o][2], y[o][3]));
                     }
-                    *reinterpret_cast<uint2*>(bvb + tc::sw128_off(f, r4, DV)) =
-                        make_uint2(tc::pack_f16(yv[0], yv[1]), tc::pack_f16(yv[2], yv[3]));
                 }
                 if (warp == 0) {  // inclusive scan of g over the chunk, two rows per lane
                     const float2 g0 = sm.gb[2 * lane], g1 = sm.gb[2 * lane + 1];
@@ -378,26 +429,24 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                     sm.bge[2 * lane + 1] = g1.y * __expf(incl);
                 }
             }
-            bool okv = true;
-            if (j == 0) okv = tc::mbar_wait(bar, ph_mma);  // D1
-            ok = __syncthreads_and(okv);
-            if (!ok) break;
             if (j == 0) {
-                ph_mma ^= 1;
-                tc::fence_after_sync();
+                ok = wait_mma();  // D1, and the barrier that publishes the gates
+            } else {
+                __syncthreads();
             }
-            // ---- A (sub-partitions 0-1: k.k rows) into shared memory and the masked decayed q.k tile
-            // (2-3: q.k rows) straight to global memory, from D1; the warps of a sub-partition take one
-            // group of C / NCG columns each.  The exponents are formed without branches (a masked entry
-            // gets -inf, whose exponential is 0); a block wholly above the diagonal only gets zeros.
+            if (!ok) break;
+            // ---- from D1: A's diagonal 16x16 blocks (fp32) and its strictly block-lower part L (fp16 tile
+            // 1) from the k.k rows (sub-partitions 0-1), the masked decayed q.k tile straight to global
+            // memory from the q.k rows (2-3); the warps of a sub-partition take one group of 32 columns
+            // each.  The exponents are formed without branches (a masked entry gets -inf, whose
+            // exponential is 0); a block wholly above the diagonal only gets zeros.
             {
                 char* AQg = reinterpret_cast<char*>(p.AQ + ch_h * (C * C));
-                constexpr int NC = C / NCG;
-                static_assert(NC % 16 == 0, "16-column loads");
+                char* Lt = tile_b(1);
                 const int r = (sp & 1) * 32 + lane;
                 const bool qrow = sp >= 2;
 #pragma unroll
-                for (int c0 = NC * cg; c0 < NC * (cg + 1); c0 += 16) {
+                for (int c0 = 32 * cg; c0 < 32 * cg + 32; c0 += 16) {
                     const bool live = c0 <= (sp & 1) * 32 + 31;  // warp-uniform
                     float v[16], e[16];
                     if (live) {
@@ -422,142 +471,139 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                     if (!qrow) {
                         const float br = sm.beta[r];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) inv.a[r][c0 + i] = br * e[i];
+                        for (int i = 0; i < 16; ++i) e[i] *= br;
+                        if (c0 == 16 * (r >> 4)) {  // the diagonal block: fp32, and zeros in L
+#pragma unroll
+                            for (int q = 0; q < 16; q += 4)
+                                *reinterpret_cast<float4*>(&inv.dg[r >> 4][r & 15][q]) =
+                                    make_float4(e[q], e[q + 1], e[q + 2], e[q + 3]);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) e[i] = 0.f;
+                        }
+                        store_h8(Lt, tc::sw128_off(r, c0, C), e);
+                        store_h8(Lt, tc::sw128_off(r, c0 + 8, C), e + 8);
                     } else {
-                        store_h8_global(AQg, tc::sw128_off(r, c0, C), e);
-                        store_h8_global(AQg, tc::sw128_off(r, c0 + 8, C), e + 8);
+                        store_h8(AQg, tc::sw128_off(r, c0, C), e);
+                        store_h8(AQg, tc::sw128_off(r, c0 + 8, C), e + 8);
                     }
                 }
             }
-            tc::fence_before_sync();
             __syncthreads();
-            tc::fence_after_sync();
-            // T = (I + A)^{-1}, by blocks.  Every final entry goes straight into the fp16 tiles of
-            // T diag(beta) and T diag(beta e^gamma) (the A operands of U and W); the fp32 copy tf holds
-            // what the next level reads.
-            //   level 1: the four diagonal 16x16 blocks by forward substitution, one column per lane held
-            //            in registers (t_r = [r == c] - sum_{s<r} A_rs t_s; the s = r-1 term goes last so
-            //            one FMA per row sits on the dependent chain); the other warps write gamma.
-            //   level 2: within each 32x32 diagonal block, X = -D2 (A21 D1).
-            //   level 3: T21 = -T22 (A21 T11) for the lower-left 32x32 block.
-            char* tb = reinterpret_cast<char*>(sm.t);
-            char* teb = reinterpret_cast<char*>(sm.te);
-            auto put_t = [&](int r, int c, float v) {  // T entry (r, c) into both operand tiles
-                const uint32_t off = tc::sw128_off(r, c, C);
-                const uint32_t wv = tc::pack_f16(v * sm.beta[c], v * sm.bge[c]);
-                *reinterpret_cast<uint16_t*>(tb + off) = (uint16_t)(wv & 0xffffu);
-                *reinterpret_cast<uint16_t*>(teb + off) = (uint16_t)(wv >> 16);
-            };
-            auto fma4 = [](float4& acc, float a, const float4& b) {
-                acc.x = fmaf(a, b.x, acc.x);
-                acc.y = fmaf(a, b.y, acc.y);
-                acc.z = fmaf(a, b.z, acc.z);
-                acc.w = fmaf(a, b.w, acc.w);
-            };
-            if (warp < 4) {
-                if (lane < 16) {
-                    const int o = 16 * warp, c = lane;
-                    float t[16];
+            // ---- D = the inverses of A's diagonal 16x16 blocks, by forward substitution in fp32 (warps
+            // 0-1: lane (block, column c), t_r = [r == c] - sum_{s<r} A_rs t_s), into fp16 tile 0, whose
+            // other blocks warps 2-7 clear; warps 4-5 also write the state pass's gate vectors
+            if (warp < 2) {
+                const int bk = 2 * warp + (lane >> 4), c = lane & 15;
+                float t[16];
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        const float* arow = &inv.a[o + r][o];
-                        float acc[2] = {r == c ? 1.f : 0.f, 0.f};
+                for (int r = 0; r < 16; ++r) {
+                    const float* arow = inv.dg[bk][r];
+                    float acc[2] = {r == c ? 1.f : 0.f, 0.f};
 #pragma unroll
-                        for (int s = 0; s + 1 < r; ++s) acc[s & 1] = fmaf(-arow[s], t[s], acc[s & 1]);
-                        const float b2 = acc[0] + acc[1];
-                        t[r] = r > 0 ? fmaf(-arow[r - 1], t[r - 1], b2) : b2;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        inv.tf[warp >> 1][16 * (warp & 1) + r][16 * (warp & 1) + c] = t[r];
-                        put_t(o + r, o + c, t[r]);
-                    }
-                } else if ((warp & 1) == 0) {  // the 16x16 corner above the diagonal of 32x32 block warp / 2
-                    float4* row = reinterpret_cast<float4*>(&inv.tf[warp >> 1][lane - 16][16]);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) row[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int s = 0; s + 1 < r; ++s) acc[s & 1] = fmaf(-arow[s], t[s], acc[s & 1]);
+                    const float b2 = acc[0] + acc[1];
+                    t[r] = r > 0 ? fmaf(-arow[r - 1], t[r - 1], b2) : b2;
                 }
-                bar_sync_n(kInvBarrier, 128);
-                {  // level 2 (threads 0..127): 32-block bb, row r, columns c4 .. c4 + 3
-                    const int bb = tid >> 6, r = (tid >> 2) & 15, c4 = 4 * (tid & 3);
-                    const int o0 = 32 * bb, o1 = o0 + 16;
-                    {
-                        float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
+                char* Dt = tile_b(0);
 #pragma unroll
-                        for (int s = 0; s < 16; ++s)  // Y = A21 D1
-                            fma4(yv, inv.a[o1 + r][o0 + s], *reinterpret_cast<const float4*>(&inv.tf[bb][s][c4]));
-                        *reinterpret_cast<float4*>(&inv.y[bb][r][c4]) = yv;
-                    }
-                    bar_sync_n(kInvBarrier, 128);
-                    {
-                        float4 xq = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                        for (int s = 0; s < 16; ++s)  // X = -D2 Y
-                            fma4(xq, inv.tf[bb][16 + r][16 + s], *reinterpret_cast<const float4*>(&inv.y[bb][s][c4]));
-                        xq = make_float4(-xq.x, -xq.y, -xq.z, -xq.w);
-                        *reinterpret_cast<float4*>(&inv.tf[bb][16 + r][c4]) = xq;
-                        put_t(o1 + r, o0 + c4, xq.x);
-                        put_t(o1 + r, o0 + c4 + 1, xq.y);
-                        put_t(o1 + r, o0 + c4 + 2, xq.z);
-                        put_t(o1 + r, o0 + c4 + 3, xq.w);
-                    }
+                for (int r = 0; r < 16; ++r)
+                    *reinterpret_cast<__half*>(Dt + tc::sw128_off(16 * bk + r, 16 * bk + c, C)) = __float2half_rn(t[r]);
+            } else {
+                // the chunks of tile 0 outside the diagonal blocks: in row r, every 16-byte chunk but the
+                // two that hold columns 16 (r / 16) .. 16 (r / 16) + 15
+                char* Dt = tile_b(0);
+                for (int e = tid - 64; e < C * 6; e += NT - 64) {
+                    const int r = e / 6, k = e % 6;
+                    const int c8 = k < 2 * (r >> 4) ? k : k + 2;
+                    *reinterpret_cast<uint4*>(Dt + tc::sw128_off(r, 8 * c8, C)) = make_uint4(0u, 0u, 0u, 0u);
                 }
-            } else if (tid - 128 < C) {  // the state pass's per-row gate vector
-                const int r = tid - 128;
-                const float gr = sm.gam[r], gn = sm.gam[n - 1];
-                p.GV[ch_h * C + r] = make_float4(__expf(gr), r < n ? __expf(gn - gr) : 0.f, gr, __expf(gn));
-            }
-            __syncthreads();
-            // Level 3 reads one operand as a warp-wide broadcast and skips the zero blocks of the
-            // triangular factors: T11[s][c] = 0 for s < c and T22[r][s] = 0 for s > r.
-            static_assert(NT / 32 == 8, "level 3 maps 8 column groups, then row groups, onto the warps");
-            {  // level 3a: P = A21 T11; warp w takes columns 4w .. 4w + 3, lane = row
-                const int r = lane, c4 = 4 * warp;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-                for (int s = c4; s < 32; ++s)
-                    fma4(acc, inv.a[32 + r][s], *reinterpret_cast<const float4*>(&inv.tf[0][s][c4]));
-                *reinterpret_cast<float4*>(&inv.m[r][c4]) = acc;
-            }
-            __syncthreads();
-            {  // level 3b: T21 = -T22 P; warp w takes 4 consecutive rows of the block, lane = column
-                constexpr int RPW = 4;
-                const int r0 = RPW * warp, c = lane;
-                float acc[RPW];
-#pragma unroll
-                for (int i = 0; i < RPW; ++i) acc[i] = 0.f;
-                for (int s4 = 0; s4 < r0 + RPW; s4 += 4) {
-                    const float p0 = inv.m[s4][c], p1 = inv.m[s4 + 1][c], p2 = inv.m[s4 + 2][c], p3 = inv.m[s4 + 3][c];
-#pragma unroll
-                    for (int i = 0; i < RPW; ++i) {
-                        const float4 t = *reinterpret_cast<const float4*>(&inv.tf[1][r0 + i][s4]);
-                        acc[i] = fmaf(t.x, p0, fmaf(t.y, p1, fmaf(t.z, p2, fmaf(t.w, p3, acc[i]))));
-                    }
+                if (warp >= 4 && warp < 6) {  // the state pass's gate vectors: e^gamma, f, gamma, e^{gamma_n}
+                    const int r = tid - 128;
+                    const float gr = sm.gam[r], gn = sm.gam[n - 1];
+                    float* gv = reinterpret_cast<float*>(p.GV + ch_h * C);
+                    gv[r] = __expf(gr);
+                    gv[C + r] = r < n ? __expf(gn - gr) : 0.f;
+                    gv[2 * C + r] = gr;
+                    gv[3 * C + r] = __expf(gn);
                 }
-#pragma unroll
-                for (int i = 0; i < RPW; ++i) put_t(32 + r0 + i, c, -acc[i]);
             }
             tc::fence_smem_to_async();
             tc::fence_before_sync();
             __syncthreads();
             tc::fence_after_sync();
+            // ---- T = (I - E)(I + E^2) D with E = D L: four fp16 products, each result rounded once
+            constexpr uint32_t i64 = tc::idesc_f16(64, 64) | tc::kTransposeB;
+            // issue a 64 x 64 x 64 product of tile `a` (K-major) and tile `b` (read MN-major) into `acc`
+            auto product = [&](uint32_t acc, int a, int b) {
+                if (tid == 0) {
+#pragma unroll
+                    for (int s = 0; s < C / 16; ++s)
+                        tc::mma_f16(acc, tc::desc_sw128_k(tile_s(a), C, s), tc::desc_sw128_mn(tile_s(b), C, s), i64, s > 0);
+                    tc::mma_commit(bar);
+                }
+                return wait_mma();
+            };
+            auto publish = [&]() {  // the tiles written above are complete and visible to the tensor core
+                tc::fence_smem_to_async();
+                tc::fence_before_sync();
+                __syncthreads();
+                tc::fence_after_sync();
+            };
+            if (!(ok = product(tX1, 0, 1))) break;  // E = D L
+            read64(tX1, [&](int m, int c0, const float* v) {  // E -> tile 2, I - E -> tile 3
+                float ne[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ne[i] = (c0 + i == m ? 1.f : 0.f) - v[i];
+                store_h8(tile_b(2), tc::sw128_off(m, c0, C), v);
+                store_h8(tile_b(2), tc::sw128_off(m, c0 + 8, C), v + 8);
+                store_h8(tile_b(3), tc::sw128_off(m, c0, C), ne);
+                store_h8(tile_b(3), tc::sw128_off(m, c0 + 8, C), ne + 8);
+            });
+            publish();
+            if (!(ok = product(tX2, 2, 2))) break;  // E^2 = E E
+            read64(tX2, [&](int m, int c0, const float* v) {  // I + E^2 -> tile 1 (L is no longer needed)
+                float pe[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pe[i] = (c0 + i == m ? 1.f : 0.f) + v[i];
+                store_h8(tile_b(1), tc::sw128_off(m, c0, C), pe);
+                store_h8(tile_b(1), tc::sw128_off(m, c0 + 8, C), pe + 8);
+            });
+            publish();
+            if (!(ok = product(tX1, 1, 0))) break;  // P = (I + E^2) D
+            read64(tX1, [&](int m, int c0, const float* v) {  // P -> tile 2 (E is no longer needed)
+                store_h8(tile_b(2), tc::sw128_off(m, c0, C), v);
+                store_h8(tile_b(2), tc::sw128_off(m, c0 + 8, C), v + 8);
+            });
+            publish();
+            if (!(ok = product(tX2, 3, 2))) break;  // T = (I - E) P
+            read64(tX2, [&](int m, int c0, const float* v) {  // T diag(beta) -> tile 0, T diag(beta e^gamma) -> 3
+                float tb[16], te[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    tb[i] = v[i] * sm.beta[c0 + i];
+                    te[i] = v[i] * sm.bge[c0 + i];
+                    amax = fmaxf(amax, fmaxf(fabsf(tb[i]), fabsf(te[i])));
+                }
+                store_h8(tile_b(0), tc::sw128_off(m, c0, C), tb);
+                store_h8(tile_b(0), tc::sw128_off(m, c0 + 8, C), tb + 8);
+                store_h8(tile_b(3), tc::sw128_off(m, c0, C), te);
+                store_h8(tile_b(3), tc::sw128_off(m, c0 + 8, C), te + 8);
+            });
+            publish();
             if (tid == 0) {  // W = (T diag(beta e^gamma)) K (M = 64, K read MN-major from the [K ; Q] tile),
-                             // U^T = V^T (T diag(beta))^T (M = DV)
-                const uint32_t bt = tc::smem_u32(sm.t), bte = tc::smem_u32(sm.te), bkq = tc::smem_u32(sm.kq);
-                const uint32_t bvv = tc::smem_u32(sm.bv);
-                constexpr uint32_t iw = tc::idesc_f16(64, DK) | tc::kTransposeB, iu = tc::idesc_f16(DV, 64);
+                             // U^T = V^T (T diag(beta))^T (M = DV, V read MN-major)
+                const uint32_t bkq = tc::smem_u32(sm.kq), bvr = tc::smem_u32(sm.vr);
+                constexpr uint32_t iw = tc::idesc_f16(64, DK) | tc::kTransposeB;
+                constexpr uint32_t iu = tc::idesc_f16(DV, 64) | tc::kTransposeA;
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    tc::mma_f16(tW, tc::desc_sw128_k(bte, C, s), tc::desc_sw128_mn(bkq, 2 * C, s), iw, s > 0);
+                    tc::mma_f16(tW, tc::desc_sw128_k(tile_s(3), C, s), tc::desc_sw128_mn(bkq, 2 * C, s), iw, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    tc::mma_f16(tU, tc::desc_sw128_k(bvv, DV, s), tc::desc_sw128_k(bt, C, s), iu, s > 0);
+                    tc::mma_f16(tU, tc::desc_sw128_mn(bvr, C, s), tc::desc_sw128_k(tile_s(0), C, s), iu, s > 0);
                 tc::mma_commit(bar);
             }
-            ok = __syncthreads_and(tc::mbar_wait(bar, ph_mma));
-            ph_mma ^= 1;
-            if (!ok) break;
-            tc::fence_after_sync();
+            if (!(ok = wait_mma())) break;
             {  // W rows -> the W tile; U -> the U^T tile (both fp16, swizzled, straight to global memory).
                // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15; the warps
                // of a sub-partition take one group of columns each
@@ -566,25 +612,29 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 const bool valid = lane < 16;
                 const int r = sp * 16 + lane;
 #pragma unroll
-                for (int c0 = cg * (DK / NCG); c0 < (cg + 1) * (DK / NCG); c0 += 16) {
+                for (int c0 = cg * (DK / 2); c0 < (cg + 1) * (DK / 2); c0 += 16) {
                     float v[16];
                     tc::tmem_ld16(tW + lane_base + c0, v);
                     tc::tmem_ld_wait();
                     if (valid) {
-                        store_h8_global(Wg, tc::sw128_off(r, c0, C), v);
-                        store_h8_global(Wg, tc::sw128_off(r, c0 + 8, C), v + 8);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                        store_h8(Wg, tc::sw128_off(r, c0, C), v);
+                        store_h8(Wg, tc::sw128_off(r, c0 + 8, C), v + 8);
                     }
                 }
                 const bool vj = DV == 128 || lane < 16;
                 const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
 #pragma unroll
-                for (int c0 = cg * (C / NCG); c0 < (cg + 1) * (C / NCG); c0 += 16) {
+                for (int c0 = cg * (C / 2); c0 < (cg + 1) * (C / 2); c0 += 16) {
                     float v[16];
                     tc::tmem_ld16(tU + lane_base + c0, v);
                     tc::tmem_ld_wait();
                     if (vj) {
-                        store_h8_global(Ug, tc::sw128_off(jr, c0, DV), v);
-                        store_h8_global(Ug, tc::sw128_off(jr, c0 + 8, DV), v + 8);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                        store_h8(Ug, tc::sw128_off(jr, c0, DV), v);
+                        store_h8(Ug, tc::sw128_off(jr, c0 + 8, DV), v + 8);
                     }
                 }
             }
@@ -598,6 +648,7 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
         item = sm.next_item;
     }
     if (!ok && tid == 0) raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
+    report_f16_range(p.hdr, amax);
     if (tid == 0) tc::bulk_wait_read_all();
     tc::fence_before_sync();
     __syncthreads();

@@ -66,6 +66,13 @@ __device__ __forceinline__ void raise_error(int32_t* hdr, int bits) {
     if (hdr) atomicOr(reinterpret_cast<int*>(hdr) + kHdrError, bits);
 }
 
+// Largest finite fp16 magnitude.  The prefill rounds its tensor-core operands to fp16; a kernel keeps
+// the largest magnitude it rounded in a register (amax) and reports any above this bound once per warp.
+constexpr float kF16Max = 65504.0f;
+__device__ __forceinline__ void report_f16_range(int32_t* hdr, float amax) {
+    if (__any_sync(0xffffffffu, !(amax <= kF16Max)) && (threadIdx.x & 31) == 0) raise_error(hdr, GDN_DEVERR_FP16_RANGE);
+}
+
 // ---- launch argument blocks ----------------------------------------------
 
 struct DecodeArgs {
@@ -140,7 +147,8 @@ struct ExtendArgs {
     uint16_t* W;        // [max_chunks, HV, C*dk]    W = T diag(beta e^gamma) K, C rows x dk
     uint16_t* U;        // [max_chunks, HV, dv*C]    U^T = (T diag(beta) V)^T, dv rows x C
     uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, C rows x C
-    float4* GV;         // [max_chunks, HV, C]       per row: e^{gamma_r}, f_r = e^{gamma_n - gamma_r}
+    float4* GV;         // [max_chunks, HV, C]       gate vectors, each block of C float4 read as
+                        //                           float[4][C]: e^{gamma_r}, f_r = e^{gamma_n - gamma_r}
                         //                           (0 past the chunk end), gamma_r, e^{gamma_n}
 };
 
@@ -187,6 +195,15 @@ void mark_launch(cudaStream_t s, int i);
 int record_cuda_failure(cudaError_t e);
 
 size_t extend_workspace_bytes(const LayerDims& d, int max_N, int max_T, int* max_chunks_out);
+
+// Host checks of an extend call's arguments other than its workspace (configuration, parameters,
+// sizes, required pointers, alignment).  Returns GDN_OK or the GDN_ERR_* code gdn_extend returns for
+// them; *nothing is set when the batch is empty (N == 0 or T == 0), in which case the pointers are
+// not checked.
+int check_extend_args(const gdn_config_t* cfg, const gdn_params_t* params, const void* mixed_qkv, const void* a,
+                      const void* b, const int32_t* cu_seqlens, int32_t N, int32_t T, const int32_t* state_indices,
+                      const int32_t* has_initial_state, const void* conv_state, const float* ssm_state, int32_t P,
+                      const void* out, LayerDims* d, bool* nothing);
 void carve_extend_workspace(ExtendArgs& e, void* ws, int max_N, int max_T);
 
 cudaError_t launch_decode(const DecodeArgs& args, int dtype, cudaStream_t s);

@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
     const char* Wg = reinterpret_cast<const char*>(p.W + (id * d.HV + h) * (C * DK));
     const char* KQg = reinterpret_cast<const char*>(p.KQ + (id * d.HK + h / d.G) * (2 * C * DK));
     const char* Ug = reinterpret_cast<const char*>(p.U + (id * d.HV + h) * (DV * C));
-    const float4* gv = p.GV + (id * d.HV + h) * C;  // .z = gamma
+    const float* gam = reinterpret_cast<const float*>(p.GV + (id * d.HV + h) * C) + 2 * C;  // gamma
     auto h2f = [](const char* q) { return __half2float(*reinterpret_cast<const __half*>(q)); };
     for (int e = tid; e < DK * DVS / 4; e += 256) {
         const int f = e / (DVS / 4), j4 = e % (DVS / 4);
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
         Wf[e] = h2f(Wg + tc::sw128_off(sr, f, C));
         Kf[e] = h2f(KQg + tc::sw128_off(sr, f, 2 * C));
     }
-    if (tid < m) coef[tid] = expf(gv[m - 1].z - gv[tid].z);
+    if (tid < m) coef[tid] = expf(gam[m - 1] - gam[tid]);
     __syncthreads();
     for (int e = tid; e < m * DVS; e += 256) {  // v'_s[j] = u_s[j] - sum_f w_s[f] S_c[f][j]
         const int sr = e / DVS, jl = e % DVS;
@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
         Vp[e] = acc;
     }
     __syncthreads();
-    const float eg = expf(gv[m - 1].z);
+    const float eg = expf(gam[m - 1]);
     for (int e = tid; e < DK * DVS; e += 256) {
         const int f = e / DVS, jl = e % DVS;
         float acc = eg * Sc[e];

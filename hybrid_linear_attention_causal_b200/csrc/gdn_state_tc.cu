@@ -25,12 +25,14 @@
 //   - V' is formed in two halves of the chunk's rows, each released on its own
 //     barrier, so the state product issues its first k-steps meanwhile;
 //   - the output products run on the tensor core while the CUDA cores form V'
-//     and update the state; a chunk's outputs are read, scaled and staged while
-//     the next chunk's state product runs, and stored after its update.
-// A ninth warp only issues MMAs; a tenth issues every bulk copy, refilling
-// each double-buffered tile as soon as its last reader releases it.  The two
-// compute warps of a TMEM sub-partition share its 32 accumulator rows and
-// take one half of the columns each.
+//     and update the state; a chunk's outputs are read, scaled and staged once
+//     the next chunk's state update has released that chunk's X, and their
+//     accumulators are handed back to the next output products on a barrier.
+// A ninth warp only issues MMAs, from descriptors formed once per buffer; a
+// tenth issues every bulk copy, refilling each double-buffered tile as soon as
+// its last reader releases it and prefetching tiles into L2 a few chunks ahead.
+// The two compute warps of a TMEM sub-partition share its 32 accumulator rows
+// and take one half of the columns each.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -41,9 +43,9 @@ namespace {
 constexpr int C = kChunk;
 constexpr int NCW = 8;                  // compute warps
 constexpr int ISSUER = NCW * 32;        // lane 0 of the ninth warp
-constexpr int COPIER = (NCW + 1) * 32;  // lane 0 of the tenth warp
 constexpr int NT = (NCW + 2) * 32;
 constexpr int kCwBarrier = 1;           // named barrier of the compute warps
+constexpr int kPrefetchAhead = 4;       // chunks between a tile's L2 prefetch and its use
 
 // bf16 outputs are staged in shared memory and leave as 16-byte vectors; fp32 outputs (whose
 // staging tiles would not fit) are stored by each thread
@@ -61,11 +63,11 @@ struct StateSmem {
     uint16_t vt[DV * C];         // V'^T: A of Oq
     uint16_t vs[DV * C];         // Vs'^T: A of Snew
     T ostage[kStageOut<T> ? 2 : 1][kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV]
-    float4 gv[2][C];             // per row: e^{gamma_r}, f_r, gamma_r, e^{gamma_n}
-    float eg[2][C];              // e^{gamma_r} of the chunk whose outputs are pending
+    alignas(16) float gv[2][4][C];  // per row: e^{gamma_r}, f_r, gamma_r, e^{gamma_n} (a bulk-copy target)
+    alignas(16) float eg[2][C];     // e^{gamma_r} of the chunk whose outputs are pending
     unsigned long long full_kq[2], full_w[2], full_u[2], full_aq[2];
     unsigned long long free_kq[2], free_w[2], free_u[2], free_aq[2];
-    unsigned long long bar_x, bar_s, bar_o, bar_vp[2], bar_sa[2];
+    unsigned long long bar_x, bar_s, bar_o, bar_vp[2], bar_sa[2], out_free[2];
     uint32_t tmem_base;
 };
 
@@ -74,6 +76,9 @@ constexpr size_t state_smem_bytes() {
     return sizeof(StateSmem<T, DK, DV>) + 1024;  // + room to align the tiles on 1024 bytes
 }
 static_assert(state_smem_bytes<__nv_bfloat16, 128, 128>() <= 227 * 1024, "state pass shared memory");
+using StateSmemF32 = StateSmem<float, 64, 64>;
+static_assert(offsetof(StateSmemF32, gv) % 16 == 0 && offsetof(StateSmemF32, eg) % 16 == 0,
+              "bulk-copy and vector targets stay 16-byte aligned whatever the output type");
 static_assert(state_smem_bytes<float, 128, 128>() <= 227 * 1024, "state pass shared memory");
 
 // barrier among the compute warps; true when `pred` holds in all of them
@@ -131,27 +136,29 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     constexpr uint32_t KQ_BYTES = 2 * C * DK * 2, W_BYTES = C * DK * 2, U_BYTES = DV * C * 2, AQ_BYTES = C * C * 2,
                        GV_BYTES = C * 16;
     auto bar = [](unsigned long long& m) { return tc::smem_u32(&m); };
-    auto fetch_kq = [&](int id) {
+    auto src_kq = [&](int id) { return p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK); };
+    auto src_w = [&](int id) { return p.W + ((size_t)id * HV + h) * (C * DK); };
+    auto src_u = [&](int id) { return p.U + ((size_t)id * HV + h) * (DV * C); };
+    auto src_gv = [&](int id) { return p.GV + ((size_t)id * HV + h) * C; };
+    auto src_aq = [&](int id) { return p.AQ + ((size_t)id * HV + h) * (C * C); };
+    auto fetch = [&](int id) {  // every tile of chunk id into its buffers, on their "full" barriers
         const int bb = (id - c_begin) & 1;
         tc::mbar_expect_tx(bar(sm.full_kq[bb]), KQ_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.kq[bb]), p.KQ + ((size_t)id * d.HK + hk) * (2 * C * DK), KQ_BYTES,
-                     bar(sm.full_kq[bb]));
-    };
-    auto fetch_w = [&](int id) {
-        const int bb = (id - c_begin) & 1;
+        tc::bulk_g2s(tc::smem_u32(sm.kq[bb]), src_kq(id), KQ_BYTES, bar(sm.full_kq[bb]));
         tc::mbar_expect_tx(bar(sm.full_w[bb]), W_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.w[bb]), p.W + ((size_t)id * HV + h) * (C * DK), W_BYTES, bar(sm.full_w[bb]));
-    };
-    auto fetch_u = [&](int id) {
-        const int bb = (id - c_begin) & 1;
+        tc::bulk_g2s(tc::smem_u32(sm.w[bb]), src_w(id), W_BYTES, bar(sm.full_w[bb]));
         tc::mbar_expect_tx(bar(sm.full_u[bb]), U_BYTES + GV_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.ut[bb]), p.U + ((size_t)id * HV + h) * (DV * C), U_BYTES, bar(sm.full_u[bb]));
-        tc::bulk_g2s(tc::smem_u32(sm.gv[bb]), p.GV + ((size_t)id * HV + h) * C, GV_BYTES, bar(sm.full_u[bb]));
-    };
-    auto fetch_aq = [&](int id) {
-        const int bb = (id - c_begin) & 1;
+        tc::bulk_g2s(tc::smem_u32(sm.ut[bb]), src_u(id), U_BYTES, bar(sm.full_u[bb]));
+        tc::bulk_g2s(tc::smem_u32(sm.gv[bb]), src_gv(id), GV_BYTES, bar(sm.full_u[bb]));
         tc::mbar_expect_tx(bar(sm.full_aq[bb]), AQ_BYTES);
-        tc::bulk_g2s(tc::smem_u32(sm.aq[bb]), p.AQ + ((size_t)id * HV + h) * (C * C), AQ_BYTES, bar(sm.full_aq[bb]));
+        tc::bulk_g2s(tc::smem_u32(sm.aq[bb]), src_aq(id), AQ_BYTES, bar(sm.full_aq[bb]));
+    };
+    auto prefetch = [&](int id) {  // chunk id's tiles into L2
+        tc::bulk_prefetch_l2(src_kq(id), KQ_BYTES);
+        tc::bulk_prefetch_l2(src_w(id), W_BYTES);
+        tc::bulk_prefetch_l2(src_u(id), U_BYTES);
+        tc::bulk_prefetch_l2(src_gv(id), GV_BYTES);
+        tc::bulk_prefetch_l2(src_aq(id), AQ_BYTES);
     };
     if (warp == 0) tc::tmem_alloc(&sm.tmem_base, 512);
     if (tid == ISSUER) {
@@ -166,17 +173,14 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             tc::mbar_init(bar(sm.free_aq[bb]), NCW + 1);  // the output product's commit + every compute warp
             tc::mbar_init(bar(sm.bar_vp[bb]), NCW / 2);
             tc::mbar_init(bar(sm.bar_sa[bb]), NCW / 2);
+            tc::mbar_init(bar(sm.out_free[bb]), NCW);
         }
         tc::mbar_init(bar(sm.bar_x), 1);
         tc::mbar_init(bar(sm.bar_s), 1);
         tc::mbar_init(bar(sm.bar_o), 1);
         tc::fence_mbar_init();
-        for (int id = c_begin; id < c_end && id < c_begin + 2; ++id) {
-            fetch_kq(id);
-            fetch_w(id);
-            fetch_u(id);
-            fetch_aq(id);
-        }
+        for (int id = c_begin; id < c_end && id < c_begin + 2; ++id) fetch(id);
+        for (int id = c_begin + 2; id < c_end && id < c_begin + kPrefetchAhead; ++id) prefetch(id);
     }
 
     // compute warps: thread (sp, half, lane) owns row j of S^T, columns half * DK/2 .. + DK/2
@@ -231,14 +235,16 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 #pragma unroll
         for (int cc = 0; cc < C / 2; cc += 16) {
             const int c0 = half * (C / 2) + cc;
-            float oi[16], oq[16];
+            float oi[16], oq[16], eg[16];
             tc::tmem_ld16(tOi(bb) + lane_base + c0, oi);
             tc::tmem_ld16(tOq(bb) + lane_base + c0, oq);
+#pragma unroll
+            for (int q = 0; q < 16; q += 4) *reinterpret_cast<float4*>(eg + q) = *reinterpret_cast<const float4*>(&sm.eg[bb][c0 + q]);
             tc::tmem_ld_wait();
             if (rowv)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float o = fmaf(sm.eg[bb][c0 + i], oi[i], oq[i]);
+                    const float o = fmaf(eg[i], oi[i], oq[i]);
                     if constexpr (kStageOut<T>) sm.ostage[bb][(c0 + i) * DV + j] = from_f<T>(o);
                     else if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + j] = from_f<T>(o);
                 }
@@ -259,33 +265,57 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     bool ok = true;
     if (warp == NCW + 1) {
         // ---- the copier: each buffer is refilled for the chunk two ahead as soon as its readers have
-        // released it (W after X, [K ; Q] after the state product, U^T and the gate vectors once V'
-        // and the output scale have been formed, Aqk once its product and the outputs are done).
-        // The next release of a buffer needs the copy issued here, so none of these barriers can
-        // complete twice before this lane has seen the first.
+        // released it (W after X, U^T and the gate vectors once V' has been formed, [K ; Q] after the
+        // state product, Aqk once its product and the outputs are done).  The next release of a buffer
+        // needs the copy issued here, so none of these barriers can complete twice before this lane
+        // has seen the first.
         if (lane == 0) {
             for (int id = c_begin; id + 2 < c_end && ok; ++id) {
                 const int it = id - c_begin, bb = it & 1;
                 const uint32_t pb = (uint32_t)(it >> 1) & 1u;
+                if (id + kPrefetchAhead < c_end) prefetch(id + kPrefetchAhead);
+                const int nx = id + 2, nb = bb;  // the chunk two ahead lands in this chunk's buffers
                 ok = tc::mbar_wait(bar(sm.free_w[bb]), pb);
-                if (ok) fetch_w(id + 2);
+                if (ok) {
+                    tc::mbar_expect_tx(bar(sm.full_w[nb]), W_BYTES);
+                    tc::bulk_g2s(tc::smem_u32(sm.w[nb]), src_w(nx), W_BYTES, bar(sm.full_w[nb]));
+                }
                 if (ok) ok = tc::mbar_wait(bar(sm.free_u[bb]), pb);
-                if (ok) fetch_u(id + 2);
+                if (ok) {
+                    tc::mbar_expect_tx(bar(sm.full_u[nb]), U_BYTES + GV_BYTES);
+                    tc::bulk_g2s(tc::smem_u32(sm.ut[nb]), src_u(nx), U_BYTES, bar(sm.full_u[nb]));
+                    tc::bulk_g2s(tc::smem_u32(sm.gv[nb]), src_gv(nx), GV_BYTES, bar(sm.full_u[nb]));
+                }
                 if (ok) ok = tc::mbar_wait(bar(sm.free_kq[bb]), pb);
-                if (ok) fetch_kq(id + 2);
+                if (ok) {
+                    tc::mbar_expect_tx(bar(sm.full_kq[nb]), KQ_BYTES);
+                    tc::bulk_g2s(tc::smem_u32(sm.kq[nb]), src_kq(nx), KQ_BYTES, bar(sm.full_kq[nb]));
+                }
                 if (ok) ok = tc::mbar_wait(bar(sm.free_aq[bb]), pb);
-                if (ok) fetch_aq(id + 2);
+                if (ok) {
+                    tc::mbar_expect_tx(bar(sm.full_aq[nb]), AQ_BYTES);
+                    tc::bulk_g2s(tc::smem_u32(sm.aq[nb]), src_aq(nx), AQ_BYTES, bar(sm.full_aq[nb]));
+                }
             }
         }
     } else if (warp == NCW) {
-        // ---- the MMA issuer
+        // ---- the MMA issuer, from descriptors formed once per buffer and advanced by constant offsets
         if (lane == 0) {
+            // buffer 1's descriptors are buffer 0's advanced by the buffer stride
+            const uint64_t dW0 = tc::desc_sw128_k(tc::smem_u32(sm.w[0]), C, 0);
+            const uint64_t dQ0 = tc::desc_sw128_k(tc::smem_u32(sm.kq[0]) + C * 128, 2 * C, 0);  // Q: rows C .. 2C-1
+            const uint64_t dK0 = tc::desc_sw128_mn(tc::smem_u32(sm.kq[0]), 2 * C, 0);
+            const uint64_t dA0 = tc::desc_sw128_k(tc::smem_u32(sm.aq[0]), C, 0);
+            constexpr uint32_t kW1 = C * DK * 2, kKQ1 = 2 * C * DK * 2, kA1 = C * C * 2;
+            const uint64_t dVs = tc::desc_sw128_k(tc::smem_u32(sm.vs), DV, 0);
+            const uint64_t dVt = tc::desc_sw128_k(tc::smem_u32(sm.vt), DV, 0);
+            constexpr uint32_t ix = tc::idesc_f16(DV, 64), is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
             for (int id = c_begin; id < c_end && ok; ++id) {
                 const int it = id - c_begin, bb = it & 1;
                 const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
+                const uint64_t dWb = tc::desc_add(dW0, bb * kW1), dQb = tc::desc_add(dQ0, bb * kKQ1),
+                               dKb = tc::desc_add(dK0, bb * kKQ1), dAb = tc::desc_add(dA0, bb * kA1);
                 ok = tc::mbar_wait(bar(sm.full_w[bb]), pb) && tc::mbar_wait(bar(sm.full_kq[bb]), pb);
-                const uint32_t bw = tc::smem_u32(sm.w[bb]), bkq = tc::smem_u32(sm.kq[bb]);
-                constexpr uint32_t ix = tc::idesc_f16(DV, 64);
                 // X^T = S^T W^T, each half of S^T's columns as soon as the update has written it
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -294,18 +324,18 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     if (ok)
 #pragma unroll
                         for (int k = hh * (DK / 32); k < (hh + 1) * (DK / 32); ++k)
-                            tc::mma_f16_ta(tX, tA + 8 * k, tc::desc_sw128_k(bw, C, k), ix, k > 0);
+                            tc::mma_f16_ta(tX, tA + 8 * k, tc::desc_add(dWb, tc::sw128_kstep(C, k)), ix, k > 0);
                 }
                 if (!ok) break;
                 tc::mma_commit(bar(sm.bar_x));
                 tc::mma_commit(bar(sm.free_w[bb]));
-                // Oi^T = S^T Q^T (Q: rows C .. 2C-1 of the [K ; Q] tile)
+                // Oi^T = S^T Q^T, once the outputs two chunks back have left its accumulator
+                if (it >= 2) ok = tc::mbar_wait(bar(sm.out_free[bb]), (uint32_t)((it >> 1) - 1) & 1u);
+                if (!ok) break;
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k)
-                    tc::mma_f16_ta(tOi(bb), tA + 8 * k, tc::desc_sw128_k(bkq + C * 128, 2 * C, k), ix, k > 0);
+                    tc::mma_f16_ta(tOi(bb), tA + 8 * k, tc::desc_add(dQb, tc::sw128_kstep(2 * C, k)), ix, k > 0);
                 // Snew^T = Vs'^T K (K read MN-major), each half of the rows as soon as it is formed
-                const uint32_t bvs = tc::smem_u32(sm.vs), bvt = tc::smem_u32(sm.vt);
-                constexpr uint32_t is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     ok = tc::mbar_wait(bar(sm.bar_vp[hh]), ph);
@@ -313,7 +343,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     if (!ok) break;
 #pragma unroll
                     for (int k = 2 * hh; k < 2 * hh + 2; ++k)
-                        tc::mma_f16(tSn, tc::desc_sw128_k(bvs, DV, k), tc::desc_sw128_mn(bkq, 2 * C, k), is, k > 0);
+                        tc::mma_f16(tSn, tc::desc_add(dVs, tc::sw128_kstep(DV, k)), tc::desc_add(dKb, 2048u * k), is,
+                                    k > 0);
                 }
                 if (!ok) break;
                 tc::mma_commit(bar(sm.bar_s));
@@ -321,11 +352,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 // Oq^T = V'^T Aqk^T: queued behind the state product, off the chain
                 ok = tc::mbar_wait(bar(sm.full_aq[bb]), pb);
                 if (!ok) break;
-                constexpr uint32_t io = tc::idesc_f16(DV, 64);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    tc::mma_f16(tOq(bb), tc::desc_sw128_k(bvt, DV, k), tc::desc_sw128_k(tc::smem_u32(sm.aq[bb]), C, k),
-                                io, k > 0);
+                    tc::mma_f16(tOq(bb), tc::desc_add(dVt, tc::sw128_kstep(DV, k)),
+                                tc::desc_add(dAb, tc::sw128_kstep(C, k)), ix, k > 0);
                 tc::mma_commit(bar(sm.bar_o));
                 tc::mma_commit(bar(sm.free_aq[bb]));
             }
@@ -335,6 +365,12 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         // and the compute warps agree on the outcome at one barrier per chunk, so they stop together.
         int prev_t0 = 0, prev_n = 0;
         int4 chn = p.chunk_tab[c_begin];
+        float amax = 0.f;  // largest magnitude this thread rounded to fp16 among V', f V' and S's copy
+#pragma unroll
+        for (int i = 0; i < DK / 2; ++i) amax = fmaxf(amax, fabsf(s[i]));  // the starting state's copy
+        // row j's 16-byte chunk c of a swizzled DV x 64 tile (U^T, V'^T, Vs'^T)
+        const uint32_t jrow = (uint32_t)j * 128, jx = (uint32_t)(j & 7);
+        auto uoff = [&](int c) { return jrow + ((((uint32_t)c >> 3) ^ jx) << 4); };
         for (int id = c_begin; id < c_end; ++id) {
             const int it = id - c_begin, bb = it & 1;
             const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
@@ -355,31 +391,33 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 #pragma unroll
                 for (int cc = 0; cc < C / 2; cc += 16) {
                     const int c0 = half * (C / 2) + cc;
-                    float xv[16];
+                    float xv[16], f[16];
                     tc::tmem_ld16(tX + lane_base + c0, xv);
+#pragma unroll
+                    for (int q = 0; q < 16; q += 4) *reinterpret_cast<float4*>(f + q) = *reinterpret_cast<const float4*>(&sm.gv[bb][1][c0 + q]);
                     tc::tmem_ld_wait();
                     if (rowv)
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {  // 8 fp16 values per 16-byte vector
-                            const uint32_t off = tc::sw128_off(j, c0 + 8 * q, DV);
+                            const uint32_t off = uoff(c0 + 8 * q);
                             const uint4 u = *reinterpret_cast<const uint4*>(utb + off);
                             const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
                             uint32_t vw[4], sw[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const float2 uu = tc::unpack_f16(uw[e]);
-                                const int cl = c0 + 8 * q + 2 * e;
                                 const float v0 = uu.x - xv[8 * q + 2 * e], v1 = uu.y - xv[8 * q + 2 * e + 1];
+                                amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));  // |f| <= 1: covers f V' too
                                 vw[e] = tc::pack_f16(v0, v1);
-                                sw[e] = tc::pack_f16(v0 * sm.gv[bb][cl].y, v1 * sm.gv[bb][cl + 1].y);
+                                sw[e] = tc::pack_f16(v0 * f[8 * q + 2 * e], v1 * f[8 * q + 2 * e + 1]);
                             }
                             *reinterpret_cast<uint4*>(vtb + off) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
                             *reinterpret_cast<uint4*>(vsb + off) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
                         }
                 }
                 if (warp == 0 || warp == 4)  // the output scale of this chunk, for its outputs one chunk later
-                    sm.eg[bb][half * 32 + lane] = sm.gv[bb][half * 32 + lane].x;
-                egn = sm.gv[bb][0].w;  // e^{gamma_n}
+                    sm.eg[bb][half * 32 + lane] = sm.gv[bb][0][half * 32 + lane];
+                egn = sm.gv[bb][3][0];  // e^{gamma_n}
                 tc::fence_smem_to_async();
                 tc::fence_before_sync();
                 __syncwarp();
@@ -387,15 +425,6 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     tc::mbar_arrive(bar(sm.bar_vp[half]));
                     tc::mbar_arrive(bar(sm.free_u[bb]));
                 }
-            }
-            // the previous chunk's outputs, while the state product runs (their products completed before
-            // this chunk's X did: a commit covers every earlier product of the issuing thread)
-            if (okl && it > 0) {
-                tc::fence_after_sync();
-                put_out(it - 1, prev_t0, prev_n);
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(sm.free_aq[bb ^ 1]));
             }
             // S^T <- e^{gamma_n} S^T + Snew^T, and its fp16 copy for the next chunk, half by half
             if (okl) okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_s), ph));
@@ -409,13 +438,29 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     tc::tmem_ld16(tSn + lane_base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[cc + i] = fmaf(egn, s[cc + i], v[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        s[cc + i] = fmaf(egn, s[cc + i], v[i]);
+                        amax = fmaxf(amax, fabsf(s[cc + i]));
+                    }
                     put_sa32(tA_row + cc / 2, &s[cc]);
                 }
                 tc::tmem_st_wait();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
+            }
+            // the previous chunk's outputs, while the next chunk's X runs (their products completed before
+            // this chunk's X did: a commit covers every earlier product of the issuing thread); their
+            // accumulators and the Aqk buffer are then released
+            if (okl && it > 0) {
+                tc::fence_after_sync();
+                put_out(it - 1, prev_t0, prev_n);
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    tc::mbar_arrive(bar(sm.out_free[bb ^ 1]));
+                    tc::mbar_arrive(bar(sm.free_aq[bb ^ 1]));
+                }
             }
             ok = cw_and(okl);  // also orders the output scale and the staged outputs between the warps
             if (!ok) break;
@@ -431,7 +476,10 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 put_out(it, prev_t0, prev_n);
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(sm.free_aq[it & 1]));
+                if (lane == 0) {
+                    tc::mbar_arrive(bar(sm.out_free[it & 1]));
+                    tc::mbar_arrive(bar(sm.free_aq[it & 1]));
+                }
             }
             ok = cw_and(okl);
             if (ok) send_out(it, prev_t0, prev_n);
@@ -439,6 +487,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 #pragma unroll
                 for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
         }
+        if (!rowv) amax = 0.f;  // lanes past a 64-row tile hold no row
+        report_f16_range(p.hdr, amax);
     }
     ok = __syncthreads_and(ok);  // the chain, the issuer, the copier and the idle lanes agree
     if (!ok && tid == ISSUER) {

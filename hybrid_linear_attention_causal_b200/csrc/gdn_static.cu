@@ -54,12 +54,15 @@ extern "C" int gdn_extend_static_scratch(const gdn_config_t* cfg, const gdn_para
                                          const int32_t* state_indices, const int32_t* has_initial_state,
                                          void* conv_state, float* ssm_state, int32_t P, void* out,
                                          gdn_stream_t stream) {
-    if (N < 0 || T < 0) return GDN_ERR_INVALID_ARG;
-    const size_t need = gdn_extend_workspace_size(cfg, N, T);
-    if (need == 0)  // invalid configuration: let gdn_extend name the error
-        return gdn_extend(cfg, params, mixed_qkv, a, b, cu_seqlens, N, T, state_indices, has_initial_state,
-                          conv_state, ssm_state, P, out, nullptr, 0, stream);
-    if (need > (size_t)GDN_EXTEND_STATIC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    // every host-side check first, so that only a call that will launch kernels touches the shared array
+    gdn::LayerDims d;
+    bool nothing = false;
+    const int rc = gdn::check_extend_args(cfg, params, mixed_qkv, a, b, cu_seqlens, N, T, state_indices,
+                                          has_initial_state, conv_state, ssm_state, P, out, &d, &nothing);
+    if (rc != GDN_OK) return rc;
+    if (nothing) return GDN_OK;
+    if (gdn::extend_workspace_bytes(d, N, T, nullptr) > (size_t)GDN_EXTEND_STATIC_SCRATCH_BYTES)
+        return GDN_ERR_WORKSPACE;
     void* scratch = nullptr;
     cudaError_t e = scratch_address(&scratch);
     if (e == cudaSuccess)  // the header holds the chunk count and the error word: start from zero

@@ -93,6 +93,15 @@ __device__ __forceinline__ uint64_t desc_sw128_k(uint32_t base, int R, int s) {
     return make_desc_sw128(base + (uint32_t)(s >> 2) * (uint32_t)(R * 128) + (uint32_t)(s & 3) * 32, 16, 1024);
 }
 
+// A descriptor advanced by `bytes` (a multiple of 16): the start address is the low 14-bit field, in
+// 16-byte units, and shared-memory addresses stay below 256 KB, so the sum never carries out of it.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
+// byte offset of k-step `s` (16 fp16) inside a K-major swizzled tile with R rows (see desc_sw128_k)
+__host__ __device__ constexpr uint32_t sw128_kstep(int R, int s) {
+    return (uint32_t)(s >> 2) * (uint32_t)(R * 128) + (uint32_t)(s & 3) * 32;
+}
+
 // MN-major k-step `s` (16 rows along K) of a swizzled tile with R rows
 __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t base, int R, int s) {
     return make_desc_sw128(base + (uint32_t)s * 2048, (uint32_t)(R * 128), 1024);

@@ -34,9 +34,15 @@
  *
  * Conventions shared by all calls
  *   - Every pointer argument is DEVICE memory owned by the caller unless its
- *     comment says host.  The library allocates nothing and keeps no mutable
- *     global state; calls on different streams with disjoint outputs may run
- *     concurrently.
+ *     comment says host.  The library allocates no device memory.  The state
+ *     it does keep: per host thread and device, a second stream with its fork
+ *     and join events (created by that thread's first extend call on the
+ *     device, kept until the process exits; see gdn_extend); per host thread,
+ *     the profiling events set by gdn_set_launch_events; and, per device, the
+ *     one scratch array behind gdn_extend_static_scratch.  Calls on different
+ *     streams with disjoint outputs and workspaces may run concurrently, with
+ *     one exception: gdn_extend_static_scratch calls share that array, so
+ *     calls of it that overlap on the GPU race (see there).
  *   - Every call is asynchronous and stream-ordered on `stream` (a
  *     cudaStream_t; NULL is the legacy default stream).  No call synchronises
  *     the host, so decode and verify can be captured in a CUDA graph, and so
@@ -97,6 +103,8 @@ typedef struct CUstream_st* gdn_stream_t; /* same type as cudaStream_t */
 #define GDN_DEVERR_ACCEPT_RANGE 0x8 /* a commit's accepted count was outside 0..D; that request was skipped */
 #define GDN_DEVERR_CKPT_RANGE 0x10  /* a checkpoint boundary outside its sequence or a row >= num_ckpt; skipped */
 #define GDN_DEVERR_TREE 0x20        /* a draft tree parent outside -1 .. t-1; that request was treated as padded */
+#define GDN_DEVERR_FP16_RANGE 0x40  /* a prefill value staged as an fp16 tensor-core operand exceeded 65504 in
+                                       magnitude (see gdn_extend); that batch's results are invalid */
 
 /* element types */
 #define GDN_DTYPE_F32 0
@@ -123,8 +131,10 @@ typedef struct {
 
 /*
  * Workspace bytes for gdn_extend over at most max_N sequences and max_T
- * packed tokens (holds the chunk table and the fp32 intermediates of the
- * chunked prefill).  Returns 0 for an invalid configuration.
+ * packed tokens: the chunk table, and per chunk of 64 rows the fp16 tiles the
+ * per-chunk step hands the serial state pass ([K ; Q] per qk head; W, U^T and
+ * the decayed q.k per value head) plus a 16-byte fp32 gate vector per row and
+ * value head.  Returns 0 for an invalid configuration.
  */
 GDN_API size_t gdn_extend_workspace_size(const gdn_config_t* cfg, int32_t max_N, int32_t max_T);
 
@@ -204,8 +214,8 @@ GDN_API int gdn_extend_checkpoints(const gdn_config_t* cfg, const gdn_params_t* 
  * no allocating library routine.
  *   - Sizes whose gdn_extend_workspace_size(cfg, N, T) exceeds
  *     GDN_EXTEND_STATIC_SCRATCH_BYTES are rejected with GDN_ERR_WORKSPACE and
- *     nothing is launched (one sequence of up to 1151 tokens for the
- *     16/32-head, dk = dv = 128 layer; 9151 for the 4/8-head, 64 layer).
+ *     nothing is launched (one sequence of up to 2175 tokens for the
+ *     16/32-head, dk = dv = 128 layer; 15807 for the 4/8-head, 64 layer).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and keeps it, and,
  *     like gdn_extend, creates the library's second stream and its two
@@ -311,19 +321,37 @@ GDN_API int gdn_get_device_error(const void* workspace, int32_t* err_out, gdn_st
 GDN_API int gdn_reset_device_error(void* workspace, gdn_stream_t stream);
 
 /*
+ * Self-check of the failure path that keeps a stuck tensor-core kernel from
+ * hanging the GPU.  Every wait of the prefill and SSD kernels on an mbarrier
+ * phase (a tensor-core product, a bulk copy, another warp's hand-off) gives up
+ * after a time limit, raises GDN_DEVERR_TIMEOUT in the workspace error word,
+ * lets its copies in flight land and returns.  This call runs that same wait
+ * in a one-thread kernel on `stream`: on an mbarrier the kernel completes
+ * itself before waiting (arrive != 0: the wait succeeds at once) or that
+ * nothing ever completes (arrive == 0: the wait runs out after limit_ns
+ * nanoseconds, 0 < limit_ns <= 1e9, the bit is raised and the kernel
+ * returns).  Read the result with gdn_get_device_error.  The workspace is
+ * any buffer of at least 512 bytes (a decode workspace will do); the call is
+ * asynchronous.  GDN_ERR_INVALID_ARG for a limit outside that range or a
+ * null or misaligned workspace, GDN_ERR_WORKSPACE for one under 512 bytes.
+ */
+GDN_API int gdn_check_bounded_wait(int32_t arrive, int64_t limit_ns, void* workspace, size_t workspace_bytes,
+                                   gdn_stream_t stream);
+
+/*
  * Profiling aid (off by default).  With n > 0, the calling thread's later
  * gdn_extend / gdn_decode / gdn_verify / gdn_commit calls record events[i] (each a
  * cudaEvent_t created by the caller) at fixed points of the call; indices
  * >= n are not recorded.  n == 0 turns recording off.
  *   decode, verify, commit: 0 before the kernel, 1 after it (on `stream`).
  *   extend: on `stream`: 0 start, 1 after the chunk table, 2 after the
- *     conv + norm + gate pass, 3 after the conv-state update, 4 after the
- *     last intra-chunk segment, 5 end (second stream joined); on the
- *     library's second stream: 6 before the first and 7 after the last
- *     state-pass segment.  The batch is processed in segments of chunks
- *     (about one per 16384 packed rows, at most 16): the state pass of segment
- *     k runs on the second stream alongside the intra-chunk pass of segment
- *     k+1, so the two spans overlap.
+ *     last per-chunk segment (conv + SiLU, L2 norm, gates and the intra-chunk
+ *     products), 3 after the conv-state update, 5 end (second stream
+ *     joined); index 4 is not recorded; on the library's second stream: 6
+ *     before the first and 7 after the last state-pass segment.  The batch is
+ *     processed in segments of chunks (about one per 16384 packed rows, at
+ *     most 16): the state pass of segment k runs on the second stream
+ *     alongside the per-chunk step of segment k+1, so the two spans overlap.
  * Returns GDN_ERR_INVALID_ARG for n < 0, n > 16 or events == NULL with n > 0.
  */
 GDN_API int gdn_set_launch_events(void* const* events, int32_t n);

@@ -49,7 +49,11 @@ def test_workspace_sizes():
     small = gdn.gdn_extend_workspace_size(c, 1, 64)
     big = gdn.gdn_extend_workspace_size(c, 8, 32768)
     assert 0 < small < big
-    assert gdn.gdn_extend_workspace_size(c, 8, 32768) >= 32768 * (2 * 16 * 128 + 32 * 128) * 4
+    # every chunk of 64 rows holds the tiles the per-chunk step hands the state pass: fp16 [K ; Q] per qk
+    # head (128 x dk), and per value head fp16 W (64 x dk), U^T (dv x 64), Aqk (64 x 64) and a 16-byte
+    # gate vector per row
+    per_chunk = 16 * 128 * 128 * 2 + 32 * (64 * 128 * 2 + 128 * 64 * 2 + 64 * 64 * 2 + 64 * 16)
+    assert big >= (32768 // 64) * per_chunk
     assert gdn.gdn_decode_workspace_size(c, 256) == B.HEADER_BYTES
     assert gdn.gdn_verify_workspace_size(c, 256, 4) == B.HEADER_BYTES
     assert gdn.gdn_verify_workspace_size(c, 256, 17) == 0
@@ -232,3 +236,15 @@ def test_ssd_workload_recipe_is_seeded_and_shaped():
     assert w.T == 32768 and len(w.lengths) == 8 and all(512 <= n <= 16384 for n in w.lengths)
     none = W.ssd_case(spec, [4], seed=1, with_D=False, with_z=False, with_bias=False, init_random=False)
     assert none.D is None and none.z is None and none.dt_bias is None and none.init is None
+
+
+def test_bounded_wait_check_rejects_bad_arguments_before_launching():
+    """gdn_check_bounded_wait validates on the host (no GPU needed): the time limit must lie in
+    (0, 1e9] ns and the workspace must be a non-null, 16-byte aligned buffer of at least 512 bytes."""
+    L = B.lib()
+    assert L.gdn_check_bounded_wait(0, 0, FAKE, 512, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_check_bounded_wait(0, -5, FAKE, 512, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_check_bounded_wait(0, 1_000_000_001, FAKE, 512, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_check_bounded_wait(0, 1000, None, 512, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_check_bounded_wait(0, 1000, FAKE_MIS, 512, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_check_bounded_wait(0, 1000, FAKE, 256, None) == gdn.GDN_ERR_WORKSPACE

@@ -14,8 +14,7 @@ import torch
 import hybrid_linear_attention_causal_b200 as gdn
 from hybrid_linear_attention_causal_b200 import binding as B
 from hybrid_linear_attention_causal_b200 import workloads as W
-from tests.gpu_util import f64, gpu_extend, same_bits, to_device
-from tests.tolerances import assert_out_close, assert_state_close
+from tests.gpu_util import gpu_extend, same_bits, to_device
 
 
 def _static_call(wd):
@@ -37,17 +36,16 @@ def _static_call(wd):
 
 
 def _compare(wd, got, ref):
+    """The static path runs gdn_extend's kernels on the same (N, T), and extend is bit-reproducible, so
+    the outputs and every slot of both pools must match gdn_extend's bit for bit; a scratch array that
+    kept something stale from an earlier call would show here."""
     out, conv, ssm = got
     r_out, r_conv, r_ssm, err = ref
     assert err == 0
-    assert_out_close(f64(out), f64(r_out))
-    named = set(wd.state_indices.tolist())
+    assert same_bits(out, r_out), "outputs differ from gdn_extend's"
     for s in range(wd.P):
-        if s in named:
-            assert_state_close(f64(ssm[s]), f64(r_ssm[s]), what=f"slot {s}")
-        else:
-            assert same_bits(ssm[s], r_ssm[s])
-        assert same_bits(conv[s], r_conv[s])
+        assert same_bits(ssm[s], r_ssm[s]), f"ssm slot {s} differs from gdn_extend's"
+        assert same_bits(conv[s], r_conv[s]), f"conv slot {s} differs from gdn_extend's"
 
 
 @pytest.mark.gpu

@@ -17,7 +17,7 @@
 //   A   = beta_r e^{gamma_r-gamma_s} (k_r.k_s)        s < r   (strictly lower)
 //   Aqk = e^{gamma_r-gamma_s} (q_r.k_s)               s <= r
 //   T   = (I + A)^{-1}
-//   W   = T diag(beta e^gamma) K              (fp16 MMA, M=64 N=dk K=64; K read MN-major)
+//   W^T = K^T (T diag(beta e^gamma))^T        (fp16 MMA, M=dk N=64 K=64; K read MN-major)
 //   U^T = V^T (T diag(beta))^T                (fp16 MMA, M=dv N=64 K=64; V read MN-major)
 //
 // (the WY/UT form of the gated delta rule, Gated DeltaNet, Yang, Kautz and
@@ -25,18 +25,20 @@
 // four 16x16 diagonal blocks of I + A by forward substitution in fp32 on the
 // CUDA cores (D = their inverses, block diagonal), then, with L the strictly
 // block-lower part of A and E = D L (nilpotent: E^4 = 0),
-//   T = (I + E)^{-1} D = (I - E)(I + E^2) D
-// as four fp16 products on the tensor core (E, E^2, P = (I + E^2) D and
-// T = (I - E) P), each result rounded to fp16 once on its way back to shared
-// memory.  T's diagonal blocks are D itself and E's entries are L's scaled by
+//   T = (I + E)^{-1} D = (I + E^2)(I - E) D
+// in three rounds of fp16 products on the tensor core (E; E^2 and
+// Q = (I - E) D together; T = (I + E^2) Q), each result rounded to fp16 once
+// on its way back to shared memory.  T's diagonal blocks are D itself and E's entries are L's scaled by
 // D, so these roundings add nothing measurable to the fp16 rounding of
 // T diag(beta) that W and U need anyway.
 //
 // The item writes, as fp16 tiles in the tensor core's 128-byte swizzled
 // shared-memory layout (so the state pass copies them verbatim): [K ; Q] once
-// per (chunk, qk head), and per (chunk, value head) W, U^T and the masked
-// decayed q.k; plus a per-row gate vector in fp32.  Rows past the end of a
-// ragged chunk are zero in every tile.  One thread issues the MMAs; the eight
+// per (chunk, qk head), and per (chunk, value head) W^T, U^T and the masked
+// decayed q.k; plus a per-row gate vector in fp32.  The chunk's rows past the
+// end of a ragged chunk are zero in every tile.  The rows of the next value
+// head and of the next item are copied into shared memory asynchronously while
+// the current one computes.  One thread issues the MMAs; the eight
 // warps read their sub-partition's 32-lane slice of tensor memory (two warps
 // per slice, one group of columns each) for the CUDA-core steps.  Two CTAs
 // share an SM (half of its tensor memory and shared memory each), so one
@@ -53,7 +55,7 @@ namespace {
 constexpr int C = kChunk;
 constexpr int NT = 256;        // 8 warps; warp w reads TMEM sub-partition w % 4
 constexpr int kCtasPerSm = 2;
-constexpr uint32_t kTmemCols = 256;  // D1 (64 columns) + W (DK) + U^T (64), a half of tensor memory
+constexpr uint32_t kTmemCols = 256;  // D1, X1 / W^T, X2 / U^T: 64 columns each, a half of tensor memory
 constexpr int kItemsPerCta = 2;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 
@@ -63,8 +65,6 @@ struct ChunkShape {
     static constexpr int LDQK = 2 * DK + PADE;           // staged q,k row: k channels, then q channels
     static constexpr int LDV = DV + PADE;                // staged v row
     static constexpr size_t XQK = (size_t)(C + 3) * LDQK * sizeof(T);
-    static constexpr size_t XV = (size_t)(C + 3) * LDV * sizeof(T);
-    static constexpr size_t XMAX = XQK > XV ? XQK : XV;
 };
 
 template <typename T, int DK, int DV>
@@ -79,8 +79,9 @@ struct ChunkSmem {
                                   // finally T diag(beta) in D's and T diag(beta e^gamma) in I - E's
         float dg[4][16][20];      // the diagonal 16x16 blocks of A (fp32), rows padded
     };
-    static constexpr size_t UBYTES = S::XMAX > sizeof(Inv) ? S::XMAX : sizeof(Inv);
+    static constexpr size_t UBYTES = S::XQK > sizeof(Inv) ? S::XQK : sizeof(Inv);
     alignas(1024) unsigned char u[UBYTES];
+    alignas(16) T xv[(C + 3) * S::LDV];  // the staged v rows of one value head
     alignas(16) T wq[2 * DK * 4];  // conv taps of the item's k then q channels
     alignas(16) T wv[DV * 4];      // conv taps of the current value head's channels
     float2 gb[C];                  // (g, beta) of the current value head
@@ -204,10 +205,10 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = sm.tmem_base;
-    // D1: 64 columns; the inverse's accumulators X1, X2 (64 columns each, M = 64 layout) and then W
-    // (DK columns) at tm + 64; U^T (M = DV, 64 columns) at tm + 64 + DK
-    const uint32_t tD1 = tm, tX1 = tm + 64, tX2 = tm + 128, tW = tm + 64, tU = tm + 64 + DK;
-    static_assert(64 + DK + 64 <= (int)kTmemCols && 192 <= 64 + DK + 64, "tensor-memory layout");
+    // D1 at tm; the inverse's accumulators X1, X2 (M = 64 layout) at tm + 64 and tm + 128, then W^T
+    // (M = DK) and U^T (M = DV) in their places: 64 columns each
+    const uint32_t tD1 = tm, tX1 = tm + 64, tX2 = tm + 128, tW = tm + 64, tU = tm + 128;
+    static_assert(192 <= (int)kTmemCols, "tensor-memory layout");
     const int sp = warp & 3, cg = warp >> 2;  // TMEM sub-partition, column group
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     uint32_t ph_mma = 0;
@@ -233,59 +234,98 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
         }
     };
 
+    constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
+    // where an item's rows are: packed row t0 .. t0+n-1 of sequence seq, chunk cidx of it
+    struct Pos {
+        int id, hk, t0, n, cidx;
+        bool init;
+        const T* cs;  // the sequence's conv-state slot
+    };
+    auto pos_of = [&](int it) {
+        Pos q;
+        q.id = it / HK;
+        q.hk = it % HK;
+        const int4 ch = p.chunk_tab[q.id];
+        q.t0 = ch.y;
+        q.n = ch.z;
+        q.cidx = ch.w;
+        q.init = p.has_init ? p.has_init[ch.x] != 0 : true;
+        q.cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)p.slots[ch.x] * d.conv_dim * 3;
+        return q;
+    };
+    // Staging: packed rows t0-3 .. t0+n-1 of some channels into shared rows of stride `ld` (staged row i
+    // <-> packed row t0 - 3 + i), vector v (VE elements) of a row from global channel chan(v), by
+    // asynchronous 16-byte copies; for a sequence's first chunk the 3 rows before it come from the
+    // conv-state slot (channel-major there, so element by element, synchronously).
+    auto stage_rows = [&](T* dst, int ld, int vpr, const Pos& q, auto&& chan) {
+        const int r_lo = q.cidx > 0 ? 0 : 3;
+        const int nv = (q.n + 3 - r_lo) * vpr;
+        for (int e = tid; e < nv; e += NT) {
+            const int i = r_lo + e / vpr, v = e % vpr;
+            tc::cp_async16(dst + (size_t)i * ld + v * VE, x + (size_t)(q.t0 - 3 + i) * d.conv_dim + chan(v));
+        }
+        if (q.cidx == 0)
+            for (int e = tid; e < 3 * vpr * VE; e += NT) {
+                const int i = e / (vpr * VE), c = e % (vpr * VE);
+                dst[(size_t)i * ld + c] = q.init ? q.cs[(size_t)(chan(c / VE) + c % VE) * 3 + i] : from_f<T>(0.f);
+            }
+    };
+    // the q,k rows (columns k then q) and their taps
+    auto stage_qk = [&](const Pos& q) {
+        const int ck0 = d.HK * DK + q.hk * DK, cq0 = q.hk * DK;
+        constexpr int VPR = 2 * DK / VE, VK = DK / VE;
+        stage_rows(xs, S::LDQK, VPR, q, [&](int v) { return v < VK ? ck0 + v * VE : cq0 + (v - VK) * VE; });
+        constexpr int WV = DK * 4 / VE;  // vectors of one part's taps
+        for (int e = tid; e < 2 * WV; e += NT)
+            tc::cp_async16(sm.wq + (e < WV ? 0 : DK * 4) + (e % WV) * VE,
+                           w + (size_t)(e < WV ? ck0 : cq0) * 4 + (e % WV) * VE);
+    };
+    // value head h's rows and taps
+    auto stage_v = [&](const Pos& q, int h) {
+        const int cv0 = 2 * d.HK * DK + h * DV;
+        stage_rows(sm.xv, S::LDV, DV / VE, q, [&](int v) { return cv0 + v * VE; });
+        for (int e = tid; e < DV * 4 / VE; e += NT) tc::cp_async16(sm.wv + e * VE, w + (size_t)cv0 * 4 + e * VE);
+    };
+    // the raw gate inputs of value head h (threads NT-C .. NT-1, one row each), held in registers until
+    // commit_gates turns them into (g, beta) in shared memory
+    float ga = 0.f, gbv = 0.f;
+    auto load_gates = [&](const Pos& q, int h) {
+        if (tid >= NT - C) {
+            const int r = tid - (NT - C);
+            ga = gbv = 0.f;
+            if (r < q.n) {
+                const size_t row = (size_t)(q.t0 + r) * HV + h;
+                ga = to_f(reinterpret_cast<const T*>(p.a)[row]);
+                gbv = to_f(reinterpret_cast<const T*>(p.b)[row]);
+            }
+        }
+    };
+    auto commit_gates = [&](int n, int h) {  // zero past the end of the chunk
+        if (tid >= NT - C) {
+            const int r = tid - (NT - C);
+            sm.gb[r] = r < n ? make_float2(-expf(p.A_log[h]) * softplus_f(ga + p.dt_bias[h]), sigmoid_f(gbv))
+                             : make_float2(0.f, 0.f);
+        }
+    };
+    {
+        const Pos q = pos_of(item);
+        stage_qk(q);
+        stage_v(q, q.hk * G);
+        load_gates(q, q.hk * G);
+    }
+
     while (ok && item >= 0) {
         int nxt = -1;
         // At most kItemsPerCta items, then the CTA ends: its SM goes to whatever waits, first of all a
         // state-pass CTA of the previous segment (its stream has the higher priority).
         if (tid == 0 && ++done < kItemsPerCta) nxt = grab();
         if (tid == 0) sm.prefetch_item = nxt;  // read by every thread after the staging barrier
-        const int id = item / HK, hk = item % HK;
-        const int4 ch = p.chunk_tab[id];
-        const int seq = ch.x, t0 = ch.y, n = ch.z, cidx = ch.w;
-        const int slot = p.slots[seq];
-        const bool init = p.has_init ? p.has_init[seq] != 0 : true;
+        const Pos q = pos_of(item);
+        const int id = q.id, hk = q.hk, n = q.n;
         const int ck0 = d.HK * DK + hk * DK, cq0 = hk * DK;  // first k / q channel
-        const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
-        constexpr int VE = 16 / (int)sizeof(T);  // elements per 16-byte vector
-        // ---- stage the q,k rows (staged row i <-> packed row t0 - 3 + i; columns k then q) and taps
-        {
-            constexpr int VPR = 2 * DK / VE;  // vectors per staged row
-            const int nv = n * VPR;
-            for (int b0 = 0; b0 < nv; b0 += NT * 4) {
-                uint4 v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = b0 + u * NT + tid;
-                    if (e < nv) {
-                        const int r = e / VPR, c = (e % VPR) * VE;
-                        const int gc = c < DK ? ck0 + c : cq0 + (c - DK);
-                        v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + r) * d.conv_dim + gc);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = b0 + u * NT + tid;
-                    if (e < nv) {
-                        const int r = e / VPR, c = (e % VPR) * VE;
-                        *reinterpret_cast<uint4*>(xs + (size_t)(r + 3) * S::LDQK + c) = v[u];
-                    }
-                }
-            }
-            for (int e = tid; e < 3 * 2 * DK; e += NT) {
-                const int i = e / (2 * DK), c = e % (2 * DK);
-                const int gc = c < DK ? ck0 + c : cq0 + (c - DK);
-                T v;
-                if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + gc];
-                else v = init ? cs[(size_t)gc * 3 + i] : from_f<T>(0.f);
-                xs[(size_t)i * S::LDQK + c] = v;
-            }
-            constexpr int WV = DK * 4 / VE;  // vectors of one part's taps
-            for (int e = tid; e < 2 * WV; e += NT) {
-                const int c0 = e < WV ? ck0 : cq0, o = (e % WV) * VE;
-                *reinterpret_cast<uint4*>(sm.wq + (e < WV ? 0 : DK * 4) + o) =
-                    *reinterpret_cast<const uint4*>(w + (size_t)c0 * 4 + o);
-            }
-        }
+        // the item's rows and the first value head's, staged by the copies issued before
+        commit_gates(n, hk * G);
+        tc::cp_async_wait_all();
         __syncthreads();
         {  // the next item's rows into L2 while this one computes: one 128-byte line per prefetch, spread
            // over every thread (its q, k and v pieces of each row: 2 DK + G DV elements)
@@ -350,47 +390,6 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
             const int h = hk * G + j;
             const size_t ch_h = (size_t)id * HV + h;
             const int cv0 = 2 * d.HK * DK + h * DV;  // first v channel of this head
-            // ---- stage this value head's v rows and taps (the q,k rows are no longer needed), and gates
-            {
-                constexpr int VPR = DV / VE;
-                const int nv = n * VPR;
-                for (int b0 = 0; b0 < nv; b0 += NT * 4) {
-                    uint4 v[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = b0 + u * NT + tid;
-                        if (e < nv)
-                            v[u] = *reinterpret_cast<const uint4*>(x + (size_t)(t0 + e / VPR) * d.conv_dim + cv0 +
-                                                                   (e % VPR) * VE);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = b0 + u * NT + tid;
-                        if (e < nv) *reinterpret_cast<uint4*>(xs + (size_t)(e / VPR + 3) * S::LDV + (e % VPR) * VE) = v[u];
-                    }
-                }
-                for (int e = tid; e < 3 * DV; e += NT) {
-                    const int i = e / DV, c = e % DV;
-                    T v;
-                    if (cidx > 0) v = x[(size_t)(t0 - 3 + i) * d.conv_dim + cv0 + c];
-                    else v = init ? cs[(size_t)(cv0 + c) * 3 + i] : from_f<T>(0.f);
-                    xs[(size_t)i * S::LDV + c] = v;
-                }
-                for (int e = tid; e < DV * 4 / VE; e += NT)
-                    *reinterpret_cast<uint4*>(sm.wv + e * VE) = *reinterpret_cast<const uint4*>(w + (size_t)cv0 * 4 + e * VE);
-                if (tid >= NT - C) {  // gates of the chunk's rows (zero past the end)
-                    const int r = tid - (NT - C);
-                    float2 gb = make_float2(0.f, 0.f);
-                    if (r < n) {
-                        const size_t row = (size_t)(t0 + r) * HV + h;
-                        const float av = to_f(reinterpret_cast<const T*>(p.a)[row]);
-                        const float bv2 = to_f(reinterpret_cast<const T*>(p.b)[row]);
-                        gb = make_float2(-expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]), sigmoid_f(bv2));
-                    }
-                    sm.gb[r] = gb;
-                }
-            }
-            __syncthreads();
             // ---- V rows (conv + SiLU) into the V tile: a task is 8 rows of DV / 4 lanes; warp 0 also
             // scans the gates
             {
@@ -400,7 +399,7 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 for (int task = warp * VPW + lane / LPV; task < C / 8; task += 8 * VPW) {
                     const int r0 = 8 * task;
                     float y[8][4];
-                    conv8x4(xs + 4 * l, S::LDV, sm.wv + 16 * l, cbias ? cbias + cv0 + 4 * l : nullptr, r0, n, y);
+                    conv8x4(sm.xv + 4 * l, S::LDV, sm.wv + 16 * l, cbias ? cbias + cv0 + 4 * l : nullptr, r0, n, y);
 #pragma unroll
                     for (int o = 0; o < 8; ++o) {
 #pragma unroll
@@ -435,6 +434,10 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 __syncthreads();
             }
             if (!ok) break;
+            if (j + 1 < G) {  // the next value head's rows, taps and gates, while this one computes
+                stage_v(q, h + 1);
+                load_gates(q, h + 1);
+            }
             // ---- from D1: A's diagonal 16x16 blocks (fp32) and its strictly block-lower part L (fp16 tile
             // 1) from the k.k rows (sub-partitions 0-1), the masked decayed q.k tile straight to global
             // memory from the q.k rows (2-3); the warps of a sub-partition take one group of 32 columns
@@ -445,38 +448,40 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 char* Lt = tile_b(1);
                 const int r = (sp & 1) * 32 + lane;
                 const bool qrow = sp >= 2;
+                float v[32];
+                const bool live0 = 32 * cg <= (sp & 1) * 32 + 31, live1 = 32 * cg + 16 <= (sp & 1) * 32 + 31;
+                if (live0) tc::tmem_ld16(tD1 + lane_base + 32 * cg, *reinterpret_cast<float(*)[16]>(v));
+                if (live1) tc::tmem_ld16(tD1 + lane_base + 32 * cg + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+                tc::tmem_ld_wait();
+                const float gr = sm.gam2[r];
+                const float br = qrow ? 1.f : sm.beta[r];
 #pragma unroll
-                for (int c0 = 32 * cg; c0 < 32 * cg + 32; c0 += 16) {
-                    const bool live = c0 <= (sp & 1) * 32 + 31;  // warp-uniform
-                    float v[16], e[16];
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c0 = 32 * cg + 16 * hh;
+                    const bool live = hh == 0 ? live0 : live1;  // warp-uniform
+                    float e[16];
                     if (live) {
-                        tc::tmem_ld16(tD1 + lane_base + c0, v);
-                        tc::tmem_ld_wait();
                         const int lim = r < n ? r - c0 + (qrow ? 1 : 0) : 0;
-                        const float gr = sm.gam2[r];
 #pragma unroll
-                        for (int q = 0; q < 16; q += 4) {
-                            const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[c0 + q]);
+                        for (int qq = 0; qq < 16; qq += 4) {
+                            const float4 gs = *reinterpret_cast<const float4*>(&sm.gam2[c0 + qq]);
                             const float gq[4] = {gs.x, gs.y, gs.z, gs.w};
 #pragma unroll
                             for (int u = 0; u < 4; ++u)
-                                e[q + u] = q + u < lim ? gr - gq[u] : __int_as_float(0xff800000u);  // -inf
+                                e[qq + u] = qq + u < lim ? gr - gq[u] : __int_as_float(0xff800000u);  // -inf
                         }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) e[i] = tc::ex2_approx(e[i]) * v[i];
+                        for (int i = 0; i < 16; ++i) e[i] = tc::ex2_approx(e[i]) * v[16 * hh + i] * br;
                     } else {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) e[i] = 0.f;
                     }
                     if (!qrow) {
-                        const float br = sm.beta[r];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) e[i] *= br;
                         if (c0 == 16 * (r >> 4)) {  // the diagonal block: fp32, and zeros in L
 #pragma unroll
-                            for (int q = 0; q < 16; q += 4)
-                                *reinterpret_cast<float4*>(&inv.dg[r >> 4][r & 15][q]) =
-                                    make_float4(e[q], e[q + 1], e[q + 2], e[q + 3]);
+                            for (int qq = 0; qq < 16; qq += 4)
+                                *reinterpret_cast<float4*>(&inv.dg[r >> 4][r & 15][qq]) =
+                                    make_float4(e[qq], e[qq + 1], e[qq + 2], e[qq + 3]);
 #pragma unroll
                             for (int i = 0; i < 16; ++i) e[i] = 0.f;
                         }
@@ -489,6 +494,7 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 }
             }
             __syncthreads();
+            if (j + 1 < G) commit_gates(n, h + 1);  // the scan of this head's gates is done
             // ---- D = the inverses of A's diagonal 16x16 blocks, by forward substitution in fp32 (warps
             // 0-1: lane (block, column c), t_r = [r == c] - sum_{s<r} A_rs t_s), into fp16 tile 0, whose
             // other blocks warps 2-7 clear; warps 4-5 also write the state pass's gate vectors
@@ -531,17 +537,14 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
             tc::fence_before_sync();
             __syncthreads();
             tc::fence_after_sync();
-            // ---- T = (I - E)(I + E^2) D with E = D L: four fp16 products, each result rounded once
+            // ---- T = (I + E)^{-1} D = (I + E^2)(I - E) D with E = D L, in three rounds of fp16 products
+            // (E; then E^2 and (I - E) D together; then T), each result rounded once
             constexpr uint32_t i64 = tc::idesc_f16(64, 64) | tc::kTransposeB;
-            // issue a 64 x 64 x 64 product of tile `a` (K-major) and tile `b` (read MN-major) into `acc`
-            auto product = [&](uint32_t acc, int a, int b) {
-                if (tid == 0) {
+            // a 64 x 64 x 64 product of tile `a` (K-major) and tile `b` (read MN-major) into `acc` (thread 0)
+            auto issue = [&](uint32_t acc, int a, int b) {
 #pragma unroll
-                    for (int s = 0; s < C / 16; ++s)
-                        tc::mma_f16(acc, tc::desc_sw128_k(tile_s(a), C, s), tc::desc_sw128_mn(tile_s(b), C, s), i64, s > 0);
-                    tc::mma_commit(bar);
-                }
-                return wait_mma();
+                for (int s = 0; s < C / 16; ++s)
+                    tc::mma_f16(acc, tc::desc_sw128_k(tile_s(a), C, s), tc::desc_sw128_mn(tile_s(b), C, s), i64, s > 0);
             };
             auto publish = [&]() {  // the tiles written above are complete and visible to the tensor core
                 tc::fence_smem_to_async();
@@ -549,7 +552,11 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 __syncthreads();
                 tc::fence_after_sync();
             };
-            if (!(ok = product(tX1, 0, 1))) break;  // E = D L
+            if (tid == 0) {  // E = D L
+                issue(tX1, 0, 1);
+                tc::mma_commit(bar);
+            }
+            if (!(ok = wait_mma())) break;
             read64(tX1, [&](int m, int c0, const float* v) {  // E -> tile 2, I - E -> tile 3
                 float ne[16];
 #pragma unroll
@@ -560,7 +567,12 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 store_h8(tile_b(3), tc::sw128_off(m, c0 + 8, C), ne + 8);
             });
             publish();
-            if (!(ok = product(tX2, 2, 2))) break;  // E^2 = E E
+            if (tid == 0) {  // E^2 = E E and Q = (I - E) D
+                issue(tX2, 2, 2);
+                issue(tX1, 3, 0);
+                tc::mma_commit(bar);
+            }
+            if (!(ok = wait_mma())) break;
             read64(tX2, [&](int m, int c0, const float* v) {  // I + E^2 -> tile 1 (L is no longer needed)
                 float pe[16];
 #pragma unroll
@@ -568,14 +580,16 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 store_h8(tile_b(1), tc::sw128_off(m, c0, C), pe);
                 store_h8(tile_b(1), tc::sw128_off(m, c0 + 8, C), pe + 8);
             });
-            publish();
-            if (!(ok = product(tX1, 1, 0))) break;  // P = (I + E^2) D
-            read64(tX1, [&](int m, int c0, const float* v) {  // P -> tile 2 (E is no longer needed)
+            read64(tX1, [&](int m, int c0, const float* v) {  // Q -> tile 2 (E is no longer needed)
                 store_h8(tile_b(2), tc::sw128_off(m, c0, C), v);
                 store_h8(tile_b(2), tc::sw128_off(m, c0 + 8, C), v + 8);
             });
             publish();
-            if (!(ok = product(tX2, 3, 2))) break;  // T = (I - E) P
+            if (tid == 0) {  // T = (I + E^2) Q
+                issue(tX2, 1, 2);
+                tc::mma_commit(bar);
+            }
+            if (!(ok = wait_mma())) break;
             read64(tX2, [&](int m, int c0, const float* v) {  // T diag(beta) -> tile 0, T diag(beta e^gamma) -> 3
                 float tb[16], te[16];
 #pragma unroll
@@ -590,54 +604,55 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                 store_h8(tile_b(3), tc::sw128_off(m, c0 + 8, C), te + 8);
             });
             publish();
-            if (tid == 0) {  // W = (T diag(beta e^gamma)) K (M = 64, K read MN-major from the [K ; Q] tile),
-                             // U^T = V^T (T diag(beta))^T (M = DV, V read MN-major)
+            if (tid == 0) {  // W^T = K^T (T diag(beta e^gamma))^T (M = DK, K read MN-major from the [K ; Q]
+                             // tile), U^T = V^T (T diag(beta))^T (M = DV, V read MN-major)
                 const uint32_t bkq = tc::smem_u32(sm.kq), bvr = tc::smem_u32(sm.vr);
-                constexpr uint32_t iw = tc::idesc_f16(64, DK) | tc::kTransposeB;
+                constexpr uint32_t iw = tc::idesc_f16(DK, 64) | tc::kTransposeA;
                 constexpr uint32_t iu = tc::idesc_f16(DV, 64) | tc::kTransposeA;
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    tc::mma_f16(tW, tc::desc_sw128_k(tile_s(3), C, s), tc::desc_sw128_mn(bkq, 2 * C, s), iw, s > 0);
+                    tc::mma_f16(tW, tc::desc_sw128_mn(bkq, 2 * C, s), tc::desc_sw128_k(tile_s(3), C, s), iw, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
                     tc::mma_f16(tU, tc::desc_sw128_mn(bvr, C, s), tc::desc_sw128_k(tile_s(0), C, s), iu, s > 0);
                 tc::mma_commit(bar);
             }
             if (!(ok = wait_mma())) break;
-            {  // W rows -> the W tile; U -> the U^T tile (both fp16, swizzled, straight to global memory).
-               // M = 64 layout: lanes 0-15 of sub-partition sp hold rows 16 sp .. 16 sp + 15; the warps
-               // of a sub-partition take one group of columns each
+            if (j + 1 == G && sm.prefetch_item >= 0) {
+                // the next item's rows (into the staging space, which the inverse's tiles have just left)
+                // and its first value head's, while this head's W and U leave
+                const Pos qn = pos_of(sm.prefetch_item);
+                stage_qk(qn);
+                stage_v(qn, qn.hk * G);
+                load_gates(qn, qn.hk * G);
+            }
+            {  // W^T and U^T -> their tiles (fp16, swizzled, straight to global memory).  A row per lane
+               // (M = 64: lanes 0-15 of each sub-partition); the warps of a sub-partition take one group of
+               // 32 columns each
                 char* Wg = reinterpret_cast<char*>(p.W + ch_h * (C * DK));
                 char* Ug = reinterpret_cast<char*>(p.U + ch_h * (DV * C));
-                const bool valid = lane < 16;
-                const int r = sp * 16 + lane;
+                float wv_[32], uv[32];
+                tc::tmem_ld16(tW + lane_base + 32 * cg, *reinterpret_cast<float(*)[16]>(wv_));
+                tc::tmem_ld16(tW + lane_base + 32 * cg + 16, *reinterpret_cast<float(*)[16]>(wv_ + 16));
+                tc::tmem_ld16(tU + lane_base + 32 * cg, *reinterpret_cast<float(*)[16]>(uv));
+                tc::tmem_ld16(tU + lane_base + 32 * cg + 16, *reinterpret_cast<float(*)[16]>(uv + 16));
+                tc::tmem_ld_wait();
+                if (DK == 128 || lane < 16) {
+                    const int ir = DK == 128 ? sp * 32 + lane : sp * 16 + lane;
 #pragma unroll
-                for (int c0 = cg * (DK / 2); c0 < (cg + 1) * (DK / 2); c0 += 16) {
-                    float v[16];
-                    tc::tmem_ld16(tW + lane_base + c0, v);
-                    tc::tmem_ld_wait();
-                    if (valid) {
+                    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(wv_[i]));
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                        store_h8(Wg, tc::sw128_off(r, c0, C), v);
-                        store_h8(Wg, tc::sw128_off(r, c0 + 8, C), v + 8);
-                    }
+                    for (int c8 = 0; c8 < 4; ++c8) store_h8(Wg, tc::sw128_off(ir, 32 * cg + 8 * c8, DK), wv_ + 8 * c8);
                 }
-                const bool vj = DV == 128 || lane < 16;
-                const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
+                if (DV == 128 || lane < 16) {
+                    const int jr = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
 #pragma unroll
-                for (int c0 = cg * (C / 2); c0 < (cg + 1) * (C / 2); c0 += 16) {
-                    float v[16];
-                    tc::tmem_ld16(tU + lane_base + c0, v);
-                    tc::tmem_ld_wait();
-                    if (vj) {
+                    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(uv[i]));
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                        store_h8(Ug, tc::sw128_off(jr, c0, DV), v);
-                        store_h8(Ug, tc::sw128_off(jr, c0 + 8, DV), v + 8);
-                    }
+                    for (int c8 = 0; c8 < 4; ++c8) store_h8(Ug, tc::sw128_off(jr, 32 * cg + 8 * c8, DV), uv + 8 * c8);
                 }
             }
+            if (j + 1 < G) tc::cp_async_wait_all();  // the next value head's rows
             tc::fence_before_sync();
             __syncthreads();  // tensor memory and the staging space are free for the next head
             tc::fence_after_sync();

@@ -144,7 +144,7 @@ struct ExtendArgs {
     // 128-byte swizzled shared-memory layout, so the state pass copies them verbatim.  Rows past the
     // end of a ragged chunk are zero.
     uint16_t* KQ;       // [max_chunks, HK, 2*C*dk]  [K ; Q*scale] (L2-normalised), 128 rows x dk
-    uint16_t* W;        // [max_chunks, HV, C*dk]    W = T diag(beta e^gamma) K, C rows x dk
+    uint16_t* W;        // [max_chunks, HV, dk*C]    W^T, W = T diag(beta e^gamma) K: dk rows x C
     uint16_t* U;        // [max_chunks, HV, dv*C]    U^T = (T diag(beta) V)^T, dv rows x C
     uint16_t* AQ;       // [max_chunks, HV, C*C]     masked decayed q.k, C rows x C
     float4* GV;         // [max_chunks, HV, C]       gate vectors, each block of C float4 read as

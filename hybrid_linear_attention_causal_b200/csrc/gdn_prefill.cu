@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(256) ckpt_finish_kernel(ExtendArgs p) {
     }
     for (int e = tid; e < m * DK; e += 256) {
         const int sr = e / DK, f = e % DK;
-        Wf[e] = h2f(Wg + tc::sw128_off(sr, f, C));
+        Wf[e] = h2f(Wg + tc::sw128_off(f, sr, DK));  // the tile holds W^T
         Kf[e] = h2f(KQg + tc::sw128_off(sr, f, 2 * C));
     }
     if (tid < m) coef[tid] = expf(gam[m - 1] - gam[tid]);

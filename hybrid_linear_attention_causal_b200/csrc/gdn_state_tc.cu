@@ -4,7 +4,7 @@
 // One CTA per (sequence, value head), looping over the sequence's chunks.  The
 // products are formed transposed, with the value dimension (dv) as the MMA's
 // M, so that every accumulator row belongs to one thread.  Per chunk, from the
-// tiles the per-chunk step wrote ([K ; Q], W, U^T, Aqk and the gate vectors):
+// tiles the per-chunk step wrote ([K ; Q], W^T, U^T, Aqk and the gate vectors):
 //
 //   X^T     = S^T W^T                       M=dv N=64 K=dk   (on the chain)
 //   Oi^T    = S^T Q^T                       M=dv N=64 K=dk   (off the chain)
@@ -57,7 +57,7 @@ struct StateSmem {
     // fp16 operand tiles in the 128-byte swizzled layout (1024-byte aligned), double-buffered and
     // copied two chunks ahead
     uint16_t kq[2][2 * C * DK];  // [K ; Q]: K rows (MN-major B of Snew), Q rows (B of Oi)
-    uint16_t w[2][C * DK];       // W (B of X)
+    uint16_t w[2][C * DK];       // W^T (B of X, read MN-major)
     uint16_t ut[2][DV * C];      // U^T
     uint16_t aq[2][C * C];       // Aqk (B of Oq)
     uint16_t vt[DV * C];         // V'^T: A of Oq
@@ -302,14 +302,15 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         // ---- the MMA issuer, from descriptors formed once per buffer and advanced by constant offsets
         if (lane == 0) {
             // buffer 1's descriptors are buffer 0's advanced by the buffer stride
-            const uint64_t dW0 = tc::desc_sw128_k(tc::smem_u32(sm.w[0]), C, 0);
+            const uint64_t dW0 = tc::desc_sw128_mn(tc::smem_u32(sm.w[0]), DK, 0);  // W^T, read MN-major
             const uint64_t dQ0 = tc::desc_sw128_k(tc::smem_u32(sm.kq[0]) + C * 128, 2 * C, 0);  // Q: rows C .. 2C-1
             const uint64_t dK0 = tc::desc_sw128_mn(tc::smem_u32(sm.kq[0]), 2 * C, 0);
             const uint64_t dA0 = tc::desc_sw128_k(tc::smem_u32(sm.aq[0]), C, 0);
             constexpr uint32_t kW1 = C * DK * 2, kKQ1 = 2 * C * DK * 2, kA1 = C * C * 2;
             const uint64_t dVs = tc::desc_sw128_k(tc::smem_u32(sm.vs), DV, 0);
             const uint64_t dVt = tc::desc_sw128_k(tc::smem_u32(sm.vt), DV, 0);
-            constexpr uint32_t ix = tc::idesc_f16(DV, 64), is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
+            constexpr uint32_t ix = tc::idesc_f16(DV, 64), ixw = ix | tc::kTransposeB,
+                               is = tc::idesc_f16(DV, DK) | tc::kTransposeB;
             for (int id = c_begin; id < c_end && ok; ++id) {
                 const int it = id - c_begin, bb = it & 1;
                 const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     if (ok)
 #pragma unroll
                         for (int k = hh * (DK / 32); k < (hh + 1) * (DK / 32); ++k)
-                            tc::mma_f16_ta(tX, tA + 8 * k, tc::desc_add(dWb, tc::sw128_kstep(C, k)), ix, k > 0);
+                            tc::mma_f16_ta(tX, tA + 8 * k, tc::desc_add(dWb, 2048u * k), ixw, k > 0);
                 }
                 if (!ok) break;
                 tc::mma_commit(bar(sm.bar_x));

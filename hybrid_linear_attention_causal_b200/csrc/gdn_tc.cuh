@@ -292,6 +292,13 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // Waits until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// Per-thread asynchronous 16-byte copy global -> shared (both 16-byte aligned), cached in L2 only;
+// cp_async_wait_all waits for every such copy this thread issued.
+__device__ __forceinline__ void cp_async16(const void* sdst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // One non-blocking test of the phase with parity `parity` of the mbarrier.
 __device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
     uint32_t done = 0;

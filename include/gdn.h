@@ -132,7 +132,7 @@ typedef struct {
 /*
  * Workspace bytes for gdn_extend over at most max_N sequences and max_T
  * packed tokens: the chunk table, and per chunk of 64 rows the fp16 tiles the
- * per-chunk step hands the serial state pass ([K ; Q] per qk head; W, U^T and
+ * per-chunk step hands the serial state pass ([K ; Q] per qk head; W^T, U^T and
  * the decayed q.k per value head) plus a 16-byte fp32 gate vector per row and
  * value head.  Returns 0 for an invalid configuration.
  */

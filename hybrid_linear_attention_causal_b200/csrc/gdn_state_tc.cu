@@ -25,9 +25,10 @@
 //   - V' is formed in two halves of the chunk's rows, each released on its own
 //     barrier, so the state product issues its first k-steps meanwhile;
 //   - the output products run on the tensor core while the CUDA cores form V'
-//     and update the state; a chunk's outputs are read, scaled and staged once
-//     the next chunk's state update has released that chunk's X, and their
-//     accumulators are handed back to the next output products on a barrier.
+//     and update the state, and four output warps (one per TMEM
+//     sub-partition) read, scale, stage and store each chunk's outputs once
+//     its products complete, handing the accumulators back to the next output
+//     products on a barrier, so no output work sits on the chain.
 // A ninth warp only issues MMAs, from descriptors formed once per buffer; a
 // tenth issues every bulk copy, refilling each double-buffered tile as soon as
 // its last reader releases it and prefetching tiles into L2 a few chunks ahead.
@@ -41,10 +42,13 @@ namespace gdn {
 namespace {
 
 constexpr int C = kChunk;
-constexpr int NCW = 8;                  // compute warps
+constexpr int NCW = 8;                  // compute warps 0-7
 constexpr int ISSUER = NCW * 32;        // lane 0 of the ninth warp
-constexpr int NT = (NCW + 2) * 32;
+constexpr int OW0 = NCW + 2;            // output warps OW0 .. OW0 + NOW - 1
+constexpr int NOW = 4;
+constexpr int NT = (OW0 + NOW) * 32;
 constexpr int kCwBarrier = 1;           // named barrier of the compute warps
+constexpr int kOwBarrier = 2;           // named barrier of the output warps
 constexpr int kPrefetchAhead = 4;       // chunks between a tile's L2 prefetch and its use
 
 // bf16 outputs are staged in shared memory and leave as 16-byte vectors; fp32 outputs (whose
@@ -64,10 +68,10 @@ struct StateSmem {
     uint16_t vs[DV * C];         // Vs'^T: A of Snew
     T ostage[kStageOut<T> ? 2 : 1][kStageOut<T> ? C * DV : 1];  // a chunk's outputs O [C][DV]
     alignas(16) float gv[2][4][C];  // per row: e^{gamma_r}, f_r, gamma_r, e^{gamma_n} (a bulk-copy target)
-    alignas(16) float eg[2][C];     // e^{gamma_r} of the chunk whose outputs are pending
+    alignas(16) float eg[2][C];     // e^{gamma_r} of a chunk, the output warps' copy
     unsigned long long full_kq[2], full_w[2], full_u[2], full_aq[2];
     unsigned long long free_kq[2], free_w[2], free_u[2], free_aq[2];
-    unsigned long long bar_x, bar_s, bar_o, bar_vp[2], bar_sa[2], out_free[2];
+    unsigned long long bar_x, bar_s, bar_o[2], bar_vp[2], bar_sa[2], out_free[2];
     uint32_t tmem_base;
 };
 
@@ -81,8 +85,8 @@ static_assert(offsetof(StateSmemF32, gv) % 16 == 0 && offsetof(StateSmemF32, eg)
               "bulk-copy and vector targets stay 16-byte aligned whatever the output type");
 static_assert(state_smem_bytes<float, 128, 128>() <= 227 * 1024, "state pass shared memory");
 
-// barrier among the compute warps; true when `pred` holds in all of them
-__device__ __forceinline__ bool cw_and(bool pred) {
+// barrier among `nthreads` threads on named barrier `id`; true when `pred` holds in all of them
+__device__ __forceinline__ bool group_and(bool pred, int id, int nthreads) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -90,10 +94,12 @@ __device__ __forceinline__ bool cw_and(bool pred) {
         "barrier.red.and.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "r"(kCwBarrier), "r"(NCW * 32)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
 }
+__device__ __forceinline__ bool cw_and(bool pred) { return group_and(pred, kCwBarrier, NCW * 32); }
+__device__ __forceinline__ bool ow_and(bool pred) { return group_and(pred, kOwBarrier, NOW * 32); }
 
 // fp16 copy of 32 consecutive values of S^T row j (this thread's lane) into 16 columns of the
 // tensor-memory A operand: two fp16 per column, the even column of S^T in the low half
@@ -169,15 +175,15 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             tc::mbar_init(bar(sm.full_aq[bb]), 1);
             tc::mbar_init(bar(sm.free_kq[bb]), 1);
             tc::mbar_init(bar(sm.free_w[bb]), 1);
-            tc::mbar_init(bar(sm.free_u[bb]), NCW);
-            tc::mbar_init(bar(sm.free_aq[bb]), NCW + 1);  // the output product's commit + every compute warp
+            tc::mbar_init(bar(sm.free_u[bb]), NCW + NOW);  // V' formed + the output warps' copy of e^gamma
+            tc::mbar_init(bar(sm.free_aq[bb]), 1);          // the output product's commit
             tc::mbar_init(bar(sm.bar_vp[bb]), NCW / 2);
             tc::mbar_init(bar(sm.bar_sa[bb]), NCW / 2);
-            tc::mbar_init(bar(sm.out_free[bb]), NCW);
+            tc::mbar_init(bar(sm.out_free[bb]), NOW);
+            tc::mbar_init(bar(sm.bar_o[bb]), 1);
         }
         tc::mbar_init(bar(sm.bar_x), 1);
         tc::mbar_init(bar(sm.bar_s), 1);
-        tc::mbar_init(bar(sm.bar_o), 1);
         tc::fence_mbar_init();
         for (int id = c_begin; id < c_end && id < c_begin + 2; ++id) fetch(id);
         for (int id = c_begin + 2; id < c_end && id < c_begin + kPrefetchAhead; ++id) prefetch(id);
@@ -228,45 +234,11 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
     }
 
-    // the outputs of chunk `it` (rows t < n at packed row t0), this thread's column j and half of the
-    // rows: o = e^{gamma_r} Oi + Oq, staged (bf16) or stored (fp32)
-    auto put_out = [&](int it, int t0, int n) {
-        const int bb = it & 1;
-#pragma unroll
-        for (int cc = 0; cc < C / 2; cc += 16) {
-            const int c0 = half * (C / 2) + cc;
-            float oi[16], oq[16], eg[16];
-            tc::tmem_ld16(tOi(bb) + lane_base + c0, oi);
-            tc::tmem_ld16(tOq(bb) + lane_base + c0, oq);
-#pragma unroll
-            for (int q = 0; q < 16; q += 4) *reinterpret_cast<float4*>(eg + q) = *reinterpret_cast<const float4*>(&sm.eg[bb][c0 + q]);
-            tc::tmem_ld_wait();
-            if (rowv)
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float o = fmaf(eg[i], oi[i], oq[i]);
-                    if constexpr (kStageOut<T>) sm.ostage[bb][(c0 + i) * DV + j] = from_f<T>(o);
-                    else if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + j] = from_f<T>(o);
-                }
-        }
-    };
-    // (compute warps, after the named barrier) the staged rows t < n leave as 16-byte vectors
-    auto send_out = [&](int it, int t0, int n) {
-        if constexpr (kStageOut<T>) {
-            constexpr int VPR = DV * (int)sizeof(T) / 16;  // vectors per row
-            for (int e = tid; e < n * VPR; e += NCW * 32) {
-                const int r = e / VPR, v = e % VPR;
-                reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * HV + h) * DV)[v] =
-                    reinterpret_cast<const uint4*>(sm.ostage[it & 1] + r * DV)[v];
-            }
-        }
-    };
-
     bool ok = true;
     if (warp == NCW + 1) {
         // ---- the copier: each buffer is refilled for the chunk two ahead as soon as its readers have
         // released it (W after X, U^T and the gate vectors once V' has been formed, [K ; Q] after the
-        // state product, Aqk once its product and the outputs are done).  The next release of a buffer
+        // state product, Aqk once its product is done).  The next release of a buffer
         // needs the copy issued here, so none of these barriers can complete twice before this lane
         // has seen the first.
         if (lane == 0) {
@@ -357,15 +329,13 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 for (int k = 0; k < C / 16; ++k)
                     tc::mma_f16(tOq(bb), tc::desc_add(dVt, tc::sw128_kstep(DV, k)),
                                 tc::desc_add(dAb, tc::sw128_kstep(C, k)), ix, k > 0);
-                tc::mma_commit(bar(sm.bar_o));
+                tc::mma_commit(bar(sm.bar_o[bb]));
                 tc::mma_commit(bar(sm.free_aq[bb]));
             }
         }
-    } else {
+    } else if (warp < NCW) {
         // ---- the compute warps.  Every wait is bounded; a failed one skips the work that needed it,
         // and the compute warps agree on the outcome at one barrier per chunk, so they stop together.
-        int prev_t0 = 0, prev_n = 0;
-        int4 chn = p.chunk_tab[c_begin];
         float amax = 0.f;  // largest magnitude this thread rounded to fp16 among V', f V' and S's copy
 #pragma unroll
         for (int i = 0; i < DK / 2; ++i) amax = fmaxf(amax, fabsf(s[i]));  // the starting state's copy
@@ -375,8 +345,6 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         for (int id = c_begin; id < c_end; ++id) {
             const int it = id - c_begin, bb = it & 1;
             const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
-            const int4 ch = chn;
-            if (id + 1 < c_end) chn = p.chunk_tab[id + 1];
             if (id == ck_chunk && rowv)  // the state entering the checkpoint's chunk: column j of S
 #pragma unroll
                 for (int i = 0; i < DK / 2; ++i) ck_dst[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
@@ -390,34 +358,30 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 char* vsb = reinterpret_cast<char*>(sm.vs);
                 const char* utb = reinterpret_cast<const char*>(sm.ut[bb]);
 #pragma unroll
-                for (int cc = 0; cc < C / 2; cc += 16) {
+                for (int cc = 0; cc < C / 2; cc += 8) {  // 8 fp16 values per 16-byte vector
                     const int c0 = half * (C / 2) + cc;
-                    float xv[16], f[16];
-                    tc::tmem_ld16(tX + lane_base + c0, xv);
+                    float xv[8], f[8];
+                    tc::tmem_ld8(tX + lane_base + c0, xv);
 #pragma unroll
-                    for (int q = 0; q < 16; q += 4) *reinterpret_cast<float4*>(f + q) = *reinterpret_cast<const float4*>(&sm.gv[bb][1][c0 + q]);
+                    for (int q = 0; q < 8; q += 4) *reinterpret_cast<float4*>(f + q) = *reinterpret_cast<const float4*>(&sm.gv[bb][1][c0 + q]);
                     tc::tmem_ld_wait();
-                    if (rowv)
+                    if (rowv) {
+                        const uint32_t off = uoff(c0);
+                        const uint4 u = *reinterpret_cast<const uint4*>(utb + off);
+                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                        uint32_t vw[4], sw[4];
 #pragma unroll
-                        for (int q = 0; q < 2; ++q) {  // 8 fp16 values per 16-byte vector
-                            const uint32_t off = uoff(c0 + 8 * q);
-                            const uint4 u = *reinterpret_cast<const uint4*>(utb + off);
-                            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-                            uint32_t vw[4], sw[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 uu = tc::unpack_f16(uw[e]);
-                                const float v0 = uu.x - xv[8 * q + 2 * e], v1 = uu.y - xv[8 * q + 2 * e + 1];
-                                amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));  // |f| <= 1: covers f V' too
-                                vw[e] = tc::pack_f16(v0, v1);
-                                sw[e] = tc::pack_f16(v0 * f[8 * q + 2 * e], v1 * f[8 * q + 2 * e + 1]);
-                            }
-                            *reinterpret_cast<uint4*>(vtb + off) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-                            *reinterpret_cast<uint4*>(vsb + off) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 uu = tc::unpack_f16(uw[e]);
+                            const float v0 = uu.x - xv[2 * e], v1 = uu.y - xv[2 * e + 1];
+                            amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));  // |f| <= 1: covers f V' too
+                            vw[e] = tc::pack_f16(v0, v1);
+                            sw[e] = tc::pack_f16(v0 * f[2 * e], v1 * f[2 * e + 1]);
                         }
+                        *reinterpret_cast<uint4*>(vtb + off) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+                        *reinterpret_cast<uint4*>(vsb + off) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+                    }
                 }
-                if (warp == 0 || warp == 4)  // the output scale of this chunk, for its outputs one chunk later
-                    sm.eg[bb][half * 32 + lane] = sm.gv[bb][0][half * 32 + lane];
                 egn = sm.gv[bb][3][0];  // e^{gamma_n}
                 tc::fence_smem_to_async();
                 tc::fence_before_sync();
@@ -432,66 +396,93 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             if (okl) {
                 tc::fence_after_sync();
 #pragma unroll
-                for (int cc = 0; cc < DK / 2; cc += 32) {
-                    const int c0 = half * (DK / 2) + cc;
-                    float v[32];
-                    tc::tmem_ld16(tSn + lane_base + c0, *reinterpret_cast<float(*)[16]>(v));
-                    tc::tmem_ld16(tSn + lane_base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+                for (int cc = 0; cc < DK / 2; cc += 16) {
+                    float v[16];
+                    tc::tmem_ld16(tSn + lane_base + half * (DK / 2) + cc, v);
                     tc::tmem_ld_wait();
+                    uint32_t wv[8];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         s[cc + i] = fmaf(egn, s[cc + i], v[i]);
                         amax = fmaxf(amax, fabsf(s[cc + i]));
                     }
-                    put_sa32(tA_row + cc / 2, &s[cc]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) wv[i] = tc::pack_f16(s[cc + 2 * i], s[cc + 2 * i + 1]);
+                    tc::tmem_st8(tA_row + cc / 2, wv);
                 }
                 tc::tmem_st_wait();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
             }
-            // the previous chunk's outputs, while the next chunk's X runs (their products completed before
-            // this chunk's X did: a commit covers every earlier product of the issuing thread); their
-            // accumulators and the Aqk buffer are then released
-            if (okl && it > 0) {
-                tc::fence_after_sync();
-                put_out(it - 1, prev_t0, prev_n);
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(bar(sm.out_free[bb ^ 1]));
-                    tc::mbar_arrive(bar(sm.free_aq[bb ^ 1]));
-                }
-            }
-            ok = cw_and(okl);  // also orders the output scale and the staged outputs between the warps
-            if (!ok) break;
-            if (it > 0) send_out(it - 1, prev_t0, prev_n);  // the previous chunk's staged outputs leave
-            prev_t0 = ch.y;
-            prev_n = ch.z;
-        }
-        if (ok) {  // the last chunk's outputs and the final state
-            const int it = c_end - 1 - c_begin;
-            bool okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_o), (uint32_t)it & 1u));
-            if (okl) {
-                tc::fence_after_sync();
-                put_out(it, prev_t0, prev_n);
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(bar(sm.out_free[it & 1]));
-                    tc::mbar_arrive(bar(sm.free_aq[it & 1]));
-                }
-            }
             ok = cw_and(okl);
-            if (ok) send_out(it, prev_t0, prev_n);
-            if (ok && rowv)  // final state: column j of S
-#pragma unroll
-                for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
+            if (!ok) break;
         }
+        if (ok && rowv)  // final state: column j of S
+#pragma unroll
+            for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
         if (!rowv) amax = 0.f;  // lanes past a 64-row tile hold no row
         report_f16_range(p.hdr, amax);
+    } else {
+        // ---- the output warps: warp OW0 + w reads sub-partition (OW0 + w) % 4, a row j of Oi^T and
+        // Oq^T with all of the chunk's 64 columns.  Per chunk: the chunk's e^{gamma_r} is copied while
+        // its gate vector is in (then released to the copier); once the output products complete,
+        // o = e^{gamma_r} Oi + Oq is staged (bf16) or stored (fp32) and the accumulators are handed
+        // back; the staged rows then leave as 16-byte vectors.
+        const int osp = warp & 3, ot = tid - OW0 * 32;
+        const uint32_t olane = (uint32_t)(osp * 32) << 16;
+        const bool orow = DV == 128 || lane < 16;
+        const int oj = DV == 128 ? osp * 32 + lane : osp * 16 + lane;
+        for (int id = c_begin; id < c_end && ok; ++id) {
+            const int it = id - c_begin, bb = it & 1;
+            const uint32_t pb = (uint32_t)(it >> 1) & 1u;
+            const int4 ch = p.chunk_tab[id];
+            const int t0 = ch.y, n = ch.z;
+            bool okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.full_u[bb]), pb));
+            if (okl) {
+                if (ot < C) sm.eg[bb][ot] = sm.gv[bb][0][ot];
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(sm.free_u[bb]));
+            }
+            okl = ow_and(okl);  // the copy of e^gamma is complete
+            if (okl) okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_o[bb]), pb));
+            if (okl) {
+                tc::fence_after_sync();
+#pragma unroll
+                for (int c0 = 0; c0 < C; c0 += 16) {
+                    float oi[16], oq[16], eg[16];
+                    tc::tmem_ld16(tOi(bb) + olane + c0, oi);
+                    tc::tmem_ld16(tOq(bb) + olane + c0, oq);
+#pragma unroll
+                    for (int q = 0; q < 16; q += 4)
+                        *reinterpret_cast<float4*>(eg + q) = *reinterpret_cast<const float4*>(&sm.eg[bb][c0 + q]);
+                    tc::tmem_ld_wait();
+                    if (orow)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float o = fmaf(eg[i], oi[i], oq[i]);
+                            if constexpr (kStageOut<T>) sm.ostage[bb][(c0 + i) * DV + oj] = from_f<T>(o);
+                            else if (c0 + i < n) out[((size_t)(t0 + c0 + i) * HV + h) * DV + oj] = from_f<T>(o);
+                        }
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(sm.out_free[bb]));
+            }
+            ok = ow_and(okl);  // the staged rows are complete
+            if (ok) {
+                if constexpr (kStageOut<T>) {
+                    constexpr int VPR = DV * (int)sizeof(T) / 16;  // vectors per row
+                    for (int e = ot; e < n * VPR; e += NOW * 32) {
+                        const int r = e / VPR, v = e % VPR;
+                        reinterpret_cast<uint4*>(out + ((size_t)(t0 + r) * HV + h) * DV)[v] =
+                            reinterpret_cast<const uint4*>(sm.ostage[bb] + r * DV)[v];
+                    }
+                }
+            }
+        }
     }
-    ok = __syncthreads_and(ok);  // the chain, the issuer, the copier and the idle lanes agree
+    ok = __syncthreads_and(ok);  // the chain, the issuer, the copier, the output warps and the idle lanes agree
     if (!ok && tid == ISSUER) {
         raise_error(p.hdr, GDN_DEVERR_TIMEOUT);
         // let copies and products already in flight finish before the CTA's shared and tensor
@@ -503,7 +494,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 tc::mbar_wait(bar(sm.full_u[bb]), par, 100000000ull);
                 tc::mbar_wait(bar(sm.full_aq[bb]), par, 100000000ull);
             }
-            tc::mbar_wait(bar(sm.bar_o), par, 100000000ull);
+            tc::mbar_wait(bar(sm.bar_o[0]), par, 100000000ull);
+            tc::mbar_wait(bar(sm.bar_o[1]), par, 100000000ull);
         }
     }
     if (ok && tid == ISSUER) {  // the releases nobody waited for, so that none lands after the CTA is gone

@@ -129,15 +129,51 @@ __device__ __forceinline__ void store_h8(char* tile, uint32_t off, const float* 
                                                        tc::pack_f16(v[4], v[5]), tc::pack_f16(v[6], v[7]));
 }
 
+// two fp32 lanes at once: d = a * b + c and d = a * b, each lane rounded exactly as fmaf / __fmul_rn
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 r;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return r;
+}
+// SiLU of two values (see silu_fast)
+__device__ __forceinline__ float2 silu2(float2 x) {
+    const float2 h = fmul2(make_float2(0.5f, 0.5f), x);
+    float2 t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(h.y));
+    return ffma2(h, t, h);
+}
+
 // conv1d (K = 4) + SiLU of 8 consecutive output rows r0 .. r0+7 (rows >= n give 0) of 4 consecutive
 // channels, from staged rows r0 .. r0+10 (staged row i holds packed row t0 - 3 + i) with a sliding
-// window; `xs` points at the first of the 4 channels in staged row 0, `w` at their 16 taps.
+// window; `xs` points at the first of the 4 channels in staged row 0, `w` at their 16 taps.  Channels
+// go in pairs through the two-lane FMA, each channel's taps accumulated in the same order as one
+// fmaf chain would.
 template <typename T>
 __device__ __forceinline__ void conv8x4(const T* xs, int ld, const T* w, const T* bias, int r0, int n,
                                         float (&y)[8][4]) {
     float wt[4][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) load4(w + 4 * u, wt[u]);
+    float2 w01[4], w23[4];  // tap j of channels (0, 1) and (2, 3)
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        w01[jj] = make_float2(wt[0][jj], wt[1][jj]);
+        w23[jj] = make_float2(wt[2][jj], wt[3][jj]);
+    }
     float b[4] = {0.f, 0.f, 0.f, 0.f};
     if (bias) load4(bias, b);
     float win[4][4];
@@ -146,13 +182,23 @@ __device__ __forceinline__ void conv8x4(const T* xs, int ld, const T* w, const T
 #pragma unroll
     for (int o = 0; o < 8; ++o) {
         load4(xs + (size_t)(r0 + o + 3) * ld, win[(o + 3) & 3]);
+        float2 a01 = make_float2(b[0], b[1]), a23 = make_float2(b[2], b[3]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            float acc = b[u];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc = fmaf(wt[u][j], win[(o + j) & 3][u], acc);
-            y[o][u] = r0 + o < n ? silu_fast(acc) : 0.f;
+        for (int jj = 0; jj < 4; ++jj) {
+            const float* wr = win[(o + jj) & 3];
+            a01 = ffma2(w01[jj], make_float2(wr[0], wr[1]), a01);
+            a23 = ffma2(w23[jj], make_float2(wr[2], wr[3]), a23);
         }
+        if (r0 + o < n) {
+            a01 = silu2(a01);
+            a23 = silu2(a23);
+        } else {
+            a01 = a23 = make_float2(0.f, 0.f);
+        }
+        y[o][0] = a01.x;
+        y[o][1] = a01.y;
+        y[o][2] = a23.x;
+        y[o][3] = a23.y;
     }
 }
 
@@ -286,24 +332,23 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
         stage_rows(sm.xv, S::LDV, DV / VE, q, [&](int v) { return cv0 + v * VE; });
         for (int e = tid; e < DV * 4 / VE; e += NT) tc::cp_async16(sm.wv + e * VE, w + (size_t)cv0 * 4 + e * VE);
     };
-    // the raw gate inputs of value head h (threads NT-C .. NT-1, one row each), held in registers until
-    // commit_gates turns them into (g, beta) in shared memory
-    float ga = 0.f, gbv = 0.f;
+    // the raw gate inputs of value head h (threads NT-C .. NT-1, one row each), held in registers as
+    // loaded (nothing waits for the loads) until commit_gates turns them into (g, beta) in shared memory
+    T ga = from_f<T>(0.f), gbv = from_f<T>(0.f);
     auto load_gates = [&](const Pos& q, int h) {
         if (tid >= NT - C) {
             const int r = tid - (NT - C);
-            ga = gbv = 0.f;
             if (r < q.n) {
                 const size_t row = (size_t)(q.t0 + r) * HV + h;
-                ga = to_f(reinterpret_cast<const T*>(p.a)[row]);
-                gbv = to_f(reinterpret_cast<const T*>(p.b)[row]);
+                ga = reinterpret_cast<const T*>(p.a)[row];
+                gbv = reinterpret_cast<const T*>(p.b)[row];
             }
         }
     };
     auto commit_gates = [&](int n, int h) {  // zero past the end of the chunk
         if (tid >= NT - C) {
             const int r = tid - (NT - C);
-            sm.gb[r] = r < n ? make_float2(-expf(p.A_log[h]) * softplus_f(ga + p.dt_bias[h]), sigmoid_f(gbv))
+            sm.gb[r] = r < n ? make_float2(-expf(p.A_log[h]) * softplus_f(to_f(ga) + p.dt_bias[h]), sigmoid_f(to_f(gbv)))
                              : make_float2(0.f, 0.f);
         }
     };
@@ -344,6 +389,12 @@ __global__ void __launch_bounds__(NT, kCtasPerSm) chunk_tc_kernel(ExtendArgs p, 
                                              : row + 2 * d.HK * DK + hkn * G * DV + (l - 2 * LQ) * (128 / sizeof(T));
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(a_));
                 }
+                // and its gate inputs: rows t0 .. t0+n-1 of a and b are one contiguous span each
+                const char* ga0 = reinterpret_cast<const char*>(reinterpret_cast<const T*>(p.a) + (size_t)chn.y * HV);
+                const char* gb0 = reinterpret_cast<const char*>(reinterpret_cast<const T*>(p.b) + (size_t)chn.y * HV);
+                const int glines = (int)(((size_t)chn.z * HV * sizeof(T) + 127) / 128);
+                for (int e = tid; e < 2 * glines; e += NT)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"((e < glines ? ga0 : gb0) + (size_t)(e % glines) * 128));
             }
         }
         // ---- conv + SiLU + L2 norm of k (tile rows 0..63) and q*scale (rows 64..127).  A task is 8 rows

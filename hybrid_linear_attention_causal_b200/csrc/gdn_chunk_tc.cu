@@ -729,7 +729,7 @@ cudaError_t launch_chunk(const ExtendArgs& p, int seg, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     // CTAs of up to kItemsPerCta (chunk, qk head) items each, enough for the most a segment can hold
-    const long long items = ((long long)p.max_chunks + p.nseg - 1) / p.nseg * p.d.HK;
+    const long long items = seg_max_piece(p.max_chunks, p.nseg) * p.d.HK;
     const int grid = (int)((items + kItemsPerCta - 1) / kItemsPerCta);
     chunk_tc_kernel<T, DK, DV><<<grid, NT, shm, s>>>(p, seg);
     return cudaGetLastError();

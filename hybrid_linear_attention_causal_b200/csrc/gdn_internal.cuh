@@ -19,7 +19,7 @@ constexpr int kMaxVerifyDraft = 16; // D limit of gdn_verify
 constexpr int kHdrError = 0;        // sticky GDN_DEVERR_* bits
 constexpr int kHdrNumChunks = 1;    // chunk count of the current extend batch
 constexpr int kMaxSegments = 16;    // segments of an extend batch (see below)
-constexpr int kHdrSegLen = 2;       // P: chunks per segment (the last may hold fewer)
+constexpr int kHdrSegLen = 2;       // chunks in the largest segment
 constexpr int kHdrSegOff = 3;       // [kMaxSegments]: first chunk_list entry of segment k
 constexpr int kHdrSegCnt = kHdrSegOff + kMaxSegments;    // [kMaxSegments]: chunks in segment k
 constexpr int kHdrSegSeqs = kHdrSegCnt + kMaxSegments;   // [kMaxSegments]: sequences with chunks in segment k
@@ -35,6 +35,33 @@ static_assert((kHdrSegRank + kMaxSegments) * 4 <= kHeaderBytes, "header too smal
 // and continuing from the state the previous piece left in its slot,
 // alongside intra of segment k+1.  A piece holds few sequences, so its state
 // pass needs few SMs; the shortest sequences come last.
+//
+// The pieces grow geometrically by kSegGrowth: the chain cannot start before
+// the first piece's per-chunk step ends, and the per-chunk step runs a little
+// faster per chunk than the chain, so a short first piece starts the chain
+// early while each later piece is still ready before the chain reaches it.
+// Piece k holds list entries [seg_bound(k), seg_bound(k + 1)).
+constexpr double kSegGrowth = 1.12;
+
+__host__ __device__ inline int seg_bound(int k, int nseg, int total) {
+    if (k <= 0) return 0;
+    if (k >= nseg) return total;
+    double rk = 1.0, rn = 1.0;
+    for (int i = 0; i < nseg; ++i) {
+        if (i < k) rk *= kSegGrowth;
+        rn *= kSegGrowth;
+    }
+    const int b = (int)((double)total * (rk - 1.0) / (rn - 1.0));
+    return b < 0 ? 0 : (b > total ? total : b);
+}
+
+// an upper bound on the entries of the largest piece of a list of at most `chunks` entries
+__host__ inline long long seg_max_piece(long long chunks, int nseg) {
+    if (nseg <= 1) return chunks;
+    double rn = 1.0;
+    for (int i = 0; i < nseg; ++i) rn *= kSegGrowth;
+    return (long long)((double)chunks * (rn / kSegGrowth) * (kSegGrowth - 1.0) / (rn - 1.0)) + 2;
+}
 
 struct LayerDims {
     int HK, HV, dk, dv, G;  // G = HV / HK

@@ -120,11 +120,10 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
     if (tid == 0) p.rank_off[p.N] = total;
     __threadfence_block();
     __syncthreads();
-    // Segments: the list cut into nseg pieces of P chunks.  The state pass of segment k takes, for
-    // each sequence, its chunks inside piece k, continuing from the state the previous piece left.
-    const int P = max(1, (total + p.nseg - 1) / p.nseg);
+    // Segments: the list cut into nseg pieces growing by kSegGrowth.  The state pass of segment k takes,
+    // for each sequence, its chunks inside piece k, continuing from the state the previous piece left.
     if (tid < kMaxSegments) {
-        const int k = tid, lo = min(k * P, total), hi = min(lo + P, total);
+        const int k = tid, lo = seg_bound(k, p.nseg, total), hi = k < p.nseg ? seg_bound(k + 1, p.nseg, total) : lo;
         p.hdr[kHdrSegOff + k] = lo;
         p.hdr[kHdrSegCnt + k] = hi - lo;
         p.hdr[kHdrItemNext + k] = 0;
@@ -146,7 +145,7 @@ __global__ void __launch_bounds__(1024) chunk_map_kernel(ExtendArgs p) {
         p.hdr[kHdrSegRank + k] = first;
         p.hdr[kHdrSegSeqs + k] = last - first + 1;
     }
-    if (tid == 0) p.hdr[kHdrSegLen] = P;
+    if (tid == 0) p.hdr[kHdrSegLen] = seg_bound(p.nseg, p.nseg, total) - seg_bound(p.nseg - 1, p.nseg, total);
     for (int id = tid; id < total; id += 1024) {
         int lo = 0, hi = p.N - 1;  // last sequence whose first chunk id <= id
         while (lo < hi) {

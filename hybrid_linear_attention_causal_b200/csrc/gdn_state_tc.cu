@@ -520,7 +520,7 @@ cudaError_t launch_state(const ExtendArgs& p, int seg, cudaStream_t s) {
         cudaFuncSetAttribute(state_tc_kernel<T, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shm);
     if (e != cudaSuccess) return e;
     // a piece of P chunks touches at most P + 1 sequences
-    const long long piece = ((long long)p.max_chunks + p.nseg - 1) / p.nseg;
+    const long long piece = seg_max_piece(p.max_chunks, p.nseg);
     const long long seqs = piece + 1 < p.N ? piece + 1 : p.N;
     state_tc_kernel<T, DK, DV><<<(unsigned)(seqs * p.d.HV), NT, shm, s>>>(p, seg);
     return cudaGetLastError();

@@ -187,8 +187,9 @@ int extend_impl(const gdn_config_t* cfg, const gdn_params_t* params, const void*
     e.ck_states = ck.ck_states;
     e.ck_conv = ck.ck_conv;
     e.num_ck = ck.num_ck;
-    // about one segment per 16384 packed rows (measured best on B200 among 4096 .. 40000): a
-    // segment's intra work then hides the previous segment's state pass, and each launch's
+    // about one segment per 16384 packed rows (measured best on B200 among 4096 .. 40000; 8192 and
+    // 4096 again slower on the 8-sequence 32768-row batch with the fused per-chunk step): a
+    // segment's per-chunk work then hides the previous segment's state pass, and each launch's
     // ramp-up and tail stay small against its work
     e.nseg = T / 16384 < 1 ? 1 : (T / 16384 > gdn::kMaxSegments ? gdn::kMaxSegments : T / 16384);
     gdn::carve_extend_workspace(e, workspace, N, T);

@@ -23,17 +23,17 @@ constexpr int kHdrSegLen = 2;       // chunks in the largest segment
 constexpr int kHdrSegOff = 3;       // [kMaxSegments]: first chunk_list entry of segment k
 constexpr int kHdrSegCnt = kHdrSegOff + kMaxSegments;    // [kMaxSegments]: chunks in segment k
 constexpr int kHdrSegSeqs = kHdrSegCnt + kMaxSegments;   // [kMaxSegments]: sequences with chunks in segment k
-constexpr int kHdrItemNext = kHdrSegSeqs + kMaxSegments; // [kMaxSegments]: next intra item of segment k
+constexpr int kHdrItemNext = kHdrSegSeqs + kMaxSegments; // [kMaxSegments]: next per-chunk item of segment k
 constexpr int kHdrSegRank = kHdrItemNext + kMaxSegments; // [kMaxSegments]: first rank with chunks in segment k
 static_assert((kHdrSegRank + kMaxSegments) * 4 <= kHeaderBytes, "header too small");
 
 // An extend batch is cut into S segments (S chosen by the host, at most
-// kMaxSegments): the chunks, listed longest sequence first, in S pieces of P
-// consecutive list entries.  The intra step runs segment by segment on the
+// kMaxSegments): the chunks, listed longest sequence first, in S pieces of
+// consecutive list entries.  The per-chunk step runs segment by segment on the
 // caller's stream; the state pass of segment k runs on a second stream once
-// intra has finished segment k, taking each sequence's chunks inside the piece
-// and continuing from the state the previous piece left in its slot,
-// alongside intra of segment k+1.  A piece holds few sequences, so its state
+// the per-chunk step has finished segment k, taking each sequence's chunks
+// inside the piece and continuing from the state the previous piece left in
+// its slot, alongside the per-chunk step of segment k+1.  A piece holds few sequences, so its state
 // pass needs few SMs; the shortest sequences come last.
 //
 // The pieces grow geometrically by kSegGrowth: the chain cannot start before

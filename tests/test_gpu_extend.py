@@ -144,7 +144,7 @@ def test_many_sequences(HK, HV, dk, dv, dtype):
 ])
 def test_segmented_batches(lengths, slots, hi):
     """Batches of 32768 packed rows or more run as several segments (the state
-    pass of segment k alongside intra of segment k+1, each segment a piece of
+    pass of segment k alongside the per-chunk step of segment k+1, each segment a piece of
     the chunks listed longest sequence first); every sequence's chain must
     continue across the segment boundaries."""
     spec = W.LayerSpec(HK=2, HV=4, dk=128, dv=128, dtype=torch.bfloat16)

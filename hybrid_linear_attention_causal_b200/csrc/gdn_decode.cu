@@ -109,6 +109,16 @@ __device__ __forceinline__ void state_step(float4 (&s)[RPT], const float* qv, co
     }
 }
 
+// The states of value heads h0 .. h0 + nh - 1 of a slot (contiguous in the pool) into L2, one
+// 128-byte line per prefetch spread over the CTA, so that the state read overlaps work that does not
+// need it yet (the conv, norm and gate phase; the previous head's tokens).
+template <int DK, int DV>
+__device__ __forceinline__ void prefetch_states_l2(const float* pool, int slot, int HV, int h0, int nh, int tid) {
+    const char* base = reinterpret_cast<const char*>(pool + ((size_t)slot * HV + (size_t)h0) * DK * DV);
+    const int lines = nh * DK * DV * 4 / 128;
+    for (int l = tid; l < lines; l += kNT) asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (size_t)l * 128));
+}
+
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kNT) decode_kernel(DecodeArgs p) {
     constexpr int CG = DV / 4, RSTEP = kNT / CG, RPT = DK / RSTEP;
@@ -130,6 +140,7 @@ __global__ void __launch_bounds__(kNT) decode_kernel(DecodeArgs p) {
         for (int i = tid; i < G * DV; i += kNT) out[i] = from_f<T>(0.f);
         return;
     }
+    prefetch_states_l2<DK, DV>(p.ssm_state, slot, d.HV, hk * G, G, tid);
     // conv window update + SiLU for every owned channel
     {
         const T* x = reinterpret_cast<const T*>(p.x) + (size_t)req * d.conv_dim;
@@ -217,6 +228,9 @@ __global__ void __launch_bounds__(kNT) verify_kernel(DecodeArgs p) {
         }
         return;
     }
+    // the first value head's state at the start; each next one while the previous head's tokens run
+    // (measured faster than all of them at the start)
+    prefetch_states_l2<DK, DV>(p.ssm_state, slot, d.HV, hk * G, 1, tid);
     {
         const T* cs = reinterpret_cast<const T*>(p.conv_state) + (size_t)slot * d.conv_dim * 3;
         const T* w = reinterpret_cast<const T*>(p.conv_w);
@@ -277,6 +291,7 @@ __global__ void __launch_bounds__(kNT) verify_kernel(DecodeArgs p) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k)
             s[k] = __ldcs(reinterpret_cast<const float4*>(Sp + (size_t)(r0 + k * RSTEP) * DV) + cg);
+        if (j + 1 < G) prefetch_states_l2<DK, DV>(p.ssm_state, slot, d.HV, h + 1, 1, tid);
         int cur = -1;  // the tree node whose state the registers hold
         for (int t = 0; t < D; ++t) {
             if (par[t] != cur) {  // a branch: continue from the parent's checkpoint (or the slot), which

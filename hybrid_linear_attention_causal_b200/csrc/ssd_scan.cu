@@ -204,7 +204,9 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
     // each of 8 rows and eight consecutive threads later store one 128-byte core-matrix block
     constexpr int NBX = SP / 8, NBB = N / 8, KX = SC * NBX / SNT, KB = SC * NBB / SNT;
     uint4 rx[KX], rz[KX], rb[KB], rc[KB];
-    float rdt0 = 0.f, rdt1 = 0.f;  // (warp 0) raw steps of rows lane and lane + 32
+    // (warp 0) raw steps of rows lane and lane + 32, held as loaded (nothing waits for the loads until
+    // the next chunk's step phase)
+    __nv_bfloat16 rdt0 = __float2bfloat16(0.f), rdt1 = __float2bfloat16(0.f);
     auto chunk_len = [&](int t0) {  // up to 64 rows, cut at the checkpoint boundary
         int len = min(SC, s1 - t0);
         if (ck_b > t0 && ck_b < t0 + len) len = ck_b - t0;
@@ -232,8 +234,8 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
             }
         }
         if (warp == 0) {
-            rdt0 = lane < len ? __bfloat162float(p.dt[(size_t)(t0 + lane) * p.H + h]) : 0.f;
-            rdt1 = lane + 32 < len ? __bfloat162float(p.dt[(size_t)(t0 + lane + 32) * p.H + h]) : 0.f;
+            if (lane < len) rdt0 = p.dt[(size_t)(t0 + lane) * p.H + h];
+            if (lane + 32 < len) rdt1 = p.dt[(size_t)(t0 + lane + 32) * p.H + h];
         }
     };
     int len = s0 < s1 ? chunk_len(s0) : 0;
@@ -244,8 +246,8 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
     for (int t0 = s0; t0 < s1; ph ^= 1u) {
         // ---- processed steps and in-chunk cumulative decay (warp 0, rows lane and lane + 32)
         if (warp == 0) {
-            const float d0 = lane < len ? ssd_step(p, rdt0, h) : 0.f;
-            const float d1 = lane + 32 < len ? ssd_step(p, rdt1, h) : 0.f;
+            const float d0 = lane < len ? ssd_step(p, __bfloat162float(rdt0), h) : 0.f;
+            const float d1 = lane + 32 < len ? ssd_step(p, __bfloat162float(rdt1), h) : 0.f;
             float c0 = d0 * Ah2, c1 = d1 * Ah2;  // base-2 exponents
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {

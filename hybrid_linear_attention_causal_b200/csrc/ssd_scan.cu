@@ -80,9 +80,10 @@ struct SsdSmem {
     uint16_t ht[N * SP];   // fp16 copy of h^T: rows n x P (R = N)
     __nv_bfloat16 xs[SC][SP + 8];  // the chunk's x rows (bf16) and gates silu(z) (fp32), rows padded by
     float zs[SC][SP + 4];          // 16 bytes so that the threads reading one row each spread over the banks
-    float g2[SC];          // gamma_r log2(e) (rows past the chunk repeat the last row's)
-    float dd[SC];          // processed step d_r (0 past the chunk)
-    float wl[SC];          // d_s e^{gamma_last - gamma_s}
+    // per chunk, double-buffered (the next chunk's are formed while this one's products run):
+    float g2[2][SC];       // gamma_r log2(e) (rows past the chunk repeat the last row's)
+    float dd[2][SC];       // processed step d_r (0 past the chunk)
+    float wl[2][SC];       // d_s e^{gamma_last - gamma_s}
     unsigned long long bar1, bar2;
     uint32_t tmem_base;
 };
@@ -238,34 +239,37 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
             if (lane + 32 < len) rdt1 = p.dt[(size_t)(t0 + lane + 32) * p.H + h];
         }
     };
+    // (warp 0) processed steps and in-chunk cumulative decay of a chunk of `ln` rows (rows lane and
+    // lane + 32) into step buffer sb, from the raw steps fetched with its rows
+    auto form_steps = [&](int sb, int ln) {
+        const float d0 = lane < ln ? ssd_step(p, __bfloat162float(rdt0), h) : 0.f;
+        const float d1 = lane + 32 < ln ? ssd_step(p, __bfloat162float(rdt1), h) : 0.f;
+        float c0 = d0 * Ah2, c1 = d1 * Ah2;  // base-2 exponents
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v0 = __shfl_up_sync(0xffffffffu, c0, o), v1 = __shfl_up_sync(0xffffffffu, c1, o);
+            if (lane >= o) {
+                c0 += v0;
+                c1 += v1;
+            }
+        }
+        c1 += __shfl_sync(0xffffffffu, c0, 31);
+        const float gl = __shfl_sync(0xffffffffu, c1, 31);  // rows past the chunk add nothing
+        sm.g2[sb][lane] = c0;
+        sm.g2[sb][lane + 32] = c1;
+        sm.dd[sb][lane] = d0;
+        sm.dd[sb][lane + 32] = d1;
+        sm.wl[sb][lane] = d0 * tc::ex2_approx(gl - c0);
+        sm.wl[sb][lane + 32] = d1 * tc::ex2_approx(gl - c1);
+    };
     int len = s0 < s1 ? chunk_len(s0) : 0;
     if (len > 0) fetch(s0, len);
+    if (len > 0 && warp == 0) form_steps(0, len);
 
     bool ok = true, okw = true;
     uint32_t ph = 0;
     for (int t0 = s0; t0 < s1; ph ^= 1u) {
-        // ---- processed steps and in-chunk cumulative decay (warp 0, rows lane and lane + 32)
-        if (warp == 0) {
-            const float d0 = lane < len ? ssd_step(p, __bfloat162float(rdt0), h) : 0.f;
-            const float d1 = lane + 32 < len ? ssd_step(p, __bfloat162float(rdt1), h) : 0.f;
-            float c0 = d0 * Ah2, c1 = d1 * Ah2;  // base-2 exponents
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v0 = __shfl_up_sync(0xffffffffu, c0, o), v1 = __shfl_up_sync(0xffffffffu, c1, o);
-                if (lane >= o) {
-                    c0 += v0;
-                    c1 += v1;
-                }
-            }
-            c1 += __shfl_sync(0xffffffffu, c0, 31);
-            const float gl = __shfl_sync(0xffffffffu, c1, 31);  // rows past the chunk add nothing
-            sm.g2[lane] = c0;
-            sm.g2[lane + 32] = c1;
-            sm.dd[lane] = d0;
-            sm.dd[lane + 32] = d1;
-            sm.wl[lane] = d0 * tc::ex2_approx(gl - c0);
-            sm.wl[lane + 32] = d1 * tc::ex2_approx(gl - c1);
-        }
+        const int cur = (int)ph;  // this chunk's step buffer
         ok = __syncthreads_and(okw) != 0;  // (also: the previous chunk's outputs are all read)
         if (!ok) break;
         // ---- the fetched rows into the fp16 operand tiles (zero past the chunk) and the bf16
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
             bf16x8(rx[k], f);
             const uint32_t off = tc::kmajor_off16(r, cb * 8, SC);
             st16(sm.xt, off, f16x8(f));
-            const float w = sm.wl[r];
+            const float w = sm.wl[cur][r];
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[i] *= w;
             st16(sm.xw, off, f16x8(f));
@@ -318,10 +322,15 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
                 tc::mma_f16(tS, tc::desc_mnmajor16(bt, SC, k), tc::desc_mnmajor16(xw, SC, k), iH, k > 0);
             tc::mma_commit(bar1);
         }
+        // the next chunk's rows load (into the registers this chunk's staging has just emptied) while
+        // this chunk's products, state update and outputs run; warp 0 forms its steps meanwhile
+        const int t0n = t0 + len, lenn = t0n < s1 ? chunk_len(t0n) : 0;
+        if (lenn > 0) fetch(t0n, lenn);
+        if (lenn > 0 && warp == 0) form_steps(cur ^ 1, lenn);
         okw = tc::mbar_wait(bar1, ph);
         tc::fence_after_sync();
         {  // h^T <- e^{gamma_last} h^T + Hnew^T
-            const float egl = tc::ex2_approx(sm.g2[SC - 1]);
+            const float egl = tc::ex2_approx(sm.g2[cur][SC - 1]);
 #pragma unroll
             for (int c0 = 0; c0 < SP; c0 += 16) {
                 float v[16];
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
         }
         put_ht();
         {  // Lm row r_own: e^{gamma_r - gamma_s} d_s Gm[r, s] for s <= r
-            const float gr = sm.g2[r_own];
+            const float gr = sm.g2[cur][r_own];
             const bool rv = lane < 16 && r_own < len;
 #pragma unroll
             for (int c0 = 0; c0 < SC; c0 += 16) {
@@ -347,7 +356,7 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int s = c0 + q + i;
-                            f[i] = (rv && s <= r_own) ? v[q + i] * sm.dd[s] * tc::ex2_approx(gr - sm.g2[s]) : 0.f;
+                            f[i] = (rv && s <= r_own) ? v[q + i] * sm.dd[cur][s] * tc::ex2_approx(gr - sm.g2[cur][s]) : 0.f;
                         }
                         st16(sm.lm, tc::kmajor_off16(r_own, c0 + q, SC), f16x8(f));
                     }
@@ -366,14 +375,11 @@ __global__ void __launch_bounds__(SNT, 2) ssd_scan_kernel(SsdArgs p) {
                 tc::mma_f16(tY, tc::desc_kmajor(lm, SC, k), tc::desc_mnmajor16(xt, SC, k), iZ, k > 0);
             tc::mma_commit(bar2);
         }
-        // the next chunk's rows load while Y and this chunk's outputs complete
-        const int t0n = t0 + len, lenn = t0n < s1 ? chunk_len(t0n) : 0;
-        if (lenn > 0) fetch(t0n, lenn);
         okw = tc::mbar_wait(bar2, ph);
         tc::fence_after_sync();
         {  // y_r = Y_r + e^{gamma_r} Z_r, skip term, gate
             const bool live = okw && lane < 16 && r_own < len;
-            const float eg = tc::ex2_approx(sm.g2[r_own]);
+            const float eg = tc::ex2_approx(sm.g2[cur][r_own]);
             const size_t row = ((size_t)(t0 + r_own) * p.H + h) * SP;
 #pragma unroll
             for (int c0 = 0; c0 < SP; c0 += 16) {

@@ -114,15 +114,6 @@ __device__ __forceinline__ void load4(const float* p, float* v) {
     v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
 }
 
-// SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x / 2, with the hardware tanh (one MUFU operation;
-// its error is below the fp16 rounding every conv output goes through)
-__device__ __forceinline__ float silu_fast(float x) {
-    const float h = 0.5f * x;
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
-    return fmaf(h, t, h);
-}
-
 // 8 floats -> 8 fp16 (one 16-byte store) at byte offset `off` of a tile
 __device__ __forceinline__ void store_h8(char* tile, uint32_t off, const float* v) {
     *reinterpret_cast<uint4*>(tile + off) = make_uint4(tc::pack_f16(v[0], v[1]), tc::pack_f16(v[2], v[3]),
@@ -148,7 +139,8 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return r;
 }
-// SiLU of two values (see silu_fast)
+// SiLU of two values: SiLU(x) = x sigmoid(x) = h + h tanh(h), h = x / 2, with the hardware tanh (one
+// MUFU operation; its error is below the fp16 rounding every conv output goes through)
 __device__ __forceinline__ float2 silu2(float2 x) {
     const float2 h = fmul2(make_float2(0.5f, 0.5f), x);
     float2 t;

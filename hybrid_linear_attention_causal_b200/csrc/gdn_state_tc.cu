@@ -20,10 +20,10 @@
 // first half:
 //   - the state update writes the fp16 copy of S^T (the A operand of X and Oi,
 //     in tensor memory) in two column halves, each released on its own
-//     barrier, so the next chunk's X issues its first k-steps while the second
-//     half is still being updated;
-//   - V' is formed in two halves of the chunk's rows, each released on its own
-//     barrier, so the state product issues its first k-steps meanwhile;
+//     barrier once every compute warp has written its part of it, so the next
+//     chunk's X issues its first k-steps while the second half is updated;
+//   - V' is formed in two halves of the chunk's rows the same way, so the
+//     state product issues its first k-steps while the second half is formed;
 //   - the output products run on the tensor core while the CUDA cores form V'
 //     and update the state, and four output warps (one per TMEM
 //     sub-partition) read, scale, stage and store each chunk's outputs once
@@ -33,7 +33,8 @@
 // tenth issues every bulk copy, refilling each double-buffered tile as soon as
 // its last reader releases it and prefetching tiles into L2 a few chunks ahead.
 // The two compute warps of a TMEM sub-partition share its 32 accumulator rows
-// and take one half of the columns each.
+// and take one quarter of the columns each in either half, the first half
+// first.
 
 #include "gdn_internal.cuh"
 #include "gdn_tc.cuh"
@@ -101,13 +102,13 @@ __device__ __forceinline__ bool group_and(bool pred, int id, int nthreads) {
 __device__ __forceinline__ bool cw_and(bool pred) { return group_and(pred, kCwBarrier, NCW * 32); }
 __device__ __forceinline__ bool ow_and(bool pred) { return group_and(pred, kOwBarrier, NOW * 32); }
 
-// fp16 copy of 32 consecutive values of S^T row j (this thread's lane) into 16 columns of the
+// fp16 copy of 16 consecutive values of S^T row j (this thread's lane) into 8 columns of the
 // tensor-memory A operand: two fp16 per column, the even column of S^T in the low half
-__device__ __forceinline__ void put_sa32(uint32_t taddr, const float* v) {
-    uint32_t wv[16];
+__device__ __forceinline__ void put_sa16(uint32_t taddr, const float* v) {
+    uint32_t wv[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) wv[i] = tc::pack_f16(v[2 * i], v[2 * i + 1]);
-    tc::tmem_st16(taddr, wv);
+    for (int i = 0; i < 8; ++i) wv[i] = tc::pack_f16(v[2 * i], v[2 * i + 1]);
+    tc::tmem_st8(taddr, wv);
 }
 
 template <typename T, int DK, int DV>
@@ -177,8 +178,8 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             tc::mbar_init(bar(sm.free_w[bb]), 1);
             tc::mbar_init(bar(sm.free_u[bb]), NCW + NOW);  // V' formed + the output warps' copy of e^gamma
             tc::mbar_init(bar(sm.free_aq[bb]), 1);          // the output product's commit
-            tc::mbar_init(bar(sm.bar_vp[bb]), NCW / 2);
-            tc::mbar_init(bar(sm.bar_sa[bb]), NCW / 2);
+            tc::mbar_init(bar(sm.bar_vp[bb]), NCW);
+            tc::mbar_init(bar(sm.bar_sa[bb]), NCW);
             tc::mbar_init(bar(sm.out_free[bb]), NOW);
             tc::mbar_init(bar(sm.bar_o[bb]), 1);
         }
@@ -189,8 +190,14 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
         for (int id = c_begin + 2; id < c_end && id < c_begin + kPrefetchAhead; ++id) prefetch(id);
     }
 
-    // compute warps: thread (sp, half, lane) owns row j of S^T, columns half * DK/2 .. + DK/2
-    const int sp = warp & 3, half = (warp >> 2) & 1;
+    // compute warps: thread (sp, hw, lane) owns row j of S^T and, in each half of its columns, the
+    // quarter hw: columns q * DK/2 + hw * DK/4 .. + DK/4 for q = 0, 1 (register s[q * DK/4 + i]).
+    // Every compute warp finishes its part of the first half before it starts on the second, so
+    // each half's barrier completes half-way through the phase and the products waiting on it start
+    // while the second half is formed.  (V'^T's chunk rows are shared out the same way.)
+    const int sp = warp & 3, hw = (warp >> 2) & 1;
+    constexpr int QW = DK / 4;
+    auto col_of = [&](int i) { return (i / QW) * (DK / 2) + hw * QW + i % QW; };
     const uint32_t lane_base = (uint32_t)(sp * 32) << 16;
     const bool rowv = warp < NCW && (DV == 128 || lane < 16);
     const int j = DV == 128 ? sp * 32 + lane : sp * 16 + lane;
@@ -199,7 +206,7 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     float* Sg = p.ssm_state + ((size_t)slot * HV + h) * DK * DV;
     float s[DK / 2];
 #pragma unroll
-    for (int i = 0; i < DK / 2; ++i) s[i] = (init && rowv) ? Sg[(size_t)(half * (DK / 2) + i) * DV + j] : 0.f;
+    for (int i = 0; i < DK / 2; ++i) s[i] = (init && rowv) ? Sg[(size_t)col_of(i) * DV + j] : 0.f;
     // a state checkpoint of this sequence: the state entering the chunk that holds its boundary is
     // stored when that chunk comes up (a boundary at the very end belongs to the last chunk); the
     // rows of that chunk before the boundary are added afterwards, off the chain
@@ -224,14 +231,18 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
     auto tOi = [&](int bb) { return tm + 128 + 64 * bb; };
     auto tOq = [&](int bb) { return tm + 256 + 64 * bb; };
     static_assert(DK <= 128 && DV <= 128, "tensor-memory layout");
-    const uint32_t tA_row = tA + lane_base + half * (DK / 4);
+    // S^T column c of row j sits in tensor-memory column c / 2 of lane j's row of the A operand
+    auto tA_at = [&](int i) { return tA + lane_base + (uint32_t)(col_of(i) / 2); };
     if (warp < NCW) {  // the starting state's fp16 copy, released as both halves of the first chunk's X
 #pragma unroll
-        for (int cc = 0; cc < DK / 2; cc += 32) put_sa32(tA_row + cc / 2, &s[cc]);
-        tc::tmem_st_wait();
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
+        for (int q = 0; q < 2; ++q) {
+#pragma unroll
+            for (int cc = 0; cc < QW; cc += 16) put_sa16(tA_at(q * QW + cc), &s[q * QW + cc]);
+            tc::tmem_st_wait();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[q]));
+        }
     }
 
     bool ok = true;
@@ -347,9 +358,9 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
             const uint32_t ph = (uint32_t)it & 1u, pb = (uint32_t)(it >> 1) & 1u;
             if (id == ck_chunk && rowv)  // the state entering the checkpoint's chunk: column j of S
 #pragma unroll
-                for (int i = 0; i < DK / 2; ++i) ck_dst[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
-            // V'^T row j = U^T row j - X^T row j over this warp's half of the chunk's rows, and
-            // Vs'^T = V'^T diag(f)
+                for (int i = 0; i < DK / 2; ++i) ck_dst[(size_t)col_of(i) * DV + j] = s[i];
+            // V'^T row j = U^T row j - X^T row j and Vs'^T = V'^T diag(f), over this warp's quarter hw of
+            // each half of the chunk's rows, the first half first
             bool okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_x), ph) && tc::mbar_wait(bar(sm.full_u[bb]), pb));
             float egn = 0.f;
             if (okl) {
@@ -358,69 +369,76 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                 char* vsb = reinterpret_cast<char*>(sm.vs);
                 const char* utb = reinterpret_cast<const char*>(sm.ut[bb]);
 #pragma unroll
-                for (int cc = 0; cc < C / 2; cc += 8) {  // 8 fp16 values per 16-byte vector
-                    const int c0 = half * (C / 2) + cc;
-                    float xv[8], f[8];
-                    tc::tmem_ld8(tX + lane_base + c0, xv);
+                for (int q = 0; q < 2; ++q) {
 #pragma unroll
-                    for (int q = 0; q < 8; q += 4) *reinterpret_cast<float4*>(f + q) = *reinterpret_cast<const float4*>(&sm.gv[bb][1][c0 + q]);
-                    tc::tmem_ld_wait();
-                    if (rowv) {
-                        const uint32_t off = uoff(c0);
-                        const uint4 u = *reinterpret_cast<const uint4*>(utb + off);
-                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-                        uint32_t vw[4], sw[4];
+                    for (int cc = 0; cc < C / 4; cc += 8) {  // 8 fp16 values per 16-byte vector
+                        const int c0 = q * (C / 2) + hw * (C / 4) + cc;
+                        float xv[8], f[8];
+                        tc::tmem_ld8(tX + lane_base + c0, xv);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 uu = tc::unpack_f16(uw[e]);
-                            const float v0 = uu.x - xv[2 * e], v1 = uu.y - xv[2 * e + 1];
-                            amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));  // |f| <= 1: covers f V' too
-                            vw[e] = tc::pack_f16(v0, v1);
-                            sw[e] = tc::pack_f16(v0 * f[2 * e], v1 * f[2 * e + 1]);
+                        for (int k4 = 0; k4 < 8; k4 += 4)
+                            *reinterpret_cast<float4*>(f + k4) = *reinterpret_cast<const float4*>(&sm.gv[bb][1][c0 + k4]);
+                        tc::tmem_ld_wait();
+                        if (rowv) {
+                            const uint32_t off = uoff(c0);
+                            const uint4 u = *reinterpret_cast<const uint4*>(utb + off);
+                            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                            uint32_t vw[4], sw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 uu = tc::unpack_f16(uw[e]);
+                                const float v0 = uu.x - xv[2 * e], v1 = uu.y - xv[2 * e + 1];
+                                amax = fmaxf(amax, fmaxf(fabsf(v0), fabsf(v1)));  // |f| <= 1: covers f V' too
+                                vw[e] = tc::pack_f16(v0, v1);
+                                sw[e] = tc::pack_f16(v0 * f[2 * e], v1 * f[2 * e + 1]);
+                            }
+                            *reinterpret_cast<uint4*>(vtb + off) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+                            *reinterpret_cast<uint4*>(vsb + off) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
                         }
-                        *reinterpret_cast<uint4*>(vtb + off) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-                        *reinterpret_cast<uint4*>(vsb + off) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
                     }
+                    tc::fence_smem_to_async();
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(sm.bar_vp[q]));
                 }
                 egn = sm.gv[bb][3][0];  // e^{gamma_n}
-                tc::fence_smem_to_async();
-                tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(bar(sm.bar_vp[half]));
-                    tc::mbar_arrive(bar(sm.free_u[bb]));
-                }
+                if (lane == 0) tc::mbar_arrive(bar(sm.free_u[bb]));
             }
-            // S^T <- e^{gamma_n} S^T + Snew^T, and its fp16 copy for the next chunk, half by half
+            // S^T <- e^{gamma_n} S^T + Snew^T, and its fp16 copy for the next chunk, the first half first
             if (okl) okl = __all_sync(0xffffffffu, tc::mbar_wait(bar(sm.bar_s), ph));
             if (okl) {
                 tc::fence_after_sync();
 #pragma unroll
-                for (int cc = 0; cc < DK / 2; cc += 16) {
-                    float v[16];
-                    tc::tmem_ld16(tSn + lane_base + half * (DK / 2) + cc, v);
-                    tc::tmem_ld_wait();
-                    uint32_t wv[8];
+                for (int q = 0; q < 2; ++q) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        s[cc + i] = fmaf(egn, s[cc + i], v[i]);
-                        amax = fmaxf(amax, fabsf(s[cc + i]));
+                    for (int cc = 0; cc < QW; cc += 16) {
+                        const int i0 = q * QW + cc;
+                        float v[16];
+                        tc::tmem_ld16(tSn + lane_base + col_of(i0), v);
+                        tc::tmem_ld_wait();
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            s[i0 + i] = fmaf(egn, s[i0 + i], v[i]);
+                            amax = fmaxf(amax, fabsf(s[i0 + i]));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) wv[i] = tc::pack_f16(s[i0 + 2 * i], s[i0 + 2 * i + 1]);
+                        tc::tmem_st8(tA_at(i0), wv);
                     }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) wv[i] = tc::pack_f16(s[cc + 2 * i], s[cc + 2 * i + 1]);
-                    tc::tmem_st8(tA_row + cc / 2, wv);
+                    tc::tmem_st_wait();
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[q]));
                 }
-                tc::tmem_st_wait();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(sm.bar_sa[half]));
             }
             ok = cw_and(okl);
             if (!ok) break;
         }
         if (ok && rowv)  // final state: column j of S
 #pragma unroll
-            for (int i = 0; i < DK / 2; ++i) Sg[(size_t)(half * (DK / 2) + i) * DV + j] = s[i];
+            for (int i = 0; i < DK / 2; ++i) Sg[(size_t)col_of(i) * DV + j] = s[i];
         if (!rowv) amax = 0.f;  // lanes past a 64-row tile hold no row
         report_f16_range(p.hdr, amax);
     } else {

@@ -319,9 +319,13 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k)
                     tc::mma_f16_ta(tOi(bb), tA + 8 * k, tc::desc_add(dQb, tc::sw128_kstep(2 * C, k)), ix, k > 0);
-                // Snew^T = Vs'^T K (K read MN-major), each half of the rows as soon as it is formed
+                // Snew^T = Vs'^T K (K read MN-major) and Oq^T = V'^T Aqk^T, each half of the chunk's rows as
+                // soon as it is formed: the state product's k-steps of a half first, then Oq's (off the
+                // chain), so that Oq's first half fills the wait for V's second half and only its second
+                // half sits between the state product and the next chunk's X
+                ok = tc::mbar_wait(bar(sm.full_aq[bb]), pb);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
+                for (int hh = 0; hh < 2 && ok; ++hh) {
                     ok = tc::mbar_wait(bar(sm.bar_vp[hh]), ph);
                     tc::fence_after_sync();
                     if (!ok) break;
@@ -329,17 +333,16 @@ __global__ void __launch_bounds__(NT, 1) state_tc_kernel(ExtendArgs p, int seg) 
                     for (int k = 2 * hh; k < 2 * hh + 2; ++k)
                         tc::mma_f16(tSn, tc::desc_add(dVs, tc::sw128_kstep(DV, k)), tc::desc_add(dKb, 2048u * k), is,
                                     k > 0);
+                    if (hh == 1) {
+                        tc::mma_commit(bar(sm.bar_s));
+                        tc::mma_commit(bar(sm.free_kq[bb]));
+                    }
+#pragma unroll
+                    for (int k = 2 * hh; k < 2 * hh + 2; ++k)
+                        tc::mma_f16(tOq(bb), tc::desc_add(dVt, tc::sw128_kstep(DV, k)),
+                                    tc::desc_add(dAb, tc::sw128_kstep(C, k)), ix, k > 0);
                 }
                 if (!ok) break;
-                tc::mma_commit(bar(sm.bar_s));
-                tc::mma_commit(bar(sm.free_kq[bb]));
-                // Oq^T = V'^T Aqk^T: queued behind the state product, off the chain
-                ok = tc::mbar_wait(bar(sm.full_aq[bb]), pb);
-                if (!ok) break;
-#pragma unroll
-                for (int k = 0; k < C / 16; ++k)
-                    tc::mma_f16(tOq(bb), tc::desc_add(dVt, tc::sw128_kstep(DV, k)),
-                                tc::desc_add(dAb, tc::sw128_kstep(C, k)), ix, k > 0);
                 tc::mma_commit(bar(sm.bar_o[bb]));
                 tc::mma_commit(bar(sm.free_aq[bb]));
             }
